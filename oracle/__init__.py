@@ -1,0 +1,220 @@
+"""CPU oracle for MXFP8 quantisation and GEMM -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline /
+reference arm of ``bench.py`` may import this package.  The product path
+(``moe_grouped_gemm_mx_b200``) never imports it, and it never imports the
+product path.  The arithmetic lives in ``mx_oracle.c`` (plain C, fp64); this
+module only builds that library and marshals numpy arrays into it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mx_oracle.c")
+_LIB = os.path.join(_HERE, "libmx_oracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math, OpenMP across rows)."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < max(
+        os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "mx_oracle.h")))
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c99", "-D_DEFAULT_SOURCE", "-fopenmp", "-shared", "-fPIC",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I32 = ctypes.c_int32
+        L.mxo_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.mxo_e4m3_decode.restype = ctypes.c_double
+        L.mxo_e4m3_encode.argtypes = [ctypes.c_double]
+        L.mxo_e4m3_encode.restype = ctypes.c_uint8
+        L.mxo_ue8m0_decode.argtypes = [ctypes.c_uint8]
+        L.mxo_ue8m0_decode.restype = ctypes.c_double
+        L.mxo_floor_log2.argtypes = [ctypes.c_double]
+        L.mxo_floor_log2.restype = ctypes.c_int
+        L.mxo_e4m3_table.argtypes = [P]
+        L.mxo_e4m3_table.restype = None
+        L.mxo_quantize_block.argtypes = [P, P, P]
+        L.mxo_quantize_block.restype = None
+        L.mxo_quantize.argtypes = [P, I64, I64, P, P]
+        L.mxo_quantize.restype = None
+        L.mxo_scale_bytes.argtypes = [I64, I64]
+        L.mxo_scale_bytes.restype = I64
+        L.mxo_sf_offset.argtypes = [I64, I64, I64]
+        L.mxo_sf_offset.restype = I64
+        L.mxo_sf_tile.argtypes = [P, I64, I64, P]
+        L.mxo_sf_tile.restype = None
+        L.mxo_sf_untile.argtypes = [P, I64, I64, P]
+        L.mxo_sf_untile.restype = None
+        L.mxo_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P, P]
+        L.mxo_gemm.restype = None
+        L.mxo_grouped_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, P, I64, P, P]
+        L.mxo_grouped_contiguous.restype = None
+        L.mxo_grouped_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P]
+        L.mxo_grouped_masked.restype = None
+        L.mxo_num_threads.argtypes = []
+        L.mxo_num_threads.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _u16(x) -> np.ndarray:
+    """Accept a numpy uint16 array or a torch bfloat16 tensor (its raw bits)."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch  # only for turning a bf16 tensor into its bit pattern
+    assert x.dtype == torch.bfloat16
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+# ---------------------------------------------------------------- scalars
+
+def e4m3_decode(code: int) -> float:
+    return lib().mxo_e4m3_decode(code)
+
+
+def e4m3_encode(v: float) -> int:
+    return lib().mxo_e4m3_encode(v)
+
+
+def ue8m0_decode(code: int) -> float:
+    return lib().mxo_ue8m0_decode(code)
+
+
+def floor_log2(a: float) -> int:
+    return lib().mxo_floor_log2(a)
+
+
+def e4m3_table() -> np.ndarray:
+    out = np.zeros(256, dtype=np.float64)
+    lib().mxo_e4m3_table(_p(out))
+    return out
+
+
+# ---------------------------------------------------------------- quantiser
+
+def quantize_block(x_bits: np.ndarray):
+    x = _u16(x_bits).reshape(32)
+    q = np.zeros(32, dtype=np.uint8)
+    s = np.zeros(1, dtype=np.uint8)
+    lib().mxo_quantize_block(_p(x), _p(q), _p(s))
+    return q, int(s[0])
+
+
+def quantize(x):
+    """BF16 [..., k] -> (q uint8 [rows, k], sf uint8 row-major [rows, k/32]),
+    rows = product of the leading dimensions."""
+    xb = _u16(x)
+    k = xb.shape[-1]
+    rows = xb.size // k if k else 0
+    assert k % 32 == 0
+    q = np.zeros((rows, k), dtype=np.uint8)
+    sf = np.zeros((rows, k // 32), dtype=np.uint8)
+    lib().mxo_quantize(_p(xb), rows, k, _p(q), _p(sf))
+    return q, sf
+
+
+def scale_bytes(rows: int, k: int) -> int:
+    return lib().mxo_scale_bytes(rows, k)
+
+
+def sf_offset(r: int, c: int, k: int) -> int:
+    return lib().mxo_sf_offset(r, c, k)
+
+
+def sf_tile(sf_rm: np.ndarray, rows: int, k: int) -> np.ndarray:
+    sf_rm = np.ascontiguousarray(sf_rm, dtype=np.uint8)
+    out = np.zeros(scale_bytes(rows, k), dtype=np.uint8)
+    lib().mxo_sf_tile(_p(sf_rm), rows, k, _p(out))
+    return out
+
+
+def sf_untile(tiled: np.ndarray, rows: int, k: int) -> np.ndarray:
+    tiled = np.ascontiguousarray(tiled, dtype=np.uint8)
+    out = np.zeros((rows, k // 32), dtype=np.uint8)
+    lib().mxo_sf_untile(_p(tiled), rows, k, _p(out))
+    return out
+
+
+# ---------------------------------------------------------------- GEMMs
+
+def gemm(qa, sfa, qb, sfb, rows=None):
+    """D = deq(A) * deq(B)^T in fp64 for the listed rows (all if None).
+
+    Returns (d, abssum), both [nrows, n] float64; abssum = sum_k |a*b|."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qb = np.ascontiguousarray(qb, dtype=np.uint8)
+    sfa = np.ascontiguousarray(sfa, dtype=np.uint8)
+    sfb = np.ascontiguousarray(sfb, dtype=np.uint8)
+    m, k = qa.shape
+    n = qb.shape[0]
+    ids = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = m if ids is None else len(ids)
+    d = np.zeros((nrows, n), dtype=np.float64)
+    a = np.zeros((nrows, n), dtype=np.float64)
+    lib().mxo_gemm(_p(qa), _p(sfa), _p(qb), _p(sfb), m, n, k, _p(ids), nrows, _p(d), _p(a))
+    return d, a
+
+
+def grouped_contiguous(qa, sfa, qb, sfb, offsets, rows=None):
+    """qa [m_total, k], qb [groups, n, k]; offsets int32 [groups+1]."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qb = np.ascontiguousarray(qb, dtype=np.uint8)
+    sfa = np.ascontiguousarray(sfa, dtype=np.uint8)
+    sfb = np.ascontiguousarray(sfb, dtype=np.uint8)
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    groups = len(off) - 1
+    _, n, k = qb.shape
+    ids = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = int(off[-1]) if ids is None else len(ids)
+    d = np.zeros((nrows, n), dtype=np.float64)
+    a = np.zeros((nrows, n), dtype=np.float64)
+    lib().mxo_grouped_contiguous(_p(qa), _p(sfa), _p(qb), _p(sfb), _p(off), groups, n, k,
+                                 _p(ids), nrows, _p(d), _p(a))
+    return d, a
+
+
+def grouped_masked(qa, sfa, qb, sfb, masked_m):
+    """qa [groups, max_m, k], qb [groups, n, k]; rows >= masked_m[e] are NaN."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qb = np.ascontiguousarray(qb, dtype=np.uint8)
+    sfa = np.ascontiguousarray(sfa, dtype=np.uint8)
+    sfb = np.ascontiguousarray(sfb, dtype=np.uint8)
+    mm = np.ascontiguousarray(masked_m, dtype=np.int32)
+    groups, max_m, k = qa.shape
+    n = qb.shape[1]
+    d = np.zeros((groups, max_m, n), dtype=np.float64)
+    a = np.zeros((groups, max_m, n), dtype=np.float64)
+    lib().mxo_grouped_masked(_p(qa), _p(sfa), _p(qb), _p(sfb), _p(mm), groups, max_m, n, k,
+                             _p(d), _p(a))
+    return d, a
+
+
+def num_threads() -> int:
+    return lib().mxo_num_threads()

@@ -1,0 +1,348 @@
+/*
+ * mx_oracle.c -- plain, slow CPU oracle for MXFP8 quantisation and GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * bench's CPU-baseline / reference arm may load this library.  The CUDA
+ * path never calls it and shares no code, header or table with it.
+ *
+ * What it computes, and where each step comes from:
+ *  - MXFP8 = 8-bit floating-point elements that share one power-of-two
+ *    exponent per block of 32 consecutive elements along K
+ *    ("PyTorch and Nebius ... DeepSeek-V3 MoE training on B200", glossary
+ *    entry on microscaling FP8, and its pointer to the OCP Microscaling
+ *    specification).  Elements are E4M3 (bias 7, no infinities, S.1111.111
+ *    is NaN, largest finite 448); the shared scale is UE8M0, value
+ *    2^(code-127), code 0xFF = NaN.
+ *  - Scale choice: X = floor(log2(amax)) - 8 (8 = exponent of the largest
+ *    E4M3 power of two, 256), clamped to [-127, 127]; elements are v*2^-X
+ *    rounded to nearest-even and saturated to +-448.
+ *  - The pipeline "BF16 -> MXFP8 -> grouped GEMM -> BF16" (same page,
+ *    diagram description of the MXFP8 flow from router input to all-to-all
+ *    combine).  The GEMM here is the exact sum of products of the
+ *    dequantised operands, accumulated in double, k ascending.
+ *  - Grouped GEMMs in contiguous and masked layouts ("DeepGEMM" summary
+ *    page, list of MoE grouped GEMM layouts; the DeepGEMM release page,
+ *    section 4 "MoE optimisation").  Both are defined as a dense GEMM per
+ *    group.
+ *
+ * Readings where the pages are silent (each one is listed in the design
+ * notes of the repository):
+ *  - an all-zero block gets scale code 0x00 (X = -127);
+ *  - a block holding any NaN or +-Inf gets scale 0xFF and every element 0x7F;
+ *  - a result that rounds to zero keeps the sign of its input (0x80 for -0);
+ *  - the scale bytes are stored in 128-row x 4-column tiles of 512 bytes,
+ *    byte (r%32)*16 + ((r%128)/32)*4 + (c%4), tiles ordered row-block major.
+ *
+ * Plain C99 + OpenMP across independent output rows only.  Build:
+ *   gcc -O2 -fopenmp -shared -fPIC -o libmx_oracle.so mx_oracle.c -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "mx_oracle.h"
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---------------------------------------------------------------- E4M3 */
+
+/* Value of one E4M3 code, by the format's definition: sign s, 4 exponent
+ * bits e (bias 7), 3 mantissa bits m.  e == 0 is subnormal (m/8 * 2^-6);
+ * S.1111.111 is NaN; there is no infinity. */
+double mxo_e4m3_decode(uint8_t code)
+{
+    int s = (code >> 7) & 1;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double mag;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+void mxo_e4m3_table(double out[256])
+{
+    for (int c = 0; c < 256; ++c)
+        out[c] = mxo_e4m3_decode((uint8_t)c);
+}
+
+/* Encode an already-scaled value v' as E4M3, round to nearest with ties to
+ * the even code, saturating: |v'| >= 448 gives +-448.  The search runs over
+ * the 127 finite non-negative codes 0x00..0x7E, whose values increase
+ * strictly with the code, so "even code" is "even mantissa LSB". */
+static double e4m3_mag[127]; /* values of codes 0x00..0x7E, filled at load */
+
+__attribute__((constructor)) static void fill_e4m3_mag(void)
+{
+    for (int c = 0; c < 127; ++c)
+        e4m3_mag[c] = mxo_e4m3_decode((uint8_t)c);
+}
+
+uint8_t mxo_e4m3_encode(double v)
+{
+    const double *mag = e4m3_mag;
+    if (isnan(v))
+        return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a >= 448.0)
+        return sign | 0x7E;
+    /* largest lo with mag[lo] <= a (binary search; mag[0] = 0 <= a) */
+    int lo = 0, hi = 126;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (mag[mid] <= a)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    int code;
+    if (mag[lo] == a) {
+        code = lo;
+    } else {
+        /* a lies strictly between mag[lo] and mag[lo+1] (a < 448 = mag[126]) */
+        double dlo = a - mag[lo];
+        double dhi = mag[lo + 1] - a;
+        if (dlo < dhi)
+            code = lo;
+        else if (dhi < dlo)
+            code = lo + 1;
+        else
+            code = (lo % 2 == 0) ? lo : lo + 1;
+    }
+    return sign | (uint8_t)code;
+}
+
+/* ---------------------------------------------------------------- UE8M0 */
+
+double mxo_ue8m0_decode(uint8_t code)
+{
+    if (code == 0xFF)
+        return NAN;
+    return ldexp(1.0, (int)code - 127);
+}
+
+/* floor(log2(a)) for finite a > 0, from the C library's exact frexp:
+ * a = f * 2^e with f in [0.5, 1), so floor(log2 a) = e - 1. */
+int mxo_floor_log2(double a)
+{
+    int e;
+    (void)frexp(a, &e);
+    return e - 1;
+}
+
+/* ---------------------------------------------------------------- BF16 */
+
+double mxo_bf16_to_double(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------- block quantiser */
+
+/* Quantise one block of 32 BF16 values: scale selection, then each element
+ * scaled by 2^-X (exact in double) and encoded. */
+void mxo_quantize_block(const uint16_t *x, uint8_t *q, uint8_t *scale)
+{
+    double v[32];
+    double amax = 0.0;
+    int nonfinite = 0;
+    for (int i = 0; i < 32; ++i) {
+        v[i] = mxo_bf16_to_double(x[i]);
+        if (!isfinite(v[i]))
+            nonfinite = 1;
+        else if (fabs(v[i]) > amax)
+            amax = fabs(v[i]);
+    }
+    if (nonfinite) {
+        *scale = 0xFF;
+        for (int i = 0; i < 32; ++i)
+            q[i] = 0x7F;
+        return;
+    }
+    int X;
+    if (amax == 0.0)
+        X = -127;
+    else
+        X = mxo_floor_log2(amax) - 8;
+    if (X < -127)
+        X = -127;
+    if (X > 127)
+        X = 127;
+    *scale = (uint8_t)(X + 127);
+    for (int i = 0; i < 32; ++i)
+        q[i] = mxo_e4m3_encode(ldexp(v[i], -X));
+}
+
+/* Quantise a row-major [rows, k] BF16 matrix (k % 32 == 0) along k.
+ * q is [rows, k] bytes; sf is the PLAIN row-major [rows, k/32] scale matrix. */
+void mxo_quantize(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, uint8_t *sf)
+{
+    int64_t kb = k / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < kb; ++c)
+            mxo_quantize_block(x + r * k + c * 32, q + r * k + c * 32, sf + r * kb + c);
+}
+
+/* ------------------------------------------------------ scale tile layout */
+
+int64_t mxo_scale_bytes(int64_t rows, int64_t k)
+{
+    int64_t kb = k / 32;
+    int64_t rpad = (rows + 127) / 128 * 128;
+    int64_t kbpad = (kb + 3) / 4 * 4;
+    return rpad * kbpad;
+}
+
+/* Byte offset of scale (r, c) -- row r, K-block c -- in the tiled layout. */
+int64_t mxo_sf_offset(int64_t r, int64_t c, int64_t k)
+{
+    int64_t kb = k / 32;
+    int64_t kbpad = (kb + 3) / 4 * 4;
+    int64_t tile = (r / 128) * (kbpad / 4) + c / 4;
+    return tile * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+}
+
+void mxo_sf_tile(const uint8_t *sf_rm, int64_t rows, int64_t k, uint8_t *tiled)
+{
+    int64_t kb = k / 32;
+    memset(tiled, 0, (size_t)mxo_scale_bytes(rows, k));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < kb; ++c)
+            tiled[mxo_sf_offset(r, c, k)] = sf_rm[r * kb + c];
+}
+
+void mxo_sf_untile(const uint8_t *tiled, int64_t rows, int64_t k, uint8_t *sf_rm)
+{
+    int64_t kb = k / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < kb; ++c)
+            sf_rm[r * kb + c] = tiled[mxo_sf_offset(r, c, k)];
+}
+
+/* ------------------------------------------------------------------ GEMM */
+
+static double deq(const double *tab, uint8_t qv, uint8_t sfv)
+{
+    return tab[qv] * mxo_ue8m0_decode(sfv);
+}
+
+/* One output row: d[j] = sum_k deq(a[i,k]) * deq(b[j,k]) for j < n, k
+ * ascending, in double; abssum[j] = sum_k |deq(a) * deq(b)|. */
+static void gemm_row(const double *tab, const uint8_t *qa_row, const uint8_t *sfa_row,
+                     const uint8_t *qb, const uint8_t *sfb, int64_t n, int64_t k,
+                     double *d_row, double *abs_row)
+{
+    int64_t kb = k / 32;
+    for (int64_t j = 0; j < n; ++j) {
+        const uint8_t *qb_row = qb + j * k;
+        const uint8_t *sfb_row = sfb + j * kb;
+        double acc = 0.0, aacc = 0.0;
+        for (int64_t kk = 0; kk < k; ++kk) {
+            double p = deq(tab, qa_row[kk], sfa_row[kk / 32]) * deq(tab, qb_row[kk], sfb_row[kk / 32]);
+            acc += p;
+            aacc += fabs(p);
+        }
+        d_row[j] = acc;
+        if (abs_row)
+            abs_row[j] = aacc;
+    }
+}
+
+/* D = A * B^T for the listed rows of A (all rows when row_ids is NULL).
+ * qa [m, k], sfa row-major [m, k/32], qb [n, k], sfb row-major [n, k/32].
+ * d and abssum are [nrows, n] (row t holds A-row row_ids[t]). */
+void mxo_gemm(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb, const uint8_t *sfb,
+              int64_t m, int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows,
+              double *d, double *abssum)
+{
+    double tab[256];
+    mxo_e4m3_table(tab);
+    int64_t kb = k / 32;
+    if (!row_ids)
+        nrows = m;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < nrows; ++t) {
+        int64_t i = row_ids ? row_ids[t] : t;
+        gemm_row(tab, qa + i * k, sfa + i * kb, qb, sfb, n, k, d + t * n,
+                 abssum ? abssum + t * n : NULL);
+    }
+}
+
+/* Contiguous grouped GEMM: rows [off[e], off[e+1]) of A use expert e's B.
+ * qb is [groups, n, k], sfb row-major [groups, n, k/32].  Only listed rows
+ * (or all rows of all groups when row_ids is NULL, in which case nrows must
+ * be off[groups]) are computed; a row outside every group gives NaN. */
+void mxo_grouped_contiguous(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                            const uint8_t *sfb, const int32_t *offsets, int32_t groups,
+                            int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows,
+                            double *d, double *abssum)
+{
+    double tab[256];
+    mxo_e4m3_table(tab);
+    int64_t kb = k / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < nrows; ++t) {
+        int64_t i = row_ids ? row_ids[t] : t;
+        int e = -1;
+        for (int g = 0; g < groups; ++g)
+            if (i >= offsets[g] && i < offsets[g + 1])
+                e = g;
+        if (e < 0) {
+            for (int64_t j = 0; j < n; ++j) {
+                d[t * n + j] = NAN;
+                if (abssum)
+                    abssum[t * n + j] = NAN;
+            }
+            continue;
+        }
+        gemm_row(tab, qa + i * k, sfa + i * kb, qb + (int64_t)e * n * k,
+                 sfb + (int64_t)e * n * kb, n, k, d + t * n, abssum ? abssum + t * n : NULL);
+    }
+}
+
+/* Masked grouped GEMM: A is [groups, max_m, k]; for group e only rows
+ * r < masked_m[e] are products (d[e, r, :] = A[e, r, :] * B[e]^T); the
+ * other rows are left as NaN here and must stay untouched on the device. */
+void mxo_grouped_masked(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                        const uint8_t *sfb, const int32_t *masked_m, int32_t groups,
+                        int64_t max_m, int64_t n, int64_t k, double *d, double *abssum)
+{
+    double tab[256];
+    mxo_e4m3_table(tab);
+    int64_t kb = k / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < (int64_t)groups * max_m; ++t) {
+        int64_t e = t / max_m, r = t % max_m;
+        if (r >= masked_m[e]) {
+            for (int64_t j = 0; j < n; ++j) {
+                d[t * n + j] = NAN;
+                if (abssum)
+                    abssum[t * n + j] = NAN;
+            }
+            continue;
+        }
+        gemm_row(tab, qa + t * k, sfa + t * kb, qb + e * n * k, sfb + e * n * kb, n, k,
+                 d + t * n, abssum ? abssum + t * n : NULL);
+    }
+}
+
+int mxo_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

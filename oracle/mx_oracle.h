@@ -1,0 +1,44 @@
+/*
+ * mx_oracle.h -- declarations of the CPU oracle (test infrastructure only).
+ * See mx_oracle.c for the definitions each function follows.
+ */
+#ifndef MX_ORACLE_H
+#define MX_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+double mxo_e4m3_decode(uint8_t code);
+void mxo_e4m3_table(double out[256]);
+uint8_t mxo_e4m3_encode(double v);
+double mxo_ue8m0_decode(uint8_t code);
+int mxo_floor_log2(double a);
+double mxo_bf16_to_double(uint16_t bits);
+
+void mxo_quantize_block(const uint16_t *x, uint8_t *q, uint8_t *scale);
+void mxo_quantize(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, uint8_t *sf);
+
+int64_t mxo_scale_bytes(int64_t rows, int64_t k);
+int64_t mxo_sf_offset(int64_t r, int64_t c, int64_t k);
+void mxo_sf_tile(const uint8_t *sf_rm, int64_t rows, int64_t k, uint8_t *tiled);
+void mxo_sf_untile(const uint8_t *tiled, int64_t rows, int64_t k, uint8_t *sf_rm);
+
+void mxo_gemm(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb, const uint8_t *sfb,
+              int64_t m, int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows,
+              double *d, double *abssum);
+void mxo_grouped_contiguous(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                            const uint8_t *sfb, const int32_t *offsets, int32_t groups,
+                            int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows,
+                            double *d, double *abssum);
+void mxo_grouped_masked(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                        const uint8_t *sfb, const int32_t *masked_m, int32_t groups,
+                        int64_t max_m, int64_t n, int64_t k, double *d, double *abssum);
+int mxo_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

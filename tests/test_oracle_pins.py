@@ -1,0 +1,368 @@
+"""Pins for the CPU oracle: each check ties the oracle to something other than
+itself -- hand-derived golden blocks, torch's own float8_e4m3fn codec, the
+BF16 bit layout, closed forms, invariants and brute force on tiny inputs.
+
+No GPU is needed; these run in the CPU suite.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "blocks.txt")
+
+
+def _expand(items):
+    out = []
+    i = 0
+    while i < len(items):
+        tok = items[i]
+        if i + 1 < len(items) and items[i + 1].startswith("x") and items[i + 1][1:].isdigit():
+            out.extend([tok] * int(items[i + 1][1:]))
+            i += 2
+        else:
+            out.append(tok)
+            i += 1
+    return out
+
+
+def load_golden_blocks():
+    cases, cur = [], None
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, _, val = line.partition(":")
+        val = val.strip()
+        if key == "case":
+            cur = {"name": val}
+            cases.append(cur)
+        elif key == "input":
+            cur["input"] = [float(t) for t in _expand(val.split())]
+        elif key == "scale":
+            cur["scale"] = int(val, 16)
+        elif key == "codes":
+            cur["codes"] = [int(t, 16) for t in _expand(val.split())]
+    for c in cases:
+        assert len(c["input"]) == 32 and len(c["codes"]) == 32, c["name"]
+    return cases
+
+
+def bf16_bits(values):
+    t = torch.tensor(values, dtype=torch.float64).to(torch.bfloat16)
+    assert torch.equal(t.double().isnan(), torch.tensor(values, dtype=torch.float64).isnan())
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def all_bf16():
+    """Every BF16 bit pattern as (uint16 bits, float64 values)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    return bits, vals
+
+
+# ---------------------------------------------------------------- E4M3 table
+
+def test_e4m3_table_matches_torch_float8(oracle):
+    tab = oracle.e4m3_table()
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(tab), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(tab[fin], ref[fin])
+    assert np.array_equal(np.signbit(tab[fin]), np.signbit(ref[fin]))
+
+
+def test_e4m3_table_landmarks(oracle):
+    tab = oracle.e4m3_table()
+    assert tab[0x7E] == 448.0
+    assert tab[0x78] == 256.0
+    assert tab[0x01] == 2.0 ** -9
+    assert tab[0x08] == 2.0 ** -6          # smallest normal
+    assert tab[0x07] == 7 * 2.0 ** -9      # largest subnormal
+    assert tab[0x80] == 0.0 and math.copysign(1.0, tab[0x80]) == -1.0
+    assert math.isnan(tab[0x7F]) and math.isnan(tab[0xFF])
+    assert np.sum(np.isnan(tab)) == 2
+    pos = tab[0x00:0x7F]
+    assert np.all(np.diff(pos) > 0)        # strictly increasing 0x00..0x7E
+    assert np.array_equal(tab[0x80:0xFF], -pos)
+
+
+def test_e4m3_roundtrip_all_finite_codes(oracle):
+    for c in list(range(0x00, 0x7F)) + list(range(0x80, 0xFF)):
+        assert oracle.e4m3_encode(oracle.e4m3_decode(c)) == c, hex(c)
+
+
+def test_e4m3_encode_matches_torch_cast_exhaustive(oracle):
+    """Every BF16 value v, scaled by 2^j for several j, encoded by the oracle
+    equals torch's RNE float->float8_e4m3fn cast wherever torch does not
+    overflow (|v| <= 464); above that the oracle saturates to +-448."""
+    bits, vals = all_bf16()
+    fin = np.isfinite(vals)
+    for j in (0, -8, 4, 9):
+        v = np.ldexp(vals[fin], j)
+        ours = np.array([oracle.e4m3_encode(float(x)) for x in v[::7]], dtype=np.uint8)
+        vs = v[::7]
+        small = np.abs(vs) <= 464.0
+        ref = torch.from_numpy(vs[small]).float().to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(ours[small], ref), f"j={j}"
+        big = ~small
+        assert np.all(ours[big] == np.where(np.signbit(vs[big]), 0xFE, 0x7E))
+
+
+def test_e4m3_encode_dense_sweep_against_torch(oracle):
+    """Values on a grid finer than the E4M3 spacing over the full range,
+    including exact midpoints (ties) between neighbouring codes."""
+    tab = oracle.e4m3_table()
+    pos = tab[0x00:0x7F]
+    mids = (pos[:-1] + pos[1:]) / 2
+    grid = np.concatenate([pos, mids, mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20)])
+    grid = np.concatenate([grid, -grid])
+    ours = np.array([oracle.e4m3_encode(float(x)) for x in grid], dtype=np.uint8)
+    ref = torch.from_numpy(grid).float().to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    # float32 conversion of the grid is exact for pos/mids; the +-2^-20 nudges
+    # stay on their side of the midpoint in float32 too.
+    assert np.array_equal(ours, ref)
+
+
+# ---------------------------------------------------------------- scale
+
+def test_ue8m0_decode(oracle):
+    assert oracle.ue8m0_decode(127) == 1.0
+    assert oracle.ue8m0_decode(0) == 2.0 ** -127
+    assert oracle.ue8m0_decode(254) == 2.0 ** 127
+    assert math.isnan(oracle.ue8m0_decode(255))
+
+
+def test_floor_log2_matches_bf16_exponent_field(oracle):
+    """floor(log2 |v|) for every positive finite BF16 value, against the
+    value's own bit fields: exponent-127 for normals, and for subnormals
+    (m * 2^-133) the index of m's top bit minus 133."""
+    bits, vals = all_bf16()
+    sel = (vals > 0) & np.isfinite(vals)
+    for b, v in zip(bits[sel][::3], vals[sel][::3]):
+        e = (int(b) >> 7) & 0xFF
+        m = int(b) & 0x7F
+        want = e - 127 if e > 0 else m.bit_length() - 1 - 133
+        assert oracle.floor_log2(float(v)) == want, (hex(b), v)
+
+
+@pytest.mark.parametrize("case", load_golden_blocks(), ids=lambda c: c["name"])
+def test_golden_blocks(oracle, case):
+    q, s = oracle.quantize_block(bf16_bits(case["input"]))
+    assert s == case["scale"]
+    assert q.tolist() == case["codes"]
+
+
+def test_scale_invariance_power_of_two(oracle):
+    """Multiplying a block by 2^j (no clamping) keeps every element code and
+    shifts the scale code by +j."""
+    rng = np.random.default_rng(0)
+    for t in range(200):
+        x = rng.standard_normal(32) * 2.0 ** rng.integers(-20, 20)
+        base = bf16_bits(list(x))
+        xb = torch.from_numpy(base.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+        q0, s0 = oracle.quantize_block(base)
+        for j in (-30, -5, 1, 7, 40):
+            xs = np.ldexp(xb, j)
+            if not (1e-30 < np.max(np.abs(xs)) < 1e30):
+                continue
+            q1, s1 = oracle.quantize_block(bf16_bits(list(xs)))
+            if 0 < s0 + j < 255 and s0 != 0:
+                assert s1 == s0 + j
+                assert np.array_equal(q1, q0)
+
+
+def test_roundtrip_exactly_representable_blocks(oracle):
+    """Blocks built as e4m3(c_i) * 2^X with amax in [256, 448]*2^X quantise
+    back to exactly (c_i, X+127)."""
+    rng = np.random.default_rng(1)
+    tab = oracle.e4m3_table()
+    for t in range(300):
+        X = int(rng.integers(-100, 100))
+        codes = rng.integers(0, 0x7F, size=32).astype(np.uint8)
+        codes[rng.integers(0, 32)] = rng.integers(0x78, 0x7F)  # amax in [256, 448]
+        signs = rng.integers(0, 2, size=32).astype(np.uint8) << 7
+        codes = codes | signs
+        vals = np.ldexp(tab[codes], X)
+        q, s = oracle.quantize_block(bf16_bits(list(vals)))
+        assert s == X + 127
+        # -0 and +0 both decode to 0; the sign survives
+        assert np.array_equal(q, codes)
+
+
+def test_dequantised_error_bound(oracle):
+    """|deq(q) - v| <= half an E4M3 ulp at v's binade (relative 2^-4), or the
+    subnormal spacing 2^(X-10), except for saturated elements."""
+    rng = np.random.default_rng(2)
+    tab = oracle.e4m3_table()
+    x = torch.from_numpy(rng.standard_normal((64, 256)) * 3).to(torch.bfloat16)
+    q, sf = oracle.quantize(x)
+    v = x.double().numpy()
+    deq = tab[q] * np.ldexp(1.0, sf.astype(np.int64) - 127).repeat(32, axis=1)
+    X = sf.astype(np.int64).repeat(32, axis=1) - 127
+    err = np.abs(deq - v)
+    sat = np.abs(v) * np.ldexp(1.0, -X) >= 448
+    bound = np.maximum(np.abs(v) * 2.0 ** -4, np.ldexp(1.0, X - 10))
+    assert np.all(err[~sat] <= bound[~sat])
+
+
+# ---------------------------------------------------------------- layout
+
+def test_scale_layout_is_bijection(oracle):
+    for rows, k in [(1, 32), (128, 128), (129, 160), (300, 512), (64, 7168)]:
+        kb = k // 32
+        nbytes = oracle.scale_bytes(rows, k)
+        assert nbytes == ((rows + 127) // 128 * 128) * ((kb + 3) // 4 * 4)
+        rpad = (rows + 127) // 128 * 128
+        kbpad = (kb + 3) // 4 * 4
+        offs = {oracle.sf_offset(r, c, k) for r in range(rpad) for c in range(kbpad)}
+        assert offs == set(range(nbytes))
+
+
+def test_scale_layout_tile_geometry(oracle):
+    """Inside a 128x4 tile: 4 consecutive K-blocks of one row are 4
+    consecutive bytes; rows r, r+32, r+64, r+96 share one 16-byte line."""
+    k = 512
+    for r in range(128):
+        base = oracle.sf_offset(r, 0, k)
+        assert [oracle.sf_offset(r, c, k) - base for c in range(4)] == [0, 1, 2, 3]
+        assert base // 16 == r % 32
+        assert (base % 16) // 4 == r // 32
+    assert oracle.sf_offset(0, 4, k) == 512            # next K tile
+    assert oracle.sf_offset(128, 0, k) == 512 * 4      # next row block (kb=16 -> 4 K tiles)
+
+
+def test_scale_tile_untile_roundtrip(oracle):
+    rng = np.random.default_rng(3)
+    for rows, k in [(1, 32), (130, 96), (256, 512)]:
+        sf = rng.integers(0, 256, size=(rows, k // 32)).astype(np.uint8)
+        t = oracle.sf_tile(sf, rows, k)
+        assert np.array_equal(oracle.sf_untile(t, rows, k), sf)
+        mask = np.zeros(t.shape, bool)
+        for r in range(rows):
+            for c in range(k // 32):
+                mask[oracle.sf_offset(r, c, k)] = True
+        assert np.all(t[~mask] == 0)
+
+
+# ---------------------------------------------------------------- GEMM
+
+def _int_block_matrix(rng, rows, k):
+    """Integers in [-4, 4] with a +-4 in every 32-block (so X = 2-8 = -6 and
+    every element v*64 is an exact E4M3 value)."""
+    m = rng.integers(-4, 5, size=(rows, k)).astype(np.float64)
+    for c in range(k // 32):
+        m[np.arange(rows), c * 32 + rng.integers(0, 32, size=rows)] = 4.0 * rng.choice([-1, 1], size=rows)
+    return m
+
+
+def test_gemm_exact_on_small_integers(oracle):
+    rng = np.random.default_rng(4)
+    for m, n, k in [(5, 7, 32), (16, 9, 64), (3, 33, 96)]:
+        a = _int_block_matrix(rng, m, k)
+        b = _int_block_matrix(rng, n, k)
+        qa, sfa = oracle.quantize(torch.from_numpy(a).to(torch.bfloat16))
+        qb, sfb = oracle.quantize(torch.from_numpy(b).to(torch.bfloat16))
+        assert np.all(sfa == 121) and np.all(sfb == 121)
+        d, absd = oracle.gemm(qa, sfa, qb, sfb)
+        want = a.astype(np.int64) @ b.astype(np.int64).T
+        assert np.array_equal(d, want.astype(np.float64))
+        assert np.array_equal(absd, (np.abs(a) @ np.abs(b).T))
+
+
+def test_gemm_identity_and_permutation(oracle):
+    rng = np.random.default_rng(5)
+    k = 64
+    b = torch.from_numpy(rng.standard_normal((10, k))).to(torch.bfloat16)
+    qb, sfb = oracle.quantize(b)
+    tab = oracle.e4m3_table()
+    deq_b = tab[qb] * np.ldexp(1.0, sfb.astype(np.int64) - 127).repeat(32, axis=1)
+    perm = rng.permutation(k)[:7]
+    a = np.zeros((7, k))
+    a[np.arange(7), perm] = 1.0
+    qa, sfa = oracle.quantize(torch.from_numpy(a).to(torch.bfloat16))
+    d, _ = oracle.gemm(qa, sfa, qb, sfb)
+    assert np.array_equal(d, deq_b[:, perm].T)
+
+
+def test_gemm_matches_torch_matmul_fp64(oracle):
+    rng = np.random.default_rng(6)
+    m, n, k = 33, 40, 160
+    a = torch.from_numpy(rng.standard_normal((m, k)) * 3).to(torch.bfloat16)
+    b = torch.from_numpy(rng.standard_normal((n, k)) * 0.02).to(torch.bfloat16)
+    qa, sfa = oracle.quantize(a)
+    qb, sfb = oracle.quantize(b)
+    tab = oracle.e4m3_table()
+    da = tab[qa] * np.ldexp(1.0, sfa.astype(np.int64) - 127).repeat(32, axis=1)
+    db = tab[qb] * np.ldexp(1.0, sfb.astype(np.int64) - 127).repeat(32, axis=1)
+    want = (torch.from_numpy(da) @ torch.from_numpy(db).T).numpy()
+    d, absd = oracle.gemm(qa, sfa, qb, sfb)
+    assert np.allclose(d, want, rtol=0, atol=1e-12 * np.max(absd))
+    # a row subset gives the same rows
+    rows = np.array([0, 5, 32])
+    d2, _ = oracle.gemm(qa, sfa, qb, sfb, rows=rows)
+    assert np.array_equal(d2, d[rows])
+
+
+def test_gemm_quantisation_error_within_stated_tolerance(oracle):
+    """The oracle's MXFP8 product stays within 1e-2*sum|a*b| + 1e-3 of the
+    unquantised BF16 product for this data -- a loose sanity pin that a
+    wrong scale sign or a dropped 2^X would break by orders of magnitude."""
+    rng = np.random.default_rng(7)
+    a = torch.from_numpy(rng.standard_normal((20, 256))).to(torch.bfloat16)
+    b = torch.from_numpy(rng.standard_normal((24, 256)) * 0.02).to(torch.bfloat16)
+    qa, sfa = oracle.quantize(a)
+    qb, sfb = oracle.quantize(b)
+    d, absd = oracle.gemm(qa, sfa, qb, sfb)
+    exact = a.double().numpy() @ b.double().numpy().T
+    assert np.all(np.abs(d - exact) <= 0.1 * absd + 1e-3)
+
+
+# ---------------------------------------------------------------- grouped
+
+def test_grouped_contiguous_equals_dense_per_group(oracle):
+    rng = np.random.default_rng(8)
+    k, n = 64, 24
+    counts = [3, 0, 130, 1]
+    off = [0]
+    for c in counts:
+        off.append(off[-1] + (c + 127) // 128 * 128)
+    m_total = off[-1]
+    a = torch.from_numpy(rng.standard_normal((m_total, k))).to(torch.bfloat16)
+    b = torch.from_numpy(rng.standard_normal((len(counts), n, k)) * 0.02).to(torch.bfloat16)
+    qa, sfa = oracle.quantize(a)
+    qb, sfb = oracle.quantize(b)
+    qb = qb.reshape(len(counts), n, k)
+    d, _ = oracle.grouped_contiguous(qa, sfa, qb, sfb, np.array(off, np.int32))
+    sfb3 = sfb.reshape(len(counts), n, k // 32)
+    for e in range(len(counts)):
+        lo, hi = off[e], off[e + 1]
+        if hi == lo:
+            continue
+        de, _ = oracle.gemm(qa[lo:hi], sfa[lo:hi], qb[e], sfb3[e])
+        assert np.array_equal(d[lo:hi], de)
+    # one group == dense
+    d1, _ = oracle.grouped_contiguous(qa[:128], sfa[:128], qb[:1], sfb3[:1].reshape(-1, k // 32),
+                                      np.array([0, 128], np.int32))
+    dd, _ = oracle.gemm(qa[:128], sfa[:128], qb[0], sfb3[0])
+    assert np.array_equal(d1, dd)
+
+
+def test_grouped_masked_equals_dense_per_group(oracle):
+    rng = np.random.default_rng(9)
+    E, max_m, n, k = 3, 40, 16, 96
+    mm = np.array([0, 40, 7], np.int32)
+    a = torch.from_numpy(rng.standard_normal((E, max_m, k))).to(torch.bfloat16)
+    b = torch.from_numpy(rng.standard_normal((E, n, k)) * 0.02).to(torch.bfloat16)
+    qa, sfa = oracle.quantize(a)
+    qb, sfb = oracle.quantize(b)
+    qa3, sfa3 = qa.reshape(E, max_m, k), sfa.reshape(E, max_m, k // 32)
+    qb3, sfb3 = qb.reshape(E, n, k), sfb.reshape(E, n, k // 32)
+    d, _ = oracle.grouped_masked(qa3, sfa, qb3, sfb, mm)
+    for e in range(E):
+        assert np.all(np.isnan(d[e, mm[e]:]))
+        if mm[e]:
+            de, _ = oracle.gemm(qa3[e, :mm[e]], sfa3[e, :mm[e]], qb3[e], sfb3[e])
+            assert np.array_equal(d[e, :mm[e]], de)
