@@ -1,0 +1,647 @@
+#!/usr/bin/env python
+"""MXFP8 GEMM / grouped-GEMM throughput on B200, one JSON line on stdout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole path over one batch of synthetic BF16 input
+already resident in HBM: quantise the activations (BF16 -> MXFP8 with tiled
+UE8M0 scales), quantise the weights, and run the GEMM(s) with the fused BF16
+epilogue.  The step is captured once in a CUDA graph and replayed; each kernel
+is bracketed by graph-captured CUDA events, so per-kernel device times come
+from the timed replays themselves.  L2 is flushed (a 512 MiB write) before
+every timed step, outside the step's events.
+
+Workloads (shapes from the pages; data synthetic and seeded):
+  page        dense 64x2112x7168, 64x24576x1536, 128x7168x2048 (default)
+  pr1         dense 128x256x512
+  large       dense M=8192, (N,K) in {(7168,2048),(2112,7168),(4096,7168)}
+  contiguous  MoE grouped, 32 experts, 8192 tokens top-8 Zipf: gate/up N=4096 K=7168,
+              then down N=7168 K=2048
+  masked      MoE masked grouped, 32 experts x 256 rows, masked_m ~ U{0..256}, N=4096 K=7168
+
+With torchrun (N > 1) every rank runs its own independent batch (the work
+units are independent problems; no data-path collective), the step time is
+the max over ranks and `value` counts the work of all ranks ("weak" scaling).
+`--impl reference` times the CPU oracle (rank 0 only) on a bounded sample of
+the same workload, in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+QUANT_BYTES_PER_ELT = 2.0 + 1.0 + 1.0 / 32.0
+METRIC = "MXFP8 GEMM & grouped-GEMM TFLOPS on 1 B200; % of dense FP8 tensor peak"
+
+
+def static_config(name: str, seed: int) -> dict:
+    """Workload description shared by both arms (no GPU needed)."""
+    import mx_inputs as I
+    cfg = {"workload": name, "seed": seed}
+    if name == "pr1":
+        cfg.update({"shapes": ["128x256x512"], "a": "N(0,1)", "b": "N(0,0.02)"})
+    elif name == "page":
+        cfg.update({"shapes": [f"{m}x{n}x{k}" for m, n, k in I.PAGE_SHAPES],
+                    "a": "N(0,1) with 0.5% x64 outliers", "b": "N(0,0.02)"})
+    elif name == "large":
+        cfg.update({"shapes": [f"{I.LARGE_M}x{n}x{k}" for n, k in I.LARGE_NK],
+                    "a": "row-wise 2^U[-4,4] * N(0,1)", "b": "N(0,0.02)"})
+    elif name == "contiguous":
+        counts = I.zipf_routing_counts(seed=seed)
+        cfg.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "topk": I.MOE_TOPK,
+                    "zipf_s": I.MOE_ZIPF_S, "real_rows": int(counts.sum()),
+                    "padded_rows": int(I.padded_offsets(counts)[-1]),
+                    "gemms": ["gate_up N=4096 K=7168", "down N=7168 K=2048"]})
+    elif name == "masked":
+        mm = I.masked_counts(seed=seed)
+        cfg.update({"experts": I.MASKED_EXPERTS, "max_m": I.MASKED_MAX_M, "n": I.MASKED_NK[0],
+                    "k": I.MASKED_NK[1], "valid_rows": int(mm.sum()), "active_experts": int((mm > 0).sum())})
+    cfg["step"] = "quantise activations + quantise weights + GEMM(s) with BF16 epilogue"
+    return cfg
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked"])
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-flush", action="store_true", help="skip the L2 flush (for ncu launch lists)")
+    p.add_argument("--eager", action="store_true", help="launch kernels directly instead of a CUDA graph")
+    p.add_argument("--seed", type=int, default=0)
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- peaks / clocks
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling every 200 ms while the GPU is under load."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ts, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        inside = [r for r in rows if t0 <= r[0] <= t1] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in inside:
+            for nm, v in zip(names, r[4][1:]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "power_w_max": max(r[3] for r in inside), "reasons": sorted(reasons),
+                "samples": len(inside), "samples_in_timed_region": sum(1 for r in rows if t0 <= r[0] <= t1)}
+
+
+# ---------------------------------------------------------------- workloads
+
+class Workload:
+    """Device-resident inputs/outputs and the list of kernel launches of one step."""
+
+    def __init__(self, name, dev, seed, mx, inputs):
+        import torch
+        self.name = name
+        self.dev = dev
+        self.mx = mx
+        self.launches = []      # (kind, label, fn, algorithmic bytes, algorithmic flops)
+        self.host_inputs = []   # (host pinned tensor, device tensor) pairs for e2e
+        self.outputs = []       # device tensors read back for e2e
+        self.flops = 0.0
+        self.config = {"workload": name}
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        getattr(self, "_build_" + name)(seed, inputs)
+
+    # -- helpers
+    def _quant(self, x, label):
+        import torch
+        mx = self.mx
+        groups = 1 if x.dim() == 2 else x.shape[0]
+        rows, k = x.shape[-2], x.shape[-1]
+        q = torch.empty(x.shape, dtype=torch.uint8, device=self.dev)
+        sf = torch.empty(groups * mx.scale_bytes(rows, k), dtype=torch.uint8, device=self.dev)
+        nbytes = x.numel() * QUANT_BYTES_PER_ELT
+        self.launches.append(("quant", label, lambda: mx.mx_quantize_bf16_to_e4m3(x, q=q, sf=sf), nbytes, 0.0))
+        return q, sf
+
+    def _add_input(self, t):
+        import torch
+        self.host_inputs.append((torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu()), t))
+
+    def _gemm_bytes(self, m_rows, n, k, b_experts=1):
+        # minimum traffic: A and B bytes once, their scales, D once
+        return m_rows * k * (1 + 1 / 32) + b_experts * n * k * (1 + 1 / 32) + 2 * m_rows * n
+
+    def _dense(self, a, b, label):
+        import torch
+        mx = self.mx
+        m, k = a.shape
+        n = b.shape[0]
+        self._add_input(a)
+        self._add_input(b)
+        qa, sfa = self._quant(a, label + ":A")
+        qb, sfb = self._quant(b, label + ":B")
+        d = torch.empty((m, n), dtype=torch.bfloat16, device=self.dev)
+        self.outputs.append(d)
+        fl = 2.0 * m * n * k
+        self.launches.append(("gemm", label, lambda: mx.mx_gemm(qa, sfa, qb, sfb, d=d, dev_status=self.status),
+                              self._gemm_bytes(m, n, k), fl))
+        self.flops += fl
+
+    # -- workloads
+    def _build_pr1(self, seed, I):
+        a, b = I.dense_problem(128, 256, 512, seed=seed, device=self.dev)
+        self._dense(a, b, "128x256x512")
+        self.config.update({"shapes": ["128x256x512"]})
+
+    def _build_page(self, seed, I):
+        for (m, n, k) in I.PAGE_SHAPES:
+            a, b = I.dense_problem(m, n, k, seed=seed, kind="outlier", device=self.dev)
+            self._dense(a, b, f"{m}x{n}x{k}")
+        self.config.update({"shapes": [f"{m}x{n}x{k}" for m, n, k in I.PAGE_SHAPES],
+                            "a": "N(0,1) with 0.5% x64 outliers", "b": "N(0,0.02)"})
+
+    def _build_large(self, seed, I):
+        for (n, k) in I.LARGE_NK:
+            a, b = I.dense_problem(I.LARGE_M, n, k, seed=seed, kind="loguniform", device=self.dev)
+            self._dense(a, b, f"{I.LARGE_M}x{n}x{k}")
+        self.config.update({"shapes": [f"{I.LARGE_M}x{n}x{k}" for n, k in I.LARGE_NK],
+                            "a": "row-wise 2^U[-4,4] * N(0,1)", "b": "N(0,0.02)"})
+
+    def _build_contiguous(self, seed, I):
+        import torch
+        mx = self.mx
+        counts = I.zipf_routing_counts(seed=seed)
+        real = int(counts.sum())
+        for (n, k), tag in ((I.MOE_GATE_NK, "gate_up"), (I.MOE_DOWN_NK, "down")):
+            prob = I.contiguous_problem(n=n, k=k, seed=seed + (0 if tag == "gate_up" else 100),
+                                        counts=counts, device=self.dev)
+            self._add_input(prob.a)
+            self._add_input(prob.b)
+            qa, sfa = self._quant(prob.a, tag + ":A")
+            qb, sfb = self._quant(prob.b, tag + ":B")
+            off = prob.offsets.to(self.dev)
+            m_total = prob.a.shape[0]
+            d = torch.empty((m_total, n), dtype=torch.bfloat16, device=self.dev)
+            self.outputs.append(d)
+            fl = 2.0 * real * n * k
+            experts = int((counts > 0).sum())
+            self.launches.append(("gemm", tag, lambda qa=qa, sfa=sfa, qb=qb, sfb=sfb, off=off, d=d:
+                                  mx.mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, off, d=d, dev_status=self.status),
+                                  self._gemm_bytes(m_total, n, k, experts), fl))
+            self.flops += fl
+        self.config.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "topk": I.MOE_TOPK,
+                            "zipf_s": I.MOE_ZIPF_S, "real_rows": real,
+                            "padded_rows": int(I.padded_offsets(counts)[-1]),
+                            "gemms": ["gate_up N=4096 K=7168", "down N=7168 K=2048"]})
+
+    def _build_masked(self, seed, I):
+        import torch
+        mx = self.mx
+        n, k = I.MASKED_NK
+        prob = I.masked_problem(n=n, k=k, seed=seed, device=self.dev)
+        self._add_input(prob.a)
+        self._add_input(prob.b)
+        qa, sfa = self._quant(prob.a, "A")
+        qb, sfb = self._quant(prob.b, "B")
+        mm = prob.masked_m.to(self.dev)
+        e, max_m, _ = prob.a.shape
+        d = torch.empty((e, max_m, n), dtype=torch.bfloat16, device=self.dev)
+        self.outputs.append(d)
+        rows = int(prob.masked_m.sum())
+        active = int((prob.masked_m > 0).sum())
+        fl = 2.0 * rows * n * k
+        self.launches.append(("gemm", "masked", lambda: mx.mx_grouped_gemm_masked(
+            qa, sfa, qb, sfb, mm, d=d, dev_status=self.status), self._gemm_bytes(rows, n, k, active), fl))
+        self.flops += fl
+        self.config.update({"experts": e, "max_m": max_m, "n": n, "k": k, "valid_rows": rows,
+                            "active_experts": active})
+
+    def run_eager(self):
+        for _, _, fn, _, _ in self.launches:
+            fn()
+
+
+# ---------------------------------------------------------------- oracle (CPU) timing
+
+def oracle_sample(name, seed, target_s=10.0):
+    """Time the CPU oracle on a bounded sample of the workload.
+
+    Returns (flops_per_second, description, threads)."""
+    import numpy as np
+    import oracle
+    import mx_inputs as I
+    oracle.build()
+    L = oracle
+
+    def dense_sample(a, b, rows):
+        qa, sfa = L.quantize(a[:rows] if rows else a)
+        qb, sfb = L.quantize(b)
+        L.gemm(qa, sfa, qb, sfb)
+        m = qa.shape[0]
+        return 2.0 * m * b.shape[0] * b.shape[1]
+
+    jobs = []
+    if name == "pr1":
+        a, b = I.dense_problem(128, 256, 512, seed=seed)
+        jobs.append(lambda: dense_sample(a, b, None))
+        desc = "full 128x256x512 step (quantise A and B, GEMM)"
+    elif name == "page":
+        probs = [I.dense_problem(m, n, k, seed=seed, kind="outlier") for (m, n, k) in I.PAGE_SHAPES]
+        jobs.append(lambda: sum(dense_sample(a, b, None) for a, b in probs))
+        desc = "full page-shapes step (quantise A and B, GEMM, all three shapes)"
+    elif name == "large":
+        probs = [I.dense_problem(64, n, k, seed=seed, kind="loguniform") for (n, k) in I.LARGE_NK]
+        jobs.append(lambda: sum(dense_sample(a, b, None) for a, b in probs))
+        desc = "a 64-row slice of A per shape (quantise it and all of B, GEMM it)"
+    elif name == "contiguous":
+        counts = I.zipf_routing_counts(seed=seed)
+        n, k = I.MOE_GATE_NK
+        g = np.random.default_rng(seed)
+        a = I.normal_bf16((64, k), 1.0, seed + 7)
+        b = I.normal_bf16((2, n, k), 0.02, seed + 8)
+
+        def job():
+            qa, sfa = L.quantize(a)
+            qb, sfb = L.quantize(b)
+            off = np.array([0, 32, 64], dtype=np.int32)
+            L.grouped_contiguous(qa, sfa, qb.reshape(2, n, k), sfb, off)
+            return 2.0 * 64 * n * k
+        jobs.append(job)
+        desc = "gate/up GEMM on 64 rows over 2 experts (quantise rows and both experts' weights)"
+        del counts, g
+    else:  # masked
+        n, k = I.MASKED_NK
+        prob = I.masked_problem(n=n, k=k, experts=2, max_m=32, seed=seed,
+                                masked_m=__import__("torch").tensor([32, 32], dtype=__import__("torch").int32))
+
+        def job():
+            qa, sfa = L.quantize(prob.a)
+            qb, sfb = L.quantize(prob.b)
+            L.grouped_masked(qa.reshape(2, 32, k), sfa, qb.reshape(2, n, k), sfb, prob.masked_m.numpy())
+            return 2.0 * 64 * n * k
+        jobs.append(job)
+        desc = "2 experts x 32 valid rows of the masked decode GEMM (N=4096, K=7168)"
+
+    flops = 0.0
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        for j in jobs:
+            flops += j()
+        reps += 1
+        if time.perf_counter() - t0 >= target_s:
+            break
+    dt = time.perf_counter() - t0
+    return flops / dt, f"{desc}; {reps} repetition(s) in {dt:.1f} s", L.num_threads()
+
+
+# ---------------------------------------------------------------- main paths
+
+def dist_init(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float, dev) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    per_step = []
+    flops_rate = None
+    desc, threads = "", 1
+    target = max(1.0, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        rate, desc, threads = oracle_sample(args.workload, args.seed, target_s=target)
+        if i >= args.warmup:
+            per_step.append(rate)
+    flops_rate = statistics.median(per_step)
+    value = flops_rate / 1e12
+    line = {"impl": "reference", "metric": METRIC,
+            "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": static_config(args.workload, args.seed),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "moe_grouped_gemm_mx_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def lookup_traffic(kernel_kind: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            tab = json.load(f)
+        ent = tab.get(f"{kernel_kind}:{workload}")
+        if ent and ent.get("source_hash") == kernel_source_hash():
+            return float(ent["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        return None
+    return None
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the library has no CPU path)")
+    import moe_grouped_gemm_mx_b200 as mx
+    import mx_inputs
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+
+    wl = Workload(args.workload, dev, args.seed + 1000 * rank, mx, mx_inputs)
+    stream = torch.cuda.Stream(device=dev)
+    flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    n_k = len(wl.launches)
+
+    # one eager pass (sets kernel attributes), then capture the step
+    with torch.cuda.stream(stream):
+        wl.run_eager()
+    torch.cuda.synchronize()
+    if int(wl.status.item()) != 0:
+        raise SystemExit(f"device status {int(wl.status.item()):#x} after the first step")
+
+    k_start = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_k)]
+    k_end = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_k)]
+    graph = None
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i, (_, _, fn, _, _) in enumerate(wl.launches):
+                k_start[i].record()
+                fn()
+                k_end[i].record()
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            for i, (_, _, fn, _, _) in enumerate(wl.launches):
+                k_start[i].record()
+                fn()
+                k_end[i].record()
+
+    s_ev = torch.cuda.Event(enable_timing=True)
+    e_ev = torch.cuda.Event(enable_timing=True)
+
+    try:
+        smi_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001 - fall back to the index
+        smi_id = str(local)
+    sampler = ClockSampler(smi_id)
+    sampler.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            if not args.no_flush:
+                flush_buf.zero_()
+            step()
+    torch.cuda.synchronize()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    step_ms = []
+    kern_ms = [[] for _ in range(n_k)]
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            if not args.no_flush:
+                flush_buf.zero_()
+            s_ev.record()
+            step()
+            e_ev.record()
+            e_ev.synchronize()
+            step_ms.append(s_ev.elapsed_time(e_ev))
+            for i in range(n_k):
+                kern_ms[i].append(k_start[i].elapsed_time(k_end[i]))
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall1 = time.time()
+    sampler.stop()
+    clocks = sampler.summary(t_wall0 - 0.25, t_wall1 + 0.25)
+
+    st = int(wl.status.item())
+    if st != 0:
+        raise SystemExit(f"device status {st:#x} during the timed steps")
+
+    ms_step = statistics.mean(step_ms)
+    ms_step_max = max_over_ranks(world, ms_step, dev)
+    value = world * wl.flops / (ms_step_max * 1e-3) / 1e12
+
+    # per-kernel breakdown and the roofline of the dominant kernel kind
+    per_launch = []
+    for i, (kind, label, _, nbytes, fl) in enumerate(wl.launches):
+        per_launch.append({"kind": kind, "label": label, "ms": statistics.mean(kern_ms[i]),
+                           "bytes": nbytes, "flops": fl})
+    kinds = {}
+    for r in per_launch:
+        kk = kinds.setdefault(r["kind"], {"ms": 0.0, "bytes": 0.0, "flops": 0.0, "launches": 0})
+        kk["ms"] += r["ms"]
+        kk["bytes"] += r["bytes"]
+        kk["flops"] += r["flops"]
+        kk["launches"] += 1
+    dom = max(kinds, key=lambda k: kinds[k]["ms"])
+    dk = kinds[dom]
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    ridge = fp8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    tensor_bound = dom == "gemm" and dk["flops"] / max(dk["bytes"], 1.0) > ridge
+    sec = dk["ms"] * 1e-3
+    if tensor_bound:
+        achieved = dk["flops"] / sec / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp8_peak}
+        peak_note = f"fp8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']}"
+    else:
+        achieved = dk["bytes"] / sec / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+        peak_note = f"{peaks['source']} hbm copy bandwidth"
+    trf = lookup_traffic(dom, args.workload)
+    roof["traffic"] = None if trf is None else trf
+    roof.update({"kernel": dom, "launches_per_step": dk["launches"], "avg_launch_ms": dk["ms"] / dk["launches"],
+                 "peak_source": peak_note})
+
+    # end to end through the public API: pinned host inputs -> device, step, result -> host
+    e2e = None
+    if not args.no_e2e:
+        h2d = sum(h.numel() * h.element_size() for h, _ in wl.host_inputs)
+        host_out = [torch.empty(d.shape, dtype=d.dtype, pin_memory=True) for d in wl.outputs]
+        d2h = sum(d.numel() * d.element_size() for d in wl.outputs)
+        e2e_steps = max(3, min(args.steps, 20))
+        times = []
+        with torch.cuda.stream(stream):
+            for it in range(e2e_steps + 2):
+                s_ev.record()
+                for h, dd in wl.host_inputs:
+                    dd.copy_(h, non_blocking=True)
+                wl.run_eager()
+                for dd, h in zip(wl.outputs, host_out):
+                    h.copy_(dd, non_blocking=True)
+                e_ev.record()
+                e_ev.synchronize()
+                if it >= 2:
+                    times.append(s_ev.elapsed_time(e_ev))
+        e2e_ms = max_over_ranks(world, statistics.mean(times), dev)
+        e2e = {"value": world * wl.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, threads = oracle_sample(args.workload, args.seed, target_s=10.0)
+        cpu = {"value": rate / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    launches_per_step = sum(1 for r in per_launch)
+    line = {
+        "metric": METRIC,
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3", "data": "synthetic",
+        "config": dict(static_config(args.workload, args.seed),
+                       l2="flushed (512 MiB write) before every timed step",
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                       graph=graph is not None),
+        "pct_of_fp8_peak": value / world / fp8_peak,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "kernels": [{"kind": r["kind"], "label": r["label"], "ms": round(r["ms"], 5),
+                     "GB/s": round(r["bytes"] / (r["ms"] * 1e-3) / 1e9, 1),
+                     "TFLOP/s": round(r["flops"] / (r["ms"] * 1e-3) / 1e12, 1)} for r in per_launch],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    return 0
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_init(args)
+    try:
+        if args.impl == "reference":
+            rc = run_reference(args, world, rank)
+        else:
+            rc = run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,154 @@
+/*
+ * mx.h -- C ABI of the B200 (sm_100a) MXFP8 GEMM library.
+ *
+ * What the library computes
+ * -------------------------
+ * MXFP8 ("PyTorch and Nebius optimise DeepSeek-V3 MoE training on B200
+ * clusters", glossary entry on microscaling FP8, and the OCP Microscaling
+ * specification it cites): 8-bit E4M3 elements that share one UE8M0
+ * power-of-two scale per block of 32 consecutive elements along K.  The
+ * pipeline is BF16 -> MXFP8 -> (grouped) GEMM with FP32 accumulation -> BF16
+ * (same page, diagram of the MXFP8 flow from router input to the all-to-all
+ * combine).  The GEMM family -- one dense GEMM and MoE grouped GEMMs in a
+ * contiguous and a masked layout -- is the one the DeepGEMM pages describe
+ * ("DeepGEMM" summary page, introduction and the MoE grouped GEMM note;
+ * DeepGEMM release page, section 4 "MoE optimisation").
+ *
+ * Conventions for every call
+ * --------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library allocates no memory per call and keeps no reference to any
+ *    pointer after the call returns.
+ *  - Row-major layouts with K contiguous.  A is [M, K], B is [N, K] (one
+ *    expert) or [E, N, K]; the product is D = A * B^T, [M, N] BF16.
+ *  - Quantised elements: one byte per element (E4M3), same shape as the
+ *    BF16 source.
+ *  - Scales: UE8M0 bytes (value 2^(c-127), 0xFF = NaN) in the tiled layout
+ *    the tensor cores consume.  For a matrix of R rows and Kb = K/32 blocks,
+ *    rows are padded to a multiple of 128 and Kb to a multiple of 4; the
+ *    scale of row r, block c sits at byte
+ *        ((r/128)*(Kb_pad/4) + c/4) * 512 + (r%32)*16 + ((r%128)/32)*4 + c%4.
+ *    Padding bytes are written as 0x00 by the quantiser.  For 3-D operands
+ *    each group has its own such region of mx_scale_bytes(rows, K) bytes,
+ *    placed back to back.
+ *  - Every call is asynchronous on `stream` (NULL = legacy default stream).
+ *    Argument errors are reported synchronously through the return value
+ *    and nothing is launched.  Data-dependent errors found on the device
+ *    (bad group offsets, masked_m out of range, an internal wait that timed
+ *    out) are OR-ed into *dev_status as MX_DEV_* bits when dev_status is
+ *    not NULL, otherwise into a library-internal word readable with
+ *    mx_read_internal_status().  Kernels never trap.
+ *  - No exceptions cross this boundary.
+ */
+#ifndef MX_H
+#define MX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *mx_stream_t;
+
+typedef enum mx_status {
+    MX_OK = 0,
+    MX_ERR_INVALID_ARGUMENT = 1, /* NULL pointer, negative size, bad count */
+    MX_ERR_UNSUPPORTED_SHAPE = 2, /* K not a multiple of 32 (quantiser) / 128 (GEMM), N % 16 != 0 */
+    MX_ERR_MISALIGNED = 3,       /* a pointer not 16-byte aligned */
+    MX_ERR_CUDA = 4              /* a CUDA runtime / driver call failed */
+} mx_status;
+
+/* Device-side status bits (OR-ed into *dev_status). */
+#define MX_DEV_BAD_OFFSETS 0x1 /* group_offsets not monotone, not multiples of 128, or > m_total */
+#define MX_DEV_BAD_MASK 0x2    /* masked_m[e] outside [0, max_m] (clamped) */
+#define MX_DEV_TIMEOUT 0x4     /* an internal pipeline wait exceeded its limit; output invalid */
+
+/* Human-readable name of a status code; never NULL. */
+const char *mx_status_string(int status);
+
+/* Bytes of the tiled scale region for a [rows, k] operand:
+ * ceil(rows/128)*128 * ceil(k/32/4)*4.  Returns 0 for rows <= 0 or k <= 0. */
+size_t mx_scale_bytes(int64_t rows, int64_t k);
+
+/*
+ * BF16 -> MXFP8 quantisation along K.
+ *   x_bf16   [rows, k] BF16, row-major, 16-byte aligned.
+ *   q_e4m3   [rows, k] bytes out, 16-byte aligned.
+ *   sf_ue8m0 mx_scale_bytes(rows, k) bytes out (tiled layout above).
+ * Per 32-element block: amax over |x|; X = floor(log2 amax) - 8 clamped to
+ * [-127, 127] (amax = 0 gives X = -127); scale byte X+127; each element
+ * x*2^-X rounded to nearest-even and saturated to +-448.  A block holding a
+ * NaN or +-Inf gets scale 0xFF and elements 0x7F.  Requires k % 32 == 0.
+ * rows == 0 is a no-op.
+ */
+mx_status mx_quantize_bf16_to_e4m3(const void *x_bf16, int64_t rows, int64_t k, void *q_e4m3,
+                                   void *sf_ue8m0, mx_stream_t stream);
+
+/*
+ * Same as mx_quantize_bf16_to_e4m3 for a 3-D [groups, rows, k] tensor whose
+ * scales are stored per group: group g's scales start at
+ * g * mx_scale_bytes(rows, k).  (When rows % 128 == 0 this equals the 2-D
+ * call on groups*rows rows.)
+ */
+mx_status mx_quantize_bf16_to_e4m3_grouped(const void *x_bf16, int64_t groups, int64_t rows,
+                                           int64_t k, void *q_e4m3, void *sf_ue8m0,
+                                           mx_stream_t stream);
+
+/*
+ * Dense MXFP8 GEMM, D = A * B^T ("DeepGEMM" summary page: the plain FP8
+ * GEMM; the dense shapes of its CUTLASS comparison table).
+ *   qa [m, k], sfa = scales of A (mx_scale_bytes(m, k));
+ *   qb [n, k], sfb = scales of B (mx_scale_bytes(n, k));
+ *   d_bf16 [m, n] BF16 out.  FP32 accumulation, BF16 round-to-nearest-even.
+ * Requires k % 128 == 0, k > 0, n % 16 == 0, 16-byte aligned pointers.
+ * m == 0 or n == 0 is a no-op.
+ */
+mx_status mx_gemm(const void *qa, const void *sfa, const void *qb, const void *sfb, void *d_bf16,
+                  int64_t m, int64_t n, int64_t k, int32_t *dev_status, mx_stream_t stream);
+
+/*
+ * Contiguous-layout MoE grouped GEMM ("DeepGEMM" release page, section 4:
+ * token sequences of all experts grouped into one M dimension).
+ *   qa [m_total, k] holds the groups back to back; group e owns rows
+ *   [group_offsets[e], group_offsets[e+1]).  Every offset must be a multiple
+ *   of 128 (pad each group with rows; padded rows are multiplied like any
+ *   other row).  sfa = scales of the whole [m_total, k] operand.
+ *   qb [groups, n, k], sfb = groups back-to-back regions of
+ *   mx_scale_bytes(n, k) bytes.
+ *   group_offsets: DEVICE int32[groups + 1], read by the kernel (no host
+ *   synchronisation).
+ *   d_bf16 [m_total, n]: rows inside a group are written; rows at or beyond
+ *   group_offsets[groups] are left untouched.
+ */
+mx_status mx_grouped_gemm_contiguous(const void *qa, const void *sfa, const void *qb,
+                                     const void *sfb, const int32_t *group_offsets,
+                                     int32_t groups, int64_t m_total, int64_t n, int64_t k,
+                                     void *d_bf16, int32_t *dev_status, mx_stream_t stream);
+
+/*
+ * Masked-layout MoE grouped GEMM ("DeepGEMM" release page, section 4:
+ * efficient when expert activation is sparse).
+ *   qa [groups, max_m, k], sfa = groups back-to-back regions of
+ *   mx_scale_bytes(max_m, k) bytes; qb [groups, n, k], sfb likewise with
+ *   mx_scale_bytes(n, k).  masked_m: DEVICE int32[groups], valid rows of
+ *   each group.  d_bf16 [groups, max_m, n]: for group e only rows
+ *   r < masked_m[e] are written; all other rows are left untouched (their
+ *   A rows may hold anything, NaN included).
+ */
+mx_status mx_grouped_gemm_masked(const void *qa, const void *sfa, const void *qb,
+                                 const void *sfb, const int32_t *masked_m, int32_t groups,
+                                 int64_t max_m, int64_t n, int64_t k, void *d_bf16,
+                                 int32_t *dev_status, mx_stream_t stream);
+
+/* Copies the library-internal device status word (used when a call got
+ * dev_status == NULL) to *host_out and, if clear != 0, resets it.
+ * Synchronises the device. */
+mx_status mx_read_internal_status(int32_t *host_out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MX_H */

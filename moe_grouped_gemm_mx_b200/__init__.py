@@ -1,0 +1,210 @@
+"""MXFP8 quantisation, dense GEMM and MoE grouped GEMMs on B200 (sm_100a).
+
+A thin ctypes binding over ``libmx.so`` (declared in ``include/mx.h``): it
+only checks tensor dtypes/devices, allocates outputs with torch when the
+caller does not pass them, and forwards raw device pointers plus the current
+CUDA stream.  Every arithmetic step runs in the library's CUDA kernels; there
+is no CPU or PyTorch fallback -- if the library is missing, importing this
+package raises.
+
+Function names match the C ABI:
+
+    q, sf = mx_quantize_bf16_to_e4m3(x)                 # x: bf16 [..., K] (3-D -> per-group scales)
+    d     = mx_gemm(qa, sfa, qb, sfb)                   # D = A B^T, bf16 [M, N]
+    d     = mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, group_offsets)
+    d     = mx_grouped_gemm_masked(qa, sfa, qb, sfb, masked_m)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "MXError", "lib_path", "scale_bytes", "mx_quantize_bf16_to_e4m3", "mx_gemm",
+    "mx_grouped_gemm_contiguous", "mx_grouped_gemm_masked", "read_internal_status",
+    "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "C_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libmx.so")
+
+MX_DEV_BAD_OFFSETS = 0x1
+MX_DEV_BAD_MASK = 0x2
+MX_DEV_TIMEOUT = 0x4
+
+# every symbol include/mx.h declares
+C_SYMBOLS = [
+    "mx_status_string", "mx_scale_bytes", "mx_quantize_bf16_to_e4m3",
+    "mx_quantize_bf16_to_e4m3_grouped", "mx_gemm", "mx_grouped_gemm_contiguous",
+    "mx_grouped_gemm_masked", "mx_read_internal_status",
+]
+
+
+class MXError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib.mx_status_string(status).decode()} ({status})")
+
+
+def _load():
+    if not os.path.exists(lib_path):
+        raise ImportError(
+            f"moe_grouped_gemm_mx_b200: CUDA library {lib_path} is missing; build it with "
+            "`python -m moe_grouped_gemm_mx_b200._build` (or __graft_entry__.build())")
+    L = ctypes.CDLL(lib_path)
+    P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    L.mx_status_string.argtypes = [ctypes.c_int]
+    L.mx_status_string.restype = ctypes.c_char_p
+    L.mx_scale_bytes.argtypes = [I64, I64]
+    L.mx_scale_bytes.restype = ctypes.c_size_t
+    L.mx_quantize_bf16_to_e4m3.argtypes = [P, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3.restype = ctypes.c_int
+    L.mx_quantize_bf16_to_e4m3_grouped.argtypes = [P, I64, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3_grouped.restype = ctypes.c_int
+    L.mx_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
+    L.mx_gemm.restype = ctypes.c_int
+    L.mx_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
+    L.mx_grouped_gemm_contiguous.restype = ctypes.c_int
+    L.mx_grouped_gemm_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
+    L.mx_grouped_gemm_masked.restype = ctypes.c_int
+    L.mx_read_internal_status.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
+    L.mx_read_internal_status.restype = ctypes.c_int
+    return L
+
+
+_lib = _load()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _check(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _raise(st: int, what: str):
+    if st != 0:
+        raise MXError(st, what)
+
+
+def scale_bytes(rows: int, k: int) -> int:
+    """Bytes of the tiled UE8M0 scale region of a [rows, k] operand."""
+    return int(_lib.mx_scale_bytes(rows, k))
+
+
+def mx_quantize_bf16_to_e4m3(x: torch.Tensor, q: torch.Tensor | None = None,
+                             sf: torch.Tensor | None = None, stream=None):
+    """BF16 [rows, K] or [groups, rows, K] -> (q uint8 same shape, sf uint8 tiled).
+
+    For a 3-D input the scales are stored per group (each group a
+    ``scale_bytes(rows, K)`` region, back to back)."""
+    _check(x, torch.bfloat16, "x")
+    if x.dim() not in (2, 3):
+        raise ValueError("x must be 2-D [rows, K] or 3-D [groups, rows, K]")
+    groups = 1 if x.dim() == 2 else x.shape[0]
+    rows, k = x.shape[-2], x.shape[-1]
+    if q is None:
+        q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(groups * scale_bytes(rows, k), dtype=torch.uint8, device=x.device)
+    _check(q, torch.uint8, "q")
+    _check(sf, torch.uint8, "sf")
+    if q.numel() != x.numel() or sf.numel() < groups * scale_bytes(rows, k):
+        raise ValueError("output buffers too small")
+    if x.dim() == 2:
+        st = _lib.mx_quantize_bf16_to_e4m3(_ptr(x), rows, k, _ptr(q), _ptr(sf), _stream(stream))
+    else:
+        st = _lib.mx_quantize_bf16_to_e4m3_grouped(_ptr(x), groups, rows, k, _ptr(q), _ptr(sf),
+                                                   _stream(stream))
+    _raise(st, "mx_quantize_bf16_to_e4m3")
+    return q, sf
+
+
+def _status_arg(dev_status):
+    if dev_status is None:
+        return None
+    _check(dev_status, torch.int32, "dev_status")
+    return dev_status.data_ptr()
+
+
+def mx_gemm(qa, sfa, qb, sfb, d: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """D = deq(A) deq(B)^T, qa uint8 [M, K], qb uint8 [N, K] -> bf16 [M, N]."""
+    for t, nm in ((qa, "qa"), (sfa, "sfa"), (qb, "qb"), (sfb, "sfb")):
+        _check(t, torch.uint8, nm)
+    m, k = qa.shape
+    n = qb.shape[0]
+    if qb.shape[1] != k:
+        raise ValueError("K mismatch")
+    if d is None:
+        d = torch.empty((m, n), dtype=torch.bfloat16, device=qa.device)
+    _check(d, torch.bfloat16, "d")
+    st = _lib.mx_gemm(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(d), m, n, k,
+                      _status_arg(dev_status), _stream(stream))
+    _raise(st, "mx_gemm")
+    return d
+
+
+def mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, group_offsets: torch.Tensor,
+                               d: torch.Tensor | None = None,
+                               dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """qa uint8 [M_total, K], qb uint8 [E, N, K], group_offsets int32 [E+1] (device)."""
+    for t, nm in ((qa, "qa"), (sfa, "sfa"), (qb, "qb"), (sfb, "sfb")):
+        _check(t, torch.uint8, nm)
+    _check(group_offsets, torch.int32, "group_offsets")
+    m_total, k = qa.shape
+    groups, n, kb = qb.shape
+    if kb != k or group_offsets.numel() != groups + 1:
+        raise ValueError("shape mismatch")
+    if d is None:
+        d = torch.empty((m_total, n), dtype=torch.bfloat16, device=qa.device)
+    _check(d, torch.bfloat16, "d")
+    st = _lib.mx_grouped_gemm_contiguous(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(group_offsets),
+                                         groups, m_total, n, k, _ptr(d), _status_arg(dev_status),
+                                         _stream(stream))
+    _raise(st, "mx_grouped_gemm_contiguous")
+    return d
+
+
+def mx_grouped_gemm_masked(qa, sfa, qb, sfb, masked_m: torch.Tensor, d: torch.Tensor | None = None,
+                           dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """qa uint8 [E, max_m, K], qb uint8 [E, N, K], masked_m int32 [E] (device)."""
+    for t, nm in ((qa, "qa"), (sfa, "sfa"), (qb, "qb"), (sfb, "sfb")):
+        _check(t, torch.uint8, nm)
+    _check(masked_m, torch.int32, "masked_m")
+    groups, max_m, k = qa.shape
+    g2, n, kb = qb.shape
+    if g2 != groups or kb != k or masked_m.numel() != groups:
+        raise ValueError("shape mismatch")
+    if d is None:
+        d = torch.empty((groups, max_m, n), dtype=torch.bfloat16, device=qa.device)
+    _check(d, torch.bfloat16, "d")
+    st = _lib.mx_grouped_gemm_masked(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(masked_m), groups,
+                                     max_m, n, k, _ptr(d), _status_arg(dev_status), _stream(stream))
+    _raise(st, "mx_grouped_gemm_masked")
+    return d
+
+
+def read_internal_status(clear: bool = True) -> int:
+    """Device-status bits accumulated by calls made without ``dev_status``."""
+    out = ctypes.c_int32(0)
+    _raise(_lib.mx_read_internal_status(ctypes.byref(out), int(clear)), "mx_read_internal_status")
+    return int(out.value)

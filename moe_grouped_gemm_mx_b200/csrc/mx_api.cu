@@ -1,0 +1,162 @@
+// mx_api.cu -- the extern "C" boundary declared in include/mx.h: argument
+// validation, then one kernel launch per call on the caller's stream.  No
+// memory is allocated per call; the only device memory the library owns is the
+// 4-byte internal status word below.
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/mx.h"
+
+#include "mx_launch.h"
+
+namespace {
+
+constexpr int64_t kMaxGroups = 1024;
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+__device__ int32_t g_internal_status = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static int cached_dev = -1, cached = 0;
+  if (dev != cached_dev) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached = v;
+    cached_dev = dev;
+  }
+  return cached;
+}
+
+int32_t* internal_status_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_internal_status) != cudaSuccess) return nullptr;
+  return static_cast<int32_t*>(p);
+}
+
+mx_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mx_status_string(int status) {
+  switch (status) {
+    case MX_OK: return "MX_OK";
+    case MX_ERR_INVALID_ARGUMENT: return "MX_ERR_INVALID_ARGUMENT";
+    case MX_ERR_UNSUPPORTED_SHAPE: return "MX_ERR_UNSUPPORTED_SHAPE";
+    case MX_ERR_MISALIGNED: return "MX_ERR_MISALIGNED";
+    case MX_ERR_CUDA: return "MX_ERR_CUDA";
+    default: return "MX_ERR_UNKNOWN";
+  }
+}
+
+size_t mx_scale_bytes(int64_t rows, int64_t k) {
+  if (rows <= 0 || k <= 0) return 0;
+  const int64_t kb = (k + 31) / 32;
+  return static_cast<size_t>(((rows + 127) / 128) * 128 * ((kb + 3) / 4) * 4);
+}
+
+static mx_status quantize_impl(const void* x, int64_t groups, int64_t rows, int64_t k, void* q, void* sf,
+                               mx_stream_t stream) {
+  if (groups < 0 || rows < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k % 32 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (groups == 0 || rows == 0 || k == 0) return MX_OK;
+  if (!x || !q || !sf) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return MX_ERR_MISALIGNED;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  return from_cuda(mxk::launch_quant(x, groups, rows, k, q, sf, static_cast<int64_t>(mx_scale_bytes(rows, k)),
+                                     sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+mx_status mx_quantize_bf16_to_e4m3(const void* x_bf16, int64_t rows, int64_t k, void* q_e4m3, void* sf_ue8m0,
+                                   mx_stream_t stream) {
+  return quantize_impl(x_bf16, 1, rows, k, q_e4m3, sf_ue8m0, stream);
+}
+
+mx_status mx_quantize_bf16_to_e4m3_grouped(const void* x_bf16, int64_t groups, int64_t rows, int64_t k,
+                                           void* q_e4m3, void* sf_ue8m0, mx_stream_t stream) {
+  return quantize_impl(x_bf16, groups, rows, k, q_e4m3, sf_ue8m0, stream);
+}
+
+static mx_status check_gemm_common(const void* qa, const void* sfa, const void* qb, const void* sfb, void* d,
+                                   int64_t m, int64_t n, int64_t k, int64_t groups) {
+  if (m < 0 || n < 0 || k < 0 || groups < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k == 0 || k % 128 != 0 || n % 16 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (m > kMaxDim || n > kMaxDim || k > kMaxDim || groups > kMaxGroups) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (!qa || !sfa || !qb || !sfb || !d) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(qa) || !aligned16(sfa) || !aligned16(qb) || !aligned16(sfb) || !aligned16(d))
+    return MX_ERR_MISALIGNED;
+  return MX_OK;
+}
+
+mx_status mx_gemm(const void* qa, const void* sfa, const void* qb, const void* sfb, void* d_bf16, int64_t m,
+                  int64_t n, int64_t k, int32_t* dev_status, mx_stream_t stream) {
+  if (m < 0 || n < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (m == 0 || n == 0) {
+    if (k % 128 != 0 || k == 0 || n % 16 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+    return MX_OK;
+  }
+  mx_status st = check_gemm_common(qa, sfa, qb, sfb, d_bf16, m, n, k, 1);
+  if (st != MX_OK) return st;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  mxk::GemmProblem p{qa, sfa, qb, sfb, d_bf16, nullptr, nullptr, status, m, n, k, 1, 0};
+  return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+mx_status mx_grouped_gemm_contiguous(const void* qa, const void* sfa, const void* qb, const void* sfb,
+                                     const int32_t* group_offsets, int32_t groups, int64_t m_total, int64_t n,
+                                     int64_t k, void* d_bf16, int32_t* dev_status, mx_stream_t stream) {
+  if (groups < 0 || m_total < 0 || n < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k == 0 || k % 128 != 0 || n % 16 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (groups == 0 || m_total == 0 || n == 0) return MX_OK;
+  if (!group_offsets) return MX_ERR_INVALID_ARGUMENT;
+  mx_status st = check_gemm_common(qa, sfa, qb, sfb, d_bf16, m_total, n, k, groups);
+  if (st != MX_OK) return st;
+  if (reinterpret_cast<uintptr_t>(group_offsets) & 3u) return MX_ERR_MISALIGNED;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  mxk::GemmProblem p{qa, sfa, qb, sfb, d_bf16, group_offsets, nullptr, status, m_total, n, k, groups, 1};
+  return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+mx_status mx_grouped_gemm_masked(const void* qa, const void* sfa, const void* qb, const void* sfb,
+                                 const int32_t* masked_m, int32_t groups, int64_t max_m, int64_t n, int64_t k,
+                                 void* d_bf16, int32_t* dev_status, mx_stream_t stream) {
+  if (groups < 0 || max_m < 0 || n < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k == 0 || k % 128 != 0 || n % 16 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (groups == 0 || max_m == 0 || n == 0) return MX_OK;
+  if (!masked_m) return MX_ERR_INVALID_ARGUMENT;
+  if (groups * max_m > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  mx_status st = check_gemm_common(qa, sfa, qb, sfb, d_bf16, max_m, n, k, groups);
+  if (st != MX_OK) return st;
+  if (reinterpret_cast<uintptr_t>(masked_m) & 3u) return MX_ERR_MISALIGNED;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  mxk::GemmProblem p{qa, sfa, qb, sfb, d_bf16, nullptr, masked_m, status, max_m, n, k, groups, 2};
+  return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+mx_status mx_read_internal_status(int32_t* host_out, int clear) {
+  if (!host_out) return MX_ERR_INVALID_ARGUMENT;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MX_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(host_out, g_internal_status, sizeof(int32_t)) != cudaSuccess) return MX_ERR_CUDA;
+  if (clear) {
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_internal_status, &zero, sizeof(int32_t)) != cudaSuccess) return MX_ERR_CUDA;
+  }
+  return MX_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,484 @@
+// mx_gemm.cu -- MXFP8 block-scaled GEMM kernels for sm_100a (B200).
+//
+// One persistent, warp-specialised kernel serves the three GEMM forms the
+// DeepGEMM pages list ("DeepGEMM" summary page: a plain FP8 GEMM plus MoE
+// grouped GEMMs in contiguous and masked layouts; DeepGEMM release page,
+// section 4), in the MXFP8 number format of the B200 MoE-training page
+// (32-element UE8M0 block scales, FP32 accumulation, BF16 output).
+//
+//   D[m, n] = sum_b 2^(sa[m,b] + sb[n,b]) * sum_{k in b} e4m3(qa[m,k]) * e4m3(qb[n,k])
+//
+// CTA layout (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A/B tiles (128-byte swizzled, 3-D tensor maps so
+//               experts never bleed into each other) and the 512-byte scale
+//               tiles (plain bulk copies) into a STAGES-deep shared-memory ring.
+//   warp 1      TMEM owner + MMA issuer: per K-tile, tcgen05.cp the scale tiles
+//               into TMEM, then 4 x tcgen05.mma kind::mxf8f6f4.block_scale
+//               (K = 32 each, scale byte k selected by the scale-factor ids),
+//               accumulating a 128 x BN FP32 tile in TMEM.  tcgen05.commit
+//               frees ring slots and publishes finished accumulators.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (each warp owns the TMEM
+//               lane quarter its warp id selects), round to BF16 and store the
+//               valid rows/columns.
+// The tile scheduler is a static stride over a linear tile index; grouped
+// forms map the index to (expert, m-block, n-block) with a table built in
+// shared memory from the device-resident offsets / masks, so no host
+// synchronisation is needed.  The Hopper-era two-level CUDA-core accumulation
+// of the pages is unnecessary here: the tensor core accumulates in FP32 in TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "mx_launch.h"
+#include "mx_ptx.cuh"
+
+namespace mxk {
+
+constexpr int BM = 128;              // MMA M (rows of A per tile)
+constexpr int BK = 128;              // K elements per pipeline stage (4 scale blocks)
+constexpr int kMaxGroups = 1024;
+constexpr int kGemmThreads = 192;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+
+enum GemmMode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+
+struct GemmArgs {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  __nv_bfloat16* d;
+  const int32_t* group_offsets;  // contiguous: [groups+1]
+  const int32_t* masked_m;       // masked: [groups]
+  int32_t* status;
+  int64_t sfa_group_bytes;  // masked: tiled scale bytes per expert of A
+  int64_t sfb_group_bytes;  // grouped: tiled scale bytes per expert of B
+  int m;                    // dense: M; contiguous: m_total; masked: max_m
+  int n;
+  int k_tiles;              // K / 128 (also the 512-byte scale tiles per 128-row block)
+  int n_tiles;              // ceil(N / BN)
+  int n_sf_tiles;           // ceil(N / 128)
+  int groups;
+  int mode;
+};
+
+template <int BN, int STAGES, int ACC>
+struct Layout {
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int SFA_BYTES = 512;
+  static constexpr int SFB_TILES = BN / 128;
+  static constexpr int SFB_BYTES = SFB_TILES * 512;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+  static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC + 1;  // + drain barrier
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_TAB0 = OFF_MISC + 16;
+  static constexpr int OFF_TAB1 = OFF_TAB0 + (kMaxGroups + 1) * 4;
+  static constexpr int BYTES = OFF_TAB1 + (kMaxGroups + 1) * 4;
+  static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024 B
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t SFA_COL = ACC * BN;
+  static constexpr uint32_t SFB_COL = SFA_COL + 4;
+  static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
+  static_assert(SFB_COL + 4 * SFB_TILES <= TMEM_COLS, "TMEM budget");
+  static_assert(OFF_B % 1024 == 0 && OFF_SFA % 1024 == 0, "swizzled tiles need 1024-B alignment");
+  static_assert(BYTES + 1024 <= 232448, "shared memory budget");
+};
+
+struct Tile {
+  int group;
+  int m_blk;  // 128-row block inside the group (masked) or inside A (dense/contiguous)
+  int n_blk;
+};
+
+// Index of the last entry <= v in the non-decreasing table t[0..n] (n+1 entries).
+__device__ __forceinline__ int last_le(const int32_t* t, int n, int32_t v) {
+  int lo = 0, hi = n;  // invariant: t[lo] <= v
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (t[mid] <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int32_t* tab0, int t) {
+  Tile r;
+  if (a.mode == kMasked) {
+    const int e = last_le(tab0, a.groups, t);  // tab0 = prefix of tiles per expert
+    const int local = t - tab0[e];
+    r.group = e;
+    r.m_blk = local / a.n_tiles;
+    r.n_blk = local - r.m_blk * a.n_tiles;
+  } else {
+    const int mb = t / a.n_tiles;
+    r.n_blk = t - mb * a.n_tiles;
+    if (a.mode == kContiguous) {
+      r.m_blk = tab0[0] / BM + mb;                               // tab0 = group offsets
+      r.group = last_le(tab0, a.groups, r.m_blk * BM);
+      if (r.group >= a.groups) r.group = a.groups - 1;
+    } else {
+      r.m_blk = mb;
+      r.group = 0;
+    }
+  }
+  return r;
+}
+
+__device__ __forceinline__ void report(int32_t* status, int bits) {
+  atomicOr(status, bits);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(lo_f32), __uint_as_float(hi_f32));
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int BN, int STAGES, int ACC>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                   const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+  using L = Layout<BN, STAGES, ACC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile uint32_t* tmem_slot = misc + 0;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* total_slot = reinterpret_cast<volatile int*>(misc + 2);
+  int32_t* tab0 = reinterpret_cast<int32_t*>(smem + L::OFF_TAB0);
+  int32_t* tab1 = reinterpret_cast<int32_t*>(smem + L::OFF_TAB1);
+
+  auto full_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * s; };
+  auto empty_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (STAGES + s); };
+  auto accf_bar = [&](int a) { return sbase + L::OFF_BAR + 8u * (2 * STAGES + a); };
+  auto acce_bar = [&](int a) { return sbase + L::OFF_BAR + 8u * (2 * STAGES + ACC + a); };
+  const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 2 * ACC);
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < ACC; ++a) {
+      mbar_init(accf_bar(a), 1);
+      mbar_init(acce_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+
+  // scheduling tables
+  int bad = 0;
+  if (args.mode == kContiguous) {
+    for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) tab0[i] = __ldg(args.group_offsets + i);
+    __syncthreads();
+    for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) {
+      const int32_t v = tab0[i];
+      if (v < 0 || (v % BM) != 0 || v > args.m) bad = 1;
+      if (i > 0 && v < tab0[i - 1]) bad = 1;
+    }
+  } else if (args.mode == kMasked) {
+    for (int i = threadIdx.x; i < args.groups; i += blockDim.x) {
+      int32_t mm = __ldg(args.masked_m + i);
+      if (mm < 0 || mm > args.m) {
+        bad = 1;
+        mm = mm < 0 ? 0 : args.m;
+      }
+      tab1[i] = mm;
+    }
+    __syncthreads();
+    if (warp == 0) {  // exclusive prefix of tiles per expert, one warp
+      const int per = (args.groups + 31) / 32;
+      const int lo = lane * per;
+      int sum = 0;
+      for (int i = lo; i < lo + per && i < args.groups; ++i) sum += (tab1[i] + BM - 1) / BM * args.n_tiles;
+      int incl = sum;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int run = incl - sum;
+      for (int i = lo; i < lo + per && i < args.groups; ++i) {
+        tab0[i] = run;
+        run += (tab1[i] + BM - 1) / BM * args.n_tiles;
+      }
+      if (lane == 31) tab0[args.groups] = incl;
+    }
+  }
+  const int any_bad = __syncthreads_or(bad);
+
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    int total;
+    if (args.mode == kDense) {
+      total = ((args.m + BM - 1) / BM) * args.n_tiles;
+    } else if (args.mode == kContiguous) {
+      total = any_bad ? 0 : (tab0[args.groups] - tab0[0]) / BM * args.n_tiles;
+      if (any_bad) report(args.status, 0x1);
+    } else {
+      total = tab0[args.groups];
+      if (any_bad) report(args.status, 0x2);
+    }
+    *total_slot = total;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = *total_slot;
+
+  // ---------------------------------------------------------------- roles
+  if (warp == 0) {
+    if (lane == 0) {
+      // ===== TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(args, tab0, t);
+        const int a_row = tl.m_blk * BM;
+        const int a_z = (args.mode == kMasked) ? tl.group : 0;
+        const int b_z = (args.mode == kDense) ? 0 : tl.group;
+        const uint8_t* sfa_base = args.sfa + (args.mode == kMasked ? tl.group * args.sfa_group_bytes : 0) +
+                                  static_cast<int64_t>(tl.m_blk) * args.k_tiles * 512;
+        const uint8_t* sfb_grp = args.sfb + (args.mode == kDense ? 0 : tl.group * args.sfb_group_bytes);
+        const int sfb_tile0 = tl.n_blk * L::SFB_TILES;
+        int nsfb = args.n_sf_tiles - sfb_tile0;
+        nsfb = nsfb > L::SFB_TILES ? L::SFB_TILES : nsfb;
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          const uint32_t bytes = L::A_BYTES + L::B_BYTES + L::SFA_BYTES + 512u * nsfb;
+          mbar_arrive_expect_tx(full_bar(stage), bytes);
+          tma_load_3d(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, full_bar(stage), kt * BK, a_row, a_z);
+          tma_load_3d(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, full_bar(stage), kt * BK,
+                      tl.n_blk * BN, b_z);
+          bulk_load(sbase + L::OFF_SFA + stage * L::SFA_BYTES, sfa_base + kt * 512, 512, full_bar(stage));
+          for (int j = 0; j < nsfb; ++j)
+            bulk_load(sbase + L::OFF_SFB + stage * L::SFB_BYTES + j * 512,
+                      sfb_grp + (static_cast<int64_t>(sfb_tile0 + j) * args.k_tiles + kt) * 512, 512,
+                      full_bar(stage));
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        report(args.status, 0x4);
+        *abort_flag = 1;
+        // give copies already in flight time to land before the CTA can exit
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 1000000ull) { }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ===== MMA issuer
+      const uint32_t idesc0 = idesc_mxf8_e4m3(BM, BN);
+      const uint32_t sfa_t = tmem_base + L::SFA_COL;
+      const uint32_t sfb_t = tmem_base + L::SFB_COL;
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_t = tmem_base + acc * BN;
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          tc_cp_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + stage * L::SFA_BYTES));
+#pragma unroll
+          for (int j = 0; j < L::SFB_TILES; ++j)
+            tc_cp_32x128b_warpx4(sfb_t + 4 * j,
+                                 desc_sf_32x16(sbase + L::OFF_SFB + stage * L::SFB_BYTES + j * 512));
+          const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES;
+          const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint32_t idesc = idesc_with_sf_ids(idesc0, kb, kb);
+            tc_mma_mxf8(d_t, desc_kmajor_sw128(a_addr + 32 * kb), desc_kmajor_sw128(b_addr + 32 * kb), idesc,
+                        sfa_t | (static_cast<uint32_t>(kb) << 30), sfb_t | (static_cast<uint32_t>(kb) << 30),
+                        (kt | kb) != 0);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(acc));
+        if (++acc == ACC) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) {
+        report(args.status, 0x4);
+        *abort_flag = 1;
+        // every MMA / copy this thread issued must finish before TMEM is freed
+        tc_commit(drain_bar);
+        mbar_wait(drain_bar, 0, nullptr, 100000000ull);
+      }
+    }
+  } else {
+    // ===== epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
+    const int quarter = warp & 3;
+    const int r_local = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      // every lane polls; the vote re-converges the warp before the
+      // warp-collective (.sync.aligned) TMEM loads below
+      const bool got = mbar_wait(accf_bar(acc), acc_phase, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xFFFFFFFFu, got)) {
+        if (lane == 0) report(args.status, 0x4);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const Tile tl = decode_tile(args, tab0, t);
+      int64_t drow;
+      bool valid;
+      if (args.mode == kMasked) {
+        const int r = tl.m_blk * BM + r_local;
+        valid = r < tab1[tl.group];
+        drow = static_cast<int64_t>(tl.group) * args.m + r;
+      } else {
+        const int r = tl.m_blk * BM + r_local;
+        valid = r < args.m;
+        drow = r;
+      }
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+      __nv_bfloat16* drow_ptr = args.d + drow * args.n;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tc_ld_32x32b_x32(t_row + c * 32, v);
+        tc_wait_ld();
+        const int col0 = tl.n_blk * BN + c * 32;
+        if (valid) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = col0 + g * 8;
+            if (col < args.n) {
+              uint4 w;
+              w.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+              w.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+              w.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+              w.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+              *reinterpret_cast<uint4*>(drow_ptr + col) = w;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acce_bar(acc));
+      if (++acc == ACC) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+// ======================================================================= host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D byte tensor [depth, rows, k] (k contiguous) read in boxes of box_rows x 128 bytes.
+static bool make_tmap(CUtensorMap* m, const void* base, int64_t k, int64_t rows, int64_t depth, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(depth)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(k * rows)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, int ACC>
+static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
+  using L = Layout<BN, STAGES, ACC>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(mx_gemm_kernel<BN, STAGES, ACC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  CUtensorMap ta, tb;
+  const int64_t a_depth = p.mode == kMasked ? p.groups : 1;
+  const int64_t b_depth = p.mode == kDense ? 1 : p.groups;
+  if (!make_tmap(&ta, p.qa, p.k, p.m, a_depth, BM)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tb, p.qb, p.k, p.n, b_depth, BN)) return cudaErrorInvalidValue;
+
+  GemmArgs a;
+  a.sfa = static_cast<const uint8_t*>(p.sfa);
+  a.sfb = static_cast<const uint8_t*>(p.sfb);
+  a.d = static_cast<__nv_bfloat16*>(p.d);
+  a.group_offsets = p.group_offsets;
+  a.masked_m = p.masked_m;
+  a.status = p.status;
+  a.k_tiles = static_cast<int>(p.k / BK);
+  a.sfa_group_bytes = ((p.m + 127) / 128) * 128 * (p.k / 32);
+  a.sfb_group_bytes = ((p.n + 127) / 128) * 128 * (p.k / 32);
+  a.m = static_cast<int>(p.m);
+  a.n = static_cast<int>(p.n);
+  a.n_tiles = static_cast<int>((p.n + BN - 1) / BN);
+  a.n_sf_tiles = static_cast<int>((p.n + 127) / 128);
+  a.groups = static_cast<int>(p.groups);
+  a.mode = p.mode;
+
+  int64_t m_tiles_bound;
+  if (p.mode == kMasked)
+    m_tiles_bound = p.groups * ((p.m + BM - 1) / BM);
+  else
+    m_tiles_bound = (p.m + BM - 1) / BM;
+  const int64_t tiles_bound = m_tiles_bound * a.n_tiles;
+  if (tiles_bound == 0) return cudaSuccess;
+  const int grid = static_cast<int>(tiles_bound < num_sms ? tiles_bound : num_sms);
+  mx_gemm_kernel<BN, STAGES, ACC><<<grid, kGemmThreads, L::ALLOC, stream>>>(ta, tb, a);
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
+  return launch_gemm_cfg<256, 4, 1>(p, num_sms, stream, launches);
+}
+
+}  // namespace mxk

@@ -1,0 +1,28 @@
+// mx_launch.h -- host-side launch entry points shared by the C ABI (mx_api.cu)
+// and the kernel translation units.  Internal to the library.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace mxk {
+
+cudaError_t launch_quant(const void* x, int64_t groups, int64_t rows, int64_t k, void* q, void* sf,
+                         int64_t sf_group_bytes, int num_sms, cudaStream_t stream, int* launches);
+
+struct GemmProblem {
+  const void* qa;
+  const void* sfa;
+  const void* qb;
+  const void* sfb;
+  void* d;
+  const int32_t* group_offsets;  // contiguous form only (device, groups + 1)
+  const int32_t* masked_m;       // masked form only (device, groups)
+  int32_t* status;               // device status word, never null
+  int64_t m, n, k;               // m: dense M / contiguous m_total / masked max_m
+  int64_t groups;                // experts (1 for the dense form)
+  int mode;                      // 0 dense, 1 contiguous, 2 masked
+};
+
+cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches);
+
+}  // namespace mxk

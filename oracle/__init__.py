@@ -68,7 +68,7 @@ def lib():
         L.mxo_gemm.restype = None
         L.mxo_grouped_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, P, I64, P, P]
         L.mxo_grouped_contiguous.restype = None
-        L.mxo_grouped_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P]
+        L.mxo_grouped_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, I64, P, P]
         L.mxo_grouped_masked.restype = None
         L.mxo_num_threads.argtypes = []
         L.mxo_num_threads.restype = ctypes.c_int
@@ -200,8 +200,11 @@ def grouped_contiguous(qa, sfa, qb, sfb, offsets, rows=None):
     return d, a
 
 
-def grouped_masked(qa, sfa, qb, sfb, masked_m):
-    """qa [groups, max_m, k], qb [groups, n, k]; rows >= masked_m[e] are NaN."""
+def grouped_masked(qa, sfa, qb, sfb, masked_m, rows=None):
+    """qa [groups, max_m, k], qb [groups, n, k]; rows >= masked_m[e] are NaN.
+
+    Without ``rows`` returns (d, abssum) of shape [groups, max_m, n]; with
+    ``rows`` (flat indices e*max_m + r) returns [len(rows), n]."""
     qa = np.ascontiguousarray(qa, dtype=np.uint8)
     qb = np.ascontiguousarray(qb, dtype=np.uint8)
     sfa = np.ascontiguousarray(sfa, dtype=np.uint8)
@@ -209,10 +212,14 @@ def grouped_masked(qa, sfa, qb, sfb, masked_m):
     mm = np.ascontiguousarray(masked_m, dtype=np.int32)
     groups, max_m, k = qa.shape
     n = qb.shape[1]
-    d = np.zeros((groups, max_m, n), dtype=np.float64)
-    a = np.zeros((groups, max_m, n), dtype=np.float64)
+    ids = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = groups * max_m if ids is None else len(ids)
+    d = np.zeros((nrows, n), dtype=np.float64)
+    a = np.zeros((nrows, n), dtype=np.float64)
     lib().mxo_grouped_masked(_p(qa), _p(sfa), _p(qb), _p(sfb), _p(mm), groups, max_m, n, k,
-                             _p(d), _p(a))
+                             _p(ids), nrows, _p(d), _p(a))
+    if ids is None:
+        return d.reshape(groups, max_m, n), a.reshape(groups, max_m, n)
     return d, a
 
 

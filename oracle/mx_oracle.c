@@ -233,14 +233,23 @@ void mxo_sf_untile(const uint8_t *tiled, int64_t rows, int64_t k, uint8_t *sf_rm
 
 /* ------------------------------------------------------------------ GEMM */
 
-static double deq(const double *tab, uint8_t qv, uint8_t sfv)
+/* Value tables: the 256 E4M3 codes and the 256 UE8M0 codes (2^(c-127),
+ * 0xFF = NaN).  A dequantised element is tab[q] * stab[sf]. */
+struct mxo_tables {
+    double tab[256];
+    double stab[256];
+};
+
+static void fill_tables(struct mxo_tables *t)
 {
-    return tab[qv] * mxo_ue8m0_decode(sfv);
+    mxo_e4m3_table(t->tab);
+    for (int c = 0; c < 256; ++c)
+        t->stab[c] = mxo_ue8m0_decode((uint8_t)c);
 }
 
 /* One output row: d[j] = sum_k deq(a[i,k]) * deq(b[j,k]) for j < n, k
  * ascending, in double; abssum[j] = sum_k |deq(a) * deq(b)|. */
-static void gemm_row(const double *tab, const uint8_t *qa_row, const uint8_t *sfa_row,
+static void gemm_row(const struct mxo_tables *t, const uint8_t *qa_row, const uint8_t *sfa_row,
                      const uint8_t *qb, const uint8_t *sfb, int64_t n, int64_t k,
                      double *d_row, double *abs_row)
 {
@@ -250,7 +259,9 @@ static void gemm_row(const double *tab, const uint8_t *qa_row, const uint8_t *sf
         const uint8_t *sfb_row = sfb + j * kb;
         double acc = 0.0, aacc = 0.0;
         for (int64_t kk = 0; kk < k; ++kk) {
-            double p = deq(tab, qa_row[kk], sfa_row[kk / 32]) * deq(tab, qb_row[kk], sfb_row[kk / 32]);
+            double a = t->tab[qa_row[kk]] * t->stab[sfa_row[kk / 32]];
+            double b = t->tab[qb_row[kk]] * t->stab[sfb_row[kk / 32]];
+            double p = a * b;
             acc += p;
             aacc += fabs(p);
         }
@@ -267,74 +278,80 @@ void mxo_gemm(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb, const ui
               int64_t m, int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows,
               double *d, double *abssum)
 {
-    double tab[256];
-    mxo_e4m3_table(tab);
+    struct mxo_tables t;
+    fill_tables(&t);
     int64_t kb = k / 32;
     if (!row_ids)
         nrows = m;
 #pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t t = 0; t < nrows; ++t) {
-        int64_t i = row_ids ? row_ids[t] : t;
-        gemm_row(tab, qa + i * k, sfa + i * kb, qb, sfb, n, k, d + t * n,
-                 abssum ? abssum + t * n : NULL);
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = row_ids ? row_ids[r] : r;
+        gemm_row(&t, qa + i * k, sfa + i * kb, qb, sfb, n, k, d + r * n,
+                 abssum ? abssum + r * n : NULL);
     }
 }
 
 /* Contiguous grouped GEMM: rows [off[e], off[e+1]) of A use expert e's B.
  * qb is [groups, n, k], sfb row-major [groups, n, k/32].  Only listed rows
- * (or all rows of all groups when row_ids is NULL, in which case nrows must
- * be off[groups]) are computed; a row outside every group gives NaN. */
+ * (or all rows 0..nrows-1 when row_ids is NULL) are computed; a row outside
+ * every group gives NaN (such rows are never written on the device). */
 void mxo_grouped_contiguous(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
                             const uint8_t *sfb, const int32_t *offsets, int32_t groups,
                             int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows,
                             double *d, double *abssum)
 {
-    double tab[256];
-    mxo_e4m3_table(tab);
+    struct mxo_tables t;
+    fill_tables(&t);
     int64_t kb = k / 32;
 #pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t t = 0; t < nrows; ++t) {
-        int64_t i = row_ids ? row_ids[t] : t;
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = row_ids ? row_ids[r] : r;
         int e = -1;
         for (int g = 0; g < groups; ++g)
             if (i >= offsets[g] && i < offsets[g + 1])
                 e = g;
         if (e < 0) {
             for (int64_t j = 0; j < n; ++j) {
-                d[t * n + j] = NAN;
+                d[r * n + j] = NAN;
                 if (abssum)
-                    abssum[t * n + j] = NAN;
+                    abssum[r * n + j] = NAN;
             }
             continue;
         }
-        gemm_row(tab, qa + i * k, sfa + i * kb, qb + (int64_t)e * n * k,
-                 sfb + (int64_t)e * n * kb, n, k, d + t * n, abssum ? abssum + t * n : NULL);
+        gemm_row(&t, qa + i * k, sfa + i * kb, qb + (int64_t)e * n * k, sfb + (int64_t)e * n * kb, n, k,
+                 d + r * n, abssum ? abssum + r * n : NULL);
     }
 }
 
-/* Masked grouped GEMM: A is [groups, max_m, k]; for group e only rows
- * r < masked_m[e] are products (d[e, r, :] = A[e, r, :] * B[e]^T); the
- * other rows are left as NaN here and must stay untouched on the device. */
+/* Masked grouped GEMM: A is [groups, max_m, k]; for expert e only rows
+ * r < masked_m[e] are products (d[e, r, :] = A[e, r, :] * B[e]^T).  Rows are
+ * addressed by flat index e*max_m + r: the listed ones, or all of them when
+ * row_ids is NULL (nrows = groups*max_m).  Rows at or beyond masked_m[e] give
+ * NaN here; on the device they must stay untouched. */
 void mxo_grouped_masked(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
                         const uint8_t *sfb, const int32_t *masked_m, int32_t groups,
-                        int64_t max_m, int64_t n, int64_t k, double *d, double *abssum)
+                        int64_t max_m, int64_t n, int64_t k, const int64_t *row_ids,
+                        int64_t nrows, double *d, double *abssum)
 {
-    double tab[256];
-    mxo_e4m3_table(tab);
+    struct mxo_tables t;
+    fill_tables(&t);
     int64_t kb = k / 32;
+    if (!row_ids)
+        nrows = (int64_t)groups * max_m;
 #pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t t = 0; t < (int64_t)groups * max_m; ++t) {
-        int64_t e = t / max_m, r = t % max_m;
-        if (r >= masked_m[e]) {
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t flat = row_ids ? row_ids[r] : r;
+        int64_t e = flat / max_m, i = flat % max_m;
+        if (i >= masked_m[e]) {
             for (int64_t j = 0; j < n; ++j) {
-                d[t * n + j] = NAN;
+                d[r * n + j] = NAN;
                 if (abssum)
-                    abssum[t * n + j] = NAN;
+                    abssum[r * n + j] = NAN;
             }
             continue;
         }
-        gemm_row(tab, qa + t * k, sfa + t * kb, qb + e * n * k, sfb + e * n * kb, n, k,
-                 d + t * n, abssum ? abssum + t * n : NULL);
+        gemm_row(&t, qa + flat * k, sfa + flat * kb, qb + e * n * k, sfb + e * n * kb, n, k,
+                 d + r * n, abssum ? abssum + r * n : NULL);
     }
 }
 

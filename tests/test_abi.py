@@ -1,0 +1,99 @@
+"""CPU-only checks of the C ABI: the library loads without a GPU, exports
+every function include/mx.h declares, and rejects bad arguments on the host
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mx.h")
+LIB = os.path.join(ROOT, "moe_grouped_gemm_mx_b200", "libmx.so")
+
+MX_OK, MX_ERR_INVALID_ARGUMENT, MX_ERR_UNSUPPORTED_SHAPE, MX_ERR_MISALIGNED = 0, 1, 2, 3
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mx_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from moe_grouped_gemm_mx_b200 import _build
+        _build.build()
+    L = ctypes.CDLL(LIB)
+    P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    L.mx_scale_bytes.argtypes = [I64, I64]
+    L.mx_scale_bytes.restype = ctypes.c_size_t
+    L.mx_status_string.argtypes = [ctypes.c_int]
+    L.mx_status_string.restype = ctypes.c_char_p
+    L.mx_quantize_bf16_to_e4m3.argtypes = [P, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3_grouped.argtypes = [P, I64, I64, I64, P, P, P]
+    L.mx_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
+    L.mx_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
+    L.mx_grouped_gemm_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
+    return L
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "mx_gemm" in names and "mx_grouped_gemm_masked" in names
+    for name in names:
+        assert hasattr(lib, name), name
+    import moe_grouped_gemm_mx_b200 as mx
+    assert sorted(mx.C_SYMBOLS) == names
+
+
+def test_scale_bytes_matches_oracle(lib, oracle):
+    for rows, k in [(1, 32), (128, 512), (129, 160), (64, 7168), (2112, 7168), (300, 96)]:
+        assert lib.mx_scale_bytes(rows, k) == oracle.scale_bytes(rows, k)
+    assert lib.mx_scale_bytes(0, 128) == 0
+    assert lib.mx_scale_bytes(-1, 128) == 0
+
+
+def test_status_strings(lib):
+    assert lib.mx_status_string(0) == b"MX_OK"
+    assert lib.mx_status_string(3) == b"MX_ERR_MISALIGNED"
+    assert lib.mx_status_string(99) == b"MX_ERR_UNKNOWN"
+
+
+FAKE = 0x10000  # a 16-byte aligned non-null value; never dereferenced by these calls
+
+
+def test_quantize_argument_checks(lib):
+    q = lib.mx_quantize_bf16_to_e4m3
+    assert q(FAKE, 4, 33, FAKE, FAKE, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert q(FAKE, -1, 32, FAKE, FAKE, None) == MX_ERR_INVALID_ARGUMENT
+    assert q(None, 4, 32, FAKE, FAKE, None) == MX_ERR_INVALID_ARGUMENT
+    assert q(FAKE + 8, 4, 32, FAKE, FAKE, None) == MX_ERR_MISALIGNED
+    assert q(None, 0, 32, None, None, None) == MX_OK  # empty is a no-op
+    g = lib.mx_quantize_bf16_to_e4m3_grouped
+    assert g(FAKE, -2, 4, 32, FAKE, FAKE, None) == MX_ERR_INVALID_ARGUMENT
+    assert g(None, 0, 4, 32, None, None, None) == MX_OK
+
+
+def test_gemm_argument_checks(lib):
+    f = lib.mx_gemm
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 100, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 24, 128, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 0, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, FAKE, None, FAKE, FAKE, 128, 256, 128, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE + 4, 128, 256, 128, None, None) == MX_ERR_MISALIGNED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 256, 128, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert f(None, None, None, None, None, 0, 256, 128, None, None) == MX_OK
+
+
+def test_grouped_argument_checks(lib):
+    c = lib.mx_grouped_gemm_contiguous
+    assert c(FAKE, FAKE, FAKE, FAKE, None, 4, 512, 256, 128, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert c(FAKE, FAKE, FAKE, FAKE, FAKE, 2000, 512, 256, 128, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert c(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 512, 256, 128, FAKE, None, None) == MX_ERR_MISALIGNED
+    assert c(None, None, None, None, None, 0, 512, 256, 128, None, None, None) == MX_OK
+    m = lib.mx_grouped_gemm_masked
+    assert m(FAKE, FAKE, FAKE, FAKE, None, 4, 256, 256, 128, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert m(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 250, 128, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert m(None, None, None, None, None, 4, 0, 256, 128, None, None, None) == MX_OK
