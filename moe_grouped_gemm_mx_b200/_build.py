@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmx.so")
 SOURCES = ["mx_api.cu", "mx_gemm.cu", "mx_quant.cu"]
-HEADERS = ["mx_ptx.cuh", "mx_launch.h"]
+HEADERS = ["mx_ptx.cuh", "mx_launch.h", "mx_fastdiv.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

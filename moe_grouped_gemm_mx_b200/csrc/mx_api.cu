@@ -67,6 +67,8 @@ static mx_status quantize_impl(const void* x, int64_t groups, int64_t rows, int6
   if (groups == 0 || rows == 0 || k == 0) return MX_OK;
   if (!x || !q || !sf) return MX_ERR_INVALID_ARGUMENT;
   if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return MX_ERR_MISALIGNED;
+  if (rows > kMaxDim || groups * rows > kMaxDim || groups * rows * (k / 32) >= (int64_t(1) << 31))
+    return MX_ERR_UNSUPPORTED_SHAPE;
   const int sms = num_sms();
   if (sms <= 0) return MX_ERR_CUDA;
   return from_cuda(mxk::launch_quant(x, groups, rows, k, q, sf, static_cast<int64_t>(mx_scale_bytes(rows, k)),

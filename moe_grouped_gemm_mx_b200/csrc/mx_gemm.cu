@@ -29,6 +29,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <cstdlib>
 
 #include "mx_launch.h"
 #include "mx_ptx.cuh"
@@ -59,9 +60,10 @@ struct GemmArgs {
   int n_sf_tiles;           // ceil(N / 128)
   int groups;
   int mode;
+  int sf_bufs;              // 1 or 2 TMEM buffers for the per-K-tile scale factors
 };
 
-template <int BN, int STAGES, int ACC>
+template <int BN, int STAGES, int ACC, int SPLIT = 1>
 struct Layout {
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = BN * BK;
@@ -80,12 +82,21 @@ struct Layout {
   static constexpr int BYTES = OFF_TAB1 + (kMaxGroups + 1) * 4;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024 B
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t SFA_COL = ACC * BN;
-  static constexpr uint32_t SFB_COL = SFA_COL + 4;
+  // scale factors in TMEM: up to two buffers of [SFA 4 cols | SFB 4 cols per 128 rows]
+  static constexpr uint32_t SF_COLS = 4 + 4 * SFB_TILES;
+  static constexpr uint32_t SF_COL0 = ACC * BN;
   static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
-  static_assert(SFB_COL + 4 * SFB_TILES <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(OFF_B % 1024 == 0 && OFF_SFA % 1024 == 0, "swizzled tiles need 1024-B alignment");
   static_assert(BYTES + 1024 <= 232448, "shared memory budget");
+  // split-K reduction buffer (reuses the operand ring once the mainloop is
+  // done): SPLIT partial slices of 128 rows x BN/SPLIT FP32 columns, rows
+  // padded by 4 floats to spread shared-memory banks.
+  static constexpr int SLICE = BN / SPLIT;
+  static constexpr int RED_STRIDE = SLICE + 4;
+  static constexpr int RED_BYTES = SPLIT * BM * RED_STRIDE * 4;
+  static_assert(SPLIT == 1 || RED_BYTES <= OFF_BAR, "reduction buffer must fit in the operand ring");
+  static_assert(SPLIT == 1 || SLICE % 4 == 0, "slices are moved as float4");
 };
 
 struct Tile {
@@ -136,11 +147,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int BN, int STAGES, int ACC>
+template <int BN, int STAGES, int ACC, int SPLIT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
-  using L = Layout<BN, STAGES, ACC>;
+  using L = Layout<BN, STAGES, ACC, SPLIT>;
+  // SPLIT > 1 (dense form only): a cluster of SPLIT CTAs shares one output
+  // tile, each CTA accumulating a contiguous share of the K tiles; the FP32
+  // partials are reduced through distributed shared memory.
+  const int split_rank = SPLIT > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT : static_cast<int>(blockIdx.x);
+  const int kt_begin = SPLIT > 1 ? split_rank * args.k_tiles / SPLIT : 0;
+  const int kt_end = SPLIT > 1 ? (split_rank + 1) * args.k_tiles / SPLIT : args.k_tiles;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -179,6 +197,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
   }
+  // Everything above touches only this CTA's shared memory and the kernel
+  // parameters.  With programmatic dependent launch the next kernel may begin
+  // its own prologue now, and from here on we need the previous kernel's
+  // results (operands, offsets) and may overwrite what it reads.
+  pdl_launch_dependents();
+  pdl_wait_prior();
 
   // scheduling tables
   int bad = 0;
@@ -251,7 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
         const Tile tl = decode_tile(args, tab0, t);
         const int a_row = tl.m_blk * BM;
         const int a_z = (args.mode == kMasked) ? tl.group : 0;
@@ -262,7 +286,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int sfb_tile0 = tl.n_blk * L::SFB_TILES;
         int nsfb = args.n_sf_tiles - sfb_tile0;
         nsfb = nsfb > L::SFB_TILES ? L::SFB_TILES : nsfb;
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        for (int kt = kt_begin; kt < kt_end; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           const uint32_t bytes = L::A_BYTES + L::B_BYTES + L::SFA_BYTES + 512u * nsfb;
           mbar_arrive_expect_tx(full_bar(stage), bytes);
@@ -290,20 +314,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       // ===== MMA issuer
       const uint32_t idesc0 = idesc_mxf8_e4m3(BM, BN);
-      const uint32_t sfa_t = tmem_base + L::SFA_COL;
-      const uint32_t sfb_t = tmem_base + L::SFB_COL;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
+      uint32_t sf_buf = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_t = tmem_base + acc * BN;
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        for (int kt = kt_begin; kt < kt_end; ++kt) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
+          // scale factors of this K tile -> TMEM (alternating buffers when two
+          // are configured, so the copy never targets columns the previous
+          // K tile's MMAs may still be reading)
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + sf_buf * L::SF_COLS;
+          const uint32_t sfb_t = sfa_t + 4;
+          sf_buf = (sf_buf + 1 == static_cast<uint32_t>(args.sf_bufs)) ? 0u : sf_buf + 1;
           tc_cp_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + stage * L::SFA_BYTES));
 #pragma unroll
           for (int j = 0; j < L::SFB_TILES; ++j)
@@ -316,7 +345,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t idesc = idesc_with_sf_ids(idesc0, kb, kb);
             tc_mma_mxf8(d_t, desc_kmajor_sw128(a_addr + 32 * kb), desc_kmajor_sw128(b_addr + 32 * kb), idesc,
                         sfa_t | (static_cast<uint32_t>(kb) << 30), sfb_t | (static_cast<uint32_t>(kb) << 30),
-                        (kt | kb) != 0);
+                        (kt != kt_begin || kb != 0) ? 1u : 0u);
           }
           tc_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -339,7 +368,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    for (int t = t_first; t < total; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
       // every lane polls; the vote re-converges the warp before the
       // warp-collective (.sync.aligned) TMEM loads below
       const bool got = mbar_wait(accf_bar(acc), acc_phase, abort_flag, kWaitLimitNs);
@@ -349,6 +378,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
+      if (SPLIT > 1) break;  // the split-K reduction below finishes this tile
       const Tile tl = decode_tile(args, tab0, t);
       int64_t drow;
       bool valid;
@@ -387,6 +417,68 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       mbar_arrive(acce_bar(acc));
       if (++acc == ACC) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  if constexpr (SPLIT > 1) {
+    // ---------------------------------------------------------- split-K reduction
+    // 1) every CTA of the cluster is past its mainloop, so every operand ring
+    //    is free to receive partials; 2) each CTA sends column slice j of its
+    //    FP32 partial to CTA j; 3) each CTA sums the SPLIT partials of its
+    //    slice in rank order (deterministic) and stores BF16.
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const int quarter = warp & 3;
+    const int r_local = quarter * 32 + lane;
+    const Tile tl = decode_tile(args, tab0, t_first);
+    const int row = tl.m_blk * BM + r_local;
+    const bool valid = row < args.m && !*abort_flag;
+    if (warp >= 2 && t_first < total) {
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tc_ld_32x32b_x32(t_row + c * 32, v);
+        tc_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const int col = c * 32 + q4 * 4;
+            const int owner = col / L::SLICE;
+            const int cin = col - owner * L::SLICE;
+            const uint32_t local = sbase + ((split_rank * BM + r_local) * L::RED_STRIDE + cin) * 4;
+            st_cluster_v4(map_to_rank(local, owner), v[q4 * 4 + 0], v[q4 * 4 + 1], v[q4 * 4 + 2], v[q4 * 4 + 3]);
+          }
+        }
+      }
+    }
+    cluster_sync();
+    if (warp >= 2 && t_first < total && valid) {
+      const float* red = reinterpret_cast<const float*>(smem);
+      __nv_bfloat16* drow_ptr = args.d + static_cast<int64_t>(row) * args.n;
+      const int col_base = tl.n_blk * BN + split_rank * L::SLICE;
+#pragma unroll 1
+      for (int j = 0; j < L::SLICE; j += 8) {
+        float sum[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sum[e] = 0.f;
+        for (int src = 0; src < SPLIT; ++src) {
+          const float4* p = reinterpret_cast<const float4*>(red + (src * BM + r_local) * L::RED_STRIDE + j);
+          const float4 x0 = p[0], x1 = p[1];
+          sum[0] += x0.x; sum[1] += x0.y; sum[2] += x0.z; sum[3] += x0.w;
+          sum[4] += x1.x; sum[5] += x1.y; sum[6] += x1.z; sum[7] += x1.w;
+        }
+        const int col = col_base + j;
+        if (col < args.n) {
+          uint4 w;
+          w.x = pack_bf16x2(__float_as_uint(sum[0]), __float_as_uint(sum[1]));
+          w.y = pack_bf16x2(__float_as_uint(sum[2]), __float_as_uint(sum[3]));
+          w.z = pack_bf16x2(__float_as_uint(sum[4]), __float_as_uint(sum[5]));
+          w.w = pack_bf16x2(__float_as_uint(sum[6]), __float_as_uint(sum[7]));
+          *reinterpret_cast<uint4*>(drow_ptr + col) = w;
+        }
+      }
     }
   }
 
@@ -431,15 +523,60 @@ static bool make_tmap(CUtensorMap* m, const void* base, int64_t k, int64_t rows,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, int ACC>
+// Number of TMEM scale-factor buffers (tuning override MX_GEMM_SFBUF = 1 | 2).
+static int sf_buffers() {
+  static int v = 0;
+  if (v == 0) {
+    const char* env = getenv("MX_GEMM_SFBUF");
+    v = (env && atoi(env) == 1) ? 1 : 2;
+  }
+  return v;
+}
+
+// Raise the kernel's dynamic shared-memory limit (once per process).
+template <int BN, int STAGES, int ACC, int SPLIT>
+static cudaError_t prepare_kernel() {
+  static cudaError_t state = cudaErrorNotReady;
+  if (state == cudaErrorNotReady)
+    state = cudaFuncSetAttribute(mx_gemm_kernel<BN, STAGES, ACC, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Layout<BN, STAGES, ACC, SPLIT>::ALLOC);
+  return state;
+}
+
+// How many clusters of the split-K kernel the GPU can hold at once (so a
+// launch is sized to a single wave); 0 if the query fails.
+template <int SPLIT>
+static int max_active_clusters() {
+  static int v = -1;
+  if (v < 0) {
+    v = 0;
+    if (prepare_kernel<128, 6, 1, SPLIT>() == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      cfg.gridDim = dim3(SPLIT, 1, 1);
+      cfg.blockDim = dim3(kGemmThreads, 1, 1);
+      cfg.dynamicSmemBytes = Layout<128, 6, 1, SPLIT>::ALLOC;
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = SPLIT;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_kernel<128, 6, 1, SPLIT>, &cfg) == cudaSuccess) v = n;
+      cudaGetLastError();
+    }
+  }
+  return v;
+}
+
+template <int BN, int STAGES, int ACC, int SPLIT>
 static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
-  using L = Layout<BN, STAGES, ACC>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(mx_gemm_kernel<BN, STAGES, ACC>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  using L = Layout<BN, STAGES, ACC, SPLIT>;
+  auto kern = mx_gemm_kernel<BN, STAGES, ACC, SPLIT>;
+  {
+    cudaError_t e = prepare_kernel<BN, STAGES, ACC, SPLIT>();
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   CUtensorMap ta, tb;
   const int64_t a_depth = p.mode == kMasked ? p.groups : 1;
@@ -463,6 +600,7 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
   a.n_sf_tiles = static_cast<int>((p.n + 127) / 128);
   a.groups = static_cast<int>(p.groups);
   a.mode = p.mode;
+  a.sf_bufs = sf_buffers();
 
   int64_t m_tiles_bound;
   if (p.mode == kMasked)
@@ -471,14 +609,82 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
     m_tiles_bound = (p.m + BM - 1) / BM;
   const int64_t tiles_bound = m_tiles_bound * a.n_tiles;
   if (tiles_bound == 0) return cudaSuccess;
-  const int grid = static_cast<int>(tiles_bound < num_sms ? tiles_bound : num_sms);
-  mx_gemm_kernel<BN, STAGES, ACC><<<grid, kGemmThreads, L::ALLOC, stream>>>(ta, tb, a);
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  if (SPLIT > 1) {
+    // one cluster of SPLIT CTAs per output tile
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_bound * SPLIT), 1, 1);
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = SPLIT;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+  } else {
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_bound < num_sms ? tiles_bound : num_sms), 1, 1);
+    attr[0] = pdl;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
+  if (e != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaGetLastError();
 }
 
+// Tile configuration for one problem.  Large problems (at least a wave of
+// 128x256 tiles) use the persistent 128x256 kernel; smaller ones first try
+// 128x128 tiles with a double-buffered accumulator, and dense problems that
+// still leave most SMs idle split K across a cluster of 2, 4 or 8 CTAs.
+enum GemmConfig : int { kCfg256 = 0, kCfg128 = 1, kCfgSplit2 = 2, kCfgSplit4 = 3, kCfgSplit8 = 4 };
+
+static int choose_config(const GemmProblem& p, int num_sms) {
+  static int forced = -2;
+  if (forced == -2) {
+    const char* env = getenv("MX_GEMM_CONFIG");  // tuning override: 0..4
+    forced = env ? atoi(env) : -1;
+  }
+  const int64_t k_tiles = p.k / BK;
+  const int64_t m_blocks = (p.mode == kMasked ? p.groups : 1) * ((p.m + BM - 1) / BM);
+  const int64_t t256 = m_blocks * ((p.n + 255) / 256);
+  const int64_t t128 = m_blocks * ((p.n + 127) / 128);
+  int c;
+  if (t256 >= num_sms || p.mode != kDense) {
+    c = t256 >= num_sms ? kCfg256 : (t128 >= num_sms / 2 ? kCfg128 : kCfg256);
+  } else if (t128 >= (num_sms * 3) / 4) {
+    c = kCfg128;
+  } else if (t128 * 8 <= num_sms && k_tiles >= 8 && t128 <= max_active_clusters<8>()) {
+    c = kCfgSplit8;
+  } else if (t128 * 4 <= num_sms && k_tiles >= 4 && t128 <= max_active_clusters<4>()) {
+    c = kCfgSplit4;
+  } else if (t128 * 2 <= num_sms && k_tiles >= 2 && t128 <= max_active_clusters<2>()) {
+    c = kCfgSplit2;
+  } else {
+    c = kCfg128;
+  }
+  if (forced >= 0 && forced <= 4) {
+    const int need = forced == kCfgSplit2 ? 2 : forced == kCfgSplit4 ? 4 : forced == kCfgSplit8 ? 8 : 1;
+    if (forced < kCfgSplit2 || (p.mode == kDense && k_tiles >= need)) c = forced;
+  }
+  return c;
+}
+
 cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
-  return launch_gemm_cfg<256, 4, 1>(p, num_sms, stream, launches);
+  switch (choose_config(p, num_sms)) {
+    case kCfg128: return launch_gemm_cfg<128, 6, 2, 1>(p, num_sms, stream, launches);
+    case kCfgSplit2: return launch_gemm_cfg<128, 6, 1, 2>(p, num_sms, stream, launches);
+    case kCfgSplit4: return launch_gemm_cfg<128, 6, 1, 4>(p, num_sms, stream, launches);
+    case kCfgSplit8: return launch_gemm_cfg<128, 6, 1, 8>(p, num_sms, stream, launches);
+    default: return launch_gemm_cfg<256, 4, 1, 1>(p, num_sms, stream, launches);
+  }
 }
 
 }  // namespace mxk

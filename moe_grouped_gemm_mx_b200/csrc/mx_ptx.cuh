@@ -208,3 +208,52 @@ __device__ __forceinline__ uint32_t idesc_with_sf_ids(uint32_t base, uint32_t a_
 }
 
 }  // namespace mxk
+
+// ------------------------------------------------------------------ clusters
+
+namespace mxk {
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Arrive-and-wait on the cluster-wide barrier (every thread of every CTA in
+// the cluster takes part).  Release/acquire orders shared-memory accesses
+// made by other CTAs of the cluster before the barrier with ours after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Shared-memory address of the same location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local_smem, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+}  // namespace mxk
+
+// ------------------------------------------------------------------ programmatic dependent launch
+
+namespace mxk {
+
+// Let the next kernel in the stream (launched with programmatic stream
+// serialization) start its prologue while this grid is still running.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Block until the preceding kernel in the stream has completed and its
+// memory is visible (a no-op when this grid was launched without PDL).
+__device__ __forceinline__ void pdl_wait_prior() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+}  // namespace mxk

@@ -7,20 +7,24 @@
 //
 // Kernel design (HBM-bound: 2 B read, 1 + 1/32 B written per element):
 //  * The [rows, K] source is contiguous, so 32-element block b is the 64-byte
-//    chunk at byte 64*b regardless of row boundaries.  Four lanes own one
-//    block (16 B each); a warp covers 8 consecutive blocks = 512 contiguous
-//    bytes, and each thread keeps U such 16-byte loads in flight.
-//  * amax is reduced on the integer magnitude bits (bits & 0x7fff) with two
-//    xor-shuffles; for non-negative IEEE values integer order is value order,
-//    and any pattern >= 0x7f80 is Inf/NaN, so a non-finite block is detected
-//    by the same max (an fmaxf reduction would silently drop NaN).
+//    chunk at byte 64*b regardless of row boundaries.  One lane owns one
+//    block (four 16-byte loads), a warp 32 consecutive blocks (2 KiB), and
+//    every thread keeps two blocks' loads in flight.  One lane per block keeps
+//    the per-element instruction count low: amax, exponent and the scale
+//    address are computed once per 32 elements.
+//  * amax is reduced on the integer magnitude bits (bits & 0x7fff, two BF16
+//    values per 32-bit SIMD max); for non-negative IEEE patterns integer
+//    order is value order, and any pattern >= 0x7f80 is Inf/NaN, so a
+//    non-finite block is detected by the same max (an fmaxf reduction would
+//    silently drop NaN).
 //  * floor(log2 amax) comes from the exponent field (normal) or the position
 //    of the top mantissa bit (subnormal); no log2f.
 //  * Elements are scaled by the exact power of two 2^-X in fp32 and converted
 //    with the hardware's saturating round-to-nearest-even cvt (e4m3x2).
 //  * Four consecutive blocks of a row (K-block c..c+3, c % 4 == 0) land in 4
 //    consecutive scale bytes, so their scales are gathered into one 32-bit
-//    store when K/32 is a multiple of 4.
+//    store when K/32 is a multiple of 4.  Row / K-block / group indices use
+//    32-bit division by launch-time constants (multiply-high and shift).
 //  * Extra CTAs beyond the streaming grid write 0x00 into the scale-tile
 //    padding (rows up to a multiple of 128, K-blocks up to a multiple of 4).
 #include <cuda_bf16.h>
@@ -28,29 +32,32 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "mx_fastdiv.h"
 #include "mx_launch.h"
 
 namespace mxk {
 
 constexpr int kQuantThreads = 256;
-constexpr int kQuantUnroll = 4;  // 16-byte loads in flight per thread
+constexpr int kQuantUnroll = 2;  // 32-element blocks per thread per loop trip (8 x 16 B loads in flight)
 
 struct QuantArgs {
   const uint4* x;          // BF16 source viewed as 16-byte vectors
   uint2* q;                // E4M3 output viewed as 8-byte vectors
   uint8_t* sf;             // tiled scale output
-  int64_t nblk;            // total 32-element blocks = groups*rows*kb
-  int64_t kb;              // blocks per row = k/32
-  int64_t rows;            // rows per group
-  int64_t groups;
+  uint32_t nblk;           // total 32-element blocks = groups*rows*kb (< 2^31)
+  uint32_t kb;             // blocks per row = k/32
+  uint32_t rows;           // rows per group
+  uint32_t groups;
+  FastDiv div_kb;          // divide by kb
+  FastDiv div_rows;        // divide by rows
   int64_t sf_group_bytes;  // tiled scale bytes per group
-  int64_t sf_ktiles;       // ceil(kb/4): 512-byte tiles along K
+  uint32_t sf_ktiles;      // ceil(kb/4): 512-byte tiles along K
   int main_blocks;         // CTAs that stream blocks; the rest write padding
   int kb4;                 // kb % 4 == 0
 };
 
-__device__ __forceinline__ int64_t sf_tiled_offset(int64_t r, int64_t c, int64_t sf_ktiles) {
-  return ((r >> 7) * sf_ktiles + (c >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
+__device__ __forceinline__ uint32_t sf_tiled_offset(uint32_t r, uint32_t c, uint32_t sf_ktiles) {
+  return ((r >> 7) * sf_ktiles + (c >> 2)) * 512u + (r & 31u) * 16u + ((r & 127u) >> 5) * 4u + (c & 3u);
 }
 
 // Scale exponent X for a block whose largest magnitude has BF16 bits `amax_bits`
@@ -78,18 +85,19 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint32_t max_mag(uint32_t w) {
-  return max(w & 0x7FFFu, (w >> 16) & 0x7FFFu);
-}
-
 __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const QuantArgs a) {
+  // with programmatic dependent launch the next kernel may start its
+  // prologue now; our own reads and writes wait for the previous kernel
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (static_cast<int>(blockIdx.x) >= a.main_blocks) {
     // ---- padding of the scale tiles: rows [rows, rpad) x all kb_pad, and
     // rows [0, rows) x blocks [kb, kb_pad), for every group.
-    const int64_t kbpad = a.sf_ktiles * 4;
-    const int64_t rpad = (a.rows + 127) / 128 * 128;
-    const int64_t n1 = (rpad - a.rows) * kbpad;
-    const int64_t n2 = a.rows * (kbpad - a.kb);
+    const int64_t kbpad = static_cast<int64_t>(a.sf_ktiles) * 4;
+    const int64_t rows = a.rows;
+    const int64_t rpad = (rows + 127) / 128 * 128;
+    const int64_t n1 = (rpad - rows) * kbpad;
+    const int64_t n2 = rows * (kbpad - a.kb);
     const int64_t per_group = n1 + n2;
     const int64_t total = per_group * a.groups;
     const int64_t stride = static_cast<int64_t>(gridDim.x - a.main_blocks) * blockDim.x;
@@ -99,7 +107,7 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const QuantArgs
       const int64_t j = i - g * per_group;
       int64_t r, c;
       if (j < n1) {
-        r = a.rows + j / kbpad;
+        r = rows + j / kbpad;
         c = j % kbpad;
       } else {
         const int64_t jj = j - n1;
@@ -107,90 +115,119 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const QuantArgs
         r = jj / w;
         c = a.kb + jj % w;
       }
-      a.sf[g * a.sf_group_bytes + sf_tiled_offset(r, c, a.sf_ktiles)] = 0;
+      a.sf[g * a.sf_group_bytes + sf_tiled_offset(static_cast<uint32_t>(r), static_cast<uint32_t>(c), a.sf_ktiles)] = 0;
     }
     return;
   }
 
-  const int lane = threadIdx.x & 31;
-  const int sub = lane & 3;   // which 16-byte quarter of the block
-  const int blk = lane >> 2;  // which of the warp's 8 blocks
-  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(a.main_blocks) * blockDim.x) >> 5;
-  constexpr int kWarpBlocks = 8 * kQuantUnroll;
+  // ---- streaming part: one lane owns one 32-element block (64 contiguous
+  // bytes: four 16-byte loads), so amax, exponent and scale bookkeeping are
+  // done once per block with no shuffles; a warp covers 32 consecutive blocks
+  // (2 KiB) per unrolled slot.
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t warp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (static_cast<uint32_t>(a.main_blocks) * blockDim.x) >> 5;
+  constexpr uint32_t kWarpBlocks = 32 * kQuantUnroll;
 
-  for (int64_t base = warp_id * kWarpBlocks; base < a.nblk; base += nwarps * kWarpBlocks) {
-    uint4 v[kQuantUnroll];
+  for (uint32_t base = warp_id * kWarpBlocks; base < a.nblk; base += nwarps * kWarpBlocks) {
+    uint4 v[kQuantUnroll][4];
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t b = base + u * 8 + blk;
-      v[u] = b < a.nblk ? __ldcs(a.x + b * 4 + sub) : make_uint4(0, 0, 0, 0);
+      const uint32_t b = base + u * 32 + lane;
+      const uint4* src = a.x + static_cast<size_t>(b) * 4;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[u][j] = b < a.nblk ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
-      const int64_t b = base + u * 8 + blk;
-      uint32_t m = max(max(max_mag(v[u].x), max_mag(v[u].y)), max(max_mag(v[u].z), max_mag(v[u].w)));
-      m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-      m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+      const uint32_t b = base + u * 32 + lane;
+      // amax of |x| on the magnitude bits, two BF16 lanes at a time
+      uint32_t m2 = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m2 = __vmaxu2(m2, v[u][j].x & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[u][j].y & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[u][j].z & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[u][j].w & 0x7FFF7FFFu);
+      }
+      const uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
       uint32_t scode;
-      uint2 out;
+      uint4 out0, out1;
       if (m >= 0x7F80u) {  // Inf or NaN somewhere in the block
         scode = 0xFFu;
-        out = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
+        out0 = out1 = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
       } else {
         const int X = block_exponent(m);
         scode = static_cast<uint32_t>(X + 127);
         const float mult = __uint_as_float(static_cast<uint32_t>(127 - X) << 23);  // 2^-X
-        out.x = pack_e4m3x4(bf16_lo(v[u].x) * mult, bf16_hi(v[u].x) * mult,
-                            bf16_lo(v[u].y) * mult, bf16_hi(v[u].y) * mult);
-        out.y = pack_e4m3x4(bf16_lo(v[u].z) * mult, bf16_hi(v[u].z) * mult,
-                            bf16_lo(v[u].w) * mult, bf16_hi(v[u].w) * mult);
-      }
-      if (b < a.nblk) __stcs(a.q + b * 4 + sub, out);
-
-      // scale byte(s)
-      const int64_t row = b / a.kb;
-      const int64_t c = b - row * a.kb;
-      const int64_t g = row / a.rows;
-      const int64_t rl = row - g * a.rows;
-      if (a.kb4) {
-        // lanes 0 and 16 each store the 4 scales of blocks blk..blk+3 (one row,
-        // K-blocks c..c+3 with c % 4 == 0).
-        const int src = lane & 16;
-        const uint32_t s0 = __shfl_sync(0xFFFFFFFFu, scode, src + 0);
-        const uint32_t s1 = __shfl_sync(0xFFFFFFFFu, scode, src + 4);
-        const uint32_t s2 = __shfl_sync(0xFFFFFFFFu, scode, src + 8);
-        const uint32_t s3 = __shfl_sync(0xFFFFFFFFu, scode, src + 12);
-        if ((lane & 15) == 0 && b < a.nblk) {
-          *reinterpret_cast<uint32_t*>(a.sf + g * a.sf_group_bytes + sf_tiled_offset(rl, c, a.sf_ktiles)) =
-              s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        uint32_t o[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          o[2 * j] = pack_e4m3x4(bf16_lo(v[u][j].x) * mult, bf16_hi(v[u][j].x) * mult,
+                                 bf16_lo(v[u][j].y) * mult, bf16_hi(v[u][j].y) * mult);
+          o[2 * j + 1] = pack_e4m3x4(bf16_lo(v[u][j].z) * mult, bf16_hi(v[u][j].z) * mult,
+                                     bf16_lo(v[u][j].w) * mult, bf16_hi(v[u][j].w) * mult);
         }
-      } else if (sub == 0 && b < a.nblk) {
-        a.sf[g * a.sf_group_bytes + sf_tiled_offset(rl, c, a.sf_ktiles)] = static_cast<uint8_t>(scode);
+        out0 = make_uint4(o[0], o[1], o[2], o[3]);
+        out1 = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+      if (b < a.nblk) {
+        uint4* dst = reinterpret_cast<uint4*>(a.q) + static_cast<size_t>(b) * 2;
+        __stcs(dst, out0);
+        __stcs(dst + 1, out1);
+      }
+
+      // scale byte(s): row / K-block of this block, then its group
+      const uint32_t row = fdiv(b, a.div_kb);
+      const uint32_t c = b - row * a.kb;
+      uint32_t g = 0, rl = row;
+      if (a.groups > 1) {
+        g = fdiv(row, a.div_rows);
+        rl = row - g * a.rows;
+      }
+      uint8_t* sfp = a.sf + static_cast<int64_t>(g) * a.sf_group_bytes + sf_tiled_offset(rl, c, a.sf_ktiles);
+      if (a.kb4) {
+        // lanes 4j..4j+3 hold K-blocks c..c+3 (c % 4 == 0) of one row: their
+        // four scale bytes are adjacent, so lane 4j stores them as one word.
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, scode, 1);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, scode, 2);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, scode, 3);
+        if ((lane & 3u) == 0 && b < a.nblk)
+          *reinterpret_cast<uint32_t*>(sfp) = scode | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      } else if (b < a.nblk) {
+        *sfp = static_cast<uint8_t>(scode);
       }
     }
   }
 }
 
-// Launch helper used by the C ABI (validation happens there).
+// Launch helper used by the C ABI (validation happens there).  Needs
+// groups*rows*(k/32) < 2^31 blocks.
 cudaError_t launch_quant(const void* x, int64_t groups, int64_t rows, int64_t k, void* q, void* sf,
                          int64_t sf_group_bytes, int num_sms, cudaStream_t stream, int* launches) {
+  static int resident = 0;  // CTAs of the kernel one SM holds (same for every B200)
+  if (resident == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, mx_quant_kernel, kQuantThreads, 0);
+    if (e != cudaSuccess || resident <= 0) resident = 2048 / kQuantThreads;
+  }
   QuantArgs a;
   a.x = static_cast<const uint4*>(x);
   a.q = static_cast<uint2*>(q);
   a.sf = static_cast<uint8_t*>(sf);
-  a.kb = k / 32;
-  a.rows = rows;
-  a.groups = groups;
-  a.nblk = groups * rows * a.kb;
+  a.kb = static_cast<uint32_t>(k / 32);
+  a.rows = static_cast<uint32_t>(rows);
+  a.groups = static_cast<uint32_t>(groups);
+  a.nblk = static_cast<uint32_t>(groups * rows * (k / 32));
+  a.div_kb = make_fastdiv(a.kb);
+  a.div_rows = make_fastdiv(a.rows);
   a.sf_group_bytes = sf_group_bytes;
   a.sf_ktiles = (a.kb + 3) / 4;
   a.kb4 = (a.kb % 4) == 0;
-  const int64_t warps_needed = (a.nblk + 8 * kQuantUnroll - 1) / (8 * kQuantUnroll);
+  const int64_t warps_needed = (static_cast<int64_t>(a.nblk) + 32 * kQuantUnroll - 1) / (32 * kQuantUnroll);
   const int64_t ctas_needed = (warps_needed + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
-  const int64_t max_ctas = static_cast<int64_t>(num_sms) * (2048 / kQuantThreads);
+  const int64_t max_ctas = static_cast<int64_t>(num_sms) * resident;
   a.main_blocks = static_cast<int>(ctas_needed < max_ctas ? ctas_needed : max_ctas);
-  const int64_t kbpad = a.sf_ktiles * 4;
+  const int64_t kbpad = static_cast<int64_t>(a.sf_ktiles) * 4;
   const int64_t rpad = (rows + 127) / 128 * 128;
   const int64_t pad_entries = ((rpad - rows) * kbpad + rows * (kbpad - a.kb)) * groups;
   int pad_blocks = 0;
@@ -200,7 +237,18 @@ cudaError_t launch_quant(const void* x, int64_t groups, int64_t rows, int64_t k,
   }
   const int grid = a.main_blocks + pad_blocks;
   if (grid == 0) return cudaSuccess;
-  mx_quant_kernel<<<grid, kQuantThreads, 0, stream>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kQuantThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mx_quant_kernel, a);
+  if (e != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaGetLastError();
 }
