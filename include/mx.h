@@ -98,6 +98,25 @@ mx_status mx_quantize_bf16_to_e4m3_grouped(const void *x_bf16, int64_t groups, i
                                            mx_stream_t stream);
 
 /*
+ * Several quantisations in one kernel launch (for the operands of one step:
+ * fewer launches, one launch latency).  Each job is exactly the
+ * mx_quantize_bf16_to_e4m3_grouped call with the same fields (groups == 1
+ * for a 2-D tensor); jobs with a zero extent are skipped.  Every job is
+ * validated before anything is launched; up to 8 jobs share a launch.  The
+ * jobs must not overlap in memory.
+ */
+typedef struct mx_quant_job {
+    const void *x_bf16; /* [groups, rows, k] BF16 */
+    int64_t groups;
+    int64_t rows;
+    int64_t k;
+    void *q_e4m3;       /* [groups, rows, k] bytes out */
+    void *sf_ue8m0;     /* groups * mx_scale_bytes(rows, k) bytes out */
+} mx_quant_job;
+
+mx_status mx_quantize_bf16_to_e4m3_multi(const mx_quant_job *jobs, int32_t count, mx_stream_t stream);
+
+/*
  * Dense MXFP8 GEMM, D = A * B^T ("DeepGEMM" summary page: the plain FP8
  * GEMM; the dense shapes of its CUTLASS comparison table).
  *   qa [m, k], sfa = scales of A (mx_scale_bytes(m, k));

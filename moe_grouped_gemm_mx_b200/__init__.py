@@ -22,7 +22,8 @@ import os
 import torch
 
 __all__ = [
-    "MXError", "lib_path", "scale_bytes", "mx_quantize_bf16_to_e4m3", "mx_gemm",
+    "MXError", "lib_path", "scale_bytes", "mx_quantize_bf16_to_e4m3", "mx_quantize_bf16_to_e4m3_multi",
+    "mx_gemm",
     "mx_grouped_gemm_contiguous", "mx_grouped_gemm_masked", "read_internal_status",
     "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "C_SYMBOLS",
 ]
@@ -37,9 +38,15 @@ MX_DEV_TIMEOUT = 0x4
 # every symbol include/mx.h declares
 C_SYMBOLS = [
     "mx_status_string", "mx_scale_bytes", "mx_quantize_bf16_to_e4m3",
-    "mx_quantize_bf16_to_e4m3_grouped", "mx_gemm", "mx_grouped_gemm_contiguous",
+    "mx_quantize_bf16_to_e4m3_grouped", "mx_quantize_bf16_to_e4m3_multi", "mx_gemm",
+    "mx_grouped_gemm_contiguous",
     "mx_grouped_gemm_masked", "mx_read_internal_status",
 ]
+
+
+class _QuantJob(ctypes.Structure):
+    _fields_ = [("x_bf16", ctypes.c_void_p), ("groups", ctypes.c_int64), ("rows", ctypes.c_int64),
+                ("k", ctypes.c_int64), ("q_e4m3", ctypes.c_void_p), ("sf_ue8m0", ctypes.c_void_p)]
 
 
 class MXError(RuntimeError):
@@ -63,6 +70,8 @@ def _load():
     L.mx_quantize_bf16_to_e4m3.restype = ctypes.c_int
     L.mx_quantize_bf16_to_e4m3_grouped.argtypes = [P, I64, I64, I64, P, P, P]
     L.mx_quantize_bf16_to_e4m3_grouped.restype = ctypes.c_int
+    L.mx_quantize_bf16_to_e4m3_multi.argtypes = [ctypes.POINTER(_QuantJob), I32, P]
+    L.mx_quantize_bf16_to_e4m3_multi.restype = ctypes.c_int
     L.mx_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
     L.mx_gemm.restype = ctypes.c_int
     L.mx_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
@@ -136,6 +145,34 @@ def mx_quantize_bf16_to_e4m3(x: torch.Tensor, q: torch.Tensor | None = None,
                                                    _stream(stream))
     _raise(st, "mx_quantize_bf16_to_e4m3")
     return q, sf
+
+
+def mx_quantize_bf16_to_e4m3_multi(xs, outs=None, stream=None):
+    """Quantise several BF16 tensors ([rows, K] or [groups, rows, K]) in one
+    kernel launch.  ``outs`` optionally gives a (q, sf) pair per tensor.
+    Returns the list of (q, sf)."""
+    xs = list(xs)
+    res = []
+    jobs = (_QuantJob * max(1, len(xs)))()
+    for i, x in enumerate(xs):
+        _check(x, torch.bfloat16, f"xs[{i}]")
+        if x.dim() not in (2, 3):
+            raise ValueError("each tensor must be 2-D or 3-D")
+        groups = 1 if x.dim() == 2 else x.shape[0]
+        rows, k = x.shape[-2], x.shape[-1]
+        if outs is not None:
+            q, sf = outs[i]
+        else:
+            q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+            sf = torch.empty(groups * scale_bytes(rows, k), dtype=torch.uint8, device=x.device)
+        _check(q, torch.uint8, f"q[{i}]")
+        _check(sf, torch.uint8, f"sf[{i}]")
+        if q.numel() != x.numel() or sf.numel() < groups * scale_bytes(rows, k):
+            raise ValueError("output buffers too small")
+        jobs[i] = _QuantJob(_ptr(x), groups, rows, k, _ptr(q), _ptr(sf))
+        res.append((q, sf))
+    _raise(_lib.mx_quantize_bf16_to_e4m3_multi(jobs, len(xs), _stream(stream)), "mx_quantize_bf16_to_e4m3_multi")
+    return res
 
 
 def _status_arg(dev_status):

@@ -60,19 +60,32 @@ size_t mx_scale_bytes(int64_t rows, int64_t k) {
   return static_cast<size_t>(((rows + 127) / 128) * 128 * ((kb + 3) / 4) * 4);
 }
 
-static mx_status quantize_impl(const void* x, int64_t groups, int64_t rows, int64_t k, void* q, void* sf,
-                               mx_stream_t stream) {
+// Host-side checks of one quantisation job; MX_OK with *empty set for a no-op.
+static mx_status check_quant_job(const void* x, int64_t groups, int64_t rows, int64_t k, const void* q,
+                                 const void* sf, bool* empty) {
+  *empty = false;
   if (groups < 0 || rows < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
   if (k % 32 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
-  if (groups == 0 || rows == 0 || k == 0) return MX_OK;
+  if (groups == 0 || rows == 0 || k == 0) {
+    *empty = true;
+    return MX_OK;
+  }
   if (!x || !q || !sf) return MX_ERR_INVALID_ARGUMENT;
   if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return MX_ERR_MISALIGNED;
   if (rows > kMaxDim || groups * rows > kMaxDim || groups * rows * (k / 32) >= (int64_t(1) << 31))
     return MX_ERR_UNSUPPORTED_SHAPE;
+  return MX_OK;
+}
+
+static mx_status quantize_impl(const void* x, int64_t groups, int64_t rows, int64_t k, void* q, void* sf,
+                               mx_stream_t stream) {
+  bool empty = false;
+  mx_status st = check_quant_job(x, groups, rows, k, q, sf, &empty);
+  if (st != MX_OK || empty) return st;
   const int sms = num_sms();
   if (sms <= 0) return MX_ERR_CUDA;
-  return from_cuda(mxk::launch_quant(x, groups, rows, k, q, sf, static_cast<int64_t>(mx_scale_bytes(rows, k)),
-                                     sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+  mxk::QuantSpec spec{x, q, sf, groups, rows, k, static_cast<int64_t>(mx_scale_bytes(rows, k))};
+  return from_cuda(mxk::launch_quant_batch(&spec, 1, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
 }
 
 mx_status mx_quantize_bf16_to_e4m3(const void* x_bf16, int64_t rows, int64_t k, void* q_e4m3, void* sf_ue8m0,
@@ -83,6 +96,40 @@ mx_status mx_quantize_bf16_to_e4m3(const void* x_bf16, int64_t rows, int64_t k, 
 mx_status mx_quantize_bf16_to_e4m3_grouped(const void* x_bf16, int64_t groups, int64_t rows, int64_t k,
                                            void* q_e4m3, void* sf_ue8m0, mx_stream_t stream) {
   return quantize_impl(x_bf16, groups, rows, k, q_e4m3, sf_ue8m0, stream);
+}
+
+mx_status mx_quantize_bf16_to_e4m3_multi(const mx_quant_job* jobs, int32_t count, mx_stream_t stream) {
+  if (count < 0 || (count > 0 && !jobs)) return MX_ERR_INVALID_ARGUMENT;
+  // validate everything before launching anything
+  int nonempty = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    bool empty = false;
+    mx_status st = check_quant_job(jobs[i].x_bf16, jobs[i].groups, jobs[i].rows, jobs[i].k, jobs[i].q_e4m3,
+                                   jobs[i].sf_ue8m0, &empty);
+    if (st != MX_OK) return st;
+    nonempty += empty ? 0 : 1;
+  }
+  if (nonempty == 0) return MX_OK;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  mxk::QuantSpec specs[mxk::kMaxQuantJobs];
+  int n = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    const mx_quant_job& j = jobs[i];
+    if (j.groups == 0 || j.rows == 0 || j.k == 0) continue;
+    specs[n++] = mxk::QuantSpec{j.x_bf16, j.q_e4m3, j.sf_ue8m0, j.groups, j.rows, j.k,
+                                static_cast<int64_t>(mx_scale_bytes(j.rows, j.k))};
+    if (n == mxk::kMaxQuantJobs) {
+      cudaError_t e = mxk::launch_quant_batch(specs, n, sms, reinterpret_cast<cudaStream_t>(stream), nullptr);
+      if (e != cudaSuccess) return MX_ERR_CUDA;
+      n = 0;
+    }
+  }
+  if (n > 0) {
+    cudaError_t e = mxk::launch_quant_batch(specs, n, sms, reinterpret_cast<cudaStream_t>(stream), nullptr);
+    if (e != cudaSuccess) return MX_ERR_CUDA;
+  }
+  return MX_OK;
 }
 
 static mx_status check_gemm_common(const void* qa, const void* sfa, const void* qb, const void* sfb, void* d,

@@ -6,8 +6,17 @@
 
 namespace mxk {
 
-cudaError_t launch_quant(const void* x, int64_t groups, int64_t rows, int64_t k, void* q, void* sf,
-                         int64_t sf_group_bytes, int num_sms, cudaStream_t stream, int* launches);
+constexpr int kMaxQuantJobs = 8;  // tensors one quantiser launch handles
+
+struct QuantSpec {
+  const void* x;            // BF16 [groups, rows, k]
+  void* q;                  // E4M3 out, same shape
+  void* sf;                 // tiled scales out, groups regions of sf_group_bytes
+  int64_t groups, rows, k;
+  int64_t sf_group_bytes;
+};
+
+cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, cudaStream_t stream, int* launches);
 
 struct GemmProblem {
   const void* qa;

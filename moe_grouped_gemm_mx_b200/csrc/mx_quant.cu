@@ -38,13 +38,17 @@
 namespace mxk {
 
 constexpr int kQuantThreads = 256;
-constexpr int kQuantUnroll = 2;  // 32-element blocks per thread per loop trip (8 x 16 B loads in flight)
+constexpr int kQuantUnroll = 2;   // 32-element blocks per lane per loop trip (8 x 16 B loads in flight)
+constexpr uint32_t kSlotBlocks = 32 * kQuantUnroll;  // blocks one warp handles per loop trip
 
-struct QuantArgs {
+// One tensor to quantise.  Several are processed by one launch: their block
+// ranges are laid end to end in "slots" of kSlotBlocks blocks (each job
+// starts on a slot boundary, so a warp's slot never spans two jobs).
+struct QuantJob {
   const uint4* x;          // BF16 source viewed as 16-byte vectors
-  uint2* q;                // E4M3 output viewed as 8-byte vectors
+  uint4* q;                // E4M3 output viewed as 16-byte vectors
   uint8_t* sf;             // tiled scale output
-  uint32_t nblk;           // total 32-element blocks = groups*rows*kb (< 2^31)
+  uint32_t nblk;           // 32-element blocks = groups*rows*kb (< 2^31)
   uint32_t kb;             // blocks per row = k/32
   uint32_t rows;           // rows per group
   uint32_t groups;
@@ -52,8 +56,19 @@ struct QuantArgs {
   FastDiv div_rows;        // divide by rows
   int64_t sf_group_bytes;  // tiled scale bytes per group
   uint32_t sf_ktiles;      // ceil(kb/4): 512-byte tiles along K
+  uint32_t kb4;            // kb % 4 == 0
+  uint32_t slot0;          // first slot of this job
+  int64_t pad0;            // first scale-padding entry of this job
+  int64_t pad_n1;          // per group: padding entries in rows [rows, rpad)
+  int64_t pad_per_group;   // per group: all padding entries
+};
+
+struct QuantBatch {
+  QuantJob job[kMaxQuantJobs];
+  int count;
+  uint32_t total_slots;
   int main_blocks;         // CTAs that stream blocks; the rest write padding
-  int kb4;                 // kb % 4 == 0
+  int64_t pad_total;
 };
 
 __device__ __forceinline__ uint32_t sf_tiled_offset(uint32_t r, uint32_t c, uint32_t sf_ktiles) {
@@ -85,63 +100,67 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const QuantArgs a) {
+// Scale-tile padding entry i of one job: rows [rows, rpad) x all kb_pad
+// blocks, then rows [0, rows) x blocks [kb, kb_pad), for every group.
+__device__ void write_padding(const QuantJob& jb, int64_t i) {
+  const int64_t kbpad = static_cast<int64_t>(jb.sf_ktiles) * 4;
+  const int64_t g = i / jb.pad_per_group;
+  const int64_t j = i - g * jb.pad_per_group;
+  int64_t r, c;
+  if (j < jb.pad_n1) {
+    r = jb.rows + j / kbpad;
+    c = j % kbpad;
+  } else {
+    const int64_t jj = j - jb.pad_n1;
+    const int64_t w = kbpad - jb.kb;
+    r = jj / w;
+    c = jb.kb + jj % w;
+  }
+  jb.sf[g * jb.sf_group_bytes + sf_tiled_offset(static_cast<uint32_t>(r), static_cast<uint32_t>(c), jb.sf_ktiles)] = 0;
+}
+
+__global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_constant__ QuantBatch B) {
   // with programmatic dependent launch the next kernel may start its
   // prologue now; our own reads and writes wait for the previous kernel
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (static_cast<int>(blockIdx.x) >= a.main_blocks) {
-    // ---- padding of the scale tiles: rows [rows, rpad) x all kb_pad, and
-    // rows [0, rows) x blocks [kb, kb_pad), for every group.
-    const int64_t kbpad = static_cast<int64_t>(a.sf_ktiles) * 4;
-    const int64_t rows = a.rows;
-    const int64_t rpad = (rows + 127) / 128 * 128;
-    const int64_t n1 = (rpad - rows) * kbpad;
-    const int64_t n2 = rows * (kbpad - a.kb);
-    const int64_t per_group = n1 + n2;
-    const int64_t total = per_group * a.groups;
-    const int64_t stride = static_cast<int64_t>(gridDim.x - a.main_blocks) * blockDim.x;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x - a.main_blocks) * blockDim.x + threadIdx.x;
-         i < total; i += stride) {
-      const int64_t g = i / per_group;
-      const int64_t j = i - g * per_group;
-      int64_t r, c;
-      if (j < n1) {
-        r = rows + j / kbpad;
-        c = j % kbpad;
-      } else {
-        const int64_t jj = j - n1;
-        const int64_t w = kbpad - a.kb;
-        r = jj / w;
-        c = a.kb + jj % w;
-      }
-      a.sf[g * a.sf_group_bytes + sf_tiled_offset(static_cast<uint32_t>(r), static_cast<uint32_t>(c), a.sf_ktiles)] = 0;
+  if (static_cast<int>(blockIdx.x) >= B.main_blocks) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x - B.main_blocks) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x - B.main_blocks) * blockDim.x + threadIdx.x; i < B.pad_total;
+         i += stride) {
+      int j = 0;
+      while (j + 1 < B.count && i >= B.job[j + 1].pad0) ++j;
+      write_padding(B.job[j], i - B.job[j].pad0);
     }
     return;
   }
 
   // ---- streaming part: one lane owns one 32-element block (64 contiguous
   // bytes: four 16-byte loads), so amax, exponent and scale bookkeeping are
-  // done once per block with no shuffles; a warp covers 32 consecutive blocks
-  // (2 KiB) per unrolled slot.
+  // done once per block with no shuffles; a warp covers 32 consecutive
+  // blocks (2 KiB) per unrolled step.
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t warp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const uint32_t nwarps = (static_cast<uint32_t>(a.main_blocks) * blockDim.x) >> 5;
-  constexpr uint32_t kWarpBlocks = 32 * kQuantUnroll;
+  const uint32_t nwarps = (static_cast<uint32_t>(B.main_blocks) * blockDim.x) >> 5;
 
-  for (uint32_t base = warp_id * kWarpBlocks; base < a.nblk; base += nwarps * kWarpBlocks) {
+  for (uint32_t slot = warp_id; slot < B.total_slots; slot += nwarps) {
+    int jn = 0;  // warp-uniform job of this slot
+    while (jn + 1 < B.count && slot >= B.job[jn + 1].slot0) ++jn;
+    const QuantJob& jb = B.job[jn];
+    const uint32_t base = (slot - jb.slot0) * kSlotBlocks;
+
     uint4 v[kQuantUnroll][4];
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const uint32_t b = base + u * 32 + lane;
-      const uint4* src = a.x + static_cast<size_t>(b) * 4;
+      const uint4* src = jb.x + static_cast<size_t>(b) * 4;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[u][j] = b < a.nblk ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < 4; ++j) v[u][j] = b < jb.nblk ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const uint32_t b = base + u * 32 + lane;
-      // amax of |x| on the magnitude bits, two BF16 lanes at a time
+      // amax of |x| on the magnitude bits, two BF16 values per SIMD max
       uint32_t m2 = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -171,72 +190,86 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const QuantArgs
         out0 = make_uint4(o[0], o[1], o[2], o[3]);
         out1 = make_uint4(o[4], o[5], o[6], o[7]);
       }
-      if (b < a.nblk) {
-        uint4* dst = reinterpret_cast<uint4*>(a.q) + static_cast<size_t>(b) * 2;
+      if (b < jb.nblk) {
+        uint4* dst = jb.q + static_cast<size_t>(b) * 2;
         __stcs(dst, out0);
         __stcs(dst + 1, out1);
       }
 
       // scale byte(s): row / K-block of this block, then its group
-      const uint32_t row = fdiv(b, a.div_kb);
-      const uint32_t c = b - row * a.kb;
+      const uint32_t row = fdiv(b, jb.div_kb);
+      const uint32_t c = b - row * jb.kb;
       uint32_t g = 0, rl = row;
-      if (a.groups > 1) {
-        g = fdiv(row, a.div_rows);
-        rl = row - g * a.rows;
+      if (jb.groups > 1) {
+        g = fdiv(row, jb.div_rows);
+        rl = row - g * jb.rows;
       }
-      uint8_t* sfp = a.sf + static_cast<int64_t>(g) * a.sf_group_bytes + sf_tiled_offset(rl, c, a.sf_ktiles);
-      if (a.kb4) {
+      uint8_t* sfp = jb.sf + static_cast<int64_t>(g) * jb.sf_group_bytes + sf_tiled_offset(rl, c, jb.sf_ktiles);
+      if (jb.kb4) {
         // lanes 4j..4j+3 hold K-blocks c..c+3 (c % 4 == 0) of one row: their
         // four scale bytes are adjacent, so lane 4j stores them as one word.
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, scode, 1);
         const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, scode, 2);
         const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, scode, 3);
-        if ((lane & 3u) == 0 && b < a.nblk)
+        if ((lane & 3u) == 0 && b < jb.nblk)
           *reinterpret_cast<uint32_t*>(sfp) = scode | (s1 << 8) | (s2 << 16) | (s3 << 24);
-      } else if (b < a.nblk) {
+      } else if (b < jb.nblk) {
         *sfp = static_cast<uint8_t>(scode);
       }
     }
   }
 }
 
-// Launch helper used by the C ABI (validation happens there).  Needs
-// groups*rows*(k/32) < 2^31 blocks.
-cudaError_t launch_quant(const void* x, int64_t groups, int64_t rows, int64_t k, void* q, void* sf,
-                         int64_t sf_group_bytes, int num_sms, cudaStream_t stream, int* launches) {
-  static int resident = 0;  // CTAs of the kernel one SM holds (same for every B200)
+// Launch helper used by the C ABI (validation happens there): up to
+// kMaxQuantJobs tensors in one launch.  Each job needs groups*rows*(k/32) < 2^31.
+cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, cudaStream_t stream, int* launches) {
+  static int resident = 0;  // CTAs of the kernel one SM holds
   if (resident == 0) {
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, mx_quant_kernel, kQuantThreads, 0);
     if (e != cudaSuccess || resident <= 0) resident = 2048 / kQuantThreads;
   }
-  QuantArgs a;
-  a.x = static_cast<const uint4*>(x);
-  a.q = static_cast<uint2*>(q);
-  a.sf = static_cast<uint8_t*>(sf);
-  a.kb = static_cast<uint32_t>(k / 32);
-  a.rows = static_cast<uint32_t>(rows);
-  a.groups = static_cast<uint32_t>(groups);
-  a.nblk = static_cast<uint32_t>(groups * rows * (k / 32));
-  a.div_kb = make_fastdiv(a.kb);
-  a.div_rows = make_fastdiv(a.rows);
-  a.sf_group_bytes = sf_group_bytes;
-  a.sf_ktiles = (a.kb + 3) / 4;
-  a.kb4 = (a.kb % 4) == 0;
-  const int64_t warps_needed = (static_cast<int64_t>(a.nblk) + 32 * kQuantUnroll - 1) / (32 * kQuantUnroll);
-  const int64_t ctas_needed = (warps_needed + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
+  QuantBatch B = {};
+  uint32_t slots = 0;
+  int64_t pads = 0;
+  int n = 0;
+  for (int i = 0; i < count; ++i) {
+    const QuantSpec& sp = specs[i];
+    if (sp.groups == 0 || sp.rows == 0 || sp.k == 0) continue;
+    QuantJob& jb = B.job[n++];
+    jb.x = static_cast<const uint4*>(sp.x);
+    jb.q = static_cast<uint4*>(sp.q);
+    jb.sf = static_cast<uint8_t*>(sp.sf);
+    jb.kb = static_cast<uint32_t>(sp.k / 32);
+    jb.rows = static_cast<uint32_t>(sp.rows);
+    jb.groups = static_cast<uint32_t>(sp.groups);
+    jb.nblk = static_cast<uint32_t>(sp.groups * sp.rows * (sp.k / 32));
+    jb.div_kb = make_fastdiv(jb.kb);
+    jb.div_rows = make_fastdiv(jb.rows);
+    jb.sf_group_bytes = sp.sf_group_bytes;
+    jb.sf_ktiles = (jb.kb + 3) / 4;
+    jb.kb4 = (jb.kb % 4) == 0;
+    jb.slot0 = slots;
+    slots += (jb.nblk + kSlotBlocks - 1) / kSlotBlocks;
+    const int64_t kbpad = static_cast<int64_t>(jb.sf_ktiles) * 4;
+    const int64_t rpad = (sp.rows + 127) / 128 * 128;
+    jb.pad_n1 = (rpad - sp.rows) * kbpad;
+    jb.pad_per_group = jb.pad_n1 + sp.rows * (kbpad - jb.kb);
+    jb.pad0 = pads;
+    pads += jb.pad_per_group * sp.groups;
+  }
+  if (n == 0) return cudaSuccess;
+  B.count = n;
+  B.total_slots = slots;
+  B.pad_total = pads;
+  const int64_t ctas_needed = (static_cast<int64_t>(slots) + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
   const int64_t max_ctas = static_cast<int64_t>(num_sms) * resident;
-  a.main_blocks = static_cast<int>(ctas_needed < max_ctas ? ctas_needed : max_ctas);
-  const int64_t kbpad = static_cast<int64_t>(a.sf_ktiles) * 4;
-  const int64_t rpad = (rows + 127) / 128 * 128;
-  const int64_t pad_entries = ((rpad - rows) * kbpad + rows * (kbpad - a.kb)) * groups;
+  B.main_blocks = static_cast<int>(ctas_needed < max_ctas ? ctas_needed : max_ctas);
   int pad_blocks = 0;
-  if (pad_entries > 0) {
-    const int64_t want = (pad_entries + kQuantThreads - 1) / kQuantThreads;
+  if (pads > 0) {
+    const int64_t want = (pads + kQuantThreads - 1) / kQuantThreads;
     pad_blocks = static_cast<int>(want < num_sms ? want : num_sms);
   }
-  const int grid = a.main_blocks + pad_blocks;
-  if (grid == 0) return cudaSuccess;
+  const int grid = B.main_blocks + pad_blocks;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(grid, 1, 1);
@@ -247,7 +280,7 @@ cudaError_t launch_quant(const void* x, int64_t groups, int64_t rows, int64_t k,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, mx_quant_kernel, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mx_quant_kernel, B);
   if (e != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaGetLastError();

@@ -33,6 +33,7 @@ def lib():
     L.mx_status_string.restype = ctypes.c_char_p
     L.mx_quantize_bf16_to_e4m3.argtypes = [P, I64, I64, P, P, P]
     L.mx_quantize_bf16_to_e4m3_grouped.argtypes = [P, I64, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3_multi.argtypes = [P, I32, P]
     L.mx_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
     L.mx_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
@@ -97,3 +98,19 @@ def test_grouped_argument_checks(lib):
     assert m(FAKE, FAKE, FAKE, FAKE, None, 4, 256, 256, 128, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
     assert m(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 250, 128, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
     assert m(None, None, None, None, None, 4, 0, 256, 128, None, None, None) == MX_OK
+
+
+def test_quantize_multi_argument_checks(lib):
+    import moe_grouped_gemm_mx_b200 as mx
+    J = mx._QuantJob
+    f = lib.mx_quantize_bf16_to_e4m3_multi
+    jobs = (J * 3)(J(FAKE, 1, 4, 64, FAKE, FAKE), J(FAKE, 1, 4, 48, FAKE, FAKE), J(FAKE, 1, 4, 64, FAKE, FAKE))
+    addr = ctypes.addressof(jobs)
+    assert f(addr, 3, None) == MX_ERR_UNSUPPORTED_SHAPE          # second job: k % 32 != 0, nothing launched
+    jobs[1] = J(FAKE + 8, 1, 4, 64, FAKE, FAKE)
+    assert f(addr, 3, None) == MX_ERR_MISALIGNED
+    assert f(None, 2, None) == MX_ERR_INVALID_ARGUMENT
+    assert f(addr, -1, None) == MX_ERR_INVALID_ARGUMENT
+    assert f(None, 0, None) == MX_OK
+    empty = (J * 2)(J(None, 0, 4, 64, None, None), J(None, 1, 0, 64, None, None))
+    assert f(ctypes.addressof(empty), 2, None) == MX_OK

@@ -115,6 +115,28 @@ def test_page_shapes_full(mx, oracle):
         check_against_oracle(mx, oracle, b)
 
 
+def test_multi_matches_single_and_oracle(mx, oracle):
+    """Nine tensors of assorted shapes (2-D, 3-D, ragged K, one empty) in one
+    batched call: every output bit-identical to the one-tensor call and to
+    the oracle (more than 8 tensors exercises the split into two launches)."""
+    shapes = [(64, 7168), (2112, 256), (3, 130, 160), (1, 32), (0, 64), (300, 224), (129, 96),
+              (2, 128, 512), (5, 7168)]
+    xs = [mx_inputs.outlier_bf16(s, seed=i).cuda() for i, s in enumerate(shapes)]
+    outs = mx.mx_quantize_bf16_to_e4m3_multi(xs)
+    torch.cuda.synchronize()
+    for x, (q, sf) in zip(xs, outs):
+        if x.numel() == 0:
+            continue
+        q1, sf1 = mx.mx_quantize_bf16_to_e4m3(x)
+        torch.cuda.synchronize()
+        assert torch.equal(q, q1) and torch.equal(sf, sf1)
+        groups = 1 if x.dim() == 2 else x.shape[0]
+        rows, k = x.shape[-2], x.shape[-1]
+        q_ref, sf_ref = oracle_quantize(oracle, x.cpu())
+        assert np.array_equal(q.cpu().numpy().reshape(-1, k), q_ref)
+        assert np.array_equal(gpu_sf_rowmajor(oracle, sf, groups, rows, k), sf_ref)
+
+
 def test_empty_is_noop(mx):
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     q, sf = mx.mx_quantize_bf16_to_e4m3(x)
