@@ -74,7 +74,11 @@ struct Layout {
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-  static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+  // epilogue staging: two 128-row x 32-column BF16 chunks (64-byte rows,
+  // 64-byte swizzle) that TMA stores read while the next chunk is written
+  static constexpr int STG_BYTES = BM * 32 * 2;
+  static constexpr int OFF_STG = (OFF_SFB + STAGES * SFB_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_BAR = OFF_STG + 2 * STG_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC + 1;  // + drain barrier
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB0 = OFF_MISC + 16;
@@ -149,8 +153,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32
 
 template <int BN, int STAGES, int ACC, int SPLIT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                   const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ CUtensorMap tmap_d, const GemmArgs args) {
   using L = Layout<BN, STAGES, ACC, SPLIT>;
   // SPLIT > 1 (dense form only): a cluster of SPLIT CTAs shares one output
   // tile, each CTA accumulating a contiguous share of the K tiles; the FP32
@@ -196,6 +200,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_d);
   }
   // Everything above touches only this CTA's shared memory and the kernel
   // parameters.  With programmatic dependent launch the next kernel may begin
@@ -368,12 +373,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t stg_count = 0;  // staging chunks used so far (buffer = count & 1)
     for (int t = t_first; t < total; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
-      // every lane polls; the vote re-converges the warp before the
-      // warp-collective (.sync.aligned) TMEM loads below
+      // every lane polls; the vote over all four epilogue warps re-converges
+      // them before the warp-collective (.sync.aligned) TMEM loads and makes
+      // the give-up decision uniform (the warps share named barriers below)
       const bool got = mbar_wait(accf_bar(acc), acc_phase, abort_flag, kWaitLimitNs);
-      if (!__all_sync(0xFFFFFFFFu, got)) {
-        if (lane == 0) report(args.status, 0x4);
+      if (!named_barrier_and(2, 128, got)) {
+        if (threadIdx.x == 64) report(args.status, 0x4);
         *abort_flag = 1;
         break;
       }
@@ -392,32 +399,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         drow = r;
       }
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
-      __nv_bfloat16* drow_ptr = args.d + drow * args.n;
+      // full tiles leave through TMA stores (the tensor map clips rows and
+      // columns outside D); a masked-layout tile that ends inside the
+      // expert's valid rows is stored row by row from registers
+      const bool use_tma = args.mode != kMasked || (tl.m_blk + 1) * BM <= tab1[tl.group];
+      if (use_tma) {
+        const int z = args.mode == kMasked ? tl.group : 0;
+        const int row0 = tl.m_blk * BM;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tc_ld_32x32b_x32(t_row + c * 32, v);
-        tc_wait_ld();
-        const int col0 = tl.n_blk * BN + c * 32;
-        if (valid) {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tc_ld_32x32b_x32(t_row + c * 32, v);
+          tc_wait_ld();
+          if (c == BN / 32 - 1) {  // accumulator fully read: hand TMEM back to the MMA warp
+            tc_fence_before();
+            mbar_arrive(acce_bar(acc));
+          }
+          const uint32_t buf = stg_count & 1u;
+          const uint32_t stg = sbase + L::OFF_STG + buf * L::STG_BYTES;
+          // the store issued from this buffer two chunks ago must have read it
+          if (threadIdx.x == 64) bulk_wait_group_read<1>();
+          named_barrier_sync(1, 128);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = col0 + g * 8;
-            if (col < args.n) {
-              uint4 w;
-              w.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-              w.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-              w.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-              w.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
-              *reinterpret_cast<uint4*>(drow_ptr + col) = w;
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t w0 = pack_bf16x2(v[j * 8 + 0], v[j * 8 + 1]);
+            const uint32_t w1 = pack_bf16x2(v[j * 8 + 2], v[j * 8 + 3]);
+            const uint32_t w2 = pack_bf16x2(v[j * 8 + 4], v[j * 8 + 5]);
+            const uint32_t w3 = pack_bf16x2(v[j * 8 + 6], v[j * 8 + 7]);
+            const uint32_t off = r_local * 64 + ((j ^ ((r_local >> 1) & 3)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + off), "r"(w0), "r"(w1), "r"(w2),
+                         "r"(w3)
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          named_barrier_sync(1, 128);
+          if (threadIdx.x == 64) {
+            tma_store_3d(&tmap_d, stg, tl.n_blk * BN + c * 32, row0, z);
+            bulk_commit_group();
+          }
+          ++stg_count;
+        }
+      } else {
+        __nv_bfloat16* drow_ptr = args.d + drow * args.n;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tc_ld_32x32b_x32(t_row + c * 32, v);
+          tc_wait_ld();
+          const int col0 = tl.n_blk * BN + c * 32;
+          if (valid) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int col = col0 + g * 8;
+              if (col < args.n) {
+                uint4 w;
+                w.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+                w.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+                w.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+                w.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+                *reinterpret_cast<uint4*>(drow_ptr + col) = w;
+              }
             }
           }
         }
+        tc_fence_before();
+        mbar_arrive(acce_bar(acc));
       }
-      tc_fence_before();
-      mbar_arrive(acce_bar(acc));
       if (++acc == ACC) { acc = 0; acc_phase ^= 1u; }
     }
+    // every TMA store of this CTA must be complete before the CTA exits
+    if (threadIdx.x == 64) bulk_wait_group_all();
   }
 
   if constexpr (SPLIT > 1) {
@@ -509,6 +560,21 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+// 3-D BF16 tensor [depth, rows, n] written in boxes of 128 rows x 32 columns
+// (64-byte rows, 64-byte swizzle, matching the epilogue's staging layout).
+static bool make_tmap_d(CUtensorMap* m, void* base, int64_t n, int64_t rows, int64_t depth) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(depth)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(n * 2), static_cast<cuuint64_t>(n * 2 * rows)};
+  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(BM), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // 3-D byte tensor [depth, rows, k] (k contiguous) read in boxes of box_rows x 128 bytes.
 static bool make_tmap(CUtensorMap* m, const void* base, int64_t k, int64_t rows, int64_t depth, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
@@ -578,11 +644,13 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
     cudaError_t e = prepare_kernel<BN, STAGES, ACC, SPLIT>();
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb;  // operands
   const int64_t a_depth = p.mode == kMasked ? p.groups : 1;
   const int64_t b_depth = p.mode == kDense ? 1 : p.groups;
   if (!make_tmap(&ta, p.qa, p.k, p.m, a_depth, BM)) return cudaErrorInvalidValue;
   if (!make_tmap(&tb, p.qb, p.k, p.n, b_depth, BN)) return cudaErrorInvalidValue;
+  CUtensorMap td;
+  if (!make_tmap_d(&td, p.d, p.n, p.m, a_depth)) return cudaErrorInvalidValue;
 
   GemmArgs a;
   a.sfa = static_cast<const uint8_t*>(p.sfa);
@@ -634,7 +702,7 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, a);
   if (e != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaGetLastError();
