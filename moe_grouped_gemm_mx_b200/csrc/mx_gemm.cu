@@ -31,41 +31,17 @@
 #include <cstdint>
 #include <cstdlib>
 
+#include "mx_gemm_common.cuh"
 #include "mx_launch.h"
-#include "mx_ptx.cuh"
 
 namespace mxk {
 
-constexpr int BM = 128;              // MMA M (rows of A per tile)
-constexpr int BK = 128;              // K elements per pipeline stage (4 scale blocks)
-constexpr int kMaxGroups = 1024;
-constexpr int kGemmThreads = 192;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
-
-enum GemmMode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
-
-struct GemmArgs {
-  const uint8_t* sfa;
-  const uint8_t* sfb;
-  __nv_bfloat16* d;
-  const int32_t* group_offsets;  // contiguous: [groups+1]
-  const int32_t* masked_m;       // masked: [groups]
-  int32_t* status;
-  int64_t sfa_group_bytes;  // masked: tiled scale bytes per expert of A
-  int64_t sfb_group_bytes;  // grouped: tiled scale bytes per expert of B
-  int m;                    // dense: M; contiguous: m_total; masked: max_m
-  int n;
-  int k_tiles;              // K / 128 (also the 512-byte scale tiles per 128-row block)
-  int n_tiles;              // ceil(N / BN)
-  int n_sf_tiles;           // ceil(N / 128)
-  int groups;
-  int mode;
-  int sf_bufs;              // 1 or 2 TMEM buffers for the per-K-tile scale factors
-};
-
-template <int BN, int STAGES, int ACC, int SPLIT = 1>
+// BMA: rows of A one stage holds (128, or 64 for a dense M <= 64, which frees
+// shared memory for deeper pipelining; the M=128 MMA then also reads the next
+// 64 rows of shared memory, which only feed accumulator rows never stored).
+template <int BN, int STAGES, int ACC, int SPLIT = 1, int BMA = BM>
 struct Layout {
-  static constexpr int A_BYTES = BM * BK;
+  static constexpr int A_BYTES = BMA * BK;
   static constexpr int B_BYTES = BN * BK;
   static constexpr int SFA_BYTES = 512;
   static constexpr int SFB_TILES = BN / 128;
@@ -96,66 +72,24 @@ struct Layout {
   // split-K reduction buffer (reuses the operand ring once the mainloop is
   // done): SPLIT partial slices of 128 rows x BN/SPLIT FP32 columns, rows
   // padded by 4 floats to spread shared-memory banks.
-  static constexpr int SLICE = BN / SPLIT;
-  static constexpr int RED_STRIDE = SLICE + 4;
-  static constexpr int RED_BYTES = SPLIT * BM * RED_STRIDE * 4;
+  // Columns are dealt out in quads of 4: CTA o of the cluster owns quads
+  // [ceil(o*QUADS/SPLIT), ceil((o+1)*QUADS/SPLIT)).
+  static constexpr int QUADS = BN / 4;
+  // Receive buffer: [source rank][quad of the slice][row] of float4, rows
+  // fastest, so the 32 lanes of a warp (32 consecutive rows) write 512
+  // contiguous bytes per remote store and read them back conflict-free.
+  static constexpr int MAX_SLICE_QUADS = (QUADS + SPLIT - 1) / SPLIT;
+  static constexpr int RED_BYTES = SPLIT * MAX_SLICE_QUADS * BM * 16;
   static_assert(SPLIT == 1 || RED_BYTES <= OFF_BAR, "reduction buffer must fit in the operand ring");
-  static_assert(SPLIT == 1 || SLICE % 4 == 0, "slices are moved as float4");
+  __host__ __device__ static constexpr int slice_start(int o) { return (o * QUADS + SPLIT - 1) / SPLIT; }
+  __host__ __device__ static constexpr int quad_owner(int q) { return (q * SPLIT) / QUADS; }
 };
 
-struct Tile {
-  int group;
-  int m_blk;  // 128-row block inside the group (masked) or inside A (dense/contiguous)
-  int n_blk;
-};
-
-// Index of the last entry <= v in the non-decreasing table t[0..n] (n+1 entries).
-__device__ __forceinline__ int last_le(const int32_t* t, int n, int32_t v) {
-  int lo = 0, hi = n;  // invariant: t[lo] <= v
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (t[mid] <= v) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-__device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int32_t* tab0, int t) {
-  Tile r;
-  if (a.mode == kMasked) {
-    const int e = last_le(tab0, a.groups, t);  // tab0 = prefix of tiles per expert
-    const int local = t - tab0[e];
-    r.group = e;
-    r.m_blk = local / a.n_tiles;
-    r.n_blk = local - r.m_blk * a.n_tiles;
-  } else {
-    const int mb = t / a.n_tiles;
-    r.n_blk = t - mb * a.n_tiles;
-    if (a.mode == kContiguous) {
-      r.m_blk = tab0[0] / BM + mb;                               // tab0 = group offsets
-      r.group = last_le(tab0, a.groups, r.m_blk * BM);
-      if (r.group >= a.groups) r.group = a.groups - 1;
-    } else {
-      r.m_blk = mb;
-      r.group = 0;
-    }
-  }
-  return r;
-}
-
-__device__ __forceinline__ void report(int32_t* status, int bits) {
-  atomicOr(status, bits);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(lo_f32), __uint_as_float(hi_f32));
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-template <int BN, int STAGES, int ACC, int SPLIT>
+template <int BN, int STAGES, int ACC, int SPLIT, int BMA>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_d, const GemmArgs args) {
-  using L = Layout<BN, STAGES, ACC, SPLIT>;
+  using L = Layout<BN, STAGES, ACC, SPLIT, BMA>;
   // SPLIT > 1 (dense form only): a cluster of SPLIT CTAs shares one output
   // tile, each CTA accumulating a contiguous share of the K tiles; the FP32
   // partials are reduced through distributed shared memory.
@@ -293,7 +227,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         nsfb = nsfb > L::SFB_TILES ? L::SFB_TILES : nsfb;
         for (int kt = kt_begin; kt < kt_end; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          const uint32_t bytes = L::A_BYTES + L::B_BYTES + L::SFA_BYTES + 512u * nsfb;
+          // only the A rows that exist are loaded when M is small; the MMA's
+          // remaining A rows read stale shared memory and only feed
+          // accumulator rows that are never stored
+          const uint32_t bytes = args.a_box_rows * BK + L::B_BYTES + L::SFA_BYTES + 512u * nsfb;
           mbar_arrive_expect_tx(full_bar(stage), bytes);
           tma_load_3d(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, full_bar(stage), kt * BK, a_row, a_z);
           tma_load_3d(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, full_bar(stage), kt * BK,
@@ -329,22 +266,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_t = tmem_base + acc * BN;
-        for (int kt = kt_begin; kt < kt_end; ++kt) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          tc_fence_after();
-          // scale factors of this K tile -> TMEM (alternating buffers when two
-          // are configured, so the copy never targets columns the previous
-          // K tile's MMAs may still be reading)
-          const uint32_t sfa_t = tmem_base + L::SF_COL0 + sf_buf * L::SF_COLS;
-          const uint32_t sfb_t = sfa_t + 4;
-          sf_buf = (sf_buf + 1 == static_cast<uint32_t>(args.sf_bufs)) ? 0u : sf_buf + 1;
-          tc_cp_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + stage * L::SFA_BYTES));
+        // The scale factors of K tile kt+1 are copied into the other TMEM
+        // buffer before the MMAs of K tile kt are issued, so the copy does not
+        // sit between two K tiles' MMAs in the tensor pipe.
+        auto copy_scales = [&](int st, uint32_t buf) {
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + buf * L::SF_COLS;
+          tc_cp_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + st * L::SFA_BYTES));
 #pragma unroll
           for (int j = 0; j < L::SFB_TILES; ++j)
-            tc_cp_32x128b_warpx4(sfb_t + 4 * j,
-                                 desc_sf_32x16(sbase + L::OFF_SFB + stage * L::SFB_BYTES + j * 512));
-          const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES;
-          const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES;
+            tc_cp_32x128b_warpx4(sfa_t + 4 + 4 * j,
+                                 desc_sf_32x16(sbase + L::OFF_SFB + st * L::SFB_BYTES + j * 512));
+        };
+        if (kt_begin < kt_end) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          copy_scales(stage, sf_buf);
+        }
+        for (int kt = kt_begin; kt < kt_end; ++kt) {
+          const int cur = stage;
+          const uint32_t cur_buf = sf_buf;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          sf_buf ^= 1u;
+          if (kt + 1 < kt_end) {
+            if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+            tc_fence_after();
+            copy_scales(stage, sf_buf);
+          }
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + cur_buf * L::SF_COLS;
+          const uint32_t sfb_t = sfa_t + 4;
+          const uint32_t a_addr = sbase + L::OFF_A + cur * L::A_BYTES;
+          const uint32_t b_addr = sbase + L::OFF_B + cur * L::B_BYTES;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             const uint32_t idesc = idesc_with_sf_ids(idesc0, kb, kb);
@@ -352,8 +303,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         sfa_t | (static_cast<uint32_t>(kb) << 30), sfb_t | (static_cast<uint32_t>(kb) << 30),
                         (kt != kt_begin || kb != 0) ? 1u : 0u);
           }
-          tc_commit(empty_bar(stage));
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          tc_commit(empty_bar(cur));
         }
         if (!ok) break;
         tc_commit(accf_bar(acc));
@@ -404,41 +354,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // expert's valid rows is stored row by row from registers
       const bool use_tma = args.mode != kMasked || (tl.m_blk + 1) * BM <= tab1[tl.group];
       if (use_tma) {
-        const int z = args.mode == kMasked ? tl.group : 0;
-        const int row0 = tl.m_blk * BM;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tc_ld_32x32b_x32(t_row + c * 32, v);
-          tc_wait_ld();
-          if (c == BN / 32 - 1) {  // accumulator fully read: hand TMEM back to the MMA warp
-            tc_fence_before();
-            mbar_arrive(acce_bar(acc));
-          }
-          const uint32_t buf = stg_count & 1u;
-          const uint32_t stg = sbase + L::OFF_STG + buf * L::STG_BYTES;
-          // the store issued from this buffer two chunks ago must have read it
-          if (threadIdx.x == 64) bulk_wait_group_read<1>();
-          named_barrier_sync(1, 128);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t w0 = pack_bf16x2(v[j * 8 + 0], v[j * 8 + 1]);
-            const uint32_t w1 = pack_bf16x2(v[j * 8 + 2], v[j * 8 + 3]);
-            const uint32_t w2 = pack_bf16x2(v[j * 8 + 4], v[j * 8 + 5]);
-            const uint32_t w3 = pack_bf16x2(v[j * 8 + 6], v[j * 8 + 7]);
-            const uint32_t off = r_local * 64 + ((j ^ ((r_local >> 1) & 3)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + off), "r"(w0), "r"(w1), "r"(w2),
-                         "r"(w3)
-                         : "memory");
-          }
-          fence_proxy_async_smem();
-          named_barrier_sync(1, 128);
-          if (threadIdx.x == 64) {
-            tma_store_3d(&tmap_d, stg, tl.n_blk * BN + c * 32, row0, z);
-            bulk_commit_group();
-          }
-          ++stg_count;
-        }
+        // drain the whole accumulator row into registers first so TMEM goes
+        // back to the MMA warp before any store is made
+        uint32_t packed[BN / 2];
+        tmem_row_to_bf16<BN>(t_row, packed);
+        tc_fence_before();
+        mbar_arrive(acce_bar(acc));
+        store_rows_tma<BN>(packed, r_local, sbase + L::OFF_STG, stg_count, &tmap_d, tl.n_blk * BN, tl.m_blk * BM,
+                           args.mode == kMasked ? tl.group : 0);
       } else {
         __nv_bfloat16* drow_ptr = args.d + drow * args.n;
 #pragma unroll 1
@@ -495,10 +418,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (valid) {
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
-            const int col = c * 32 + q4 * 4;
-            const int owner = col / L::SLICE;
-            const int cin = col - owner * L::SLICE;
-            const uint32_t local = sbase + ((split_rank * BM + r_local) * L::RED_STRIDE + cin) * 4;
+            const int q = c * 8 + q4;
+            const int owner = L::quad_owner(q);
+            const int cin = (q - L::slice_start(owner)) * 4;
+            const uint32_t local = sbase + ((split_rank * L::MAX_SLICE_QUADS + cin / 4) * BM + r_local) * 16;
             st_cluster_v4(map_to_rank(local, owner), v[q4 * 4 + 0], v[q4 * 4 + 1], v[q4 * 4 + 2], v[q4 * 4 + 3]);
           }
         }
@@ -508,26 +431,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp >= 2 && t_first < total && valid) {
       const float* red = reinterpret_cast<const float*>(smem);
       __nv_bfloat16* drow_ptr = args.d + static_cast<int64_t>(row) * args.n;
-      const int col_base = tl.n_blk * BN + split_rank * L::SLICE;
+      const int q_begin = L::slice_start(split_rank);
+      const int q_end = L::slice_start(split_rank + 1);
 #pragma unroll 1
-      for (int j = 0; j < L::SLICE; j += 8) {
-        float sum[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sum[e] = 0.f;
+      for (int q = q_begin; q < q_end; ++q) {
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int src = 0; src < SPLIT; ++src) {
-          const float4* p = reinterpret_cast<const float4*>(red + (src * BM + r_local) * L::RED_STRIDE + j);
-          const float4 x0 = p[0], x1 = p[1];
-          sum[0] += x0.x; sum[1] += x0.y; sum[2] += x0.z; sum[3] += x0.w;
-          sum[4] += x1.x; sum[5] += x1.y; sum[6] += x1.z; sum[7] += x1.w;
+          const float4 x = *reinterpret_cast<const float4*>(
+              red + ((src * L::MAX_SLICE_QUADS + (q - q_begin)) * BM + r_local) * 4);
+          sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
         }
-        const int col = col_base + j;
+        const int col = tl.n_blk * BN + q * 4;
         if (col < args.n) {
-          uint4 w;
-          w.x = pack_bf16x2(__float_as_uint(sum[0]), __float_as_uint(sum[1]));
-          w.y = pack_bf16x2(__float_as_uint(sum[2]), __float_as_uint(sum[3]));
-          w.z = pack_bf16x2(__float_as_uint(sum[4]), __float_as_uint(sum[5]));
-          w.w = pack_bf16x2(__float_as_uint(sum[6]), __float_as_uint(sum[7]));
-          *reinterpret_cast<uint4*>(drow_ptr + col) = w;
+          uint2 w;
+          w.x = pack_bf16x2(__float_as_uint(sum.x), __float_as_uint(sum.y));
+          w.y = pack_bf16x2(__float_as_uint(sum.z), __float_as_uint(sum.w));
+          *reinterpret_cast<uint2*>(drow_ptr + col) = w;
         }
       }
     }
@@ -544,68 +463,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ======================================================================= host
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 3-D BF16 tensor [depth, rows, n] written in boxes of 128 rows x 32 columns
-// (64-byte rows, 64-byte swizzle, matching the epilogue's staging layout).
-static bool make_tmap_d(CUtensorMap* m, void* base, int64_t n, int64_t rows, int64_t depth) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(n), static_cast<cuuint64_t>(rows),
-                              static_cast<cuuint64_t>(depth)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(n * 2), static_cast<cuuint64_t>(n * 2 * rows)};
-  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(BM), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-// 3-D byte tensor [depth, rows, k] (k contiguous) read in boxes of box_rows x 128 bytes.
-static bool make_tmap(CUtensorMap* m, const void* base, int64_t k, int64_t rows, int64_t depth, int box_rows) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows),
-                              static_cast<cuuint64_t>(depth)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(k * rows)};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// Number of TMEM scale-factor buffers (tuning override MX_GEMM_SFBUF = 1 | 2).
-static int sf_buffers() {
-  static int v = 0;
-  if (v == 0) {
-    const char* env = getenv("MX_GEMM_SFBUF");
-    v = (env && atoi(env) == 1) ? 1 : 2;
-  }
-  return v;
-}
-
 // Raise the kernel's dynamic shared-memory limit (once per process).
-template <int BN, int STAGES, int ACC, int SPLIT>
+template <int BN, int STAGES, int ACC, int SPLIT, int BMA>
 static cudaError_t prepare_kernel() {
   static cudaError_t state = cudaErrorNotReady;
   if (state == cudaErrorNotReady)
-    state = cudaFuncSetAttribute(mx_gemm_kernel<BN, STAGES, ACC, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Layout<BN, STAGES, ACC, SPLIT>::ALLOC);
+    state = cudaFuncSetAttribute(mx_gemm_kernel<BN, STAGES, ACC, SPLIT, BMA>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Layout<BN, STAGES, ACC, SPLIT, BMA>::ALLOC);
   return state;
 }
 
@@ -616,12 +481,12 @@ static int max_active_clusters() {
   static int v = -1;
   if (v < 0) {
     v = 0;
-    if (prepare_kernel<128, 6, 1, SPLIT>() == cudaSuccess) {
+    if (prepare_kernel<128, 6, 1, SPLIT, BM>() == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
       cfg.gridDim = dim3(SPLIT, 1, 1);
       cfg.blockDim = dim3(kGemmThreads, 1, 1);
-      cfg.dynamicSmemBytes = Layout<128, 6, 1, SPLIT>::ALLOC;
+      cfg.dynamicSmemBytes = Layout<128, 6, 1, SPLIT, BM>::ALLOC;
       attr[0].id = cudaLaunchAttributeClusterDimension;
       attr[0].val.clusterDim.x = SPLIT;
       attr[0].val.clusterDim.y = 1;
@@ -629,25 +494,27 @@ static int max_active_clusters() {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_kernel<128, 6, 1, SPLIT>, &cfg) == cudaSuccess) v = n;
+      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_kernel<128, 6, 1, SPLIT, BM>, &cfg) == cudaSuccess) v = n;
       cudaGetLastError();
     }
   }
   return v;
 }
 
-template <int BN, int STAGES, int ACC, int SPLIT>
+template <int BN, int STAGES, int ACC, int SPLIT, int BMA = BM>
 static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
-  using L = Layout<BN, STAGES, ACC, SPLIT>;
-  auto kern = mx_gemm_kernel<BN, STAGES, ACC, SPLIT>;
+  using L = Layout<BN, STAGES, ACC, SPLIT, BMA>;
+  auto kern = mx_gemm_kernel<BN, STAGES, ACC, SPLIT, BMA>;
   {
-    cudaError_t e = prepare_kernel<BN, STAGES, ACC, SPLIT>();
+    cudaError_t e = prepare_kernel<BN, STAGES, ACC, SPLIT, BMA>();
     if (e != cudaSuccess) return e;
   }
   CUtensorMap ta, tb;  // operands
   const int64_t a_depth = p.mode == kMasked ? p.groups : 1;
   const int64_t b_depth = p.mode == kDense ? 1 : p.groups;
-  if (!make_tmap(&ta, p.qa, p.k, p.m, a_depth, BM)) return cudaErrorInvalidValue;
+  const int a_box_rows = (p.mode == kDense && p.m <= 32) ? 32 : (p.mode == kDense && p.m <= 64) ? 64 : BM;
+  if (a_box_rows > BMA) return cudaErrorInvalidValue;
+  if (!make_tmap(&ta, p.qa, p.k, p.m, a_depth, a_box_rows)) return cudaErrorInvalidValue;
   if (!make_tmap(&tb, p.qb, p.k, p.n, b_depth, BN)) return cudaErrorInvalidValue;
   CUtensorMap td;
   if (!make_tmap_d(&td, p.d, p.n, p.m, a_depth)) return cudaErrorInvalidValue;
@@ -668,7 +535,8 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
   a.n_sf_tiles = static_cast<int>((p.n + 127) / 128);
   a.groups = static_cast<int>(p.groups);
   a.mode = p.mode;
-  a.sf_bufs = sf_buffers();
+  a.sf_bufs = 2;
+  a.a_box_rows = a_box_rows;
 
   int64_t m_tiles_bound;
   if (p.mode == kMasked)
@@ -712,12 +580,37 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
 // 128x256 tiles) use the persistent 128x256 kernel; smaller ones first try
 // 128x128 tiles with a double-buffered accumulator, and dense problems that
 // still leave most SMs idle split K across a cluster of 2, 4 or 8 CTAs.
-enum GemmConfig : int { kCfg256 = 0, kCfg128 = 1, kCfgSplit2 = 2, kCfgSplit4 = 3, kCfgSplit8 = 4 };
+enum GemmConfig : int {
+  kCfg256 = 0, kCfg128 = 1, kCfgSplit2 = 2, kCfgSplit4 = 3, kCfgSplit8 = 4, kCfgSplit3 = 5, kCfgSplit6 = 6,
+  kCfgPair = 7
+};
+
+static int split_of(int c) {
+  switch (c) {
+    case kCfgSplit2: return 2;
+    case kCfgSplit3: return 3;
+    case kCfgSplit4: return 4;
+    case kCfgSplit6: return 6;
+    case kCfgSplit8: return 8;
+    default: return 1;
+  }
+}
+
+static int max_clusters_of(int split) {
+  switch (split) {
+    case 2: return max_active_clusters<2>();
+    case 3: return max_active_clusters<3>();
+    case 4: return max_active_clusters<4>();
+    case 6: return max_active_clusters<6>();
+    case 8: return max_active_clusters<8>();
+    default: return 0;
+  }
+}
 
 static int choose_config(const GemmProblem& p, int num_sms) {
   static int forced = -2;
   if (forced == -2) {
-    const char* env = getenv("MX_GEMM_CONFIG");  // tuning override: 0..4
+    const char* env = getenv("MX_GEMM_CONFIG");  // tuning override: 0..7
     forced = env ? atoi(env) : -1;
   }
   const int64_t k_tiles = p.k / BK;
@@ -726,30 +619,49 @@ static int choose_config(const GemmProblem& p, int num_sms) {
   const int64_t t128 = m_blocks * ((p.n + 127) / 128);
   int c;
   if (t256 >= num_sms || p.mode != kDense) {
-    c = t256 >= num_sms ? kCfg256 : (t128 >= num_sms / 2 ? kCfg128 : kCfg256);
+    c = t256 >= num_sms ? kCfgPair : (t128 >= num_sms / 2 ? kCfg128 : kCfgPair);
   } else if (t128 >= (num_sms * 3) / 4) {
     c = kCfg128;
-  } else if (t128 * 8 <= num_sms && k_tiles >= 8 && t128 <= max_active_clusters<8>()) {
-    c = kCfgSplit8;
-  } else if (t128 * 4 <= num_sms && k_tiles >= 4 && t128 <= max_active_clusters<4>()) {
-    c = kCfgSplit4;
-  } else if (t128 * 2 <= num_sms && k_tiles >= 2 && t128 <= max_active_clusters<2>()) {
-    c = kCfgSplit2;
   } else {
+    // the largest split whose clusters all fit at once and leave no SM doubled up
     c = kCfg128;
+    const int order[5] = {kCfgSplit8, kCfgSplit6, kCfgSplit4, kCfgSplit3, kCfgSplit2};
+    for (int i = 0; i < 5; ++i) {
+      const int sp = split_of(order[i]);
+      if (t128 * sp <= num_sms && k_tiles >= sp && t128 <= max_clusters_of(sp)) {
+        c = order[i];
+        break;
+      }
+    }
   }
-  if (forced >= 0 && forced <= 4) {
-    const int need = forced == kCfgSplit2 ? 2 : forced == kCfgSplit4 ? 4 : forced == kCfgSplit8 ? 8 : 1;
-    if (forced < kCfgSplit2 || (p.mode == kDense && k_tiles >= need)) c = forced;
+  if (forced >= 0 && forced <= 7) {
+    const int need = split_of(forced);
+    if (need == 1 || (p.mode == kDense && k_tiles >= need)) c = forced;
   }
   return c;
 }
 
 cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
-  switch (choose_config(p, num_sms)) {
+  const int c = choose_config(p, num_sms);
+  if (c == kCfgPair) return launch_gemm_pair(p, num_sms, stream, launches);
+  if (p.mode == kDense && p.m <= 64) {
+    // A stages of 64 rows: 8 stages in flight instead of 6
+    switch (c) {
+      case kCfg128: return launch_gemm_cfg<128, 8, 2, 1, 64>(p, num_sms, stream, launches);
+      case kCfgSplit2: return launch_gemm_cfg<128, 8, 1, 2, 64>(p, num_sms, stream, launches);
+      case kCfgSplit3: return launch_gemm_cfg<128, 8, 1, 3, 64>(p, num_sms, stream, launches);
+      case kCfgSplit4: return launch_gemm_cfg<128, 8, 1, 4, 64>(p, num_sms, stream, launches);
+      case kCfgSplit6: return launch_gemm_cfg<128, 8, 1, 6, 64>(p, num_sms, stream, launches);
+      case kCfgSplit8: return launch_gemm_cfg<128, 8, 1, 8, 64>(p, num_sms, stream, launches);
+      default: return launch_gemm_cfg<256, 4, 1, 1>(p, num_sms, stream, launches);
+    }
+  }
+  switch (c) {
     case kCfg128: return launch_gemm_cfg<128, 6, 2, 1>(p, num_sms, stream, launches);
     case kCfgSplit2: return launch_gemm_cfg<128, 6, 1, 2>(p, num_sms, stream, launches);
+    case kCfgSplit3: return launch_gemm_cfg<128, 6, 1, 3>(p, num_sms, stream, launches);
     case kCfgSplit4: return launch_gemm_cfg<128, 6, 1, 4>(p, num_sms, stream, launches);
+    case kCfgSplit6: return launch_gemm_cfg<128, 6, 1, 6>(p, num_sms, stream, launches);
     case kCfgSplit8: return launch_gemm_cfg<128, 6, 1, 8>(p, num_sms, stream, launches);
     default: return launch_gemm_cfg<256, 4, 1, 1>(p, num_sms, stream, launches);
   }

@@ -1,0 +1,515 @@
+// mx_gemm2.cu -- CTA-pair MXFP8 GEMM (tcgen05 cta_group::2) for large problems.
+//
+// Same computation and C ABI as the one-CTA kernel in mx_gemm.cu (dense,
+// contiguous-grouped and masked-grouped forms, FP32 accumulation, BF16 out),
+// but two CTAs of a cluster share one 256 x 256 output tile: CTA r holds A
+// rows [128r, 128r+128) and B rows [128r, 128r+128) of the tile in its own
+// shared memory, and one 2-SM MMA, issued by the leader CTA (rank 0), reads
+// both.  Per K step each CTA therefore stages half the B bytes a one-CTA
+// 128 x 256 tile needs for the same math, which lowers the operand feed each
+// SM must sustain -- the limit of the one-CTA kernel on large problems.
+//
+//   warp 0 (both CTAs)   TMA producer: own A half, own B half, the 512-byte
+//                        scale chunk of its own 128 A rows and the two chunks
+//                        of all 256 B rows (every CTA's MMA half needs all N
+//                        scales).  Every load completes on the LEADER's
+//                        full barrier; the leader announces both CTAs' bytes.
+//   warp 1 (leader)      scale chunks -> TMEM (tcgen05.cp, both CTAs), 4 pair
+//                        MMAs per K tile, commits multicast to both CTAs'
+//                        "empty" / "accumulator full" barriers.
+//   warps 2-5 (both)     epilogue of the CTA's own 128 accumulator rows
+//                        (TMEM -> BF16 -> swizzled staging -> TMA store),
+//                        then an arrival on the leader's "accumulator empty".
+//
+// Grouped forms: a pair tile covers 256 rows of ONE expert; with groups
+// aligned to 128 rows, the second CTA's half of an expert's last tile may be
+// past the expert's rows, in which case it is computed but not stored.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "mx_gemm_common.cuh"
+#include "mx_launch.h"
+
+namespace mxk {
+
+constexpr int kPairN = 256;  // N of the pair tile (128 B rows per CTA)
+constexpr int kPairM = 256;  // M of the pair tile (128 A rows per CTA)
+
+template <int STAGES>
+struct PairLayout {
+  static constexpr int A_BYTES = 128 * BK;
+  static constexpr int B_BYTES = 128 * BK;
+  static constexpr int SFA_BYTES = 512;
+  static constexpr int SFB_BYTES = 1024;  // both 128-row scale chunks of the 256 B rows
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+  static constexpr int STG_BYTES = 128 * 32 * 2;
+  static constexpr int OFF_STG = (OFF_SFB + STAGES * SFB_BYTES + 1023) / 1024 * 1024;
+  static constexpr int OFF_BAR = OFF_STG + 2 * STG_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 3;  // full/empty per stage, accf, acce, drain
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_TAB0 = OFF_MISC + 16;
+  static constexpr int OFF_TAB1 = OFF_TAB0 + (kMaxGroups + 1) * 4;
+  static constexpr int BYTES = OFF_TAB1 + (kMaxGroups + 1) * 4;
+  static constexpr int ALLOC = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t SF_COLS = 4 + 8;
+  static constexpr uint32_t SF_COL0 = kPairN;
+  static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(OFF_B % 1024 == 0 && OFF_SFA % 1024 == 0, "swizzled tiles need 1024-B alignment");
+  static_assert(ALLOC <= 232448, "shared memory budget");
+};
+
+struct PairTile {
+  int group;
+  int row0;      // first of the tile's 256 A/D rows (absolute for dense/contiguous, within the expert if masked)
+  int rows_end;  // rows at or beyond this are not stored
+  int n_blk;     // 256-wide column block
+};
+
+__device__ __forceinline__ PairTile decode_pair_tile(const GemmArgs& a, const int32_t* tab0, const int32_t* tab1,
+                                                     int t) {
+  PairTile r;
+  if (a.mode == kDense) {
+    const int mb = t / a.n_tiles;
+    r.group = 0;
+    r.n_blk = t - mb * a.n_tiles;
+    r.row0 = mb * kPairM;
+    r.rows_end = a.m;
+  } else {
+    const int e = last_le(tab0, a.groups, t);  // tab0: prefix of pair tiles per expert
+    const int local = t - tab0[e];
+    const int mb = local / a.n_tiles;
+    r.group = e;
+    r.n_blk = local - mb * a.n_tiles;
+    if (a.mode == kContiguous) {  // tab1: group offsets
+      r.row0 = tab1[e] + mb * kPairM;
+      r.rows_end = tab1[e + 1];
+    } else {  // tab1: clamped masked_m
+      r.row0 = mb * kPairM;
+      r.rows_end = tab1[e];
+    }
+  }
+  return r;
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                        const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ CUtensorMap tmap_sfa,
+                        const __grid_constant__ CUtensorMap tmap_sfb, const GemmArgs args) {
+  using L = PairLayout<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
+  const int pair = static_cast<int>(blockIdx.x) >> 1;
+  const int npairs = static_cast<int>(gridDim.x) >> 1;
+
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile uint32_t* tmem_slot = misc + 0;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* total_slot = reinterpret_cast<volatile int*>(misc + 2);
+  int32_t* tab0 = reinterpret_cast<int32_t*>(smem + L::OFF_TAB0);
+  int32_t* tab1 = reinterpret_cast<int32_t*>(smem + L::OFF_TAB1);
+
+  auto full_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * s; };
+  auto empty_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (STAGES + s); };
+  const uint32_t accf_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES);
+  const uint32_t acce_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 1);
+  const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 2);
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);   // the leader's producer announces both CTAs' bytes
+      mbar_init(empty_bar(s), 1);  // the leader's commit, multicast to both CTAs
+    }
+    mbar_init(accf_bar, 1);
+    mbar_init(acce_bar, 256);      // every epilogue thread of both CTAs
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_d);
+    prefetch_tmap(&tmap_sfa);
+    prefetch_tmap(&tmap_sfb);
+  }
+  pdl_launch_dependents();
+  pdl_wait_prior();
+
+  // scheduling tables: tab1 = offsets (contiguous) / clamped masks (masked),
+  // tab0 = exclusive prefix of pair tiles per expert
+  int bad = 0;
+  if (args.mode != kDense) {
+    if (args.mode == kContiguous) {
+      for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) tab1[i] = __ldg(args.group_offsets + i);
+      __syncthreads();
+      for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) {
+        const int32_t v = tab1[i];
+        if (v < 0 || (v % BM) != 0 || v > args.m) bad = 1;
+        if (i > 0 && v < tab1[i - 1]) bad = 1;
+      }
+    } else {
+      for (int i = threadIdx.x; i < args.groups; i += blockDim.x) {
+        int32_t mm = __ldg(args.masked_m + i);
+        if (mm < 0 || mm > args.m) {
+          bad = 1;
+          mm = mm < 0 ? 0 : args.m;
+        }
+        tab1[i] = mm;
+      }
+    }
+    bad = __syncthreads_or(bad);
+    if (warp == 0) {
+      const int per = (args.groups + 31) / 32;
+      const int lo = lane * per;
+      auto tiles_of = [&](int e) -> int {
+        const int rows = args.mode == kContiguous ? (bad ? 0 : tab1[e + 1] - tab1[e]) : tab1[e];
+        return (rows + kPairM - 1) / kPairM * args.n_tiles;
+      };
+      int sum = 0;
+      for (int i = lo; i < lo + per && i < args.groups; ++i) sum += tiles_of(i);
+      int incl = sum;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int run = incl - sum;
+      for (int i = lo; i < lo + per && i < args.groups; ++i) {
+        tab0[i] = run;
+        run += tiles_of(i);
+      }
+      if (lane == 31) tab0[args.groups] = incl;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(const_cast<uint32_t*>(tmem_slot)), L::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (threadIdx.x == 0) {
+    int total;
+    if (args.mode == kDense) {
+      total = ((args.m + kPairM - 1) / kPairM) * args.n_tiles;
+    } else {
+      total = tab0[args.groups];
+      if (bad && rank == 0) report(args.status, args.mode == kContiguous ? 0x1 : 0x2);
+    }
+    *total_slot = total;
+  }
+  // barriers initialised and TMEM allocated in BOTH CTAs before any cross-CTA traffic
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = *total_slot;
+
+  // ---------------------------------------------------------------- roles
+  if (warp == 0) {
+    if (lane == 0) {
+      // ===== TMA producer (both CTAs); every load completes on the leader's full barrier
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const PairTile tl = decode_pair_tile(args, tab0, tab1, t);
+        const int a_row = tl.row0 + 128 * static_cast<int>(rank);
+        const int a_z = args.mode == kMasked ? tl.group : 0;
+        const int b_z = args.mode == kDense ? 0 : tl.group;
+        const int b_row = tl.n_blk * kPairN + 128 * static_cast<int>(rank);
+        // scale chunks (512 B each) are addressed in units of chunks
+        const int sfa_chunk0 = (args.mode == kMasked ? tl.group * static_cast<int>(args.sfa_group_bytes / 512) : 0) +
+                               (a_row / 128) * args.k_tiles;
+        const int sfb_grp = args.mode == kDense ? 0 : tl.group * static_cast<int>(args.sfb_group_bytes / 512);
+        int nsfb = args.n_sf_tiles - tl.n_blk * 2;
+        nsfb = nsfb > 2 ? 2 : nsfb;
+        // the leader announces the bytes of both CTAs' loads for this stage
+        const uint32_t bytes_pair = 2u * (L::A_BYTES + L::B_BYTES + L::SFA_BYTES + 512u * nsfb);
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          const uint32_t fb = map_to_rank(full_bar(stage), 0);
+          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), bytes_pair);
+          tma_load_3d_pair(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, fb, kt * BK, a_row, a_z);
+          tma_load_3d_pair(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, fb, kt * BK, b_row, b_z);
+          tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, fb, 0, 0, sfa_chunk0 + kt);
+          for (int j = 0; j < nsfb; ++j)
+            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES + j * 512, &tmap_sfb, fb, 0, 0,
+                             sfb_grp + (tl.n_blk * 2 + j) * args.k_tiles + kt);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        report(args.status, 0x4);
+        *abort_flag = 1;
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 1000000ull) { }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ===== MMA issuer (leader only)
+      const uint32_t idesc0 = idesc_mxf8_e4m3(kPairM, kPairN);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase = 0;
+      uint32_t sf_buf = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        if (!mbar_wait(acce_bar, acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        // scale factors of K tile kt+1 go into the other TMEM buffer before
+        // the MMAs of K tile kt are issued
+        auto copy_scales = [&](int st, uint32_t buf) {
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + buf * L::SF_COLS;
+          tc_cp_pair_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + st * L::SFA_BYTES));
+          tc_cp_pair_32x128b_warpx4(sfa_t + 4, desc_sf_32x16(sbase + L::OFF_SFB + st * L::SFB_BYTES));
+          tc_cp_pair_32x128b_warpx4(sfa_t + 8, desc_sf_32x16(sbase + L::OFF_SFB + st * L::SFB_BYTES + 512));
+        };
+        if (args.k_tiles > 0) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          copy_scales(stage, sf_buf);
+        }
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          const int cur = stage;
+          const uint32_t cur_buf = sf_buf;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          sf_buf ^= 1u;
+          if (kt + 1 < args.k_tiles) {
+            if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+            tc_fence_after();
+            copy_scales(stage, sf_buf);
+          }
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + cur_buf * L::SF_COLS;
+          const uint32_t sfb_t = sfa_t + 4;
+          const uint32_t a_addr = sbase + L::OFF_A + cur * L::A_BYTES;
+          const uint32_t b_addr = sbase + L::OFF_B + cur * L::B_BYTES;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint32_t idesc = idesc_with_sf_ids(idesc0, kb, kb);
+            tc_mma_pair_mxf8(tmem_base, desc_kmajor_sw128(a_addr + 32 * kb), desc_kmajor_sw128(b_addr + 32 * kb),
+                             idesc, sfa_t | (static_cast<uint32_t>(kb) << 30),
+                             sfb_t | (static_cast<uint32_t>(kb) << 30), (kt != 0 || kb != 0) ? 1u : 0u);
+          }
+          tc_commit_pair_multicast(empty_bar(cur), 0x3);
+        }
+        if (!ok) break;
+        tc_commit_pair_multicast(accf_bar, 0x3);
+        acc_phase ^= 1u;
+      }
+      if (!ok) {
+        report(args.status, 0x4);
+        *abort_flag = 1;
+        tc_commit_pair_multicast(drain_bar, 0x1);
+        mbar_wait(drain_bar, 0, nullptr, 100000000ull);
+      }
+    }
+  } else {
+    // ===== epilogue (both CTAs): this CTA's 128 accumulator rows
+    const int quarter = warp & 3;
+    const int r_local = quarter * 32 + lane;
+    const uint32_t acce_leader = map_to_rank(acce_bar, 0);
+    uint32_t acc_phase = 0;
+    uint32_t stg_count = 0;
+    for (int t = pair; t < total; t += npairs) {
+      const bool got = mbar_wait(accf_bar, acc_phase, abort_flag, kWaitLimitNs);
+      if (!named_barrier_and(2, 128, got)) {
+        if (threadIdx.x == 64) report(args.status, 0x4);
+        *abort_flag = 1;
+        break;
+      }
+      acc_phase ^= 1u;
+      tc_fence_after();
+      const PairTile tl = decode_pair_tile(args, tab0, tab1, t);
+      const int my_row0 = tl.row0 + 128 * static_cast<int>(rank);
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+      // dense rows past M are clipped by the tensor map; grouped rows past the
+      // expert are not ours to write
+      const bool full = args.mode == kDense ? my_row0 < tl.rows_end : my_row0 + 128 <= tl.rows_end;
+      const bool none = my_row0 >= tl.rows_end;
+      if (none) {
+        tc_fence_before();
+        mbar_arrive_cluster(acce_leader);
+      } else if (full) {
+        uint32_t packed[kPairN / 2];
+        tmem_row_to_bf16<kPairN>(t_row, packed);
+        tc_fence_before();
+        mbar_arrive_cluster(acce_leader);  // TMEM back to the leader's MMA warp before any store
+        store_rows_tma<kPairN>(packed, r_local, sbase + L::OFF_STG, stg_count, &tmap_d, tl.n_blk * kPairN, my_row0,
+                               args.mode == kMasked ? tl.group : 0);
+      } else {
+        // masked expert ending inside this CTA's rows: row-predicated stores
+        const int r = my_row0 + r_local;
+        const bool valid = r < tl.rows_end;
+        __nv_bfloat16* drow_ptr = args.d + (static_cast<int64_t>(tl.group) * args.m + r) * args.n;
+#pragma unroll 1
+        for (int c = 0; c < kPairN / 32; ++c) {
+          uint32_t v[32];
+          tc_ld_32x32b_x32(t_row + c * 32, v);
+          tc_wait_ld();
+          const int col0 = tl.n_blk * kPairN + c * 32;
+          if (valid) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int col = col0 + g * 8;
+              if (col < args.n) {
+                uint4 w;
+                w.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+                w.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+                w.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+                w.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+                *reinterpret_cast<uint4*>(drow_ptr + col) = w;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(acce_leader);
+      }
+    }
+    if (threadIdx.x == 64) bulk_wait_group_all();
+  }
+
+  // ---------------------------------------------------------------- teardown
+  // neither CTA may leave while its peer can still signal its barriers,
+  // read its shared memory or write its TMEM
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::TMEM_COLS);
+  }
+}
+
+// ======================================================================= host
+
+// Scale-factor region viewed as 3-D bytes {16, 32, chunks}: one box is one
+// 512-byte chunk (32 rows x 16 bytes), the tcgen05.cp source matrix.
+static bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t bytes) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {16, 32, static_cast<cuuint64_t>(bytes / 512)};
+  const cuuint64_t strides[2] = {16, 512};
+  const cuuint32_t box[3] = {16, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int STAGES>
+static cudaError_t prepare_pair_kernel() {
+  static cudaError_t state = cudaErrorNotReady;
+  if (state == cudaErrorNotReady)
+    state = cudaFuncSetAttribute(mx_gemm_pair_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 PairLayout<STAGES>::ALLOC);
+  return state;
+}
+
+// Pairs the GPU holds at once (one per two SMs when nothing else runs).
+int pair_kernel_max_pairs(int num_sms) {
+  static int v = -1;
+  if (v < 0) {
+    v = num_sms / 2;
+    if (prepare_pair_kernel<6>() == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      cfg.gridDim = dim3(2, 1, 1);
+      cfg.blockDim = dim3(kGemmThreads, 1, 1);
+      cfg.dynamicSmemBytes = PairLayout<6>::ALLOC;
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_pair_kernel<6>, &cfg) == cudaSuccess && n > 0) v = n;
+      cudaGetLastError();
+    }
+  }
+  return v;
+}
+
+cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
+  constexpr int STAGES = 6;
+  using L = PairLayout<STAGES>;
+  {
+    cudaError_t e = prepare_pair_kernel<STAGES>();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap ta, tb, td, tsa, tsb;
+  const int64_t a_depth = p.mode == kMasked ? p.groups : 1;
+  const int64_t b_depth = p.mode == kDense ? 1 : p.groups;
+  const int64_t sfa_bytes = a_depth * (((p.m + 127) / 128) * 128 * (p.k / 32));
+  const int64_t sfb_bytes = b_depth * (((p.n + 127) / 128) * 128 * (p.k / 32));
+  if (!make_tmap(&ta, p.qa, p.k, p.m, a_depth, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tb, p.qb, p.k, p.n, b_depth, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_d(&td, p.d, p.n, p.m, a_depth)) return cudaErrorInvalidValue;
+  if (!make_tmap_sf(&tsa, p.sfa, sfa_bytes)) return cudaErrorInvalidValue;
+  if (!make_tmap_sf(&tsb, p.sfb, sfb_bytes)) return cudaErrorInvalidValue;
+
+  GemmArgs a = {};
+  a.sfa = static_cast<const uint8_t*>(p.sfa);
+  a.sfb = static_cast<const uint8_t*>(p.sfb);
+  a.d = static_cast<__nv_bfloat16*>(p.d);
+  a.group_offsets = p.group_offsets;
+  a.masked_m = p.masked_m;
+  a.status = p.status;
+  a.k_tiles = static_cast<int>(p.k / BK);
+  a.sfa_group_bytes = ((p.m + 127) / 128) * 128 * (p.k / 32);
+  a.sfb_group_bytes = ((p.n + 127) / 128) * 128 * (p.k / 32);
+  a.m = static_cast<int>(p.m);
+  a.n = static_cast<int>(p.n);
+  a.n_tiles = static_cast<int>((p.n + kPairN - 1) / kPairN);
+  a.n_sf_tiles = static_cast<int>((p.n + 127) / 128);
+  a.groups = static_cast<int>(p.groups);
+  a.mode = p.mode;
+  a.sf_bufs = 2;
+  a.a_box_rows = 128;
+
+  // upper bound of pair tiles (grouped forms: every expert full)
+  int64_t m_blocks;
+  if (p.mode == kDense)
+    m_blocks = (p.m + kPairM - 1) / kPairM;
+  else if (p.mode == kMasked)
+    m_blocks = p.groups * ((p.m + kPairM - 1) / kPairM);
+  else
+    m_blocks = p.m / 128 / 2 + p.groups;  // each expert adds at most one half-used pair tile
+  const int64_t tiles_bound = m_blocks * a.n_tiles;
+  if (tiles_bound == 0) return cudaSuccess;
+  const int64_t max_pairs = pair_kernel_max_pairs(num_sms);
+  const int64_t pairs = tiles_bound < max_pairs ? tiles_bound : max_pairs;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.gridDim = dim3(static_cast<unsigned>(pairs * 2), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::ALLOC;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<STAGES>, ta, tb, td, tsa, tsb, a);
+  if (e != cudaSuccess) return e;
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
+}  // namespace mxk

@@ -34,4 +34,7 @@ struct GemmProblem {
 
 cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches);
 
+// CTA-pair (2-SM MMA) kernel for large problems, any of the three forms.
+cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches);
+
 }  // namespace mxk
