@@ -8,15 +8,21 @@
 //
 //   D[m, n] = sum_b 2^(sa[m,b] + sb[n,b]) * sum_{k in b} e4m3(qa[m,k]) * e4m3(qb[n,k])
 //
-// CTA layout (192 threads, one CTA per SM):
+// CTA layout (224 threads, one CTA per SM):
 //   warp 0      TMA producer: A/B tiles (128-byte swizzled, 3-D tensor maps so
 //               experts never bleed into each other) and the 512-byte scale
 //               tiles (plain bulk copies) into a STAGES-deep shared-memory ring.
-//   warp 1      TMEM owner + MMA issuer: per K-tile, tcgen05.cp the scale tiles
-//               into TMEM, then 4 x tcgen05.mma kind::mxf8f6f4.block_scale
-//               (K = 32 each, scale byte k selected by the scale-factor ids),
-//               accumulating a 128 x BN FP32 tile in TMEM.  tcgen05.commit
-//               frees ring slots and publishes finished accumulators.
+//   warp 6      scale copier: as each stage lands, tcgen05.cp its scale tiles
+//               into that stage's own TMEM scale buffer and commit to the
+//               stage's "scales ready" barrier.
+//   warp 1      TMEM owner + MMA issuer: per K-tile, wait for "scales ready",
+//               then 4 x tcgen05.mma kind::mxf8f6f4.block_scale (K = 32 each,
+//               scale byte k selected by the scale-factor ids), accumulating a
+//               128 x BN FP32 tile in TMEM.  tcgen05.commit frees ring slots
+//               and publishes finished accumulators.  One 128 x 256 x 32 MMA
+//               keeps the tensor pipe busy for about as long as a thread needs
+//               to issue two tcgen05 instructions, so the issuer does nothing
+//               but wait, issue the MMAs and commit.
 //   warps 2..5  epilogue: tcgen05.ld the accumulator (each warp owns the TMEM
 //               lane quarter its warp id selects), round to BF16 and store the
 //               valid rows/columns.
@@ -55,18 +61,21 @@ struct Layout {
   static constexpr int STG_BYTES = BM * 32 * 2;
   static constexpr int OFF_STG = (OFF_SFB + STAGES * SFB_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = OFF_STG + 2 * STG_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC + 1;  // + drain barrier
+  // full / empty / scales-ready per stage, full / empty per accumulator, and
+  // the two drain barriers (MMA issuer, scale copier) used when giving up
+  static constexpr int NUM_BARS = 3 * STAGES + 2 * ACC + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB0 = OFF_MISC + 16;
   static constexpr int OFF_TAB1 = OFF_TAB0 + (kMaxGroups + 1) * 4;
   static constexpr int BYTES = OFF_TAB1 + (kMaxGroups + 1) * 4;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024 B
   static constexpr uint32_t TMEM_COLS = 512;
-  // scale factors in TMEM: up to two buffers of [SFA 4 cols | SFB 4 cols per 128 rows]
+  // scale factors in TMEM: one buffer per pipeline stage of
+  // [SFA 4 cols | SFB 4 cols per 128 rows of B]
   static constexpr uint32_t SF_COLS = 4 + 4 * SFB_TILES;
   static constexpr uint32_t SF_COL0 = ACC * BN;
   static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
-  static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(OFF_B % 1024 == 0 && OFF_SFA % 1024 == 0, "swizzled tiles need 1024-B alignment");
   static_assert(BYTES + 1024 <= 232448, "shared memory budget");
   // split-K reduction buffer (reuses the operand ring once the mainloop is
@@ -115,19 +124,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto empty_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (STAGES + s); };
   auto accf_bar = [&](int a) { return sbase + L::OFF_BAR + 8u * (2 * STAGES + a); };
   auto acce_bar = [&](int a) { return sbase + L::OFF_BAR + 8u * (2 * STAGES + ACC + a); };
-  const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 2 * ACC);
+  auto sfready_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (2 * STAGES + 2 * ACC + s); };
+  const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (3 * STAGES + 2 * ACC);
+  const uint32_t sf_drain_bar = drain_bar + 8u;
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
+      mbar_init(sfready_bar(s), 1);
     }
     for (int a = 0; a < ACC; ++a) {
       mbar_init(accf_bar(a), 1);
       mbar_init(acce_bar(a), 128);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(sf_drain_bar, 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -260,42 +273,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      uint32_t sf_buf = 0;
       bool ok = true;
       for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_t = tmem_base + acc * BN;
-        // The scale factors of K tile kt+1 are copied into the other TMEM
-        // buffer before the MMAs of K tile kt are issued, so the copy does not
-        // sit between two K tiles' MMAs in the tensor pipe.
-        auto copy_scales = [&](int st, uint32_t buf) {
-          const uint32_t sfa_t = tmem_base + L::SF_COL0 + buf * L::SF_COLS;
-          tc_cp_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + st * L::SFA_BYTES));
-#pragma unroll
-          for (int j = 0; j < L::SFB_TILES; ++j)
-            tc_cp_32x128b_warpx4(sfa_t + 4 + 4 * j,
-                                 desc_sf_32x16(sbase + L::OFF_SFB + st * L::SFB_BYTES + j * 512));
-        };
-        if (kt_begin < kt_end) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          tc_fence_after();
-          copy_scales(stage, sf_buf);
-        }
         for (int kt = kt_begin; kt < kt_end; ++kt) {
-          const int cur = stage;
-          const uint32_t cur_buf = sf_buf;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          sf_buf ^= 1u;
-          if (kt + 1 < kt_end) {
-            if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-            tc_fence_after();
-            copy_scales(stage, sf_buf);
-          }
-          const uint32_t sfa_t = tmem_base + L::SF_COL0 + cur_buf * L::SF_COLS;
+          // the copier's commit implies the stage's operands have landed too
+          if (!mbar_wait(sfready_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
           const uint32_t sfb_t = sfa_t + 4;
-          const uint32_t a_addr = sbase + L::OFF_A + cur * L::A_BYTES;
-          const uint32_t b_addr = sbase + L::OFF_B + cur * L::B_BYTES;
+          const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES;
+          const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             const uint32_t idesc = idesc_with_sf_ids(idesc0, kb, kb);
@@ -303,7 +293,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         sfa_t | (static_cast<uint32_t>(kb) << 30), sfb_t | (static_cast<uint32_t>(kb) << 30),
                         (kt != kt_begin || kb != 0) ? 1u : 0u);
           }
-          tc_commit(empty_bar(cur));
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         tc_commit(accf_bar(acc));
@@ -312,10 +303,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) {
         report(args.status, 0x4);
         *abort_flag = 1;
-        // every MMA / copy this thread issued must finish before TMEM is freed
+        // every MMA this thread issued must finish before TMEM is freed
         tc_commit(drain_bar);
         mbar_wait(drain_bar, 0, nullptr, 100000000ull);
       }
+    }
+  } else if (warp == 6) {
+    if (lane == 0) {
+      // ===== scale copier: stage s's scale tiles -> TMEM scale buffer s.
+      // The buffer is free again once the stage's MMAs completed, which the
+      // producer has seen (empty) before it refilled the stage (full).
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
+        for (int kt = kt_begin; kt < kt_end; ++kt) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
+          tc_cp_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + stage * L::SFA_BYTES));
+#pragma unroll
+          for (int j = 0; j < L::SFB_TILES; ++j)
+            tc_cp_32x128b_warpx4(sfa_t + 4 + 4 * j,
+                                 desc_sf_32x16(sbase + L::OFF_SFB + stage * L::SFB_BYTES + j * 512));
+          tc_commit(sfready_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        report(args.status, 0x4);
+        *abort_flag = 1;
+      }
+      // copies still in flight must land before TMEM is freed
+      tc_commit(sf_drain_bar);
+      mbar_wait(sf_drain_bar, 0, nullptr, 100000000ull);
     }
   } else {
     // ===== epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
@@ -408,7 +429,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const Tile tl = decode_tile(args, tab0, t_first);
     const int row = tl.m_blk * BM + r_local;
     const bool valid = row < args.m && !*abort_flag;
-    if (warp >= 2 && t_first < total) {
+    if (warp >= 2 && warp <= 5 && t_first < total) {
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -428,7 +449,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     cluster_sync();
-    if (warp >= 2 && t_first < total && valid) {
+    if (warp >= 2 && warp <= 5 && t_first < total && valid) {
       const float* red = reinterpret_cast<const float*>(smem);
       __nv_bfloat16* drow_ptr = args.d + static_cast<int64_t>(row) * args.n;
       const int q_begin = L::slice_start(split_rank);

@@ -14,9 +14,12 @@
 //                        of all 256 B rows (every CTA's MMA half needs all N
 //                        scales).  Every load completes on the LEADER's
 //                        full barrier; the leader announces both CTAs' bytes.
-//   warp 1 (leader)      scale chunks -> TMEM (tcgen05.cp, both CTAs), 4 pair
-//                        MMAs per K tile, commits multicast to both CTAs'
-//                        "empty" / "accumulator full" barriers.
+//   warp 6 (leader)      scale chunks of each landed stage -> that stage's
+//                        TMEM scale buffer (tcgen05.cp, both CTAs), commit
+//                        to the stage's "scales ready" barrier.
+//   warp 1 (leader)      4 pair MMAs per K tile once its scales are ready,
+//                        commits multicast to both CTAs' "empty" /
+//                        "accumulator full" barriers.
 //   warps 2-5 (both)     epilogue of the CTA's own 128 accumulator rows
 //                        (TMEM -> BF16 -> swizzled staging -> TMA store),
 //                        then an arrival on the leader's "accumulator empty".
@@ -50,7 +53,9 @@ struct PairLayout {
   static constexpr int STG_BYTES = 128 * 32 * 2;
   static constexpr int OFF_STG = (OFF_SFB + STAGES * SFB_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = OFF_STG + 2 * STG_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 3;  // full/empty per stage, accf, acce, drain
+  // full / empty / scales-ready per stage, accf, acce, and the drain barriers
+  // of the MMA issuer and the scale copier
+  static constexpr int NUM_BARS = 3 * STAGES + 4;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB0 = OFF_MISC + 16;
   static constexpr int OFF_TAB1 = OFF_TAB0 + (kMaxGroups + 1) * 4;
@@ -59,7 +64,7 @@ struct PairLayout {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t SF_COLS = 4 + 8;
   static constexpr uint32_t SF_COL0 = kPairN;
-  static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");  // one scale buffer per stage
   static_assert(OFF_B % 1024 == 0 && OFF_SFA % 1024 == 0, "swizzled tiles need 1024-B alignment");
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
@@ -125,16 +130,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t accf_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES);
   const uint32_t acce_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 1);
   const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 2);
+  const uint32_t sf_drain_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 3);
+  auto sfready_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (2 * STAGES + 4 + s); };
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);   // the leader's producer announces both CTAs' bytes
       mbar_init(empty_bar(s), 1);  // the leader's commit, multicast to both CTAs
+      mbar_init(sfready_bar(s), 1);  // the leader's scale-copy commit (leader only)
     }
     mbar_init(accf_bar, 1);
     mbar_init(acce_bar, 256);      // every epilogue thread of both CTAs
     mbar_init(drain_bar, 1);
+    mbar_init(sf_drain_bar, 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -242,10 +251,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), bytes_pair);
           tma_load_3d_pair(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, fb, kt * BK, a_row, a_z);
           tma_load_3d_pair(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, fb, kt * BK, b_row, b_z);
-          tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, fb, 0, 0, sfa_chunk0 + kt);
+          tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, fb, 0, sfa_chunk0 + kt, 0);
           for (int j = 0; j < nsfb; ++j)
-            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES + j * 512, &tmap_sfb, fb, 0, 0,
-                             sfb_grp + (tl.n_blk * 2 + j) * args.k_tiles + kt);
+            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES + j * 512, &tmap_sfb, fb, 0,
+                             sfb_grp + (tl.n_blk * 2 + j) * args.k_tiles + kt, 0);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -258,43 +267,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      // ===== MMA issuer (leader only)
+      // ===== MMA issuer (leader only): wait for a stage's scales, 4 pair MMAs, commit
       const uint32_t idesc0 = idesc_mxf8_e4m3(kPairM, kPairN);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0;
-      uint32_t sf_buf = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs) {
         if (!mbar_wait(acce_bar, acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
-        // scale factors of K tile kt+1 go into the other TMEM buffer before
-        // the MMAs of K tile kt are issued
-        auto copy_scales = [&](int st, uint32_t buf) {
-          const uint32_t sfa_t = tmem_base + L::SF_COL0 + buf * L::SF_COLS;
-          tc_cp_pair_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + st * L::SFA_BYTES));
-          tc_cp_pair_32x128b_warpx4(sfa_t + 4, desc_sf_32x16(sbase + L::OFF_SFB + st * L::SFB_BYTES));
-          tc_cp_pair_32x128b_warpx4(sfa_t + 8, desc_sf_32x16(sbase + L::OFF_SFB + st * L::SFB_BYTES + 512));
-        };
-        if (args.k_tiles > 0) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          tc_fence_after();
-          copy_scales(stage, sf_buf);
-        }
         for (int kt = 0; kt < args.k_tiles; ++kt) {
-          const int cur = stage;
-          const uint32_t cur_buf = sf_buf;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          sf_buf ^= 1u;
-          if (kt + 1 < args.k_tiles) {
-            if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-            tc_fence_after();
-            copy_scales(stage, sf_buf);
-          }
-          const uint32_t sfa_t = tmem_base + L::SF_COL0 + cur_buf * L::SF_COLS;
+          // the copier's commit implies both CTAs' operands of the stage have landed
+          if (!mbar_wait(sfready_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
           const uint32_t sfb_t = sfa_t + 4;
-          const uint32_t a_addr = sbase + L::OFF_A + cur * L::A_BYTES;
-          const uint32_t b_addr = sbase + L::OFF_B + cur * L::B_BYTES;
+          const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES;
+          const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             const uint32_t idesc = idesc_with_sf_ids(idesc0, kb, kb);
@@ -302,7 +291,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              idesc, sfa_t | (static_cast<uint32_t>(kb) << 30),
                              sfb_t | (static_cast<uint32_t>(kb) << 30), (kt != 0 || kb != 0) ? 1u : 0u);
           }
-          tc_commit_pair_multicast(empty_bar(cur), 0x3);
+          tc_commit_pair_multicast(empty_bar(stage), 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         tc_commit_pair_multicast(accf_bar, 0x3);
@@ -314,6 +304,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_commit_pair_multicast(drain_bar, 0x1);
         mbar_wait(drain_bar, 0, nullptr, 100000000ull);
       }
+    }
+  } else if (warp == 6) {
+    if (lane == 0 && rank == 0) {
+      // ===== scale copier (leader only): once both CTAs' stage s has landed,
+      // copy each CTA's scale chunks into its TMEM scale buffer s.  Buffer s
+      // is free again once the stage's MMAs completed, which both producers
+      // have seen (empty) before refilling the stage (full).
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
+          tc_cp_pair_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + stage * L::SFA_BYTES));
+          tc_cp_pair_32x128b_warpx4(sfa_t + 4, desc_sf_32x16(sbase + L::OFF_SFB + stage * L::SFB_BYTES));
+          tc_cp_pair_32x128b_warpx4(sfa_t + 8, desc_sf_32x16(sbase + L::OFF_SFB + stage * L::SFB_BYTES + 512));
+          tc_commit_pair_multicast(sfready_bar(stage), 0x1);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        report(args.status, 0x4);
+        *abort_flag = 1;
+      }
+      // copies still in flight must land before TMEM is freed
+      tc_commit_pair_multicast(sf_drain_bar, 0x1);
+      mbar_wait(sf_drain_bar, 0, nullptr, 100000000ull);
     }
   } else {
     // ===== epilogue (both CTAs): this CTA's 128 accumulator rows
@@ -394,16 +413,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ======================================================================= host
 
-// Scale-factor region viewed as 3-D bytes {16, 32, chunks}: one box is one
-// 512-byte chunk (32 rows x 16 bytes), the tcgen05.cp source matrix.
+// Scale-factor region viewed as rows of 512 bytes (one 512-byte chunk = the
+// tcgen05.cp source matrix per row), typed as 128 x 32-bit words so a whole
+// chunk is one box row: the TMA unit handles it as one request rather than
+// the 32 it needs for a box of 32 rows x 16 bytes.
 static bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t bytes) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[3] = {16, 32, static_cast<cuuint64_t>(bytes / 512)};
-  const cuuint64_t strides[2] = {16, 512};
-  const cuuint32_t box[3] = {16, 32, 1};
+  const cuuint64_t chunks = static_cast<cuuint64_t>(bytes / 512);
+  const cuuint64_t dims[3] = {128, chunks, 1};
+  const cuuint64_t strides[2] = {512, 512 * chunks};
+  const cuuint32_t box[3] = {128, 1, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

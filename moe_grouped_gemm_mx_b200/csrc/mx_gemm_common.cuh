@@ -14,7 +14,7 @@ namespace mxk {
 constexpr int BM = 128;              // MMA M (rows of A per tile)
 constexpr int BK = 128;              // K elements per pipeline stage (4 scale blocks)
 constexpr int kMaxGroups = 1024;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;  // 7 warps: producer, MMA, 4 epilogue, scale copier
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
 enum GemmMode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
