@@ -597,10 +597,12 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
   return cudaGetLastError();
 }
 
-// Tile configuration for one problem.  Large problems (at least a wave of
-// 128x256 tiles) use the persistent 128x256 kernel; smaller ones first try
-// 128x128 tiles with a double-buffered accumulator, and dense problems that
-// still leave most SMs idle split K across a cluster of 2, 4 or 8 CTAs.
+// Tile configuration for one problem.  Large dense and contiguous-grouped
+// problems (at least a wave of 256-row tiles) use the CTA-pair 256x256
+// kernel; masked-grouped problems use the one-CTA persistent 128x256 kernel;
+// smaller ones first try 128x128 tiles with a double-buffered accumulator,
+// and dense problems that still leave most SMs idle split K across a cluster
+// of 2, 3, 4, 6 or 8 CTAs.
 enum GemmConfig : int {
   kCfg256 = 0, kCfg128 = 1, kCfgSplit2 = 2, kCfgSplit4 = 3, kCfgSplit8 = 4, kCfgSplit3 = 5, kCfgSplit6 = 6,
   kCfgPair = 7
@@ -639,7 +641,11 @@ static int choose_config(const GemmProblem& p, int num_sms) {
   const int64_t t256 = m_blocks * ((p.n + 255) / 256);
   const int64_t t128 = m_blocks * ((p.n + 127) / 128);
   int c;
-  if (t256 >= num_sms || p.mode != kDense) {
+  if (p.mode == kMasked) {
+    // decode-style problems stream every expert's weights once: the one-CTA
+    // 128x256 tiles keep the most weight bytes in flight per SM
+    c = t256 >= num_sms ? kCfg256 : kCfg128;
+  } else if (t256 >= num_sms || p.mode != kDense) {
     c = t256 >= num_sms ? kCfgPair : (t128 >= num_sms / 2 ? kCfg128 : kCfgPair);
   } else if (t128 >= (num_sms * 3) / 4) {
     c = kCfg128;

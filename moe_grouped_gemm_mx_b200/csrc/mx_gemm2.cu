@@ -39,13 +39,21 @@ namespace mxk {
 
 constexpr int kPairN = 256;  // N of the pair tile (128 B rows per CTA)
 constexpr int kPairM = 256;  // M of the pair tile (128 A rows per CTA)
+constexpr int kPairKC = 2;   // 128-byte K chunks per pipeline stage (K = 256 per stage)
+constexpr int kPairStages = 3;
 
+// One pipeline stage holds two K chunks of 128 bytes for A and B (each chunk
+// a 128-row x 128-byte swizzled tile, as the MMA descriptor expects) and the
+// matching scale chunks.  Fetching two chunks per TMA operation and issuing 8
+// MMAs per barrier wait and commit halves the per-stage fixed costs (TMA
+// operations, mbarrier round trips) that bounded 128-K stages.
 template <int STAGES>
 struct PairLayout {
-  static constexpr int A_BYTES = 128 * BK;
-  static constexpr int B_BYTES = 128 * BK;
-  static constexpr int SFA_BYTES = 512;
-  static constexpr int SFB_BYTES = 1024;  // both 128-row scale chunks of the 256 B rows
+  static constexpr int CHUNK = 128 * BK;              // 16 KB
+  static constexpr int A_BYTES = kPairKC * CHUNK;
+  static constexpr int B_BYTES = kPairKC * CHUNK;
+  static constexpr int SFA_BYTES = kPairKC * 512;     // [K chunk] of 512-byte scale chunks
+  static constexpr int SFB_BYTES = 2 * kPairKC * 512; // [B 128-row half][K chunk]
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
@@ -62,7 +70,9 @@ struct PairLayout {
   static constexpr int BYTES = OFF_TAB1 + (kMaxGroups + 1) * 4;
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t SF_COLS = 4 + 8;
+  // TMEM scale buffer of one stage: per K chunk [SFA 4 cols | SFB 8 cols]
+  static constexpr uint32_t SF_CHUNK_COLS = 4 + 8;
+  static constexpr uint32_t SF_COLS = kPairKC * SF_CHUNK_COLS;
   static constexpr uint32_t SF_COL0 = kPairN;
   static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");  // one scale buffer per stage
   static_assert(OFF_B % 1024 == 0 && OFF_SFA % 1024 == 0, "swizzled tiles need 1024-B alignment");
@@ -231,30 +241,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      const int k_stages = (args.k_tiles + kPairKC - 1) / kPairKC;
+      // the leader announces the bytes of both CTAs' loads for a stage (boxes
+      // reaching past the tensor are zero-filled and still count in full)
+      const uint32_t bytes_pair = 2u * (L::A_BYTES + L::B_BYTES + L::SFA_BYTES + L::SFB_BYTES);
       for (int t = pair; t < total && ok; t += npairs) {
         const PairTile tl = decode_pair_tile(args, tab0, tab1, t);
         const int a_row = tl.row0 + 128 * static_cast<int>(rank);
         const int a_z = args.mode == kMasked ? tl.group : 0;
         const int b_z = args.mode == kDense ? 0 : tl.group;
         const int b_row = tl.n_blk * kPairN + 128 * static_cast<int>(rank);
-        // scale chunks (512 B each) are addressed in units of chunks
-        const int sfa_chunk0 = (args.mode == kMasked ? tl.group * static_cast<int>(args.sfa_group_bytes / 512) : 0) +
-                               (a_row / 128) * args.k_tiles;
-        const int sfb_grp = args.mode == kDense ? 0 : tl.group * static_cast<int>(args.sfb_group_bytes / 512);
-        int nsfb = args.n_sf_tiles - tl.n_blk * 2;
-        nsfb = nsfb > 2 ? 2 : nsfb;
-        // the leader announces the bytes of both CTAs' loads for this stage
-        const uint32_t bytes_pair = 2u * (L::A_BYTES + L::B_BYTES + L::SFA_BYTES + 512u * nsfb);
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        // scale regions as [128-row block][K chunk] of 512-byte chunks
+        const int sfa_blk =
+            (args.mode == kMasked ? tl.group * static_cast<int>(args.sfa_group_bytes / 512 / args.k_tiles) : 0) +
+            a_row / 128;
+        const int sfb_blk = (args.mode == kDense ? 0 : tl.group * args.n_sf_tiles) + tl.n_blk * 2;
+        for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
           if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), bytes_pair);
-          tma_load_3d_pair(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, fb, kt * BK, a_row, a_z);
-          tma_load_3d_pair(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, fb, kt * BK, b_row, b_z);
-          tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, fb, 0, sfa_chunk0 + kt, 0);
-          for (int j = 0; j < nsfb; ++j)
-            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES + j * 512, &tmap_sfb, fb, 0,
-                             sfb_grp + (tl.n_blk * 2 + j) * args.k_tiles + kt, 0);
+          const int kc = ks * kPairKC;
+          tma_load_4d_pair(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, fb, 0, a_row, kc, a_z);
+          tma_load_4d_pair(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, fb, 0, b_row, kc, b_z);
+          tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, fb, 0, kc, sfa_blk);
+          tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES, &tmap_sfb, fb, 0, kc, sfb_blk);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -276,20 +286,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = pair; t < total && ok; t += npairs) {
         if (!mbar_wait(acce_bar, acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        const int k_stages = (args.k_tiles + kPairKC - 1) / kPairKC;
+        for (int ks = 0; ks < k_stages; ++ks) {
           // the copier's commit implies both CTAs' operands of the stage have landed
           if (!mbar_wait(sfready_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
-          const uint32_t sfb_t = sfa_t + 4;
-          const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES;
-          const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES;
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t idesc = idesc_with_sf_ids(idesc0, kb, kb);
-            tc_mma_pair_mxf8(tmem_base, desc_kmajor_sw128(a_addr + 32 * kb), desc_kmajor_sw128(b_addr + 32 * kb),
-                             idesc, sfa_t | (static_cast<uint32_t>(kb) << 30),
-                             sfb_t | (static_cast<uint32_t>(kb) << 30), (kt != 0 || kb != 0) ? 1u : 0u);
+          for (int c = 0; c < kPairKC; ++c) {
+            // a chunk past K holds zeros with zero-code scales and adds nothing
+            const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS + c * L::SF_CHUNK_COLS;
+            const uint32_t sfb_t = sfa_t + 4;
+            const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES + c * L::CHUNK;
+            const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES + c * L::CHUNK;
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint32_t idesc = idesc_with_sf_ids(idesc0, kb, kb);
+              tc_mma_pair_mxf8(tmem_base, desc_kmajor_sw128(a_addr + 32 * kb),
+                               desc_kmajor_sw128(b_addr + 32 * kb), idesc,
+                               sfa_t | (static_cast<uint32_t>(kb) << 30), sfb_t | (static_cast<uint32_t>(kb) << 30),
+                               (ks != 0 || c != 0 || kb != 0) ? 1u : 0u);
+            }
           }
           tc_commit_pair_multicast(empty_bar(stage), 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -315,13 +331,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs) {
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        const int k_stages = (args.k_tiles + kPairKC - 1) / kPairKC;
+        for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
-          tc_cp_pair_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + stage * L::SFA_BYTES));
-          tc_cp_pair_32x128b_warpx4(sfa_t + 4, desc_sf_32x16(sbase + L::OFF_SFB + stage * L::SFB_BYTES));
-          tc_cp_pair_32x128b_warpx4(sfa_t + 8, desc_sf_32x16(sbase + L::OFF_SFB + stage * L::SFB_BYTES + 512));
+#pragma unroll
+          for (int c = 0; c < kPairKC; ++c) {
+            const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS + c * L::SF_CHUNK_COLS;
+            const uint32_t sfb_s = sbase + L::OFF_SFB + stage * L::SFB_BYTES + c * 512;
+            tc_cp_pair_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + stage * L::SFA_BYTES + c * 512));
+            tc_cp_pair_32x128b_warpx4(sfa_t + 4, desc_sf_32x16(sfb_s));
+            tc_cp_pair_32x128b_warpx4(sfa_t + 8, desc_sf_32x16(sfb_s + kPairKC * 512));
+          }
           tc_commit_pair_multicast(sfready_bar(stage), 0x1);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -413,17 +434,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ======================================================================= host
 
-// Scale-factor region viewed as rows of 512 bytes (one 512-byte chunk = the
-// tcgen05.cp source matrix per row), typed as 128 x 32-bit words so a whole
-// chunk is one box row: the TMA unit handles it as one request rather than
-// the 32 it needs for a box of 32 rows x 16 bytes.
-static bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t bytes) {
+// Operand [depth, rows, k] bytes viewed as 4-D {128, rows, k/128, depth}: one
+// box of {128, 128, kPairKC, 1} brings kPairKC consecutive K chunks of 128
+// rows, each landing as its own 16 KB 128-byte-swizzled tile.
+static bool make_tmap_kc(CUtensorMap* m, const void* base, int64_t k, int64_t rows, int64_t depth) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  const cuuint64_t chunks = static_cast<cuuint64_t>(bytes / 512);
-  const cuuint64_t dims[3] = {128, chunks, 1};
-  const cuuint64_t strides[2] = {512, 512 * chunks};
-  const cuuint32_t box[3] = {128, 1, 1};
+  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(k / 128),
+                              static_cast<cuuint64_t>(depth)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(k), 128, static_cast<cuuint64_t>(k * rows)};
+  const cuuint32_t box[4] = {128, 128, kPairKC, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tiled scale region viewed as 3-D {128 words, K chunks, 128-row blocks}: one
+// 512-byte chunk is one box row of 32-bit words (a single TMA request), and a
+// box of {128, kPairKC, blocks} brings the chunks of kPairKC consecutive K
+// chunks for `blocks` consecutive 128-row blocks.  Chunks past K are
+// zero-filled (scale code 0x00), so they scale zeros to zero.
+static bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t bytes, int64_t k_chunks, int blocks) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t nblk = static_cast<cuuint64_t>(bytes / 512 / k_chunks);
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(k_chunks), nblk};
+  const cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(512 * k_chunks)};
+  const cuuint32_t box[3] = {128, kPairKC, static_cast<cuuint32_t>(blocks)};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -444,12 +482,12 @@ int pair_kernel_max_pairs(int num_sms) {
   static int v = -1;
   if (v < 0) {
     v = num_sms / 2;
-    if (prepare_pair_kernel<6>() == cudaSuccess) {
+    if (prepare_pair_kernel<kPairStages>() == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
       cfg.gridDim = dim3(2, 1, 1);
       cfg.blockDim = dim3(kGemmThreads, 1, 1);
-      cfg.dynamicSmemBytes = PairLayout<6>::ALLOC;
+      cfg.dynamicSmemBytes = PairLayout<kPairStages>::ALLOC;
       attr[0].id = cudaLaunchAttributeClusterDimension;
       attr[0].val.clusterDim.x = 2;
       attr[0].val.clusterDim.y = 1;
@@ -457,7 +495,7 @@ int pair_kernel_max_pairs(int num_sms) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_pair_kernel<6>, &cfg) == cudaSuccess && n > 0) v = n;
+      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_pair_kernel<kPairStages>, &cfg) == cudaSuccess && n > 0) v = n;
       cudaGetLastError();
     }
   }
@@ -465,7 +503,7 @@ int pair_kernel_max_pairs(int num_sms) {
 }
 
 cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
-  constexpr int STAGES = 6;
+  constexpr int STAGES = kPairStages;
   using L = PairLayout<STAGES>;
   {
     cudaError_t e = prepare_pair_kernel<STAGES>();
@@ -476,11 +514,11 @@ cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t str
   const int64_t b_depth = p.mode == kDense ? 1 : p.groups;
   const int64_t sfa_bytes = a_depth * (((p.m + 127) / 128) * 128 * (p.k / 32));
   const int64_t sfb_bytes = b_depth * (((p.n + 127) / 128) * 128 * (p.k / 32));
-  if (!make_tmap(&ta, p.qa, p.k, p.m, a_depth, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap(&tb, p.qb, p.k, p.n, b_depth, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_kc(&ta, p.qa, p.k, p.m, a_depth)) return cudaErrorInvalidValue;
+  if (!make_tmap_kc(&tb, p.qb, p.k, p.n, b_depth)) return cudaErrorInvalidValue;
   if (!make_tmap_d(&td, p.d, p.n, p.m, a_depth)) return cudaErrorInvalidValue;
-  if (!make_tmap_sf(&tsa, p.sfa, sfa_bytes)) return cudaErrorInvalidValue;
-  if (!make_tmap_sf(&tsb, p.sfb, sfb_bytes)) return cudaErrorInvalidValue;
+  if (!make_tmap_sf(&tsa, p.sfa, sfa_bytes, p.k / BK, 1)) return cudaErrorInvalidValue;
+  if (!make_tmap_sf(&tsb, p.sfb, sfb_bytes, p.k / BK, 2)) return cudaErrorInvalidValue;
 
   GemmArgs a = {};
   a.sfa = static_cast<const uint8_t*>(p.sfa);
