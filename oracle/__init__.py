@@ -56,6 +56,14 @@ def lib():
         L.mxo_quantize_block.restype = None
         L.mxo_quantize.argtypes = [P, I64, I64, P, P]
         L.mxo_quantize.restype = None
+        L.mxo_quantize_block_f32.argtypes = [P, P, P]
+        L.mxo_quantize_block_f32.restype = None
+        L.mxo_quantize_f32.argtypes = [P, I64, I64, P, P]
+        L.mxo_quantize_f32.restype = None
+        L.mxo_silu.argtypes = [ctypes.c_double]
+        L.mxo_silu.restype = ctypes.c_double
+        L.mxo_swiglu.argtypes = [P, P, I64, P]
+        L.mxo_swiglu.restype = None
         L.mxo_scale_bytes.argtypes = [I64, I64]
         L.mxo_scale_bytes.restype = I64
         L.mxo_sf_offset.argtypes = [I64, I64, I64]
@@ -138,6 +146,41 @@ def quantize(x):
     sf = np.zeros((rows, k // 32), dtype=np.uint8)
     lib().mxo_quantize(_p(xb), rows, k, _p(q), _p(sf))
     return q, sf
+
+
+def quantize_block_f32(x: np.ndarray):
+    x = np.ascontiguousarray(x, dtype=np.float32).reshape(32)
+    q = np.zeros(32, dtype=np.uint8)
+    s = np.zeros(1, dtype=np.uint8)
+    lib().mxo_quantize_block_f32(_p(x), _p(q), _p(s))
+    return q, int(s[0])
+
+
+def quantize_f32(x: np.ndarray):
+    """FP32 [..., k] -> (q uint8 [rows, k], sf uint8 row-major [rows, k/32]),
+    the same scale and rounding rule as ``quantize``."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    k = x.shape[-1]
+    rows = x.size // k if k else 0
+    assert k % 32 == 0
+    q = np.zeros((rows, k), dtype=np.uint8)
+    sf = np.zeros((rows, k // 32), dtype=np.uint8)
+    lib().mxo_quantize_f32(_p(x), rows, k, _p(q), _p(sf))
+    return q, sf
+
+
+def silu(x: float) -> float:
+    return lib().mxo_silu(x)
+
+
+def swiglu(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """h = silu(g) * u elementwise, fp64."""
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    u = np.ascontiguousarray(u, dtype=np.float64)
+    assert g.shape == u.shape
+    h = np.zeros(g.shape, dtype=np.float64)
+    lib().mxo_swiglu(_p(g), _p(u), g.size, _p(h))
+    return h
 
 
 def scale_bytes(rows: int, k: int) -> int:

@@ -150,15 +150,14 @@ double mxo_bf16_to_double(uint16_t bits)
 
 /* ------------------------------------------------------- block quantiser */
 
-/* Quantise one block of 32 BF16 values: scale selection, then each element
- * scaled by 2^-X (exact in double) and encoded. */
-void mxo_quantize_block(const uint16_t *x, uint8_t *q, uint8_t *scale)
+/* Quantise one block of 32 values (each exactly representable in double):
+ * scale selection, then each element scaled by 2^-X (exact in double) and
+ * encoded. */
+static void quantize_values(const double *v, uint8_t *q, uint8_t *scale)
 {
-    double v[32];
     double amax = 0.0;
     int nonfinite = 0;
     for (int i = 0; i < 32; ++i) {
-        v[i] = mxo_bf16_to_double(x[i]);
         if (!isfinite(v[i]))
             nonfinite = 1;
         else if (fabs(v[i]) > amax)
@@ -184,6 +183,25 @@ void mxo_quantize_block(const uint16_t *x, uint8_t *q, uint8_t *scale)
         q[i] = mxo_e4m3_encode(ldexp(v[i], -X));
 }
 
+/* Quantise one block of 32 BF16 values. */
+void mxo_quantize_block(const uint16_t *x, uint8_t *q, uint8_t *scale)
+{
+    double v[32];
+    for (int i = 0; i < 32; ++i)
+        v[i] = mxo_bf16_to_double(x[i]);
+    quantize_values(v, q, scale);
+}
+
+/* Quantise one block of 32 FP32 values (the same scale and rounding rule;
+ * FP32 is the precision of a GEMM epilogue that requantises its result). */
+void mxo_quantize_block_f32(const float *x, uint8_t *q, uint8_t *scale)
+{
+    double v[32];
+    for (int i = 0; i < 32; ++i)
+        v[i] = (double)x[i];
+    quantize_values(v, q, scale);
+}
+
 /* Quantise a row-major [rows, k] BF16 matrix (k % 32 == 0) along k.
  * q is [rows, k] bytes; sf is the PLAIN row-major [rows, k/32] scale matrix. */
 void mxo_quantize(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, uint8_t *sf)
@@ -193,6 +211,33 @@ void mxo_quantize(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, uint8_
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t c = 0; c < kb; ++c)
             mxo_quantize_block(x + r * k + c * 32, q + r * k + c * 32, sf + r * kb + c);
+}
+
+/* Quantise a row-major [rows, k] FP32 matrix (k % 32 == 0) along k; q and
+ * the plain row-major sf as in mxo_quantize. */
+void mxo_quantize_f32(const float *x, int64_t rows, int64_t k, uint8_t *q, uint8_t *sf)
+{
+    int64_t kb = k / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < kb; ++c)
+            mxo_quantize_block_f32(x + r * k + c * 32, q + r * k + c * 32, sf + r * kb + c);
+}
+
+/* ------------------------------------------------------ SwiGLU */
+
+/* SiLU (the "swish" gate of SwiGLU): x * sigmoid(x) = x / (1 + e^-x). */
+double mxo_silu(double x)
+{
+    return x / (1.0 + exp(-x));
+}
+
+/* h = silu(g) * u elementwise over n values (the expert activation between
+ * the gate/up and the down GEMM of a DeepSeek-V3 MoE expert). */
+void mxo_swiglu(const double *g, const double *u, int64_t n, double *h)
+{
+    for (int64_t i = 0; i < n; ++i)
+        h[i] = mxo_silu(g[i]) * u[i];
 }
 
 /* ------------------------------------------------------ scale tile layout */

@@ -20,6 +20,10 @@ double mxo_bf16_to_double(uint16_t bits);
 
 void mxo_quantize_block(const uint16_t *x, uint8_t *q, uint8_t *scale);
 void mxo_quantize(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, uint8_t *sf);
+void mxo_quantize_block_f32(const float *x, uint8_t *q, uint8_t *scale);
+void mxo_quantize_f32(const float *x, int64_t rows, int64_t k, uint8_t *q, uint8_t *sf);
+double mxo_silu(double x);
+void mxo_swiglu(const double *g, const double *u, int64_t n, double *h);
 
 int64_t mxo_scale_bytes(int64_t rows, int64_t k);
 int64_t mxo_sf_offset(int64_t r, int64_t c, int64_t k);

@@ -366,3 +366,96 @@ def test_grouped_masked_equals_dense_per_group(oracle):
         if mm[e]:
             de, _ = oracle.gemm(qa3[e, :mm[e]], sfa3[e, :mm[e]], qb3[e], sfb3[e])
             assert np.array_equal(d[e, :mm[e]], de)
+
+
+# ---------------------------------------------------------------- SwiGLU and the FP32 quantiser
+# (the fused MoE expert MLP: gate/up GEMM -> silu(gate) * up -> MXFP8 -> down GEMM)
+
+@pytest.mark.parametrize("x", [0.1, 0.5, 1.0, 2.5, 7.0, 19.0, 60.0])
+def test_silu_odd_part_identity(oracle, x):
+    """silu(x) - silu(-x) = x * (sigmoid(x) + sigmoid(-x)) = x exactly."""
+    assert oracle.silu(x) - oracle.silu(-x) == pytest.approx(x, rel=1e-15, abs=1e-300)
+
+
+def test_silu_closed_forms(oracle):
+    assert oracle.silu(0.0) == 0.0
+    # sigmoid(ln 3) = 3/4
+    assert oracle.silu(math.log(3.0)) == pytest.approx(0.75 * math.log(3.0), rel=1e-15)
+    # sigmoid(-ln 3) = 1/4
+    assert oracle.silu(-math.log(3.0)) == pytest.approx(-0.25 * math.log(3.0), rel=1e-15)
+    # saturation: silu(x) -> x for large x, -> 0- for very negative x
+    assert oracle.silu(40.0) == pytest.approx(40.0, rel=1e-15)
+    assert -1e-15 < oracle.silu(-40.0) < 0.0
+    # minimum of silu is about -0.2785 at x about -1.2785 (W(1/e) + 1 solution)
+    xs = np.linspace(-3, 0, 30001)
+    vals = np.array([oracle.silu(float(v)) for v in xs])
+    assert vals.min() == pytest.approx(-0.278464542761074, abs=1e-9)
+
+
+def test_swiglu_definition(oracle):
+    rng = np.random.default_rng(5)
+    g = rng.standard_normal(1000) * 3
+    u = rng.standard_normal(1000)
+    h = oracle.swiglu(g, u)
+    # u = 1 gives silu; u = 0 gives zeros; the gate and up roles are not symmetric
+    np.testing.assert_array_equal(oracle.swiglu(g, np.ones_like(g)), [oracle.silu(float(v)) for v in g])
+    assert not oracle.swiglu(g, np.zeros_like(g)).any()
+    assert np.abs(oracle.swiglu(u, g) - h).max() > 0.1
+    assert oracle.swiglu(np.array([math.log(3.0)]), np.array([2.0]))[0] == pytest.approx(1.5 * math.log(3.0),
+                                                                                        rel=1e-15)
+
+
+def test_quantize_f32_equals_bf16_quantiser_on_bf16_values(oracle):
+    """On values exactly representable in BF16 the FP32 quantiser must give the
+    BF16 quantiser's bytes (one rule for both input precisions)."""
+    g = torch.Generator().manual_seed(11)
+    x = (torch.randn(64, 256, generator=g) * torch.exp2(torch.randint(-20, 20, (64, 1), generator=g).float()))
+    x = x.to(torch.bfloat16)
+    x[3, 5] = 0.0
+    x[7, :32] = 0.0
+    x[9, 40] = float("nan")
+    x[10, 70] = float("-inf")
+    q16, s16 = oracle.quantize(x)
+    q32, s32 = oracle.quantize_f32(x.float().numpy())
+    np.testing.assert_array_equal(q32, q16)
+    np.testing.assert_array_equal(s32, s16)
+
+
+def test_quantize_f32_keeps_fp32_precision(oracle):
+    """A tie at BF16 precision is broken by the extra FP32 bits: with amax 1.75
+    (X = -8), 1.0625 scales to 272, exactly between the E4M3 values 256 and
+    288, and ties to the even code 0x78; 1.0625 * (1 + 2^-20) scales just above
+    the tie and must round up to 0x79.  Both inputs are exact FP32 values."""
+    blk = np.full(32, 0.5, dtype=np.float32)
+    blk[0] = 1.75
+    blk[1] = 1.0625
+    blk[2] = np.float32(1.0625 * (1.0 + 2.0 ** -20))
+    blk[3] = -np.float32(1.0625 * (1.0 + 2.0 ** -20))
+    q, s = oracle.quantize_block_f32(blk)
+    assert s == 127 - 8
+    assert q[0] == 0x7E  # 1.75 * 256 = 448, the largest finite E4M3 value
+    assert q[1] == 0x78
+    assert q[2] == 0x79
+    assert q[3] == 0xF9
+
+
+def test_quantize_f32_special_blocks(oracle):
+    # FP32 subnormals: amax = 2^-130 < 2^-126 -> X clamps to -127, so values
+    # scale by 2^127: 2^-130 -> 2^-3 (code 0x20), 2^-140 -> 2^-13, below half
+    # the smallest E4M3 subnormal 2^-9, -> +0
+    blk = np.zeros(32, dtype=np.float32)
+    blk[0] = np.float32(2.0 ** -130)
+    blk[1] = np.float32(2.0 ** -140)
+    q, s = oracle.quantize_block_f32(blk)
+    assert s == 0
+    assert q[0] == 0x20 and oracle.e4m3_decode(0x20) == 2.0 ** -3
+    assert q[1] == 0x00
+    # non-finite FP32 -> scale 0xFF, elements 0x7F
+    blk = np.ones(32, dtype=np.float32)
+    blk[31] = np.float32("inf")
+    q, s = oracle.quantize_block_f32(blk)
+    assert s == 0xFF and (q == 0x7F).all()
+    # large FP32 magnitudes: amax = 2^100 -> X = 92
+    blk = np.full(32, 2.0 ** 100, dtype=np.float32)
+    q, s = oracle.quantize_block_f32(blk)
+    assert s == 127 + 92 and (q == 0x78).all()
