@@ -162,6 +162,47 @@ mx_status mx_grouped_gemm_masked(const void *qa, const void *sfa, const void *qb
                                  int64_t max_m, int64_t n, int64_t k, void *d_bf16,
                                  int32_t *dev_status, mx_stream_t stream);
 
+/*
+ * Fused first half of an MoE expert MLP: the gate/up GEMM, SwiGLU, and MXFP8
+ * requantisation of the result in one kernel, so the activation never goes
+ * to memory in BF16 (the B200 MoE-training page describes MXFP8 expert
+ * layers between a BF16 -> MXFP8 quantise and the BF16 restore; the
+ * activation between the two expert GEMMs is DeepSeek-V3's SwiGLU).
+ *
+ *   G = A * gate^T, U = A * up^T (FP32 accumulation, as in mx_gemm);
+ *   H = silu(G) * U with silu(x) = x / (1 + e^-x), in FP32;
+ *   H is quantised along its columns in 32-element blocks by the rule of
+ *   mx_quantize_bf16_to_e4m3 applied to the FP32 values.
+ *
+ * qb holds, per expert, the 2*i_dim rows of the gate/up projection stacked as
+ * [gate (i_dim rows); up (i_dim rows)], row-major [groups, 2*i_dim, k]; sfb
+ * its scales (groups regions of mx_scale_bytes(2*i_dim, k) bytes).  qa/sfa
+ * as in the matching plain call.  Outputs: qh E4M3 [rows, i_dim] (row
+ * layout of the matching plain call's D) and sfh its tiled scales
+ * (mx_scale_bytes(rows, i_dim) bytes; per expert for the masked form).
+ * (qh, sfh) is directly the A operand of the down GEMM (K = i_dim).
+ *
+ * Requires k % 128 == 0, i_dim % 128 == 0, 16-byte aligned pointers.  Rows
+ * the plain call leaves untouched (contiguous: at or beyond
+ * group_offsets[groups]; masked: at or beyond masked_m[e]) are left
+ * untouched in qh and sfh too; the dense form writes 0x00 into the scale
+ * padding rows of its last 128-row block.  Errors as for the plain calls.
+ */
+mx_status mx_gemm_swiglu_quant(const void *qa, const void *sfa, const void *qb, const void *sfb, void *qh,
+                               void *sfh, int64_t m, int64_t i_dim, int64_t k, int32_t *dev_status,
+                               mx_stream_t stream);
+
+mx_status mx_grouped_gemm_contiguous_swiglu_quant(const void *qa, const void *sfa, const void *qb,
+                                                  const void *sfb, const int32_t *group_offsets,
+                                                  int32_t groups, int64_t m_total, int64_t i_dim, int64_t k,
+                                                  void *qh, void *sfh, int32_t *dev_status,
+                                                  mx_stream_t stream);
+
+mx_status mx_grouped_gemm_masked_swiglu_quant(const void *qa, const void *sfa, const void *qb,
+                                              const void *sfb, const int32_t *masked_m, int32_t groups,
+                                              int64_t max_m, int64_t i_dim, int64_t k, void *qh, void *sfh,
+                                              int32_t *dev_status, mx_stream_t stream);
+
 /* Copies the library-internal device status word (used when a call got
  * dev_status == NULL) to *host_out and, if clear != 0, resets it.
  * Synchronises the device. */

@@ -24,7 +24,8 @@ import torch
 __all__ = [
     "MXError", "lib_path", "scale_bytes", "mx_quantize_bf16_to_e4m3", "mx_quantize_bf16_to_e4m3_multi",
     "mx_gemm",
-    "mx_grouped_gemm_contiguous", "mx_grouped_gemm_masked", "read_internal_status",
+    "mx_grouped_gemm_contiguous", "mx_grouped_gemm_masked", "mx_gemm_swiglu_quant",
+    "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant", "read_internal_status",
     "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "C_SYMBOLS",
 ]
 
@@ -40,7 +41,8 @@ C_SYMBOLS = [
     "mx_status_string", "mx_scale_bytes", "mx_quantize_bf16_to_e4m3",
     "mx_quantize_bf16_to_e4m3_grouped", "mx_quantize_bf16_to_e4m3_multi", "mx_gemm",
     "mx_grouped_gemm_contiguous",
-    "mx_grouped_gemm_masked", "mx_read_internal_status",
+    "mx_grouped_gemm_masked", "mx_read_internal_status", "mx_gemm_swiglu_quant",
+    "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant",
 ]
 
 
@@ -78,6 +80,12 @@ def _load():
     L.mx_grouped_gemm_contiguous.restype = ctypes.c_int
     L.mx_grouped_gemm_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_masked.restype = ctypes.c_int
+    L.mx_gemm_swiglu_quant.argtypes = [P, P, P, P, P, P, I64, I64, I64, P, P]
+    L.mx_gemm_swiglu_quant.restype = ctypes.c_int
+    L.mx_grouped_gemm_contiguous_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
+    L.mx_grouped_gemm_contiguous_swiglu_quant.restype = ctypes.c_int
+    L.mx_grouped_gemm_masked_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
+    L.mx_grouped_gemm_masked_swiglu_quant.restype = ctypes.c_int
     L.mx_read_internal_status.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
     L.mx_read_internal_status.restype = ctypes.c_int
     return L
@@ -238,6 +246,79 @@ def mx_grouped_gemm_masked(qa, sfa, qb, sfb, masked_m: torch.Tensor, d: torch.Te
                                      max_m, n, k, _ptr(d), _status_arg(dev_status), _stream(stream))
     _raise(st, "mx_grouped_gemm_masked")
     return d
+
+
+def _swiglu_out(rows_shape, i_dim, groups, rows_per_group, qh, sfh, device):
+    if qh is None:
+        qh = torch.empty(rows_shape + (i_dim,), dtype=torch.uint8, device=device)
+    if sfh is None:
+        sfh = torch.empty(groups * scale_bytes(rows_per_group, i_dim), dtype=torch.uint8, device=device)
+    _check(qh, torch.uint8, "qh")
+    _check(sfh, torch.uint8, "sfh")
+    if qh.numel() != int(torch.tensor(rows_shape).prod()) * i_dim or \
+            sfh.numel() < groups * scale_bytes(rows_per_group, i_dim):
+        raise ValueError("output buffers too small")
+    return qh, sfh
+
+
+def mx_gemm_swiglu_quant(qa, sfa, qb, sfb, qh: torch.Tensor | None = None, sfh: torch.Tensor | None = None,
+                         dev_status: torch.Tensor | None = None, stream=None):
+    """Fused gate/up GEMM + SwiGLU + MXFP8: qa uint8 [M, K], qb uint8
+    [2I, K] = [gate; up] -> (qh uint8 [M, I], sfh tiled scales)."""
+    for t, nm in ((qa, "qa"), (sfa, "sfa"), (qb, "qb"), (sfb, "sfb")):
+        _check(t, torch.uint8, nm)
+    m, k = qa.shape
+    n2, kb = qb.shape
+    if kb != k or n2 % 2:
+        raise ValueError("shape mismatch")
+    i_dim = n2 // 2
+    qh, sfh = _swiglu_out((m,), i_dim, 1, m, qh, sfh, qa.device)
+    st = _lib.mx_gemm_swiglu_quant(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(qh), _ptr(sfh), m, i_dim, k,
+                                   _status_arg(dev_status), _stream(stream))
+    _raise(st, "mx_gemm_swiglu_quant")
+    return qh, sfh
+
+
+def mx_grouped_gemm_contiguous_swiglu_quant(qa, sfa, qb, sfb, group_offsets: torch.Tensor,
+                                            qh: torch.Tensor | None = None, sfh: torch.Tensor | None = None,
+                                            dev_status: torch.Tensor | None = None, stream=None):
+    """Contiguous layout: qa uint8 [M_total, K], qb uint8 [E, 2I, K] ([gate; up]
+    per expert), group_offsets int32 [E+1] -> (qh uint8 [M_total, I], sfh)."""
+    for t, nm in ((qa, "qa"), (sfa, "sfa"), (qb, "qb"), (sfb, "sfb")):
+        _check(t, torch.uint8, nm)
+    _check(group_offsets, torch.int32, "group_offsets")
+    m_total, k = qa.shape
+    groups, n2, kb = qb.shape
+    if kb != k or n2 % 2 or group_offsets.numel() != groups + 1:
+        raise ValueError("shape mismatch")
+    i_dim = n2 // 2
+    qh, sfh = _swiglu_out((m_total,), i_dim, 1, m_total, qh, sfh, qa.device)
+    st = _lib.mx_grouped_gemm_contiguous_swiglu_quant(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(group_offsets),
+                                                      groups, m_total, i_dim, k, _ptr(qh), _ptr(sfh),
+                                                      _status_arg(dev_status), _stream(stream))
+    _raise(st, "mx_grouped_gemm_contiguous_swiglu_quant")
+    return qh, sfh
+
+
+def mx_grouped_gemm_masked_swiglu_quant(qa, sfa, qb, sfb, masked_m: torch.Tensor,
+                                        qh: torch.Tensor | None = None, sfh: torch.Tensor | None = None,
+                                        dev_status: torch.Tensor | None = None, stream=None):
+    """Masked layout: qa uint8 [E, max_m, K], qb uint8 [E, 2I, K], masked_m int32
+    [E] -> (qh uint8 [E, max_m, I], sfh with one scale region per expert)."""
+    for t, nm in ((qa, "qa"), (sfa, "sfa"), (qb, "qb"), (sfb, "sfb")):
+        _check(t, torch.uint8, nm)
+    _check(masked_m, torch.int32, "masked_m")
+    groups, max_m, k = qa.shape
+    g2, n2, kb = qb.shape
+    if g2 != groups or kb != k or n2 % 2 or masked_m.numel() != groups:
+        raise ValueError("shape mismatch")
+    i_dim = n2 // 2
+    qh, sfh = _swiglu_out((groups, max_m), i_dim, groups, max_m, qh, sfh, qa.device)
+    st = _lib.mx_grouped_gemm_masked_swiglu_quant(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(masked_m),
+                                                  groups, max_m, i_dim, k, _ptr(qh), _ptr(sfh),
+                                                  _status_arg(dev_status), _stream(stream))
+    _raise(st, "mx_grouped_gemm_masked_swiglu_quant")
+    return qh, sfh
 
 
 def read_internal_status(clear: bool = True) -> int:

@@ -197,6 +197,83 @@ mx_status mx_grouped_gemm_masked(const void* qa, const void* sfa, const void* qb
   return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
 }
 
+// ---------------------------------------------------------------- fused SwiGLU + MXFP8 (expert MLP, first half)
+
+static mx_status check_swiglu(const void* qh, const void* sfh, int64_t i_dim) {
+  if (i_dim <= 0) return MX_ERR_INVALID_ARGUMENT;
+  if (i_dim % 128 != 0 || 2 * i_dim > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (!qh || !sfh) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(qh) || !aligned16(sfh)) return MX_ERR_MISALIGNED;
+  return MX_OK;
+}
+
+mx_status mx_gemm_swiglu_quant(const void* qa, const void* sfa, const void* qb, const void* sfb, void* qh,
+                               void* sfh, int64_t m, int64_t i_dim, int64_t k, int32_t* dev_status,
+                               mx_stream_t stream) {
+  if (m < 0 || i_dim < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k == 0 || k % 128 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (m == 0) return i_dim % 128 == 0 ? MX_OK : MX_ERR_UNSUPPORTED_SHAPE;
+  mx_status st = check_swiglu(qh, sfh, i_dim);
+  if (st != MX_OK) return st;
+  st = check_gemm_common(qa, sfa, qb, sfb, qh, m, 2 * i_dim, k, 1);
+  if (st != MX_OK) return st;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  mxk::GemmProblem p{qa, sfa, qb, sfb, qh, nullptr, nullptr, status, m, 2 * i_dim, k, 1, 0};
+  p.i_dim = i_dim;
+  p.sf_out = sfh;
+  return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+mx_status mx_grouped_gemm_contiguous_swiglu_quant(const void* qa, const void* sfa, const void* qb, const void* sfb,
+                                                  const int32_t* group_offsets, int32_t groups, int64_t m_total,
+                                                  int64_t i_dim, int64_t k, void* qh, void* sfh,
+                                                  int32_t* dev_status, mx_stream_t stream) {
+  if (groups < 0 || m_total < 0 || i_dim < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k == 0 || k % 128 != 0 || i_dim % 128 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (groups == 0 || m_total == 0 || i_dim == 0) return MX_OK;
+  if (!group_offsets) return MX_ERR_INVALID_ARGUMENT;
+  mx_status st = check_swiglu(qh, sfh, i_dim);
+  if (st != MX_OK) return st;
+  st = check_gemm_common(qa, sfa, qb, sfb, qh, m_total, 2 * i_dim, k, groups);
+  if (st != MX_OK) return st;
+  if (reinterpret_cast<uintptr_t>(group_offsets) & 3u) return MX_ERR_MISALIGNED;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  mxk::GemmProblem p{qa, sfa, qb, sfb, qh, group_offsets, nullptr, status, m_total, 2 * i_dim, k, groups, 1};
+  p.i_dim = i_dim;
+  p.sf_out = sfh;
+  return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+mx_status mx_grouped_gemm_masked_swiglu_quant(const void* qa, const void* sfa, const void* qb, const void* sfb,
+                                              const int32_t* masked_m, int32_t groups, int64_t max_m, int64_t i_dim,
+                                              int64_t k, void* qh, void* sfh, int32_t* dev_status,
+                                              mx_stream_t stream) {
+  if (groups < 0 || max_m < 0 || i_dim < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k == 0 || k % 128 != 0 || i_dim % 128 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (groups == 0 || max_m == 0 || i_dim == 0) return MX_OK;
+  if (!masked_m) return MX_ERR_INVALID_ARGUMENT;
+  if (groups * max_m > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  mx_status st = check_swiglu(qh, sfh, i_dim);
+  if (st != MX_OK) return st;
+  st = check_gemm_common(qa, sfa, qb, sfb, qh, max_m, 2 * i_dim, k, groups);
+  if (st != MX_OK) return st;
+  if (reinterpret_cast<uintptr_t>(masked_m) & 3u) return MX_ERR_MISALIGNED;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  mxk::GemmProblem p{qa, sfa, qb, sfb, qh, nullptr, masked_m, status, max_m, 2 * i_dim, k, groups, 2};
+  p.i_dim = i_dim;
+  p.sf_out = sfh;
+  return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
 mx_status mx_read_internal_status(int32_t* host_out, int clear) {
   if (!host_out) return MX_ERR_INVALID_ARGUMENT;
   if (cudaDeviceSynchronize() != cudaSuccess) return MX_ERR_CUDA;

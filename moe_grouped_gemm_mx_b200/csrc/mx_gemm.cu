@@ -540,7 +540,7 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
   CUtensorMap td;
   if (!make_tmap_d(&td, p.d, p.n, p.m, a_depth)) return cudaErrorInvalidValue;
 
-  GemmArgs a;
+  GemmArgs a = {};
   a.sfa = static_cast<const uint8_t*>(p.sfa);
   a.sfb = static_cast<const uint8_t*>(p.sfb);
   a.d = static_cast<__nv_bfloat16*>(p.d);
@@ -556,7 +556,6 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
   a.n_sf_tiles = static_cast<int>((p.n + 127) / 128);
   a.groups = static_cast<int>(p.groups);
   a.mode = p.mode;
-  a.sf_bufs = 2;
   a.a_box_rows = a_box_rows;
 
   int64_t m_tiles_bound;
@@ -669,6 +668,7 @@ static int choose_config(const GemmProblem& p, int num_sms) {
 }
 
 cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
+  if (p.i_dim > 0) return launch_gemm_pair(p, num_sms, stream, launches);  // fused SwiGLU: CTA-pair kernel only
   const int c = choose_config(p, num_sms);
   if (c == kCfgPair) return launch_gemm_pair(p, num_sms, stream, launches);
   if (p.mode == kDense && p.m <= 64) {

@@ -29,6 +29,7 @@
 // past the expert's rows, in which case it is computed but not stored.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -112,7 +113,54 @@ __device__ __forceinline__ PairTile decode_pair_tile(const GemmArgs& a, const in
   return r;
 }
 
-template <int STAGES>
+// ---------------------------------------------------------------- fused SwiGLU + MXFP8 epilogue
+
+// h = silu(g) * u in FP32, with the logistic function evaluated on -|g| so
+// that neither the exponential nor the division can overflow.
+__device__ __forceinline__ float swiglu_f32(float g, float u) {
+  const float t = __expf(-fabsf(g));       // (0, 1]
+  const float r = __fdividef(1.0f, 1.0f + t);  // sigmoid(|g|)
+  const float sig = g >= 0.0f ? r : t * r;     // sigmoid(g)
+  return g * sig * u;
+}
+
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// MXFP8 quantisation of 32 FP32 values (the BF16 quantiser's rule applied to
+// FP32 input): X = floor(log2 amax) - 8 clamped to [-127, 127] (amax 0 gives
+// -127), elements x * 2^-X with saturating round-to-nearest-even; a block
+// holding NaN or Inf gets scale 0xFF and elements 0x7F.  amax is taken on the
+// integer magnitude bits (order-preserving for IEEE patterns, and >= 0x7f800000
+// exactly for Inf/NaN).  Returns the scale byte; q receives 32 bytes.
+__device__ __forceinline__ uint32_t quant_block32_f32(const float (&h)[32], uint32_t (&q)[8]) {
+  uint32_t amax = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) amax = max(amax, __float_as_uint(h[j]) & 0x7FFFFFFFu);
+  if (amax >= 0x7F800000u) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = 0x7F7F7F7Fu;
+    return 0xFFu;
+  }
+  int x = -127;
+  if (amax != 0) {
+    const int e = static_cast<int>(amax >> 23);
+    const int fl = e > 0 ? e - 127 : (31 - __clz(amax & 0x7FFFFFu)) - 149;  // subnormal: m * 2^-149
+    x = fl - 8;
+    x = x < -127 ? -127 : (x > 127 ? 127 : x);
+  }
+  // 2^-X as an FP32 bit pattern: finite FP32 input keeps X <= 119, so the
+  // exponent field 127 - X lies in [8, 254]
+  const float s = __uint_as_float(static_cast<uint32_t>(127 - x) << 23);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = e4m3x4(h[4 * i] * s, h[4 * i + 1] * s, h[4 * i + 2] * s, h[4 * i + 3] * s);
+  return static_cast<uint32_t>(x + 127);
+}
+
+template <int STAGES, bool SWIGLU>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                         const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ CUtensorMap tmap_sfa,
@@ -250,12 +298,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int a_row = tl.row0 + 128 * static_cast<int>(rank);
         const int a_z = args.mode == kMasked ? tl.group : 0;
         const int b_z = args.mode == kDense ? 0 : tl.group;
-        const int b_row = tl.n_blk * kPairN + 128 * static_cast<int>(rank);
+        // SwiGLU: CTA 0 takes the 128 gate rows and CTA 1 the matching 128 up
+        // rows of the column block, so each CTA's accumulator row holds
+        // [gate | up] of the same 128 output columns
+        const int b_row = SWIGLU ? (rank != 0 ? args.swiglu_i : 0) + tl.n_blk * 128
+                                 : tl.n_blk * kPairN + 128 * static_cast<int>(rank);
         // scale regions as [128-row block][K chunk] of 512-byte chunks
         const int sfa_blk =
             (args.mode == kMasked ? tl.group * static_cast<int>(args.sfa_group_bytes / 512 / args.k_tiles) : 0) +
             a_row / 128;
-        const int sfb_blk = (args.mode == kDense ? 0 : tl.group * args.n_sf_tiles) + tl.n_blk * 2;
+        const int sfb_grp = args.mode == kDense ? 0 : tl.group * args.n_sf_tiles;
+        const int sfb_blk = sfb_grp + (SWIGLU ? tl.n_blk : tl.n_blk * 2);
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
@@ -264,7 +317,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_4d_pair(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, fb, 0, a_row, kc, a_z);
           tma_load_4d_pair(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, fb, 0, b_row, kc, b_z);
           tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, fb, 0, kc, sfa_blk);
-          tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES, &tmap_sfb, fb, 0, kc, sfb_blk);
+          if (SWIGLU) {  // gate and up scale blocks are i/128 blocks apart: two boxes of one block
+            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES, &tmap_sfb, fb, 0, kc, sfb_blk);
+            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES + kPairKC * 512, &tmap_sfb, fb, 0, kc,
+                             sfb_blk + args.swiglu_i / 128);
+          } else {
+            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES, &tmap_sfb, fb, 0, kc, sfb_blk);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -378,6 +437,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // expert are not ours to write
       const bool full = args.mode == kDense ? my_row0 < tl.rows_end : my_row0 + 128 <= tl.rows_end;
       const bool none = my_row0 >= tl.rows_end;
+      if constexpr (SWIGLU) {
+        // ---- H = silu(gate) * up, requantised to MXFP8 along its columns:
+        // each thread owns one row, so a 32-column block is thread-local
+        if (none) {
+          tc_fence_before();
+          mbar_arrive_cluster(acce_leader);
+          continue;
+        }
+        uint32_t qw[32];  // the row's 128 E4M3 bytes
+        uint32_t sfw = 0; // its 4 scale bytes (column blocks 4*n_blk .. 4*n_blk+3)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          uint32_t g[32], u[32];
+          tc_ld_32x32b_x32(t_row + b * 32, g);
+          tc_ld_32x32b_x32(t_row + 128 + b * 32, u);
+          tc_wait_ld();
+          float h[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) h[j] = swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]));
+          uint32_t q8[8];
+          sfw |= quant_block32_f32(h, q8) << (8 * b);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) qw[b * 8 + i] = q8[i];
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(acce_leader);  // TMEM back to the leader's MMA warp before any store
+        const int r = my_row0 + r_local;   // absolute row (dense, contiguous) or row within the expert (masked)
+        const bool valid = r < tl.rows_end;
+        // scales: the 4 bytes of this row for column blocks 4*n_blk..+3 are
+        // adjacent in the tiled layout (rows padded to 128, i/128 tiles per row block)
+        uint8_t* sfh = args.sfh + (args.mode == kMasked ? tl.group * args.sfh_group_bytes : 0);
+        const int64_t sf_off = (static_cast<int64_t>(r >> 7) * (args.swiglu_i / 128) + tl.n_blk) * 512 +
+                               (r & 31) * 16 + ((r & 127) >> 5) * 4;
+        if (valid)
+          *reinterpret_cast<uint32_t*>(sfh + sf_off) = sfw;
+        else if (args.mode == kDense)
+          *reinterpret_cast<uint32_t*>(sfh + sf_off) = 0u;  // scale padding rows of the last row block
+        if (full) {
+          store_words_tma<32, 64>(qw, r_local, sbase + L::OFF_STG, stg_count, &tmap_d, tl.n_blk * 128, my_row0,
+                                  args.mode == kMasked ? tl.group : 0);
+        } else if (valid) {
+          // masked expert ending inside this CTA's rows: row-predicated stores
+          uint4* hrow = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(args.d) +
+                                                 (static_cast<int64_t>(tl.group) * args.m + r) * args.swiglu_i +
+                                                 tl.n_blk * 128);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) hrow[i] = make_uint4(qw[4 * i], qw[4 * i + 1], qw[4 * i + 2], qw[4 * i + 3]);
+        }
+        continue;
+      }
       if (none) {
         tc_fence_before();
         mbar_arrive_cluster(acce_leader);
@@ -468,11 +577,11 @@ static bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t bytes, int64_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int STAGES>
+template <int STAGES, bool SWIGLU>
 static cudaError_t prepare_pair_kernel() {
   static cudaError_t state = cudaErrorNotReady;
   if (state == cudaErrorNotReady)
-    state = cudaFuncSetAttribute(mx_gemm_pair_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    state = cudaFuncSetAttribute(mx_gemm_pair_kernel<STAGES, SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  PairLayout<STAGES>::ALLOC);
   return state;
 }
@@ -482,7 +591,7 @@ int pair_kernel_max_pairs(int num_sms) {
   static int v = -1;
   if (v < 0) {
     v = num_sms / 2;
-    if (prepare_pair_kernel<kPairStages>() == cudaSuccess) {
+    if (prepare_pair_kernel<kPairStages, false>() == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
       cfg.gridDim = dim3(2, 1, 1);
@@ -495,20 +604,23 @@ int pair_kernel_max_pairs(int num_sms) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_pair_kernel<kPairStages>, &cfg) == cudaSuccess && n > 0) v = n;
+      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_pair_kernel<kPairStages, false>, &cfg) == cudaSuccess && n > 0) v = n;
       cudaGetLastError();
     }
   }
   return v;
 }
 
-cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
+template <bool SWIGLU>
+static cudaError_t launch_pair(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
   constexpr int STAGES = kPairStages;
   using L = PairLayout<STAGES>;
   {
-    cudaError_t e = prepare_pair_kernel<STAGES>();
+    cudaError_t e = prepare_pair_kernel<STAGES, SWIGLU>();
     if (e != cudaSuccess) return e;
   }
+  if (SWIGLU && (p.i_dim <= 0 || p.i_dim % 128 != 0 || p.n != 2 * p.i_dim || !p.sf_out))
+    return cudaErrorInvalidValue;
   CUtensorMap ta, tb, td, tsa, tsb;
   const int64_t a_depth = p.mode == kMasked ? p.groups : 1;
   const int64_t b_depth = p.mode == kDense ? 1 : p.groups;
@@ -516,9 +628,13 @@ cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t str
   const int64_t sfb_bytes = b_depth * (((p.n + 127) / 128) * 128 * (p.k / 32));
   if (!make_tmap_kc(&ta, p.qa, p.k, p.m, a_depth)) return cudaErrorInvalidValue;
   if (!make_tmap_kc(&tb, p.qb, p.k, p.n, b_depth)) return cudaErrorInvalidValue;
-  if (!make_tmap_d(&td, p.d, p.n, p.m, a_depth)) return cudaErrorInvalidValue;
+  if (SWIGLU) {
+    if (!make_tmap_h(&td, p.d, p.i_dim, p.m, a_depth)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_tmap_d(&td, p.d, p.n, p.m, a_depth)) return cudaErrorInvalidValue;
+  }
   if (!make_tmap_sf(&tsa, p.sfa, sfa_bytes, p.k / BK, 1)) return cudaErrorInvalidValue;
-  if (!make_tmap_sf(&tsb, p.sfb, sfb_bytes, p.k / BK, 2)) return cudaErrorInvalidValue;
+  if (!make_tmap_sf(&tsb, p.sfb, sfb_bytes, p.k / BK, SWIGLU ? 1 : 2)) return cudaErrorInvalidValue;
 
   GemmArgs a = {};
   a.sfa = static_cast<const uint8_t*>(p.sfa);
@@ -532,12 +648,17 @@ cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t str
   a.sfb_group_bytes = ((p.n + 127) / 128) * 128 * (p.k / 32);
   a.m = static_cast<int>(p.m);
   a.n = static_cast<int>(p.n);
-  a.n_tiles = static_cast<int>((p.n + kPairN - 1) / kPairN);
+  // a SwiGLU tile yields 128 output columns from 128 gate + 128 up rows
+  a.n_tiles = SWIGLU ? static_cast<int>(p.i_dim / 128) : static_cast<int>((p.n + kPairN - 1) / kPairN);
   a.n_sf_tiles = static_cast<int>((p.n + 127) / 128);
   a.groups = static_cast<int>(p.groups);
   a.mode = p.mode;
-  a.sf_bufs = 2;
   a.a_box_rows = 128;
+  if (SWIGLU) {
+    a.swiglu_i = static_cast<int>(p.i_dim);
+    a.sfh = static_cast<uint8_t*>(p.sf_out);
+    a.sfh_group_bytes = ((p.m + 127) / 128) * 128 * (p.i_dim / 32);
+  }
 
   // upper bound of pair tiles (grouped forms: every expert full)
   int64_t m_blocks;
@@ -566,10 +687,14 @@ cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t str
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<STAGES>, ta, tb, td, tsa, tsb, a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<STAGES, SWIGLU>, ta, tb, td, tsa, tsb, a);
   if (e != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
+  return p.i_dim > 0 ? launch_pair<true>(p, num_sms, stream, launches) : launch_pair<false>(p, num_sms, stream, launches);
 }
 
 }  // namespace mxk

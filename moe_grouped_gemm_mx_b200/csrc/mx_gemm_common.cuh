@@ -35,8 +35,13 @@ struct GemmArgs {
   int n_sf_tiles;           // ceil(N / 128)
   int groups;
   int mode;
-  int sf_bufs;              // 1 or 2 TMEM buffers for the per-K-tile scale factors
   int a_box_rows;           // rows of A one TMA box brings (128, or 64/32 for a dense M <= 64)
+  // fused SwiGLU + MXFP8 epilogue (CTA-pair kernel only): B holds [gate; up]
+  // rows per expert, 2 * swiglu_i of them; the output is E4M3 H = silu(gate)
+  // * up [rows, swiglu_i] (through the D tensor map) plus its tiled scales
+  int swiglu_i;             // 0: plain BF16 epilogue
+  uint8_t* sfh;             // tiled UE8M0 scales of H
+  int64_t sfh_group_bytes;  // masked form: tiled scale bytes of H per expert
 };
 
 struct Tile {
@@ -120,6 +125,22 @@ inline bool make_tmap_d(CUtensorMap* m, void* base, int64_t n, int64_t rows, int
          CUDA_SUCCESS;
 }
 
+// 3-D byte tensor [depth, rows, cols] written in boxes of 128 rows x 64 bytes
+// (64-byte swizzle, the epilogue's staging layout): the E4M3 output of the
+// fused SwiGLU epilogue.
+inline bool make_tmap_h(CUtensorMap* m, void* base, int64_t cols, int64_t rows, int64_t depth) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(depth)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(cols * rows)};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(BM), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // 3-D byte tensor [depth, rows, k] (k contiguous) read in boxes of box_rows x 128 bytes.
 inline bool make_tmap(CUtensorMap* m, const void* base, int64_t k, int64_t rows, int64_t depth, int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
@@ -155,15 +176,17 @@ __device__ __forceinline__ void tmem_row_to_bf16(uint32_t t_row, uint32_t (&pack
 }
 
 // Epilogue, step 2 (the 128 epilogue threads, thread 64 issuing): write the
-// packed rows of a 128-row tile through two 64-byte-swizzled 8 KiB staging
-// chunks (128 rows x 32 columns) with TMA stores at (x0 + 32c, y0, z); the
-// tensor map clips what lies outside D.  `stg_count` alternates the chunks.
-template <int NCOLS>
-__device__ __forceinline__ void store_rows_tma(const uint32_t (&packed)[NCOLS / 2], int r_local, uint32_t stg_base,
-                                               uint32_t& stg_count, const CUtensorMap* tmap_d, int x0, int y0,
-                                               int z) {
+// WORDS 32-bit words of each row of a 128-row tile through two
+// 64-byte-swizzled 8 KiB staging chunks (128 rows x 64 bytes) with TMA stores
+// at (x0 + c * CHUNK_ELEMS, y0, z), CHUNK_ELEMS = elements of the tensor map
+// per 64 bytes (32 for BF16 D, 64 for E4M3 H); the tensor map clips what lies
+// outside the tensor.  `stg_count` alternates the chunks.
+template <int WORDS, int CHUNK_ELEMS = 32>
+__device__ __forceinline__ void store_words_tma(const uint32_t (&packed)[WORDS], int r_local, uint32_t stg_base,
+                                                uint32_t& stg_count, const CUtensorMap* tmap_d, int x0, int y0,
+                                                int z) {
 #pragma unroll
-  for (int c = 0; c < NCOLS / 32; ++c) {
+  for (int c = 0; c < WORDS / 16; ++c) {
     const uint32_t stg = stg_base + (stg_count & 1u) * 8192u;
     // the store issued from this chunk two rounds ago must have read it
     if (threadIdx.x == 64) bulk_wait_group_read<1>();
@@ -178,11 +201,19 @@ __device__ __forceinline__ void store_rows_tma(const uint32_t (&packed)[NCOLS / 
     fence_proxy_async_smem();
     named_barrier_sync(1, 128);
     if (threadIdx.x == 64) {
-      tma_store_3d(tmap_d, stg, x0 + c * 32, y0, z);
+      tma_store_3d(tmap_d, stg, x0 + c * CHUNK_ELEMS, y0, z);
       bulk_commit_group();
     }
     ++stg_count;
   }
+}
+
+// BF16 rows of NCOLS columns (NCOLS / 2 packed words).
+template <int NCOLS>
+__device__ __forceinline__ void store_rows_tma(const uint32_t (&packed)[NCOLS / 2], int r_local, uint32_t stg_base,
+                                               uint32_t& stg_count, const CUtensorMap* tmap_d, int x0, int y0,
+                                               int z) {
+  store_words_tma<NCOLS / 2, 32>(packed, r_local, stg_base, stg_count, tmap_d, x0, y0, z);
 }
 
 }  // namespace mxk

@@ -30,6 +30,11 @@ struct GemmProblem {
   int64_t m, n, k;               // m: dense M / contiguous m_total / masked max_m
   int64_t groups;                // experts (1 for the dense form)
   int mode;                      // 0 dense, 1 contiguous, 2 masked
+  // fused SwiGLU + MXFP8 requantisation epilogue (i_dim > 0): qb holds
+  // [gate; up] = 2 * i_dim rows per expert, d receives E4M3 H [.., i_dim]
+  // and sf_out its tiled scales
+  int64_t i_dim = 0;
+  void* sf_out = nullptr;
 };
 
 cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches);

@@ -37,6 +37,9 @@ def lib():
     L.mx_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
     L.mx_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
+    L.mx_gemm_swiglu_quant.argtypes = [P, P, P, P, P, P, I64, I64, I64, P, P]
+    L.mx_grouped_gemm_contiguous_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
+    L.mx_grouped_gemm_masked_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
     return L
 
 
@@ -114,3 +117,24 @@ def test_quantize_multi_argument_checks(lib):
     assert f(None, 0, None) == MX_OK
     empty = (J * 2)(J(None, 0, 4, 64, None, None), J(None, 1, 0, 64, None, None))
     assert f(ctypes.addressof(empty), 2, None) == MX_OK
+
+
+def test_swiglu_quant_argument_checks(lib):
+    f = lib.mx_gemm_swiglu_quant
+    # i_dim must be a positive multiple of 128 (the fused epilogue's column block)
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 192, 256, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 0, 256, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 96, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 128, 256, 256, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4, 128, 256, 256, None, None) == MX_ERR_MISALIGNED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE + 8, FAKE, 128, 256, 256, None, None) == MX_ERR_MISALIGNED
+    assert f(None, None, None, None, None, None, 0, 256, 256, None, None) == MX_OK
+    c = lib.mx_grouped_gemm_contiguous_swiglu_quant
+    assert c(FAKE, FAKE, FAKE, FAKE, None, 4, 512, 256, 128, FAKE, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert c(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 512, 200, 128, FAKE, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert c(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 512, 256, 128, FAKE, FAKE, None, None) == MX_ERR_MISALIGNED
+    assert c(None, None, None, None, None, 0, 512, 256, 128, None, None, None, None) == MX_OK
+    m = lib.mx_grouped_gemm_masked_swiglu_quant
+    assert m(FAKE, FAKE, FAKE, FAKE, None, 4, 256, 256, 128, FAKE, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert m(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 130, FAKE, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert m(None, None, None, None, None, 4, 0, 256, 128, None, None, None, None) == MX_OK
