@@ -68,12 +68,23 @@ def static_config(name: str, seed: int) -> dict:
                     "zipf_s": I.MOE_ZIPF_S, "real_rows": int(counts.sum()),
                     "padded_rows": int(I.padded_offsets(counts)[-1]),
                     "gemms": ["gate_up N=4096 K=7168", "down N=7168 K=2048"]})
+    elif name == "moe_mlp":
+        counts = I.zipf_routing_counts(seed=seed)
+        cfg.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "topk": I.MOE_TOPK,
+                    "zipf_s": I.MOE_ZIPF_S, "real_rows": int(counts.sum()),
+                    "padded_rows": int(I.padded_offsets(counts)[-1]),
+                    "gemms": ["gate/up N=2x2048 K=7168 with fused SwiGLU + MXFP8 requantisation",
+                              "down N=7168 K=2048 on the requantised activation"]})
     elif name == "masked":
         mm = I.masked_counts(seed=seed)
         cfg.update({"experts": I.MASKED_EXPERTS, "max_m": I.MASKED_MAX_M, "n": I.MASKED_NK[0],
                     "k": I.MASKED_NK[1], "valid_rows": int(mm.sum()), "active_experts": int((mm > 0).sum())})
-    cfg["step"] = ("quantise activations + weights (one batched launch), then the GEMM(s) "
-                   "with BF16 epilogue")
+    if name == "moe_mlp":
+        cfg["step"] = ("quantise tokens + gate/up and down weights (one batched launch), then the fused "
+                       "gate/up GEMM -> SwiGLU -> MXFP8 kernel and the down GEMM with BF16 epilogue")
+    else:
+        cfg["step"] = ("quantise activations + weights (one batched launch), then the GEMM(s) "
+                       "with BF16 epilogue")
     return cfg
 
 
@@ -82,7 +93,7 @@ def parse_args():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked"])
+    p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -285,6 +296,41 @@ class Workload:
                             "padded_rows": int(I.padded_offsets(counts)[-1]),
                             "gemms": ["gate_up N=4096 K=7168", "down N=7168 K=2048"]})
 
+    def _build_moe_mlp(self, seed, I):
+        """One MoE expert layer: [gate; up] GEMM with the SwiGLU + MXFP8 epilogue,
+        then the down GEMM on its output (the contiguous workload's shapes)."""
+        import torch
+        mx = self.mx
+        counts = I.zipf_routing_counts(seed=seed)
+        real = int(counts.sum())
+        n13, k = I.MOE_GATE_NK
+        n2, i_dim = I.MOE_DOWN_NK
+        assert n13 == 2 * i_dim
+        prob = I.contiguous_problem(n=n13, k=k, seed=seed, counts=counts, device=self.dev)
+        w2 = I.normal_bf16((len(counts), n2, i_dim), 0.02, seed + 4_000_037, self.dev)
+        for t in (prob.a, prob.b, w2):
+            self._add_input(t)
+        qa, sfa = self._quant(prob.a, "A")
+        q13, sf13 = self._quant(prob.b, "W13")
+        q2, sf2 = self._quant(w2, "W2")
+        off = prob.offsets.to(self.dev)
+        m_total = prob.a.shape[0]
+        qh = torch.empty((m_total, i_dim), dtype=torch.uint8, device=self.dev)
+        sfh = torch.empty(mx.scale_bytes(m_total, i_dim), dtype=torch.uint8, device=self.dev)
+        y = torch.empty((m_total, n2), dtype=torch.bfloat16, device=self.dev)
+        self.outputs.append(y)
+        experts = int((counts > 0).sum())
+        fl1 = 2.0 * real * n13 * k
+        bytes1 = (m_total * k + experts * n13 * k + m_total * i_dim) * (1 + 1 / 32)
+        self.launches.append(("gemm", "gate_up+swiglu", lambda: mx.mx_grouped_gemm_contiguous_swiglu_quant(
+            qa, sfa, q13, sf13, off, qh=qh, sfh=sfh, dev_status=self.status), bytes1, fl1))
+        fl2 = 2.0 * real * n2 * i_dim
+        self.launches.append(("gemm", "down", lambda: mx.mx_grouped_gemm_contiguous(
+            qh, sfh, q2, sf2, off, d=y, dev_status=self.status), self._gemm_bytes(m_total, n2, i_dim, experts), fl2))
+        self.flops += fl1 + fl2
+        self.config.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "real_rows": real,
+                            "padded_rows": m_total})
+
     def _build_masked(self, seed, I):
         import torch
         mx = self.mx
@@ -360,6 +406,30 @@ def oracle_sample(name, seed, target_s=10.0):
         jobs.append(job)
         desc = "gate/up GEMM on 64 rows over 2 experts (quantise rows and both experts' weights)"
         del counts, g
+    elif name == "moe_mlp":
+        n13, k = I.MOE_GATE_NK
+        n2, i_dim = I.MOE_DOWN_NK
+        a = I.normal_bf16((64, k), 1.0, seed + 7)
+        w13 = I.normal_bf16((2, n13, k), 0.02, seed + 8)
+        w2 = I.normal_bf16((2, n2, i_dim), 0.02, seed + 9)
+
+        def job():
+            qa, sfa = L.quantize(a)
+            q13, sf13 = L.quantize(w13)
+            q2, sf2 = L.quantize(w2)
+            off = np.array([0, 32, 64], dtype=np.int32)
+            q13 = q13.reshape(2, n13, k)
+            sf13 = sf13.reshape(2, n13, k // 32)
+            g, _ = L.grouped_contiguous(qa, sfa, np.ascontiguousarray(q13[:, :i_dim]),
+                                        np.ascontiguousarray(sf13[:, :i_dim]).reshape(-1, k // 32), off)
+            u, _ = L.grouped_contiguous(qa, sfa, np.ascontiguousarray(q13[:, i_dim:]),
+                                        np.ascontiguousarray(sf13[:, i_dim:]).reshape(-1, k // 32), off)
+            qh, sfh = L.quantize_f32(L.swiglu(g, u).astype(np.float32))
+            L.grouped_contiguous(qh, sfh, q2.reshape(2, n2, i_dim), sf2, off)
+            return 2.0 * 64 * n13 * k + 2.0 * 64 * n2 * i_dim
+        jobs.append(job)
+        desc = ("one expert layer on 64 rows over 2 experts: quantise rows and weights, gate/up GEMM, "
+                "SwiGLU, requantise, down GEMM")
     else:  # masked
         n, k = I.MASKED_NK
         prob = I.masked_problem(n=n, k=k, experts=2, max_m=32, seed=seed,
