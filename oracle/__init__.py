@@ -78,6 +78,8 @@ def lib():
         L.mxo_grouped_contiguous.restype = None
         L.mxo_grouped_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, I64, P, P]
         L.mxo_grouped_masked.restype = None
+        L.mxo_grouped_kgrouped.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, I64, P, P]
+        L.mxo_grouped_kgrouped.restype = None
         L.mxo_num_threads.argtypes = []
         L.mxo_num_threads.restype = ctypes.c_int
         _lib = L
@@ -263,6 +265,44 @@ def grouped_masked(qa, sfa, qb, sfb, masked_m, rows=None):
                              _p(ids), nrows, _p(d), _p(a))
     if ids is None:
         return d.reshape(groups, max_m, n), a.reshape(groups, max_m, n)
+    return d, a
+
+
+def quantize_transposed(x):
+    """Quantisation along the ROW dimension of x [..., rows, cols] (blocks of
+    32 consecutive rows of one column), returned in the transposed layout:
+    by definition the row-wise quantisation of x^T.  For a 3-D x each group
+    is transposed on its own: q [groups*cols, rows], sf [groups*cols, rows/32]."""
+    xb = _u16(x)
+    if xb.ndim == 2:
+        xb = xb[None]
+    xt = np.ascontiguousarray(np.swapaxes(xb, -1, -2))
+    return quantize(xt)
+
+
+def grouped_kgrouped(qa, sfa, qb, sfb, offsets, rows=None):
+    """d[e] = deq(A[:, off[e]:off[e+1]]) * deq(B[:, off[e]:off[e+1]])^T in fp64.
+
+    qa [m, k_total], qb [n, k_total] (the token dimension is the reduction
+    dimension), sfa / sfb row-major [., k_total/32]; offsets int32
+    [groups+1].  Returns (d, abssum) of shape [groups, m, n], or
+    [len(rows), n] for the listed flat indices e*m + i."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qb = np.ascontiguousarray(qb, dtype=np.uint8)
+    sfa = np.ascontiguousarray(sfa, dtype=np.uint8)
+    sfb = np.ascontiguousarray(sfb, dtype=np.uint8)
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    groups = len(off) - 1
+    m, k_total = qa.shape
+    n = qb.shape[0]
+    ids = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = groups * m if ids is None else len(ids)
+    d = np.zeros((nrows, n), dtype=np.float64)
+    a = np.zeros((nrows, n), dtype=np.float64)
+    lib().mxo_grouped_kgrouped(_p(qa), _p(sfa), _p(qb), _p(sfb), _p(off), groups, m, n, k_total,
+                               _p(ids), nrows, _p(d), _p(a))
+    if ids is None:
+        return d.reshape(groups, m, n), a.reshape(groups, m, n)
     return d, a
 
 

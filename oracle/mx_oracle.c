@@ -400,6 +400,48 @@ void mxo_grouped_masked(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb
     }
 }
 
+/* K-grouped GEMM (the weight gradient of an MoE expert layer: the
+ * reduction runs over tokens, and each expert owns a range of them).  For
+ * expert e and k ranging over [off[e], off[e+1]):
+ *   d[e, i, j] = sum_k deq(a[i, k]) * deq(b[j, k]),  k ascending, in double.
+ * qa [m, k_total], qb [n, k_total], scales row-major [., k_total/32]
+ * (blocks of 32 along the token dimension).  An expert with no tokens gives
+ * zeros.  Only the listed flat indices e*m + i are computed when row_ids is
+ * given; d and abssum are [nrows, n]. */
+void mxo_grouped_kgrouped(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                          const uint8_t *sfb, const int32_t *offsets, int32_t groups,
+                          int64_t m, int64_t n, int64_t k_total, const int64_t *row_ids,
+                          int64_t nrows, double *d, double *abssum)
+{
+    struct mxo_tables t;
+    fill_tables(&t);
+    int64_t kb = k_total / 32;
+    if (!row_ids)
+        nrows = (int64_t)groups * m;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t flat = row_ids ? row_ids[r] : r;
+        int64_t e = flat / m, i = flat % m;
+        const uint8_t *qa_row = qa + i * k_total;
+        const uint8_t *sfa_row = sfa + i * kb;
+        for (int64_t j = 0; j < n; ++j) {
+            const uint8_t *qb_row = qb + j * k_total;
+            const uint8_t *sfb_row = sfb + j * kb;
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t kk = offsets[e]; kk < offsets[e + 1]; ++kk) {
+                double a = t.tab[qa_row[kk]] * t.stab[sfa_row[kk / 32]];
+                double b = t.tab[qb_row[kk]] * t.stab[sfb_row[kk / 32]];
+                double p = a * b;
+                acc += p;
+                aacc += fabs(p);
+            }
+            d[r * n + j] = acc;
+            if (abssum)
+                abssum[r * n + j] = aacc;
+        }
+    }
+}
+
 int mxo_num_threads(void)
 {
 #ifdef _OPENMP

@@ -41,6 +41,10 @@ void mxo_grouped_masked(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb
                         const uint8_t *sfb, const int32_t *masked_m, int32_t groups,
                         int64_t max_m, int64_t n, int64_t k, const int64_t *row_ids,
                         int64_t nrows, double *d, double *abssum);
+void mxo_grouped_kgrouped(const uint8_t *qa, const uint8_t *sfa, const uint8_t *qb,
+                          const uint8_t *sfb, const int32_t *offsets, int32_t groups,
+                          int64_t m, int64_t n, int64_t k_total, const int64_t *row_ids,
+                          int64_t nrows, double *d, double *abssum);
 int mxo_num_threads(void);
 
 #ifdef __cplusplus

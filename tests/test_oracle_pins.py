@@ -459,3 +459,68 @@ def test_quantize_f32_special_blocks(oracle):
     blk = np.full(32, 2.0 ** 100, dtype=np.float32)
     q, s = oracle.quantize_block_f32(blk)
     assert s == 127 + 92 and (q == 0x78).all()
+
+
+# ---------------------------------------------------------------- training-side GEMMs
+# (quantisation along the token dimension and the K-grouped weight-gradient GEMM)
+
+def test_quantize_transposed_hand_example(oracle):
+    """Blocks run down a column: x [64, 3]; column 0 all ones (amax 1 -> X = -8,
+    scale 0x77, elements 256 -> 0x78); column 1 = row index r in rows 0..31
+    (amax 31 -> X = -4, r*16: 0..496, 31*16 = 496 saturates to 448 = 0x7E)
+    and zeros in rows 32..63 (scale 0x00, codes 0x00); column 2 = -2 everywhere
+    (X = -7, -256 -> 0xF8).  Output layout: q[c, r] is the code of x[r, c]."""
+    x = np.zeros((64, 3), dtype=np.float32)
+    x[:, 0] = 1.0
+    x[:32, 1] = np.arange(32)
+    x[:, 2] = -2.0
+    q, sf = oracle.quantize_transposed(torch.from_numpy(x).to(torch.bfloat16))
+    assert q.shape == (3, 64) and sf.shape == (3, 2)
+    assert list(sf[0]) == [0x77, 0x77] and np.all(q[0] == 0x78)
+    assert list(sf[1]) == [127 - 4, 0x00]
+    assert q[1, 1] == oracle.e4m3_encode(16.0) and q[1, 31] == 0x7E and q[1, 30] == oracle.e4m3_encode(480.0)
+    assert np.all(q[1, 32:] == 0x00)
+    assert list(sf[2]) == [127 - 7, 127 - 7] and np.all(q[2] == 0xF8)
+
+
+def _kgrouped_operands(oracle, rng, m, n, tokens):
+    a = _int_block_matrix(rng, m, tokens)   # [m, tokens], blocks of 32 tokens share amax 4
+    b = _int_block_matrix(rng, n, tokens)
+    qa, sfa = oracle.quantize(torch.from_numpy(a).to(torch.bfloat16))
+    qb, sfb = oracle.quantize(torch.from_numpy(b).to(torch.bfloat16))
+    return a, b, qa, sfa, qb, sfb
+
+
+def test_kgrouped_exact_on_small_integers(oracle):
+    """Integer operands whose every 32-token block has amax 4 are exact in
+    MXFP8, and all partial sums are small integers: each expert's result must
+    equal the integer matmul over its own token range."""
+    rng = np.random.default_rng(21)
+    a, b, qa, sfa, qb, sfb = _kgrouped_operands(oracle, rng, 6, 5, 256)
+    off = np.array([0, 64, 64, 96, 256], dtype=np.int32)   # expert 1 has no tokens
+    d, absd = oracle.grouped_kgrouped(qa, sfa, qb, sfb, off)
+    for e in range(4):
+        s0, s1 = off[e], off[e + 1]
+        want = a[:, s0:s1].astype(np.int64) @ b[:, s0:s1].astype(np.int64).T
+        assert np.array_equal(d[e], want.astype(np.float64)), e
+        assert np.array_equal(absd[e], np.abs(a[:, s0:s1]) @ np.abs(b[:, s0:s1]).T)
+    assert not d[1].any()
+
+
+def test_kgrouped_one_group_equals_dense_and_sum_over_groups(oracle):
+    g = torch.Generator().manual_seed(5)
+    a = torch.randn(40, 384, generator=g).to(torch.bfloat16)
+    b = (torch.randn(24, 384, generator=g) * 0.3).to(torch.bfloat16)
+    qa, sfa = oracle.quantize(a)
+    qb, sfb = oracle.quantize(b)
+    dense, dabs = oracle.gemm(qa, sfa, qb, sfb)
+    one, oabs = oracle.grouped_kgrouped(qa, sfa, qb, sfb, np.array([0, 384], dtype=np.int32))
+    np.testing.assert_array_equal(one[0], dense)
+    np.testing.assert_array_equal(oabs[0], dabs)
+    # the experts partition the tokens, so their gradients sum to the dense product
+    parts, _ = oracle.grouped_kgrouped(qa, sfa, qb, sfb, np.array([0, 128, 160, 160, 384], dtype=np.int32))
+    np.testing.assert_allclose(parts.sum(axis=0), dense, rtol=1e-12, atol=1e-12)
+    # sampled rows (flat e*m + i) agree with the full result
+    ids = np.array([0, 39, 40 + 7, 3 * 40 + 39], dtype=np.int64)
+    sub, _ = oracle.grouped_kgrouped(qa, sfa, qb, sfb, np.array([0, 128, 160, 160, 384], dtype=np.int32), rows=ids)
+    np.testing.assert_array_equal(sub, parts.reshape(-1, 24)[ids])
