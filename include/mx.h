@@ -163,6 +163,45 @@ mx_status mx_grouped_gemm_masked(const void *qa, const void *sfa, const void *qb
                                  int32_t *dev_status, mx_stream_t stream);
 
 /*
+ * Quantisation along the ROW dimension, written transposed: for x
+ * [groups, rows, cols] BF16 (row-major) the output is q [groups, cols, rows]
+ * E4M3, each 32 consecutive rows of a column sharing one UE8M0 scale, with
+ * per-group tiled scales of the [cols, rows] operand
+ * (groups * mx_scale_bytes(cols, rows) bytes; rows play the role of K).
+ * Same scale and rounding rule as mx_quantize_bf16_to_e4m3.  Used for the
+ * training-side MoE GEMMs (the B200 MoE-training page applies MXFP8 to
+ * DeepSeek-V3 training): the weight gradient reduces over tokens, so the
+ * output gradient and the layer input [tokens, features] are quantised along
+ * tokens; the input gradient reduces over the layer's output features, so the
+ * expert weights [E, N, K] are quantised along N into [E, K, N].
+ * Requires rows % 32 == 0, cols % 8 == 0, 16-byte aligned pointers.  Scale
+ * padding bytes are written as 0x00.
+ */
+mx_status mx_quantize_bf16_to_e4m3_transposed(const void *x_bf16, int64_t groups, int64_t rows, int64_t cols,
+                                              void *q_e4m3, void *sf_ue8m0, mx_stream_t stream);
+
+/*
+ * K-grouped MoE GEMM: the weight gradient of an expert layer, where the
+ * reduction runs over tokens and each expert owns a contiguous range of them
+ * (the contiguous layout of mx_grouped_gemm_contiguous, seen from the
+ * backward pass).  For expert e and k in [group_offsets[e], group_offsets[e+1]):
+ *   D[e, i, j] = sum_k deq(A[i, k]) * deq(B[j, k])   (FP32 accumulation, BF16 out)
+ *   qa [m, k_total] E4M3 (e.g. the output gradient transposed, m = N of the
+ *   layer), sfa = mx_scale_bytes(m, k_total) tiled scales (blocks of 32
+ *   tokens); qb [n, k_total] (e.g. the layer input transposed), sfb
+ *   likewise; both from mx_quantize_bf16_to_e4m3_transposed.
+ *   group_offsets: DEVICE int32[groups + 1], multiples of 128, non-decreasing,
+ *   at most k_total (else MX_DEV_BAD_OFFSETS and nothing is written).
+ *   d_bf16 [groups, m, n]: every expert's block is written; an expert with
+ *   no tokens gets zeros.
+ * Requires k_total > 0, k_total % 128 == 0, n % 16 == 0, 16-byte aligned
+ * pointers.
+ */
+mx_status mx_grouped_gemm_kgrouped(const void *qa, const void *sfa, const void *qb, const void *sfb,
+                                   const int32_t *group_offsets, int32_t groups, int64_t m, int64_t n,
+                                   int64_t k_total, void *d_bf16, int32_t *dev_status, mx_stream_t stream);
+
+/*
  * Fused first half of an MoE expert MLP: the gate/up GEMM, SwiGLU, and MXFP8
  * requantisation of the result in one kernel, so the activation never goes
  * to memory in BF16 (the B200 MoE-training page describes MXFP8 expert

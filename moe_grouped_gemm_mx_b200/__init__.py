@@ -25,7 +25,8 @@ __all__ = [
     "MXError", "lib_path", "scale_bytes", "mx_quantize_bf16_to_e4m3", "mx_quantize_bf16_to_e4m3_multi",
     "mx_gemm",
     "mx_grouped_gemm_contiguous", "mx_grouped_gemm_masked", "mx_gemm_swiglu_quant",
-    "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant", "read_internal_status",
+    "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant",
+    "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped", "read_internal_status",
     "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "C_SYMBOLS",
 ]
 
@@ -43,6 +44,7 @@ C_SYMBOLS = [
     "mx_grouped_gemm_contiguous",
     "mx_grouped_gemm_masked", "mx_read_internal_status", "mx_gemm_swiglu_quant",
     "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant",
+    "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped",
 ]
 
 
@@ -86,6 +88,10 @@ def _load():
     L.mx_grouped_gemm_contiguous_swiglu_quant.restype = ctypes.c_int
     L.mx_grouped_gemm_masked_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
     L.mx_grouped_gemm_masked_swiglu_quant.restype = ctypes.c_int
+    L.mx_quantize_bf16_to_e4m3_transposed.argtypes = [P, I64, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3_transposed.restype = ctypes.c_int
+    L.mx_grouped_gemm_kgrouped.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
+    L.mx_grouped_gemm_kgrouped.restype = ctypes.c_int
     L.mx_read_internal_status.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
     L.mx_read_internal_status.restype = ctypes.c_int
     return L
@@ -183,6 +189,30 @@ def mx_quantize_bf16_to_e4m3_multi(xs, outs=None, stream=None):
     return res
 
 
+def mx_quantize_bf16_to_e4m3_transposed(x: torch.Tensor, q: torch.Tensor | None = None,
+                                        sf: torch.Tensor | None = None, stream=None):
+    """Quantise along the ROWS of x ([rows, cols] or [groups, rows, cols] BF16)
+    into the transposed layout: q uint8 [cols, rows] / [groups, cols, rows] and
+    per-group tiled scales of the [cols, rows] operand."""
+    _check(x, torch.bfloat16, "x")
+    if x.dim() not in (2, 3):
+        raise ValueError("x must be 2-D [rows, cols] or 3-D [groups, rows, cols]")
+    groups = 1 if x.dim() == 2 else x.shape[0]
+    rows, cols = x.shape[-2], x.shape[-1]
+    shape = (cols, rows) if x.dim() == 2 else (groups, cols, rows)
+    if q is None:
+        q = torch.empty(shape, dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(groups * scale_bytes(cols, rows), dtype=torch.uint8, device=x.device)
+    _check(q, torch.uint8, "q")
+    _check(sf, torch.uint8, "sf")
+    if q.numel() != x.numel() or sf.numel() < groups * scale_bytes(cols, rows):
+        raise ValueError("output buffers too small")
+    st = _lib.mx_quantize_bf16_to_e4m3_transposed(_ptr(x), groups, rows, cols, _ptr(q), _ptr(sf), _stream(stream))
+    _raise(st, "mx_quantize_bf16_to_e4m3_transposed")
+    return q, sf
+
+
 def _status_arg(dev_status):
     if dev_status is None:
         return None
@@ -245,6 +275,31 @@ def mx_grouped_gemm_masked(qa, sfa, qb, sfb, masked_m: torch.Tensor, d: torch.Te
     st = _lib.mx_grouped_gemm_masked(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(masked_m), groups,
                                      max_m, n, k, _ptr(d), _status_arg(dev_status), _stream(stream))
     _raise(st, "mx_grouped_gemm_masked")
+    return d
+
+
+def mx_grouped_gemm_kgrouped(qa, sfa, qb, sfb, group_offsets: torch.Tensor, groups: int | None = None,
+                             d: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                             stream=None) -> torch.Tensor:
+    """K-grouped MoE GEMM (weight gradient): qa uint8 [M, K_total], qb uint8
+    [N, K_total], group_offsets int32 [E+1] along K -> bf16 [E, M, N] with
+    D[e] = deq(A[:, off[e]:off[e+1]]) deq(B[:, off[e]:off[e+1]])^T."""
+    for t, nm in ((qa, "qa"), (sfa, "sfa"), (qb, "qb"), (sfb, "sfb")):
+        _check(t, torch.uint8, nm)
+    _check(group_offsets, torch.int32, "group_offsets")
+    m, k_total = qa.shape
+    n, kb = qb.shape
+    if kb != k_total:
+        raise ValueError("K mismatch")
+    groups = group_offsets.numel() - 1 if groups is None else groups
+    if group_offsets.numel() != groups + 1:
+        raise ValueError("group_offsets must hold groups + 1 entries")
+    if d is None:
+        d = torch.empty((groups, m, n), dtype=torch.bfloat16, device=qa.device)
+    _check(d, torch.bfloat16, "d")
+    st = _lib.mx_grouped_gemm_kgrouped(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(group_offsets), groups,
+                                       m, n, k_total, _ptr(d), _status_arg(dev_status), _stream(stream))
+    _raise(st, "mx_grouped_gemm_kgrouped")
     return d
 
 

@@ -132,6 +132,20 @@ mx_status mx_quantize_bf16_to_e4m3_multi(const mx_quant_job* jobs, int32_t count
   return MX_OK;
 }
 
+mx_status mx_quantize_bf16_to_e4m3_transposed(const void* x_bf16, int64_t groups, int64_t rows, int64_t cols,
+                                              void* q_e4m3, void* sf_ue8m0, mx_stream_t stream) {
+  if (groups < 0 || rows < 0 || cols < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (rows % 32 != 0 || cols % 8 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (groups == 0 || rows == 0 || cols == 0) return MX_OK;
+  if (!x_bf16 || !q_e4m3 || !sf_ue8m0) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(sf_ue8m0)) return MX_ERR_MISALIGNED;
+  if (rows > kMaxDim || cols > kMaxDim || groups * rows * cols / 32 >= (int64_t(1) << 40))
+    return MX_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(mxk::launch_quant_transposed(x_bf16, groups, rows, cols, q_e4m3, sf_ue8m0,
+                                                static_cast<int64_t>(mx_scale_bytes(cols, rows)),
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 static mx_status check_gemm_common(const void* qa, const void* sfa, const void* qb, const void* sfb, void* d,
                                    int64_t m, int64_t n, int64_t k, int64_t groups) {
   if (m < 0 || n < 0 || k < 0 || groups < 0) return MX_ERR_INVALID_ARGUMENT;
@@ -194,6 +208,25 @@ mx_status mx_grouped_gemm_masked(const void* qa, const void* sfa, const void* qb
   int32_t* status = dev_status ? dev_status : internal_status_ptr();
   if (!status) return MX_ERR_CUDA;
   mxk::GemmProblem p{qa, sfa, qb, sfb, d_bf16, nullptr, masked_m, status, max_m, n, k, groups, 2};
+  return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+mx_status mx_grouped_gemm_kgrouped(const void* qa, const void* sfa, const void* qb, const void* sfb,
+                                   const int32_t* group_offsets, int32_t groups, int64_t m, int64_t n,
+                                   int64_t k_total, void* d_bf16, int32_t* dev_status, mx_stream_t stream) {
+  if (groups < 0 || m < 0 || n < 0 || k_total < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k_total == 0 || k_total % 128 != 0 || n % 16 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (groups == 0 || m == 0 || n == 0) return MX_OK;
+  if (!group_offsets) return MX_ERR_INVALID_ARGUMENT;
+  if (groups * m > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  mx_status st = check_gemm_common(qa, sfa, qb, sfb, d_bf16, m, n, k_total, groups);
+  if (st != MX_OK) return st;
+  if (reinterpret_cast<uintptr_t>(group_offsets) & 3u) return MX_ERR_MISALIGNED;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  mxk::GemmProblem p{qa, sfa, qb, sfb, d_bf16, group_offsets, nullptr, status, m, n, k_total, groups, 3};
   return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
 }
 

@@ -668,7 +668,8 @@ static int choose_config(const GemmProblem& p, int num_sms) {
 }
 
 cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches) {
-  if (p.i_dim > 0) return launch_gemm_pair(p, num_sms, stream, launches);  // fused SwiGLU: CTA-pair kernel only
+  // fused SwiGLU and K-grouped (weight-gradient) forms: CTA-pair kernel only
+  if (p.i_dim > 0 || p.mode == kKGrouped) return launch_gemm_pair(p, num_sms, stream, launches);
   const int c = choose_config(p, num_sms);
   if (c == kCfgPair) return launch_gemm_pair(p, num_sms, stream, launches);
   if (p.mode == kDense && p.m <= 64) {

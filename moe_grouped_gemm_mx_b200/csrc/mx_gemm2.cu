@@ -34,6 +34,7 @@
 #include <cstdint>
 
 #include "mx_gemm_common.cuh"
+#include "mx_mxfp8.cuh"
 #include "mx_launch.h"
 
 namespace mxk {
@@ -105,6 +106,9 @@ __device__ __forceinline__ PairTile decode_pair_tile(const GemmArgs& a, const in
     if (a.mode == kContiguous) {  // tab1: group offsets
       r.row0 = tab1[e] + mb * kPairM;
       r.rows_end = tab1[e + 1];
+    } else if (a.mode == kKGrouped) {  // every expert has the full [m, n] output
+      r.row0 = mb * kPairM;
+      r.rows_end = a.m;
     } else {  // tab1: clamped masked_m
       r.row0 = mb * kPairM;
       r.rows_end = tab1[e];
@@ -122,42 +126,6 @@ __device__ __forceinline__ float swiglu_f32(float g, float u) {
   const float r = __fdividef(1.0f, 1.0f + t);  // sigmoid(|g|)
   const float sig = g >= 0.0f ? r : t * r;     // sigmoid(g)
   return g * sig * u;
-}
-
-__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
-  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
-  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-}
-
-// MXFP8 quantisation of 32 FP32 values (the BF16 quantiser's rule applied to
-// FP32 input): X = floor(log2 amax) - 8 clamped to [-127, 127] (amax 0 gives
-// -127), elements x * 2^-X with saturating round-to-nearest-even; a block
-// holding NaN or Inf gets scale 0xFF and elements 0x7F.  amax is taken on the
-// integer magnitude bits (order-preserving for IEEE patterns, and >= 0x7f800000
-// exactly for Inf/NaN).  Returns the scale byte; q receives 32 bytes.
-__device__ __forceinline__ uint32_t quant_block32_f32(const float (&h)[32], uint32_t (&q)[8]) {
-  uint32_t amax = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) amax = max(amax, __float_as_uint(h[j]) & 0x7FFFFFFFu);
-  if (amax >= 0x7F800000u) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] = 0x7F7F7F7Fu;
-    return 0xFFu;
-  }
-  int x = -127;
-  if (amax != 0) {
-    const int e = static_cast<int>(amax >> 23);
-    const int fl = e > 0 ? e - 127 : (31 - __clz(amax & 0x7FFFFFu)) - 149;  // subnormal: m * 2^-149
-    x = fl - 8;
-    x = x < -127 ? -127 : (x > 127 ? 127 : x);
-  }
-  // 2^-X as an FP32 bit pattern: finite FP32 input keeps X <= 119, so the
-  // exponent field 127 - X lies in [8, 254]
-  const float s = __uint_as_float(static_cast<uint32_t>(127 - x) << 23);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = e4m3x4(h[4 * i] * s, h[4 * i + 1] * s, h[4 * i + 2] * s, h[4 * i + 3] * s);
-  return static_cast<uint32_t>(x + 127);
 }
 
 template <int STAGES, bool SWIGLU>
@@ -219,12 +187,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // tab0 = exclusive prefix of pair tiles per expert
   int bad = 0;
   if (args.mode != kDense) {
-    if (args.mode == kContiguous) {
+    if (args.mode == kContiguous || args.mode == kKGrouped) {
+      // offsets along M (contiguous) or along K (K-grouped: the token ranges)
+      const int limit = args.mode == kContiguous ? args.m : args.k_tiles * BK;
       for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) tab1[i] = __ldg(args.group_offsets + i);
       __syncthreads();
       for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) {
         const int32_t v = tab1[i];
-        if (v < 0 || (v % BM) != 0 || v > args.m) bad = 1;
+        if (v < 0 || (v % BM) != 0 || v > limit) bad = 1;
         if (i > 0 && v < tab1[i - 1]) bad = 1;
       }
     } else {
@@ -242,6 +212,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int per = (args.groups + 31) / 32;
       const int lo = lane * per;
       auto tiles_of = [&](int e) -> int {
+        if (args.mode == kKGrouped) return bad ? 0 : (args.m + kPairM - 1) / kPairM * args.n_tiles;
         const int rows = args.mode == kContiguous ? (bad ? 0 : tab1[e + 1] - tab1[e]) : tab1[e];
         return (rows + kPairM - 1) / kPairM * args.n_tiles;
       };
@@ -271,7 +242,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       total = ((args.m + kPairM - 1) / kPairM) * args.n_tiles;
     } else {
       total = tab0[args.groups];
-      if (bad && rank == 0) report(args.status, args.mode == kContiguous ? 0x1 : 0x2);
+      if (bad && rank == 0) report(args.status, args.mode == kMasked ? 0x2 : 0x1);
     }
     *total_slot = total;
   }
@@ -281,6 +252,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = *total_slot;
+  // K range of a tile in 128-byte chunks: all of K, or (K-grouped) the
+  // expert's own token range [off[e], off[e+1])
+  auto tile_kc0 = [&](const PairTile& tl) -> int {
+    return args.mode == kKGrouped ? tab1[tl.group] / BK : 0;
+  };
+  auto tile_chunks = [&](const PairTile& tl) -> int {
+    return args.mode == kKGrouped ? (tab1[tl.group + 1] - tab1[tl.group]) / BK : args.k_tiles;
+  };
 
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
@@ -289,7 +268,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      const int k_stages = (args.k_tiles + kPairKC - 1) / kPairKC;
       // the leader announces the bytes of both CTAs' loads for a stage (boxes
       // reaching past the tensor are zero-filled and still count in full)
       const uint32_t bytes_pair = 2u * (L::A_BYTES + L::B_BYTES + L::SFA_BYTES + L::SFB_BYTES);
@@ -297,7 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const PairTile tl = decode_pair_tile(args, tab0, tab1, t);
         const int a_row = tl.row0 + 128 * static_cast<int>(rank);
         const int a_z = args.mode == kMasked ? tl.group : 0;
-        const int b_z = args.mode == kDense ? 0 : tl.group;
+        const int b_z = (args.mode == kDense || args.mode == kKGrouped) ? 0 : tl.group;
         // SwiGLU: CTA 0 takes the 128 gate rows and CTA 1 the matching 128 up
         // rows of the column block, so each CTA's accumulator row holds
         // [gate | up] of the same 128 output columns
@@ -307,13 +285,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int sfa_blk =
             (args.mode == kMasked ? tl.group * static_cast<int>(args.sfa_group_bytes / 512 / args.k_tiles) : 0) +
             a_row / 128;
-        const int sfb_grp = args.mode == kDense ? 0 : tl.group * args.n_sf_tiles;
+        const int sfb_grp = (args.mode == kDense || args.mode == kKGrouped) ? 0 : tl.group * args.n_sf_tiles;
         const int sfb_blk = sfb_grp + (SWIGLU ? tl.n_blk : tl.n_blk * 2);
+        const int kc0 = tile_kc0(tl);
+        const int k_stages = (tile_chunks(tl) + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
           if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), bytes_pair);
-          const int kc = ks * kPairKC;
+          const int kc = kc0 + ks * kPairKC;
           tma_load_4d_pair(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, fb, 0, a_row, kc, a_z);
           tma_load_4d_pair(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, fb, 0, b_row, kc, b_z);
           tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, fb, 0, kc, sfa_blk);
@@ -345,14 +325,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = pair; t < total && ok; t += npairs) {
         if (!mbar_wait(acce_bar, acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
-        const int k_stages = (args.k_tiles + kPairKC - 1) / kPairKC;
+        const int chunks = tile_chunks(decode_pair_tile(args, tab0, tab1, t));
+        const int k_stages = (chunks + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
           // the copier's commit implies both CTAs' operands of the stage have landed
           if (!mbar_wait(sfready_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < kPairKC; ++c) {
-            // a chunk past K holds zeros with zero-code scales and adds nothing
+            // a chunk past K holds zeros with zero-code scales and adds nothing;
+            // in the K-grouped form a chunk past the expert's tokens belongs to
+            // the next expert and is skipped
+            if (args.mode == kKGrouped && ks * kPairKC + c >= chunks) break;
             const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS + c * L::SF_CHUNK_COLS;
             const uint32_t sfb_t = sfa_t + 4;
             const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES + c * L::CHUNK;
@@ -390,7 +374,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs) {
-        const int k_stages = (args.k_tiles + kPairKC - 1) / kPairKC;
+        const int k_stages = (tile_chunks(decode_pair_tile(args, tab0, tab1, t)) + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
@@ -435,7 +419,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
       // dense rows past M are clipped by the tensor map; grouped rows past the
       // expert are not ours to write
-      const bool full = args.mode == kDense ? my_row0 < tl.rows_end : my_row0 + 128 <= tl.rows_end;
+      const bool dense_rows = args.mode == kDense || args.mode == kKGrouped;
+      const bool full = dense_rows ? my_row0 < tl.rows_end : my_row0 + 128 <= tl.rows_end;
       const bool none = my_row0 >= tl.rows_end;
       if constexpr (SWIGLU) {
         // ---- H = silu(gate) * up, requantised to MXFP8 along its columns:
@@ -492,11 +477,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_arrive_cluster(acce_leader);
       } else if (full) {
         uint32_t packed[kPairN / 2];
-        tmem_row_to_bf16<kPairN>(t_row, packed);
+        if (args.mode == kKGrouped && tile_chunks(tl) == 0) {
+#pragma unroll
+          for (int j = 0; j < kPairN / 2; ++j) packed[j] = 0u;  // an expert with no tokens has a zero gradient
+        } else {
+          tmem_row_to_bf16<kPairN>(t_row, packed);
+        }
         tc_fence_before();
         mbar_arrive_cluster(acce_leader);  // TMEM back to the leader's MMA warp before any store
         store_rows_tma<kPairN>(packed, r_local, sbase + L::OFF_STG, stg_count, &tmap_d, tl.n_blk * kPairN, my_row0,
-                               args.mode == kMasked ? tl.group : 0);
+                               (args.mode == kMasked || args.mode == kKGrouped) ? tl.group : 0);
       } else {
         // masked expert ending inside this CTA's rows: row-predicated stores
         const int r = my_row0 + r_local;
@@ -623,15 +613,16 @@ static cudaError_t launch_pair(const GemmProblem& p, int num_sms, cudaStream_t s
     return cudaErrorInvalidValue;
   CUtensorMap ta, tb, td, tsa, tsb;
   const int64_t a_depth = p.mode == kMasked ? p.groups : 1;
-  const int64_t b_depth = p.mode == kDense ? 1 : p.groups;
+  const int64_t b_depth = (p.mode == kDense || p.mode == kKGrouped) ? 1 : p.groups;
+  const int64_t d_depth = (p.mode == kMasked || p.mode == kKGrouped) ? p.groups : 1;  // K-grouped: D [groups, m, n]
   const int64_t sfa_bytes = a_depth * (((p.m + 127) / 128) * 128 * (p.k / 32));
   const int64_t sfb_bytes = b_depth * (((p.n + 127) / 128) * 128 * (p.k / 32));
   if (!make_tmap_kc(&ta, p.qa, p.k, p.m, a_depth)) return cudaErrorInvalidValue;
   if (!make_tmap_kc(&tb, p.qb, p.k, p.n, b_depth)) return cudaErrorInvalidValue;
   if (SWIGLU) {
-    if (!make_tmap_h(&td, p.d, p.i_dim, p.m, a_depth)) return cudaErrorInvalidValue;
+    if (!make_tmap_h(&td, p.d, p.i_dim, p.m, d_depth)) return cudaErrorInvalidValue;
   } else {
-    if (!make_tmap_d(&td, p.d, p.n, p.m, a_depth)) return cudaErrorInvalidValue;
+    if (!make_tmap_d(&td, p.d, p.n, p.m, d_depth)) return cudaErrorInvalidValue;
   }
   if (!make_tmap_sf(&tsa, p.sfa, sfa_bytes, p.k / BK, 1)) return cudaErrorInvalidValue;
   if (!make_tmap_sf(&tsb, p.sfb, sfb_bytes, p.k / BK, SWIGLU ? 1 : 2)) return cudaErrorInvalidValue;
@@ -664,7 +655,7 @@ static cudaError_t launch_pair(const GemmProblem& p, int num_sms, cudaStream_t s
   int64_t m_blocks;
   if (p.mode == kDense)
     m_blocks = (p.m + kPairM - 1) / kPairM;
-  else if (p.mode == kMasked)
+  else if (p.mode == kMasked || p.mode == kKGrouped)
     m_blocks = p.groups * ((p.m + kPairM - 1) / kPairM);
   else
     m_blocks = p.m / 128 / 2 + p.groups;  // each expert adds at most one half-used pair tile

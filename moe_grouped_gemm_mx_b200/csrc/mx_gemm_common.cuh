@@ -17,7 +17,7 @@ constexpr int kMaxGroups = 1024;
 constexpr int kGemmThreads = 224;  // 7 warps: producer, MMA, 4 epilogue, scale copier
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
-enum GemmMode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+enum GemmMode : int { kDense = 0, kContiguous = 1, kMasked = 2, kKGrouped = 3 };
 
 struct GemmArgs {
   const uint8_t* sfa;

@@ -38,6 +38,8 @@ def lib():
     L.mx_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_masked.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_gemm_swiglu_quant.argtypes = [P, P, P, P, P, P, I64, I64, I64, P, P]
+    L.mx_quantize_bf16_to_e4m3_transposed.argtypes = [P, I64, I64, I64, P, P, P]
+    L.mx_grouped_gemm_kgrouped.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_contiguous_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
     L.mx_grouped_gemm_masked_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
     return L
@@ -138,3 +140,20 @@ def test_swiglu_quant_argument_checks(lib):
     assert m(FAKE, FAKE, FAKE, FAKE, None, 4, 256, 256, 128, FAKE, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
     assert m(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 130, FAKE, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
     assert m(None, None, None, None, None, 4, 0, 256, 128, None, None, None, None) == MX_OK
+
+
+def test_training_side_argument_checks(lib):
+    t = lib.mx_quantize_bf16_to_e4m3_transposed
+    assert t(FAKE, 1, 48, 64, FAKE, FAKE, None) == MX_ERR_UNSUPPORTED_SHAPE   # rows % 32
+    assert t(FAKE, 1, 64, 60, FAKE, FAKE, None) == MX_ERR_UNSUPPORTED_SHAPE   # cols % 8
+    assert t(FAKE, -1, 64, 64, FAKE, FAKE, None) == MX_ERR_INVALID_ARGUMENT
+    assert t(None, 1, 64, 64, FAKE, FAKE, None) == MX_ERR_INVALID_ARGUMENT
+    assert t(FAKE, 1, 64, 64, FAKE + 8, FAKE, None) == MX_ERR_MISALIGNED
+    assert t(None, 0, 64, 64, None, None, None) == MX_OK
+    k = lib.mx_grouped_gemm_kgrouped
+    assert k(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 200, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert k(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 0, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert k(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 250, 256, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert k(FAKE, FAKE, FAKE, FAKE, None, 4, 256, 256, 256, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert k(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 256, 256, 256, FAKE, None, None) == MX_ERR_MISALIGNED
+    assert k(None, None, None, None, None, 0, 256, 256, 256, None, None, None) == MX_OK
