@@ -75,11 +75,21 @@ def static_config(name: str, seed: int) -> dict:
                     "padded_rows": int(I.padded_offsets(counts)[-1]),
                     "gemms": ["gate/up N=2x2048 K=7168 with fused SwiGLU + MXFP8 requantisation",
                               "down N=7168 K=2048 on the requantised activation"]})
+    elif name == "moe_bwd":
+        counts = I.zipf_routing_counts(seed=seed)
+        cfg.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "topk": I.MOE_TOPK,
+                    "zipf_s": I.MOE_ZIPF_S, "real_rows": int(counts.sum()),
+                    "padded_rows": int(I.padded_offsets(counts)[-1]),
+                    "gemms": ["dgrad dX[T,7168] = dY[T,4096] W13 (contiguous, W13 quantised along N)",
+                              "wgrad dW13[32,4096,7168] = dY^T X per expert (K-grouped over tokens)"]})
     elif name == "masked":
         mm = I.masked_counts(seed=seed)
         cfg.update({"experts": I.MASKED_EXPERTS, "max_m": I.MASKED_MAX_M, "n": I.MASKED_NK[0],
                     "k": I.MASKED_NK[1], "valid_rows": int(mm.sum()), "active_experts": int((mm > 0).sum())})
-    if name == "moe_mlp":
+    if name == "moe_bwd":
+        cfg["step"] = ("backward of the MoE gate/up projection: quantise dY row-wise, W13 along N, dY and X "
+                       "along tokens (transposed), then the dgrad and the K-grouped wgrad GEMMs, BF16 out")
+    elif name == "moe_mlp":
         cfg["step"] = ("quantise tokens + gate/up and down weights (one batched launch), then the fused "
                        "gate/up GEMM -> SwiGLU -> MXFP8 kernel and the down GEMM with BF16 epilogue")
     else:
@@ -93,7 +103,7 @@ def parse_args():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp"])
+    p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp", "moe_bwd"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -331,6 +341,52 @@ class Workload:
         self.config.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "real_rows": real,
                             "padded_rows": m_total})
 
+    def _build_moe_bwd(self, seed, I):
+        """Backward of the MoE gate/up projection (the contiguous workload's
+        first GEMM): input gradient dX = dY W13 per expert and weight gradient
+        dW13[e] = dY_e^T X_e over each expert's tokens."""
+        import torch
+        mx = self.mx
+        counts = I.zipf_routing_counts(seed=seed)
+        real = int(counts.sum())
+        n_out, k_in = I.MOE_GATE_NK
+        off_cpu = I.padded_offsets(counts)
+        t = int(off_cpu[-1])
+        experts = len(counts)
+        x = I.contiguous_problem(n=16, k=k_in, seed=seed, counts=counts, device=self.dev).a  # zero padding rows
+        dy = I.contiguous_problem(n=16, k=n_out, seed=seed + 1, counts=counts, device=self.dev).a
+        w = I.normal_bf16((experts, n_out, k_in), 0.02, seed + 5_000_011, self.dev)
+        for tt in (x, dy, w):
+            self._add_input(tt)
+        q_dy, sf_dy = self._quant(dy, "dY")
+        q_wt = torch.empty((experts, k_in, n_out), dtype=torch.uint8, device=self.dev)
+        sf_wt = torch.empty(experts * mx.scale_bytes(k_in, n_out), dtype=torch.uint8, device=self.dev)
+        q_dyt = torch.empty((n_out, t), dtype=torch.uint8, device=self.dev)
+        sf_dyt = torch.empty(mx.scale_bytes(n_out, t), dtype=torch.uint8, device=self.dev)
+        q_xt = torch.empty((k_in, t), dtype=torch.uint8, device=self.dev)
+        sf_xt = torch.empty(mx.scale_bytes(k_in, t), dtype=torch.uint8, device=self.dev)
+        qb = QUANT_BYTES_PER_ELT
+        self.launches.append(("quant", "W13 along N", lambda: mx.mx_quantize_bf16_to_e4m3_transposed(
+            w, q=q_wt, sf=sf_wt), w.numel() * qb, 0.0))
+        self.launches.append(("quant", "dY along tokens", lambda: mx.mx_quantize_bf16_to_e4m3_transposed(
+            dy, q=q_dyt, sf=sf_dyt), dy.numel() * qb, 0.0))
+        self.launches.append(("quant", "X along tokens", lambda: mx.mx_quantize_bf16_to_e4m3_transposed(
+            x, q=q_xt, sf=sf_xt), x.numel() * qb, 0.0))
+        off = off_cpu.to(self.dev)
+        dx = torch.empty((t, k_in), dtype=torch.bfloat16, device=self.dev)
+        dw = torch.empty((experts, n_out, k_in), dtype=torch.bfloat16, device=self.dev)
+        self.outputs += [dx, dw]
+        active = int((counts > 0).sum())
+        fl = 2.0 * real * n_out * k_in
+        self.launches.append(("gemm", "dgrad", lambda: mx.mx_grouped_gemm_contiguous(
+            q_dy, sf_dy, q_wt, sf_wt, off, d=dx, dev_status=self.status),
+            self._gemm_bytes(t, k_in, n_out, active), fl))
+        wbytes = (n_out + k_in) * t * (1 + 1 / 32) + 2.0 * experts * n_out * k_in
+        self.launches.append(("gemm", "wgrad", lambda: mx.mx_grouped_gemm_kgrouped(
+            q_dyt, sf_dyt, q_xt, sf_xt, off, groups=experts, d=dw, dev_status=self.status), wbytes, fl))
+        self.flops += 2 * fl
+        self.config.update({"experts": experts, "tokens": I.MOE_TOKENS, "real_rows": real, "padded_rows": t})
+
     def _build_masked(self, seed, I):
         import torch
         mx = self.mx
@@ -406,6 +462,24 @@ def oracle_sample(name, seed, target_s=10.0):
         jobs.append(job)
         desc = "gate/up GEMM on 64 rows over 2 experts (quantise rows and both experts' weights)"
         del counts, g
+    elif name == "moe_bwd":
+        n_out, k_in = I.MOE_GATE_NK
+        dy = I.normal_bf16((64, n_out), 1.0, seed + 7)
+        x = I.normal_bf16((64, k_in), 1.0, seed + 8)
+        w = I.normal_bf16((2, n_out, k_in), 0.02, seed + 9)
+
+        def job():
+            off = np.array([0, 32, 64], dtype=np.int32)
+            qdy, sdy = L.quantize(dy)
+            qwt, swt = L.quantize_transposed(w)
+            L.grouped_contiguous(qdy, sdy, qwt.reshape(2, k_in, n_out), swt, off)   # dgrad
+            qdyt, sdyt = L.quantize_transposed(dy)
+            qxt, sxt = L.quantize_transposed(x)
+            L.grouped_kgrouped(qdyt, sdyt, qxt, sxt, off, rows=np.arange(64, dtype=np.int64))  # wgrad, 64 rows
+            return 2.0 * 64 * n_out * k_in + 2.0 * 64 * 32 * k_in
+        jobs.append(job)
+        desc = ("backward of the gate/up projection on 64 tokens over 2 experts: quantise dY, W13 along N, "
+                "dY and X along tokens; dgrad for all 64 tokens, wgrad for 64 output rows")
     elif name == "moe_mlp":
         n13, k = I.MOE_GATE_NK
         n2, i_dim = I.MOE_DOWN_NK

@@ -18,9 +18,10 @@
 // shared-memory store) into a 32 KiB row-major staging buffer; then thread j
 // walks column j down the 128 rows -- a warp reads 64 contiguous bytes of a
 // staged row per step, free of bank conflicts -- and quantises its four
-// 32-row blocks with the FP32 block rule (exact for BF16 input), writing the
-// column's 128 bytes as one contiguous run of the output row and its four
-// scale bytes, adjacent in the tiled layout, as one 32-bit store.  Scale
+// 32-row blocks with the FP32 block rule (exact for BF16 input); its four
+// scale bytes, adjacent in the tiled layout, leave as one 32-bit store.  The
+// E4M3 tile is restaged in (swizzled) shared memory and written out as
+// 128-byte row runs by groups of 8 threads.  Scale
 // padding (rows of the transposed operand up to a multiple of 128, blocks up
 // to a multiple of 4) is written as 0x00 by the CTAs that own it.
 #include <cuda_bf16.h>
@@ -81,24 +82,48 @@ __global__ void __launch_bounds__(kTQThreads) mx_quant_t_kernel(const TQArgs a) 
   // scale bytes of (transposed row c, blocks 4*rt .. 4*rt+3): one 32-bit word
   const int64_t sf_off = (static_cast<int64_t>(c >> 7) * a.sf_ktiles + rt) * 512 + (c & 31) * 16 + ((c & 127) >> 5) * 4;
   const int c_pad = (a.cols + 127) / 128 * 128;
-  if (t >= cols_here) {
-    if (c < c_pad) *reinterpret_cast<uint32_t*>(sfg + sf_off) = 0u;  // scale padding rows
-    return;
-  }
-  uint8_t* qrow = a.q + (static_cast<int64_t>(g) * a.cols + c) * a.rows + r0;
+  uint32_t qv[32];  // this column's 128 output bytes
   uint32_t sfw = 0;
+  if (t < cols_here) {
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    if (b * 32 >= rows_here) break;  // blocks past the rows stay 0x00 (scale padding)
-    float h[32];
+    for (int b = 0; b < 4; ++b) {
+      if (b * 32 < rows_here) {  // blocks past the rows stay 0x00 (scale padding)
+        float h[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) h[j] = __uint_as_float(static_cast<uint32_t>(tile[b * 32 + j][t]) << 16);
-    uint32_t q8[8];
-    sfw |= quant_block32_f32(h, q8) << (8 * b);
-    *reinterpret_cast<uint4*>(qrow + b * 32) = make_uint4(q8[0], q8[1], q8[2], q8[3]);
-    *reinterpret_cast<uint4*>(qrow + b * 32 + 16) = make_uint4(q8[4], q8[5], q8[6], q8[7]);
+        for (int j = 0; j < 32; ++j) h[j] = __uint_as_float(static_cast<uint32_t>(tile[b * 32 + j][t]) << 16);
+        uint32_t q8[8];
+        sfw |= quant_block32_f32(h, q8) << (8 * b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qv[b * 8 + i] = q8[i];
+      }
+    }
+    *reinterpret_cast<uint32_t*>(sfg + sf_off) = sfw;
+  } else if (c < c_pad) {
+    *reinterpret_cast<uint32_t*>(sfg + sf_off) = 0u;  // scale padding rows
   }
-  *reinterpret_cast<uint32_t*>(sfg + sf_off) = sfw;
+  // ---- restage the [128 columns x 128 rows] E4M3 tile so every output row
+  // leaves as contiguous 128-byte runs (a lane-per-row store pattern would
+  // send 16-byte pieces to 32 different rows per instruction).  Row t of the
+  // staging area holds column t's bytes; its 16-byte chunk j sits at slot
+  // j ^ (t & 7) so that 8 consecutive rows spread over all banks.
+  __syncthreads();  // every thread is done reading the BF16 tile
+  uint4* stg = reinterpret_cast<uint4*>(&tile[0][0]);  // 16 KiB of the 32 KiB buffer
+  if (t < cols_here) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      stg[t * 8 + (j ^ (t & 7))] = make_uint4(qv[4 * j], qv[4 * j + 1], qv[4 * j + 2], qv[4 * j + 3]);
+  }
+  __syncthreads();
+  const int chunks = rows_here / 16;  // valid 16-byte chunks per output row
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = i * 16 + (t >> 3);  // output row = column c0 + row
+    const int j = t & 7;
+    if (row < cols_here && j < chunks) {
+      uint8_t* dst = a.q + (static_cast<int64_t>(g) * a.cols + c0 + row) * a.rows + r0 + j * 16;
+      *reinterpret_cast<uint4*>(dst) = stg[row * 8 + (j ^ (row & 7))];
+    }
+  }
 }
 
 cudaError_t launch_quant_transposed(const void* x, int64_t groups, int64_t rows, int64_t cols, void* q, void* sf,
