@@ -50,6 +50,17 @@ QUANT_BYTES_PER_ELT = 2.0 + 1.0 + 1.0 / 32.0
 METRIC = "MXFP8 GEMM & grouped-GEMM TFLOPS on 1 B200; % of dense FP8 tensor peak"
 
 
+# MoE problem size: the configured 32 experts x 8192 tokens unless
+# --experts / --tokens override it (used only to make small ncu captures)
+MOE_OVERRIDE = {"experts": None, "tokens": None}
+
+
+def moe_counts(I, seed):
+    experts = MOE_OVERRIDE["experts"] or I.MOE_EXPERTS
+    tokens = MOE_OVERRIDE["tokens"] or I.MOE_TOKENS
+    return I.zipf_routing_counts(tokens=tokens, experts=experts, topk=min(I.MOE_TOPK, experts), seed=seed)
+
+
 def static_config(name: str, seed: int) -> dict:
     """Workload description shared by both arms (no GPU needed)."""
     import mx_inputs as I
@@ -63,21 +74,21 @@ def static_config(name: str, seed: int) -> dict:
         cfg.update({"shapes": [f"{I.LARGE_M}x{n}x{k}" for n, k in I.LARGE_NK],
                     "a": "row-wise 2^U[-4,4] * N(0,1)", "b": "N(0,0.02)"})
     elif name == "contiguous":
-        counts = I.zipf_routing_counts(seed=seed)
-        cfg.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "topk": I.MOE_TOPK,
+        counts = moe_counts(I, seed)
+        cfg.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "topk": I.MOE_TOPK,
                     "zipf_s": I.MOE_ZIPF_S, "real_rows": int(counts.sum()),
                     "padded_rows": int(I.padded_offsets(counts)[-1]),
                     "gemms": ["gate_up N=4096 K=7168", "down N=7168 K=2048"]})
     elif name == "moe_mlp":
-        counts = I.zipf_routing_counts(seed=seed)
-        cfg.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "topk": I.MOE_TOPK,
+        counts = moe_counts(I, seed)
+        cfg.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "topk": I.MOE_TOPK,
                     "zipf_s": I.MOE_ZIPF_S, "real_rows": int(counts.sum()),
                     "padded_rows": int(I.padded_offsets(counts)[-1]),
                     "gemms": ["gate/up N=2x2048 K=7168 with fused SwiGLU + MXFP8 requantisation",
                               "down N=7168 K=2048 on the requantised activation"]})
     elif name == "moe_bwd":
-        counts = I.zipf_routing_counts(seed=seed)
-        cfg.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "topk": I.MOE_TOPK,
+        counts = moe_counts(I, seed)
+        cfg.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "topk": I.MOE_TOPK,
                     "zipf_s": I.MOE_ZIPF_S, "real_rows": int(counts.sum()),
                     "padded_rows": int(I.padded_offsets(counts)[-1]),
                     "gemms": ["dgrad dX[T,7168] = dY[T,4096] W13 (contiguous, W13 quantised along N)",
@@ -110,6 +121,10 @@ def parse_args():
     p.add_argument("--no-flush", action="store_true", help="skip the L2 flush (for ncu launch lists)")
     p.add_argument("--eager", action="store_true", help="launch kernels directly instead of a CUDA graph")
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--experts", type=int, default=None,
+                   help="MoE workloads: experts instead of the configured 32 (small profiling captures only)")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="MoE workloads: tokens instead of the configured 8192 (small profiling captures only)")
     p.add_argument("--ref-seconds", type=float, default=None,
                    help="CPU seconds per reference-arm step (default: sized so the run ends in ~2 min)")
     return p.parse_args()
@@ -282,7 +297,7 @@ class Workload:
     def _build_contiguous(self, seed, I):
         import torch
         mx = self.mx
-        counts = I.zipf_routing_counts(seed=seed)
+        counts = moe_counts(I, seed)
         real = int(counts.sum())
         for (n, k), tag in ((I.MOE_GATE_NK, "gate_up"), (I.MOE_DOWN_NK, "down")):
             prob = I.contiguous_problem(n=n, k=k, seed=seed + (0 if tag == "gate_up" else 100),
@@ -301,7 +316,7 @@ class Workload:
                                   mx.mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, off, d=d, dev_status=self.status),
                                   self._gemm_bytes(m_total, n, k, experts), fl))
             self.flops += fl
-        self.config.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "topk": I.MOE_TOPK,
+        self.config.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "topk": I.MOE_TOPK,
                             "zipf_s": I.MOE_ZIPF_S, "real_rows": real,
                             "padded_rows": int(I.padded_offsets(counts)[-1]),
                             "gemms": ["gate_up N=4096 K=7168", "down N=7168 K=2048"]})
@@ -311,7 +326,7 @@ class Workload:
         then the down GEMM on its output (the contiguous workload's shapes)."""
         import torch
         mx = self.mx
-        counts = I.zipf_routing_counts(seed=seed)
+        counts = moe_counts(I, seed)
         real = int(counts.sum())
         n13, k = I.MOE_GATE_NK
         n2, i_dim = I.MOE_DOWN_NK
@@ -338,7 +353,7 @@ class Workload:
         self.launches.append(("gemm", "down", lambda: mx.mx_grouped_gemm_contiguous(
             qh, sfh, q2, sf2, off, d=y, dev_status=self.status), self._gemm_bytes(m_total, n2, i_dim, experts), fl2))
         self.flops += fl1 + fl2
-        self.config.update({"experts": I.MOE_EXPERTS, "tokens": I.MOE_TOKENS, "real_rows": real,
+        self.config.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "real_rows": real,
                             "padded_rows": m_total})
 
     def _build_moe_bwd(self, seed, I):
@@ -347,7 +362,7 @@ class Workload:
         dW13[e] = dY_e^T X_e over each expert's tokens."""
         import torch
         mx = self.mx
-        counts = I.zipf_routing_counts(seed=seed)
+        counts = moe_counts(I, seed)
         real = int(counts.sum())
         n_out, k_in = I.MOE_GATE_NK
         off_cpu = I.padded_offsets(counts)
@@ -385,7 +400,8 @@ class Workload:
         self.launches.append(("gemm", "wgrad", lambda: mx.mx_grouped_gemm_kgrouped(
             q_dyt, sf_dyt, q_xt, sf_xt, off, groups=experts, d=dw, dev_status=self.status), wbytes, fl))
         self.flops += 2 * fl
-        self.config.update({"experts": experts, "tokens": I.MOE_TOKENS, "real_rows": real, "padded_rows": t})
+        self.config.update({"experts": experts, "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "real_rows": real,
+                            "padded_rows": t})
 
     def _build_masked(self, seed, I):
         import torch
@@ -447,7 +463,7 @@ def oracle_sample(name, seed, target_s=10.0):
         jobs.append(lambda: sum(dense_sample(a, b, None) for a, b in probs))
         desc = "a 64-row slice of A per shape (quantise it and all of B, GEMM it)"
     elif name == "contiguous":
-        counts = I.zipf_routing_counts(seed=seed)
+        counts = moe_counts(I, seed)
         n, k = I.MOE_GATE_NK
         g = np.random.default_rng(seed)
         a = I.normal_bf16((64, k), 1.0, seed + 7)
@@ -802,6 +818,8 @@ def run_ours(args, world, rank, local):
 
 def main():
     args = parse_args()
+    MOE_OVERRIDE["experts"] = args.experts
+    MOE_OVERRIDE["tokens"] = args.tokens
     world, rank, local = dist_init(args)
     try:
         if args.impl == "reference":
