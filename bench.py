@@ -248,7 +248,8 @@ class Workload:
         nbytes = sum(x.numel() for x in xs) * QUANT_BYTES_PER_ELT
         label = "+".join(j[3] for j in self.quant_jobs)
         assert len(xs) <= 8
-        self.launches.insert(0, ("quant", label, lambda: mx.mx_quantize_bf16_to_e4m3_multi(xs, outs), nbytes, 0.0))
+        self.launches.insert(0, ("quant", label, lambda *xs_: mx.mx_quantize_bf16_to_e4m3_multi(list(xs_), outs),
+                                 nbytes, 0.0, tuple(xs)))
 
     def _add_input(self, t):
         import torch
@@ -270,8 +271,9 @@ class Workload:
         d = torch.empty((m, n), dtype=torch.bfloat16, device=self.dev)
         self.outputs.append(d)
         fl = 2.0 * m * n * k
-        self.launches.append(("gemm", label, lambda: mx.mx_gemm(qa, sfa, qb, sfb, d=d, dev_status=self.status),
-                              self._gemm_bytes(m, n, k), fl))
+        self.launches.append(("gemm", label, lambda qa, sfa, qb, sfb: mx.mx_gemm(qa, sfa, qb, sfb, d=d,
+                                                                                dev_status=self.status),
+                              self._gemm_bytes(m, n, k), fl, (qa, sfa, qb, sfb)))
         self.flops += fl
 
     # -- workloads
@@ -312,9 +314,9 @@ class Workload:
             self.outputs.append(d)
             fl = 2.0 * real * n * k
             experts = int((counts > 0).sum())
-            self.launches.append(("gemm", tag, lambda qa=qa, sfa=sfa, qb=qb, sfb=sfb, off=off, d=d:
+            self.launches.append(("gemm", tag, lambda qa, sfa, qb, sfb, off, d=d:
                                   mx.mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, off, d=d, dev_status=self.status),
-                                  self._gemm_bytes(m_total, n, k, experts), fl))
+                                  self._gemm_bytes(m_total, n, k, experts), fl, (qa, sfa, qb, sfb, off)))
             self.flops += fl
         self.config.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "topk": I.MOE_TOPK,
                             "zipf_s": I.MOE_ZIPF_S, "real_rows": real,
@@ -347,11 +349,14 @@ class Workload:
         experts = int((counts > 0).sum())
         fl1 = 2.0 * real * n13 * k
         bytes1 = (m_total * k + experts * n13 * k + m_total * i_dim) * (1 + 1 / 32)
-        self.launches.append(("gemm", "gate_up+swiglu", lambda: mx.mx_grouped_gemm_contiguous_swiglu_quant(
-            qa, sfa, q13, sf13, off, qh=qh, sfh=sfh, dev_status=self.status), bytes1, fl1))
+        self.launches.append(("gemm", "gate_up+swiglu", lambda qa, sfa, q13, sf13, off:
+                              mx.mx_grouped_gemm_contiguous_swiglu_quant(qa, sfa, q13, sf13, off, qh=qh, sfh=sfh,
+                                                                         dev_status=self.status),
+                              bytes1, fl1, (qa, sfa, q13, sf13, off)))
         fl2 = 2.0 * real * n2 * i_dim
-        self.launches.append(("gemm", "down", lambda: mx.mx_grouped_gemm_contiguous(
-            qh, sfh, q2, sf2, off, d=y, dev_status=self.status), self._gemm_bytes(m_total, n2, i_dim, experts), fl2))
+        self.launches.append(("gemm", "down", lambda qh, sfh, q2, sf2, off: mx.mx_grouped_gemm_contiguous(
+            qh, sfh, q2, sf2, off, d=y, dev_status=self.status), self._gemm_bytes(m_total, n2, i_dim, experts), fl2,
+            (qh, sfh, q2, sf2, off)))
         self.flops += fl1 + fl2
         self.config.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "real_rows": real,
                             "padded_rows": m_total})
@@ -381,24 +386,25 @@ class Workload:
         q_xt = torch.empty((k_in, t), dtype=torch.uint8, device=self.dev)
         sf_xt = torch.empty(mx.scale_bytes(k_in, t), dtype=torch.uint8, device=self.dev)
         qb = QUANT_BYTES_PER_ELT
-        self.launches.append(("quant", "W13 along N", lambda: mx.mx_quantize_bf16_to_e4m3_transposed(
-            w, q=q_wt, sf=sf_wt), w.numel() * qb, 0.0))
-        self.launches.append(("quant", "dY along tokens", lambda: mx.mx_quantize_bf16_to_e4m3_transposed(
-            dy, q=q_dyt, sf=sf_dyt), dy.numel() * qb, 0.0))
-        self.launches.append(("quant", "X along tokens", lambda: mx.mx_quantize_bf16_to_e4m3_transposed(
-            x, q=q_xt, sf=sf_xt), x.numel() * qb, 0.0))
+        self.launches.append(("quant", "W13 along N", lambda w: mx.mx_quantize_bf16_to_e4m3_transposed(
+            w, q=q_wt, sf=sf_wt), w.numel() * qb, 0.0, (w,)))
+        self.launches.append(("quant", "dY along tokens", lambda dy: mx.mx_quantize_bf16_to_e4m3_transposed(
+            dy, q=q_dyt, sf=sf_dyt), dy.numel() * qb, 0.0, (dy,)))
+        self.launches.append(("quant", "X along tokens", lambda x: mx.mx_quantize_bf16_to_e4m3_transposed(
+            x, q=q_xt, sf=sf_xt), x.numel() * qb, 0.0, (x,)))
         off = off_cpu.to(self.dev)
         dx = torch.empty((t, k_in), dtype=torch.bfloat16, device=self.dev)
         dw = torch.empty((experts, n_out, k_in), dtype=torch.bfloat16, device=self.dev)
         self.outputs += [dx, dw]
         active = int((counts > 0).sum())
         fl = 2.0 * real * n_out * k_in
-        self.launches.append(("gemm", "dgrad", lambda: mx.mx_grouped_gemm_contiguous(
+        self.launches.append(("gemm", "dgrad", lambda q_dy, sf_dy, q_wt, sf_wt, off: mx.mx_grouped_gemm_contiguous(
             q_dy, sf_dy, q_wt, sf_wt, off, d=dx, dev_status=self.status),
-            self._gemm_bytes(t, k_in, n_out, active), fl))
+            self._gemm_bytes(t, k_in, n_out, active), fl, (q_dy, sf_dy, q_wt, sf_wt, off)))
         wbytes = (n_out + k_in) * t * (1 + 1 / 32) + 2.0 * experts * n_out * k_in
-        self.launches.append(("gemm", "wgrad", lambda: mx.mx_grouped_gemm_kgrouped(
-            q_dyt, sf_dyt, q_xt, sf_xt, off, groups=experts, d=dw, dev_status=self.status), wbytes, fl))
+        self.launches.append(("gemm", "wgrad", lambda q_dyt, sf_dyt, q_xt, sf_xt, off: mx.mx_grouped_gemm_kgrouped(
+            q_dyt, sf_dyt, q_xt, sf_xt, off, groups=experts, d=dw, dev_status=self.status), wbytes, fl,
+            (q_dyt, sf_dyt, q_xt, sf_xt, off)))
         self.flops += 2 * fl
         self.config.update({"experts": experts, "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "real_rows": real,
                             "padded_rows": t})
@@ -419,15 +425,16 @@ class Workload:
         rows = int(prob.masked_m.sum())
         active = int((prob.masked_m > 0).sum())
         fl = 2.0 * rows * n * k
-        self.launches.append(("gemm", "masked", lambda: mx.mx_grouped_gemm_masked(
-            qa, sfa, qb, sfb, mm, d=d, dev_status=self.status), self._gemm_bytes(rows, n, k, active), fl))
+        self.launches.append(("gemm", "masked", lambda qa, sfa, qb, sfb, mm: mx.mx_grouped_gemm_masked(
+            qa, sfa, qb, sfb, mm, d=d, dev_status=self.status), self._gemm_bytes(rows, n, k, active), fl,
+            (qa, sfa, qb, sfb, mm)))
         self.flops += fl
         self.config.update({"experts": e, "max_m": max_m, "n": n, "k": k, "valid_rows": rows,
                             "active_experts": active})
 
     def run_eager(self):
-        for _, _, fn, _, _ in self.launches:
-            fn()
+        for _, _, fn, _, _, inputs in self.launches:
+            fn(*inputs)
 
 
 # ---------------------------------------------------------------- oracle (CPU) timing
@@ -697,23 +704,38 @@ def run_ours(args, world, rank, local):
     barrier(world)
     t_wall1 = time.time()
 
-    # per-kernel device time: every kernel of the step launched on its own
-    # after an L2 flush, bracketed by CUDA events on its stream (events inside
-    # the captured step would add their own latency to every kernel)
-    k_start = [torch.cuda.Event(enable_timing=True) for _ in range(n_k)]
-    k_end = [torch.cuda.Event(enable_timing=True) for _ in range(n_k)]
+    # per-kernel device time: each kernel of the step replayed back to back in
+    # a CUDA graph over rotating copies of its operands (together larger than
+    # L2, so no launch finds its operands cached by the previous ones), CUDA
+    # events on the stream around the graph, divided by the number of
+    # launches.  Events recorded around every single kernel would add several
+    # microseconds of their own to each (measured: 16 vs 8 us for a page-shape
+    # GEMM), and a single kernel is what the roofline is about.
     kern_ms = [[] for _ in range(n_k)]
+    k_copies = []
     kernel_reps = max(3, min(args.steps, 10))
-    with torch.cuda.stream(stream):
-        for _ in range(kernel_reps):
-            for i, (_, _, fn, _, _) in enumerate(wl.launches):
-                if not args.no_flush:
-                    flush_buf.zero_()
-                k_start[i].record()
-                fn()
-                k_end[i].record()
-                k_end[i].synchronize()
-                kern_ms[i].append(k_start[i].elapsed_time(k_end[i]))
+    l2_cover = 256 * 1024 * 1024
+    for i, (_, _, fn, _, _, inputs) in enumerate(wl.launches):
+        in_bytes = sum(t.numel() * t.element_size() for t in inputs)
+        copies = max(1, min(32, -(-l2_cover // max(in_bytes, 1))))
+        bufs = [inputs] + [tuple(t.clone() for t in inputs) for _ in range(copies - 1)]
+        per_replay = max(copies, 4)
+        with torch.cuda.stream(stream):
+            fn(*bufs[-1])  # one eager launch on the copies before capture
+            torch.cuda.synchronize()
+            g_k = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_k, stream=stream):
+                for j in range(per_replay):
+                    fn(*bufs[j % copies])
+            for rep in range(kernel_reps + 1):
+                s_ev.record()
+                g_k.replay()
+                e_ev.record()
+                e_ev.synchronize()
+                if rep > 0:  # the first replay warms the graph
+                    kern_ms[i].append(s_ev.elapsed_time(e_ev) / per_replay)
+        k_copies.append(copies)
+        del g_k, bufs
     torch.cuda.synchronize()
     sampler.stop()
     clocks = sampler.summary(t_wall0 - 0.25, t_wall1 + 0.25)
@@ -728,7 +750,7 @@ def run_ours(args, world, rank, local):
 
     # per-kernel breakdown and the roofline of the dominant kernel kind
     per_launch = []
-    for i, (kind, label, _, nbytes, fl) in enumerate(wl.launches):
+    for i, (kind, label, _, nbytes, fl, _) in enumerate(wl.launches):
         per_launch.append({"kind": kind, "label": label, "ms": statistics.mean(kern_ms[i]),
                            "bytes": nbytes, "flops": fl})
     kinds = {}
@@ -758,8 +780,9 @@ def run_ours(args, world, rank, local):
     roof["traffic"] = None if trf is None else trf
     roof.update({"kernel": dom, "launches_per_step": dk["launches"], "avg_launch_ms": dk["ms"] / dk["launches"],
                  "peak_source": peak_note,
-                 "timing": f"each kernel of the step launched alone after an L2 flush, CUDA events on its "
-                           f"stream, mean of {kernel_reps} launches"})
+                 "timing": f"each kernel of the step replayed back to back in a CUDA graph over rotating "
+                           f"copies of its operands (together >= 256 MiB, larger than L2), CUDA events on its stream "
+                           f"around the graph, {kernel_reps} replays; operand copies per kernel: {k_copies}"})
 
     # end to end through the public API: pinned host inputs -> device, step, result -> host
     e2e = None
