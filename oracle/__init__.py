@@ -80,6 +80,12 @@ def lib():
         L.mxo_grouped_masked.restype = None
         L.mxo_grouped_kgrouped.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, I64, P, P]
         L.mxo_grouped_kgrouped.restype = None
+        L.mxo_tw_quantize_rows.argtypes = [P, I64, I64, P, P]
+        L.mxo_tw_quantize_rows.restype = None
+        L.mxo_tw_quantize_blocks.argtypes = [P, I64, I64, P, P]
+        L.mxo_tw_quantize_blocks.restype = None
+        L.mxo_tw_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P, P]
+        L.mxo_tw_gemm.restype = None
         L.mxo_num_threads.argtypes = []
         L.mxo_num_threads.restype = ctypes.c_int
         _lib = L
@@ -303,6 +309,49 @@ def grouped_kgrouped(qa, sfa, qb, sfb, offsets, rows=None):
                                _p(ids), nrows, _p(d), _p(a))
     if ids is None:
         return d.reshape(groups, m, n), a.reshape(groups, m, n)
+    return d, a
+
+
+# ---------------------------------------------------------------- tile-wise FP32-scaled FP8
+
+def tw_quantize_rows(x):
+    """BF16 [rows, k] -> (q uint8 [rows, k], s float32 [k/128, rows]): one FP32
+    scale per row and 128-element K tile."""
+    xb = _u16(x)
+    rows, k = xb.shape
+    assert k % 128 == 0
+    q = np.zeros((rows, k), dtype=np.uint8)
+    s = np.zeros((k // 128, rows), dtype=np.float32)
+    lib().mxo_tw_quantize_rows(_p(xb), rows, k, _p(q), _p(s))
+    return q, s
+
+
+def tw_quantize_blocks(x):
+    """BF16 [rows, k] -> (q uint8 [rows, k], s float32 [ceil(rows/128), k/128]):
+    one FP32 scale per 128 x 128 block."""
+    xb = _u16(x)
+    rows, k = xb.shape
+    assert k % 128 == 0
+    q = np.zeros((rows, k), dtype=np.uint8)
+    s = np.zeros(((rows + 127) // 128, k // 128), dtype=np.float32)
+    lib().mxo_tw_quantize_blocks(_p(xb), rows, k, _p(q), _p(s))
+    return q, s
+
+
+def tw_gemm(qa, sa, qb, sb, rows=None):
+    """D = deq(A) deq(B)^T in fp64 with tile-wise FP32 scales (sa [k/128, m],
+    sb [ceil(n/128), k/128]).  Returns (d, abssum) [nrows, n]."""
+    qa = np.ascontiguousarray(qa, dtype=np.uint8)
+    qb = np.ascontiguousarray(qb, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sb = np.ascontiguousarray(sb, dtype=np.float32)
+    m, k = qa.shape
+    n = qb.shape[0]
+    ids = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nrows = m if ids is None else len(ids)
+    d = np.zeros((nrows, n), dtype=np.float64)
+    a = np.zeros((nrows, n), dtype=np.float64)
+    lib().mxo_tw_gemm(_p(qa), _p(sa), _p(qb), _p(sb), m, n, k, _p(ids), nrows, _p(d), _p(a))
     return d, a
 
 

@@ -442,6 +442,103 @@ void mxo_grouped_kgrouped(const uint8_t *qa, const uint8_t *sfa, const uint8_t *
     }
 }
 
+/* ------------------------------------------------- tile-wise FP32-scaled FP8 */
+
+/* The FP8 format with fine-grained FP32 scales that DeepGEMM's GEMMs take
+ * (the pages: "tile-wise" scaling of the FP8 mixed-precision recipe, and
+ * DeepGEMM's FP32 two-level accumulation).  One FP32 scale per tile of
+ * elements: s = amax / 448 in FP32 (448 = largest E4M3 value), each element
+ * x / s in FP32 (IEEE division, round to nearest) encoded as E4M3 with
+ * round-to-nearest-even and saturation.  An all-zero tile gets s = 1; a tile
+ * holding NaN or +-Inf gets s = NaN and every element 0x7F.  FP32 arithmetic
+ * is done in float on purpose: the device quantiser computes the same
+ * correctly rounded FP32 quotients. */
+static void tw_quantize_tile(const uint16_t *x, int64_t stride, int rows, int cols, uint8_t *q,
+                             int64_t qstride, float *scale)
+{
+    float amax = 0.0f;
+    int nonfinite = 0;
+    for (int r = 0; r < rows; ++r)
+        for (int c = 0; c < cols; ++c) {
+            float v = (float)mxo_bf16_to_double(x[r * stride + c]);
+            if (!isfinite(v))
+                nonfinite = 1;
+            else if (fabsf(v) > amax)
+                amax = fabsf(v);
+        }
+    if (nonfinite) {
+        *scale = NAN;
+        for (int r = 0; r < rows; ++r)
+            for (int c = 0; c < cols; ++c)
+                q[r * qstride + c] = 0x7F;
+        return;
+    }
+    volatile float s = amax == 0.0f ? 1.0f : amax / 448.0f;
+    *scale = s;
+    for (int r = 0; r < rows; ++r)
+        for (int c = 0; c < cols; ++c) {
+            volatile float v = (float)mxo_bf16_to_double(x[r * stride + c]) / s;
+            q[r * qstride + c] = mxo_e4m3_encode((double)v);
+        }
+}
+
+/* Activations: one scale per row and 128-element K tile ("1 x 128").
+ * x [rows, k] BF16, k % 128 == 0; q [rows, k]; s [k/128, rows] (K-tile major). */
+void mxo_tw_quantize_rows(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, float *s)
+{
+    int64_t kt = k / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t t = 0; t < kt; ++t)
+            tw_quantize_tile(x + r * k + t * 128, k, 1, 128, q + r * k + t * 128, k, s + t * rows + r);
+}
+
+/* Weights: one scale per 128 x 128 block ("128 x 128"; a last block of
+ * fewer than 128 rows covers what there is).  x [rows, k] BF16, k % 128 == 0;
+ * q [rows, k]; s [ceil(rows/128), k/128]. */
+void mxo_tw_quantize_blocks(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, float *s)
+{
+    int64_t kt = k / 128, rb = (rows + 127) / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < rb; ++b) {
+        int nr = (int)(rows - b * 128 < 128 ? rows - b * 128 : 128);
+        for (int64_t t = 0; t < kt; ++t)
+            tw_quantize_tile(x + b * 128 * k + t * 128, k, nr, 128, q + b * 128 * k + t * 128, k,
+                             s + b * kt + t);
+    }
+}
+
+/* D = deq(A) * deq(B)^T in double, k ascending, for the listed rows (all when
+ * row_ids is NULL): deq(a[i, kk]) = e4m3(qa[i, kk]) * sa[kk/128, i],
+ * deq(b[j, kk]) = e4m3(qb[j, kk]) * sb[j/128, kk/128].  d, abssum [nrows, n]. */
+void mxo_tw_gemm(const uint8_t *qa, const float *sa, const uint8_t *qb, const float *sb, int64_t m,
+                 int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows, double *d,
+                 double *abssum)
+{
+    double tab[256];
+    mxo_e4m3_table(tab);
+    int64_t kt = k / 128;
+    if (!row_ids)
+        nrows = m;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = row_ids ? row_ids[r] : r;
+        for (int64_t j = 0; j < n; ++j) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t kk = 0; kk < k; ++kk) {
+                double a = tab[qa[i * k + kk]] * (double)sa[(kk / 128) * m + i];
+                double b = tab[qb[j * k + kk]] * (double)sb[(j / 128) * kt + kk / 128];
+                double p = a * b;
+                acc += p;
+                aacc += fabs(p);
+            }
+            d[r * n + j] = acc;
+            if (abssum)
+                abssum[r * n + j] = aacc;
+        }
+    }
+}
+
 int mxo_num_threads(void)
 {
 #ifdef _OPENMP

@@ -45,6 +45,11 @@ void mxo_grouped_kgrouped(const uint8_t *qa, const uint8_t *sfa, const uint8_t *
                           const uint8_t *sfb, const int32_t *offsets, int32_t groups,
                           int64_t m, int64_t n, int64_t k_total, const int64_t *row_ids,
                           int64_t nrows, double *d, double *abssum);
+void mxo_tw_quantize_rows(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, float *s);
+void mxo_tw_quantize_blocks(const uint16_t *x, int64_t rows, int64_t k, uint8_t *q, float *s);
+void mxo_tw_gemm(const uint8_t *qa, const float *sa, const uint8_t *qb, const float *sb, int64_t m,
+                 int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows, double *d,
+                 double *abssum);
 int mxo_num_threads(void);
 
 #ifdef __cplusplus

@@ -524,3 +524,75 @@ def test_kgrouped_one_group_equals_dense_and_sum_over_groups(oracle):
     ids = np.array([0, 39, 40 + 7, 3 * 40 + 39], dtype=np.int64)
     sub, _ = oracle.grouped_kgrouped(qa, sfa, qb, sfb, np.array([0, 128, 160, 160, 384], dtype=np.int32), rows=ids)
     np.testing.assert_array_equal(sub, parts.reshape(-1, 24)[ids])
+
+
+# ---------------------------------------------------------------- tile-wise FP32-scaled FP8 (DeepGEMM format)
+
+def test_tw_quantize_power_of_two_scales_are_exact(oracle):
+    """amax = 448 * 2^j gives s = 2^j exactly, so every BF16 value that is an
+    E4M3 value times 2^j quantises to that E4M3 code."""
+    table = oracle.e4m3_table()
+    finite = [c for c in range(0x7F) if c not in (0x7F,)]
+    rng = np.random.default_rng(3)
+    for j in (-10, -3, 0, 4, 20):
+        codes = rng.choice(finite, size=128).astype(np.uint8)
+        codes[5] = 0x7E                     # amax = 448 * 2^j
+        signs = rng.choice([0, 0x80], size=128).astype(np.uint8)
+        vals = np.array([table[c] for c in codes]) * 2.0 ** j
+        vals = np.where(signs == 0x80, -vals, vals)
+        x = torch.from_numpy(vals).to(torch.bfloat16)
+        q, s = oracle.tw_quantize_rows(x.reshape(1, 128))
+        assert s[0, 0] == np.float32(2.0 ** j)
+        want = codes | signs
+        want[(codes == 0) & (signs == 0x80)] = 0x80   # -0 keeps its sign
+        assert np.array_equal(q[0], want), j
+
+
+def test_tw_quantize_matches_torch_division_and_cast(oracle):
+    """Independent path: FP32 division in torch and torch's own float8_e4m3fn
+    cast of the quotient give the oracle's codes; s is amax / 448 in FP32."""
+    g = torch.Generator().manual_seed(8)
+    x = (torch.randn(64, 512, generator=g) * torch.exp2(torch.randint(-8, 8, (64, 1), generator=g).float())
+         ).to(torch.bfloat16)
+    q, s = oracle.tw_quantize_rows(x)
+    xf = x.float().reshape(64, 4, 128)
+    amax = xf.abs().amax(dim=2)
+    s_t = amax / torch.tensor(448.0)
+    assert np.array_equal(s.T, s_t.numpy())
+    codes = (xf / s_t[:, :, None]).to(torch.float8_e4m3fn).view(torch.uint8).reshape(64, 512).numpy()
+    assert np.array_equal(q, codes)
+    # every tile's largest element lands on +-448
+    assert np.all((q.reshape(64, 4, 128) & 0x7F).max(axis=2) == 0x7E)
+
+
+def test_tw_quantize_blocks_and_special_tiles(oracle):
+    g = torch.Generator().manual_seed(9)
+    x = torch.randn(200, 256, generator=g).to(torch.bfloat16)   # 2 row blocks (128 + 72) x 2 K tiles
+    x[128:, 128:] = 0.0                                         # an all-zero block
+    x[3, 7] = float("inf")                                      # a non-finite block
+    q, s = oracle.tw_quantize_blocks(x)
+    assert s.shape == (2, 2)
+    assert np.isnan(s[0, 0]) and np.all(q[:128, :128] == 0x7F)
+    assert s[1, 1] == 1.0 and np.all((q[128:, 128:] & 0x7F) == 0)
+    blk = x[:128, 128:].float()
+    assert s[0, 1] == np.float32(blk.abs().max().item()) / np.float32(448.0)
+    assert s[1, 0] == np.float32(x[128:, :128].float().abs().max().item()) / np.float32(448.0)
+
+
+def test_tw_gemm_equals_mxfp8_gemm_on_power_of_two_scales(oracle):
+    """With tile scales that are powers of two the tile-wise dequantisation is
+    an MXFP8 dequantisation with the same exponent in every 32-block of the
+    tile, so the two oracle GEMMs must agree exactly."""
+    rng = np.random.default_rng(12)
+    m, n, k = 9, 140, 256
+    qa = rng.integers(0, 0x7F, size=(m, k)).astype(np.uint8) | rng.choice([0, 0x80], size=(m, k)).astype(np.uint8)
+    qb = rng.integers(0, 0x7F, size=(n, k)).astype(np.uint8)
+    ja = rng.integers(-6, 6, size=(k // 128, m))
+    jb = rng.integers(-6, 6, size=((n + 127) // 128, k // 128))
+    sa = np.exp2(ja).astype(np.float32)
+    sb = np.exp2(jb).astype(np.float32)
+    d_tw, a_tw = oracle.tw_gemm(qa, sa, qb, sb)
+    sfa = (127 + np.repeat(ja.T, 4, axis=1)).astype(np.uint8)                    # [m, k/32]
+    sfb = (127 + np.repeat(np.repeat(jb, 128, axis=0)[:n], 4, axis=1)).astype(np.uint8)  # [n, k/32]
+    d_mx, a_mx = oracle.gemm(qa, sfa, qb, sfb)
+    assert np.array_equal(d_tw, d_mx) and np.array_equal(a_tw, a_mx)
