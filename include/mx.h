@@ -242,6 +242,44 @@ mx_status mx_grouped_gemm_masked_swiglu_quant(const void *qa, const void *sfa, c
                                               int64_t max_m, int64_t i_dim, int64_t k, void *qh, void *sfh,
                                               int32_t *dev_status, mx_stream_t stream);
 
+/*
+ * Tile-wise FP32-scaled FP8: the format with fine-grained FP32 scales that
+ * DeepGEMM's GEMMs take (the pages: "tile-wise" scaling in the FP8
+ * mixed-precision recipe; DeepGEMM's FP32 two-level accumulation), with
+ * DeepSeek-V3's tiles: 1 x 128 for activations, 128 x 128 for weights.
+ * Per tile: s = amax / 448 in FP32 (IEEE division), element x / s (IEEE FP32
+ * division) as E4M3 with saturating round-to-nearest-even; an all-zero tile
+ * gets s = 1, a tile holding NaN or +-Inf gets s = NaN (0x7FC00000) and
+ * elements 0x7F.  Scales are plain FP32 arrays:
+ *   1 x 128:   scales [k/128, rows]          (K-tile major)
+ *   128 x 128: scales [ceil(rows/128), k/128]
+ * x [rows, k] BF16 16-byte aligned, q [rows, k]; requires k % 128 == 0.
+ */
+mx_status mx_quantize_bf16_to_e4m3_tile1x128(const void *x_bf16, int64_t rows, int64_t k, void *q_e4m3,
+                                             float *scales, mx_stream_t stream);
+mx_status mx_quantize_bf16_to_e4m3_block128x128(const void *x_bf16, int64_t rows, int64_t k, void *q_e4m3,
+                                                float *scales, mx_stream_t stream);
+
+/*
+ * GEMM on tile-wise FP32-scaled FP8 operands:
+ *   D[i, j] = sum_kt sa[kt, i] * sb[j/128, kt] * sum_{k in K tile kt} e4m3(a[i,k]) * e4m3(b[j,k])
+ * qa [m, k] with sa [k/128, m] (1 x 128 tiles); qb [n, k] with sb
+ * [ceil(n/128), k/128] (128 x 128 blocks); d_bf16 [m, n].  Each K tile's
+ * products are summed by the tensor core into a TMEM accumulator and
+ * promoted into FP32 with its two scales (DeepGEMM's two-level accumulation,
+ * "DeepSeek drops DeepGEMM" page, section 1).  Requires k % 128 == 0,
+ * n % 16 == 0, 16-byte aligned qa/qb/d, 4-byte aligned scales.
+ * The contiguous grouped form follows mx_grouped_gemm_contiguous: qb
+ * [groups, n, k], sb [groups, ceil(n/128), k/128], device group_offsets
+ * (multiples of 128), sa [k/128, m_total].
+ */
+mx_status mx_gemm_tilewise(const void *qa, const float *sa, const void *qb, const float *sb, void *d_bf16,
+                           int64_t m, int64_t n, int64_t k, int32_t *dev_status, mx_stream_t stream);
+mx_status mx_grouped_gemm_contiguous_tilewise(const void *qa, const float *sa, const void *qb, const float *sb,
+                                              const int32_t *group_offsets, int32_t groups, int64_t m_total,
+                                              int64_t n, int64_t k, void *d_bf16, int32_t *dev_status,
+                                              mx_stream_t stream);
+
 /* Copies the library-internal device status word (used when a call got
  * dev_status == NULL) to *host_out and, if clear != 0, resets it.
  * Synchronises the device. */

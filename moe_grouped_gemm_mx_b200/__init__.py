@@ -26,8 +26,9 @@ __all__ = [
     "mx_gemm",
     "mx_grouped_gemm_contiguous", "mx_grouped_gemm_masked", "mx_gemm_swiglu_quant",
     "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant",
-    "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped", "read_internal_status",
-    "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "C_SYMBOLS",
+    "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped", "mx_quantize_bf16_to_e4m3_tile1x128",
+    "mx_quantize_bf16_to_e4m3_block128x128", "mx_gemm_tilewise", "mx_grouped_gemm_contiguous_tilewise",
+    "read_internal_status", "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "C_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,7 +45,8 @@ C_SYMBOLS = [
     "mx_grouped_gemm_contiguous",
     "mx_grouped_gemm_masked", "mx_read_internal_status", "mx_gemm_swiglu_quant",
     "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant",
-    "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped",
+    "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped", "mx_quantize_bf16_to_e4m3_tile1x128",
+    "mx_quantize_bf16_to_e4m3_block128x128", "mx_gemm_tilewise", "mx_grouped_gemm_contiguous_tilewise",
 ]
 
 
@@ -63,7 +65,7 @@ def _load():
     if not os.path.exists(lib_path):
         raise ImportError(
             f"moe_grouped_gemm_mx_b200: CUDA library {lib_path} is missing; build it with "
-            "`python -m moe_grouped_gemm_mx_b200._build` (or __graft_entry__.build())")
+            "`python moe_grouped_gemm_mx_b200/_build.py` (or __graft_entry__.build())")
     L = ctypes.CDLL(lib_path)
     P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
     L.mx_status_string.argtypes = [ctypes.c_int]
@@ -92,6 +94,14 @@ def _load():
     L.mx_quantize_bf16_to_e4m3_transposed.restype = ctypes.c_int
     L.mx_grouped_gemm_kgrouped.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_kgrouped.restype = ctypes.c_int
+    L.mx_quantize_bf16_to_e4m3_tile1x128.argtypes = [P, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3_tile1x128.restype = ctypes.c_int
+    L.mx_quantize_bf16_to_e4m3_block128x128.argtypes = [P, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3_block128x128.restype = ctypes.c_int
+    L.mx_gemm_tilewise.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
+    L.mx_gemm_tilewise.restype = ctypes.c_int
+    L.mx_grouped_gemm_contiguous_tilewise.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
+    L.mx_grouped_gemm_contiguous_tilewise.restype = ctypes.c_int
     L.mx_read_internal_status.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
     L.mx_read_internal_status.restype = ctypes.c_int
     return L
@@ -300,6 +310,79 @@ def mx_grouped_gemm_kgrouped(qa, sfa, qb, sfb, group_offsets: torch.Tensor, grou
     st = _lib.mx_grouped_gemm_kgrouped(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(group_offsets), groups,
                                        m, n, k_total, _ptr(d), _status_arg(dev_status), _stream(stream))
     _raise(st, "mx_grouped_gemm_kgrouped")
+    return d
+
+
+def _tw_quant(fn, name, x, q, s, scale_shape, stream):
+    _check(x, torch.bfloat16, "x")
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [rows, K]")
+    rows, k = x.shape
+    if q is None:
+        q = torch.empty((rows, k), dtype=torch.uint8, device=x.device)
+    if s is None:
+        s = torch.empty(scale_shape, dtype=torch.float32, device=x.device)
+    _check(q, torch.uint8, "q")
+    _check(s, torch.float32, "scales")
+    if q.numel() != x.numel() or s.numel() < int(torch.tensor(scale_shape).prod()):
+        raise ValueError("output buffers too small")
+    _raise(fn(_ptr(x), rows, k, _ptr(q), _ptr(s), _stream(stream)), name)
+    return q, s
+
+
+def mx_quantize_bf16_to_e4m3_tile1x128(x: torch.Tensor, q=None, s=None, stream=None):
+    """BF16 [rows, K] -> (q uint8 [rows, K], s float32 [K/128, rows]): one FP32
+    scale per row and 128-element K tile (s = amax/448)."""
+    rows, k = x.shape
+    return _tw_quant(_lib.mx_quantize_bf16_to_e4m3_tile1x128, "mx_quantize_bf16_to_e4m3_tile1x128", x, q, s,
+                     (k // 128, rows), stream)
+
+
+def mx_quantize_bf16_to_e4m3_block128x128(x: torch.Tensor, q=None, s=None, stream=None):
+    """BF16 [rows, K] -> (q uint8 [rows, K], s float32 [ceil(rows/128), K/128]): one
+    FP32 scale per 128 x 128 block (s = amax/448)."""
+    rows, k = x.shape
+    return _tw_quant(_lib.mx_quantize_bf16_to_e4m3_block128x128, "mx_quantize_bf16_to_e4m3_block128x128", x, q, s,
+                     ((rows + 127) // 128, k // 128), stream)
+
+
+def mx_gemm_tilewise(qa, sa, qb, sb, d: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Tile-wise FP32-scaled FP8 GEMM: qa uint8 [M, K] with sa float32 [K/128, M],
+    qb uint8 [N, K] with sb float32 [ceil(N/128), K/128] -> bf16 [M, N]."""
+    for t, nm in ((qa, "qa"), (qb, "qb")):
+        _check(t, torch.uint8, nm)
+    for t, nm in ((sa, "sa"), (sb, "sb")):
+        _check(t, torch.float32, nm)
+    m, k = qa.shape
+    n = qb.shape[0]
+    if d is None:
+        d = torch.empty((m, n), dtype=torch.bfloat16, device=qa.device)
+    _check(d, torch.bfloat16, "d")
+    _raise(_lib.mx_gemm_tilewise(_ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), _ptr(d), m, n, k, _status_arg(dev_status),
+                                 _stream(stream)), "mx_gemm_tilewise")
+    return d
+
+
+def mx_grouped_gemm_contiguous_tilewise(qa, sa, qb, sb, group_offsets: torch.Tensor, d: torch.Tensor | None = None,
+                                        dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Contiguous grouped form: qa [M_total, K], sa [K/128, M_total], qb [E, N, K],
+    sb [E, ceil(N/128), K/128], group_offsets int32 [E+1] -> bf16 [M_total, N]."""
+    for t, nm in ((qa, "qa"), (qb, "qb")):
+        _check(t, torch.uint8, nm)
+    for t, nm in ((sa, "sa"), (sb, "sb")):
+        _check(t, torch.float32, nm)
+    _check(group_offsets, torch.int32, "group_offsets")
+    m_total, k = qa.shape
+    groups, n, kb = qb.shape
+    if kb != k or group_offsets.numel() != groups + 1:
+        raise ValueError("shape mismatch")
+    if d is None:
+        d = torch.empty((m_total, n), dtype=torch.bfloat16, device=qa.device)
+    _check(d, torch.bfloat16, "d")
+    _raise(_lib.mx_grouped_gemm_contiguous_tilewise(_ptr(qa), _ptr(sa), _ptr(qb), _ptr(sb), _ptr(group_offsets),
+                                                    groups, m_total, n, k, _ptr(d), _status_arg(dev_status),
+                                                    _stream(stream)), "mx_grouped_gemm_contiguous_tilewise")
     return d
 
 

@@ -1,7 +1,10 @@
 """Ahead-of-time build of the sm_100a library ``libmx.so`` (no JIT).
 
-    python -m moe_grouped_gemm_mx_b200._build          # build if stale
-    python -m moe_grouped_gemm_mx_b200._build --force  # rebuild
+    python moe_grouped_gemm_mx_b200/_build.py          # build if stale
+    python moe_grouped_gemm_mx_b200/_build.py --force  # rebuild
+
+(run as a file, not as a package module: importing the package loads the
+library, which is what this script builds)
 
 nvcc cross-compiles for sm_100a on a machine without a GPU, so the library is
 built in-tree and travels with the source tree.
@@ -17,7 +20,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmx.so")
-SOURCES = ["mx_api.cu", "mx_gemm.cu", "mx_gemm2.cu", "mx_quant.cu", "mx_quant_t.cu"]
+SOURCES = ["mx_api.cu", "mx_gemm.cu", "mx_gemm2.cu", "mx_quant.cu", "mx_quant_t.cu", "mx_quant_tw.cu",
+           "mx_gemm_tw.cu"]
 HEADERS = ["mx_ptx.cuh", "mx_launch.h", "mx_fastdiv.h", "mx_gemm_common.cuh", "mx_mxfp8.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

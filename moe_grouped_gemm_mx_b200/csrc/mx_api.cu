@@ -230,6 +230,60 @@ mx_status mx_grouped_gemm_kgrouped(const void* qa, const void* sfa, const void* 
   return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
 }
 
+// ---------------------------------------------------------------- tile-wise FP32-scaled FP8
+
+static mx_status tw_quantize(const void* x, int64_t rows, int64_t k, void* q, float* s, bool blocks,
+                             mx_stream_t stream) {
+  if (rows < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k % 128 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0 || k == 0) return MX_OK;
+  if (!x || !q || !s) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u)) return MX_ERR_MISALIGNED;
+  if (rows > kMaxDim || k > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(mxk::launch_tw_quant(x, rows, k, q, s, blocks, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mx_status mx_quantize_bf16_to_e4m3_tile1x128(const void* x_bf16, int64_t rows, int64_t k, void* q_e4m3,
+                                             float* scales, mx_stream_t stream) {
+  return tw_quantize(x_bf16, rows, k, q_e4m3, scales, false, stream);
+}
+
+mx_status mx_quantize_bf16_to_e4m3_block128x128(const void* x_bf16, int64_t rows, int64_t k, void* q_e4m3,
+                                                float* scales, mx_stream_t stream) {
+  return tw_quantize(x_bf16, rows, k, q_e4m3, scales, true, stream);
+}
+
+static mx_status tw_gemm(const void* qa, const float* sa, const void* qb, const float* sb,
+                         const int32_t* group_offsets, int32_t groups, int64_t m, int64_t n, int64_t k, void* d,
+                         int32_t* dev_status, int mode, mx_stream_t stream) {
+  if (groups < 0 || m < 0 || n < 0 || k < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (k == 0 || k % 128 != 0 || n % 16 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (groups == 0 || m == 0 || n == 0) return MX_OK;
+  if (!qa || !sa || !qb || !sb || !d || (mode == 1 && !group_offsets)) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(qa) || !aligned16(qb) || !aligned16(d) || (reinterpret_cast<uintptr_t>(sa) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sb) & 3u) || (reinterpret_cast<uintptr_t>(group_offsets) & 3u))
+    return MX_ERR_MISALIGNED;
+  if (m > kMaxDim || n > kMaxDim || k > kMaxDim || groups > kMaxGroups) return MX_ERR_UNSUPPORTED_SHAPE;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  mxk::TwProblem p{qa, sa, qb, sb, d, group_offsets, status, m, n, k, groups, mode};
+  return from_cuda(mxk::launch_gemm_tw(p, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mx_status mx_gemm_tilewise(const void* qa, const float* sa, const void* qb, const float* sb, void* d_bf16,
+                           int64_t m, int64_t n, int64_t k, int32_t* dev_status, mx_stream_t stream) {
+  return tw_gemm(qa, sa, qb, sb, nullptr, 1, m, n, k, d_bf16, dev_status, 0, stream);
+}
+
+mx_status mx_grouped_gemm_contiguous_tilewise(const void* qa, const float* sa, const void* qb, const float* sb,
+                                              const int32_t* group_offsets, int32_t groups, int64_t m_total,
+                                              int64_t n, int64_t k, void* d_bf16, int32_t* dev_status,
+                                              mx_stream_t stream) {
+  return tw_gemm(qa, sa, qb, sb, group_offsets, groups, m_total, n, k, d_bf16, dev_status, 1, stream);
+}
+
 // ---------------------------------------------------------------- fused SwiGLU + MXFP8 (expert MLP, first half)
 
 static mx_status check_swiglu(const void* qh, const void* sfh, int64_t i_dim) {

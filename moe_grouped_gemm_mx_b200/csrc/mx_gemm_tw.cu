@@ -1,0 +1,326 @@
+// mx_gemm_tw.cu -- GEMM on tile-wise FP32-scaled FP8 operands (the format of
+// mx_quant_tw.cu: A with one FP32 scale per row and 128-element K tile, B with
+// one per 128 x 128 block), dense and contiguous-grouped:
+//
+//   D[i, j] = sum_kt sa[kt, i] * sb[j/128, kt] * sum_{k in kt} e4m3(a[i,k]) e4m3(b[j,k])
+//
+// FP32 scales cannot ride inside the tensor core's block-scaled MMA (its
+// scales are powers of two), so this is DeepGEMM's two-level accumulation
+// ("DeepSeek drops DeepGEMM" page, section 1: FP8 products accumulated by the
+// tensor core, promoted into FP32 with the scales applied on CUDA cores),
+// rebuilt for B200: the first level is a TMEM accumulator, the promotion reads
+// it with tcgen05.ld.
+//
+// CTA layout (192 threads, one CTA per SM, persistent over 128 x 128 tiles):
+//   warp 0      TMA producer: A and B tiles of one 128-element K tile per
+//               stage, STAGES-deep ring.
+//   warp 1      TMEM owner and MMA issuer: each K tile's four K = 32
+//               block-scaled MMAs (every scale factor 2^0, staged once into
+//               TMEM) go into a FRESH partial accumulator, alternating
+//               between two TMEM buffers so that the tensor core fills one
+//               while the other is being promoted.
+//   warps 2..5  promotion and epilogue: each thread owns one row of the
+//               tile; per K tile it reads the row's 128 partial sums from
+//               TMEM, releases the buffer, and adds them times
+//               sa[kt, row] * sb[n-block, kt] into FP32 registers; after the
+//               last K tile it rounds to BF16 and leaves through swizzled
+//               staging and TMA stores.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "mx_gemm_common.cuh"
+#include "mx_launch.h"
+
+namespace mxk {
+
+constexpr int kTwStages = 6;
+constexpr int kTwThreads = 192;
+
+struct TwLayout {
+  static constexpr int A_BYTES = 128 * BK;  // 16 KB
+  static constexpr int B_BYTES = 128 * BK;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + kTwStages * A_BYTES;
+  static constexpr int OFF_ONES = OFF_B + kTwStages * B_BYTES;  // 512 bytes of scale code 127 (2^0)
+  static constexpr int OFF_STG = (OFF_ONES + 512 + 1023) / 1024 * 1024;
+  static constexpr int OFF_BAR = OFF_STG + 2 * 8192;
+  static constexpr int NUM_BARS = 2 * kTwStages + 4 + 1;  // full/empty per stage, accf[2], acce[2], drain
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_TAB0 = OFF_MISC + 16;
+  static constexpr int BYTES = OFF_TAB0 + (kMaxGroups + 1) * 4;
+  static constexpr int ALLOC = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t SF_COL = 256;  // unit scales: SFA 4 columns, then SFB 4 columns
+  static_assert(OFF_B % 1024 == 0 && OFF_STG % 1024 == 0, "swizzled tiles need 1024-B alignment");
+  static_assert(ALLOC <= 232448, "shared memory budget");
+};
+
+struct TwArgs {
+  const float* sa;               // [k_tiles, m]
+  const float* sb;               // [groups, nb, k_tiles]
+  const int32_t* group_offsets;  // contiguous form: [groups + 1]
+  int32_t* status;
+  int m, n, k_tiles, n_tiles, groups, mode;  // mode 0 dense, 1 contiguous
+};
+
+__global__ void __launch_bounds__(kTwThreads, 1)
+    mx_gemm_tw_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_d, const TwArgs args) {
+  using L = TwLayout;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile uint32_t* tmem_slot = misc + 0;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* total_slot = reinterpret_cast<volatile int*>(misc + 2);
+  int32_t* tab0 = reinterpret_cast<int32_t*>(smem + L::OFF_TAB0);
+
+  auto full_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * s; };
+  auto empty_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (kTwStages + s); };
+  auto accf_bar = [&](int b) { return sbase + L::OFF_BAR + 8u * (2 * kTwStages + b); };
+  auto acce_bar = [&](int b) { return sbase + L::OFF_BAR + 8u * (2 * kTwStages + 2 + b); };
+  const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (2 * kTwStages + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTwStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 128);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+  }
+  if (warp == 1) {  // 512 bytes of UE8M0 code 127 (= 2^0) for the MMA's scale operands
+    reinterpret_cast<uint4*>(smem + L::OFF_ONES)[lane] = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    prefetch_tmap(&tmap_d);
+  }
+  pdl_launch_dependents();
+  pdl_wait_prior();
+
+  int bad = 0;
+  if (args.mode == kContiguous) {
+    for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) tab0[i] = __ldg(args.group_offsets + i);
+    __syncthreads();
+    for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) {
+      const int32_t v = tab0[i];
+      if (v < 0 || (v % BM) != 0 || v > args.m) bad = 1;
+      if (i > 0 && v < tab0[i - 1]) bad = 1;
+    }
+  }
+  const int any_bad = __syncthreads_or(bad);
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    int total;
+    if (args.mode == kContiguous) {
+      total = any_bad ? 0 : (tab0[args.groups] - tab0[0]) / BM * args.n_tiles;
+      if (any_bad) report(args.status, 0x1);
+    } else {
+      total = ((args.m + BM - 1) / BM) * args.n_tiles;
+    }
+    *total_slot = total;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = *total_slot;
+
+  // tile t -> (expert, 128-row block, 128-column block)
+  auto decode = [&](int t, int& group, int& m_blk, int& n_blk) {
+    const int mb = t / args.n_tiles;
+    n_blk = t - mb * args.n_tiles;
+    if (args.mode == kContiguous) {
+      m_blk = tab0[0] / BM + mb;
+      group = last_le(tab0, args.groups, m_blk * BM);
+      if (group >= args.groups) group = args.groups - 1;
+    } else {
+      m_blk = mb;
+      group = 0;
+    }
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ===== TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int group, m_blk, n_blk;
+        decode(t, group, m_blk, n_blk);
+        for (int kt = 0; kt < args.k_tiles; ++kt) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(stage), L::A_BYTES + L::B_BYTES);
+          tma_load_3d(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, full_bar(stage), kt * BK, m_blk * BM, 0);
+          tma_load_3d(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, full_bar(stage), kt * BK, n_blk * 128,
+                      args.mode == kContiguous ? group : 0);
+          if (++stage == kTwStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        report(args.status, 0x4);
+        *abort_flag = 1;
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 1000000ull) { }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ===== MMA issuer
+      const uint32_t sf = tmem_base + L::SF_COL;
+      tc_cp_32x128b_warpx4(sf, desc_sf_32x16(sbase + L::OFF_ONES));      // SFA: 2^0 everywhere
+      tc_cp_32x128b_warpx4(sf + 4, desc_sf_32x16(sbase + L::OFF_ONES));  // SFB
+      const uint32_t idesc0 = idesc_mxf8_e4m3(BM, 128);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t ib = 0;  // K tiles issued so far (partial buffer = ib & 1)
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int kt = 0; kt < args.k_tiles; ++kt, ++ib) {
+          const uint32_t b = ib & 1u;
+          if (!mbar_wait(acce_bar(b), ((ib >> 1) & 1u) ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES;
+          const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb)
+            tc_mma_mxf8(tmem_base + b * 128, desc_kmajor_sw128(a_addr + 32 * kb), desc_kmajor_sw128(b_addr + 32 * kb),
+                        idesc_with_sf_ids(idesc0, kb, kb), sf | (static_cast<uint32_t>(kb) << 30),
+                        (sf + 4) | (static_cast<uint32_t>(kb) << 30), kb != 0 ? 1u : 0u);
+          tc_commit(empty_bar(stage));
+          tc_commit(accf_bar(b));
+          if (++stage == kTwStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        report(args.status, 0x4);
+        *abort_flag = 1;
+        tc_commit(drain_bar);
+        mbar_wait(drain_bar, 0, nullptr, 100000000ull);
+      }
+    }
+  } else {
+    // ===== promotion and epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
+    const int quarter = warp & 3;
+    const int r_local = quarter * 32 + lane;
+    uint32_t ib = 0;
+    uint32_t stg_count = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      int group, m_blk, n_blk;
+      decode(t, group, m_blk, n_blk);
+      const int row = m_blk * BM + r_local;
+      const bool row_ok = row < args.m;
+      const float* sb_t = args.sb + (static_cast<int64_t>(group) * args.n_tiles + n_blk) * args.k_tiles;
+      float acc[128];
+#pragma unroll
+      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      for (int kt = 0; kt < args.k_tiles; ++kt, ++ib) {
+        const uint32_t b = ib & 1u;
+        const float s = (row_ok ? __ldg(args.sa + static_cast<int64_t>(kt) * args.m + row) : 0.0f) * __ldg(sb_t + kt);
+        const bool got = mbar_wait(accf_bar(b), (ib >> 1) & 1u, abort_flag, kWaitLimitNs);
+        if (!named_barrier_and(2, 128, got)) {
+          if (threadIdx.x == 64) report(args.status, 0x4);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + b * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v0[32], v1[32];
+          tc_ld_32x32b_x32(t_row + h * 64, v0);
+          tc_ld_32x32b_x32(t_row + h * 64 + 32, v1);
+          tc_wait_ld();
+          if (h == 1) {  // every column of the buffer is in registers: hand it back
+            tc_fence_before();
+            mbar_arrive(acce_bar(b));
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            acc[h * 64 + j] = fmaf(s, __uint_as_float(v0[j]), acc[h * 64 + j]);
+            acc[h * 64 + 32 + j] = fmaf(s, __uint_as_float(v1[j]), acc[h * 64 + 32 + j]);
+          }
+        }
+      }
+      if (!ok) break;
+      uint32_t packed[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) packed[j] = pack_bf16x2(__float_as_uint(acc[2 * j]), __float_as_uint(acc[2 * j + 1]));
+      store_rows_tma<128>(packed, r_local, sbase + L::OFF_STG, stg_count, &tmap_d, n_blk * 128, m_blk * BM, 0);
+    }
+    if (threadIdx.x == 64) bulk_wait_group_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+static cudaError_t prepare_tw_kernel() {
+  static cudaError_t state = cudaErrorNotReady;
+  if (state == cudaErrorNotReady)
+    state = cudaFuncSetAttribute(mx_gemm_tw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TwLayout::ALLOC);
+  return state;
+}
+
+cudaError_t launch_gemm_tw(const TwProblem& p, int num_sms, cudaStream_t stream) {
+  cudaError_t e = prepare_tw_kernel();
+  if (e != cudaSuccess) return e;
+  const int64_t b_depth = p.mode == kContiguous ? p.groups : 1;
+  CUtensorMap ta, tb, td;
+  if (!make_tmap(&ta, p.qa, p.k, p.m, 1, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tb, p.qb, p.k, p.n, b_depth, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_d(&td, p.d, p.n, p.m, 1)) return cudaErrorInvalidValue;
+  TwArgs a = {};
+  a.sa = p.sa;
+  a.sb = p.sb;
+  a.group_offsets = p.group_offsets;
+  a.status = p.status;
+  a.m = static_cast<int>(p.m);
+  a.n = static_cast<int>(p.n);
+  a.k_tiles = static_cast<int>(p.k / BK);
+  a.n_tiles = static_cast<int>((p.n + 127) / 128);
+  a.groups = static_cast<int>(p.groups);
+  a.mode = p.mode;
+  const int64_t tiles_bound = ((p.m + BM - 1) / BM) * a.n_tiles;
+  if (tiles_bound == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles_bound < num_sms ? tiles_bound : num_sms), 1, 1);
+  cfg.blockDim = dim3(kTwThreads, 1, 1);
+  cfg.dynamicSmemBytes = TwLayout::ALLOC;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, mx_gemm_tw_kernel, ta, tb, td, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace mxk

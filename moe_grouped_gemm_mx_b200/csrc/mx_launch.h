@@ -47,4 +47,24 @@ cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, 
 // CTA-pair (2-SM MMA) kernel for large problems, any of the three forms.
 cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches);
 
+// Tile-wise FP32-scaled FP8 (mx_quant_tw.cu): blocks == false -> one scale per
+// row and 128-element K tile, s [k/128, rows]; true -> one per 128 x 128 block,
+// s [ceil(rows/128), k/128].
+cudaError_t launch_tw_quant(const void* x, int64_t rows, int64_t k, void* q, float* s, bool blocks,
+                            cudaStream_t stream);
+
+struct TwProblem {
+  const void* qa;                // [m, k] E4M3
+  const float* sa;               // [k/128, m]
+  const void* qb;                // [groups, n, k] E4M3
+  const float* sb;               // [groups, ceil(n/128), k/128]
+  void* d;                       // [m, n] BF16
+  const int32_t* group_offsets;  // contiguous form only
+  int32_t* status;
+  int64_t m, n, k, groups;
+  int mode;                      // 0 dense, 1 contiguous
+};
+
+cudaError_t launch_gemm_tw(const TwProblem& p, int num_sms, cudaStream_t stream);
+
 }  // namespace mxk

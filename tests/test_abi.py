@@ -23,8 +23,8 @@ def declared_functions():
 @pytest.fixture(scope="module")
 def lib():
     if not os.path.exists(LIB):
-        from moe_grouped_gemm_mx_b200 import _build
-        _build.build()
+        import __graft_entry__
+        __graft_entry__.build()
     L = ctypes.CDLL(LIB)
     P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
     L.mx_scale_bytes.argtypes = [I64, I64]
@@ -40,6 +40,10 @@ def lib():
     L.mx_gemm_swiglu_quant.argtypes = [P, P, P, P, P, P, I64, I64, I64, P, P]
     L.mx_quantize_bf16_to_e4m3_transposed.argtypes = [P, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_kgrouped.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3_tile1x128.argtypes = [P, I64, I64, P, P, P]
+    L.mx_quantize_bf16_to_e4m3_block128x128.argtypes = [P, I64, I64, P, P, P]
+    L.mx_gemm_tilewise.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
+    L.mx_grouped_gemm_contiguous_tilewise.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_contiguous_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
     L.mx_grouped_gemm_masked_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
     return L
@@ -157,3 +161,21 @@ def test_training_side_argument_checks(lib):
     assert k(FAKE, FAKE, FAKE, FAKE, None, 4, 256, 256, 256, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
     assert k(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 256, 256, 256, FAKE, None, None) == MX_ERR_MISALIGNED
     assert k(None, None, None, None, None, 0, 256, 256, 256, None, None, None) == MX_OK
+
+
+def test_tilewise_argument_checks(lib):
+    for q in (lib.mx_quantize_bf16_to_e4m3_tile1x128, lib.mx_quantize_bf16_to_e4m3_block128x128):
+        assert q(FAKE, 4, 96, FAKE, FAKE, None) == MX_ERR_UNSUPPORTED_SHAPE       # k % 128
+        assert q(FAKE, -1, 128, FAKE, FAKE, None) == MX_ERR_INVALID_ARGUMENT
+        assert q(FAKE, 4, 128, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
+        assert q(FAKE, 4, 128, FAKE, FAKE + 2, None) == MX_ERR_MISALIGNED
+        assert q(None, 0, 128, None, None, None) == MX_OK
+    g = lib.mx_gemm_tilewise
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 96, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 24, 128, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert g(FAKE, None, FAKE, FAKE, FAKE, 128, 256, 128, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert g(FAKE, FAKE + 2, FAKE, FAKE, FAKE, 128, 256, 128, None, None) == MX_ERR_MISALIGNED
+    assert g(None, None, None, None, None, 0, 256, 128, None, None) == MX_OK
+    c = lib.mx_grouped_gemm_contiguous_tilewise
+    assert c(FAKE, FAKE, FAKE, FAKE, None, 4, 512, 256, 128, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert c(FAKE, FAKE, FAKE, FAKE, FAKE, 2000, 512, 256, 128, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE

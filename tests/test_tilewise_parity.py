@@ -1,0 +1,106 @@
+"""Tile-wise FP32-scaled FP8 (DeepGEMM's format: 1 x 128 activation tiles,
+128 x 128 weight blocks, s = amax / 448) on the GPU vs the CPU oracle: both
+quantisers bit-exact (scales compared as FP32 bit patterns, NaN included),
+and the two-level-accumulation GEMM (TMEM partial per 128-element K tile,
+promoted with its scales in FP32) in dense and contiguous-grouped form within
+the GEMM tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import mx_inputs
+from mxtest_util import assert_gemm_close, to_np_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mx():
+    import moe_grouped_gemm_mx_b200 as m
+    return m
+
+
+def bits(a: np.ndarray) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+
+
+def check_quant(mx, oracle, x, blocks: bool):
+    dev = torch.device("cuda")
+    if blocks:
+        q, s = mx.mx_quantize_bf16_to_e4m3_block128x128(x.to(dev))
+        rq, rs = oracle.tw_quantize_blocks(x)
+    else:
+        q, s = mx.mx_quantize_bf16_to_e4m3_tile1x128(x.to(dev))
+        rq, rs = oracle.tw_quantize_rows(x)
+    torch.cuda.synchronize()
+    q = q.cpu().numpy()
+    s = s.cpu().numpy()
+    assert np.array_equal(bits(s), bits(rs)), f"{(bits(s) != bits(rs)).sum()} scales differ"
+    assert np.array_equal(q, rq), f"{(q != rq).sum()} element bytes differ"
+
+
+@pytest.mark.parametrize("blocks", [False, True])
+def test_tilewise_quant_every_bf16_pattern(mx, oracle, blocks):
+    bits16 = np.random.default_rng(1).permutation(np.arange(65536, dtype=np.int64)).astype(np.uint16)
+    x = torch.from_numpy(bits16.view(np.int16).reshape(256, 256).copy()).view(torch.bfloat16)
+    check_quant(mx, oracle, x, blocks)
+
+
+@pytest.mark.parametrize("shape", [(300, 512), (64, 7168), (129, 256), (1, 128)])
+@pytest.mark.parametrize("blocks", [False, True])
+def test_tilewise_quant_shapes(mx, oracle, shape, blocks):
+    x = mx_inputs.outlier_bf16(shape, seed=21)
+    if shape[0] >= 130:
+        x[129, 128:256] = 0.0           # a zero 1x128 tile (its block stays non-zero)
+        x[0, 300] = float("nan")        # a non-finite tile / block
+    check_quant(mx, oracle, x, blocks)
+
+
+def tw_dense(mx, oracle, m, n, k, seed, rows=None):
+    dev = torch.device("cuda")
+    a = mx_inputs.outlier_bf16((m, k), seed=seed)
+    b = mx_inputs.normal_bf16((n, k), 0.02, seed + 1)
+    qa, sa = mx.mx_quantize_bf16_to_e4m3_tile1x128(a.to(dev))
+    qb, sb = mx.mx_quantize_bf16_to_e4m3_block128x128(b.to(dev))
+    d = mx.mx_gemm_tilewise(qa, sa, qb, sb)
+    torch.cuda.synchronize()
+    d_ref, absd = oracle.tw_gemm(qa.cpu().numpy(), sa.cpu().numpy(), qb.cpu().numpy(), sb.cpu().numpy(), rows=rows)
+    dg = to_np_f64(d if rows is None else d[torch.as_tensor(rows, device=d.device)])
+    assert_gemm_close(dg, d_ref, absd, f"tile-wise {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("m,n,k", [(128, 256, 512), (200, 272, 1152), (17, 400, 128), (300, 128, 2048)])
+def test_tilewise_gemm_dense(mx, oracle, m, n, k):
+    tw_dense(mx, oracle, m, n, k, seed=30)
+
+
+def test_tilewise_gemm_page_shape(mx, oracle):
+    """The first dense shape of the DeepGEMM comparison table, 64 x 2112 x 7168."""
+    tw_dense(mx, oracle, 64, 2112, 7168, seed=31)
+
+
+def test_tilewise_gemm_contiguous(mx, oracle):
+    counts = torch.tensor([0, 5, 128, 200, 1, 0, 77], dtype=torch.int64)
+    n, k = 272, 384
+    prob = mx_inputs.contiguous_problem(n=n, k=k, seed=32, counts=counts)
+    e = len(counts)
+    dev = torch.device("cuda")
+    qa, sa = mx.mx_quantize_bf16_to_e4m3_tile1x128(prob.a.to(dev))
+    # expert weights [E, N, K] quantised as one [E*N, K] matrix: with N not a
+    # multiple of 128 the blocks would straddle experts, so quantise per expert
+    qb = torch.empty((e, n, k), dtype=torch.uint8, device=dev)
+    nb = (n + 127) // 128
+    sb = torch.empty((e, nb, k // 128), dtype=torch.float32, device=dev)
+    for x in range(e):
+        mx.mx_quantize_bf16_to_e4m3_block128x128(prob.b[x].to(dev), q=qb[x], s=sb[x])
+    off = prob.offsets.to(dev)
+    d = mx.mx_grouped_gemm_contiguous_tilewise(qa, sa, qb, sb, off)
+    torch.cuda.synchronize()
+    qa_h, sa_h, qb_h, sb_h = qa.cpu().numpy(), sa.cpu().numpy(), qb.cpu().numpy(), sb.cpu().numpy()
+    offs = prob.offsets.numpy()
+    for x in range(e):
+        r0, r1 = int(offs[x]), int(offs[x + 1])
+        if r1 == r0:
+            continue
+        d_ref, absd = oracle.tw_gemm(qa_h[r0:r1], np.ascontiguousarray(sa_h[:, r0:r1]), qb_h[x], sb_h[x])
+        assert_gemm_close(to_np_f64(d[r0:r1]), d_ref, absd, f"tile-wise contiguous expert {x}")
