@@ -120,6 +120,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-flush", action="store_true", help="skip the L2 flush (for ncu launch lists)")
     p.add_argument("--eager", action="store_true", help="launch kernels directly instead of a CUDA graph")
+    p.add_argument("--fmt", default="mxfp8", choices=["mxfp8", "tilewise"],
+                   help="operand format: MXFP8 (default) or tile-wise FP32-scaled FP8 (DeepGEMM's)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--experts", type=int, default=None,
                    help="MoE workloads: experts instead of the configured 32 (small profiling captures only)")
@@ -212,7 +214,7 @@ class ClockSampler:
 class Workload:
     """Device-resident inputs/outputs and the list of kernel launches of one step."""
 
-    def __init__(self, name, dev, seed, mx, inputs):
+    def __init__(self, name, dev, seed, mx, inputs, fmt="mxfp8"):
         import torch
         self.name = name
         self.dev = dev
@@ -224,6 +226,11 @@ class Workload:
         self.config = {"workload": name}
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.quant_jobs = []
+        self.fmt = fmt
+        if fmt == "tilewise":
+            if name not in ("pr1", "page", "large", "contiguous"):
+                raise SystemExit(f"--fmt tilewise applies to the dense and contiguous workloads, not {name}")
+            self.config["format"] = "tile-wise FP32-scaled FP8 (1x128 activations, 128x128 weights)"
         getattr(self, "_build_" + name)(seed, inputs)
         self._finish()
 
@@ -240,8 +247,10 @@ class Workload:
         return q, sf
 
     def _finish(self):
-        """All quantisations of the step go in one launch (up to 8 tensors),
-        ahead of the GEMMs."""
+        """All MXFP8 quantisations of the step go in one launch (up to 8
+        tensors), ahead of the GEMMs."""
+        if not self.quant_jobs:
+            return
         mx = self.mx
         xs = [j[0] for j in self.quant_jobs]
         outs = [(j[1], j[2]) for j in self.quant_jobs]
@@ -259,6 +268,21 @@ class Workload:
         # minimum traffic: A and B bytes once, their scales, D once
         return m_rows * k * (1 + 1 / 32) + b_experts * n * k * (1 + 1 / 32) + 2 * m_rows * n
 
+    def _tw_quant(self, x, label, blocks):
+        """Register a tile-wise FP32-scaled FP8 quantisation launch (1x128 tiles,
+        or 128x128 blocks of x viewed as [rows, k])."""
+        import torch
+        mx = self.mx
+        x2 = x.reshape(-1, x.shape[-1])
+        rows, k = x2.shape
+        q = torch.empty((rows, k), dtype=torch.uint8, device=self.dev)
+        shape = ((rows + 127) // 128, k // 128) if blocks else (k // 128, rows)
+        sc = torch.empty(shape, dtype=torch.float32, device=self.dev)
+        fn = mx.mx_quantize_bf16_to_e4m3_block128x128 if blocks else mx.mx_quantize_bf16_to_e4m3_tile1x128
+        nbytes = rows * k * 3.0 + sc.numel() * 4.0
+        self.launches.append(("quant", label, lambda x2: fn(x2, q=q, s=sc), nbytes, 0.0, (x2,)))
+        return q.reshape(x.shape), sc
+
     def _dense(self, a, b, label):
         import torch
         mx = self.mx
@@ -266,6 +290,17 @@ class Workload:
         n = b.shape[0]
         self._add_input(a)
         self._add_input(b)
+        if self.fmt == "tilewise":
+            qa, sa = self._tw_quant(a, label + ":A 1x128", False)
+            qb, sb = self._tw_quant(b, label + ":B 128x128", True)
+            d = torch.empty((m, n), dtype=torch.bfloat16, device=self.dev)
+            self.outputs.append(d)
+            fl = 2.0 * m * n * k
+            nbytes = m * k + n * k + sa.numel() * 4.0 + sb.numel() * 4.0 + 2.0 * m * n
+            self.launches.append(("gemm", label, lambda qa, sa, qb, sb: mx.mx_gemm_tilewise(
+                qa, sa, qb, sb, d=d, dev_status=self.status), nbytes, fl, (qa, sa, qb, sb)))
+            self.flops += fl
+            return
         qa, sfa = self._quant(a, label + ":A")
         qb, sfb = self._quant(b, label + ":B")
         d = torch.empty((m, n), dtype=torch.bfloat16, device=self.dev)
@@ -306,14 +341,25 @@ class Workload:
                                         counts=counts, device=self.dev)
             self._add_input(prob.a)
             self._add_input(prob.b)
-            qa, sfa = self._quant(prob.a, tag + ":A")
-            qb, sfb = self._quant(prob.b, tag + ":B")
             off = prob.offsets.to(self.dev)
             m_total = prob.a.shape[0]
             d = torch.empty((m_total, n), dtype=torch.bfloat16, device=self.dev)
             self.outputs.append(d)
             fl = 2.0 * real * n * k
             experts = int((counts > 0).sum())
+            if self.fmt == "tilewise":
+                qa, sa = self._tw_quant(prob.a, tag + ":A 1x128", False)
+                qb, sb = self._tw_quant(prob.b, tag + ":B 128x128", True)   # N % 128 == 0: blocks stay in one expert
+                sb = sb.reshape(len(counts), n // 128, k // 128)
+                nbytes = (m_total * k + experts * n * k) * 1.0 + (sa.numel() + sb.numel()) * 4.0 + 2.0 * m_total * n
+                self.launches.append(("gemm", tag, lambda qa, sa, qb, sb, off, d=d:
+                                      mx.mx_grouped_gemm_contiguous_tilewise(qa, sa, qb, sb, off, d=d,
+                                                                             dev_status=self.status),
+                                      nbytes, fl, (qa, sa, qb, sb, off)))
+                self.flops += fl
+                continue
+            qa, sfa = self._quant(prob.a, tag + ":A")
+            qb, sfb = self._quant(prob.b, tag + ":B")
             self.launches.append(("gemm", tag, lambda qa, sfa, qb, sfb, off, d=d:
                                   mx.mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, off, d=d, dev_status=self.status),
                                   self._gemm_bytes(m_total, n, k, experts), fl, (qa, sfa, qb, sfb, off)))
@@ -439,7 +485,7 @@ class Workload:
 
 # ---------------------------------------------------------------- oracle (CPU) timing
 
-def oracle_sample(name, seed, target_s=10.0):
+def oracle_sample(name, seed, target_s=10.0, fmt="mxfp8"):
     """Time the CPU oracle on a bounded sample of the workload.
 
     Returns (flops_per_second, description, threads)."""
@@ -450,9 +496,14 @@ def oracle_sample(name, seed, target_s=10.0):
     L = oracle
 
     def dense_sample(a, b, rows):
-        qa, sfa = L.quantize(a[:rows] if rows else a)
-        qb, sfb = L.quantize(b)
-        L.gemm(qa, sfa, qb, sfb)
+        if fmt == "tilewise":
+            qa, sa = L.tw_quantize_rows(a[:rows] if rows else a)
+            qb, sb = L.tw_quantize_blocks(b)
+            L.tw_gemm(qa, sa, qb, sb)
+        else:
+            qa, sfa = L.quantize(a[:rows] if rows else a)
+            qb, sfb = L.quantize(b)
+            L.gemm(qa, sfa, qb, sfb)
         m = qa.shape[0]
         return 2.0 * m * b.shape[0] * b.shape[1]
 
@@ -477,6 +528,12 @@ def oracle_sample(name, seed, target_s=10.0):
         b = I.normal_bf16((2, n, k), 0.02, seed + 8)
 
         def job():
+            if fmt == "tilewise":   # two experts of 32 rows each, per-expert tile-wise GEMMs
+                qa, sa = L.tw_quantize_rows(a)
+                for e in range(2):
+                    qb, sb = L.tw_quantize_blocks(b[e])
+                    L.tw_gemm(qa[32 * e:32 * (e + 1)], np.ascontiguousarray(sa[:, 32 * e:32 * (e + 1)]), qb, sb)
+                return 2.0 * 64 * n * k
             qa, sfa = L.quantize(a)
             qb, sfb = L.quantize(b)
             off = np.array([0, 32, 64], dtype=np.int32)
@@ -594,7 +651,7 @@ def run_reference(args, world, rank):
     target = args.ref_seconds if args.ref_seconds is not None else \
         max(1.0, min(10.0, 120.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup + args.steps):
-        rate, desc, threads = oracle_sample(args.workload, args.seed, target_s=target)
+        rate, desc, threads = oracle_sample(args.workload, args.seed, target_s=target, fmt=args.fmt)
         if i >= args.warmup:
             per_step.append(rate)
     flops_rate = statistics.median(per_step)
@@ -603,7 +660,7 @@ def run_reference(args, world, rank):
             "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": static_config(args.workload, args.seed),
+            "config": dict(static_config(args.workload, args.seed), format=args.fmt),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -646,7 +703,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     peaks = load_peaks()
 
-    wl = Workload(args.workload, dev, args.seed + 1000 * rank, mx, mx_inputs)
+    wl = Workload(args.workload, dev, args.seed + 1000 * rank, mx, mx_inputs, fmt=args.fmt)
     stream = torch.cuda.Stream(device=dev)
     flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
     n_k = len(wl.launches)
@@ -810,7 +867,7 @@ def run_ours(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, threads = oracle_sample(args.workload, args.seed, target_s=10.0)
+        rate, desc, threads = oracle_sample(args.workload, args.seed, target_s=10.0, fmt=args.fmt)
         cpu = {"value": rate / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
 
     launches_per_step = sum(1 for r in per_launch)
@@ -819,7 +876,7 @@ def run_ours(args, world, rank, local):
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3", "data": "synthetic",
-        "config": dict(static_config(args.workload, args.seed),
+        "config": dict(static_config(args.workload, args.seed), format=args.fmt,
                        l2="flushed (512 MiB write) before every timed step",
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU",
                        graph=graph is not None),
