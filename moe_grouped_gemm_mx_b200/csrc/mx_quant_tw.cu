@@ -11,12 +11,13 @@
 // are correctly rounded (__fdiv_rn), so the results are exactly those of the
 // definition.
 //
-//  * rows kernel (activations, [rows, k], scales [k/128, rows]): one warp per
-//    (row, 128-element K tile), 8 bytes (4 BF16) per lane, a warp max
-//    reduction for amax; HBM-bound.
+//  * rows kernel (activations, [rows, k], scales [k/128, rows]): a half-warp
+//    per 1 x 128 tile (16 bytes per lane), 8 tiles per warp with every load in
+//    flight before the arithmetic; HBM-bound.
 //  * blocks kernel (weights, [rows, k], scales [ceil(rows/128), k/128]): one
-//    256-thread CTA per 128 x 128 block, 64 elements per thread held in
-//    registers across the block-wide amax reduction.
+//    256-thread CTA per 128 x 128 block, a half-warp per row segment, 64
+//    elements per thread held in registers across the block-wide amax
+//    reduction.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -31,38 +32,68 @@ constexpr uint32_t kTwNaN = 0x7FC00000u;  // the quiet NaN written as the scale 
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
-__global__ void __launch_bounds__(256) tw_quant_rows_kernel(const uint2* __restrict__ x, uint32_t* __restrict__ q,
+// Activations: a half-warp (16 lanes x 16 bytes) holds one 1 x 128 tile; a
+// warp takes 8 tiles, all loads issued before any arithmetic (2 KiB in flight
+// per warp).  Tiles are numbered with the row fastest, so a warp's scale
+// stores are consecutive.
+__global__ void __launch_bounds__(256) tw_quant_rows_kernel(const uint4* __restrict__ x, uint2* __restrict__ q,
                                                              float* __restrict__ s, int rows, int ktiles) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
-  const int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);  // (tile, row), row fastest
-  if (w >= static_cast<int64_t>(rows) * ktiles) return;
-  const int row = static_cast<int>(w % rows);
-  const int kt = static_cast<int>(w / rows);
-  const int64_t k4 = static_cast<int64_t>(ktiles) * 32;  // row length in 4-element units
-  const uint2 v = x[row * k4 + kt * 32 + lane];
-  float f[4] = {bf16_bits_to_f32(v.x & 0xFFFFu), bf16_bits_to_f32(v.x >> 16), bf16_bits_to_f32(v.y & 0xFFFFu),
-                bf16_bits_to_f32(v.y >> 16)};
-  uint32_t m = 0;
+  const int half = lane >> 4;
+  const int hl = lane & 15;
+  const int64_t units = static_cast<int64_t>(rows) * ktiles;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int64_t k8 = static_cast<int64_t>(ktiles) * 16;  // row length in 8-element units
+  uint4 v[4];
+  int64_t idx[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) m = max(m, __float_as_uint(f[i]) & 0x7FFFFFFFu);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  uint32_t out;
-  float sc;
-  if (m >= 0x7F800000u) {
-    sc = __uint_as_float(kTwNaN);
-    out = 0x7F7F7F7Fu;
-  } else {
-    sc = m == 0 ? 1.0f : __fdiv_rn(__uint_as_float(m), 448.0f);
-    out = e4m3x4(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc), __fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc));
+  for (int j = 0; j < 4; ++j) {
+    const int64_t u = w * 8 + j * 2 + half;
+    idx[j] = -1;
+    v[j] = make_uint4(0, 0, 0, 0);
+    if (u < units) {
+      const int64_t row = u % rows, kt = u / rows;
+      idx[j] = row * k8 + kt * 16 + hl;
+      v[j] = x[idx[j]];
+    }
   }
-  q[row * k4 + kt * 32 + lane] = out;
-  if (lane == 0) s[static_cast<int64_t>(kt) * rows + row] = sc;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m = max(m, (w4[i] << 16) & 0x7FFFFFFFu);
+      m = max(m, w4[i] & 0x7FFF0000u);
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));  // within the half-warp
+    const int64_t u = w * 8 + j * 2 + half;
+    if (idx[j] < 0) continue;
+    const bool nonfinite = m >= 0x7F800000u;
+    const float sc = nonfinite ? __uint_as_float(kTwNaN) : (m == 0 ? 1.0f : __fdiv_rn(__uint_as_float(m), 448.0f));
+    uint2 o = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
+    if (!nonfinite) {
+      float f[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __fdiv_rn(bf16_bits_to_f32(w4[i] & 0xFFFFu), sc);
+        f[2 * i + 1] = __fdiv_rn(bf16_bits_to_f32(w4[i] >> 16), sc);
+      }
+      o.x = e4m3x4(f[0], f[1], f[2], f[3]);
+      o.y = e4m3x4(f[4], f[5], f[6], f[7]);
+    }
+    q[idx[j]] = o;
+    if (hl == 0) s[u] = sc;  // scales are [k/128, rows]: index kt * rows + row == u
+  }
 }
 
-__global__ void __launch_bounds__(256) tw_quant_blocks_kernel(const uint4* __restrict__ x, uint4* __restrict__ q,
+// Weights: one 256-thread CTA per 128 x 128 block; a half-warp reads one row's
+// 256 contiguous bytes per load, a warp 16 rows (8 loads per thread, all in
+// flight); block-wide amax through shared memory.
+__global__ void __launch_bounds__(256) tw_quant_blocks_kernel(const uint4* __restrict__ x, uint2* __restrict__ q,
                                                                float* __restrict__ s, int rows, int ktiles) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -70,26 +101,34 @@ __global__ void __launch_bounds__(256) tw_quant_blocks_kernel(const uint4* __res
   const int kt = blockIdx.x % ktiles;
   const int rb = blockIdx.x / ktiles;
   const int t = threadIdx.x;
-  const int r = rb * 128 + (t >> 1);   // this thread's row
-  const int half = t & 1;              // which 64 columns of the tile's 128
-  const bool valid = r < rows;
-  const int64_t k16 = static_cast<int64_t>(ktiles) * 16;  // row length in 16-byte (8-element) units
-  const int64_t base = static_cast<int64_t>(r) * k16 + kt * 16 + half * 8;
+  const int warp = t >> 5, lane = t & 31;
+  const int hl = lane & 15;
+  const int64_t k8 = static_cast<int64_t>(ktiles) * 16;  // row length in 8-element units
   uint4 v[8];
+  int64_t idx[8];
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    v[i] = valid ? x[base + i] : make_uint4(0, 0, 0, 0);
+    const int r = rb * 128 + warp * 16 + i * 2 + (lane >> 4);
+    idx[i] = -1;
+    v[i] = make_uint4(0, 0, 0, 0);
+    if (r < rows) {
+      idx[i] = static_cast<int64_t>(r) * k8 + kt * 16 + hl;
+      v[i] = x[idx[i]];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
     const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       m = max(m, (w4[j] << 16) & 0x7FFFFFFFu);
-      m = max(m, (w4[j] & 0xFFFF0000u) & 0x7FFFFFFFu);
+      m = max(m, w4[j] & 0x7FFF0000u);
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  if ((t & 31) == 0) warp_max[t >> 5] = m;
+  if (lane == 0) warp_max[warp] = m;
   __syncthreads();
   m = warp_max[0];
 #pragma unroll
@@ -97,12 +136,9 @@ __global__ void __launch_bounds__(256) tw_quant_blocks_kernel(const uint4* __res
   const bool nonfinite = m >= 0x7F800000u;
   const float sc = nonfinite ? __uint_as_float(kTwNaN) : (m == 0 ? 1.0f : __fdiv_rn(__uint_as_float(m), 448.0f));
   if (t == 0) s[static_cast<int64_t>(rb) * ktiles + kt] = sc;
-  if (!valid) return;
-  // input unit i (8 BF16, 16 bytes) becomes 8 output bytes at the same unit
-  // index of the byte tensor viewed as 8-byte units
-  uint2* q8 = reinterpret_cast<uint2*>(q);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
+    if (idx[i] < 0) continue;
     uint2 o = make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu);
     if (!nonfinite) {
       const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
@@ -115,7 +151,7 @@ __global__ void __launch_bounds__(256) tw_quant_blocks_kernel(const uint4* __res
       o.x = e4m3x4(f[0], f[1], f[2], f[3]);
       o.y = e4m3x4(f[4], f[5], f[6], f[7]);
     }
-    q8[base + i] = o;
+    q[idx[i]] = o;  // 8 elements -> 8 bytes at the same unit index
   }
 }
 
@@ -138,11 +174,11 @@ cudaError_t launch_tw_quant(const void* x, int64_t rows, int64_t k, void* q, flo
   if (rows == 0 || kt == 0) return cudaSuccess;
   cudaError_t e;
   if (!blocks) {
-    const int64_t warps = rows * static_cast<int64_t>(kt);
+    const int64_t warps = (rows * static_cast<int64_t>(kt) + 7) / 8;  // 8 tiles per warp
     const int64_t grid = (warps + 7) / 8;
     if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    const uint2* xp = static_cast<const uint2*>(x);
-    uint32_t* qp = static_cast<uint32_t*>(q);
+    const uint4* xp = static_cast<const uint4*>(x);
+    uint2* qp = static_cast<uint2*>(q);
     void* args[] = {&xp, &qp, &s, &r, &kt};
     e = launch_pdl(reinterpret_cast<const void*>(tw_quant_rows_kernel), dim3(static_cast<unsigned>(grid)), dim3(256),
                    args, stream);
@@ -150,7 +186,7 @@ cudaError_t launch_tw_quant(const void* x, int64_t rows, int64_t k, void* q, flo
     const int64_t grid = ((rows + 127) / 128) * kt;
     if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
     const uint4* xp = static_cast<const uint4*>(x);
-    uint4* qp = static_cast<uint4*>(q);
+    uint2* qp = static_cast<uint2*>(q);
     void* args[] = {&xp, &qp, &s, &r, &kt};
     e = launch_pdl(reinterpret_cast<const void*>(tw_quant_blocks_kernel), dim3(static_cast<unsigned>(grid)), dim3(256),
                    args, stream);
