@@ -599,9 +599,10 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
 // Tile configuration for one problem.  Large dense and contiguous-grouped
 // problems (at least a wave of 256-row tiles) use the CTA-pair 256x256
 // kernel; masked-grouped problems use the one-CTA persistent 128x256 kernel;
-// smaller ones first try 128x128 tiles with a double-buffered accumulator,
-// and dense problems that still leave most SMs idle split K across a cluster
-// of 2, 3, 4, 6 or 8 CTAs.
+// dense problems that fit one wave of 128x256 tiles but not of 128x128 ones
+// take the 128x256 tiles; smaller ones first try 128x128 tiles with a
+// double-buffered accumulator, and dense problems that still leave most SMs
+// idle split K across a cluster of 2, 3, 4, 6 or 8 CTAs.
 enum GemmConfig : int {
   kCfg256 = 0, kCfg128 = 1, kCfgSplit2 = 2, kCfgSplit4 = 3, kCfgSplit8 = 4, kCfgSplit3 = 5, kCfgSplit6 = 6,
   kCfgPair = 7
@@ -646,17 +647,34 @@ static int choose_config(const GemmProblem& p, int num_sms) {
     c = t256 >= num_sms ? kCfg256 : kCfg128;
   } else if (t256 >= num_sms || p.mode != kDense) {
     c = t256 >= num_sms ? kCfgPair : (t128 >= num_sms / 2 ? kCfg128 : kCfgPair);
+  } else if (t128 > num_sms && t256 <= num_sms) {
+    // one wave of 128x256 tiles instead of more than one of 128x128: the same
+    // columns per CTA, one tile's fixed cost instead of two, half the A reads
+    c = kCfg256;
   } else if (t128 >= (num_sms * 3) / 4) {
     c = kCfg128;
   } else {
-    // the largest split whose clusters all fit at once and leave no SM doubled up
+    // Split K over a cluster only where the shorter per-CTA stream pays for
+    // the exchange of partial sums through distributed shared memory.  Time
+    // model fitted to measured kernels: a CTA streams its operands at about
+    // 90 GB/s, the GPU at about 6 TB/s, and the exchange costs about 3 us.
+    // Candidates are the splits whose clusters all fit at once and leave no
+    // SM doubled up.
+    const double a_rows = p.m <= 32 ? 32.0 : p.m <= 64 ? 64.0 : static_cast<double>(BM);
+    const double per_cta = (a_rows + 128.0) * static_cast<double>(p.k);
+    const double total = static_cast<double>(p.n + p.m) * static_cast<double>(p.k);
+    auto est = [&](int sp) {
+      const double stream = per_cta / sp / 9.0e10;
+      return (stream > total / 6.0e12 ? stream : total / 6.0e12) + (sp > 1 ? 3.0e-6 : 0.0);
+    };
     c = kCfg128;
+    double best = est(1);
     const int order[5] = {kCfgSplit8, kCfgSplit6, kCfgSplit4, kCfgSplit3, kCfgSplit2};
     for (int i = 0; i < 5; ++i) {
       const int sp = split_of(order[i]);
-      if (t128 * sp <= num_sms && k_tiles >= sp && t128 <= max_clusters_of(sp)) {
+      if (t128 * sp <= num_sms && k_tiles >= sp && t128 <= max_clusters_of(sp) && est(sp) < best) {
+        best = est(sp);
         c = order[i];
-        break;
       }
     }
   }
