@@ -668,25 +668,33 @@ def run_reference(args, world, rank):
     return 0
 
 
-def kernel_source_hash():
+# the sources each kind of MXFP8 kernel is built from (a traffic figure stays
+# valid while these files are unchanged)
+KERNEL_SOURCES = {
+    "quant": ["mx_quant.cu", "mx_fastdiv.h", "mx_launch.h"],
+    "gemm": ["mx_gemm.cu", "mx_gemm2.cu", "mx_gemm_common.cuh", "mx_ptx.cuh", "mx_mxfp8.cuh", "mx_launch.h"],
+}
+
+
+def kernel_source_hash(kernel_kind: str) -> str:
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "moe_grouped_gemm_mx_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for name in KERNEL_SOURCES[kernel_kind]:
+        with open(os.path.join(ROOT, "moe_grouped_gemm_mx_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def lookup_traffic(kernel_kind: str, workload: str):
+def lookup_traffic(kernel_kind: str, workload: str, fmt: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources; otherwise None."""
+    the current sources of that kernel; otherwise None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
+    if fmt != "mxfp8" or kernel_kind not in KERNEL_SOURCES or not os.path.exists(path):
         return None
     try:
         with open(path) as f:
             tab = json.load(f)
         ent = tab.get(f"{kernel_kind}:{workload}")
-        if ent and ent.get("source_hash") == kernel_source_hash():
+        if ent and ent.get("source_hash") == kernel_source_hash(kernel_kind):
             return float(ent["dram_bytes_per_launch"])
     except (OSError, ValueError, KeyError):
         return None
@@ -833,7 +841,7 @@ def run_ours(args, world, rank, local):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
         peak_note = f"{peaks['source']} hbm copy bandwidth"
-    trf = lookup_traffic(dom, args.workload)
+    trf = lookup_traffic(dom, args.workload, args.fmt)
     roof["traffic"] = None if trf is None else trf
     roof.update({"kernel": dom, "launches_per_step": dk["launches"], "avg_launch_ms": dk["ms"] / dk["launches"],
                  "peak_source": peak_note,
