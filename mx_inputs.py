@@ -20,6 +20,9 @@ not available here):
                    down N=7168 K=2048 (fresh N(0,1) activations).
   * ``masked``     32 experts x 256 rows, masked_m[e] ~ U{0..256}; rows at or
                    beyond masked_m[e] are NaN; N=4096 K=7168.
+  * ``moe_layer``  the ``contiguous`` routing as an explicit [8192, 8] table of
+                   expert ids (same Zipf draw) with softmax gate weights over
+                   N(0,1) logits; token activations [8192, 7168] ~ N(0,1).
 
 All draws come from ``torch.Generator`` objects seeded explicitly; on a CUDA
 device the CUDA generator is used (same recipe, different stream of numbers),
@@ -106,6 +109,26 @@ def zipf_routing_counts(tokens: int = MOE_TOKENS, experts: int = MOE_EXPERTS, to
     p = (p / p.sum()).expand(tokens, experts).contiguous()
     choice = torch.multinomial(p, topk, replacement=False, generator=g)
     return torch.bincount(choice.flatten(), minlength=experts).to(torch.int64)
+
+
+def topk_ids(tokens: int = MOE_TOKENS, topk: int = MOE_TOPK, experts: int = MOE_EXPERTS, seed: int = 0,
+             s: float = MOE_ZIPF_S):
+    """Routing table int32 numpy [tokens, topk]: each token's ``topk``
+    distinct experts, drawn without replacement with p(e) proportional to
+    (e+1)^-s (the router's choice; the router itself is not modelled)."""
+    g = _gen(seed, "cpu")
+    p = torch.arange(1, experts + 1, dtype=torch.float64).pow(-s)
+    p = (p / p.sum()).expand(tokens, experts).contiguous()
+    choice = torch.multinomial(p, topk, replacement=False, generator=g)
+    return choice.to(torch.int32).numpy()
+
+
+def gate_weights(tokens: int = MOE_TOKENS, topk: int = MOE_TOPK, seed: int = 0):
+    """Gate weights float32 numpy [tokens, topk]: a softmax over N(0,1)
+    logits per token (positive, summing to 1 like a top-k router's)."""
+    g = _gen(seed + 17, "cpu")
+    logits = torch.randn(tokens, topk, generator=g, dtype=torch.float32)
+    return torch.softmax(logits, dim=1).numpy()
 
 
 def padded_offsets(counts: torch.Tensor, align: int = 128) -> torch.Tensor:

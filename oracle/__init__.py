@@ -86,6 +86,12 @@ def lib():
         L.mxo_tw_quantize_blocks.restype = None
         L.mxo_tw_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P, P]
         L.mxo_tw_gemm.restype = None
+        L.mxo_moe_route.argtypes = [P, I64, I32, I32, P, P, P]
+        L.mxo_moe_route.restype = I64
+        L.mxo_moe_dispatch.argtypes = [P, I64, I64, P, I64, I64, P, P]
+        L.mxo_moe_dispatch.restype = None
+        L.mxo_moe_combine.argtypes = [P, I64, P, P, I64, I64, P, P]
+        L.mxo_moe_combine.restype = None
         L.mxo_num_threads.argtypes = []
         L.mxo_num_threads.restype = ctypes.c_int
         _lib = L
@@ -353,6 +359,50 @@ def tw_gemm(qa, sa, qb, sb, rows=None):
     a = np.zeros((nrows, n), dtype=np.float64)
     lib().mxo_tw_gemm(_p(qa), _p(sa), _p(qb), _p(sb), m, n, k, _p(ids), nrows, _p(d), _p(a))
     return d, a
+
+
+# ---------------------------------------------------------------- MoE expert layer
+
+def moe_route(ids, num_experts: int, pad: int = 128):
+    """Routing plan of a [T, topk] expert-id table (token-major entries).
+
+    Returns (counts int32 [E], offsets int32 [E+1] padded to ``pad``, row
+    int32 [T*topk] (-1 for an id outside [0, E)), dropped entries)."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+    counts = np.zeros(num_experts, dtype=np.int32)
+    offsets = np.zeros(num_experts + 1, dtype=np.int32)
+    row = np.zeros(ids.size, dtype=np.int32)
+    bad = lib().mxo_moe_route(_p(ids), ids.size, num_experts, pad, _p(counts), _p(offsets), _p(row))
+    return counts, offsets, row, int(bad)
+
+
+def moe_dispatch(x, row, topk: int, m_rows: int):
+    """Token rows x BF16 [T, k] -> (q uint8 [m_rows, k], sf uint8 row-major
+    [m_rows, k/32]): each token's MXFP8 row at every row it is routed to,
+    zero (E4M3 0, scale code 0) elsewhere."""
+    xb = _u16(x)
+    T, k = xb.shape
+    row = np.ascontiguousarray(row, dtype=np.int32).reshape(-1)
+    assert row.size == T * topk and k % 32 == 0
+    q = np.zeros((m_rows, k), dtype=np.uint8)
+    sf = np.zeros((m_rows, k // 32), dtype=np.uint8)
+    lib().mxo_moe_dispatch(_p(xb), T, k, _p(row), topk, m_rows, _p(q), _p(sf))
+    return q, sf
+
+
+def moe_combine(y, row, w):
+    """out[t] = sum_j w[t, j] * y[row[t, j]] (fp64); y BF16 [*, n], w float32
+    [T, topk].  Returns (out, abssum) float64 [T, n]."""
+    yb = _u16(y)
+    n = yb.shape[-1]
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    T, topk = w.shape
+    row = np.ascontiguousarray(row, dtype=np.int32).reshape(-1)
+    assert row.size == T * topk
+    out = np.zeros((T, n), dtype=np.float64)
+    a = np.zeros((T, n), dtype=np.float64)
+    lib().mxo_moe_combine(_p(yb), n, _p(row), _p(w), T, topk, _p(out), _p(a))
+    return out, a
 
 
 def num_threads() -> int:

@@ -539,6 +539,105 @@ void mxo_tw_gemm(const uint8_t *qa, const float *sa, const uint8_t *qb, const fl
     }
 }
 
+/* ------------------------------------------------------------------ MoE expert layer
+ *
+ * The data movement around the grouped GEMM in a mixture-of-experts layer:
+ * the B200 MoE-training page's diagram of the MXFP8 expert layer (router
+ * output -> BF16 -> MXFP8 -> grouped GEMM -> BF16 -> all-to-all combine) and
+ * its glossary entry on all-to-all (tokens are sent to the experts that
+ * process them and the results are gathered back); the DeepGEMM release
+ * page, section 4 (the contiguous layout: each expert's tokens grouped, one
+ * group after another).  The router itself is not part of the path: ids and
+ * gate weights are inputs.
+ */
+
+/* Routing plan.  ids [n] holds the expert of each entry (t, j) of a [T, topk]
+ * routing table in token-major order (n = T*topk).  Expert e's rows are its
+ * entries in that order, starting at offsets[e]; each group is padded to a
+ * multiple of `pad` rows: offsets[e+1] = offsets[e] + ceil(counts[e]/pad)*pad.
+ * row[i] is the row of entry i, or -1 when ids[i] is outside [0, E) (such an
+ * entry is dropped).  Returns the number of dropped entries. */
+int64_t mxo_moe_route(const int32_t *ids, int64_t n, int32_t E, int32_t pad, int32_t *counts,
+                      int32_t *offsets, int32_t *row)
+{
+    int64_t bad = 0;
+    for (int32_t e = 0; e < E; ++e)
+        counts[e] = 0;
+    for (int64_t i = 0; i < n; ++i)
+        if (ids[i] >= 0 && ids[i] < E)
+            counts[ids[i]] += 1;
+    offsets[0] = 0;
+    for (int32_t e = 0; e < E; ++e)
+        offsets[e + 1] = offsets[e] + (counts[e] + pad - 1) / pad * pad;
+    int32_t *next = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+    for (int32_t e = 0; e < E; ++e)
+        next[e] = offsets[e];
+    for (int64_t i = 0; i < n; ++i) {
+        if (ids[i] >= 0 && ids[i] < E) {
+            row[i] = next[ids[i]];
+            next[ids[i]] += 1;
+        } else {
+            row[i] = -1;
+            ++bad;
+        }
+    }
+    free(next);
+    return bad;
+}
+
+/* Dispatch into the contiguous layout: the E4M3 row and scales of token t
+ * (quantised as by mxo_quantize) are written to row[t*topk + j] for every j
+ * with row >= 0.  q [m_rows, k] and sf_rm [m_rows, k/32] are first set to
+ * zero, so every row no entry maps to (the group padding) is the quantisation
+ * of a zero row: E4M3 0x00 elements, scale code 0x00. */
+void mxo_moe_dispatch(const uint16_t *x, int64_t T, int64_t k, const int32_t *row, int64_t topk,
+                      int64_t m_rows, uint8_t *q, uint8_t *sf_rm)
+{
+    int64_t kb = k / 32;
+    memset(q, 0, (size_t)(m_rows * k));
+    memset(sf_rm, 0, (size_t)(m_rows * kb));
+    uint8_t *tq = (uint8_t *)malloc((size_t)(k > 0 ? k : 1));
+    uint8_t *ts = (uint8_t *)malloc((size_t)(kb > 0 ? kb : 1));
+    for (int64_t t = 0; t < T; ++t) {
+        mxo_quantize(x + t * k, 1, k, tq, ts);
+        for (int64_t j = 0; j < topk; ++j) {
+            int32_t r = row[t * topk + j];
+            if (r < 0)
+                continue;
+            memcpy(q + (int64_t)r * k, tq, (size_t)k);
+            memcpy(sf_rm + (int64_t)r * kb, ts, (size_t)kb);
+        }
+    }
+    free(tq);
+    free(ts);
+}
+
+/* Combine: out[t, :] = sum_j w[t, j] * y[row[t*topk + j], :] in fp64, j
+ * ascending, over the entries with row >= 0; y holds BF16 bit patterns
+ * [*, n].  abssum (optional) = sum_j |w * y|, the scale of the rounding
+ * error a reduced-precision sum may make. */
+void mxo_moe_combine(const uint16_t *y, int64_t n, const int32_t *row, const float *w, int64_t T,
+                     int64_t topk, double *out, double *abssum)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t c = 0; c < n; ++c) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t j = 0; j < topk; ++j) {
+                int32_t r = row[t * topk + j];
+                if (r < 0)
+                    continue;
+                double p = (double)w[t * topk + j] * mxo_bf16_to_double(y[(int64_t)r * n + c]);
+                acc += p;
+                aacc += fabs(p);
+            }
+            out[t * n + c] = acc;
+            if (abssum)
+                abssum[t * n + c] = aacc;
+        }
+    }
+}
+
 int mxo_num_threads(void)
 {
 #ifdef _OPENMP

@@ -50,6 +50,12 @@ void mxo_tw_quantize_blocks(const uint16_t *x, int64_t rows, int64_t k, uint8_t 
 void mxo_tw_gemm(const uint8_t *qa, const float *sa, const uint8_t *qb, const float *sb, int64_t m,
                  int64_t n, int64_t k, const int64_t *row_ids, int64_t nrows, double *d,
                  double *abssum);
+int64_t mxo_moe_route(const int32_t *ids, int64_t n, int32_t E, int32_t pad, int32_t *counts,
+                      int32_t *offsets, int32_t *row);
+void mxo_moe_dispatch(const uint16_t *x, int64_t T, int64_t k, const int32_t *row, int64_t topk,
+                      int64_t m_rows, uint8_t *q, uint8_t *sf_rm);
+void mxo_moe_combine(const uint16_t *y, int64_t n, const int32_t *row, const float *w, int64_t T,
+                     int64_t topk, double *out, double *abssum);
 int mxo_num_threads(void);
 
 #ifdef __cplusplus
