@@ -65,6 +65,7 @@ typedef enum mx_status {
 #define MX_DEV_BAD_OFFSETS 0x1 /* group_offsets not monotone, not multiples of 128, or > m_total */
 #define MX_DEV_BAD_MASK 0x2    /* masked_m[e] outside [0, max_m] (clamped) */
 #define MX_DEV_TIMEOUT 0x4     /* an internal pipeline wait exceeded its limit; output invalid */
+#define MX_DEV_BAD_INDEX 0x8   /* a row index read from device memory was out of range (access skipped) */
 
 /* Human-readable name of a status code; never NULL. */
 const char *mx_status_string(int status);
@@ -279,6 +280,76 @@ mx_status mx_grouped_gemm_contiguous_tilewise(const void *qa, const float *sa, c
                                               const int32_t *group_offsets, int32_t groups, int64_t m_total,
                                               int64_t n, int64_t k, void *d_bf16, int32_t *dev_status,
                                               mx_stream_t stream);
+
+/* ------------------------------------------------------------------ MoE expert layer
+ *
+ * The data movement around the grouped GEMM in a mixture-of-experts layer:
+ * the B200 MoE-training page's MXFP8 expert layer (router output -> BF16 ->
+ * MXFP8 -> grouped GEMM -> BF16 -> all-to-all combine; glossary entry on
+ * all-to-all: tokens are sent to their experts and the results gathered
+ * back) and DeepGEMM's contiguous layout (release page, section 4).  The
+ * router is not part of the path: expert ids and gate weights are inputs.
+ * For expert parallelism the same calls build and unpack the all-to-all
+ * buffers (route with pad = 1 orders entries by expert, i.e. by the rank that
+ * owns the expert).
+ */
+
+/* Upper bound of the rows a routing plan of n entries over `experts` groups
+ * padded to `pad` occupies, rounded up to a multiple of 128 (the scale-tile
+ * height): allocate the grouped operand with this many rows. */
+int64_t mx_moe_max_rows(int64_t n, int32_t experts, int32_t pad);
+
+/* Routing plan of a [tokens, topk] expert-id table (n = tokens*topk int32
+ * entries, token-major, device).  Expert e's rows are its entries in entry
+ * order starting at offsets[e]; every group is padded to a multiple of `pad`
+ * rows: offsets[e+1] = offsets[e] + ceil(counts[e]/pad)*pad.  Outputs
+ * (device, caller-owned): counts int32 [experts], offsets int32 [experts+1],
+ * row int32 [n] (the entry's row; -1 for an id outside [0, experts), which is
+ * dropped), dropped int32 [1] (nullable: the number of dropped entries).
+ * One CTA; 1 <= experts <= 1024, 1 <= pad <= 128, n < 2^31 - 1024. */
+mx_status mx_moe_route(const int32_t *ids, int64_t n, int32_t experts, int32_t pad, int32_t *counts,
+                       int32_t *offsets, int32_t *row, int32_t *dropped, mx_stream_t stream);
+
+/* Dispatch: each token row of x_bf16 [tokens, k] is quantised to MXFP8 once
+ * (the rule of mx_quantize_bf16_to_e4m3, bit for bit) and written to row
+ * row[t*topk + j] of q_e4m3 [m_rows, k] for every j with row >= 0; its k/32
+ * scale bytes go to the same row of sf: the tiled layout over m_rows rows
+ * (mx_scale_bytes(m_rows, k) bytes; the GEMM operand) when sf_row_major == 0,
+ * else row-major [m_rows, k/32] (an all-to-all send buffer).  When pad > 1 the
+ * padding rows of every group ([offsets[e] + counts[e], offsets[e+1]), from
+ * mx_moe_route with the same pad) are set to the quantisation of a zero row
+ * (E4M3 0x00, scale 0x00).  k % 128 == 0; m_rows % 128 == 0 for the tiled
+ * layout; 16-byte aligned x, q and sf.  A row >= m_rows is skipped and sets
+ * MX_DEV_BAD_INDEX. */
+mx_status mx_moe_dispatch_quant(const void *x_bf16, int64_t tokens, int64_t k, const int32_t *row, int32_t topk,
+                                const int32_t *counts, const int32_t *offsets, int32_t experts, int32_t pad,
+                                int64_t m_rows, void *q_e4m3, void *sf, int32_t sf_row_major,
+                                int32_t *dev_status, mx_stream_t stream);
+
+/* Scatter of already quantised rows (an all-to-all receive buffer): row i of
+ * q_src [n_src, k] with its row-major scales sf_src [n_src, k/32] goes to row
+ * dst_row[i] of q_dst [m_rows, k] / the tiled scales sf_dst (mx_scale_bytes(
+ * m_rows, k) bytes); padding rows of the plan (counts, offsets, pad) are
+ * cleared as in mx_moe_dispatch_quant.  Same shape, alignment and index rules. */
+mx_status mx_moe_scatter_rows(const void *q_src, const void *sf_src, int64_t n_src, int64_t k,
+                              const int32_t *dst_row, const int32_t *counts, const int32_t *offsets,
+                              int32_t experts, int32_t pad, int64_t m_rows, void *q_dst, void *sf_dst,
+                              int32_t *dev_status, mx_stream_t stream);
+
+/* Row gather: dst[i] = src[idx[i]] for i < n, rows of row_bytes bytes
+ * (row_bytes % 16 == 0, 16-byte aligned src and dst); an index outside
+ * [0, src_rows) gives a zero row and sets MX_DEV_BAD_INDEX. */
+mx_status mx_gather_rows(const void *src, int64_t src_rows, int64_t row_bytes, const int32_t *idx, int64_t n,
+                         void *dst, int32_t *dev_status, mx_stream_t stream);
+
+/* Combine: out[t, :] = sum_j w[t, j] * y[row[t*topk + j], :] for t < tokens,
+ * over the entries with row >= 0, FP32 fused multiply-adds in j order and one
+ * rounding to BF16 (RNE).  y_bf16 [y_rows, n_cols], w float32 [tokens, topk],
+ * row int32 [tokens*topk], out_bf16 [tokens, n_cols]; n_cols % 8 == 0,
+ * 16-byte aligned y and out, 1 <= topk <= 64.  A row >= y_rows is skipped and
+ * sets MX_DEV_BAD_INDEX. */
+mx_status mx_moe_combine(const void *y_bf16, int64_t y_rows, int64_t n_cols, const int32_t *row, const float *w,
+                         int64_t tokens, int32_t topk, void *out_bf16, int32_t *dev_status, mx_stream_t stream);
 
 /* Copies the library-internal device status word (used when a call got
  * dev_status == NULL) to *host_out and, if clear != 0, resets it.

@@ -28,7 +28,10 @@ __all__ = [
     "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant",
     "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped", "mx_quantize_bf16_to_e4m3_tile1x128",
     "mx_quantize_bf16_to_e4m3_block128x128", "mx_gemm_tilewise", "mx_grouped_gemm_contiguous_tilewise",
-    "read_internal_status", "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "C_SYMBOLS",
+    "mx_moe_max_rows", "mx_moe_route", "mx_moe_dispatch_quant", "mx_moe_scatter_rows", "mx_gather_rows",
+    "mx_moe_combine",
+    "read_internal_status", "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "MX_DEV_BAD_INDEX",
+    "C_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,6 +40,7 @@ lib_path = os.path.join(_HERE, "libmx.so")
 MX_DEV_BAD_OFFSETS = 0x1
 MX_DEV_BAD_MASK = 0x2
 MX_DEV_TIMEOUT = 0x4
+MX_DEV_BAD_INDEX = 0x8
 
 # every symbol include/mx.h declares
 C_SYMBOLS = [
@@ -47,6 +51,8 @@ C_SYMBOLS = [
     "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant",
     "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped", "mx_quantize_bf16_to_e4m3_tile1x128",
     "mx_quantize_bf16_to_e4m3_block128x128", "mx_gemm_tilewise", "mx_grouped_gemm_contiguous_tilewise",
+    "mx_moe_max_rows", "mx_moe_route", "mx_moe_dispatch_quant", "mx_moe_scatter_rows", "mx_gather_rows",
+    "mx_moe_combine",
 ]
 
 
@@ -102,6 +108,18 @@ def _load():
     L.mx_gemm_tilewise.restype = ctypes.c_int
     L.mx_grouped_gemm_contiguous_tilewise.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_contiguous_tilewise.restype = ctypes.c_int
+    L.mx_moe_max_rows.argtypes = [I64, I32, I32]
+    L.mx_moe_max_rows.restype = I64
+    L.mx_moe_route.argtypes = [P, I64, I32, I32, P, P, P, P, P]
+    L.mx_moe_route.restype = ctypes.c_int
+    L.mx_moe_dispatch_quant.argtypes = [P, I64, I64, P, I32, P, P, I32, I32, I64, P, P, I32, P, P]
+    L.mx_moe_dispatch_quant.restype = ctypes.c_int
+    L.mx_moe_scatter_rows.argtypes = [P, P, I64, I64, P, P, P, I32, I32, I64, P, P, P, P]
+    L.mx_moe_scatter_rows.restype = ctypes.c_int
+    L.mx_gather_rows.argtypes = [P, I64, I64, P, I64, P, P, P]
+    L.mx_gather_rows.restype = ctypes.c_int
+    L.mx_moe_combine.argtypes = [P, I64, I64, P, P, I64, I32, P, P, P]
+    L.mx_moe_combine.restype = ctypes.c_int
     L.mx_read_internal_status.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
     L.mx_read_internal_status.restype = ctypes.c_int
     return L
@@ -457,6 +475,128 @@ def mx_grouped_gemm_masked_swiglu_quant(qa, sfa, qb, sfb, masked_m: torch.Tensor
                                                   _status_arg(dev_status), _stream(stream))
     _raise(st, "mx_grouped_gemm_masked_swiglu_quant")
     return qh, sfh
+
+
+# ---------------------------------------------------------------- MoE expert layer
+
+def mx_moe_max_rows(n: int, experts: int, pad: int) -> int:
+    """Rows to allocate for the grouped operand of a routing plan of ``n``
+    entries (every group padded to ``pad``), rounded up to 128."""
+    return int(_lib.mx_moe_max_rows(n, experts, pad))
+
+
+def mx_moe_route(ids: torch.Tensor, experts: int, pad: int = 128, counts=None, offsets=None, row=None,
+                 dropped=None, stream=None):
+    """Routing plan of an int32 expert-id table ([tokens, topk] or flat,
+    token-major).  Returns (counts [E], offsets [E+1], row [n], dropped [1]),
+    int32 device tensors: expert e's rows are its entries in entry order from
+    offsets[e], groups padded to ``pad`` rows; row = -1 for an id outside
+    [0, experts)."""
+    _check(ids, torch.int32, "ids")
+    n = ids.numel()
+    dev = ids.device
+    counts = torch.empty(experts, dtype=torch.int32, device=dev) if counts is None else counts
+    offsets = torch.empty(experts + 1, dtype=torch.int32, device=dev) if offsets is None else offsets
+    row = torch.empty(n, dtype=torch.int32, device=dev) if row is None else row
+    dropped = torch.empty(1, dtype=torch.int32, device=dev) if dropped is None else dropped
+    for t, nm, size in ((counts, "counts", experts), (offsets, "offsets", experts + 1), (row, "row", n),
+                        (dropped, "dropped", 1)):
+        _check(t, torch.int32, nm)
+        if t.numel() < size:
+            raise ValueError(f"{nm} too small")
+    _raise(_lib.mx_moe_route(_ptr(ids), n, experts, pad, _ptr(counts), _ptr(offsets), _ptr(row), _ptr(dropped),
+                             _stream(stream)), "mx_moe_route")
+    return counts, offsets, row, dropped
+
+
+def mx_moe_dispatch_quant(x: torch.Tensor, row: torch.Tensor, topk: int, counts: torch.Tensor,
+                          offsets: torch.Tensor, pad: int, m_rows: int, q=None, sf=None, sf_row_major=False,
+                          dev_status=None, stream=None):
+    """Quantise each token of x (BF16 [tokens, K]) once and write its MXFP8
+    row at every row it is routed to (``row`` from mx_moe_route).  Returns
+    (q uint8 [m_rows, K], sf): sf tiled (the GEMM operand) or row-major
+    [m_rows, K/32].  Group padding rows (pad > 1) are zero rows."""
+    _check(x, torch.bfloat16, "x")
+    _check(row, torch.int32, "row")
+    tokens, k = x.shape
+    if row.numel() != tokens * topk:
+        raise ValueError("row must hold tokens*topk entries")
+    experts = counts.numel() if counts is not None else 0
+    if counts is not None:
+        _check(counts, torch.int32, "counts")
+        _check(offsets, torch.int32, "offsets")
+    sf_bytes = m_rows * (k // 32) if sf_row_major else scale_bytes(m_rows, k)
+    q = torch.empty((m_rows, k), dtype=torch.uint8, device=x.device) if q is None else q
+    sf = torch.empty(sf_bytes, dtype=torch.uint8, device=x.device) if sf is None else sf
+    _check(q, torch.uint8, "q")
+    _check(sf, torch.uint8, "sf")
+    if q.numel() < m_rows * k or sf.numel() < sf_bytes:
+        raise ValueError("output buffers too small")
+    _raise(_lib.mx_moe_dispatch_quant(_ptr(x), tokens, k, _ptr(row), topk, _ptr(counts), _ptr(offsets), experts,
+                                      pad, m_rows, _ptr(q), _ptr(sf), 1 if sf_row_major else 0, _ptr(dev_status),
+                                      _stream(stream)), "mx_moe_dispatch_quant")
+    return q, sf
+
+
+def mx_moe_scatter_rows(q_src: torch.Tensor, sf_src: torch.Tensor, dst_row: torch.Tensor, counts: torch.Tensor,
+                        offsets: torch.Tensor, pad: int, m_rows: int, q=None, sf=None, dev_status=None,
+                        stream=None):
+    """Place quantised rows (q_src uint8 [n, K], row-major scales sf_src
+    [n, K/32]) at dst_row of a grouped operand (q [m_rows, K], tiled sf),
+    clearing the group padding rows.  Returns (q, sf)."""
+    _check(q_src, torch.uint8, "q_src")
+    _check(sf_src, torch.uint8, "sf_src")
+    _check(dst_row, torch.int32, "dst_row")
+    n, k = q_src.shape
+    if dst_row.numel() != n or sf_src.numel() < n * (k // 32):
+        raise ValueError("dst_row / sf_src do not match q_src")
+    _check(counts, torch.int32, "counts")
+    _check(offsets, torch.int32, "offsets")
+    q = torch.empty((m_rows, k), dtype=torch.uint8, device=q_src.device) if q is None else q
+    sf = torch.empty(scale_bytes(m_rows, k), dtype=torch.uint8, device=q_src.device) if sf is None else sf
+    _check(q, torch.uint8, "q")
+    _check(sf, torch.uint8, "sf")
+    if q.numel() < m_rows * k or sf.numel() < scale_bytes(m_rows, k):
+        raise ValueError("output buffers too small")
+    _raise(_lib.mx_moe_scatter_rows(_ptr(q_src), _ptr(sf_src), n, k, _ptr(dst_row), _ptr(counts), _ptr(offsets),
+                                    counts.numel(), pad, m_rows, _ptr(q), _ptr(sf), _ptr(dev_status),
+                                    _stream(stream)), "mx_moe_scatter_rows")
+    return q, sf
+
+
+def mx_gather_rows(src: torch.Tensor, idx: torch.Tensor, out=None, dev_status=None, stream=None):
+    """out[i] = src[idx[i]] for the rows of a 2-D contiguous tensor (row size a
+    multiple of 16 bytes); an out-of-range index gives a zero row."""
+    if src.dim() != 2 or not src.is_contiguous() or src.device.type != "cuda":
+        raise ValueError("src must be a contiguous 2-D CUDA tensor")
+    _check(idx, torch.int32, "idx")
+    n = idx.numel()
+    out = torch.empty((n, src.shape[1]), dtype=src.dtype, device=src.device) if out is None else out
+    if out.dtype != src.dtype or not out.is_contiguous() or out.shape[1:] != src.shape[1:] or out.shape[0] < n:
+        raise ValueError("out does not match src")
+    row_bytes = src.shape[1] * src.element_size()
+    _raise(_lib.mx_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(idx), n, _ptr(out), _ptr(dev_status),
+                               _stream(stream)), "mx_gather_rows")
+    return out
+
+
+def mx_moe_combine(y: torch.Tensor, row: torch.Tensor, w: torch.Tensor, out=None, dev_status=None, stream=None):
+    """out[t] = sum_j w[t, j] * y[row[t, j]] (FP32 in j order, BF16 out);
+    y BF16 [rows, N], w float32 [tokens, topk], row int32 [tokens*topk]."""
+    _check(y, torch.bfloat16, "y")
+    _check(w, torch.float32, "w")
+    _check(row, torch.int32, "row")
+    tokens, topk = w.shape
+    if row.numel() != tokens * topk:
+        raise ValueError("row must hold tokens*topk entries")
+    n = y.shape[1]
+    out = torch.empty((tokens, n), dtype=torch.bfloat16, device=y.device) if out is None else out
+    _check(out, torch.bfloat16, "out")
+    if out.numel() < tokens * n:
+        raise ValueError("out too small")
+    _raise(_lib.mx_moe_combine(_ptr(y), y.shape[0], n, _ptr(row), _ptr(w), tokens, topk, _ptr(out),
+                               _ptr(dev_status), _stream(stream)), "mx_moe_combine")
+    return out
 
 
 def read_internal_status(clear: bool = True) -> int:

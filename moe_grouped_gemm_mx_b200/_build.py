@@ -21,7 +21,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmx.so")
 SOURCES = ["mx_api.cu", "mx_gemm.cu", "mx_gemm2.cu", "mx_quant.cu", "mx_quant_t.cu", "mx_quant_tw.cu",
-           "mx_gemm_tw.cu"]
+           "mx_gemm_tw.cu", "mx_moe.cu"]
 HEADERS = ["mx_ptx.cuh", "mx_launch.h", "mx_fastdiv.h", "mx_gemm_common.cuh", "mx_mxfp8.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -361,6 +361,124 @@ mx_status mx_grouped_gemm_masked_swiglu_quant(const void* qa, const void* sfa, c
   return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
 }
 
+int64_t mx_moe_max_rows(int64_t n, int32_t experts, int32_t pad) {
+  if (n < 0 || experts <= 0 || pad <= 0) return 0;
+  const int64_t rows = n + static_cast<int64_t>(experts) * (pad - 1);
+  return (rows + 127) / 128 * 128;
+}
+
+mx_status mx_moe_route(const int32_t* ids, int64_t n, int32_t experts, int32_t pad, int32_t* counts,
+                       int32_t* offsets, int32_t* row, int32_t* dropped, mx_stream_t stream) {
+  if (n < 0 || experts < 1 || experts > kMaxGroups || pad < 1 || pad > 128) return MX_ERR_INVALID_ARGUMENT;
+  if (n > kMaxDim - 1024) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (!counts || !offsets || (n > 0 && (!ids || !row))) return MX_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(ids) | reinterpret_cast<uintptr_t>(counts) | reinterpret_cast<uintptr_t>(offsets) |
+       reinterpret_cast<uintptr_t>(row) | reinterpret_cast<uintptr_t>(dropped)) & 3u)
+    return MX_ERR_MISALIGNED;
+  return from_cuda(mxk::launch_moe_route(ids, n, experts, pad, counts, offsets, row, dropped,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+static mx_status check_place(const void* src, int64_t n_src, int64_t k, const int32_t* row, int32_t fan,
+                             const int32_t* counts, const int32_t* offsets, int32_t experts, int32_t pad,
+                             int64_t m_rows, const void* q, const void* sf, bool tiled) {
+  if (n_src < 0 || k < 0 || m_rows < 0 || fan < 1 || fan > 64 || pad < 1 || pad > 128 || experts < 0 ||
+      experts > kMaxGroups)
+    return MX_ERR_INVALID_ARGUMENT;
+  if (k % 128 != 0 || (tiled && m_rows % 128 != 0)) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (k > kMaxDim || m_rows > kMaxDim || n_src > kMaxDim || n_src * static_cast<int64_t>(fan) > kMaxDim)
+    return MX_ERR_UNSUPPORTED_SHAPE;
+  if (pad > 1 && experts > 0 && (!counts || !offsets)) return MX_ERR_INVALID_ARGUMENT;
+  if (k == 0 || (n_src == 0 && (pad == 1 || experts == 0))) return MX_OK;
+  if (!q || !sf || (n_src > 0 && (!src || !row))) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(src) || !aligned16(q) || !aligned16(sf)) return MX_ERR_MISALIGNED;
+  return MX_OK;
+}
+
+mx_status mx_moe_dispatch_quant(const void* x_bf16, int64_t tokens, int64_t k, const int32_t* row, int32_t topk,
+                                const int32_t* counts, const int32_t* offsets, int32_t experts, int32_t pad,
+                                int64_t m_rows, void* q_e4m3, void* sf, int32_t sf_row_major,
+                                int32_t* dev_status, mx_stream_t stream) {
+  mx_status st = check_place(x_bf16, tokens, k, row, topk, counts, offsets, experts, pad, m_rows, q_e4m3, sf,
+                             sf_row_major == 0);
+  if (st != MX_OK) return st;
+  if (k == 0 || (tokens == 0 && (pad == 1 || experts == 0))) return MX_OK;
+  mxk::MoePlace p = {};
+  p.src = x_bf16;
+  p.row = row;
+  p.counts = counts;
+  p.offsets = offsets;
+  p.q = q_e4m3;
+  p.sf = sf;
+  p.status = dev_status ? dev_status : internal_status_ptr();
+  p.n_src = tokens;
+  p.m_rows = m_rows;
+  p.k = k;
+  p.fan = topk;
+  p.experts = experts;
+  p.pad = pad;
+  p.sf_row_major = sf_row_major != 0;
+  p.quantize = true;
+  return from_cuda(mxk::launch_moe_place(p, static_cast<cudaStream_t>(stream)));
+}
+
+mx_status mx_moe_scatter_rows(const void* q_src, const void* sf_src, int64_t n_src, int64_t k,
+                              const int32_t* dst_row, const int32_t* counts, const int32_t* offsets,
+                              int32_t experts, int32_t pad, int64_t m_rows, void* q_dst, void* sf_dst,
+                              int32_t* dev_status, mx_stream_t stream) {
+  mx_status st = check_place(q_src, n_src, k, dst_row, 1, counts, offsets, experts, pad, m_rows, q_dst, sf_dst, true);
+  if (st != MX_OK) return st;
+  if (k == 0 || (n_src == 0 && (pad == 1 || experts == 0))) return MX_OK;
+  if (n_src > 0 && !sf_src) return MX_ERR_INVALID_ARGUMENT;
+  mxk::MoePlace p = {};
+  p.src = q_src;
+  p.src_sf = sf_src;
+  p.row = dst_row;
+  p.counts = counts;
+  p.offsets = offsets;
+  p.q = q_dst;
+  p.sf = sf_dst;
+  p.status = dev_status ? dev_status : internal_status_ptr();
+  p.n_src = n_src;
+  p.m_rows = m_rows;
+  p.k = k;
+  p.fan = 1;
+  p.experts = experts;
+  p.pad = pad;
+  p.sf_row_major = 0;
+  p.quantize = false;
+  return from_cuda(mxk::launch_moe_place(p, static_cast<cudaStream_t>(stream)));
+}
+
+mx_status mx_gather_rows(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* idx, int64_t n,
+                         void* dst, int32_t* dev_status, mx_stream_t stream) {
+  if (src_rows < 0 || row_bytes < 0 || n < 0) return MX_ERR_INVALID_ARGUMENT;
+  if (row_bytes % 16 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (n > kMaxDim || src_rows > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0 || row_bytes == 0) return MX_OK;
+  if (!idx || !dst || (src_rows > 0 && !src)) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(src) || !aligned16(dst)) return MX_ERR_MISALIGNED;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  return from_cuda(mxk::launch_moe_gather(src, src_rows, row_bytes, idx, n, dst, status,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+mx_status mx_moe_combine(const void* y_bf16, int64_t y_rows, int64_t n_cols, const int32_t* row, const float* w,
+                         int64_t tokens, int32_t topk, void* out_bf16, int32_t* dev_status, mx_stream_t stream) {
+  if (y_rows < 0 || n_cols < 0 || tokens < 0 || topk < 1 || topk > 64) return MX_ERR_INVALID_ARGUMENT;
+  if (n_cols % 8 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (tokens > kMaxDim || y_rows > kMaxDim || tokens * static_cast<int64_t>(topk) > kMaxDim)
+    return MX_ERR_UNSUPPORTED_SHAPE;
+  if (tokens == 0 || n_cols == 0) return MX_OK;
+  if (!row || !w || !out_bf16 || (y_rows > 0 && !y_bf16)) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(y_bf16) || !aligned16(out_bf16) || (reinterpret_cast<uintptr_t>(w) & 3u) ||
+      (reinterpret_cast<uintptr_t>(row) & 3u))
+    return MX_ERR_MISALIGNED;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  return from_cuda(mxk::launch_moe_combine(y_bf16, y_rows, n_cols, row, w, tokens, topk, out_bf16, status,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 mx_status mx_read_internal_status(int32_t* host_out, int clear) {
   if (!host_out) return MX_ERR_INVALID_ARGUMENT;
   if (cudaDeviceSynchronize() != cudaSuccess) return MX_ERR_CUDA;

@@ -67,4 +67,27 @@ struct TwProblem {
 
 cudaError_t launch_gemm_tw(const TwProblem& p, int num_sms, cudaStream_t stream);
 
+// MoE expert-layer data movement (mx_moe.cu).
+cudaError_t launch_moe_route(const int32_t* ids, int64_t n, int E, int pad, int32_t* counts, int32_t* offsets,
+                             int32_t* row, int32_t* dropped, cudaStream_t stream);
+
+struct MoePlace {
+  const void* src;          // quantize: BF16 [n_src, k]; else E4M3 [n_src, k]
+  const void* src_sf;       // !quantize: row-major scales [n_src, k/32]
+  const int32_t* row;       // [n_src * fan] destination rows (-1: none)
+  const int32_t* counts;    // [experts]
+  const int32_t* offsets;   // [experts + 1]
+  void* q;                  // [m_rows, k]
+  void* sf;                 // tiled over m_rows, or row-major [m_rows, k/32]
+  int32_t* status;
+  int64_t n_src, m_rows, k;
+  int fan, experts, pad, sf_row_major;
+  bool quantize;
+};
+cudaError_t launch_moe_place(const MoePlace& p, cudaStream_t stream);
+cudaError_t launch_moe_gather(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* idx, int64_t n,
+                              void* dst, int32_t* status, cudaStream_t stream);
+cudaError_t launch_moe_combine(const void* y, int64_t y_rows, int64_t n_cols, const int32_t* row, const float* w,
+                               int64_t tokens, int topk, void* out, int32_t* status, cudaStream_t stream);
+
 }  // namespace mxk

@@ -1,0 +1,385 @@
+// mx_moe.cu -- the data movement around the grouped GEMM of a mixture-of-
+// experts expert layer, on sm_100a: the routing plan, the dispatch (each
+// token quantised to MXFP8 once and its row placed at every expert row it is
+// routed to, in the contiguous grouped layout), the row scatter / gather of
+// the all-to-all buffers of expert parallelism, and the gate-weighted combine.
+//
+// Sources: the B200 MoE-training page (the diagram of the MXFP8 expert layer:
+// router output -> BF16 -> MXFP8 -> grouped GEMM -> BF16 -> all-to-all
+// combine; the glossary entry on all-to-all: tokens go to the experts that
+// process them and the results are gathered back; the DeepEP section) and the
+// DeepGEMM release page, section 4 (the contiguous layout: each expert's
+// tokens grouped, one group after another, each group padded to the GEMM's
+// 128-row tile).
+//
+// Everything here is HBM-bound data movement; each kernel reads and writes
+// every byte once.  Indices that come from device memory (rows, ids) are
+// checked before any access: a bad one skips the access and sets a bit of the
+// caller's status word.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "mx_launch.h"
+#include "mx_mxfp8.cuh"
+
+namespace mxk {
+
+constexpr int kRouteThreads = 1024;
+constexpr int kRowWarps = 8;  // warps per CTA of the row kernels (one row per warp)
+constexpr int kDevBadIndex = 0x8;
+
+__device__ __forceinline__ void moe_report(int32_t* status, int bits) { atomicOr(status, bits); }
+
+// ------------------------------------------------------------------ routing plan
+// One CTA of 1024 threads: the plan is a prefix over all entries, and the
+// table (8192 tokens x top-8 = 64K entries) is tiny next to the GEMMs it
+// feeds.  Phase 1: per-expert histogram in shared memory.  Phase 2: exclusive
+// scan of the padded group sizes (one expert per thread, E <= 1024).
+// Phase 3: stable ranks, 1024 entries per step in entry order: within a warp
+// by __match_any_sync and the population count of the lower lanes, across
+// the warps of a step through a byte table of per-warp counts per expert,
+// across steps by a running next row per expert.
+__global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t* __restrict__ ids, int n, int E,
+                                                                  int pad, int32_t* __restrict__ counts,
+                                                                  int32_t* __restrict__ offsets,
+                                                                  int32_t* __restrict__ row,
+                                                                  int32_t* __restrict__ dropped) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  extern __shared__ int32_t route_smem[];
+  int32_t* hist = route_smem;       // [E]
+  int32_t* next = hist + E;         // [E] next row of each expert
+  int32_t* wsum = next + E;         // [32] warp totals of the scan
+  int32_t* nbad = wsum + 32;        // [1]
+  uint8_t* wcnt = reinterpret_cast<uint8_t*>(nbad + 1);  // [E][32] entries per warp in the current step
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
+  for (int i = tid; i < E * 32; i += blockDim.x) wcnt[i] = 0;
+  if (tid == 0) *nbad = 0;
+  __syncthreads();
+
+  int bad = 0;
+  for (int i = tid; i < n; i += blockDim.x) {
+    const int e = ids[i];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    else ++bad;
+  }
+  if (bad) atomicAdd(nbad, bad);
+  __syncthreads();
+
+  const int v = tid < E ? (hist[tid] + pad - 1) / pad * pad : 0;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = wsum[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    wsum[lane] = wi - w;
+  }
+  __syncthreads();
+  const int excl = incl - v + wsum[warp];
+  if (tid < E) {
+    counts[tid] = hist[tid];
+    offsets[tid] = excl;
+    next[tid] = excl;
+    if (tid == E - 1) offsets[E] = excl + v;
+  }
+  if (tid == 0 && dropped != nullptr) *dropped = *nbad;
+  __syncthreads();
+
+  const uint32_t lower = (1u << lane) - 1u;
+  for (int c0 = 0; c0 < n; c0 += blockDim.x) {
+    const int i = c0 + tid;
+    int e = -1;
+    if (i < n) {
+      e = ids[i];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+    const bool leader = (peers & lower) == 0;
+    if (e >= 0 && leader) wcnt[e * 32 + warp] = static_cast<uint8_t>(__popc(peers));
+    __syncthreads();
+    if (e >= 0) {
+      int pre = 0;
+      const uint8_t* wc = wcnt + e * 32;
+      for (int w = 0; w < warp; ++w) pre += wc[w];
+      row[i] = next[e] + pre + __popc(peers & lower);
+    } else if (i < n) {
+      row[i] = -1;
+    }
+    __syncthreads();
+    if (e >= 0 && leader) {
+      atomicAdd(&next[e], __popc(peers));
+      wcnt[e * 32 + warp] = 0;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ dispatch / scatter
+struct PlaceArgs {
+  const void* src;          // QUANT: BF16 tokens [n_src, k]; else E4M3 rows [n_src, k]
+  const uint8_t* src_sf;    // !QUANT: row-major scales [n_src, k/32]
+  const int32_t* row;       // destination rows [n_src * fan]
+  const int32_t* counts;    // [E] real rows per group (padding clearing)
+  const int32_t* offsets;   // [E+1] padded group starts
+  uint8_t* q;               // E4M3 rows [m_rows, k]
+  uint8_t* sf;              // scales of q: tiled, or row-major [m_rows, k/32]
+  int32_t* status;
+  int64_t n_src;
+  int64_t m_rows;
+  int k;
+  int fan;                  // destination rows per source row (top-k for the dispatch, 1 for a scatter)
+  int E;                    // groups whose padding rows are cleared (0: none)
+  int pad_slots;            // padding rows per group at most (pad - 1)
+  int sf_row_major;
+};
+
+// Scale word of blocks c..c+3 (c % 4 == 0) of row r.
+__device__ __forceinline__ uint32_t* scale_word(const PlaceArgs& a, int64_t r, uint32_t c, uint32_t kb) {
+  const int64_t off = a.sf_row_major ? r * kb + c : static_cast<int64_t>(sf_tiled_offset(static_cast<uint32_t>(r), c, kb / 4));
+  return reinterpret_cast<uint32_t*>(a.sf + off);
+}
+
+// One warp per source row (QUANT: quantise the BF16 token's 32-element
+// blocks, one per lane, with the quantiser's rule; else copy E4M3 row and
+// scales), the row then written to each of its `fan` destinations; the warps
+// after the last source row clear the group padding rows (E4M3 0, scale 0:
+// the quantisation of a zero row).
+template <bool QUANT>
+__global__ void __launch_bounds__(kRowWarps * 32) moe_place_kernel(const PlaceArgs a) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  const uint32_t kb = static_cast<uint32_t>(a.k / 32);
+  if (w < a.n_src) {
+    for (uint32_t b0 = 0; b0 < kb; b0 += 32) {
+      const uint32_t b = b0 + lane;
+      const bool on = b < kb;  // kb % 4 == 0: each group of 4 lanes is all on or all off
+      uint4 out0 = make_uint4(0, 0, 0, 0), out1 = out0;
+      uint32_t scode = 0;
+      if (QUANT) {
+        uint4 v[4];
+        const uint4* src = static_cast<const uint4*>(a.src) + (w * kb + b) * 4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = on ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
+        scode = quant_block32_bf16(v, out0, out1);
+      } else if (on) {
+        const uint4* src = static_cast<const uint4*>(a.src) + (w * kb + b) * 2;
+        out0 = __ldcs(src);
+        out1 = __ldcs(src + 1);
+        scode = a.src_sf[w * kb + b];
+      }
+      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, scode, 1);
+      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, scode, 2);
+      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, scode, 3);
+      const uint32_t word = scode | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      for (int j = 0; j < a.fan; ++j) {
+        const int32_t r = a.row[w * a.fan + j];
+        if (r < 0) continue;  // a dropped entry
+        if (r >= a.m_rows) {
+          if (lane == 0 && b0 == 0) moe_report(a.status, kDevBadIndex);
+          continue;
+        }
+        if (on) {
+          uint4* dst = reinterpret_cast<uint4*>(a.q) + (static_cast<int64_t>(r) * kb + b) * 2;
+          dst[0] = out0;
+          dst[1] = out1;
+          if ((lane & 3) == 0) *scale_word(a, r, b, kb) = word;
+        }
+      }
+    }
+    return;
+  }
+  // padding rows
+  if (a.E == 0 || a.pad_slots == 0) return;
+  const int64_t p = w - a.n_src;
+  const int e = static_cast<int>(p / a.pad_slots);
+  if (e >= a.E) return;
+  const int s = static_cast<int>(p - static_cast<int64_t>(e) * a.pad_slots);
+  const int64_t r = static_cast<int64_t>(a.offsets[e]) + a.counts[e] + s;
+  if (r >= a.offsets[e + 1]) return;
+  if (r < 0 || r >= a.m_rows) {
+    if (lane == 0) moe_report(a.status, kDevBadIndex);
+    return;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(a.q + r * a.k);
+  for (int i = lane; i < a.k / 16; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+  for (uint32_t c = 4 * lane; c < kb; c += 128) *scale_word(a, r, c, kb) = 0;
+}
+
+// ------------------------------------------------------------------ row gather
+// dst[i] = src[idx[i]] for rows of `row_vecs` 16-byte vectors; an index
+// outside [0, src_rows) gives a zero row and the status bit.  One warp per row.
+__global__ void __launch_bounds__(kRowWarps * 32) moe_gather_kernel(const uint4* __restrict__ src, int64_t src_rows,
+                                                                    int64_t row_vecs, const int32_t* __restrict__ idx,
+                                                                    int64_t n, uint4* __restrict__ dst,
+                                                                    int32_t* status) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (i >= n) return;
+  const int32_t r = idx[i];
+  uint4* d = dst + i * row_vecs;
+  if (r < 0 || r >= src_rows) {
+    if (lane == 0) moe_report(status, kDevBadIndex);
+    for (int64_t c = lane; c < row_vecs; c += 32) d[c] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const uint4* s = src + static_cast<int64_t>(r) * row_vecs;
+  for (int64_t c = lane; c < row_vecs; c += 32) d[c] = __ldcs(s + c);
+}
+
+// ------------------------------------------------------------------ combine
+// out[t, :] = sum_j w[t, j] * y[row[t*topk + j], :], FP32 fused multiply-adds
+// in j order, rounded once to BF16 (RNE).  One warp per token, 8 columns (one
+// 16-byte vector) per lane per step, four routed rows' loads in flight.
+__global__ void __launch_bounds__(kRowWarps * 32) moe_combine_kernel(const uint4* __restrict__ y, int64_t y_rows,
+                                                                     int64_t n_vecs, const int32_t* __restrict__ row,
+                                                                     const float* __restrict__ wt, int64_t tokens,
+                                                                     int topk, uint4* __restrict__ out,
+                                                                     int32_t* status) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (t >= tokens) return;
+  const int32_t* rt = row + t * topk;
+  const float* wt_t = wt + t * topk;
+  bool bad = false;
+  for (int64_t c = lane; c < n_vecs; c += 32) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int j0 = 0; j0 < topk; j0 += 4) {
+      uint4 v[4];
+      float wj[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u;
+        int32_t r = j < topk ? rt[j] : -1;
+        if (r >= y_rows) {
+          bad = true;
+          r = -1;
+        }
+        wj[u] = r >= 0 ? wt_t[j] : 0.0f;
+        v[u] = r >= 0 ? __ldcs(y + static_cast<int64_t>(r) * n_vecs + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (j0 + u >= topk) break;
+        const uint32_t x4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] = fmaf(wj[u], bf16_lo(x4[i]), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(wj[u], bf16_hi(x4[i]), acc[2 * i + 1]);
+        }
+      }
+    }
+    uint4 o;
+    uint32_t* op = &o.x;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+      op[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    out[t * n_vecs + c] = o;
+  }
+  if (bad && lane == 0) moe_report(status, kDevBadIndex);
+}
+
+// ======================================================================= host
+
+static cudaError_t launch_pdl_cfg(const void* func, dim3 grid, dim3 block, size_t smem, void** args,
+                                  cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelExC(&cfg, func, args);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_moe_route(const int32_t* ids, int64_t n, int E, int pad, int32_t* counts, int32_t* offsets,
+                             int32_t* row, int32_t* dropped, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(2 * E + 33) * 4 + static_cast<size_t>(E) * 32;
+  int ni = static_cast<int>(n);
+  void* args[] = {&ids, &ni, &E, &pad, &counts, &offsets, &row, &dropped};
+  return launch_pdl_cfg(reinterpret_cast<const void*>(moe_route_kernel), dim3(1), dim3(kRouteThreads), smem, args,
+                        stream);
+}
+
+cudaError_t launch_moe_place(const MoePlace& p, cudaStream_t stream) {
+  PlaceArgs a = {};
+  a.src = p.src;
+  a.src_sf = static_cast<const uint8_t*>(p.src_sf);
+  a.row = p.row;
+  a.counts = p.counts;
+  a.offsets = p.offsets;
+  a.q = static_cast<uint8_t*>(p.q);
+  a.sf = static_cast<uint8_t*>(p.sf);
+  a.status = p.status;
+  a.n_src = p.n_src;
+  a.m_rows = p.m_rows;
+  a.k = static_cast<int>(p.k);
+  a.fan = p.fan;
+  a.E = p.pad > 1 ? p.experts : 0;
+  a.pad_slots = p.pad > 1 ? p.pad - 1 : 0;
+  a.sf_row_major = p.sf_row_major;
+  const int64_t warps = p.n_src + static_cast<int64_t>(a.E) * a.pad_slots;
+  if (warps == 0) return cudaSuccess;
+  const int64_t grid = (warps + kRowWarps - 1) / kRowWarps;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  void* args[] = {&a};
+  const void* f = p.quantize ? reinterpret_cast<const void*>(moe_place_kernel<true>)
+                             : reinterpret_cast<const void*>(moe_place_kernel<false>);
+  return launch_pdl_cfg(f, dim3(static_cast<unsigned>(grid)), dim3(kRowWarps * 32), 0, args, stream);
+}
+
+cudaError_t launch_moe_gather(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* idx, int64_t n,
+                              void* dst, int32_t* status, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const int64_t grid = (n + kRowWarps - 1) / kRowWarps;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  const uint4* s = static_cast<const uint4*>(src);
+  uint4* d = static_cast<uint4*>(dst);
+  int64_t vecs = row_bytes / 16;
+  void* args[] = {&s, &src_rows, &vecs, &idx, &n, &d, &status};
+  return launch_pdl_cfg(reinterpret_cast<const void*>(moe_gather_kernel), dim3(static_cast<unsigned>(grid)),
+                        dim3(kRowWarps * 32), 0, args, stream);
+}
+
+cudaError_t launch_moe_combine(const void* y, int64_t y_rows, int64_t n_cols, const int32_t* row, const float* w,
+                               int64_t tokens, int topk, void* out, int32_t* status, cudaStream_t stream) {
+  if (tokens == 0) return cudaSuccess;
+  const int64_t grid = (tokens + kRowWarps - 1) / kRowWarps;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  const uint4* yp = static_cast<const uint4*>(y);
+  uint4* op = static_cast<uint4*>(out);
+  int64_t vecs = n_cols / 8;
+  void* args[] = {&yp, &y_rows, &vecs, &row, &w, &tokens, &topk, &op, &status};
+  return launch_pdl_cfg(reinterpret_cast<const void*>(moe_combine_kernel), dim3(static_cast<unsigned>(grid)),
+                        dim3(kRowWarps * 32), 0, args, stream);
+}
+
+}  // namespace mxk

@@ -34,6 +34,7 @@
 
 #include "mx_fastdiv.h"
 #include "mx_launch.h"
+#include "mx_mxfp8.cuh"
 
 namespace mxk {
 
@@ -70,35 +71,6 @@ struct QuantBatch {
   int main_blocks;         // CTAs that stream blocks; the rest write padding
   int64_t pad_total;
 };
-
-__device__ __forceinline__ uint32_t sf_tiled_offset(uint32_t r, uint32_t c, uint32_t sf_ktiles) {
-  return ((r >> 7) * sf_ktiles + (c >> 2)) * 512u + (r & 31u) * 16u + ((r & 127u) >> 5) * 4u + (c & 3u);
-}
-
-// Scale exponent X for a block whose largest magnitude has BF16 bits `amax_bits`
-// (finite).  X = floor(log2 amax) - 8, clamped to [-127, 127]; amax == 0 -> -127.
-__device__ __forceinline__ int block_exponent(uint32_t amax_bits) {
-  if (amax_bits == 0) return -127;
-  const int e = static_cast<int>(amax_bits >> 7);
-  int fl;
-  if (e > 0) {
-    fl = e - 127;
-  } else {
-    const uint32_t m = amax_bits & 0x7Fu;  // subnormal: value = m * 2^-133
-    fl = (31 - __clz(m)) - 133;
-  }
-  int X = fl - 8;
-  return X < -127 ? -127 : (X > 127 ? 127 : X);
-}
-
-__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
-  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
-  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // Scale-tile padding entry i of one job: rows [rows, rpad) x all kb_pad
 // blocks, then rows [0, rows) x blocks [kb, kb_pad), for every group.
@@ -160,36 +132,8 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_co
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const uint32_t b = base + u * 32 + lane;
-      // amax of |x| on the magnitude bits, two BF16 values per SIMD max
-      uint32_t m2 = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        m2 = __vmaxu2(m2, v[u][j].x & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, v[u][j].y & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, v[u][j].z & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, v[u][j].w & 0x7FFF7FFFu);
-      }
-      const uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
-      uint32_t scode;
       uint4 out0, out1;
-      if (m >= 0x7F80u) {  // Inf or NaN somewhere in the block
-        scode = 0xFFu;
-        out0 = out1 = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-      } else {
-        const int X = block_exponent(m);
-        scode = static_cast<uint32_t>(X + 127);
-        const float mult = __uint_as_float(static_cast<uint32_t>(127 - X) << 23);  // 2^-X
-        uint32_t o[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          o[2 * j] = pack_e4m3x4(bf16_lo(v[u][j].x) * mult, bf16_hi(v[u][j].x) * mult,
-                                 bf16_lo(v[u][j].y) * mult, bf16_hi(v[u][j].y) * mult);
-          o[2 * j + 1] = pack_e4m3x4(bf16_lo(v[u][j].z) * mult, bf16_hi(v[u][j].z) * mult,
-                                     bf16_lo(v[u][j].w) * mult, bf16_hi(v[u][j].w) * mult);
-        }
-        out0 = make_uint4(o[0], o[1], o[2], o[3]);
-        out1 = make_uint4(o[4], o[5], o[6], o[7]);
-      }
+      const uint32_t scode = quant_block32_bf16(v[u], out0, out1);
       if (b < jb.nblk) {
         uint4* dst = jb.q + static_cast<size_t>(b) * 2;
         __stcs(dst, out0);

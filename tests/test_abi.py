@@ -46,6 +46,13 @@ def lib():
     L.mx_grouped_gemm_contiguous_tilewise.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
     L.mx_grouped_gemm_contiguous_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
     L.mx_grouped_gemm_masked_swiglu_quant.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P, P]
+    L.mx_moe_max_rows.argtypes = [I64, I32, I32]
+    L.mx_moe_max_rows.restype = I64
+    L.mx_moe_route.argtypes = [P, I64, I32, I32, P, P, P, P, P]
+    L.mx_moe_dispatch_quant.argtypes = [P, I64, I64, P, I32, P, P, I32, I32, I64, P, P, I32, P, P]
+    L.mx_moe_scatter_rows.argtypes = [P, P, I64, I64, P, P, P, I32, I32, I64, P, P, P, P]
+    L.mx_gather_rows.argtypes = [P, I64, I64, P, I64, P, P, P]
+    L.mx_moe_combine.argtypes = [P, I64, I64, P, P, I64, I32, P, P, P]
     return L
 
 
@@ -179,3 +186,40 @@ def test_tilewise_argument_checks(lib):
     c = lib.mx_grouped_gemm_contiguous_tilewise
     assert c(FAKE, FAKE, FAKE, FAKE, None, 4, 512, 256, 128, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
     assert c(FAKE, FAKE, FAKE, FAKE, FAKE, 2000, 512, 256, 128, FAKE, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+
+
+def test_moe_argument_checks(lib):
+    A, B, C, D, E = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+    assert lib.mx_moe_max_rows(65536, 32, 128) == 69632          # 65536 + 32*127 -> 69600 -> x128
+    assert lib.mx_moe_max_rows(10, 4, 1) == 128
+    assert lib.mx_moe_max_rows(-1, 4, 1) == 0
+    # route: experts in [1, 1024], pad in [1, 128], 4-byte aligned pointers
+    assert lib.mx_moe_route(A, 16, 0, 128, B, C, D, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_route(A, 16, 1025, 128, B, C, D, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_route(A, 16, 8, 0, B, C, D, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_route(A, 16, 8, 129, B, C, D, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_route(None, 16, 8, 128, B, C, D, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_route(A + 2, 16, 8, 128, B, C, D, None, None) == MX_ERR_MISALIGNED
+    # dispatch: k % 128, m_rows % 128 for tiled scales, topk in [1, 64], alignment
+    assert lib.mx_moe_dispatch_quant(A, 4, 96, B, 2, C, D, 8, 128, 128, E, E, 0, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert lib.mx_moe_dispatch_quant(A, 4, 128, B, 2, C, D, 8, 128, 100, E, E, 0, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert lib.mx_moe_dispatch_quant(A, 4, 128, B, 0, C, D, 8, 128, 128, E, E, 0, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_dispatch_quant(A, 4, 128, B, 2, None, None, 8, 128, 128, E, E, 0, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_dispatch_quant(A + 8, 4, 128, B, 2, C, D, 8, 128, 128, E, E, 0, None, None) == MX_ERR_MISALIGNED
+    assert lib.mx_moe_dispatch_quant(A, 4, 128, None, 2, C, D, 8, 128, 128, E, E, 0, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_dispatch_quant(A, 0, 128, None, 2, None, None, 0, 1, 0, None, None, 1, None, None) == MX_OK
+    # scatter: same rules, plus the source scales
+    assert lib.mx_moe_scatter_rows(A, None, 4, 128, B, C, D, 8, 128, 128, E, E, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_scatter_rows(A, A, 4, 64, B, C, D, 8, 128, 128, E, E, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    # gather: rows of a multiple of 16 bytes, aligned
+    assert lib.mx_gather_rows(A, 8, 24, B, 4, C, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert lib.mx_gather_rows(A + 4, 8, 32, B, 4, C, None, None) == MX_ERR_MISALIGNED
+    assert lib.mx_gather_rows(A, 8, 32, None, 4, C, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_gather_rows(A, 8, 32, B, 0, C, None, None) == MX_OK
+    # combine: n_cols % 8, topk in [1, 64], aligned y/out and 4-byte w/row
+    assert lib.mx_moe_combine(A, 8, 12, B, C, 4, 2, D, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert lib.mx_moe_combine(A, 8, 16, B, C, 4, 0, D, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_combine(A, 8, 16, B, C, 4, 65, D, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_combine(A, 8, 16, B, C + 2, 4, 2, D, None, None) == MX_ERR_MISALIGNED
+    assert lib.mx_moe_combine(A, 8, 16, None, C, 4, 2, D, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert lib.mx_moe_combine(A, 8, 16, B, C, 0, 2, D, None, None) == MX_OK
