@@ -1,0 +1,63 @@
+"""CPU stand-ins for the library steps of the expert-parallel MoE layer,
+built on the oracle (fp64 GEMMs, exact quantisation), so the layer's
+multi-rank plumbing (count exchange, all-to-all splits, row orders, the
+return path) can run on gloo ranks without a GPU.  Scales stay row-major
+throughout: these ops both produce and consume them."""
+import numpy as np
+import torch
+
+import oracle
+
+
+def _np(t):
+    return t.detach().cpu().numpy() if isinstance(t, torch.Tensor) else np.asarray(t)
+
+
+def _bf16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+
+
+class OracleOps:
+    def max_rows(self, n, experts, pad):
+        return (n + experts * (pad - 1) + 127) // 128 * 128
+
+    def route(self, ids, experts, pad):
+        c, o, r, _ = oracle.moe_route(_np(ids).reshape(-1).astype(np.int32), experts, pad)
+        return torch.from_numpy(c), torch.from_numpy(o), torch.from_numpy(r)
+
+    def dispatch(self, x, row, topk, counts, offsets, pad, m_rows, row_major):
+        q, sf = oracle.moe_dispatch(x, _np(row), topk, m_rows)
+        return torch.from_numpy(q), torch.from_numpy(sf.reshape(-1).copy())
+
+    def scatter(self, q_src, sf_src, dst_row, counts, offsets, pad, m_rows):
+        q_src, sf_src, dst = _np(q_src), _np(sf_src), _np(dst_row)
+        q = np.zeros((m_rows, q_src.shape[1]), dtype=np.uint8)
+        sf = np.zeros((m_rows, sf_src.shape[1]), dtype=np.uint8)
+        q[dst] = q_src
+        sf[dst] = sf_src
+        return torch.from_numpy(q), torch.from_numpy(sf)
+
+    def gate_up_swiglu(self, qa, sfa, q13, sf13, offsets):
+        off = _np(offsets).astype(np.int32)
+        d, _ = oracle.grouped_contiguous(_np(qa), _np(sfa), _np(q13), _np(sf13), off)
+        i_dim = d.shape[1] // 2
+        h = oracle.swiglu(d[:, :i_dim], d[:, i_dim:]).astype(np.float32)
+        qh = np.zeros((qa.shape[0], i_dim), dtype=np.uint8)
+        sfh = np.zeros((qa.shape[0], i_dim // 32), dtype=np.uint8)
+        if len(h):
+            qh[: len(h)], sfh[: len(h)] = oracle.quantize_f32(h)
+        return torch.from_numpy(qh), torch.from_numpy(sfh)
+
+    def down(self, qh, sfh, q2, sf2, offsets):
+        off = _np(offsets).astype(np.int32)
+        d, _ = oracle.grouped_contiguous(_np(qh), _np(sfh), _np(q2), _np(sf2), off)
+        out = np.zeros((qh.shape[0], d.shape[1]), dtype=np.float64)
+        out[: len(d)] = d
+        return _bf16(out)
+
+    def gather(self, src, idx):
+        return src[torch.as_tensor(_np(idx)).long()]
+
+    def combine(self, y, row, w):
+        out, _ = oracle.moe_combine(y.contiguous(), _np(row), _np(w))
+        return _bf16(out)

@@ -275,3 +275,23 @@ def test_moe_layer_full_shape_sampled(mx, oracle):
     rng = np.random.default_rng(63)
     tokens = np.unique(np.concatenate([[0, T - 1], rng.choice(T, 94, replace=False)]))
     layer_check(mx, oracle, x, ids, w2.cpu(), gate_w, E, r, sample_tokens=tokens)
+
+
+def test_ep_layer_one_rank_matches_direct_layer(mx):
+    """The expert-parallel layer with one rank (send buffer in expert order,
+    scatter into the padded layout, gather back) computes exactly what the
+    direct single-GPU layer computes."""
+    from moe_grouped_gemm_mx_b200.ep import ep_moe_layer
+    T, topk, E, H, I, N = 300, 4, 8, 256, 256, 256
+    x = mx_inputs.normal_bf16((T, H), 1.0, 70).to(DEV)
+    ids = mx_inputs.topk_ids(T, topk, E, seed=71)
+    ids[5, 2] = -1                                   # a dropped entry
+    gate_w = mx_inputs.gate_weights(T, topk, seed=72)
+    w13 = mx_inputs.normal_bf16((E, 2 * I, H), 0.05, 73)
+    w2 = mx_inputs.normal_bf16((E, N, I), 0.05, 74)
+    r = moe_layer(mx, x, ids, w13, w2, gate_w, E)
+    q13, sf13 = mx.mx_quantize_bf16_to_e4m3(w13.to(DEV))
+    q2, sf2 = mx.mx_quantize_bf16_to_e4m3(w2.to(DEV))
+    y = ep_moe_layer(x, torch.from_numpy(ids).to(DEV), torch.from_numpy(gate_w).to(DEV), E, q13, sf13, q2, sf2)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), r["out"].view(torch.int16))

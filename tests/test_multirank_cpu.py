@@ -40,7 +40,7 @@ def _rank_main(rank, world, port, out):
 
 def test_max_over_ranks_gloo():
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
     assert out[0] == 3.0 and out[1] == 3.0
