@@ -93,6 +93,15 @@ def static_config(name: str, seed: int) -> dict:
                     "padded_rows": int(I.padded_offsets(counts)[-1]),
                     "gemms": ["dgrad dX[T,7168] = dY[T,4096] W13 (contiguous, W13 quantised along N)",
                               "wgrad dW13[32,4096,7168] = dY^T X per expert (K-grouped over tokens)"]})
+    elif name == "moe_layer":
+        import numpy as np
+        tokens = MOE_OVERRIDE["tokens"] or I.MOE_TOKENS
+        experts = MOE_OVERRIDE["experts"] or I.MOE_EXPERTS
+        c = np.bincount(I.topk_ids(tokens, I.MOE_TOPK, experts, seed=seed).reshape(-1), minlength=experts)
+        cfg.update({"experts": experts, "tokens": tokens, "topk": I.MOE_TOPK, "zipf_s": I.MOE_ZIPF_S,
+                    "hidden": I.MOE_GATE_NK[1], "intermediate": I.MOE_DOWN_NK[1], "real_rows": int(c.sum()),
+                    "padded_rows": int(((c + 127) // 128 * 128).sum()),
+                    "gate_weights": "softmax over N(0,1) logits"})
     elif name == "masked":
         mm = I.masked_counts(seed=seed)
         cfg.update({"experts": I.MASKED_EXPERTS, "max_m": I.MASKED_MAX_M, "n": I.MASKED_NK[0],
@@ -103,6 +112,10 @@ def static_config(name: str, seed: int) -> dict:
     elif name == "moe_mlp":
         cfg["step"] = ("quantise tokens + gate/up and down weights (one batched launch), then the fused "
                        "gate/up GEMM -> SwiGLU -> MXFP8 kernel and the down GEMM with BF16 epilogue")
+    elif name == "moe_layer":
+        cfg["step"] = ("quantise the gate/up and down weights (one batched launch), route the top-8 table, "
+                       "dispatch (quantise each token once into its experts' rows), fused gate/up GEMM -> "
+                       "SwiGLU -> MXFP8, down GEMM, gate-weighted combine to BF16 token outputs")
     else:
         cfg["step"] = ("quantise activations + weights (one batched launch), then the GEMM(s) "
                        "with BF16 epilogue")
@@ -114,7 +127,8 @@ def parse_args():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp", "moe_bwd"])
+    p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp", "moe_bwd",
+                                                            "moe_layer"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -407,6 +421,73 @@ class Workload:
         self.config.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "real_rows": real,
                             "padded_rows": m_total})
 
+    def _build_moe_layer(self, seed, I):
+        """One complete MoE expert layer in token order: routing plan, dispatch
+        (each token quantised to MXFP8 once and placed at its experts' rows of
+        the padded grouped layout), [gate; up] GEMM + SwiGLU + MXFP8, down GEMM,
+        gate-weighted combine back to the tokens; the expert weights are
+        quantised in the step's batched launch."""
+        import numpy as np
+        import torch
+        mx = self.mx
+        T = MOE_OVERRIDE["tokens"] or I.MOE_TOKENS
+        E = MOE_OVERRIDE["experts"] or I.MOE_EXPERTS
+        topk = I.MOE_TOPK
+        n13, hdim = I.MOE_GATE_NK
+        n2, i_dim = I.MOE_DOWN_NK
+        assert n13 == 2 * i_dim
+        ids_np = I.topk_ids(T, topk, E, seed=seed)
+        ids = torch.from_numpy(ids_np.reshape(-1).copy()).to(self.dev)
+        gw = torch.from_numpy(I.gate_weights(T, topk, seed=seed)).to(self.dev)
+        x = I.normal_bf16((T, hdim), 1.0, seed + 7, self.dev)
+        w13 = I.normal_bf16((E, n13, hdim), 0.02, seed + 2_000_003, self.dev)
+        w2 = I.normal_bf16((E, n2, i_dim), 0.02, seed + 4_000_037, self.dev)
+        for t in (x, ids, gw, w13, w2):
+            self._add_input(t)
+        q13, sf13 = self._quant(w13, "W13")
+        q2, sf2 = self._quant(w2, "W2")
+        counts_h = np.bincount(ids_np.reshape(-1), minlength=E)
+        real = int(counts_h.sum())
+        padded = int(((counts_h + 127) // 128 * 128).sum())
+        active = int((counts_h > 0).sum())
+        n = T * topk
+        m_rows = mx.mx_moe_max_rows(n, E, 128)
+        i32 = dict(dtype=torch.int32, device=self.dev)
+        counts, offsets, row, dropped = (torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(n, **i32),
+                                         torch.empty(1, **i32))
+        qa = torch.empty((m_rows, hdim), dtype=torch.uint8, device=self.dev)
+        sfa = torch.empty(mx.scale_bytes(m_rows, hdim), dtype=torch.uint8, device=self.dev)
+        qh = torch.empty((m_rows, i_dim), dtype=torch.uint8, device=self.dev)
+        sfh = torch.empty(mx.scale_bytes(m_rows, i_dim), dtype=torch.uint8, device=self.dev)
+        y = torch.empty((m_rows, n2), dtype=torch.bfloat16, device=self.dev)
+        out = torch.empty((T, n2), dtype=torch.bfloat16, device=self.dev)
+        self.outputs.append(out)
+        self.launches.append(("route", "route", lambda ids: mx.mx_moe_route(ids, E, 128, counts, offsets, row,
+                                                                               dropped),
+                              n * 8.0, 0.0, (ids,)))
+        # read each token once, write its row (and scales) per routed expert, zero the padding rows
+        dbytes = T * hdim * 2.0 + padded * hdim * (1 + 1 / 32) + n * 4.0
+        self.launches.append(("dispatch", "dispatch", lambda x, row, counts, offsets: mx.mx_moe_dispatch_quant(
+            x, row, topk, counts, offsets, 128, m_rows, q=qa, sf=sfa, dev_status=self.status), dbytes, 0.0,
+            (x, row, counts, offsets)))
+        fl1 = 2.0 * real * n13 * hdim
+        bytes1 = (padded * hdim + active * n13 * hdim + padded * i_dim) * (1 + 1 / 32)
+        self.launches.append(("gemm", "gate_up+swiglu", lambda qa, sfa, q13, sf13, offsets:
+                              mx.mx_grouped_gemm_contiguous_swiglu_quant(qa, sfa, q13, sf13, offsets, qh=qh,
+                                                                         sfh=sfh, dev_status=self.status),
+                              bytes1, fl1, (qa, sfa, q13, sf13, offsets)))
+        fl2 = 2.0 * real * n2 * i_dim
+        self.launches.append(("gemm", "down", lambda qh, sfh, q2, sf2, offsets: mx.mx_grouped_gemm_contiguous(
+            qh, sfh, q2, sf2, offsets, d=y, dev_status=self.status), self._gemm_bytes(padded, n2, i_dim, active),
+            fl2, (qh, sfh, q2, sf2, offsets)))
+        cbytes = real * n2 * 2.0 + T * n2 * 2.0 + n * 8.0
+        self.launches.append(("combine", "combine", lambda y, row, gw: mx.mx_moe_combine(
+            y, row, gw, out=out, dev_status=self.status), cbytes, 0.0, (y, row, gw)))
+        self.flops += fl1 + fl2
+        self.config.update({"experts": E, "tokens": T, "topk": topk, "zipf_s": I.MOE_ZIPF_S, "hidden": hdim,
+                            "intermediate": i_dim, "real_rows": real, "padded_rows": padded,
+                            "gate_weights": "softmax over N(0,1) logits"})
+
     def _build_moe_bwd(self, seed, I):
         """Backward of the MoE gate/up projection (the contiguous workload's
         first GEMM): input gradient dX = dY W13 per expert and weight gradient
@@ -584,6 +665,43 @@ def oracle_sample(name, seed, target_s=10.0, fmt="mxfp8"):
         jobs.append(job)
         desc = ("one expert layer on 64 rows over 2 experts: quantise rows and weights, gate/up GEMM, "
                 "SwiGLU, requantise, down GEMM")
+    elif name == "moe_layer":
+        n13, k = I.MOE_GATE_NK
+        n2, i_dim = I.MOE_DOWN_NK
+        T, topk, E = 8, I.MOE_TOPK, 8
+        x = I.normal_bf16((T, k), 1.0, seed + 7)
+        ids = I.topk_ids(T, topk, E, seed=seed)
+        gw = I.gate_weights(T, topk, seed=seed)
+        w13 = I.normal_bf16((E, n13, k), 0.02, seed + 8)
+        w2 = I.normal_bf16((E, n2, i_dim), 0.02, seed + 9)
+
+        def job():
+            import torch
+            q13, sf13 = L.quantize(w13)
+            q2, sf2 = L.quantize(w2)
+            counts, off, row, _ = L.moe_route(ids, E, 128)
+            m = int(off[-1])
+            qa, sfa = L.moe_dispatch(x, row, topk, m)
+            rows = np.sort(row).astype(np.int64)           # the routed rows (padding rows are not computed)
+            q13 = q13.reshape(E, n13, k)
+            sf13 = sf13.reshape(E, n13, k // 32)
+            g, _ = L.grouped_contiguous(qa, sfa, np.ascontiguousarray(q13[:, :i_dim]),
+                                        np.ascontiguousarray(sf13[:, :i_dim]), off, rows=rows)
+            u, _ = L.grouped_contiguous(qa, sfa, np.ascontiguousarray(q13[:, i_dim:]),
+                                        np.ascontiguousarray(sf13[:, i_dim:]), off, rows=rows)
+            qh = np.zeros((m, i_dim), dtype=np.uint8)
+            sfh = np.zeros((m, i_dim // 32), dtype=np.uint8)
+            qh[rows], sfh[rows] = L.quantize_f32(L.swiglu(g, u).astype(np.float32))
+            d, _ = L.grouped_contiguous(qh, sfh, q2.reshape(E, n2, i_dim), sf2.reshape(E, n2, i_dim // 32), off,
+                                        rows=rows)
+            y = np.zeros((m, n2), dtype=np.float32)
+            y[rows] = d
+            L.moe_combine(torch.from_numpy(y).to(torch.bfloat16), row, gw)
+            real = T * topk
+            return 2.0 * real * n13 * k + 2.0 * real * n2 * i_dim
+        jobs.append(job)
+        desc = (f"one expert layer on {T} tokens x top-{topk} of {E} experts: quantise the experts' weights, "
+                "route, dispatch, gate/up GEMM, SwiGLU, requantise, down GEMM, combine")
     else:  # masked
         n, k = I.MASKED_NK
         prob = I.masked_problem(n=n, k=k, experts=2, max_m=32, seed=seed,

@@ -32,14 +32,21 @@ constexpr int kDevBadIndex = 0x8;
 __device__ __forceinline__ void moe_report(int32_t* status, int bits) { atomicOr(status, bits); }
 
 // ------------------------------------------------------------------ routing plan
-// One CTA of 1024 threads: the plan is a prefix over all entries, and the
-// table (8192 tokens x top-8 = 64K entries) is tiny next to the GEMMs it
-// feeds.  Phase 1: per-expert histogram in shared memory.  Phase 2: exclusive
-// scan of the padded group sizes (one expert per thread, E <= 1024).
-// Phase 3: stable ranks, 1024 entries per step in entry order: within a warp
-// by __match_any_sync and the population count of the lower lanes, across
-// the warps of a step through a byte table of per-warp counts per expert,
-// across steps by a running next row per expert.
+// One CTA of 32 warps: the plan is a prefix over all entries, and the table
+// (8192 tokens x top-8 = 64K entries) is small next to the GEMMs it feeds.
+// Warp w owns the contiguous segment [w*seg, (w+1)*seg) of the entries, so
+// entry order is (warp, position in segment).
+//  1. each warp streams its segment 32 entries per step (four steps' loads in
+//     flight): a lane's rank among the step's entries of its expert comes
+//     from __match_any_sync, the warp's running count of that expert from its
+//     own row of a [32][E] shared-memory table; the rank within the segment
+//     is parked in row[i];
+//  2. one thread per expert turns its column of the table into exclusive
+//     per-warp prefixes and a total; a block scan over the padded totals
+//     gives the group offsets;
+//  3. each warp adds offset + warp prefix to the parked ranks (coalesced).
+constexpr int kRouteUnroll = 4;
+
 __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t* __restrict__ ids, int n, int E,
                                                                   int pad, int32_t* __restrict__ counts,
                                                                   int32_t* __restrict__ offsets,
@@ -48,27 +55,60 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ int32_t route_smem[];
-  int32_t* hist = route_smem;       // [E]
-  int32_t* next = hist + E;         // [E] next row of each expert
-  int32_t* wsum = next + E;         // [32] warp totals of the scan
-  int32_t* nbad = wsum + 32;        // [1]
-  uint8_t* wcnt = reinterpret_cast<uint8_t*>(nbad + 1);  // [E][32] entries per warp in the current step
+  int32_t* wc = route_smem;          // [32][E] per-warp counts, then per-warp exclusive prefixes
+  int32_t* base = wc + 32 * E;       // [E] group offsets
+  int32_t* wsum = base + E;          // [32] warp totals of the scan
+  int32_t* nbad = wsum + 32;         // [1]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
-  for (int i = tid; i < E * 32; i += blockDim.x) wcnt[i] = 0;
+  for (int i = tid; i < 32 * E; i += blockDim.x) wc[i] = 0;
   if (tid == 0) *nbad = 0;
   __syncthreads();
 
+  const int seg = (n + 31) / 32;
+  const int begin = warp * seg;
+  const int end = min(n, begin + seg);
+  const uint32_t lower = (1u << lane) - 1u;
+  int32_t* my = wc + warp * E;
   int bad = 0;
-  for (int i = tid; i < n; i += blockDim.x) {
-    const int e = ids[i];
-    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
-    else ++bad;
+  for (int s0 = begin; s0 < end; s0 += 32 * kRouteUnroll) {
+    int ev[kRouteUnroll];
+#pragma unroll
+    for (int u = 0; u < kRouteUnroll; ++u) {
+      const int i = s0 + u * 32 + lane;
+      ev[u] = i < end ? __ldg(ids + i) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kRouteUnroll; ++u) {
+      const int i = s0 + u * 32 + lane;
+      const bool in = i < end;
+      const bool valid = in && ev[u] >= 0 && ev[u] < E;
+      if (in && !valid) ++bad;
+      const int key = valid ? ev[u] : -1;
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
+      int b = 0;
+      if (valid) {
+        b = my[key];
+        row[i] = b + __popc(peers & lower);
+      } else if (in) {
+        row[i] = -1;
+      }
+      __syncwarp();
+      if (valid && (peers & lower) == 0) my[key] = b + __popc(peers);
+      __syncwarp();
+    }
   }
   if (bad) atomicAdd(nbad, bad);
   __syncthreads();
 
-  const int v = tid < E ? (hist[tid] + pad - 1) / pad * pad : 0;
+  int total = 0;
+  if (tid < E) {
+    for (int w = 0; w < 32; ++w) {
+      const int c = wc[w * E + tid];
+      wc[w * E + tid] = total;
+      total += c;
+    }
+  }
+  const int v = tid < E ? (total + pad - 1) / pad * pad : 0;
   int incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -90,40 +130,19 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
   __syncthreads();
   const int excl = incl - v + wsum[warp];
   if (tid < E) {
-    counts[tid] = hist[tid];
+    counts[tid] = total;
     offsets[tid] = excl;
-    next[tid] = excl;
+    base[tid] = excl;
     if (tid == E - 1) offsets[E] = excl + v;
   }
   if (tid == 0 && dropped != nullptr) *dropped = *nbad;
   __syncthreads();
 
-  const uint32_t lower = (1u << lane) - 1u;
-  for (int c0 = 0; c0 < n; c0 += blockDim.x) {
-    const int i = c0 + tid;
-    int e = -1;
-    if (i < n) {
-      e = ids[i];
-      if (e < 0 || e >= E) e = -1;
-    }
-    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
-    const bool leader = (peers & lower) == 0;
-    if (e >= 0 && leader) wcnt[e * 32 + warp] = static_cast<uint8_t>(__popc(peers));
-    __syncthreads();
-    if (e >= 0) {
-      int pre = 0;
-      const uint8_t* wc = wcnt + e * 32;
-      for (int w = 0; w < warp; ++w) pre += wc[w];
-      row[i] = next[e] + pre + __popc(peers & lower);
-    } else if (i < n) {
-      row[i] = -1;
-    }
-    __syncthreads();
-    if (e >= 0 && leader) {
-      atomicAdd(&next[e], __popc(peers));
-      wcnt[e * 32 + warp] = 0;
-    }
-    __syncthreads();
+  for (int i = begin + lane; i < end; i += 32) {
+    const int r = row[i];  // written by this thread in step 1
+    if (r < 0) continue;
+    const int e = __ldg(ids + i);
+    row[i] = base[e] + my[e] + r;
   }
 }
 
@@ -322,7 +341,11 @@ static cudaError_t launch_pdl_cfg(const void* func, dim3 grid, dim3 block, size_
 
 cudaError_t launch_moe_route(const int32_t* ids, int64_t n, int E, int pad, int32_t* counts, int32_t* offsets,
                              int32_t* row, int32_t* dropped, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(2 * E + 33) * 4 + static_cast<size_t>(E) * 32;
+  const size_t smem = static_cast<size_t>(33 * E + 33) * 4;  // at most 135 KB (E = 1024)
+  static cudaError_t attr = cudaErrorNotReady;
+  if (attr == cudaErrorNotReady)
+    attr = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * 1024 * 4 + 33 * 4);
+  if (attr != cudaSuccess) return attr;
   int ni = static_cast<int>(n);
   void* args[] = {&ids, &ni, &E, &pad, &counts, &offsets, &row, &dropped};
   return launch_pdl_cfg(reinterpret_cast<const void*>(moe_route_kernel), dim3(1), dim3(kRouteThreads), smem, args,
