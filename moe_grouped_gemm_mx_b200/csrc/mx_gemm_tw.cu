@@ -14,11 +14,12 @@
 // CTA layout (192 threads, one CTA per SM, persistent over 128 x 128 tiles):
 //   warp 0      TMA producer: A and B tiles of one 128-element K tile per
 //               stage, STAGES-deep ring.
-//   warp 1      TMEM owner and MMA issuer: each K tile's four K = 32
-//               block-scaled MMAs (every scale factor 2^0, staged once into
-//               TMEM) go into a FRESH partial accumulator, alternating
-//               between two TMEM buffers so that the tensor core fills one
-//               while the other is being promoted.
+//   warp 1      TMEM owner and MMA issuer: each K tile's four K = 32 FP8
+//               MMAs (kind::f8f6f4, no block scales) go into a FRESH partial
+//               accumulator, cycling through four 128-column TMEM buffers,
+//               so the tensor core runs up to three K tiles ahead of the
+//               promotion (a 128 x 128 x 128 tile is only ~256 MMA cycles,
+//               less than one promotion round trip).
 //   warps 2..5  promotion and epilogue: each thread owns one row of the
 //               tile; per K tile it reads the row's 128 partial sums from
 //               TMEM, releases the buffer, and adds them times
@@ -37,22 +38,22 @@ namespace mxk {
 
 constexpr int kTwStages = 6;
 constexpr int kTwThreads = 192;
+constexpr int kTwBufs = 4;  // TMEM partial buffers of 128 columns (all 512 columns)
 
 struct TwLayout {
   static constexpr int A_BYTES = 128 * BK;  // 16 KB
   static constexpr int B_BYTES = 128 * BK;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + kTwStages * A_BYTES;
-  static constexpr int OFF_ONES = OFF_B + kTwStages * B_BYTES;  // 512 bytes of scale code 127 (2^0)
-  static constexpr int OFF_STG = (OFF_ONES + 512 + 1023) / 1024 * 1024;
+  static constexpr int OFF_STG = (OFF_B + kTwStages * B_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = OFF_STG + 2 * 8192;
-  static constexpr int NUM_BARS = 2 * kTwStages + 4 + 1;  // full/empty per stage, accf[2], acce[2], drain
+  // full/empty per stage, accf/acce per partial buffer, drain
+  static constexpr int NUM_BARS = 2 * kTwStages + 2 * kTwBufs + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB0 = OFF_MISC + 16;
   static constexpr int BYTES = OFF_TAB0 + (kMaxGroups + 1) * 4;
   static constexpr int ALLOC = BYTES + 1024;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t SF_COL = 256;  // unit scales: SFA 4 columns, then SFB 4 columns
+  static constexpr uint32_t TMEM_COLS = 128 * kTwBufs;
   static_assert(OFF_B % 1024 == 0 && OFF_STG % 1024 == 0, "swizzled tiles need 1024-B alignment");
   static_assert(ALLOC <= 232448, "shared memory budget");
 };
@@ -84,25 +85,21 @@ __global__ void __launch_bounds__(kTwThreads, 1)
   auto full_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * s; };
   auto empty_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (kTwStages + s); };
   auto accf_bar = [&](int b) { return sbase + L::OFF_BAR + 8u * (2 * kTwStages + b); };
-  auto acce_bar = [&](int b) { return sbase + L::OFF_BAR + 8u * (2 * kTwStages + 2 + b); };
-  const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (2 * kTwStages + 4);
+  auto acce_bar = [&](int b) { return sbase + L::OFF_BAR + 8u * (2 * kTwStages + kTwBufs + b); };
+  const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (2 * kTwStages + 2 * kTwBufs);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTwStages; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kTwBufs; ++b) {
       mbar_init(accf_bar(b), 1);
       mbar_init(acce_bar(b), 128);
     }
     mbar_init(drain_bar, 1);
     fence_mbar_init();
     *abort_flag = 0;
-  }
-  if (warp == 1) {  // 512 bytes of UE8M0 code 127 (= 2^0) for the MMA's scale operands
-    reinterpret_cast<uint4*>(smem + L::OFF_ONES)[lane] = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
-    fence_proxy_async_smem();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
@@ -185,27 +182,23 @@ __global__ void __launch_bounds__(kTwThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ===== MMA issuer
-      const uint32_t sf = tmem_base + L::SF_COL;
-      tc_cp_32x128b_warpx4(sf, desc_sf_32x16(sbase + L::OFF_ONES));      // SFA: 2^0 everywhere
-      tc_cp_32x128b_warpx4(sf + 4, desc_sf_32x16(sbase + L::OFF_ONES));  // SFB
-      const uint32_t idesc0 = idesc_mxf8_e4m3(BM, 128);
+      const uint32_t idesc = idesc_f8_e4m3_f32(BM, 128);
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t ib = 0;  // K tiles issued so far (partial buffer = ib & 1)
+      uint32_t ib = 0;  // K tiles issued so far (partial buffer = ib % kTwBufs)
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         for (int kt = 0; kt < args.k_tiles; ++kt, ++ib) {
-          const uint32_t b = ib & 1u;
-          if (!mbar_wait(acce_bar(b), ((ib >> 1) & 1u) ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          const uint32_t b = ib % kTwBufs;
+          if (!mbar_wait(acce_bar(b), ((ib / kTwBufs) & 1u) ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES;
           const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb)
-            tc_mma_mxf8(tmem_base + b * 128, desc_kmajor_sw128(a_addr + 32 * kb), desc_kmajor_sw128(b_addr + 32 * kb),
-                        idesc_with_sf_ids(idesc0, kb, kb), sf | (static_cast<uint32_t>(kb) << 30),
-                        (sf + 4) | (static_cast<uint32_t>(kb) << 30), kb != 0 ? 1u : 0u);
+            tc_mma_f8(tmem_base + b * 128, desc_kmajor_sw128(a_addr + 32 * kb), desc_kmajor_sw128(b_addr + 32 * kb),
+                      idesc, kb != 0 ? 1u : 0u);
           tc_commit(empty_bar(stage));
           tc_commit(accf_bar(b));
           if (++stage == kTwStages) { stage = 0; phase ^= 1u; }
@@ -231,15 +224,28 @@ __global__ void __launch_bounds__(kTwThreads, 1)
       const int row = m_blk * BM + r_local;
       const bool row_ok = row < args.m;
       const float* sb_t = args.sb + (static_cast<int64_t>(group) * args.n_tiles + n_blk) * args.k_tiles;
+      const float* sa_r = args.sa + row;
+      auto sa_at = [&](int kt) { return row_ok ? __ldg(sa_r + static_cast<int64_t>(kt) * args.m) : 0.0f; };
+      // the scales of K tile kt are loaded two K tiles ahead of their use
+      float sa0 = sa_at(0), sb0 = __ldg(sb_t);
+      float sa1 = args.k_tiles > 1 ? sa_at(1) : 0.0f, sb1 = args.k_tiles > 1 ? __ldg(sb_t + 1) : 0.0f;
       float acc[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
       for (int kt = 0; kt < args.k_tiles; ++kt, ++ib) {
-        const uint32_t b = ib & 1u;
-        const float s = (row_ok ? __ldg(args.sa + static_cast<int64_t>(kt) * args.m + row) : 0.0f) * __ldg(sb_t + kt);
-        const bool got = mbar_wait(accf_bar(b), (ib >> 1) & 1u, abort_flag, kWaitLimitNs);
-        if (!named_barrier_and(2, 128, got)) {
-          if (threadIdx.x == 64) report(args.status, 0x4);
+        const uint32_t b = ib % kTwBufs;
+        const float s = sa0 * sb0;
+        sa0 = sa1;
+        sb0 = sb1;
+        if (kt + 2 < args.k_tiles) {
+          sa1 = sa_at(kt + 2);
+          sb1 = __ldg(sb_t + kt + 2);
+        }
+        // each warp reads only its own TMEM lane quarter: a warp-uniform
+        // decision is enough (the aligned TMEM loads need one)
+        const bool got = mbar_wait(accf_bar(b), (ib / kTwBufs) & 1u, abort_flag, kWaitLimitNs);
+        if (!__all_sync(0xFFFFFFFFu, got)) {
+          if (lane == 0) report(args.status, 0x4);
           *abort_flag = 1;
           ok = false;
           break;
@@ -263,7 +269,10 @@ __global__ void __launch_bounds__(kTwThreads, 1)
           }
         }
       }
-      if (!ok) break;
+      // one uniform decision per tile before the epilogue's 128-thread
+      // barriers: a warp that gave up set abort_flag, which ends the other
+      // warps' waits too, so every warp gets here
+      if (!named_barrier_and(2, 128, ok)) break;
       uint32_t packed[64];
 #pragma unroll
       for (int j = 0; j < 64; ++j) packed[j] = pack_bf16x2(__float_as_uint(acc[2 * j]), __float_as_uint(acc[2 * j + 1]));

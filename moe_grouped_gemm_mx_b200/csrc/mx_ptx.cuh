@@ -137,6 +137,17 @@ __device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D(tmem) (+)= A(smem) * B(smem)^T for FP8 operands without block scaling.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far completes.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -200,6 +211,16 @@ __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N) {
          | (0u << 10)                             // B format E4M3
          | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
          | (1u << 23)                             // scale format UE8M0
+         | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
+// Instruction descriptor for kind::f8f6f4 without scales: E4M3 x E4M3 into an
+// FP32 accumulator (bits 4-5 = 1), both operands K-major, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_f8_e4m3_f32(int M, int N) {
+  return (1u << 4)                                // D format F32
+         | (0u << 7)                              // A format E4M3
+         | (0u << 10)                             // B format E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
 
