@@ -104,3 +104,50 @@ def test_tilewise_gemm_contiguous(mx, oracle):
             continue
         d_ref, absd = oracle.tw_gemm(qa_h[r0:r1], np.ascontiguousarray(sa_h[:, r0:r1]), qb_h[x], sb_h[x])
         assert_gemm_close(to_np_f64(d[r0:r1]), d_ref, absd, f"tile-wise contiguous expert {x}")
+
+
+# ---------------------------------------------------------------- ragged shapes and experts
+
+TW_SHAPES = [(256, 512, 512), (300, 272, 1152), (17, 400, 128), (600, 2112, 384)]
+TW_COUNTS = [0, 5, 128, 300, 1, 0, 77, 256]   # ragged experts, empty ones, a row block ending mid-tile
+
+
+@pytest.mark.parametrize("m,n,k", TW_SHAPES)
+def test_tilewise_gemm_ragged(mx, oracle, m, n, k):
+    """Ragged M, N tails and a single K tile (K = 128)."""
+    dev = torch.device("cuda")
+    a = mx_inputs.outlier_bf16((m, k), seed=m + k)
+    b = mx_inputs.normal_bf16((n, k), 0.02, m + n)
+    qa, sa = mx.mx_quantize_bf16_to_e4m3_tile1x128(a.to(dev))
+    qb, sb = mx.mx_quantize_bf16_to_e4m3_block128x128(b.to(dev))
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    d = mx.mx_gemm_tilewise(qa, sa, qb, sb, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    d_ref, absd = oracle.tw_gemm(qa.cpu().numpy(), sa.cpu().numpy(), qb.cpu().numpy(), sb.cpu().numpy())
+    assert_gemm_close(to_np_f64(d), d_ref, absd, f"tile-wise {m}x{n}x{k}")
+
+
+def test_tilewise_gemm_contiguous_ragged(mx, oracle):
+    counts = torch.tensor(TW_COUNTS, dtype=torch.int64)
+    n, k = 256, 640
+    prob = mx_inputs.contiguous_problem(n=n, k=k, seed=40, counts=counts)
+    e = len(counts)
+    dev = torch.device("cuda")
+    qa, sa = mx.mx_quantize_bf16_to_e4m3_tile1x128(prob.a.to(dev))
+    qb = torch.empty((e, n, k), dtype=torch.uint8, device=dev)
+    sb = torch.empty((e, n // 128, k // 128), dtype=torch.float32, device=dev)
+    for x in range(e):
+        mx.mx_quantize_bf16_to_e4m3_block128x128(prob.b[x].to(dev), q=qb[x], s=sb[x])
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    d = mx.mx_grouped_gemm_contiguous_tilewise(qa, sa, qb, sb, prob.offsets.to(dev), dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    qa_h, sa_h, qb_h, sb_h = qa.cpu().numpy(), sa.cpu().numpy(), qb.cpu().numpy(), sb.cpu().numpy()
+    offs = prob.offsets.numpy()
+    for x in range(e):
+        r0, r1 = int(offs[x]), int(offs[x + 1])
+        if r1 == r0:
+            continue
+        d_ref, absd = oracle.tw_gemm(qa_h[r0:r1], np.ascontiguousarray(sa_h[:, r0:r1]), qb_h[x], sb_h[x])
+        assert_gemm_close(to_np_f64(d[r0:r1]), d_ref, absd, f"tile-wise contiguous expert {x}")
