@@ -789,8 +789,8 @@ def run_reference(args, world, rank):
 # the sources each kind of MXFP8 kernel is built from (a traffic figure stays
 # valid while these files are unchanged)
 KERNEL_SOURCES = {
-    "quant": ["mx_quant.cu", "mx_fastdiv.h", "mx_launch.h"],
-    "gemm": ["mx_gemm.cu", "mx_gemm2.cu", "mx_gemm_common.cuh", "mx_ptx.cuh", "mx_mxfp8.cuh", "mx_launch.h"],
+    "quant": ["mx_quant.cu", "mx_mxfp8.cuh", "mx_fastdiv.h"],
+    "gemm": ["mx_gemm.cu", "mx_gemm2.cu", "mx_gemm_common.cuh", "mx_ptx.cuh", "mx_mxfp8.cuh"],
 }
 
 
