@@ -171,11 +171,13 @@ __device__ __forceinline__ uint32_t* scale_word(const PlaceArgs& a, int64_t r, u
   return reinterpret_cast<uint32_t*>(a.sf + off);
 }
 
-// One warp per source row (QUANT: quantise the BF16 token's 32-element
-// blocks, one per lane, with the quantiser's rule; else copy E4M3 row and
-// scales), the row then written to each of its `fan` destinations; the warps
-// after the last source row clear the group padding rows (E4M3 0, scale 0:
-// the quantisation of a zero row).
+// One warp per (source row, chunk of 32 blocks = 1024 elements): QUANT
+// quantises the BF16 token's blocks, one per lane, with the quantiser's rule;
+// else it copies the E4M3 bytes and scales.  The chunk is then written to each
+// of the row's `fan` destinations.  The warps after the last source chunk
+// clear the group padding rows (E4M3 0, scale 0: the quantisation of a zero
+// row), one (padding slot, chunk) each.  Splitting rows into chunks keeps
+// enough warps in flight when there are few tokens.
 template <bool QUANT>
 __global__ void __launch_bounds__(kRowWarps * 32) moe_place_kernel(const PlaceArgs a) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -183,48 +185,68 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_place_kernel(const PlaceAr
   const int lane = threadIdx.x & 31;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
   const uint32_t kb = static_cast<uint32_t>(a.k / 32);
-  if (w < a.n_src) {
-    for (uint32_t b0 = 0; b0 < kb; b0 += 32) {
-      const uint32_t b = b0 + lane;
-      const bool on = b < kb;  // kb % 4 == 0: each group of 4 lanes is all on or all off
-      uint4 out0 = make_uint4(0, 0, 0, 0), out1 = out0;
-      uint32_t scode = 0;
-      if (QUANT) {
-        uint4 v[4];
-        const uint4* src = static_cast<const uint4*>(a.src) + (w * kb + b) * 4;
+  const int64_t chunks = (kb + 31) / 32;
+  const int64_t src_units = a.n_src * chunks;
+  if (w < src_units) {
+    const int64_t src = w / chunks;
+    const uint32_t b = static_cast<uint32_t>(w - src * chunks) * 32 + lane;
+    const bool on = b < kb;  // kb % 4 == 0: each group of 4 lanes is all on or all off
+    uint4 out0 = make_uint4(0, 0, 0, 0), out1 = out0;
+    uint32_t scode = 0;
+    if (QUANT) {
+      uint4 v[4];
+      const uint4* sp = static_cast<const uint4*>(a.src) + (src * kb + b) * 4;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = on ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
-        scode = quant_block32_bf16(v, out0, out1);
-      } else if (on) {
-        const uint4* src = static_cast<const uint4*>(a.src) + (w * kb + b) * 2;
-        out0 = __ldcs(src);
-        out1 = __ldcs(src + 1);
-        scode = a.src_sf[w * kb + b];
+      for (int j = 0; j < 4; ++j) v[j] = on ? __ldcs(sp + j) : make_uint4(0, 0, 0, 0);
+      scode = quant_block32_bf16(v, out0, out1);
+    } else if (on) {
+      const uint4* sp = static_cast<const uint4*>(a.src) + (src * kb + b) * 2;
+      out0 = __ldcs(sp);
+      out1 = __ldcs(sp + 1);
+      scode = a.src_sf[src * kb + b];
+    }
+    const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, scode, 1);
+    const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, scode, 2);
+    const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, scode, 3);
+    const uint32_t word = scode | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    // rearrange so each store instruction writes 512 contiguous bytes: bytes
+    // [16l, 16l + 16) of the chunk's first (second) 512 are half l & 1 of
+    // block l >> 1 (16 + (l >> 1))
+    const int sa = lane >> 1, sb = 16 + (lane >> 1);
+    const bool hi = lane & 1;
+    uint4 st0, st1;
+    {
+      const uint4 x0 = make_uint4(__shfl_sync(0xFFFFFFFFu, out0.x, sa), __shfl_sync(0xFFFFFFFFu, out0.y, sa),
+                                  __shfl_sync(0xFFFFFFFFu, out0.z, sa), __shfl_sync(0xFFFFFFFFu, out0.w, sa));
+      const uint4 x1 = make_uint4(__shfl_sync(0xFFFFFFFFu, out1.x, sa), __shfl_sync(0xFFFFFFFFu, out1.y, sa),
+                                  __shfl_sync(0xFFFFFFFFu, out1.z, sa), __shfl_sync(0xFFFFFFFFu, out1.w, sa));
+      const uint4 y0 = make_uint4(__shfl_sync(0xFFFFFFFFu, out0.x, sb), __shfl_sync(0xFFFFFFFFu, out0.y, sb),
+                                  __shfl_sync(0xFFFFFFFFu, out0.z, sb), __shfl_sync(0xFFFFFFFFu, out0.w, sb));
+      const uint4 y1 = make_uint4(__shfl_sync(0xFFFFFFFFu, out1.x, sb), __shfl_sync(0xFFFFFFFFu, out1.y, sb),
+                                  __shfl_sync(0xFFFFFFFFu, out1.z, sb), __shfl_sync(0xFFFFFFFFu, out1.w, sb));
+      st0 = hi ? x1 : x0;
+      st1 = hi ? y1 : y0;
+    }
+    const uint32_t b0 = b - lane;  // first block of the chunk
+    const bool on0 = b0 + sa < kb, on1 = b0 + sb < kb;
+    for (int j = 0; j < a.fan; ++j) {
+      const int32_t r = a.row[src * a.fan + j];
+      if (r < 0) continue;  // a dropped entry
+      if (r >= a.m_rows) {
+        if (lane == 0) moe_report(a.status, kDevBadIndex);
+        continue;
       }
-      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, scode, 1);
-      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, scode, 2);
-      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, scode, 3);
-      const uint32_t word = scode | (s1 << 8) | (s2 << 16) | (s3 << 24);
-      for (int j = 0; j < a.fan; ++j) {
-        const int32_t r = a.row[w * a.fan + j];
-        if (r < 0) continue;  // a dropped entry
-        if (r >= a.m_rows) {
-          if (lane == 0 && b0 == 0) moe_report(a.status, kDevBadIndex);
-          continue;
-        }
-        if (on) {
-          uint4* dst = reinterpret_cast<uint4*>(a.q) + (static_cast<int64_t>(r) * kb + b) * 2;
-          dst[0] = out0;
-          dst[1] = out1;
-          if ((lane & 3) == 0) *scale_word(a, r, b, kb) = word;
-        }
-      }
+      uint4* dst = reinterpret_cast<uint4*>(a.q) + (static_cast<int64_t>(r) * kb + b0) * 2;
+      if (on0) dst[lane] = st0;
+      if (on1) dst[32 + lane] = st1;
+      if (on && (lane & 3) == 0) *scale_word(a, r, b, kb) = word;
     }
     return;
   }
-  // padding rows
+  // padding rows, one (slot, chunk) per warp
   if (a.E == 0 || a.pad_slots == 0) return;
-  const int64_t p = w - a.n_src;
+  const int64_t p = (w - src_units) / chunks;
+  const uint32_t c = static_cast<uint32_t>((w - src_units) - p * chunks);
   const int e = static_cast<int>(p / a.pad_slots);
   if (e >= a.E) return;
   const int s = static_cast<int>(p - static_cast<int64_t>(e) * a.pad_slots);
@@ -234,9 +256,13 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_place_kernel(const PlaceAr
     if (lane == 0) moe_report(a.status, kDevBadIndex);
     return;
   }
-  uint4* dst = reinterpret_cast<uint4*>(a.q + r * a.k);
-  for (int i = lane; i < a.k / 16; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
-  for (uint32_t c = 4 * lane; c < kb; c += 128) *scale_word(a, r, c, kb) = 0;
+  const uint32_t b = c * 32 + lane;
+  if (b < kb) {
+    uint4* dst = reinterpret_cast<uint4*>(a.q) + (r * kb + b) * 2;
+    dst[0] = make_uint4(0, 0, 0, 0);
+    dst[1] = make_uint4(0, 0, 0, 0);
+    if ((lane & 3) == 0) *scale_word(a, r, b, kb) = 0;
+  }
 }
 
 // ------------------------------------------------------------------ row gather
@@ -264,8 +290,9 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_gather_kernel(const uint4*
 
 // ------------------------------------------------------------------ combine
 // out[t, :] = sum_j w[t, j] * y[row[t*topk + j], :], FP32 fused multiply-adds
-// in j order, rounded once to BF16 (RNE).  One warp per token, 8 columns (one
-// 16-byte vector) per lane per step, four routed rows' loads in flight.
+// in j order, rounded once to BF16 (RNE).  One warp per (token, chunk of 256
+// columns): 8 columns (one 16-byte vector) per lane, four routed rows' loads
+// in flight.
 __global__ void __launch_bounds__(kRowWarps * 32) moe_combine_kernel(const uint4* __restrict__ y, int64_t y_rows,
                                                                      int64_t n_vecs, const int32_t* __restrict__ row,
                                                                      const float* __restrict__ wt, int64_t tokens,
@@ -274,12 +301,15 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_combine_kernel(const uint4
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  const int64_t chunks = (n_vecs + 31) / 32;
+  const int64_t t = w / chunks;
   if (t >= tokens) return;
+  const int64_t c = (w - t * chunks) * 32 + lane;
   const int32_t* rt = row + t * topk;
   const float* wt_t = wt + t * topk;
   bool bad = false;
-  for (int64_t c = lane; c < n_vecs; c += 32) {
+  if (c < n_vecs) {
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
@@ -369,7 +399,8 @@ cudaError_t launch_moe_place(const MoePlace& p, cudaStream_t stream) {
   a.E = p.pad > 1 ? p.experts : 0;
   a.pad_slots = p.pad > 1 ? p.pad - 1 : 0;
   a.sf_row_major = p.sf_row_major;
-  const int64_t warps = p.n_src + static_cast<int64_t>(a.E) * a.pad_slots;
+  const int64_t chunks = (p.k / 32 + 31) / 32;
+  const int64_t warps = (p.n_src + static_cast<int64_t>(a.E) * a.pad_slots) * chunks;
   if (warps == 0) return cudaSuccess;
   const int64_t grid = (warps + kRowWarps - 1) / kRowWarps;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
@@ -395,7 +426,8 @@ cudaError_t launch_moe_gather(const void* src, int64_t src_rows, int64_t row_byt
 cudaError_t launch_moe_combine(const void* y, int64_t y_rows, int64_t n_cols, const int32_t* row, const float* w,
                                int64_t tokens, int topk, void* out, int32_t* status, cudaStream_t stream) {
   if (tokens == 0) return cudaSuccess;
-  const int64_t grid = (tokens + kRowWarps - 1) / kRowWarps;
+  const int64_t warps = tokens * ((n_cols / 8 + 31) / 32);
+  const int64_t grid = (warps + kRowWarps - 1) / kRowWarps;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
   const uint4* yp = static_cast<const uint4*>(y);
   uint4* op = static_cast<uint4*>(out);

@@ -134,10 +134,25 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_co
       const uint32_t b = base + u * 32 + lane;
       uint4 out0, out1;
       const uint32_t scode = quant_block32_bf16(v[u], out0, out1);
-      if (b < jb.nblk) {
-        uint4* dst = jb.q + static_cast<size_t>(b) * 2;
-        __stcs(dst, out0);
-        __stcs(dst + 1, out1);
+      // the warp's 32 blocks are 1 KB of contiguous output: rearrange it so
+      // each store instruction writes 512 contiguous bytes (bytes
+      // [16l, 16l + 16) of the first / second half are half l & 1 of block
+      // l >> 1 / 16 + (l >> 1))
+      {
+        const int sa = lane >> 1, sb = 16 + (lane >> 1);
+        const bool hi = lane & 1u;
+        const uint4 x0 = make_uint4(__shfl_sync(0xFFFFFFFFu, out0.x, sa), __shfl_sync(0xFFFFFFFFu, out0.y, sa),
+                                    __shfl_sync(0xFFFFFFFFu, out0.z, sa), __shfl_sync(0xFFFFFFFFu, out0.w, sa));
+        const uint4 x1 = make_uint4(__shfl_sync(0xFFFFFFFFu, out1.x, sa), __shfl_sync(0xFFFFFFFFu, out1.y, sa),
+                                    __shfl_sync(0xFFFFFFFFu, out1.z, sa), __shfl_sync(0xFFFFFFFFu, out1.w, sa));
+        const uint4 y0 = make_uint4(__shfl_sync(0xFFFFFFFFu, out0.x, sb), __shfl_sync(0xFFFFFFFFu, out0.y, sb),
+                                    __shfl_sync(0xFFFFFFFFu, out0.z, sb), __shfl_sync(0xFFFFFFFFu, out0.w, sb));
+        const uint4 y1 = make_uint4(__shfl_sync(0xFFFFFFFFu, out1.x, sb), __shfl_sync(0xFFFFFFFFu, out1.y, sb),
+                                    __shfl_sync(0xFFFFFFFFu, out1.z, sb), __shfl_sync(0xFFFFFFFFu, out1.w, sb));
+        const uint32_t b0 = base + u * 32;
+        uint4* dst = jb.q + static_cast<size_t>(b0) * 2;
+        if (b0 + sa < jb.nblk) __stcs(dst + lane, hi ? x1 : x0);
+        if (b0 + sb < jb.nblk) __stcs(dst + 32 + lane, hi ? y1 : y0);
       }
 
       // scale byte(s): row / K-block of this block, then its group
