@@ -1,4 +1,4 @@
-"""Expert parallelism on two gloo ranks (CPU): the layer's multi-rank
+"""Expert parallelism on two and four gloo ranks (CPU): the layer's multi-rank
 plumbing (per-expert count exchange, the row all-to-alls with uneven and
 empty splits, the receive-side plan, the return path and the combine) gives
 exactly the output of the same layer computed in one process over all
@@ -18,7 +18,7 @@ import torch.multiprocessing as mp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 TESTS = os.path.dirname(os.path.abspath(__file__))
 
-E, TOPK, H, I, N = 4, 2, 128, 128, 96
+TOPK, H, I, N = 2, 128, 128, 96
 
 
 def _free_port():
@@ -29,19 +29,21 @@ def _free_port():
     return port
 
 
-def _problem(case: str):
-    """Per-rank tokens, routing and gate weights, and the global experts."""
+def _problem(case: str, world: int):
+    """Per-rank tokens, routing and gate weights, and the global experts (two
+    per rank)."""
     sys.path[:0] = [ROOT, TESTS]
     import mx_inputs
     import oracle
+    E = 2 * world
     ranks = []
-    for r in range(2):
+    for r in range(world):
         T = 40 + 13 * r
         x = mx_inputs.normal_bf16((T, H), 1.0, 100 + r)
         ids = mx_inputs.topk_ids(T, TOPK, E, seed=200 + r)
         if case == "skewed":
             if r == 1:
-                ids = ids % 2 + 2            # rank 1 sends nothing to rank 0's experts
+                ids = ids % 2 + 2            # rank 1 sends nothing to rank 0's experts (nor rank 2's, ...)
             ids[3, 1] = -1                   # a dropped entry
         gw = mx_inputs.gate_weights(T, TOPK, seed=300 + r)
         ranks.append((x, ids, gw))
@@ -51,7 +53,7 @@ def _problem(case: str):
     q2, sf2 = oracle.quantize(w2)
     experts = (q13.reshape(E, 2 * I, H), sf13.reshape(E, 2 * I, H // 32),
                q2.reshape(E, N, I), sf2.reshape(E, N, I // 32))
-    return ranks, experts
+    return ranks, experts, E
 
 
 def _rank_main(rank, world, port, case, out):
@@ -62,7 +64,7 @@ def _rank_main(rank, world, port, case, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
     try:
-        ranks, (q13, sf13, q2, sf2) = _problem(case)
+        ranks, (q13, sf13, q2, sf2), E = _problem(case, world)
         x, ids, gw = ranks[rank]
         lo, hi = rank * (E // world), (rank + 1) * (E // world)
         y = ep_moe_layer(x, torch.from_numpy(ids), torch.from_numpy(gw), E,
@@ -82,22 +84,24 @@ def _library():
         __graft_entry__.build()
 
 
-@pytest.mark.parametrize("case", ["uniform", "skewed"])
-def test_ep_two_ranks_matches_one_process(case):
+@pytest.mark.parametrize("world,case", [(2, "uniform"), (2, "skewed"), (4, "skewed")])
+def test_ep_ranks_match_one_process(world, case):
     from ep_ref_ops import OracleOps
     from moe_grouped_gemm_mx_b200.ep import ep_moe_layer
     port = _free_port()
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.spawn(_rank_main, args=(2, port, case, out), nprocs=2, join=True)
-    ranks, (q13, sf13, q2, sf2) = _problem(case)
+    mp.spawn(_rank_main, args=(world, port, case, out), nprocs=world, join=True)
+    ranks, (q13, sf13, q2, sf2), E = _problem(case, world)
     x = torch.cat([r[0] for r in ranks])
     ids = torch.from_numpy(np.concatenate([r[1] for r in ranks]))
     gw = torch.from_numpy(np.concatenate([r[2] for r in ranks]))
     ref = ep_moe_layer(x, ids, gw, E, torch.from_numpy(q13), torch.from_numpy(sf13), torch.from_numpy(q2),
                        torch.from_numpy(sf2), ops=OracleOps())
     ref_bits = ref.view(torch.int16).numpy()
-    t0 = ranks[0][0].shape[0]
-    assert np.array_equal(out[0], ref_bits[:t0])
-    assert np.array_equal(out[1], ref_bits[t0:])
+    t0 = 0
+    for r in range(world):
+        t1 = t0 + ranks[r][0].shape[0]
+        assert np.array_equal(out[r], ref_bits[t0:t1]), f"rank {r}"
+        t0 = t1
     assert np.abs(ref.float().numpy()).max() > 0      # the layer produced something
