@@ -22,6 +22,7 @@
 
 #include "mx_launch.h"
 #include "mx_mxfp8.cuh"
+#include "mx_ptx.cuh"
 
 namespace mxk {
 
@@ -32,20 +33,31 @@ constexpr int kDevBadIndex = 0x8;
 __device__ __forceinline__ void moe_report(int32_t* status, int bits) { atomicOr(status, bits); }
 
 // ------------------------------------------------------------------ routing plan
-// One CTA of 32 warps: the plan is a prefix over all entries, and the table
-// (8192 tokens x top-8 = 64K entries) is small next to the GEMMs it feeds.
-// Warp w owns the contiguous segment [w*seg, (w+1)*seg) of the entries, so
-// entry order is (warp, position in segment).
-//  1. each warp streams its segment 32 entries per step (four steps' loads in
-//     flight): a lane's rank among the step's entries of its expert comes
-//     from __match_any_sync, the warp's running count of that expert from its
-//     own row of a [32][E] shared-memory table; the rank within the segment
-//     is parked in row[i];
-//  2. one thread per expert turns its column of the table into exclusive
-//     per-warp prefixes and a total; a block scan over the padded totals
-//     gives the group offsets;
-//  3. each warp adds offset + warp prefix to the parked ranks (coalesced).
+// A cluster of kRouteCluster CTAs of 32 warps; CTA c owns the contiguous
+// segment c of the entries and warp w of it a contiguous sub-segment, so entry
+// order is (CTA, warp, position).
+//  1. each warp streams its sub-segment 32 entries per step (four steps'
+//     loads in flight): a lane's rank among the step's entries of its expert
+//     comes from __match_any_sync, the warp's running count of that expert
+//     from its own row of a [32][E] shared-memory table; the rank within the
+//     sub-segment is parked in row[i];
+//  2. one thread per expert turns its column into exclusive per-warp
+//     prefixes and the CTA's total; after a cluster barrier each CTA reads
+//     the other CTAs' totals through distributed shared memory (the earlier
+//     CTAs' sum is its base, all of them the expert's count), and a block
+//     scan over the padded counts gives the group offsets (the same in every
+//     CTA; CTA 0 writes them out);
+//  3. each warp adds offset + CTA base + warp prefix to its parked ranks.
+// A second cluster barrier keeps every CTA resident until its peers have
+// read its totals.
 constexpr int kRouteUnroll = 4;
+constexpr int kRouteCluster = 8;
+
+__device__ __forceinline__ int32_t ld_cluster_s32(uint32_t addr) {
+  int32_t v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t* __restrict__ ids, int n, int E,
                                                                   int pad, int32_t* __restrict__ counts,
@@ -56,17 +68,22 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
   asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ int32_t route_smem[];
   int32_t* wc = route_smem;          // [32][E] per-warp counts, then per-warp exclusive prefixes
-  int32_t* base = wc + 32 * E;       // [E] group offsets
+  int32_t* tot = wc + 32 * E;        // [E] this CTA's count per expert (read by the other CTAs)
+  int32_t* base = tot + E;           // [E] group offset + earlier CTAs' counts
   int32_t* wsum = base + E;          // [32] warp totals of the scan
-  int32_t* nbad = wsum + 32;         // [1]
+  int32_t* nbad = wsum + 32;         // [1] dropped entries of this CTA (read by CTA 0)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int crank = static_cast<int>(cluster_ctarank());
   for (int i = tid; i < 32 * E; i += blockDim.x) wc[i] = 0;
   if (tid == 0) *nbad = 0;
   __syncthreads();
 
-  const int seg = (n + 31) / 32;
-  const int begin = warp * seg;
-  const int end = min(n, begin + seg);
+  const int cseg = (n + kRouteCluster - 1) / kRouteCluster;
+  const int cbeg = min(n, crank * cseg);
+  const int cend = min(n, cbeg + cseg);
+  const int seg = (cend - cbeg + 31) / 32;
+  const int begin = min(cend, cbeg + warp * seg);
+  const int end = min(cend, begin + seg);
   const uint32_t lower = (1u << lane) - 1u;
   int32_t* my = wc + warp * E;
   int bad = 0;
@@ -100,15 +117,34 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
   if (bad) atomicAdd(nbad, bad);
   __syncthreads();
 
-  int total = 0;
   if (tid < E) {
+    int t = 0;
     for (int w = 0; w < 32; ++w) {
       const int c = wc[w * E + tid];
-      wc[w * E + tid] = total;
-      total += c;
+      wc[w * E + tid] = t;
+      t += c;
+    }
+    tot[tid] = t;
+  }
+  cluster_arrive_release();  // every CTA's totals are written ...
+  cluster_wait_acquire();    // ... and visible cluster-wide
+  int pre = 0, all = 0;
+  if (tid < E) {
+    const uint32_t a = smem_u32(tot + tid);
+    for (int c = 0; c < kRouteCluster; ++c) {
+      const int v = c == crank ? tot[tid] : ld_cluster_s32(map_to_rank(a, c));
+      if (c < crank) pre += v;
+      all += v;
     }
   }
-  const int v = tid < E ? (total + pad - 1) / pad * pad : 0;
+  int nbad_all = 0;
+  if (crank == 0 && tid == 0) {
+    const uint32_t a = smem_u32(nbad);
+    for (int c = 0; c < kRouteCluster; ++c) nbad_all += c == 0 ? *nbad : ld_cluster_s32(map_to_rank(a, c));
+  }
+  cluster_arrive_release();  // done reading the other CTAs' shared memory
+
+  const int v = tid < E ? (all + pad - 1) / pad * pad : 0;
   int incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -130,12 +166,14 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
   __syncthreads();
   const int excl = incl - v + wsum[warp];
   if (tid < E) {
-    counts[tid] = total;
-    offsets[tid] = excl;
-    base[tid] = excl;
-    if (tid == E - 1) offsets[E] = excl + v;
+    base[tid] = excl + pre;
+    if (crank == 0) {
+      counts[tid] = all;
+      offsets[tid] = excl;
+      if (tid == E - 1) offsets[E] = excl + v;
+    }
   }
-  if (tid == 0 && dropped != nullptr) *dropped = *nbad;
+  if (crank == 0 && tid == 0 && dropped != nullptr) *dropped = nbad_all;
   __syncthreads();
 
   for (int i = begin + lane; i < end; i += 32) {
@@ -144,6 +182,7 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
     const int e = __ldg(ids + i);
     row[i] = base[e] + my[e] + r;
   }
+  cluster_wait_acquire();  // peers may still read this CTA's totals until here
 }
 
 // ------------------------------------------------------------------ dispatch / scatter
@@ -371,15 +410,30 @@ static cudaError_t launch_pdl_cfg(const void* func, dim3 grid, dim3 block, size_
 
 cudaError_t launch_moe_route(const int32_t* ids, int64_t n, int E, int pad, int32_t* counts, int32_t* offsets,
                              int32_t* row, int32_t* dropped, cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(33 * E + 33) * 4;  // at most 135 KB (E = 1024)
+  const size_t smem = static_cast<size_t>(34 * E + 33) * 4;  // at most 139 KB (E = 1024)
   static cudaError_t attr = cudaErrorNotReady;
   if (attr == cudaErrorNotReady)
-    attr = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * 1024 * 4 + 33 * 4);
+    attr = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 34 * 1024 * 4 + 33 * 4);
   if (attr != cudaSuccess) return attr;
   int ni = static_cast<int>(n);
   void* args[] = {&ids, &ni, &E, &pad, &counts, &offsets, &row, &dropped};
-  return launch_pdl_cfg(reinterpret_cast<const void*>(moe_route_kernel), dim3(1), dim3(kRouteThreads), smem, args,
-                        stream);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[2];
+  cfg.gridDim = dim3(kRouteCluster);
+  cfg.blockDim = dim3(kRouteThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = kRouteCluster;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(moe_route_kernel), args);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_moe_place(const MoePlace& p, cudaStream_t stream) {
