@@ -7,9 +7,10 @@
 //
 // Kernel design (HBM-bound: 2 B read, 1 + 1/32 B written per element):
 //  * The [rows, K] source is contiguous, so 32-element block b is the 64-byte
-//    chunk at byte 64*b regardless of row boundaries.  One lane owns one
-//    block (four 16-byte loads), a warp 32 consecutive blocks (2 KiB), and
-//    every thread keeps two blocks' loads in flight.  One lane per block keeps
+//    chunk at byte 64*b regardless of row boundaries.  A warp loads 32
+//    consecutive blocks (2 KiB) with four coalesced 16-byte loads per lane,
+//    two such steps in flight, staged through swizzled shared memory; then
+//    one lane owns one block.  One lane per block keeps
 //    the per-element instruction count low: amax, exponent and the scale
 //    address are computed once per 32 elements.
 //  * amax is reduced on the integer magnitude bits (bits & 0x7fff, two BF16
@@ -92,6 +93,7 @@ __device__ void write_padding(const QuantJob& jb, int64_t i) {
 }
 
 __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_constant__ QuantBatch B) {
+  __shared__ uint4 quant_stage[(kQuantThreads / 32) * kQuantUnroll * 128];  // 2 KiB per warp and step
   // with programmatic dependent launch the next kernel may start its
   // prologue now; our own reads and writes wait for the previous kernel
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -121,14 +123,43 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_co
     const QuantJob& jb = B.job[jn];
     const uint32_t base = (slot - jb.slot0) * kSlotBlocks;
 
+    // Coalesced loads: instruction j of step u brings the 16-byte piece
+    // 32j + lane of the step's 2 KiB (512 contiguous bytes per instruction);
+    // the pieces go through a per-warp shared-memory stage, swizzled (piece
+    // p at slot p ^ ((p >> 3) & 7)) so that both the writes here and each
+    // lane's read of its own block's four pieces below are free of bank
+    // conflicts.
+    uint4* stage = quant_stage + (threadIdx.x >> 5) * (kQuantUnroll * 128);
+    {
+      uint4 g[kQuantUnroll][4];
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u) {
+        const uint32_t b0 = base + u * 32;  // first block of the step
+        const uint4* src = jb.x + static_cast<size_t>(b0) * 4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t p = 32 * j + lane;  // piece p belongs to block b0 + p / 4
+          g[u][j] = b0 + (p >> 2) < jb.nblk ? __ldcs(src + p) : make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kQuantUnroll; ++u)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t p = 32 * j + lane;
+          stage[u * 128 + (p ^ ((p >> 3) & 7u))] = g[u][j];
+        }
+    }
+    __syncwarp();
     uint4 v[kQuantUnroll][4];
 #pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u) {
-      const uint32_t b = base + u * 32 + lane;
-      const uint4* src = jb.x + static_cast<size_t>(b) * 4;
+    for (int u = 0; u < kQuantUnroll; ++u)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) v[u][j] = b < jb.nblk ? __ldcs(src + j) : make_uint4(0, 0, 0, 0);
-    }
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t p = 4 * lane + q;
+        v[u][q] = stage[u * 128 + (p ^ ((p >> 3) & 7u))];
+      }
+    __syncwarp();  // the stage is rewritten by the warp's next slot
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const uint32_t b = base + u * 32 + lane;
