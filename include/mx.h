@@ -320,7 +320,8 @@ mx_status mx_moe_route(const int32_t *ids, int64_t n, int32_t experts, int32_t p
  * mx_moe_route with the same pad) are set to the quantisation of a zero row
  * (E4M3 0x00, scale 0x00).  k % 128 == 0; m_rows % 128 == 0 for the tiled
  * layout; 16-byte aligned x, q and sf.  A row >= m_rows is skipped and sets
- * MX_DEV_BAD_INDEX. */
+ * MX_DEV_BAD_INDEX.  The rows of different entries must be distinct (as
+ * mx_moe_route makes them); two entries sharing a row leave either one's data. */
 mx_status mx_moe_dispatch_quant(const void *x_bf16, int64_t tokens, int64_t k, const int32_t *row, int32_t topk,
                                 const int32_t *counts, const int32_t *offsets, int32_t experts, int32_t pad,
                                 int64_t m_rows, void *q_e4m3, void *sf, int32_t sf_row_major,
