@@ -143,6 +143,7 @@ mx_status mx_quantize_bf16_to_e4m3_transposed(const void* x_bf16, int64_t groups
     return MX_ERR_UNSUPPORTED_SHAPE;
   return from_cuda(mxk::launch_quant_transposed(x_bf16, groups, rows, cols, q_e4m3, sf_ue8m0,
                                                 static_cast<int64_t>(mx_scale_bytes(cols, rows)),
+                                                internal_status_ptr(), num_sms(),
                                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -21,7 +21,7 @@ cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, c
 // Quantisation along the rows of x [groups, rows, cols] into q [groups, cols,
 // rows] with per-group tiled scales of the [cols, rows] operand.
 cudaError_t launch_quant_transposed(const void* x, int64_t groups, int64_t rows, int64_t cols, void* q, void* sf,
-                                    int64_t sf_group_bytes, cudaStream_t stream);
+                                    int64_t sf_group_bytes, int32_t* status, int num_sms, cudaStream_t stream);
 
 struct GemmProblem {
   const void* qa;
