@@ -151,3 +151,25 @@ def test_tilewise_gemm_contiguous_ragged(mx, oracle):
             continue
         d_ref, absd = oracle.tw_gemm(qa_h[r0:r1], np.ascontiguousarray(sa_h[:, r0:r1]), qb_h[x], sb_h[x])
         assert_gemm_close(to_np_f64(d[r0:r1]), d_ref, absd, f"tile-wise contiguous expert {x}")
+
+
+@pytest.mark.parametrize("blocks", [False, True])
+def test_tilewise_quant_midpoints_and_tiny_scales(mx, oracle, blocks):
+    """Rounding corner cases of x / s: tiles scaled so that s = 1 exactly
+    with elements on E4M3 rounding midpoints (ties to even), tiles of BF16
+    subnormals (a subnormal FP32 scale), and rows spread over many binades,
+    plus a large random matrix."""
+    g = torch.Generator().manual_seed(77)
+    rows, k = 256, 512
+    x = torch.randn(rows, k, generator=g)
+    mids = torch.tensor([1.0625, 1.1875, 1.3125, 1.4375, 1.5625, 1.6875, 1.8125, 1.9375,
+                         0.0029296875, 0.0048828125, 0.0009765625, 0.001953125 * 1.5])
+    for r in range(0, 128):                       # amax 448 in every 128x128 block and 1x128 tile
+        x[r] = mids[torch.randint(0, len(mids), (k,), generator=g)] * (2.0 ** torch.randint(-6, 8, (k,), generator=g))
+        x[r, ::128] = 448.0
+    x[128:160] = torch.randn(32, k, generator=g) * 1e-39  # BF16 subnormals: a tiny scale
+    x[160] = torch.randn(k, generator=g) * (2.0 ** torch.randint(-30, 30, (k,), generator=g).float())
+    x = x.to(torch.bfloat16)
+    check_quant(mx, oracle, x, blocks)
+    big = torch.randn(2048, 1024, generator=g).to(torch.bfloat16)
+    check_quant(mx, oracle, big, blocks)
