@@ -30,6 +30,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <cstdlib>
 
 #include "mx_gemm_common.cuh"
 #include "mx_launch.h"
@@ -59,6 +60,7 @@ struct TwLayout {
 };
 
 struct TwArgs {
+  __nv_bfloat16* d;              // [m, n] (written directly by the split-K form)
   const float* sa;               // [k_tiles, m]
   const float* sb;               // [groups, nb, k_tiles]
   const int32_t* group_offsets;  // contiguous form: [groups + 1]
@@ -66,10 +68,36 @@ struct TwArgs {
   int m, n, k_tiles, n_tiles, groups, mode;  // mode 0 dense, 1 contiguous
 };
 
+// Split-K reduction buffer (reuses the operand ring after the mainloop):
+// SPLIT partial slices of 128 rows x 128/SPLIT FP32 columns, in quads of 4
+// columns; CTA o owns quads [ceil(o*32/SPLIT), ceil((o+1)*32/SPLIT)).
+// [source rank][quad of the slice][row] float4, rows fastest: the 32 lanes of
+// a warp (32 consecutive rows) write 512 contiguous bytes per remote store.
+template <int SPLIT>
+struct TwSplit {
+  static constexpr int QUADS = 32;
+  static constexpr int MAX_SLICE_QUADS = (QUADS + SPLIT - 1) / SPLIT;
+  static constexpr int RED_BYTES = SPLIT * MAX_SLICE_QUADS * BM * 16;
+  __host__ __device__ static constexpr int slice_start(int o) { return (o * QUADS + SPLIT - 1) / SPLIT; }
+  __host__ __device__ static constexpr int quad_owner(int q) { return (q * SPLIT) / QUADS; }
+  static_assert(RED_BYTES <= TwLayout::OFF_STG, "reduction buffer must fit in the operand ring");
+};
+
+// SPLIT > 1 (dense form only): a cluster of SPLIT CTAs shares one output
+// tile, each CTA promoting a contiguous share of the K tiles into its
+// registers; the FP32 sums are then exchanged through distributed shared
+// memory (each CTA sums one column slice over the cluster in rank order --
+// deterministic -- and stores it as BF16).
+template <int SPLIT>
 __global__ void __launch_bounds__(kTwThreads, 1)
     mx_gemm_tw_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_d, const TwArgs args) {
   using L = TwLayout;
+  using RS = TwSplit<SPLIT>;
+  const int split_rank = SPLIT > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT : static_cast<int>(blockIdx.x);
+  const int kt_begin = SPLIT > 1 ? split_rank * args.k_tiles / SPLIT : 0;
+  const int kt_end = SPLIT > 1 ? (split_rank + 1) * args.k_tiles / SPLIT : args.k_tiles;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -154,16 +182,22 @@ __global__ void __launch_bounds__(kTwThreads, 1)
     }
   };
 
+  // the promotion warps' FP32 accumulators (one 128-column tile row per
+  // thread); at function scope so the split-K exchange below can send them
+  float acc[128];
+  const int quarter = warp & 3;
+  const int r_local = quarter * 32 + lane;
+
   if (warp == 0) {
     if (lane == 0) {
       // ===== TMA producer
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
         int group, m_blk, n_blk;
         decode(t, group, m_blk, n_blk);
-        for (int kt = 0; kt < args.k_tiles; ++kt) {
+        for (int kt = kt_begin; kt < kt_end; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), L::A_BYTES + L::B_BYTES);
           tma_load_3d(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, full_bar(stage), kt * BK, m_blk * BM, 0);
@@ -187,8 +221,8 @@ __global__ void __launch_bounds__(kTwThreads, 1)
       uint32_t phase = 0;
       uint32_t ib = 0;  // K tiles issued so far (partial buffer = ib % kTwBufs)
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        for (int kt = 0; kt < args.k_tiles; ++kt, ++ib) {
+      for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
+        for (int kt = kt_begin; kt < kt_end; ++kt, ++ib) {
           const uint32_t b = ib % kTwBufs;
           if (!mbar_wait(acce_bar(b), ((ib / kTwBufs) & 1u) ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
@@ -213,12 +247,10 @@ __global__ void __launch_bounds__(kTwThreads, 1)
     }
   } else {
     // ===== promotion and epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
-    const int quarter = warp & 3;
-    const int r_local = quarter * 32 + lane;
     uint32_t ib = 0;
     uint32_t stg_count = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
       int group, m_blk, n_blk;
       decode(t, group, m_blk, n_blk);
       const int row = m_blk * BM + r_local;
@@ -227,17 +259,17 @@ __global__ void __launch_bounds__(kTwThreads, 1)
       const float* sa_r = args.sa + row;
       auto sa_at = [&](int kt) { return row_ok ? __ldg(sa_r + static_cast<int64_t>(kt) * args.m) : 0.0f; };
       // the scales of K tile kt are loaded two K tiles ahead of their use
-      float sa0 = sa_at(0), sb0 = __ldg(sb_t);
-      float sa1 = args.k_tiles > 1 ? sa_at(1) : 0.0f, sb1 = args.k_tiles > 1 ? __ldg(sb_t + 1) : 0.0f;
-      float acc[128];
+      float sa0 = kt_begin < kt_end ? sa_at(kt_begin) : 0.0f, sb0 = kt_begin < kt_end ? __ldg(sb_t + kt_begin) : 0.0f;
+      float sa1 = kt_begin + 1 < kt_end ? sa_at(kt_begin + 1) : 0.0f;
+      float sb1 = kt_begin + 1 < kt_end ? __ldg(sb_t + kt_begin + 1) : 0.0f;
 #pragma unroll
       for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
-      for (int kt = 0; kt < args.k_tiles; ++kt, ++ib) {
+      for (int kt = kt_begin; kt < kt_end; ++kt, ++ib) {
         const uint32_t b = ib % kTwBufs;
         const float s = sa0 * sb0;
         sa0 = sa1;
         sb0 = sb1;
-        if (kt + 2 < args.k_tiles) {
+        if (kt + 2 < kt_end) {
           sa1 = sa_at(kt + 2);
           sb1 = __ldg(sb_t + kt + 2);
         }
@@ -269,6 +301,7 @@ __global__ void __launch_bounds__(kTwThreads, 1)
           }
         }
       }
+      if constexpr (SPLIT > 1) break;  // the split-K exchange below finishes the tile
       // one uniform decision per tile before the epilogue's 128-thread
       // barriers: a warp that gave up set abort_flag, which ends the other
       // warps' waits too, so every warp gets here
@@ -281,6 +314,57 @@ __global__ void __launch_bounds__(kTwThreads, 1)
     if (threadIdx.x == 64) bulk_wait_group_all();
   }
 
+  if constexpr (SPLIT > 1) {
+    // ---------------------------------------------------------- split-K exchange
+    // 1) every CTA of the cluster is past its mainloop, so every operand
+    //    ring is free to receive; 2) each promotion thread sends column slice
+    //    o of its row to CTA o; 3) each CTA sums the SPLIT partials of its
+    //    slice in rank order and stores BF16.  Every thread of every CTA
+    //    takes both cluster barriers, whatever happened before.
+    tc_fence_before();
+    cluster_sync();
+    const bool epi = warp >= 2 && t_first < total;
+    int m_blk = 0, n_blk = 0;
+    if (epi) {
+      int group;
+      decode(t_first, group, m_blk, n_blk);
+    }
+    const int row = m_blk * BM + r_local;
+    const bool valid = epi && row < args.m;
+    if (valid) {
+#pragma unroll
+      for (int q = 0; q < RS::QUADS; ++q) {
+        const int owner = RS::quad_owner(q);
+        const uint32_t local =
+            sbase + ((split_rank * RS::MAX_SLICE_QUADS + (q - RS::slice_start(owner))) * BM + r_local) * 16;
+        st_cluster_v4(map_to_rank(local, owner), __float_as_uint(acc[4 * q]), __float_as_uint(acc[4 * q + 1]),
+                      __float_as_uint(acc[4 * q + 2]), __float_as_uint(acc[4 * q + 3]));
+      }
+    }
+    cluster_sync();
+    if (valid && !*abort_flag) {
+      const float* red = reinterpret_cast<const float*>(smem);
+      __nv_bfloat16* drow = args.d + static_cast<int64_t>(row) * args.n;
+      const int q_begin = RS::slice_start(split_rank), q_end = RS::slice_start(split_rank + 1);
+#pragma unroll 1
+      for (int q = q_begin; q < q_end; ++q) {
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int src = 0; src < SPLIT; ++src) {
+          const float4 x =
+              *reinterpret_cast<const float4*>(red + ((src * RS::MAX_SLICE_QUADS + (q - q_begin)) * BM + r_local) * 4);
+          sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
+        }
+        const int col = n_blk * 128 + q * 4;
+        if (col < args.n) {
+          uint2 w;
+          w.x = pack_bf16x2(__float_as_uint(sum.x), __float_as_uint(sum.y));
+          w.y = pack_bf16x2(__float_as_uint(sum.z), __float_as_uint(sum.w));
+          *reinterpret_cast<uint2*>(drow + col) = w;
+        }
+      }
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -289,15 +373,44 @@ __global__ void __launch_bounds__(kTwThreads, 1)
   }
 }
 
+template <int SPLIT>
 static cudaError_t prepare_tw_kernel() {
   static cudaError_t state = cudaErrorNotReady;
   if (state == cudaErrorNotReady)
-    state = cudaFuncSetAttribute(mx_gemm_tw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TwLayout::ALLOC);
+    state = cudaFuncSetAttribute(mx_gemm_tw_kernel<SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 TwLayout::ALLOC);
   return state;
 }
 
-cudaError_t launch_gemm_tw(const TwProblem& p, int num_sms, cudaStream_t stream) {
-  cudaError_t e = prepare_tw_kernel();
+// How many clusters of SPLIT CTAs the GPU holds at once (0 if unknown).
+template <int SPLIT>
+static int tw_max_clusters() {
+  static int v = -1;
+  if (v < 0) {
+    v = 0;
+    if (prepare_tw_kernel<SPLIT>() == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      cfg.gridDim = dim3(SPLIT, 1, 1);
+      cfg.blockDim = dim3(kTwThreads, 1, 1);
+      cfg.dynamicSmemBytes = TwLayout::ALLOC;
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = SPLIT;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_tw_kernel<SPLIT>, &cfg) == cudaSuccess) v = n;
+      cudaGetLastError();
+    }
+  }
+  return v;
+}
+
+template <int SPLIT>
+static cudaError_t launch_tw(const TwProblem& p, int num_sms, cudaStream_t stream) {
+  cudaError_t e = prepare_tw_kernel<SPLIT>();
   if (e != cudaSuccess) return e;
   const int64_t b_depth = p.mode == kContiguous ? p.groups : 1;
   CUtensorMap ta, tb, td;
@@ -305,6 +418,7 @@ cudaError_t launch_gemm_tw(const TwProblem& p, int num_sms, cudaStream_t stream)
   if (!make_tmap(&tb, p.qb, p.k, p.n, b_depth, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_d(&td, p.d, p.n, p.m, 1)) return cudaErrorInvalidValue;
   TwArgs a = {};
+  a.d = static_cast<__nv_bfloat16*>(p.d);
   a.sa = p.sa;
   a.sb = p.sb;
   a.group_offsets = p.group_offsets;
@@ -318,18 +432,73 @@ cudaError_t launch_gemm_tw(const TwProblem& p, int num_sms, cudaStream_t stream)
   const int64_t tiles_bound = ((p.m + BM - 1) / BM) * a.n_tiles;
   if (tiles_bound == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles_bound < num_sms ? tiles_bound : num_sms), 1, 1);
+  cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(kTwThreads, 1, 1);
   cfg.dynamicSmemBytes = TwLayout::ALLOC;
   cfg.stream = stream;
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  if (SPLIT > 1) {  // one cluster of SPLIT CTAs per output tile
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_bound * SPLIT), 1, 1);
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = SPLIT;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl;
+    cfg.numAttrs = 2;
+  } else {
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_bound < num_sms ? tiles_bound : num_sms), 1, 1);
+    attr[0] = pdl;
+    cfg.numAttrs = 1;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, mx_gemm_tw_kernel, ta, tb, td, a);
+  e = cudaLaunchKernelEx(&cfg, mx_gemm_tw_kernel<SPLIT>, ta, tb, td, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+static int tw_max_clusters_of(int split) {
+  switch (split) {
+    case 2: return tw_max_clusters<2>();
+    case 4: return tw_max_clusters<4>();
+    case 8: return tw_max_clusters<8>();
+    default: return 0;
+  }
+}
+
+// Dense problems whose 128 x 128 tiles leave most SMs idle split K over a
+// cluster of 2, 4 or 8 CTAs: the largest split whose clusters all fit at once
+// with at least two K tiles per CTA.  MX_TW_SPLIT=1|2|4|8 forces one (tests).
+cudaError_t launch_gemm_tw(const TwProblem& p, int num_sms, cudaStream_t stream) {
+  static int forced = -2;
+  if (forced == -2) {
+    const char* env = getenv("MX_TW_SPLIT");
+    forced = env ? atoi(env) : -1;
+  }
+  const int64_t k_tiles = p.k / BK;
+  const int64_t tiles = ((p.m + BM - 1) / BM) * ((p.n + 127) / 128);
+  int split = 1;
+  if (p.mode != kContiguous) {
+    if (forced == 1 || forced == 2 || forced == 4 || forced == 8) {
+      if (k_tiles >= forced) split = forced;
+    } else if (tiles * 2 <= num_sms) {
+      const int order[3] = {8, 4, 2};
+      for (int i = 0; i < 3; ++i) {
+        const int sp = order[i];
+        if (tiles * sp <= num_sms && k_tiles >= 2 * sp && tiles <= tw_max_clusters_of(sp)) {
+          split = sp;
+          break;
+        }
+      }
+    }
+  }
+  switch (split) {
+    case 2: return launch_tw<2>(p, num_sms, stream);
+    case 4: return launch_tw<4>(p, num_sms, stream);
+    case 8: return launch_tw<8>(p, num_sms, stream);
+    default: return launch_tw<1>(p, num_sms, stream);
+  }
 }
 
 }  // namespace mxk

@@ -4,6 +4,11 @@ quantisers bit-exact (scales compared as FP32 bit patterns, NaN included),
 and the two-level-accumulation GEMM (TMEM partial per 128-element K tile,
 promoted with its scales in FP32) in dense and contiguous-grouped form within
 the GEMM tolerance."""
+import os
+import subprocess
+import sys
+import tempfile
+
 import numpy as np
 import pytest
 import torch
@@ -173,3 +178,59 @@ def test_tilewise_quant_midpoints_and_tiny_scales(mx, oracle, blocks):
     check_quant(mx, oracle, x, blocks)
     big = torch.randn(2048, 1024, generator=g).to(torch.bfloat16)
     check_quant(mx, oracle, big, blocks)
+
+
+# ---------------------------------------------------------------- split-K over a cluster
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+# ragged M and N, K tiles not a multiple of the split (9 over 2/4/8), exactly
+# one K tile per CTA (8 over 8), and the page's first dense shape
+SPLIT_SHAPES = [(200, 272, 1152), (17, 400, 1152), (129, 256, 1024), (64, 2112, 7168)]
+
+SPLIT_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import moe_grouped_gemm_mx_b200 as mx, mx_inputs
+out = sys.argv[2]
+res = {}
+for (m, n, k) in %r:
+    a = mx_inputs.outlier_bf16((m, k), seed=m + k)
+    b = mx_inputs.normal_bf16((n, k), 0.02, n + k)
+    qa, sa = mx.mx_quantize_bf16_to_e4m3_tile1x128(a.cuda())
+    qb, sb = mx.mx_quantize_bf16_to_e4m3_block128x128(b.cuda())
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    buf = torch.full((m + 128, n), 7.0, dtype=torch.bfloat16, device="cuda")
+    mx.mx_gemm_tilewise(qa, sa, qb, sb, d=buf[:m], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, hex(int(st.item()))
+    res[f"{m}x{n}x{k}"] = buf.float().cpu().numpy()
+    res[f"{m}x{n}x{k}_q"] = np.concatenate([qa.cpu().numpy().ravel(), qb.cpu().numpy().ravel()])
+    res[f"{m}x{n}x{k}_sa"] = sa.cpu().numpy()
+    res[f"{m}x{n}x{k}_sb"] = sb.cpu().numpy()
+np.savez(out, **res)
+""" % (SPLIT_SHAPES,)
+
+
+@pytest.mark.parametrize("split", [1, 2, 4, 8, 0], ids=["split1", "split2", "split4", "split8", "auto"])
+def test_tilewise_gemm_split_k(oracle, split):
+    """The dense tile-wise GEMM with K split over a cluster of 1/2/4/8 CTAs
+    (forced through the library's MX_TW_SPLIT override, read once per
+    process, so each split runs in a child process) and with the library's
+    own choice; rows past M keep their sentinel."""
+    with tempfile.TemporaryDirectory() as td:
+        out = os.path.join(td, "d.npz")
+        env = dict(os.environ)
+        env.pop("MX_TW_SPLIT", None)
+        if split:
+            env["MX_TW_SPLIT"] = str(split)
+        r = subprocess.run([sys.executable, "-c", SPLIT_CHILD, ROOT, out], env=env, capture_output=True, text=True,
+                           timeout=300)
+        assert r.returncode == 0, r.stderr[-2000:]
+        got = np.load(out)
+        for (m, n, k) in SPLIT_SHAPES:
+            key = f"{m}x{n}x{k}"
+            q = got[key + "_q"]
+            qa, qb = q[:m * k].reshape(m, k), q[m * k:].reshape(n, k)
+            d_ref, absd = oracle.tw_gemm(qa, got[key + "_sa"], qb, got[key + "_sb"])
+            assert_gemm_close(got[key][:m].astype(np.float64), d_ref, absd, f"split {split} {key}")
+            assert np.all(got[key][m:] == 7.0), f"split {split} {key}: rows past M written"
