@@ -6,11 +6,15 @@
 A step is one pass of the whole path over one batch of synthetic BF16 input
 already resident in HBM: quantise the activations (BF16 -> MXFP8 with tiled
 UE8M0 scales), quantise the weights -- all tensors of the step in one batched
-quantiser launch -- and run the GEMM(s) with the fused BF16 epilogue.  The step is captured once in a CUDA graph and replayed; the step time
-comes from CUDA events around each replay.  L2 is flushed (a 512 MiB write)
-before every timed step, outside the step's events.  Per-kernel device times
-(for the roofline of the dominant kernel) come from launching each kernel of
-the step on its own after an L2 flush, bracketed by CUDA events.
+quantiser launch -- and run the GEMM(s) with the fused BF16 epilogue.  The
+step is captured once in a CUDA graph and replayed; the step time comes from
+CUDA events around each replay.  L2 is flushed (a 512 MiB write) before every
+timed step, outside the step's events ("cold"); the mean, p50 and p95 of the
+cold steps are reported, and the same number of steps without the flush
+("warm") are timed afterwards and reported beside them.  Per-kernel device
+times (for the roofline of the dominant kernel) come from replaying each
+kernel of the step back to back in a CUDA graph over rotating copies of its
+operands that together exceed L2.
 
 Workloads (shapes from the pages; data synthetic and seeded):
   page        dense 64x2112x7168, 64x24576x1536, 128x7168x2048 (default)
@@ -19,6 +23,9 @@ Workloads (shapes from the pages; data synthetic and seeded):
   contiguous  MoE grouped, 32 experts, 8192 tokens top-8 Zipf: gate/up N=4096 K=7168,
               then down N=7168 K=2048
   masked      MoE masked grouped, 32 experts x 256 rows, masked_m ~ U{0..256}, N=4096 K=7168
+  moe_mlp     the contiguous MoE with gate/up -> SwiGLU -> MXFP8 fused, then down
+  moe_bwd     the gate/up layer's backward: dgrad and the K-grouped weight gradient
+  moe_layer   a whole expert layer: route, dispatch, gate/up.SwiGLU, down, combine
 
 With torchrun (N > 1) every rank runs its own independent batch (the work
 units are independent problems; no data-path collective), the step time is
@@ -125,8 +132,8 @@ def static_config(name: str, seed: int) -> dict:
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp", "moe_bwd",
                                                             "moe_layer"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -887,6 +894,16 @@ def run_ours(args, world, rank, local):
     barrier(world)
     t_wall1 = time.time()
 
+    # warm steps: the same replays without the L2 flush in between
+    warm_ms = []
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            s_ev.record()
+            step()
+            e_ev.record()
+            e_ev.synchronize()
+            warm_ms.append(s_ev.elapsed_time(e_ev))
+
     # per-kernel device time: each kernel of the step replayed back to back in
     # a CUDA graph over rotating copies of its operands (together larger than
     # L2, so no launch finds its operands cached by the previous ones), CUDA
@@ -930,6 +947,18 @@ def run_ours(args, world, rank, local):
     ms_step = statistics.mean(step_ms)
     ms_step_max = max_over_ranks(world, ms_step, dev)
     value = world * wl.flops / (ms_step_max * 1e-3) / 1e12
+
+    def pct(xs, q):
+        ys = sorted(xs)
+        return ys[min(len(ys) - 1, int(round(q / 100.0 * (len(ys) - 1))))]
+
+    warm_mean = max_over_ranks(world, statistics.mean(warm_ms), dev)
+    step_stats = {"cold_ms_p50": max_over_ranks(world, pct(step_ms, 50), dev),
+                  "cold_ms_p95": max_over_ranks(world, pct(step_ms, 95), dev),
+                  "warm_ms_mean": warm_mean,
+                  "warm_ms_p50": max_over_ranks(world, pct(warm_ms, 50), dev),
+                  "warm_ms_p95": max_over_ranks(world, pct(warm_ms, 95), dev),
+                  "warm_value": world * wl.flops / (warm_mean * 1e-3) / 1e12}
 
     # per-kernel breakdown and the roofline of the dominant kernel kind
     per_launch = []
@@ -1000,7 +1029,7 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_step_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": ms_step_max, "step_stats": step_stats, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3", "data": "synthetic",
         "config": dict(static_config(args.workload, args.seed), format=args.fmt,
                        l2="flushed (512 MiB write) before every timed step",
