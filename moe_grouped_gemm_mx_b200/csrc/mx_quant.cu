@@ -92,6 +92,19 @@ __device__ void write_padding(const QuantJob& jb, int64_t i) {
   jb.sf[g * jb.sf_group_bytes + sf_tiled_offset(static_cast<uint32_t>(r), static_cast<uint32_t>(c), jb.sf_ktiles)] = 0;
 }
 
+// KEEP: the outputs are written with ordinary (write-back) stores, so that
+// they stay in L2 for the GEMM that reads them next; otherwise with
+// streaming stores (evict-first), which are a little faster for outputs that
+// would not fit in L2 anyway.  The BF16 input is always read streaming.
+template <bool KEEP>
+__device__ __forceinline__ void store_out(uint4* p, const uint4& v) {
+  if constexpr (KEEP)
+    *p = v;
+  else
+    __stcs(p, v);
+}
+
+template <bool KEEP>
 __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_constant__ QuantBatch B) {
   __shared__ uint4 quant_stage[(kQuantThreads / 32) * kQuantUnroll * 128];  // 2 KiB per warp and step
   // with programmatic dependent launch the next kernel may start its
@@ -182,8 +195,8 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_co
                                     __shfl_sync(0xFFFFFFFFu, out1.z, sb), __shfl_sync(0xFFFFFFFFu, out1.w, sb));
         const uint32_t b0 = base + u * 32;
         uint4* dst = jb.q + static_cast<size_t>(b0) * 2;
-        if (b0 + sa < jb.nblk) __stcs(dst + lane, hi ? x1 : x0);
-        if (b0 + sb < jb.nblk) __stcs(dst + 32 + lane, hi ? y1 : y0);
+        if (b0 + sa < jb.nblk) store_out<KEEP>(dst + lane, hi ? x1 : x0);
+        if (b0 + sb < jb.nblk) store_out<KEEP>(dst + 32 + lane, hi ? y1 : y0);
       }
 
       // scale byte(s): row / K-block of this block, then its group
@@ -214,13 +227,19 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_co
 // kMaxQuantJobs tensors in one launch.  Each job needs groups*rows*(k/32) < 2^31.
 cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, cudaStream_t stream, int* launches) {
   static int resident = 0;  // CTAs of the kernel one SM holds
+  static int64_t l2_bytes = 0;
   if (resident == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, mx_quant_kernel, kQuantThreads, 0);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, mx_quant_kernel<false>, kQuantThreads, 0);
     if (e != cudaSuccess || resident <= 0) resident = 2048 / kQuantThreads;
+    int dev = 0, l2 = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) == cudaSuccess)
+      l2_bytes = l2;
+    cudaGetLastError();
   }
   QuantBatch B = {};
   uint32_t slots = 0;
   int64_t pads = 0;
+  int64_t out_bytes = 0;
   int n = 0;
   for (int i = 0; i < count; ++i) {
     const QuantSpec& sp = specs[i];
@@ -246,6 +265,7 @@ cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, c
     jb.pad_per_group = jb.pad_n1 + sp.rows * (kbpad - jb.kb);
     jb.pad0 = pads;
     pads += jb.pad_per_group * sp.groups;
+    out_bytes += static_cast<int64_t>(jb.nblk) * 32 + sp.groups * sp.sf_group_bytes;
   }
   if (n == 0) return cudaSuccess;
   B.count = n;
@@ -270,7 +290,10 @@ cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, mx_quant_kernel, B);
+  // outputs that fit in three quarters of L2 are kept there for their consumer
+  const bool keep = out_bytes <= l2_bytes / 4 * 3;
+  cudaError_t e = keep ? cudaLaunchKernelEx(&cfg, mx_quant_kernel<true>, B)
+                       : cudaLaunchKernelEx(&cfg, mx_quant_kernel<false>, B);
   if (e != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaGetLastError();
