@@ -18,7 +18,7 @@ operands that together exceed L2.
 
 Workloads (shapes from the pages; data synthetic and seeded):
   page        dense 64x2112x7168, 64x24576x1536, 128x7168x2048 (default); the three
-              independent GEMMs run on parallel streams after the quantiser
+              independent shapes' GEMMs run on parallel streams
   pr1         dense 128x256x512
   large       dense M=8192, (N,K) in {(7168,2048),(2112,7168),(4096,7168)}
   contiguous  MoE grouped, 32 experts, 8192 tokens top-8 Zipf: gate/up N=4096 K=7168,
@@ -249,7 +249,9 @@ class Workload:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.quant_jobs = []
         self.fmt = fmt
-        self.parallel_tail = False  # launches[1:] independent: parallel branches after launches[0]
+        # independent chains of launches (lists of indices into launches), run
+        # on parallel streams / graph branches after the launches in none
+        self.branches = None
         self._side = []
         if fmt == "tilewise":
             if name not in ("pr1", "page", "large", "contiguous"):
@@ -345,12 +347,16 @@ class Workload:
         for (m, n, k) in I.PAGE_SHAPES:
             a, b = I.dense_problem(m, n, k, seed=seed, kind="outlier", device=self.dev)
             self._dense(a, b, f"{m}x{n}x{k}")
+        # the three shapes are independent problems: their GEMMs run on
+        # parallel streams (branches of the step's graph), so that their fixed
+        # costs overlap -- after the one batched quantiser launch (MXFP8), or
+        # each behind its own two quantiser launches (tile-wise)
         if self.fmt == "mxfp8":
-            # the three GEMMs are independent problems: after the one batched
-            # quantiser launch each runs on its own stream (a parallel branch
-            # of the step's graph), so their fixed costs overlap
-            self.parallel_tail = True
+            self.branches = [[1], [2], [3]]
             self.config["gemms"] = "three independent GEMMs on parallel streams / graph branches after the quantiser"
+        else:
+            self.branches = [[0, 1, 2], [3, 4, 5], [6, 7, 8]]
+            self.config["gemms"] = "per shape: quantise A, quantise B, GEMM, the three shapes on parallel streams"
         self.config.update({"shapes": [f"{m}x{n}x{k}" for m, n, k in I.PAGE_SHAPES],
                             "a": "N(0,1) with 0.5% x64 outliers", "b": "N(0,0.02)"})
 
@@ -576,26 +582,27 @@ class Workload:
                             "active_experts": active})
 
     def run_eager(self):
-        if not self.parallel_tail:
+        if not self.branches:
             for _, _, fn, _, _, inputs in self.launches:
                 fn(*inputs)
             return
         import torch
         cur = torch.cuda.current_stream()
-        tail = self.launches[1:]
-        while len(self._side) < len(tail) - 1:
-            self._side.append(torch.cuda.Stream(device=self.dev))
-        _, _, fn, _, _, inputs = self.launches[0]
-        fn(*inputs)
-        for st in self._side[:len(tail) - 1]:
-            st.wait_stream(cur)
-        for j, (_, _, fn, _, _, inputs) in enumerate(tail):
-            if j == 0:
+        in_branch = {i for br in self.branches for i in br}
+        for i, (_, _, fn, _, _, inputs) in enumerate(self.launches):
+            if i not in in_branch:
                 fn(*inputs)
-            else:
-                with torch.cuda.stream(self._side[j - 1]):
+        nside = len(self.branches) - 1
+        while len(self._side) < nside:
+            self._side.append(torch.cuda.Stream(device=self.dev))
+        for st in self._side[:nside]:
+            st.wait_stream(cur)
+        for b, br in enumerate(self.branches):
+            with torch.cuda.stream(cur if b == 0 else self._side[b - 1]):
+                for i in br:
+                    _, _, fn, _, _, inputs = self.launches[i]
                     fn(*inputs)
-        for st in self._side[:len(tail) - 1]:
+        for st in self._side[:nside]:
             cur.wait_stream(st)
 
 
