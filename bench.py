@@ -948,6 +948,7 @@ def run_ours(args, world, rank, local):
     # GEMM), and a single kernel is what the roofline is about.
     kern_ms = [[] for _ in range(n_k)]
     k_copies = []
+    t_k0 = time.time()
     kernel_reps = max(3, min(args.steps, 10))
     l2_cover = 256 * 1024 * 1024
     for i, (_, _, fn, _, _, inputs) in enumerate(wl.launches):
@@ -972,8 +973,10 @@ def run_ours(args, world, rank, local):
         k_copies.append(copies)
         del g_k, bufs
     torch.cuda.synchronize()
+    t_k1 = time.time()
     sampler.stop()
     clocks = sampler.summary(t_wall0 - 0.25, t_wall1 + 0.25)
+    k_clocks = sampler.summary(t_k0, t_k1 + 0.25)
 
     st = int(wl.status.item())
     if st != 0:
@@ -1014,10 +1017,17 @@ def run_ours(args, world, rank, local):
     tensor_bound = dom == "gemm" and dk["flops"] / max(dk["bytes"], 1.0) > ridge
     sec = dk["ms"] * 1e-3
     if tensor_bound:
+        # the burst peak for a kernel whose timed replays ran at full clock;
+        # the sustained one (a seconds-long GEMM loop under the power cap)
+        # once the power cap throttled the replays
+        capped = "sw_power_cap" in k_clocks.get("reasons", [])
+        t_peak = peaks["bf16_tflops_sustained" if capped else "bf16_tflops"] * FP8_OVER_BF16
         achieved = dk["flops"] / sec / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp8_peak}
-        peak_note = f"fp8 = 2 x {peaks['source']} bf16 burst {peaks['bf16_tflops']}"
+        roof = {"bound": "tensor", "achieved": achieved, "peak": t_peak, "unit": "TFLOP/s",
+                "frac": achieved / t_peak}
+        peak_note = (f"fp8 = 2 x {peaks['source']} bf16 "
+                     + (f"sustained {peaks['bf16_tflops_sustained']} (sw_power_cap active during the kernel's "
+                        f"timed replays)" if capped else f"burst {peaks['bf16_tflops']}"))
     else:
         achieved = dk["bytes"] / sec / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
