@@ -184,8 +184,11 @@ def test_tilewise_quant_midpoints_and_tiny_scales(mx, oracle, blocks):
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 # ragged M and N, K tiles not a multiple of the split (9 over 2/4/8), exactly
-# one K tile per CTA (8 over 8), and the page's first dense shape
-SPLIT_SHAPES = [(200, 272, 1152), (17, 400, 1152), (129, 256, 1024), (64, 2112, 7168)]
+# one K tile per CTA (8 over 8), a single row and a single 16-column block,
+# fewer K tiles than the split asks for (5: the split is not taken), and the
+# page's first dense shape
+SPLIT_SHAPES = [(200, 272, 1152), (17, 400, 1152), (129, 256, 1024), (1, 16, 1024), (256, 128, 640),
+                (64, 2112, 7168)]
 
 SPLIT_CHILD = r"""
 import sys, numpy as np, torch
