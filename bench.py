@@ -231,6 +231,27 @@ class ClockSampler:
                 "samples": len(inside), "samples_in_timed_region": sum(1 for r in rows if t0 <= r[0] <= t1)}
 
 
+def system_info(dev, smi_id: str) -> dict:
+    """GPU, driver, CUDA and compiler versions and host cores, recorded with
+    every measurement."""
+    import torch
+    info = {"gpu": torch.cuda.get_device_name(dev), "torch": torch.__version__, "cuda_runtime": torch.version.cuda,
+            "host_cores": os.cpu_count()}
+    try:
+        r = subprocess.run(["nvidia-smi", f"--id={smi_id}", "--query-gpu=driver_version", "--format=csv,noheader"],
+                           capture_output=True, text=True, timeout=20)
+        info["driver"] = r.stdout.strip().splitlines()[0] if r.returncode == 0 and r.stdout.strip() else None
+    except (OSError, subprocess.SubprocessError):
+        info["driver"] = None
+    try:
+        r = subprocess.run(["nvcc", "--version"], capture_output=True, text=True, timeout=20)
+        rel = [ln for ln in r.stdout.splitlines() if "release" in ln]
+        info["nvcc"] = rel[0].split("release", 1)[1].strip() if rel else None
+    except (OSError, subprocess.SubprocessError):
+        info["nvcc"] = None
+    return info
+
+
 # ---------------------------------------------------------------- workloads
 
 class Workload:
@@ -1086,6 +1107,7 @@ def run_ours(args, world, rank, local):
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "system": system_info(dev, smi_id),
         "kernels": [{"kind": r["kind"], "label": r["label"], "ms": round(r["ms"], 5),
                      "GB/s": round(r["bytes"] / (r["ms"] * 1e-3) / 1e9, 1),
                      "TFLOP/s": round(r["flops"] / (r["ms"] * 1e-3) / 1e12, 1)} for r in per_launch],
