@@ -88,6 +88,8 @@ def lib():
         L.mxo_tw_gemm.restype = None
         L.mxo_moe_route.argtypes = [P, I64, I32, I32, P, P, P]
         L.mxo_moe_route.restype = I64
+        L.mxo_moe_peer_plan.argtypes = [P, P, I32, I32, I32, P, P, P, P]
+        L.mxo_moe_peer_plan.restype = None
         L.mxo_moe_dispatch.argtypes = [P, I64, I64, P, I64, I64, P, P]
         L.mxo_moe_dispatch.restype = None
         L.mxo_moe_combine.argtypes = [P, I64, P, P, I64, I64, P, P]
@@ -374,6 +376,31 @@ def moe_route(ids, num_experts: int, pad: int = 128):
     row = np.zeros(ids.size, dtype=np.int32)
     bad = lib().mxo_moe_route(_p(ids), ids.size, num_experts, pad, _p(counts), _p(offsets), _p(row))
     return counts, offsets, row, int(bad)
+
+
+def moe_peer_plan(ids_list, num_experts: int, pad: int = 128):
+    """Expert-parallel placement of every rank's entries (rank r's ids are
+    ids_list[r], token-major): on the owner of expert e (rank e // (E/R)), e's
+    rows are rank 0's entries in order, then rank 1's, ...; each of the
+    owner's groups padded to ``pad``.  Returns ([(dst_rank, dst_row)] per rank,
+    counts_local int32 [R, E/R], offsets_local int32 [R, E/R+1])."""
+    ranks = len(ids_list)
+    flat = [np.ascontiguousarray(a, dtype=np.int32).reshape(-1) for a in ids_list]
+    n_of = np.array([a.size for a in flat], dtype=np.int64)
+    ids = np.ascontiguousarray(np.concatenate(flat) if flat else np.zeros(0, np.int32), dtype=np.int32)
+    el = num_experts // ranks
+    dst_rank = np.zeros(ids.size, dtype=np.int32)
+    dst_row = np.zeros(ids.size, dtype=np.int32)
+    counts = np.zeros((ranks, el), dtype=np.int32)
+    offsets = np.zeros((ranks, el + 1), dtype=np.int32)
+    lib().mxo_moe_peer_plan(_p(ids), _p(n_of), ranks, num_experts, pad, _p(dst_rank), _p(dst_row), _p(counts),
+                            _p(offsets))
+    per = []
+    pos = 0
+    for n in n_of:
+        per.append((dst_rank[pos:pos + n], dst_row[pos:pos + n]))
+        pos += n
+    return per, counts, offsets
 
 
 def moe_dispatch(x, row, topk: int, m_rows: int):

@@ -585,6 +585,55 @@ int64_t mxo_moe_route(const int32_t *ids, int64_t n, int32_t E, int32_t pad, int
     return bad;
 }
 
+/* Expert-parallel placement (the B200 MoE-training page, its DeepEP section
+ * and glossary entry on all-to-all: each token goes to the rank that holds
+ * its expert).  `ranks` ranks each hold E/ranks experts (rank o owns experts
+ * [o*E/ranks, (o+1)*E/ranks)) and their own entries: ids holds rank r's n_of[r]
+ * entries after those of ranks 0..r-1.  On the owner of expert e, e's rows
+ * are its entries of rank 0 in entry order, then those of rank 1, and so on;
+ * the owner's experts are placed one after another, each group padded to a
+ * multiple of `pad` rows.  Entry i (in ids order) goes to rank dst_rank[i],
+ * row dst_row[i]; an id outside [0, E) is dropped (-1, -1).  Owner o's plan:
+ * counts_local[o*el + l] entries of its expert l (el = E/ranks) and
+ * offsets_local[o*(el+1) + l] its padded group starts, el + 1 values. */
+void mxo_moe_peer_plan(const int32_t *ids, const int64_t *n_of, int32_t ranks, int32_t E, int32_t pad,
+                       int32_t *dst_rank, int32_t *dst_row, int32_t *counts_local, int32_t *offsets_local)
+{
+    int32_t el = E / ranks;
+    int64_t n = 0;
+    for (int32_t r = 0; r < ranks; ++r)
+        n += n_of[r];
+    int64_t *tot = (int64_t *)calloc((size_t)(E > 0 ? E : 1), sizeof(int64_t));
+    int64_t *next = (int64_t *)calloc((size_t)(E > 0 ? E : 1), sizeof(int64_t));
+    for (int64_t i = 0; i < n; ++i)
+        if (ids[i] >= 0 && ids[i] < E)
+            tot[ids[i]] += 1;
+    for (int32_t o = 0; o < ranks; ++o) {
+        int64_t start = 0;
+        for (int32_t l = 0; l < el; ++l) {
+            int32_t e = o * el + l;
+            next[e] = start;
+            counts_local[o * el + l] = (int32_t)tot[e];
+            offsets_local[o * (el + 1) + l] = (int32_t)start;
+            start += (tot[e] + pad - 1) / pad * pad;
+        }
+        offsets_local[o * (el + 1) + el] = (int32_t)start;
+    }
+    for (int64_t i = 0; i < n; ++i) {   /* rank by rank, each rank's entries in order */
+        int32_t e = ids[i];
+        if (e >= 0 && e < E) {
+            dst_rank[i] = e / el;
+            dst_row[i] = (int32_t)next[e];
+            next[e] += 1;
+        } else {
+            dst_rank[i] = -1;
+            dst_row[i] = -1;
+        }
+    }
+    free(tot);
+    free(next);
+}
+
 /* Dispatch into the contiguous layout: the E4M3 row and scales of token t
  * (quantised as by mxo_quantize) are written to row[t*topk + j] for every j
  * with row >= 0.  q [m_rows, k] and sf_rm [m_rows, k/32] are first set to

@@ -52,6 +52,8 @@ void mxo_tw_gemm(const uint8_t *qa, const float *sa, const uint8_t *qb, const fl
                  double *abssum);
 int64_t mxo_moe_route(const int32_t *ids, int64_t n, int32_t E, int32_t pad, int32_t *counts,
                       int32_t *offsets, int32_t *row);
+void mxo_moe_peer_plan(const int32_t *ids, const int64_t *n_of, int32_t ranks, int32_t E, int32_t pad,
+                       int32_t *dst_rank, int32_t *dst_row, int32_t *counts_local, int32_t *offsets_local);
 void mxo_moe_dispatch(const uint16_t *x, int64_t T, int64_t k, const int32_t *row, int64_t topk,
                       int64_t m_rows, uint8_t *q, uint8_t *sf_rm);
 void mxo_moe_combine(const uint16_t *y, int64_t n, const int32_t *row, const float *w, int64_t T,

@@ -157,3 +157,59 @@ def test_layer_grouped_rows_match_per_token_dense():
             e = int(ids[t, j])
             dt, _ = gemm(qx[t:t + 1], sfx[t:t + 1], qb[e], sfb[e])
             assert np.array_equal(d[row[t * topk + j]], dt[0])
+
+
+# ---------------------------------------------------------------- expert-parallel placement
+
+def test_peer_plan_hand_example():
+    """Two ranks, four experts (rank 0 owns 0-1, rank 1 owns 2-3), pad 2.
+    Rank 0's entries have experts 0,3,1,0 and rank 1's 2,0,3,3.  Totals: e0 3
+    (rank 0 entries 0, 3, then rank 1 entry 1), e1 1, e2 1, e3 3 (rank 0
+    entry 1, then rank 1 entries 2, 3).  Owner 0: e0 rows 0-2 (padded to 4),
+    e1 row 4 (padded to 2): offsets 0, 4, 6.  Owner 1: e2 row 0 (padded to
+    2), e3 rows 2-4 (padded to 4): offsets 0, 2, 6."""
+    from oracle import moe_peer_plan
+    per, counts, offsets = moe_peer_plan([np.array([0, 3, 1, 0]), np.array([2, 0, 3, 3])], 4, pad=2)
+    assert per[0][0].tolist() == [0, 1, 0, 0] and per[0][1].tolist() == [0, 2, 4, 1]
+    assert per[1][0].tolist() == [1, 0, 1, 1] and per[1][1].tolist() == [0, 2, 3, 4]
+    assert counts.tolist() == [[3, 1], [1, 3]]
+    assert offsets.tolist() == [[0, 4, 6], [0, 2, 6]]
+
+
+@pytest.mark.parametrize("pad", [1, 128])
+def test_peer_plan_one_rank_is_the_routing_plan(pad):
+    """With one rank the placement is the single-GPU routing plan."""
+    from oracle import moe_peer_plan, moe_route
+    ids = mx_inputs.topk_ids(300, 4, 8, seed=81)
+    ids[7, 1] = -1
+    ids[9, 0] = 8
+    per, counts, offsets = moe_peer_plan([ids], 8, pad=pad)
+    rc, ro, rr, _ = moe_route(ids, 8, pad=pad)
+    assert np.array_equal(per[0][1], rr)
+    assert np.array_equal(per[0][0], np.where(rr >= 0, 0, -1))
+    assert np.array_equal(counts[0], rc) and np.array_equal(offsets[0], ro)
+
+
+@pytest.mark.parametrize("ranks,experts", [(2, 8), (3, 6), (4, 32)])
+def test_peer_plan_is_the_owners_routing_plan(ranks, experts):
+    """On every owner, the rows are those the single-GPU routing plan gives
+    to the owner's experts over all ranks' entries taken rank by rank (the
+    entries of other owners' experts dropped), and the plan's counts and
+    offsets are that plan's."""
+    from oracle import moe_peer_plan, moe_route
+    rng = np.random.default_rng(ranks * experts)
+    ids_list = [mx_inputs.topk_ids(int(rng.integers(0, 200)), 4, experts, seed=90 + r) for r in range(ranks)]
+    ids_list[0][:3, 0] = -1                       # dropped entries
+    per, counts, offsets = moe_peer_plan(ids_list, experts, pad=128)
+    el = experts // ranks
+    allids = np.concatenate([a.reshape(-1) for a in ids_list])
+    dr = np.concatenate([p[0] for p in per])
+    drow = np.concatenate([p[1] for p in per])
+    for o in range(ranks):
+        local = np.where((allids >= o * el) & (allids < (o + 1) * el), allids - o * el, -1).astype(np.int32)
+        rc, ro, rr, _ = moe_route(local, el, pad=128)
+        mine = local >= 0
+        assert np.all(dr[mine] == o)
+        assert np.array_equal(drow[mine], rr[mine])
+        assert np.array_equal(counts[o], rc) and np.array_equal(offsets[o], ro)
+    assert np.all((dr == -1) == (allids < 0)) and np.all((drow == -1) == (allids < 0))
