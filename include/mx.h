@@ -352,6 +352,71 @@ mx_status mx_gather_rows(const void *src, int64_t src_rows, int64_t row_bytes, c
 mx_status mx_moe_combine(const void *y_bf16, int64_t y_rows, int64_t n_cols, const int32_t *row, const float *w,
                          int64_t tokens, int32_t topk, void *out_bf16, int32_t *dev_status, mx_stream_t stream);
 
+/*
+ * Expert parallelism over peer memory (the DeepEP role on the B200
+ * MoE-training page: tokens are sent to the ranks that hold their experts and
+ * the results gathered back), with the exchange fused into the dispatch and
+ * the combine: the dispatch quantises each token once and stores its MXFP8
+ * row straight into the receive buffer of the rank that owns the expert, and
+ * the combine loads the expert outputs straight from their owners' buffers.
+ * "Rank r's buffer" is any device pointer this process can dereference:
+ * another GPU's memory mapped for peer access (NVLink), or, to emulate several
+ * ranks on one GPU, a local buffer.  Pointer tables (q_peers, sf_peers,
+ * y_peers) are DEVICE arrays of `ranks` pointers, every buffer 16-byte aligned
+ * and of the same shape on every rank.  The calls only load and store: the
+ * caller orders the phases across ranks (every rank's dispatch complete
+ * before any owner's GEMM reads its receive buffer; every owner's GEMM
+ * complete before any combine reads its output; every combine complete before
+ * the buffers are written again), e.g. with a collective barrier on the stream.
+ * Rank r of R owns the experts [r*E/R, (r+1)*E/R).
+ */
+
+/* Placement plan of this rank's entries (n = tokens*topk, device).  ids are
+ * global expert ids; row_send is mx_moe_route(ids, experts, pad = 1)'s row
+ * output; count_table int32 [ranks, experts] holds every rank's counts from
+ * that route (e.g. all-gathered).  On the owner of expert e, e's rows come
+ * source rank by source rank, each source's rows in its entry order, and each
+ * local expert's group is padded to `pad` rows.  Outputs (device):
+ * dst_rank/dst_row int32 [n] (the owner and the row in its receive buffer;
+ * -1/-1 for an id outside [0, experts)), and this rank's own receive plan:
+ * counts_local int32 [experts/ranks] (rows from all sources) and
+ * offsets_local int32 [experts/ranks + 1] (padded group starts, the
+ * group_offsets of the grouped GEMMs; offsets_local[E/R] = rows in use).
+ * experts % ranks == 0; 1 <= experts, ranks <= 1024; 1 <= pad <= 128;
+ * n * ranks < 2^31.  A row_send inconsistent with count_table sets
+ * MX_DEV_BAD_INDEX and gives -1/-1. */
+mx_status mx_moe_peer_plan(const int32_t *ids, const int32_t *row_send, int64_t n, const int32_t *count_table,
+                           int32_t ranks, int32_t rank, int32_t experts, int32_t pad, int32_t *dst_rank,
+                           int32_t *dst_row, int32_t *counts_local, int32_t *offsets_local, int32_t *dev_status,
+                           mx_stream_t stream);
+
+/* Dispatch over peer memory: each token row of x_bf16 [tokens, k] is
+ * quantised to MXFP8 once (mx_quantize_bf16_to_e4m3's rule, bit for bit) and,
+ * for every j with dst_row[t*topk + j] >= 0, written to row dst_row of
+ * q_peers[dst_rank] [m_rows, k] with its scale bytes in the tiled layout of
+ * sf_peers[dst_rank] (mx_scale_bytes(m_rows, k) bytes).  This rank's own
+ * receive buffer q_local / sf_local (the entries of the tables for this rank)
+ * gets the padding rows of its plan (counts_local, offsets_local,
+ * experts_local, pad from mx_moe_peer_plan) set to the quantisation of a zero
+ * row.  k % 128 == 0, m_rows % 128 == 0, 16-byte aligned buffers.  A
+ * dst_rank outside [0, ranks) or a dst_row >= m_rows is skipped and sets
+ * MX_DEV_BAD_INDEX. */
+mx_status mx_moe_dispatch_quant_peer(const void *x_bf16, int64_t tokens, int64_t k, const int32_t *dst_rank,
+                                     const int32_t *dst_row, int32_t topk, void *const *q_peers,
+                                     void *const *sf_peers, int32_t ranks, int64_t m_rows, void *q_local,
+                                     void *sf_local, const int32_t *counts_local, const int32_t *offsets_local,
+                                     int32_t experts_local, int32_t pad, int32_t *dev_status, mx_stream_t stream);
+
+/* Combine over peer memory: out[t, :] = sum_j w[t, j] * y_peers[src_rank[t*topk+j]][src_row[t*topk+j], :]
+ * over the entries with src_row >= 0, with mx_moe_combine's arithmetic (FP32
+ * fused multiply-adds in j order, one rounding to BF16).  Every rank's output
+ * buffer is BF16 [y_rows, n_cols]; src_rank/src_row are the dispatch's
+ * dst_rank/dst_row.  A rank outside [0, ranks) or a row >= y_rows is skipped
+ * and sets MX_DEV_BAD_INDEX. */
+mx_status mx_moe_combine_peer(const void *const *y_peers, int32_t ranks, int64_t y_rows, int64_t n_cols,
+                              const int32_t *src_rank, const int32_t *src_row, const float *w, int64_t tokens,
+                              int32_t topk, void *out_bf16, int32_t *dev_status, mx_stream_t stream);
+
 /* Copies the library-internal device status word (used when a call got
  * dev_status == NULL) to *host_out and, if clear != 0, resets it.
  * Synchronises the device. */

@@ -29,7 +29,7 @@ __all__ = [
     "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped", "mx_quantize_bf16_to_e4m3_tile1x128",
     "mx_quantize_bf16_to_e4m3_block128x128", "mx_gemm_tilewise", "mx_grouped_gemm_contiguous_tilewise",
     "mx_moe_max_rows", "mx_moe_route", "mx_moe_dispatch_quant", "mx_moe_scatter_rows", "mx_gather_rows",
-    "mx_moe_combine",
+    "mx_moe_combine", "mx_moe_peer_plan", "mx_moe_dispatch_quant_peer", "mx_moe_combine_peer",
     "read_internal_status", "MX_DEV_BAD_OFFSETS", "MX_DEV_BAD_MASK", "MX_DEV_TIMEOUT", "MX_DEV_BAD_INDEX",
     "C_SYMBOLS",
 ]
@@ -52,7 +52,7 @@ C_SYMBOLS = [
     "mx_quantize_bf16_to_e4m3_transposed", "mx_grouped_gemm_kgrouped", "mx_quantize_bf16_to_e4m3_tile1x128",
     "mx_quantize_bf16_to_e4m3_block128x128", "mx_gemm_tilewise", "mx_grouped_gemm_contiguous_tilewise",
     "mx_moe_max_rows", "mx_moe_route", "mx_moe_dispatch_quant", "mx_moe_scatter_rows", "mx_gather_rows",
-    "mx_moe_combine",
+    "mx_moe_combine", "mx_moe_peer_plan", "mx_moe_dispatch_quant_peer", "mx_moe_combine_peer",
 ]
 
 
@@ -120,6 +120,12 @@ def _load():
     L.mx_gather_rows.restype = ctypes.c_int
     L.mx_moe_combine.argtypes = [P, I64, I64, P, P, I64, I32, P, P, P]
     L.mx_moe_combine.restype = ctypes.c_int
+    L.mx_moe_peer_plan.argtypes = [P, P, I64, P, I32, I32, I32, I32, P, P, P, P, P, P]
+    L.mx_moe_peer_plan.restype = ctypes.c_int
+    L.mx_moe_dispatch_quant_peer.argtypes = [P, I64, I64, P, P, I32, P, P, I32, I64, P, P, P, P, I32, I32, P, P]
+    L.mx_moe_dispatch_quant_peer.restype = ctypes.c_int
+    L.mx_moe_combine_peer.argtypes = [P, I32, I64, I64, P, P, P, I64, I32, P, P, P]
+    L.mx_moe_combine_peer.restype = ctypes.c_int
     L.mx_read_internal_status.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
     L.mx_read_internal_status.restype = ctypes.c_int
     return L
@@ -596,6 +602,100 @@ def mx_moe_combine(y: torch.Tensor, row: torch.Tensor, w: torch.Tensor, out=None
         raise ValueError("out too small")
     _raise(_lib.mx_moe_combine(_ptr(y), y.shape[0], n, _ptr(row), _ptr(w), tokens, topk, _ptr(out),
                                _ptr(dev_status), _stream(stream)), "mx_moe_combine")
+    return out
+
+
+def _ptr_table(t: torch.Tensor, ranks: int, name: str):
+    """A device int64 tensor of ``ranks`` buffer addresses (a peer pointer table)."""
+    if t.dtype != torch.int64 or t.device.type != "cuda" or not t.is_contiguous() or t.numel() != ranks:
+        raise ValueError(f"{name} must be a contiguous int64 CUDA tensor of {ranks} addresses")
+    return _ptr(t)
+
+
+def mx_moe_peer_plan(ids: torch.Tensor, row_send: torch.Tensor, count_table: torch.Tensor, rank: int,
+                     experts: int, pad: int = 128, dst_rank=None, dst_row=None, counts_local=None,
+                     offsets_local=None, dev_status=None, stream=None):
+    """Where each of this rank's entries goes under expert parallelism over
+    peer memory.  ids int32 [tokens*topk] (global expert ids), row_send the
+    row output of mx_moe_route(ids, experts, pad=1), count_table int32
+    [ranks, experts] every rank's counts of that route.  Returns (dst_rank,
+    dst_row, counts_local [E/R], offsets_local [E/R+1]) int32 device tensors:
+    the owner and the row in its receive buffer per entry, and this rank's own
+    receive plan (group offsets of its local experts, padded to ``pad``)."""
+    _check(ids, torch.int32, "ids")
+    _check(row_send, torch.int32, "row_send")
+    _check(count_table, torch.int32, "count_table")
+    n = ids.numel()
+    ranks = count_table.shape[0]
+    if count_table.dim() != 2 or count_table.shape[1] != experts or row_send.numel() != n:
+        raise ValueError("count_table must be [ranks, experts] and row_send match ids")
+    if experts % ranks:
+        raise ValueError("the experts must divide evenly over the ranks")
+    el = experts // ranks
+    dev = ids.device
+    dst_rank = torch.empty(n, dtype=torch.int32, device=dev) if dst_rank is None else dst_rank
+    dst_row = torch.empty(n, dtype=torch.int32, device=dev) if dst_row is None else dst_row
+    counts_local = torch.empty(el, dtype=torch.int32, device=dev) if counts_local is None else counts_local
+    offsets_local = torch.empty(el + 1, dtype=torch.int32, device=dev) if offsets_local is None else offsets_local
+    for t, nm, size in ((dst_rank, "dst_rank", n), (dst_row, "dst_row", n), (counts_local, "counts_local", el),
+                        (offsets_local, "offsets_local", el + 1)):
+        _check(t, torch.int32, nm)
+        if t.numel() < size:
+            raise ValueError(f"{nm} too small")
+    _raise(_lib.mx_moe_peer_plan(_ptr(ids), _ptr(row_send), n, _ptr(count_table), ranks, rank, experts, pad,
+                                 _ptr(dst_rank), _ptr(dst_row), _ptr(counts_local), _ptr(offsets_local),
+                                 _ptr(dev_status), _stream(stream)), "mx_moe_peer_plan")
+    return dst_rank, dst_row, counts_local, offsets_local
+
+
+def mx_moe_dispatch_quant_peer(x: torch.Tensor, dst_rank: torch.Tensor, dst_row: torch.Tensor, topk: int,
+                               q_ptrs: torch.Tensor, sf_ptrs: torch.Tensor, m_rows: int, q_local: torch.Tensor,
+                               sf_local: torch.Tensor, counts_local: torch.Tensor, offsets_local: torch.Tensor,
+                               pad: int = 128, dev_status=None, stream=None):
+    """Quantise each token of x (BF16 [tokens, K]) once and store its MXFP8
+    row (tiled scales) at row dst_row of rank dst_rank's receive buffer, the
+    buffers given by device address tables q_ptrs / sf_ptrs (int64 [ranks]);
+    this rank's own receive buffer (q_local [m_rows, K], sf_local) gets the
+    padding rows of its plan cleared."""
+    _check(x, torch.bfloat16, "x")
+    _check(dst_rank, torch.int32, "dst_rank")
+    _check(dst_row, torch.int32, "dst_row")
+    _check(q_local, torch.uint8, "q_local")
+    _check(sf_local, torch.uint8, "sf_local")
+    _check(counts_local, torch.int32, "counts_local")
+    _check(offsets_local, torch.int32, "offsets_local")
+    tokens, k = x.shape
+    ranks = q_ptrs.numel()
+    if dst_row.numel() != tokens * topk or dst_rank.numel() != tokens * topk:
+        raise ValueError("dst_rank / dst_row must hold tokens*topk entries")
+    if q_local.numel() < m_rows * k or sf_local.numel() < scale_bytes(m_rows, k):
+        raise ValueError("local receive buffers too small")
+    _raise(_lib.mx_moe_dispatch_quant_peer(_ptr(x), tokens, k, _ptr(dst_rank), _ptr(dst_row), topk,
+                                           _ptr_table(q_ptrs, ranks, "q_ptrs"), _ptr_table(sf_ptrs, ranks, "sf_ptrs"),
+                                           ranks, m_rows, _ptr(q_local), _ptr(sf_local), _ptr(counts_local),
+                                           _ptr(offsets_local), counts_local.numel(), pad, _ptr(dev_status),
+                                           _stream(stream)), "mx_moe_dispatch_quant_peer")
+
+
+def mx_moe_combine_peer(y_ptrs: torch.Tensor, y_rows: int, n: int, src_rank: torch.Tensor, src_row: torch.Tensor,
+                        w: torch.Tensor, out=None, dev_status=None, stream=None):
+    """out[t] = sum_j w[t, j] * (rank src_rank[t, j]'s output)[src_row[t, j]]
+    (FP32 in j order, BF16 out); every rank's output is BF16 [y_rows, n],
+    addressed by the device table y_ptrs (int64 [ranks])."""
+    _check(w, torch.float32, "w")
+    _check(src_rank, torch.int32, "src_rank")
+    _check(src_row, torch.int32, "src_row")
+    tokens, topk = w.shape
+    if src_row.numel() != tokens * topk or src_rank.numel() != tokens * topk:
+        raise ValueError("src_rank / src_row must hold tokens*topk entries")
+    ranks = y_ptrs.numel()
+    out = torch.empty((tokens, n), dtype=torch.bfloat16, device=w.device) if out is None else out
+    _check(out, torch.bfloat16, "out")
+    if out.numel() < tokens * n:
+        raise ValueError("out too small")
+    _raise(_lib.mx_moe_combine_peer(_ptr_table(y_ptrs, ranks, "y_ptrs"), ranks, y_rows, n, _ptr(src_rank),
+                                    _ptr(src_row), _ptr(w), tokens, topk, _ptr(out), _ptr(dev_status),
+                                    _stream(stream)), "mx_moe_combine_peer")
     return out
 
 

@@ -476,8 +476,90 @@ mx_status mx_moe_combine(const void* y_bf16, int64_t y_rows, int64_t n_cols, con
       (reinterpret_cast<uintptr_t>(row) & 3u))
     return MX_ERR_MISALIGNED;
   int32_t* status = dev_status ? dev_status : internal_status_ptr();
-  return from_cuda(mxk::launch_moe_combine(y_bf16, y_rows, n_cols, row, w, tokens, topk, out_bf16, status,
-                                           static_cast<cudaStream_t>(stream)));
+  return from_cuda(mxk::launch_moe_combine(y_bf16, nullptr, nullptr, 0, y_rows, n_cols, row, w, tokens, topk,
+                                           out_bf16, status, static_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------------------ expert parallelism over peer memory
+
+mx_status mx_moe_peer_plan(const int32_t* ids, const int32_t* row_send, int64_t n, const int32_t* count_table,
+                           int32_t ranks, int32_t rank, int32_t experts, int32_t pad, int32_t* dst_rank,
+                           int32_t* dst_row, int32_t* counts_local, int32_t* offsets_local, int32_t* dev_status,
+                           mx_stream_t stream) {
+  if (n < 0 || ranks < 1 || ranks > kMaxGroups || rank < 0 || rank >= ranks || experts < 1 ||
+      experts > kMaxGroups || pad < 1 || pad > 128 || experts % ranks != 0)
+    return MX_ERR_INVALID_ARGUMENT;
+  if (n * static_cast<int64_t>(ranks) > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (!count_table || !counts_local || !offsets_local || (n > 0 && (!ids || !row_send || !dst_rank || !dst_row)))
+    return MX_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(ids) | reinterpret_cast<uintptr_t>(row_send) |
+       reinterpret_cast<uintptr_t>(count_table) | reinterpret_cast<uintptr_t>(dst_rank) |
+       reinterpret_cast<uintptr_t>(dst_row) | reinterpret_cast<uintptr_t>(counts_local) |
+       reinterpret_cast<uintptr_t>(offsets_local)) & 3u)
+    return MX_ERR_MISALIGNED;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  return from_cuda(mxk::launch_moe_peer_plan(ids, row_send, n, count_table, ranks, rank, experts, pad, dst_rank,
+                                             dst_row, counts_local, offsets_local, status, sms,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+mx_status mx_moe_dispatch_quant_peer(const void* x_bf16, int64_t tokens, int64_t k, const int32_t* dst_rank,
+                                     const int32_t* dst_row, int32_t topk, void* const* q_peers,
+                                     void* const* sf_peers, int32_t ranks, int64_t m_rows, void* q_local,
+                                     void* sf_local, const int32_t* counts_local, const int32_t* offsets_local,
+                                     int32_t experts_local, int32_t pad, int32_t* dev_status, mx_stream_t stream) {
+  if (ranks < 1 || ranks > kMaxGroups) return MX_ERR_INVALID_ARGUMENT;
+  mx_status st = check_place(x_bf16, tokens, k, dst_row, topk, counts_local, offsets_local, experts_local, pad,
+                             m_rows, q_local, sf_local, true);
+  if (st != MX_OK) return st;
+  if (k == 0 || (tokens == 0 && (pad == 1 || experts_local == 0))) return MX_OK;
+  if (tokens > 0 && (!dst_rank || !q_peers || !sf_peers)) return MX_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(q_peers) | reinterpret_cast<uintptr_t>(sf_peers)) & 7u ||
+      (reinterpret_cast<uintptr_t>(dst_rank) & 3u))
+    return MX_ERR_MISALIGNED;
+  mxk::MoePlace p = {};
+  p.src = x_bf16;
+  p.row = dst_row;
+  p.counts = counts_local;
+  p.offsets = offsets_local;
+  p.q = q_local;
+  p.sf = sf_local;
+  p.status = dev_status ? dev_status : internal_status_ptr();
+  p.n_src = tokens;
+  p.m_rows = m_rows;
+  p.k = k;
+  p.fan = topk;
+  p.experts = experts_local;
+  p.pad = pad;
+  p.sf_row_major = 0;
+  p.quantize = true;
+  p.q_peers = q_peers;
+  p.sf_peers = sf_peers;
+  p.row_rank = dst_rank;
+  p.ranks = ranks;
+  return from_cuda(mxk::launch_moe_place(p, static_cast<cudaStream_t>(stream)));
+}
+
+mx_status mx_moe_combine_peer(const void* const* y_peers, int32_t ranks, int64_t y_rows, int64_t n_cols,
+                              const int32_t* src_rank, const int32_t* src_row, const float* w, int64_t tokens,
+                              int32_t topk, void* out_bf16, int32_t* dev_status, mx_stream_t stream) {
+  if (ranks < 1 || ranks > kMaxGroups || y_rows < 0 || n_cols < 0 || tokens < 0 || topk < 1 || topk > 64)
+    return MX_ERR_INVALID_ARGUMENT;
+  if (n_cols % 8 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+  if (tokens > kMaxDim || y_rows > kMaxDim || tokens * static_cast<int64_t>(topk) > kMaxDim)
+    return MX_ERR_UNSUPPORTED_SHAPE;
+  if (tokens == 0 || n_cols == 0) return MX_OK;
+  if (!y_peers || !src_rank || !src_row || !w || !out_bf16) return MX_ERR_INVALID_ARGUMENT;
+  if (!aligned16(out_bf16) || (reinterpret_cast<uintptr_t>(y_peers) & 7u) ||
+      ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(src_rank) |
+        reinterpret_cast<uintptr_t>(src_row)) & 3u))
+    return MX_ERR_MISALIGNED;
+  int32_t* status = dev_status ? dev_status : internal_status_ptr();
+  return from_cuda(mxk::launch_moe_combine(nullptr, y_peers, src_rank, ranks, y_rows, n_cols, src_row, w, tokens,
+                                           topk, out_bf16, status, static_cast<cudaStream_t>(stream)));
 }
 
 mx_status mx_read_internal_status(int32_t* host_out, int clear) {

@@ -83,11 +83,25 @@ struct MoePlace {
   int64_t n_src, m_rows, k;
   int fan, experts, pad, sf_row_major;
   bool quantize;
+  // peer form (expert parallelism over peer memory): destination j of source
+  // row i is row row[i*fan+j] of rank row_rank[i*fan+j]'s buffers, device
+  // tables q_peers / sf_peers [ranks]; q / sf are this rank's own (padding)
+  void* const* q_peers = nullptr;
+  void* const* sf_peers = nullptr;
+  const int32_t* row_rank = nullptr;
+  int ranks = 0;
 };
 cudaError_t launch_moe_place(const MoePlace& p, cudaStream_t stream);
 cudaError_t launch_moe_gather(const void* src, int64_t src_rows, int64_t row_bytes, const int32_t* idx, int64_t n,
                               void* dst, int32_t* status, cudaStream_t stream);
-cudaError_t launch_moe_combine(const void* y, int64_t y_rows, int64_t n_cols, const int32_t* row, const float* w,
-                               int64_t tokens, int topk, void* out, int32_t* status, cudaStream_t stream);
+// y_peers != nullptr: the peer form, routed row j of token t is row
+// row[t*topk+j] of rank row_rank[t*topk+j]'s output (device table [ranks]).
+cudaError_t launch_moe_combine(const void* y, const void* const* y_peers, const int32_t* row_rank, int ranks,
+                               int64_t y_rows, int64_t n_cols, const int32_t* row, const float* w, int64_t tokens,
+                               int topk, void* out, int32_t* status, cudaStream_t stream);
+cudaError_t launch_moe_peer_plan(const int32_t* ids, const int32_t* row_send, int64_t n, const int32_t* count,
+                                 int ranks, int rank, int E, int pad, int32_t* dst_rank, int32_t* dst_row,
+                                 int32_t* counts_local, int32_t* offsets_local, int32_t* status, int num_sms,
+                                 cudaStream_t stream);
 
 }  // namespace mxk

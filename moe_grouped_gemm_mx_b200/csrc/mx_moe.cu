@@ -2,7 +2,11 @@
 // experts expert layer, on sm_100a: the routing plan, the dispatch (each
 // token quantised to MXFP8 once and its row placed at every expert row it is
 // routed to, in the contiguous grouped layout), the row scatter / gather of
-// the all-to-all buffers of expert parallelism, and the gate-weighted combine.
+// the all-to-all buffers of expert parallelism, the gate-weighted combine, and
+// the peer-memory forms of dispatch and combine for expert parallelism over
+// NVLink (rows written straight into, and read straight from, the buffers of
+// the rank that owns the expert, through a device table of every rank's
+// pointers) with the plan that places each entry there.
 //
 // Sources: the B200 MoE-training page (the diagram of the MXFP8 expert layer:
 // router output -> BF16 -> MXFP8 -> grouped GEMM -> BF16 -> all-to-all
@@ -192,8 +196,12 @@ struct PlaceArgs {
   const int32_t* row;       // destination rows [n_src * fan]
   const int32_t* counts;    // [E] real rows per group (padding clearing)
   const int32_t* offsets;   // [E+1] padded group starts
-  uint8_t* q;               // E4M3 rows [m_rows, k]
+  uint8_t* q;               // E4M3 rows [m_rows, k] (PEER: this rank's receive rows, padding only)
   uint8_t* sf;              // scales of q: tiled, or row-major [m_rows, k/32]
+  uint8_t* const* q_peers;  // PEER: [ranks] every rank's receive rows [m_rows, k]
+  uint8_t* const* sf_peers; // PEER: [ranks] their tiled scales
+  const int32_t* row_rank;  // PEER: destination rank of each destination row [n_src * fan]
+  int ranks;
   int32_t* status;
   int64_t n_src;
   int64_t m_rows;
@@ -204,10 +212,10 @@ struct PlaceArgs {
   int sf_row_major;
 };
 
-// Scale word of blocks c..c+3 (c % 4 == 0) of row r.
-__device__ __forceinline__ uint32_t* scale_word(const PlaceArgs& a, int64_t r, uint32_t c, uint32_t kb) {
+// Scale word of blocks c..c+3 (c % 4 == 0) of row r of the scales at sf.
+__device__ __forceinline__ uint32_t* scale_word(const PlaceArgs& a, uint8_t* sf, int64_t r, uint32_t c, uint32_t kb) {
   const int64_t off = a.sf_row_major ? r * kb + c : static_cast<int64_t>(sf_tiled_offset(static_cast<uint32_t>(r), c, kb / 4));
-  return reinterpret_cast<uint32_t*>(a.sf + off);
+  return reinterpret_cast<uint32_t*>(sf + off);
 }
 
 // One warp per (source row, chunk of 32 blocks = 1024 elements): QUANT
@@ -216,8 +224,11 @@ __device__ __forceinline__ uint32_t* scale_word(const PlaceArgs& a, int64_t r, u
 // of the row's `fan` destinations.  The warps after the last source chunk
 // clear the group padding rows (E4M3 0, scale 0: the quantisation of a zero
 // row), one (padding slot, chunk) each.  Splitting rows into chunks keeps
-// enough warps in flight when there are few tokens.
-template <bool QUANT>
+// enough warps in flight when there are few tokens.  PEER: destination j of a
+// row is row `row` of rank `row_rank`'s receive buffer, reached through the
+// pointer tables (another GPU's memory over NVLink, by plain stores); the
+// padding rows cleared are those of this rank's own receive buffer.
+template <bool QUANT, bool PEER>
 __global__ void __launch_bounds__(kRowWarps * 32) moe_place_kernel(const PlaceArgs a) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -271,14 +282,25 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_place_kernel(const PlaceAr
     for (int j = 0; j < a.fan; ++j) {
       const int32_t r = a.row[src * a.fan + j];
       if (r < 0) continue;  // a dropped entry
+      uint8_t* qb = a.q;
+      uint8_t* sfb = a.sf;
+      if constexpr (PEER) {
+        const int32_t rk = a.row_rank[src * a.fan + j];
+        if (rk < 0 || rk >= a.ranks) {
+          if (lane == 0) moe_report(a.status, kDevBadIndex);
+          continue;
+        }
+        qb = a.q_peers[rk];
+        sfb = a.sf_peers[rk];
+      }
       if (r >= a.m_rows) {
         if (lane == 0) moe_report(a.status, kDevBadIndex);
         continue;
       }
-      uint4* dst = reinterpret_cast<uint4*>(a.q) + (static_cast<int64_t>(r) * kb + b0) * 2;
+      uint4* dst = reinterpret_cast<uint4*>(qb) + (static_cast<int64_t>(r) * kb + b0) * 2;
       if (on0) dst[lane] = st0;
       if (on1) dst[32 + lane] = st1;
-      if (on && (lane & 3) == 0) *scale_word(a, r, b, kb) = word;
+      if (on && (lane & 3) == 0) *scale_word(a, sfb, r, b, kb) = word;
     }
     return;
   }
@@ -300,7 +322,7 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_place_kernel(const PlaceAr
     uint4* dst = reinterpret_cast<uint4*>(a.q) + (r * kb + b) * 2;
     dst[0] = make_uint4(0, 0, 0, 0);
     dst[1] = make_uint4(0, 0, 0, 0);
-    if ((lane & 3) == 0) *scale_word(a, r, b, kb) = 0;
+    if ((lane & 3) == 0) *scale_word(a, a.sf, r, b, kb) = 0;
   }
 }
 
@@ -331,9 +353,15 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_gather_kernel(const uint4*
 // out[t, :] = sum_j w[t, j] * y[row[t*topk + j], :], FP32 fused multiply-adds
 // in j order, rounded once to BF16 (RNE).  One warp per (token, chunk of 256
 // columns): 8 columns (one 16-byte vector) per lane, four routed rows' loads
-// in flight.
-__global__ void __launch_bounds__(kRowWarps * 32) moe_combine_kernel(const uint4* __restrict__ y, int64_t y_rows,
-                                                                     int64_t n_vecs, const int32_t* __restrict__ row,
+// in flight.  PEER: routed row j of a token is row `row` of rank `row_rank`'s
+// expert output, read through the pointer table (another GPU's memory over
+// NVLink, by plain loads).
+template <bool PEER>
+__global__ void __launch_bounds__(kRowWarps * 32) moe_combine_kernel(const uint4* __restrict__ y,
+                                                                     const uint4* const* __restrict__ y_peers,
+                                                                     const int32_t* __restrict__ row_rank, int ranks,
+                                                                     int64_t y_rows, int64_t n_vecs,
+                                                                     const int32_t* __restrict__ row,
                                                                      const float* __restrict__ wt, int64_t tokens,
                                                                      int topk, uint4* __restrict__ out,
                                                                      int32_t* status) {
@@ -359,12 +387,22 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_combine_kernel(const uint4
       for (int u = 0; u < 4; ++u) {
         const int j = j0 + u;
         int32_t r = j < topk ? rt[j] : -1;
+        const uint4* yb = y;
+        if (PEER && r >= 0) {
+          const int32_t rk = row_rank[t * topk + j];
+          if (rk < 0 || rk >= ranks) {
+            bad = true;
+            r = -1;
+          } else {
+            yb = y_peers[rk];
+          }
+        }
         if (r >= y_rows) {
           bad = true;
           r = -1;
         }
         wj[u] = r >= 0 ? wt_t[j] : 0.0f;
-        v[u] = r >= 0 ? __ldcs(y + static_cast<int64_t>(r) * n_vecs + c) : make_uint4(0, 0, 0, 0);
+        v[u] = r >= 0 ? __ldcs(yb + static_cast<int64_t>(r) * n_vecs + c) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -387,6 +425,106 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_combine_kernel(const uint4
     out[t * n_vecs + c] = o;
   }
   if (bad && lane == 0) moe_report(status, kDevBadIndex);
+}
+
+// ------------------------------------------------------------------ expert-parallel placement plan
+// Rank `rank` of `ranks` owns the experts [rank * el, (rank + 1) * el),
+// el = E / ranks.  count[src][e] is the number of entries rank src routes to
+// (global) expert e; this rank's entries were routed with pad 1, so
+// row_send[i] = (its entries for experts before e) + (the rank of entry i
+// among its entries for e).  On the owner o = e / el, expert e's rows come
+// source rank by source rank, each source's in its own order, and every
+// local expert's group is padded to `pad` rows:
+//   dst_rank[i] = o
+//   dst_row[i]  = gstart(e) + sum_{src < rank} count[src][e] + (row_send[i] - own_start(e))
+// with gstart(e) the padded start of e among its owner's experts.  Block 0
+// also writes this rank's own receive plan: counts_local[l] = total entries
+// of expert rank * el + l over all sources, offsets_local = their padded
+// starts (el + 1 values).  An id outside [0, E) is a dropped entry (-1, -1).
+constexpr int kPlanThreads = 256;
+
+__global__ void __launch_bounds__(kPlanThreads) moe_peer_plan_kernel(
+    const int32_t* __restrict__ ids, const int32_t* __restrict__ row_send, int64_t n,
+    const int32_t* __restrict__ count, int ranks, int rank, int E, int pad, int32_t* __restrict__ dst_rank,
+    int32_t* __restrict__ dst_row, int32_t* __restrict__ counts_local, int32_t* __restrict__ offsets_local,
+    int32_t* status) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  extern __shared__ int32_t plan_sh[];
+  int32_t* tot = plan_sh;     // [E] entries of expert e over all source ranks
+  int32_t* pre = tot + E;     // [E] ... over the source ranks before this one
+  int32_t* own = pre + E;     // [E] this rank's entries of e
+  int32_t* start = own + E;   // [E] this rank's entries of the experts before e
+  int32_t* gsc = start + E;   // [E] exclusive scan of the padded totals over all experts
+  const int el = E / ranks;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t t = 0, p = 0;
+    for (int src = 0; src < ranks; ++src) {
+      const int32_t c = __ldg(count + static_cast<int64_t>(src) * E + e);
+      t += c;
+      if (src < rank) p += c;
+    }
+    tot[e] = t;
+    pre[e] = p;
+    own[e] = __ldg(count + static_cast<int64_t>(rank) * E + e);
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // two exclusive scans, 32 experts per step
+    const int lane = threadIdx.x;
+    int32_t carry_s = 0, carry_g = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane;
+      const int32_t vs = e < E ? own[e] : 0;
+      const int32_t vg = e < E ? (tot[e] + pad - 1) / pad * pad : 0;
+      int32_t xs = vs, xg = vg;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t ys = __shfl_up_sync(0xFFFFFFFFu, xs, o);
+        const int32_t yg = __shfl_up_sync(0xFFFFFFFFu, xg, o);
+        if (lane >= o) {
+          xs += ys;
+          xg += yg;
+        }
+      }
+      if (e < E) {
+        start[e] = carry_s + xs - vs;
+        gsc[e] = carry_g + xg - vg;
+      }
+      carry_s += __shfl_sync(0xFFFFFFFFu, xs, 31);
+      carry_g += __shfl_sync(0xFFFFFFFFu, xg, 31);
+    }
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    const int e0 = rank * el;
+    for (int l = threadIdx.x; l <= el; l += blockDim.x) {
+      if (l < el) {
+        counts_local[l] = tot[e0 + l];
+        offsets_local[l] = gsc[e0 + l] - gsc[e0];
+      } else {
+        offsets_local[el] = gsc[e0 + el - 1] - gsc[e0] + (tot[e0 + el - 1] + pad - 1) / pad * pad;
+      }
+    }
+  }
+  bool bad = false;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int32_t e = ids[i];
+    int32_t dr = -1, drow = -1;
+    if (e >= 0 && e < E) {
+      const int32_t within = row_send[i] - start[e];
+      if (within < 0 || within >= own[e]) {
+        bad = true;
+      } else {
+        const int o = e / el;
+        dr = o;
+        drow = gsc[e] - gsc[o * el] + pre[e] + within;
+      }
+    }
+    dst_rank[i] = dr;
+    dst_row[i] = drow;
+  }
+  if (bad) moe_report(status, kDevBadIndex);
 }
 
 // ======================================================================= host
@@ -453,14 +591,21 @@ cudaError_t launch_moe_place(const MoePlace& p, cudaStream_t stream) {
   a.E = p.pad > 1 ? p.experts : 0;
   a.pad_slots = p.pad > 1 ? p.pad - 1 : 0;
   a.sf_row_major = p.sf_row_major;
+  a.q_peers = reinterpret_cast<uint8_t* const*>(p.q_peers);
+  a.sf_peers = reinterpret_cast<uint8_t* const*>(p.sf_peers);
+  a.row_rank = p.row_rank;
+  a.ranks = p.ranks;
+  const bool peer = p.q_peers != nullptr;
   const int64_t chunks = (p.k / 32 + 31) / 32;
   const int64_t warps = (p.n_src + static_cast<int64_t>(a.E) * a.pad_slots) * chunks;
   if (warps == 0) return cudaSuccess;
   const int64_t grid = (warps + kRowWarps - 1) / kRowWarps;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
   void* args[] = {&a};
-  const void* f = p.quantize ? reinterpret_cast<const void*>(moe_place_kernel<true>)
-                             : reinterpret_cast<const void*>(moe_place_kernel<false>);
+  const void* f = peer ? (p.quantize ? reinterpret_cast<const void*>(moe_place_kernel<true, true>)
+                                     : reinterpret_cast<const void*>(moe_place_kernel<false, true>))
+                       : (p.quantize ? reinterpret_cast<const void*>(moe_place_kernel<true, false>)
+                                     : reinterpret_cast<const void*>(moe_place_kernel<false, false>));
   return launch_pdl_cfg(f, dim3(static_cast<unsigned>(grid)), dim3(kRowWarps * 32), 0, args, stream);
 }
 
@@ -477,18 +622,35 @@ cudaError_t launch_moe_gather(const void* src, int64_t src_rows, int64_t row_byt
                         dim3(kRowWarps * 32), 0, args, stream);
 }
 
-cudaError_t launch_moe_combine(const void* y, int64_t y_rows, int64_t n_cols, const int32_t* row, const float* w,
-                               int64_t tokens, int topk, void* out, int32_t* status, cudaStream_t stream) {
+cudaError_t launch_moe_combine(const void* y, const void* const* y_peers, const int32_t* row_rank, int ranks,
+                               int64_t y_rows, int64_t n_cols, const int32_t* row, const float* w, int64_t tokens,
+                               int topk, void* out, int32_t* status, cudaStream_t stream) {
   if (tokens == 0) return cudaSuccess;
   const int64_t warps = tokens * ((n_cols / 8 + 31) / 32);
   const int64_t grid = (warps + kRowWarps - 1) / kRowWarps;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
   const uint4* yp = static_cast<const uint4*>(y);
+  const uint4* const* ypp = reinterpret_cast<const uint4* const*>(y_peers);
   uint4* op = static_cast<uint4*>(out);
   int64_t vecs = n_cols / 8;
-  void* args[] = {&yp, &y_rows, &vecs, &row, &w, &tokens, &topk, &op, &status};
-  return launch_pdl_cfg(reinterpret_cast<const void*>(moe_combine_kernel), dim3(static_cast<unsigned>(grid)),
-                        dim3(kRowWarps * 32), 0, args, stream);
+  void* args[] = {&yp, &ypp, &row_rank, &ranks, &y_rows, &vecs, &row, &w, &tokens, &topk, &op, &status};
+  const void* f = y_peers ? reinterpret_cast<const void*>(moe_combine_kernel<true>)
+                          : reinterpret_cast<const void*>(moe_combine_kernel<false>);
+  return launch_pdl_cfg(f, dim3(static_cast<unsigned>(grid)), dim3(kRowWarps * 32), 0, args, stream);
+}
+
+cudaError_t launch_moe_peer_plan(const int32_t* ids, const int32_t* row_send, int64_t n, const int32_t* count,
+                                 int ranks, int rank, int E, int pad, int32_t* dst_rank, int32_t* dst_row,
+                                 int32_t* counts_local, int32_t* offsets_local, int32_t* status, int num_sms,
+                                 cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(5) * E * 4;  // at most 20 KB (E = 1024)
+  int64_t grid = (n + kPlanThreads - 1) / kPlanThreads;
+  if (grid < 1) grid = 1;  // block 0 writes the receive plan even with no entries
+  if (grid > 2 * static_cast<int64_t>(num_sms)) grid = 2 * static_cast<int64_t>(num_sms);
+  void* args[] = {&ids, &row_send, &n, &count, &ranks, &rank, &E, &pad, &dst_rank, &dst_row,
+                  &counts_local, &offsets_local, &status};
+  return launch_pdl_cfg(reinterpret_cast<const void*>(moe_peer_plan_kernel), dim3(static_cast<unsigned>(grid)),
+                        dim3(kPlanThreads), smem, args, stream);
 }
 
 }  // namespace mxk

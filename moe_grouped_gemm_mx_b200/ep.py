@@ -24,6 +24,17 @@ are NCCL all-to-alls through torch.distributed; their split sizes need one
 device-to-host read of the row counts per exchange.  Every step of the data
 path is a library kernel; this module only sequences them (``ops``), and the
 few index vectors it builds with torch are bookkeeping over the count table.
+
+``ep_moe_layer_peer`` is the same layer with the exchange fused into the
+kernels over peer memory instead of all-to-alls: every rank's receive and
+output buffers are mapped on every rank (``PeerBuffers``); after an
+all-gather of the per-expert counts, one plan kernel gives each entry its
+owner and its row there, the dispatch kernel quantises each token once and
+stores its MXFP8 row straight into the owner's receive buffer (NVLink
+stores), the owner runs its experts in place, and the combine kernel loads
+the expert outputs straight from the owners' buffers (NVLink loads) into the
+gate-weighted sum.  Stream-ordered barriers (a one-element all-reduce)
+separate the three phases; no kernel waits on another rank.
 """
 from __future__ import annotations
 
@@ -55,14 +66,24 @@ class LibraryOps:
     def gate_up_swiglu(self, qa, sfa, q13, sf13, offsets):
         return self.mx.mx_grouped_gemm_contiguous_swiglu_quant(qa, sfa, q13, sf13, offsets)
 
-    def down(self, qh, sfh, q2, sf2, offsets):
-        return self.mx.mx_grouped_gemm_contiguous(qh, sfh, q2, sf2, offsets)
+    def down(self, qh, sfh, q2, sf2, offsets, d=None):
+        return self.mx.mx_grouped_gemm_contiguous(qh, sfh, q2, sf2, offsets, d=d)
 
     def gather(self, src, idx):
         return self.mx.mx_gather_rows(src, idx)
 
     def combine(self, y, row, w):
         return self.mx.mx_moe_combine(y, row, w)
+
+    def peer_plan(self, ids, row_send, count_table, rank, experts, pad):
+        return self.mx.mx_moe_peer_plan(ids, row_send, count_table, rank, experts, pad)
+
+    def dispatch_peer(self, x, dst_rank, dst_row, topk, bufs, counts_l, offsets_l, pad):
+        self.mx.mx_moe_dispatch_quant_peer(x, dst_rank, dst_row, topk, bufs.q_ptrs, bufs.sf_ptrs, bufs.m_cap,
+                                           bufs.q, bufs.sf, counts_l, offsets_l, pad)
+
+    def combine_peer(self, bufs, n, dst_rank, dst_row, w):
+        return self.mx.mx_moe_combine_peer(bufs.y_ptrs, bufs.m_cap, n, dst_rank, dst_row, w)
 
 
 def _all_to_all_rows(src: torch.Tensor, send_rows, recv_rows, group):
@@ -132,3 +153,143 @@ def ep_moe_layer(x: torch.Tensor, ids: torch.Tensor, gate_w: torch.Tensor, exper
     else:
         y_home = y_back
     return ops.combine(y_home, row_send, gate_w)
+
+
+# ---------------------------------------------------------------- exchange over peer memory
+
+class PeerBuffers:
+    """One rank's buffers for the peer-memory exchange, and device tables of
+    every rank's addresses of the same buffers.
+
+    q  uint8 [m_cap, H]: the MXFP8 rows routed to this rank's experts;
+    sf uint8: their tiled scales (``scale_bytes(m_cap, H)``);
+    y  BF16 [m_cap, N]: this rank's expert outputs, row for row;
+    q_ptrs / sf_ptrs / y_ptrs  int64 [ranks] device tensors (rank r's address).
+    m_cap must hold the rows of the largest plan any rank receives (at most
+    mx_moe_max_rows(ranks * tokens * topk, E / ranks, pad))."""
+
+    def __init__(self, q, sf, y, q_ptrs, sf_ptrs, y_ptrs, rank):
+        self.q, self.sf, self.y = q, sf, y
+        self.q_ptrs, self.sf_ptrs, self.y_ptrs = q_ptrs, sf_ptrs, y_ptrs
+        self.rank = rank
+        self.ranks = q_ptrs.numel()
+        self.m_cap = q.shape[0]
+
+    @staticmethod
+    def _alloc(alloc, m_cap, H, N, device, scale_bytes):
+        q = alloc((m_cap, H), torch.uint8, device)
+        sf = alloc((scale_bytes(m_cap, H),), torch.uint8, device)
+        y = alloc((m_cap, N), torch.bfloat16, device)
+        return q, sf, y
+
+    @classmethod
+    def emulated(cls, ranks: int, m_cap: int, H: int, N: int, device, mx=None):
+        """``ranks`` ranks' buffers on one GPU, one PeerBuffers per emulated
+        rank, all sharing the same address tables (the kernels see exactly
+        what they would see with each buffer on its own GPU)."""
+        if mx is None:
+            import moe_grouped_gemm_mx_b200 as mx
+        bufs = [cls._alloc(lambda shape, dt, dev: torch.empty(shape, dtype=dt, device=dev), m_cap, H, N, device,
+                           mx.scale_bytes) for _ in range(ranks)]
+        tables = [torch.tensor([b[i].data_ptr() for b in bufs], dtype=torch.int64, device=device) for i in range(3)]
+        return [cls(*bufs[r], *tables, r) for r in range(ranks)]
+
+    @classmethod
+    def symmetric(cls, m_cap: int, H: int, N: int, group=None, mx=None):
+        """Buffers in torch's symmetric memory, mapped on every rank of
+        ``group`` (one process per GPU; peers reached over NVLink)."""
+        if mx is None:
+            import moe_grouped_gemm_mx_b200 as mx
+        import torch.distributed._symmetric_memory as symm
+        group = dist.group.WORLD if group is None else group
+        device = torch.device("cuda", torch.cuda.current_device())
+        bufs = cls._alloc(lambda shape, dt, dev: symm.empty(*shape, dtype=dt, device=dev), m_cap, H, N, device,
+                          mx.scale_bytes)
+        tables = []
+        for b in bufs:
+            h = symm.rendezvous(b, group)
+            tables.append(torch.tensor(list(h.buffer_ptrs), dtype=torch.int64, device=device))
+        return cls(*bufs, *tables, dist.get_rank(group))
+
+
+def peer_dispatch(x, ids, experts, count_table, bufs: PeerBuffers, ops=None, pad: int = 128):
+    """Phase 1 on one rank: plan this rank's entries against the all-ranks
+    count table and store every routed MXFP8 row in its owner's receive
+    buffer.  Returns the plan (dst_rank, dst_row, counts_local, offsets_local)."""
+    ops = LibraryOps() if ops is None else ops
+    T, topk = ids.shape
+    flat = ids.reshape(-1)
+    _, _, row_send = ops.route(flat, experts, 1)
+    dst_rank, dst_row, counts_l, offsets_l = ops.peer_plan(flat, row_send, count_table, bufs.rank, experts, pad)
+    ops.dispatch_peer(x, dst_rank, dst_row, topk, bufs, counts_l, offsets_l, pad)
+    return dst_rank, dst_row, counts_l, offsets_l
+
+
+def peer_experts(bufs: PeerBuffers, plan, q13, sf13, q2, sf2, ops=None):
+    """Phase 2 on one rank: its experts over its receive buffer, the outputs
+    left in its output buffer y (row for row)."""
+    ops = LibraryOps() if ops is None else ops
+    offsets_l = plan[3]
+    qh, sfh = ops.gate_up_swiglu(bufs.q, bufs.sf, q13, sf13, offsets_l)
+    ops.down(qh, sfh, q2, sf2, offsets_l, d=bufs.y)
+
+
+def peer_combine(bufs: PeerBuffers, plan, gate_w, n: int, ops=None):
+    """Phase 3 on one rank: the gate-weighted sum of its tokens' expert
+    outputs, loaded from their owners' output buffers."""
+    ops = LibraryOps() if ops is None else ops
+    return ops.combine_peer(bufs, n, plan[0], plan[1], gate_w)
+
+
+def route_counts(ids, experts, ops=None):
+    """This rank's entries per global expert (the row of the count table)."""
+    ops = LibraryOps() if ops is None else ops
+    counts, _, _ = ops.route(ids.reshape(-1), experts, 1)
+    return counts
+
+
+def _stream_barrier(group):
+    """Every rank's work so far on its current stream is complete before any
+    rank's later work on its stream starts (a one-element all-reduce)."""
+    t = torch.zeros(1, dtype=torch.int32, device=torch.device("cuda", torch.cuda.current_device()))
+    dist.all_reduce(t, group=group)
+
+
+def ep_moe_layer_peer(x: torch.Tensor, ids: torch.Tensor, gate_w: torch.Tensor, experts: int,
+                      q13, sf13, q2, sf2, bufs: PeerBuffers, group=None, ops=None, pad: int = 128) -> torch.Tensor:
+    """One expert-parallel MoE layer on this rank with the exchange over peer
+    memory (arguments as ep_moe_layer; ``bufs`` from PeerBuffers.symmetric).
+    Returns BF16 [T, N]."""
+    ops = LibraryOps() if ops is None else ops
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    if experts % world or bufs.ranks != world:
+        raise ValueError("the experts must divide evenly over the ranks, one buffer set per rank")
+    counts = route_counts(ids, experts, ops)
+    if world > 1:
+        table = torch.empty((world, experts), dtype=torch.int32, device=counts.device)
+        dist.all_gather_into_tensor(table, counts, group=group)
+    else:
+        table = counts.view(1, experts)
+    plan = peer_dispatch(x, ids, experts, table, bufs, ops, pad)
+    if world > 1:
+        _stream_barrier(group)
+    peer_experts(bufs, plan, q13, sf13, q2, sf2, ops)
+    if world > 1:
+        _stream_barrier(group)
+    out = peer_combine(bufs, plan, gate_w, bufs.y.shape[1], ops)
+    if world > 1:
+        _stream_barrier(group)  # the outputs are read before any rank overwrites its buffers
+    return out
+
+
+def ep_moe_layer_peer_emulated(xs, ids_list, gate_ws, experts, weights, bufs_list, ops=None, pad: int = 128):
+    """The peer-memory layer for R ranks emulated on one GPU: each phase runs
+    for every rank before the next phase starts (what the barriers of
+    ep_moe_layer_peer guarantee).  weights[r] = (q13, sf13, q2, sf2) of rank
+    r's experts.  Returns every rank's output."""
+    ops = LibraryOps() if ops is None else ops
+    table = torch.stack([route_counts(ids, experts, ops) for ids in ids_list])
+    plans = [peer_dispatch(xs[r], ids_list[r], experts, table, bufs_list[r], ops, pad) for r in range(len(xs))]
+    for r in range(len(xs)):
+        peer_experts(bufs_list[r], plans[r], *weights[r], ops)
+    return [peer_combine(bufs_list[r], plans[r], gate_ws[r], bufs_list[r].y.shape[1], ops) for r in range(len(xs))]

@@ -53,6 +53,9 @@ def lib():
     L.mx_moe_scatter_rows.argtypes = [P, P, I64, I64, P, P, P, I32, I32, I64, P, P, P, P]
     L.mx_gather_rows.argtypes = [P, I64, I64, P, I64, P, P, P]
     L.mx_moe_combine.argtypes = [P, I64, I64, P, P, I64, I32, P, P, P]
+    L.mx_moe_peer_plan.argtypes = [P, P, I64, P, I32, I32, I32, I32, P, P, P, P, P, P]
+    L.mx_moe_dispatch_quant_peer.argtypes = [P, I64, I64, P, P, I32, P, P, I32, I64, P, P, P, P, I32, I32, P, P]
+    L.mx_moe_combine_peer.argtypes = [P, I32, I64, I64, P, P, P, I64, I32, P, P, P]
     return L
 
 
@@ -223,3 +226,33 @@ def test_moe_argument_checks(lib):
     assert lib.mx_moe_combine(A, 8, 16, B, C + 2, 4, 2, D, None, None) == MX_ERR_MISALIGNED
     assert lib.mx_moe_combine(A, 8, 16, None, C, 4, 2, D, None, None) == MX_ERR_INVALID_ARGUMENT
     assert lib.mx_moe_combine(A, 8, 16, B, C, 0, 2, D, None, None) == MX_OK
+
+
+def test_moe_peer_argument_checks(lib):
+    A, B, C, D, E, F, G = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000
+    plan = lib.mx_moe_peer_plan
+    # ranks in [1, 1024], rank in [0, ranks), experts % ranks == 0, pad in [1, 128]
+    assert plan(A, B, 16, C, 0, 0, 8, 128, D, E, F, G, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert plan(A, B, 16, C, 2, 2, 8, 128, D, E, F, G, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert plan(A, B, 16, C, 3, 0, 8, 128, D, E, F, G, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert plan(A, B, 16, C, 2, 0, 8, 0, D, E, F, G, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert plan(A, B, 16, None, 2, 0, 8, 128, D, E, F, G, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert plan(A, B, 16, C, 2, 0, 8, 128, None, E, F, G, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert plan(A + 2, B, 16, C, 2, 0, 8, 128, D, E, F, G, None, None) == MX_ERR_MISALIGNED
+    assert plan(A, B, 1 << 30, C, 4, 0, 8, 128, D, E, F, G, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    disp = lib.mx_moe_dispatch_quant_peer
+    # the dispatch's rules, plus ranks and 8-byte aligned pointer tables
+    assert disp(A, 4, 128, B, C, 2, D, E, 0, 128, F, G, A, B, 4, 128, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert disp(A, 4, 96, B, C, 2, D, E, 2, 128, F, G, A, B, 4, 128, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert disp(A, 4, 128, B, C, 2, D, E, 2, 100, F, G, A, B, 4, 128, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert disp(A, 4, 128, B, C, 2, None, E, 2, 128, F, G, A, B, 4, 128, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert disp(A, 4, 128, None, C, 2, D, E, 2, 128, F, G, A, B, 4, 128, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert disp(A, 4, 128, B, C, 2, D + 4, E, 2, 128, F, G, A, B, 4, 128, None, None) == MX_ERR_MISALIGNED
+    assert disp(A, 4, 128, B, C, 2, D, E, 2, 128, F, G, None, None, 4, 128, None, None) == MX_ERR_INVALID_ARGUMENT
+    comb = lib.mx_moe_combine_peer
+    assert comb(A, 0, 8, 16, B, C, D, 4, 2, E, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert comb(A, 2, 8, 12, B, C, D, 4, 2, E, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert comb(A, 2, 8, 16, B, C, D, 4, 65, E, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert comb(None, 2, 8, 16, B, C, D, 4, 2, E, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert comb(A + 4, 2, 8, 16, B, C, D, 4, 2, E, None, None) == MX_ERR_MISALIGNED
+    assert comb(A, 2, 8, 16, B, C, D, 0, 2, E, None, None) == MX_OK
