@@ -248,10 +248,11 @@ def route_counts(ids, experts, ops=None):
     return counts
 
 
-def _stream_barrier(group):
+def _stream_barrier(group, device):
     """Every rank's work so far on its current stream is complete before any
-    rank's later work on its stream starts (a one-element all-reduce)."""
-    t = torch.zeros(1, dtype=torch.int32, device=torch.device("cuda", torch.cuda.current_device()))
+    rank's later work on its stream starts (a one-element all-reduce on the
+    stream; on CPU ranks, a plain barrier)."""
+    t = torch.zeros(1, dtype=torch.int32, device=device)
     dist.all_reduce(t, group=group)
 
 
@@ -266,19 +267,20 @@ def ep_moe_layer_peer(x: torch.Tensor, ids: torch.Tensor, gate_w: torch.Tensor, 
         raise ValueError("the experts must divide evenly over the ranks, one buffer set per rank")
     counts = route_counts(ids, experts, ops)
     if world > 1:
-        table = torch.empty((world, experts), dtype=torch.int32, device=counts.device)
-        dist.all_gather_into_tensor(table, counts, group=group)
+        parts = [torch.empty_like(counts) for _ in range(world)]
+        dist.all_gather(parts, counts, group=group)
+        table = torch.stack(parts)
     else:
         table = counts.view(1, experts)
     plan = peer_dispatch(x, ids, experts, table, bufs, ops, pad)
     if world > 1:
-        _stream_barrier(group)
+        _stream_barrier(group, x.device)
     peer_experts(bufs, plan, q13, sf13, q2, sf2, ops)
     if world > 1:
-        _stream_barrier(group)
+        _stream_barrier(group, x.device)
     out = peer_combine(bufs, plan, gate_w, bufs.y.shape[1], ops)
     if world > 1:
-        _stream_barrier(group)  # the outputs are read before any rank overwrites its buffers
+        _stream_barrier(group, x.device)  # the outputs are read before any rank overwrites its buffers
     return out
 
 

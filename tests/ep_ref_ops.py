@@ -48,12 +48,15 @@ class OracleOps:
             qh[: len(h)], sfh[: len(h)] = oracle.quantize_f32(h)
         return torch.from_numpy(qh), torch.from_numpy(sfh)
 
-    def down(self, qh, sfh, q2, sf2, offsets):
+    def down(self, qh, sfh, q2, sf2, offsets, d=None):
         off = _np(offsets).astype(np.int32)
-        d, _ = oracle.grouped_contiguous(_np(qh), _np(sfh), _np(q2), _np(sf2), off)
-        out = np.zeros((qh.shape[0], d.shape[1]), dtype=np.float64)
-        out[: len(d)] = d
-        return _bf16(out)
+        dd, _ = oracle.grouped_contiguous(_np(qh), _np(sfh), _np(q2), _np(sf2), off)
+        out = np.zeros((qh.shape[0], dd.shape[1]), dtype=np.float64)
+        out[: len(dd)] = dd
+        if d is None:
+            return _bf16(out)
+        d.copy_(_bf16(out))
+        return d
 
     def gather(self, src, idx):
         return src[torch.as_tensor(_np(idx)).long()]
@@ -61,3 +64,51 @@ class OracleOps:
     def combine(self, y, row, w):
         out, _ = oracle.moe_combine(y.contiguous(), _np(row), _np(w))
         return _bf16(out)
+
+    # -- the exchange over peer memory, with every rank's buffers as shared
+    # CPU tensors (bufs.peer_q / peer_sf / peer_y, indexed by rank)
+
+    def peer_plan(self, ids, row_send, count_table, rank, experts, pad):
+        """The placement from the count table alone (what each rank can
+        compute): owner o = e // (E/R); row = padded start of e among o's
+        experts + entries of e on the ranks before this one + the entry's
+        rank among this rank's entries of e."""
+        ids, table = _np(ids).reshape(-1), _np(count_table)
+        ranks = table.shape[0]
+        el = experts // ranks
+        tot = table.sum(0)
+        padded = (tot + pad - 1) // pad * pad
+        before = table[:rank].sum(0)
+        seen = np.zeros(experts, dtype=np.int64)
+        dst_rank = np.full(ids.size, -1, dtype=np.int32)
+        dst_row = np.full(ids.size, -1, dtype=np.int32)
+        for i, e in enumerate(ids):
+            if 0 <= e < experts:
+                o = e // el
+                dst_rank[i] = o
+                dst_row[i] = padded[o * el:e].sum() + before[e] + seen[e]
+                seen[e] += 1
+        mine = slice(rank * el, (rank + 1) * el)
+        offsets = np.concatenate([[0], np.cumsum(padded[mine])]).astype(np.int32)
+        return (torch.from_numpy(dst_rank), torch.from_numpy(dst_row), torch.from_numpy(tot[mine].astype(np.int32)),
+                torch.from_numpy(offsets))
+
+    def dispatch_peer(self, x, dst_rank, dst_row, topk, bufs, counts_l, offsets_l, pad):
+        q, sf = oracle.quantize(x)
+        for i, (rk, r) in enumerate(zip(_np(dst_rank).tolist(), _np(dst_row).tolist())):
+            if r >= 0:
+                bufs.peer_q[rk][r] = torch.from_numpy(q[i // topk])
+                bufs.peer_sf[rk][r] = torch.from_numpy(sf[i // topk])
+        cl, ol = _np(counts_l), _np(offsets_l)
+        for l in range(cl.size):                # this rank's own padding rows
+            bufs.q[ol[l] + cl[l]:ol[l + 1]] = 0
+            bufs.sf[ol[l] + cl[l]:ol[l + 1]] = 0
+
+    def combine_peer(self, bufs, n, dst_rank, dst_row, w):
+        dr, drow = _np(dst_rank).reshape(-1), _np(dst_row).reshape(-1)
+        y = torch.zeros((dr.size, n), dtype=torch.bfloat16)
+        for i, (rk, r) in enumerate(zip(dr.tolist(), drow.tolist())):
+            if r >= 0:
+                y[i] = bufs.peer_y[rk][r]
+        rows = np.where(drow >= 0, np.arange(dr.size), -1).astype(np.int32)
+        return self.combine(y, rows, w)

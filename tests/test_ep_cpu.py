@@ -2,7 +2,10 @@
 plumbing (per-expert count exchange, the row all-to-alls with uneven and
 empty splits, the receive-side plan, the return path and the combine) gives
 exactly the output of the same layer computed in one process over all
-tokens and all experts.  The steps that run as CUDA kernels on a GPU are
+tokens and all experts; so does the layer with the exchange over peer
+memory (count all-gather, placement, stores into the owners' receive
+buffers and loads from their outputs, the barriers between the phases),
+with every rank's buffers as shared-memory CPU tensors.  The steps that run as CUDA kernels on a GPU are
 replaced by oracle-backed CPU stand-ins (tests/ep_ref_ops.py), identical in
 both runs, so any difference is the plumbing's."""
 import datetime
@@ -105,3 +108,56 @@ def test_ep_ranks_match_one_process(world, case):
         assert np.array_equal(out[r], ref_bits[t0:t1]), f"rank {r}"
         t0 = t1
     assert np.abs(ref.float().numpy()).max() > 0      # the layer produced something
+
+
+def _rank_main_peer(rank, world, port, case, shared, out):
+    import torch.distributed as dist
+    sys.path[:0] = [ROOT, TESTS]
+    from ep_ref_ops import OracleOps
+    from moe_grouped_gemm_mx_b200.ep import PeerBuffers, ep_moe_layer_peer
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        ranks, (q13, sf13, q2, sf2), E = _problem(case, world)
+        x, ids, gw = ranks[rank]
+        lo, hi = rank * (E // world), (rank + 1) * (E // world)
+        q_all, sf_all, y_all = shared
+        no_table = torch.zeros(world, dtype=torch.int64)     # the CPU stand-ins index the shared tensors instead
+        bufs = PeerBuffers(q_all[rank], sf_all[rank], y_all[rank], no_table, no_table, no_table, rank)
+        bufs.peer_q, bufs.peer_sf, bufs.peer_y = q_all, sf_all, y_all
+        y = ep_moe_layer_peer(x, torch.from_numpy(ids), torch.from_numpy(gw), E,
+                              torch.from_numpy(q13[lo:hi].copy()), torch.from_numpy(sf13[lo:hi].copy()),
+                              torch.from_numpy(q2[lo:hi].copy()), torch.from_numpy(sf2[lo:hi].copy()),
+                              bufs, ops=OracleOps())
+        out[rank] = y.view(torch.int16).numpy().copy()
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,case", [(2, "uniform"), (2, "skewed"), (4, "skewed")])
+def test_ep_peer_ranks_match_one_process(world, case):
+    from ep_ref_ops import OracleOps
+    from moe_grouped_gemm_mx_b200.ep import ep_moe_layer
+    ranks, (q13, sf13, q2, sf2), E = _problem(case, world)
+    entries = sum(r[1].size for r in ranks)
+    el = E // world
+    m_cap = (entries + el * 127 + 127) // 128 * 128
+    shared = ([torch.full((m_cap, H), 0xAB, dtype=torch.uint8).share_memory_() for _ in range(world)],
+              [torch.full((m_cap, H // 32), 0xCD, dtype=torch.uint8).share_memory_() for _ in range(world)],
+              [torch.zeros((m_cap, N), dtype=torch.bfloat16).share_memory_() for _ in range(world)])
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.spawn(_rank_main_peer, args=(world, port, case, shared, out), nprocs=world, join=True)
+    x = torch.cat([r[0] for r in ranks])
+    ids = torch.from_numpy(np.concatenate([r[1] for r in ranks]))
+    gw = torch.from_numpy(np.concatenate([r[2] for r in ranks]))
+    ref = ep_moe_layer(x, ids, gw, E, torch.from_numpy(q13), torch.from_numpy(sf13), torch.from_numpy(q2),
+                       torch.from_numpy(sf2), ops=OracleOps())
+    ref_bits = ref.view(torch.int16).numpy()
+    t0 = 0
+    for r in range(world):
+        t1 = t0 + ranks[r][0].shape[0]
+        assert np.array_equal(out[r], ref_bits[t0:t1]), f"rank {r}"
+        t0 = t1
