@@ -27,6 +27,8 @@ Workloads (shapes from the pages; data synthetic and seeded):
   moe_mlp     the contiguous MoE with gate/up -> SwiGLU -> MXFP8 fused, then down
   moe_bwd     the gate/up layer's backward: dgrad and the K-grouped weight gradient
   moe_layer   a whole expert layer: route, dispatch, gate/up.SwiGLU, down, combine
+  moe_layer_peer  the same layer through the expert-parallel peer-memory kernels
+              (placement plan, dispatch and combine through pointer tables), one rank
 
 With torchrun (N > 1) every rank runs its own independent batch (the work
 units are independent problems; no data-path collective), the step time is
@@ -101,7 +103,7 @@ def static_config(name: str, seed: int) -> dict:
                     "padded_rows": int(I.padded_offsets(counts)[-1]),
                     "gemms": ["dgrad dX[T,7168] = dY[T,4096] W13 (contiguous, W13 quantised along N)",
                               "wgrad dW13[32,4096,7168] = dY^T X per expert (K-grouped over tokens)"]})
-    elif name == "moe_layer":
+    elif name in ("moe_layer", "moe_layer_peer"):
         import numpy as np
         tokens = MOE_OVERRIDE["tokens"] or I.MOE_TOKENS
         experts = MOE_OVERRIDE["experts"] or I.MOE_EXPERTS
@@ -124,6 +126,9 @@ def static_config(name: str, seed: int) -> dict:
         cfg["step"] = ("quantise the gate/up and down weights (one batched launch), route the top-8 table, "
                        "dispatch (quantise each token once into its experts' rows), fused gate/up GEMM -> "
                        "SwiGLU -> MXFP8, down GEMM, gate-weighted combine to BF16 token outputs")
+    elif name == "moe_layer_peer":
+        cfg["step"] = ("the moe_layer step through the expert-parallel peer-memory kernels on one rank: "
+                       "route (pad 1), placement plan, dispatch and combine through device pointer tables")
     else:
         cfg["step"] = ("quantise activations + weights (one batched launch), then the GEMM(s) "
                        "with BF16 epilogue")
@@ -136,7 +141,7 @@ def parse_args():
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp", "moe_bwd",
-                                                            "moe_layer"])
+                                                            "moe_layer", "moe_layer_peer"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -531,6 +536,83 @@ class Workload:
                             "intermediate": i_dim, "real_rows": real, "padded_rows": padded,
                             "gate_weights": "softmax over N(0,1) logits"})
 
+    def _build_moe_layer_peer(self, seed, I):
+        """The moe_layer step through the expert-parallel peer-memory kernels
+        on one rank: routing plan with pad 1, placement plan, dispatch through
+        the device pointer table into the (here local) receive buffer, the two
+        grouped GEMMs, combine through the pointer table.  Measures those
+        kernels' HBM rates; with more ranks their stores and loads would go to
+        other GPUs over NVLink."""
+        import numpy as np
+        import torch
+        mx = self.mx
+        T = MOE_OVERRIDE["tokens"] or I.MOE_TOKENS
+        E = MOE_OVERRIDE["experts"] or I.MOE_EXPERTS
+        topk = I.MOE_TOPK
+        n13, hdim = I.MOE_GATE_NK
+        n2, i_dim = I.MOE_DOWN_NK
+        ids_np = I.topk_ids(T, topk, E, seed=seed)
+        ids = torch.from_numpy(ids_np.reshape(-1).copy()).to(self.dev)
+        gw = torch.from_numpy(I.gate_weights(T, topk, seed=seed)).to(self.dev)
+        x = I.normal_bf16((T, hdim), 1.0, seed + 7, self.dev)
+        w13 = I.normal_bf16((E, n13, hdim), 0.02, seed + 2_000_003, self.dev)
+        w2 = I.normal_bf16((E, n2, i_dim), 0.02, seed + 4_000_037, self.dev)
+        for t in (x, ids, gw, w13, w2):
+            self._add_input(t)
+        q13, sf13 = self._quant(w13, "W13")
+        q2, sf2 = self._quant(w2, "W2")
+        counts_h = np.bincount(ids_np.reshape(-1), minlength=E)
+        real = int(counts_h.sum())
+        padded = int(((counts_h + 127) // 128 * 128).sum())
+        active = int((counts_h > 0).sum())
+        n = T * topk
+        m_rows = mx.mx_moe_max_rows(n, E, 128)
+        i32 = dict(dtype=torch.int32, device=self.dev)
+        counts, offsets, row_send, dropped = (torch.empty(E, **i32), torch.empty(E + 1, **i32),
+                                              torch.empty(n, **i32), torch.empty(1, **i32))
+        dst_rank, dst_row = torch.empty(n, **i32), torch.empty(n, **i32)
+        counts_l, offsets_l = torch.empty(E, **i32), torch.empty(E + 1, **i32)
+        qa = torch.empty((m_rows, hdim), dtype=torch.uint8, device=self.dev)
+        sfa = torch.empty(mx.scale_bytes(m_rows, hdim), dtype=torch.uint8, device=self.dev)
+        qh = torch.empty((m_rows, i_dim), dtype=torch.uint8, device=self.dev)
+        sfh = torch.empty(mx.scale_bytes(m_rows, i_dim), dtype=torch.uint8, device=self.dev)
+        y = torch.empty((m_rows, n2), dtype=torch.bfloat16, device=self.dev)
+        out = torch.empty((T, n2), dtype=torch.bfloat16, device=self.dev)
+        q_ptrs = torch.tensor([qa.data_ptr()], dtype=torch.int64, device=self.dev)
+        sf_ptrs = torch.tensor([sfa.data_ptr()], dtype=torch.int64, device=self.dev)
+        y_ptrs = torch.tensor([y.data_ptr()], dtype=torch.int64, device=self.dev)
+        self.outputs.append(out)
+        self.launches.append(("route", "route (pad 1)", lambda ids: mx.mx_moe_route(ids, E, 1, counts, offsets,
+                                                                                     row_send, dropped),
+                              n * 8.0, 0.0, (ids,)))
+        self.launches.append(("plan", "placement plan", lambda ids, row_send, counts: mx.mx_moe_peer_plan(
+            ids, row_send, counts.view(1, E), 0, E, 128, dst_rank=dst_rank, dst_row=dst_row, counts_local=counts_l,
+            offsets_local=offsets_l, dev_status=self.status), n * 16.0, 0.0, (ids, row_send, counts)))
+        dbytes = T * hdim * 2.0 + padded * hdim * (1 + 1 / 32) + n * 8.0
+        self.launches.append(("dispatch", "dispatch (peer table)", lambda x, dst_rank, dst_row, counts_l, offsets_l:
+                              mx.mx_moe_dispatch_quant_peer(x, dst_rank, dst_row, topk, q_ptrs, sf_ptrs, m_rows, qa,
+                                                            sfa, counts_l, offsets_l, 128, dev_status=self.status),
+                              dbytes, 0.0, (x, dst_rank, dst_row, counts_l, offsets_l)))
+        fl1 = 2.0 * real * n13 * hdim
+        bytes1 = (padded * hdim + active * n13 * hdim + padded * i_dim) * (1 + 1 / 32)
+        self.launches.append(("gemm", "gate_up+swiglu", lambda qa, sfa, q13, sf13, offsets_l:
+                              mx.mx_grouped_gemm_contiguous_swiglu_quant(qa, sfa, q13, sf13, offsets_l, qh=qh,
+                                                                         sfh=sfh, dev_status=self.status),
+                              bytes1, fl1, (qa, sfa, q13, sf13, offsets_l)))
+        fl2 = 2.0 * real * n2 * i_dim
+        self.launches.append(("gemm", "down", lambda qh, sfh, q2, sf2, offsets_l: mx.mx_grouped_gemm_contiguous(
+            qh, sfh, q2, sf2, offsets_l, d=y, dev_status=self.status), self._gemm_bytes(padded, n2, i_dim, active),
+            fl2, (qh, sfh, q2, sf2, offsets_l)))
+        cbytes = real * n2 * 2.0 + T * n2 * 2.0 + n * 12.0
+        self.launches.append(("combine", "combine (peer table)", lambda dst_rank, dst_row, gw: mx.mx_moe_combine_peer(
+            y_ptrs, m_rows, n2, dst_rank, dst_row, gw, out=out, dev_status=self.status), cbytes, 0.0,
+            (dst_rank, dst_row, gw)))
+        self.flops += fl1 + fl2
+        self.config.update({"experts": E, "tokens": T, "topk": topk, "zipf_s": I.MOE_ZIPF_S, "hidden": hdim,
+                            "intermediate": i_dim, "real_rows": real, "padded_rows": padded, "ranks": 1,
+                            "exchange": "peer-memory kernels through device pointer tables (one rank: local)",
+                            "gate_weights": "softmax over N(0,1) logits"})
+
     def _build_moe_bwd(self, seed, I):
         """Backward of the MoE gate/up projection (the contiguous workload's
         first GEMM): input gradient dX = dY W13 per expert and weight gradient
@@ -728,7 +810,7 @@ def oracle_sample(name, seed, target_s=10.0, fmt="mxfp8"):
         jobs.append(job)
         desc = ("one expert layer on 64 rows over 2 experts: quantise rows and weights, gate/up GEMM, "
                 "SwiGLU, requantise, down GEMM")
-    elif name == "moe_layer":
+    elif name in ("moe_layer", "moe_layer_peer"):
         n13, k = I.MOE_GATE_NK
         n2, i_dim = I.MOE_DOWN_NK
         T, topk, E = 8, I.MOE_TOPK, 8
