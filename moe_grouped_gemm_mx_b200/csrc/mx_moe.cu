@@ -33,6 +33,7 @@ namespace mxk {
 constexpr int kRouteThreads = 1024;
 constexpr int kRowWarps = 8;  // warps per CTA of the row kernels (one row per warp)
 constexpr int kDevBadIndex = 0x8;
+constexpr int kCombineBatch = 8;  // routed rows of a token whose loads the combine has in flight at once
 
 __device__ __forceinline__ void moe_report(int32_t* status, int bits) { atomicOr(status, bits); }
 
@@ -352,7 +353,7 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_gather_kernel(const uint4*
 // ------------------------------------------------------------------ combine
 // out[t, :] = sum_j w[t, j] * y[row[t*topk + j], :], FP32 fused multiply-adds
 // in j order, rounded once to BF16 (RNE).  One warp per (token, chunk of 256
-// columns): 8 columns (one 16-byte vector) per lane, four routed rows' loads
+// columns): 8 columns (one 16-byte vector) per lane, eight routed rows' loads
 // in flight.  PEER: routed row j of a token is row `row` of rank `row_rank`'s
 // expert output, read through the pointer table (another GPU's memory over
 // NVLink, by plain loads).
@@ -380,32 +381,35 @@ __global__ void __launch_bounds__(kRowWarps * 32) moe_combine_kernel(const uint4
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    for (int j0 = 0; j0 < topk; j0 += 4) {
-      uint4 v[4];
-      float wj[4];
+    for (int j0 = 0; j0 < topk; j0 += kCombineBatch) {
+      // three branch-free phases, each with the batch's loads in flight
+      // together: the rows (and ranks), the ranks' addresses, the data
+      int32_t r[kCombineBatch], rk[kCombineBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kCombineBatch; ++u) {
         const int j = j0 + u;
-        int32_t r = j < topk ? rt[j] : -1;
-        const uint4* yb = y;
-        if (PEER && r >= 0) {
-          const int32_t rk = row_rank[t * topk + j];
-          if (rk < 0 || rk >= ranks) {
-            bad = true;
-            r = -1;
-          } else {
-            yb = y_peers[rk];
-          }
-        }
-        if (r >= y_rows) {
+        r[u] = j < topk ? rt[j] : -1;
+        rk[u] = PEER && j < topk ? row_rank[t * topk + j] : 0;
+      }
+      const uint4* yb[kCombineBatch];
+#pragma unroll
+      for (int u = 0; u < kCombineBatch; ++u) {
+        const bool rank_ok = !PEER || (rk[u] >= 0 && rk[u] < ranks);
+        if (r[u] >= 0 && (!rank_ok || r[u] >= y_rows)) {
           bad = true;
-          r = -1;
+          r[u] = -1;
         }
-        wj[u] = r >= 0 ? wt_t[j] : 0.0f;
-        v[u] = r >= 0 ? __ldcs(yb + static_cast<int64_t>(r) * n_vecs + c) : make_uint4(0, 0, 0, 0);
+        yb[u] = PEER ? y_peers[r[u] >= 0 ? rk[u] : 0] : y;  // entry 0 exists: ranks >= 1
+      }
+      uint4 v[kCombineBatch];
+      float wj[kCombineBatch];
+#pragma unroll
+      for (int u = 0; u < kCombineBatch; ++u) {
+        wj[u] = r[u] >= 0 ? wt_t[j0 + u] : 0.0f;
+        v[u] = r[u] >= 0 ? __ldcs(yb[u] + static_cast<int64_t>(r[u]) * n_vecs + c) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kCombineBatch; ++u) {
         if (j0 + u >= topk) break;
         const uint32_t x4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
