@@ -17,12 +17,12 @@ kernel of the step back to back in a CUDA graph over rotating copies of its
 operands that together exceed L2.
 
 Workloads (shapes from the pages; data synthetic and seeded):
-  page        dense 64x2112x7168, 64x24576x1536, 128x7168x2048 (default); the three
+  contiguous  MoE grouped, 32 experts, 8192 tokens top-8 Zipf: gate/up N=4096 K=7168,
+              then down N=7168 K=2048 (default: the largest configuration, tensor-bound)
+  page        dense 64x2112x7168, 64x24576x1536, 128x7168x2048; the three
               independent shapes' GEMMs run on parallel streams
   pr1         dense 128x256x512
   large       dense M=8192, (N,K) in {(7168,2048),(2112,7168),(4096,7168)}
-  contiguous  MoE grouped, 32 experts, 8192 tokens top-8 Zipf: gate/up N=4096 K=7168,
-              then down N=7168 K=2048
   masked      MoE masked grouped, 32 experts x 256 rows, masked_m ~ U{0..256}, N=4096 K=7168
   moe_mlp     the contiguous MoE with gate/up -> SwiGLU -> MXFP8 fused, then down
   moe_bwd     the gate/up layer's backward: dgrad and the K-grouped weight gradient
@@ -135,12 +135,22 @@ def static_config(name: str, seed: int) -> dict:
     return cfg
 
 
+def run_config(args, world: int) -> dict:
+    """The `config` object of the JSON line, identical in both arms: the
+    workload, the operand format and how the GPU arm times it (L2 flushed
+    before every timed step, CUDA-graph replays unless --eager)."""
+    return dict(static_config(args.workload, args.seed), format=args.fmt,
+                l2="flushed (512 MiB write) before every timed step",
+                parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                graph=not args.eager)
+
+
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=10)
-    p.add_argument("--workload", default="page", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp", "moe_bwd",
+    p.add_argument("--workload", default="contiguous", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp", "moe_bwd",
                                                             "moe_layer", "moe_layer_peer"])
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
@@ -923,7 +933,7 @@ def run_reference(args, world, rank):
             "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": dict(static_config(args.workload, args.seed), format=args.fmt),
+            "config": run_config(args, world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -1179,10 +1189,7 @@ def run_ours(args, world, rank, local):
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step_max, "step_stats": step_stats, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3", "data": "synthetic",
-        "config": dict(static_config(args.workload, args.seed), format=args.fmt,
-                       l2="flushed (512 MiB write) before every timed step",
-                       parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                       graph=graph is not None),
+        "config": run_config(args, world),
         "pct_of_fp8_peak": value / world / fp8_peak,
         "roofline": roof,
         "cpu_baseline": cpu,
