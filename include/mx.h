@@ -383,7 +383,8 @@ mx_status mx_moe_combine(const void *y_bf16, int64_t y_rows, int64_t n_cols, con
  * offsets_local int32 [experts/ranks + 1] (padded group starts, the
  * group_offsets of the grouped GEMMs; offsets_local[E/R] = rows in use).
  * experts % ranks == 0; 1 <= experts, ranks <= 1024; 1 <= pad <= 128;
- * n * ranks < 2^31.  A row_send inconsistent with count_table sets
+ * n * ranks + experts * (pad - 1) < 2^31 (the largest padded offset the plan
+ * can produce), else MX_ERR_UNSUPPORTED_SHAPE.  A row_send inconsistent with count_table sets
  * MX_DEV_BAD_INDEX and gives -1/-1. */
 mx_status mx_moe_peer_plan(const int32_t *ids, const int32_t *row_send, int64_t n, const int32_t *count_table,
                            int32_t ranks, int32_t rank, int32_t experts, int32_t pad, int32_t *dst_rank,

@@ -489,7 +489,10 @@ mx_status mx_moe_peer_plan(const int32_t* ids, const int32_t* row_send, int64_t 
   if (n < 0 || ranks < 1 || ranks > kMaxGroups || rank < 0 || rank >= ranks || experts < 1 ||
       experts > kMaxGroups || pad < 1 || pad > 128 || experts % ranks != 0)
     return MX_ERR_INVALID_ARGUMENT;
-  if (n * static_cast<int64_t>(ranks) > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  // every entry of every rank plus each expert's padding: the largest row
+  // index and padded offset the plan can produce must fit in int32
+  if (n * static_cast<int64_t>(ranks) + static_cast<int64_t>(experts) * (pad - 1) > kMaxDim)
+    return MX_ERR_UNSUPPORTED_SHAPE;
   if (!count_table || !counts_local || !offsets_local || (n > 0 && (!ids || !row_send || !dst_rank || !dst_row)))
     return MX_ERR_INVALID_ARGUMENT;
   if ((reinterpret_cast<uintptr_t>(ids) | reinterpret_cast<uintptr_t>(row_send) |

@@ -43,12 +43,17 @@ import torch.distributed as dist
 
 
 class LibraryOps:
-    """The steps of the layer as calls into the CUDA library."""
+    """The steps of the layer as calls into the CUDA library.
 
-    def __init__(self, mx=None):
+    Every call ORs its data-dependent errors (bad offsets, rows beyond a
+    buffer, indices outside a table) into the int32 device word ``status``;
+    ``check()`` reads it back and raises if any step reported one."""
+
+    def __init__(self, mx=None, status: torch.Tensor | None = None):
         if mx is None:
             import moe_grouped_gemm_mx_b200 as mx
         self.mx = mx
+        self.status = status
 
     def max_rows(self, n, experts, pad):
         return self.mx.mx_moe_max_rows(n, experts, pad)
@@ -58,32 +63,60 @@ class LibraryOps:
         return counts, offsets, row
 
     def dispatch(self, x, row, topk, counts, offsets, pad, m_rows, row_major):
-        return self.mx.mx_moe_dispatch_quant(x, row, topk, counts, offsets, pad, m_rows, sf_row_major=row_major)
+        return self.mx.mx_moe_dispatch_quant(x, row, topk, counts, offsets, pad, m_rows, sf_row_major=row_major,
+                                             dev_status=self.status)
 
     def scatter(self, q_src, sf_src, dst_row, counts, offsets, pad, m_rows):
-        return self.mx.mx_moe_scatter_rows(q_src, sf_src, dst_row, counts, offsets, pad, m_rows)
+        return self.mx.mx_moe_scatter_rows(q_src, sf_src, dst_row, counts, offsets, pad, m_rows,
+                                           dev_status=self.status)
 
     def gate_up_swiglu(self, qa, sfa, q13, sf13, offsets):
-        return self.mx.mx_grouped_gemm_contiguous_swiglu_quant(qa, sfa, q13, sf13, offsets)
+        return self.mx.mx_grouped_gemm_contiguous_swiglu_quant(qa, sfa, q13, sf13, offsets, dev_status=self.status)
 
     def down(self, qh, sfh, q2, sf2, offsets, d=None):
-        return self.mx.mx_grouped_gemm_contiguous(qh, sfh, q2, sf2, offsets, d=d)
+        return self.mx.mx_grouped_gemm_contiguous(qh, sfh, q2, sf2, offsets, d=d, dev_status=self.status)
 
     def gather(self, src, idx):
-        return self.mx.mx_gather_rows(src, idx)
+        return self.mx.mx_gather_rows(src, idx, dev_status=self.status)
 
     def combine(self, y, row, w):
-        return self.mx.mx_moe_combine(y, row, w)
+        return self.mx.mx_moe_combine(y, row, w, dev_status=self.status)
 
     def peer_plan(self, ids, row_send, count_table, rank, experts, pad):
-        return self.mx.mx_moe_peer_plan(ids, row_send, count_table, rank, experts, pad)
+        return self.mx.mx_moe_peer_plan(ids, row_send, count_table, rank, experts, pad, dev_status=self.status)
 
     def dispatch_peer(self, x, dst_rank, dst_row, topk, bufs, counts_l, offsets_l, pad):
         self.mx.mx_moe_dispatch_quant_peer(x, dst_rank, dst_row, topk, bufs.q_ptrs, bufs.sf_ptrs, bufs.m_cap,
-                                           bufs.q, bufs.sf, counts_l, offsets_l, pad)
+                                           bufs.q, bufs.sf, counts_l, offsets_l, pad, dev_status=self.status)
 
     def combine_peer(self, bufs, n, dst_rank, dst_row, w):
-        return self.mx.mx_moe_combine_peer(bufs.y_ptrs, bufs.m_cap, n, dst_rank, dst_row, w)
+        return self.mx.mx_moe_combine_peer(bufs.y_ptrs, bufs.m_cap, n, dst_rank, dst_row, w, dev_status=self.status)
+
+    def check(self, what: str = "expert layer"):
+        """Raise if any call since the last check reported a device error
+        (one device-to-host read), then clear the word."""
+        if self.status is None:
+            return
+        v = int(self.status.item())
+        if v:
+            self.status.zero_()
+            raise RuntimeError(f"{what}: device status {v:#x} (bad offsets 0x1, bad mask 0x2, timeout 0x4, "
+                               f"index or row outside its buffer 0x8)")
+
+
+def _default_ops(ops, device):
+    """The caller's ops, or library ops with a fresh status word that the
+    layer checks before it returns."""
+    if ops is not None:
+        return ops, False
+    return LibraryOps(status=torch.zeros(1, dtype=torch.int32, device=device)), True
+
+
+def _check_pad(pad: int):
+    # the contiguous grouped GEMM takes groups that start on 128-row
+    # boundaries, and the routing kernels pad groups to at most 128 rows
+    if pad != 128:
+        raise ValueError(f"pad must be 128: the grouped GEMM's groups start on 128-row boundaries (got {pad})")
 
 
 def _all_to_all_rows(src: torch.Tensor, send_rows, recv_rows, group):
@@ -101,8 +134,14 @@ def ep_moe_layer(x: torch.Tensor, ids: torch.Tensor, gate_w: torch.Tensor, exper
            ids; gate_w float32 [T, topk].
     q13/sf13, q2/sf2  this rank's E/W experts, quantised: [E/W, 2I, H] and
            [E/W, N, I] E4M3 with per-expert tiled scales.
+    pad    rows each local expert's group is padded to: 128 (the grouped
+           GEMM's groups start on 128-row boundaries; anything else raises).
+    ops    the steps (default: the CUDA library, with a device status word
+           that is checked before returning -- a RuntimeError names any
+           data-dependent error a kernel reported).
     Returns BF16 [T, N]: sum_j gate_w[t, j] * expert_{ids[t,j]}(x[t])."""
-    ops = LibraryOps() if ops is None else ops
+    _check_pad(pad)
+    ops, own_status = _default_ops(ops, x.device)
     world = dist.get_world_size(group) if dist.is_initialized() else 1
     if experts % world:
         raise ValueError("the experts must divide evenly over the ranks")
@@ -152,7 +191,10 @@ def ep_moe_layer(x: torch.Tensor, ids: torch.Tensor, gate_w: torch.Tensor, exper
         y_home = _all_to_all_rows(y_back, recv_rows, send_rows, group)
     else:
         y_home = y_back
-    return ops.combine(y_home, row_send, gate_w)
+    out = ops.combine(y_home, row_send, gate_w)
+    if own_status:
+        ops.check("ep_moe_layer")
+    return out
 
 
 # ---------------------------------------------------------------- exchange over peer memory
@@ -260,8 +302,13 @@ def ep_moe_layer_peer(x: torch.Tensor, ids: torch.Tensor, gate_w: torch.Tensor, 
                       q13, sf13, q2, sf2, bufs: PeerBuffers, group=None, ops=None, pad: int = 128) -> torch.Tensor:
     """One expert-parallel MoE layer on this rank with the exchange over peer
     memory (arguments as ep_moe_layer; ``bufs`` from PeerBuffers.symmetric).
-    Returns BF16 [T, N]."""
-    ops = LibraryOps() if ops is None else ops
+    With the default ops the layer checks, before it returns, that no kernel
+    reported an error -- in particular that every owner's plan fitted its
+    receive buffer (rows beyond bufs.m_cap are skipped by the dispatch and
+    reported, and would leave stale expert outputs behind): a RuntimeError
+    otherwise.  Returns BF16 [T, N]."""
+    _check_pad(pad)
+    ops, own_status = _default_ops(ops, x.device)
     world = dist.get_world_size(group) if dist.is_initialized() else 1
     if experts % world or bufs.ranks != world:
         raise ValueError("the experts must divide evenly over the ranks, one buffer set per rank")
@@ -281,6 +328,8 @@ def ep_moe_layer_peer(x: torch.Tensor, ids: torch.Tensor, gate_w: torch.Tensor, 
     out = peer_combine(bufs, plan, gate_w, bufs.y.shape[1], ops)
     if world > 1:
         _stream_barrier(group, x.device)  # the outputs are read before any rank overwrites its buffers
+    if own_status:
+        ops.check("ep_moe_layer_peer")
     return out
 
 
@@ -288,10 +337,15 @@ def ep_moe_layer_peer_emulated(xs, ids_list, gate_ws, experts, weights, bufs_lis
     """The peer-memory layer for R ranks emulated on one GPU: each phase runs
     for every rank before the next phase starts (what the barriers of
     ep_moe_layer_peer guarantee).  weights[r] = (q13, sf13, q2, sf2) of rank
-    r's experts.  Returns every rank's output."""
-    ops = LibraryOps() if ops is None else ops
+    r's experts.  Returns every rank's output; with the default ops, raises
+    if any kernel reported an error."""
+    _check_pad(pad)
+    ops, own_status = _default_ops(ops, xs[0].device)
     table = torch.stack([route_counts(ids, experts, ops) for ids in ids_list])
     plans = [peer_dispatch(xs[r], ids_list[r], experts, table, bufs_list[r], ops, pad) for r in range(len(xs))]
     for r in range(len(xs)):
         peer_experts(bufs_list[r], plans[r], *weights[r], ops)
-    return [peer_combine(bufs_list[r], plans[r], gate_ws[r], bufs_list[r].y.shape[1], ops) for r in range(len(xs))]
+    outs = [peer_combine(bufs_list[r], plans[r], gate_ws[r], bufs_list[r].y.shape[1], ops) for r in range(len(xs))]
+    if own_status:
+        ops.check("ep_moe_layer_peer_emulated")
+    return outs

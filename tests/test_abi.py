@@ -240,6 +240,11 @@ def test_moe_peer_argument_checks(lib):
     assert plan(A, B, 16, C, 2, 0, 8, 128, None, E, F, G, None, None) == MX_ERR_INVALID_ARGUMENT
     assert plan(A + 2, B, 16, C, 2, 0, 8, 128, D, E, F, G, None, None) == MX_ERR_MISALIGNED
     assert plan(A, B, 1 << 30, C, 4, 0, 8, 128, D, E, F, G, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    # entries fit in int32 but the padded offsets could not: every expert
+    # adds up to pad - 1 rows
+    n_edge = ((1 << 31) - 1 - 1024 * 127) // 2
+    assert plan(A, B, n_edge + 1, C, 2, 0, 1024, 128, D, E, F, G, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    assert plan(A, B, n_edge, C, 2, 0, 1024, 128, None, E, F, G, None, None) == MX_ERR_INVALID_ARGUMENT
     disp = lib.mx_moe_dispatch_quant_peer
     # the dispatch's rules, plus ranks and 8-byte aligned pointer tables
     assert disp(A, 4, 128, B, C, 2, D, E, 0, 128, F, G, A, B, 4, 128, None, None) == MX_ERR_INVALID_ARGUMENT

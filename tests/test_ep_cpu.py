@@ -161,3 +161,22 @@ def test_ep_peer_ranks_match_one_process(world, case):
         t1 = t0 + ranks[r][0].shape[0]
         assert np.array_equal(out[r], ref_bits[t0:t1]), f"rank {r}"
         t0 = t1
+
+
+@pytest.mark.parametrize("pad", [1, 64, 256])
+def test_ep_layers_reject_pad_off_the_gemm_grid(pad):
+    """Both layer forms refuse a pad other than 128 before any work: the
+    grouped GEMM takes groups that start on 128-row boundaries, and a plan
+    padded otherwise would make it skip every tile."""
+    from ep_ref_ops import OracleOps
+    from moe_grouped_gemm_mx_b200.ep import PeerBuffers, ep_moe_layer, ep_moe_layer_peer
+    ranks, (q13, sf13, q2, sf2), E = _problem("uniform", 1)
+    x, ids, gw = ranks[0]
+    w = [torch.from_numpy(a) for a in (q13, sf13, q2, sf2)]
+    with pytest.raises(ValueError, match="pad"):
+        ep_moe_layer(x, torch.from_numpy(ids), torch.from_numpy(gw), E, *w, ops=OracleOps(), pad=pad)
+    table = torch.zeros(1, dtype=torch.int64)
+    bufs = PeerBuffers(torch.zeros((128, H), dtype=torch.uint8), torch.zeros((128, H // 32), dtype=torch.uint8),
+                       torch.zeros((128, N), dtype=torch.bfloat16), table, table, table, 0)
+    with pytest.raises(ValueError, match="pad"):
+        ep_moe_layer_peer(x, torch.from_numpy(ids), torch.from_numpy(gw), E, *w, bufs, ops=OracleOps(), pad=pad)

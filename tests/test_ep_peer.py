@@ -170,3 +170,33 @@ def test_peer_bad_ranks_report(mx):
                            torch.tensor([0, 0], dtype=torch.int32, device=DEV), w, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) & mx.MX_DEV_BAD_INDEX
+
+
+def test_peer_layer_undersized_buffers_raise(mx):
+    """Receive buffers too small for the plan: the dispatch skips the rows
+    past the buffer, the grouped GEMMs refuse the offsets and the combine
+    skips the rows it cannot load -- each reports it, and the layer raises
+    instead of returning the stale contents of the output buffers."""
+    from moe_grouped_gemm_mx_b200.ep import PeerBuffers, ep_moe_layer_peer_emulated
+    ranks, experts, topk, H, I, N, pad = 2, 4, 2, 128, 128, 128, 128
+    tokens = [200, 150]
+    ids_list = rank_inputs(ranks, tokens, topk, experts, seed=90)
+    xs = [mx_inputs.normal_bf16((tokens[r], H), 1.0, 91 + r).to(DEV) for r in range(ranks)]
+    gws = [torch.from_numpy(mx_inputs.gate_weights(tokens[r], topk, seed=93 + r)).to(DEV) for r in range(ranks)]
+    q13, sf13 = mx.mx_quantize_bf16_to_e4m3(mx_inputs.normal_bf16((experts, 2 * I, H), 0.05, 95).to(DEV))
+    q2, sf2 = mx.mx_quantize_bf16_to_e4m3(mx_inputs.normal_bf16((experts, N, I), 0.05, 96).to(DEV))
+    el = experts // ranks
+    per13, per2 = mx.scale_bytes(2 * I, H), mx.scale_bytes(N, I)
+    weights = [(q13[r * el:(r + 1) * el], sf13[r * el * per13:(r + 1) * el * per13],
+                q2[r * el:(r + 1) * el], sf2[r * el * per2:(r + 1) * el * per2]) for r in range(ranks)]
+    need = mx.mx_moe_max_rows(sum(tokens) * topk, el, pad)
+    assert need > 256
+    bufs = PeerBuffers.emulated(ranks, 256, H, N, DEV)      # far below the rows the plans need
+    with pytest.raises(RuntimeError, match="device status"):
+        ep_moe_layer_peer_emulated(xs, [torch.from_numpy(i).to(DEV) for i in ids_list], gws, experts, weights,
+                                   bufs, pad=pad)
+    # the same layer with buffers of the right size runs clean
+    bufs = PeerBuffers.emulated(ranks, need, H, N, DEV)
+    outs = ep_moe_layer_peer_emulated(xs, [torch.from_numpy(i).to(DEV) for i in ids_list], gws, experts, weights,
+                                      bufs, pad=pad)
+    assert all(bool(torch.isfinite(o.float()).all()) for o in outs)
