@@ -127,3 +127,17 @@ def check_swiglu_quant(oracle, qh: np.ndarray, sf_rm: np.ndarray, g_ref, u_ref, 
     same = (q_ref == qh) & np.repeat(s_ref == sf_rm, 32, axis=1)
     assert same.mean() > 0.97, f"{what}: only {same.mean():.4f} of H codes equal the oracle's"
     return h_ref
+
+
+def sampled_rows(m_end, n_random, seed=0, tile=128, extra=()):
+    """Row indices for a full-size parity check: ``n_random`` distinct random
+    rows of [0, m_end), the first and last row of every ``tile``-row block
+    (where a tile of the GEMM, and each CTA's half of a pair tile, starts and
+    ends), and ``extra``; sorted int64."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(m_end, min(n_random, m_end), replace=False).tolist())
+    for t0 in range(0, m_end, tile):
+        rows.update([t0, min(t0 + tile, m_end) - 1])
+    rows.update(int(r) for r in extra if 0 <= int(r) < m_end)
+    return np.array(sorted(rows), dtype=np.int64)

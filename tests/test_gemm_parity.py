@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import mx_inputs
-from mxtest_util import assert_gemm_close, is_sentinel, oracle_quantize, sentinel_fill, to_np_f64
+from mxtest_util import sampled_rows, assert_gemm_close, is_sentinel, oracle_quantize, sentinel_fill, to_np_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -108,8 +108,9 @@ def test_large_dense_sampled_rows(mx, oracle, nk):
     n, k = nk
     m = mx_inputs.LARGE_M
     a, b = mx_inputs.dense_problem(m, n, k, seed=0, kind="loguniform")
-    g = np.random.default_rng(0)
-    rows = np.unique(np.concatenate([g.choice(m, 200, replace=False), [0, 127, 128, m - 1]]))
+    # 256 random rows plus the first and last row of every 128-row M tile
+    rows = sampled_rows(m, 256, seed=0)
+    assert len(rows) >= 256 + 2 * (m // 128) - 8
     check_dense(mx, oracle, a, b, rows=rows, what=f"large {m}x{n}x{k}")
 
 

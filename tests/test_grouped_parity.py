@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import mx_inputs
-from mxtest_util import assert_gemm_close, is_sentinel, oracle_quantize, sentinel_fill, to_np_f64
+from mxtest_util import sampled_rows, assert_gemm_close, is_sentinel, oracle_quantize, sentinel_fill, to_np_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -94,20 +94,22 @@ def test_contiguous_bad_offsets_reported(mx, bad):
     assert bool(is_sentinel(d).all()), "nothing may be written when offsets are invalid"
 
 
-def test_contiguous_moe_gate_up_sampled(mx, oracle):
-    """Full-size MoE gate/up GEMM (32 experts, 8192 tokens x top-8, Zipf
-    routing, N=4096, K=7168) -- sampled rows against the oracle: 64 random
-    rows plus the first and last real row of every non-empty expert."""
-    n, k = mx_inputs.MOE_GATE_NK
-    prob = mx_inputs.contiguous_problem(n=n, k=k, seed=0)
+@pytest.mark.parametrize("which", ["gate_up", "down"])
+def test_contiguous_moe_sampled(mx, oracle, which):
+    """Full-size MoE grouped GEMMs (32 experts, 8192 tokens x top-8, Zipf
+    routing): gate/up (N=4096, K=7168) and down (N=7168, K=2048) -- 256
+    random rows, the first and last row of every 128-row tile (each CTA half
+    of a pair tile), and the first and last real row of every non-empty
+    expert, against the oracle."""
+    n, k = mx_inputs.MOE_GATE_NK if which == "gate_up" else mx_inputs.MOE_DOWN_NK
+    prob = mx_inputs.contiguous_problem(n=n, k=k, seed=0 if which == "gate_up" else 100)
     off = prob.offsets.numpy()
-    rng = np.random.default_rng(0)
-    rows = set(rng.choice(int(off[-1]), 64, replace=False).tolist())
+    ends = []
     for e in range(len(prob.counts)):
         if prob.counts[e] > 0:
-            rows.update([int(off[e]), int(off[e]) + int(prob.counts[e]) - 1])
-    rows = np.array(sorted(rows), dtype=np.int64)
-    check_contiguous(mx, oracle, prob, rows=rows, what="MoE gate/up")
+            ends += [int(off[e]), int(off[e]) + int(prob.counts[e]) - 1]
+    rows = sampled_rows(int(off[-1]), 256, seed=0, extra=ends)
+    check_contiguous(mx, oracle, prob, rows=rows, what=f"MoE {which}")
 
 
 # ---------------------------------------------------------------- masked
@@ -126,10 +128,11 @@ def gpu_masked(mx, prob, masked_m=None):
     return d, int(status.item())
 
 
-def check_masked(mx, oracle, prob, what="", sample_per_expert=None):
+def check_masked(mx, oracle, prob, what="", sample_per_expert=None, whole_experts=()):
     """All rows of every expert (or, with sample_per_expert, the first and
-    last valid row plus that many random valid rows) against the oracle; all
-    rows at or beyond masked_m must still hold the sentinel."""
+    last valid row plus that many random valid rows, and every valid row of
+    the experts in whole_experts) against the oracle; all rows at or beyond
+    masked_m must still hold the sentinel."""
     d, st = gpu_masked(mx, prob)
     assert st == 0, f"device status {st:#x}"
     e, max_m, k = prob.a.shape
@@ -142,7 +145,7 @@ def check_masked(mx, oracle, prob, what="", sample_per_expert=None):
     for g in range(e):
         if mm[g] == 0:
             continue
-        if sample_per_expert is None:
+        if sample_per_expert is None or g in whole_experts:
             rows.extend(g * max_m + r for r in range(mm[g]))
         else:
             pick = {0, mm[g] - 1} | set(rng.integers(0, mm[g], sample_per_expert).tolist())
@@ -183,8 +186,16 @@ def test_masked_bad_mask_reported_and_clamped(mx, oracle):
 
 def test_masked_decode_config(mx, oracle):
     """Full masked decode config: 32 experts x max 256 rows, masked_m ~
-    U{0..256}, N=4096, K=7168, NaN padding rows; first, last and 6 random
-    valid rows of every expert against the oracle."""
+    U{0..256}, N=4096, K=7168, NaN padding rows; every valid row of the four
+    experts with the most rows (a tile boundary inside each) and of the
+    expert with the fewest non-zero rows, the first, last and 8 random valid
+    rows of every other expert, against the oracle."""
     n, k = mx_inputs.MASKED_NK
     prob = mx_inputs.masked_problem(n=n, k=k, seed=0)
-    check_masked(mx, oracle, prob, "masked decode", sample_per_expert=6)
+    mm = prob.masked_m.numpy()
+    order = np.argsort(-mm, kind="stable")
+    whole = set(order[:4].tolist())
+    nz = [g for g in range(len(mm)) if mm[g] > 0]
+    whole.add(min(nz, key=lambda g: mm[g]))
+    assert sum(int(mm[g]) for g in whole) >= 4 * 128
+    check_masked(mx, oracle, prob, "masked decode", sample_per_expert=8, whole_experts=whole)

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import mx_inputs
-from mxtest_util import assert_gemm_close, is_sentinel, sentinel_fill, to_np_f64
+from mxtest_util import sampled_rows, assert_gemm_close, is_sentinel, sentinel_fill, to_np_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -157,3 +157,38 @@ def test_dgrad_on_weights_quantised_along_n(mx, oracle):
     d_ref, absd = oracle.grouped_contiguous(r_dy, rs_dy, r_wt.reshape(e, k, n), rs_wt, offsets.numpy())
     m_end = int(offsets[-1])
     assert_gemm_close(to_np_f64(dx[:m_end]), d_ref, absd, "dgrad")
+
+
+def test_dgrad_moe_shape_sampled(mx, oracle):
+    """dX = dY W13 at the MoE gate/up shape (32 experts, 8192 tokens x top-8,
+    Zipf routing, dY [T, 4096], W13 [32, 4096, 7168] quantised along N into
+    [32, 7168, 4096]): 256 random rows, the first and last row of every
+    128-row tile and of every non-empty expert, against the oracle."""
+    counts = mx_inputs.zipf_routing_counts(seed=0)
+    offsets = mx_inputs.padded_offsets(counts)
+    n_out, k_in = mx_inputs.MOE_GATE_NK
+    e = len(counts)
+    t = int(offsets[-1])
+    dev = torch.device("cuda")
+    dy = mx_inputs.normal_bf16((t, n_out), 1.0, 62)
+    pad = torch.repeat_interleave(torch.arange(e), (offsets[1:] - offsets[:-1]).long())
+    local = torch.arange(t) - offsets[:-1].long()[pad]
+    dy[local >= counts[pad]] = 0                    # padding rows of the grouped layout are zero
+    w = mx_inputs.normal_bf16((e, n_out, k_in), 0.02, 63)
+    q_dy, sf_dy = mx.mx_quantize_bf16_to_e4m3(dy.to(dev))
+    q_wt, sf_wt = mx.mx_quantize_bf16_to_e4m3_transposed(w.to(dev))     # [E, K, N]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    dx = mx.mx_grouped_gemm_contiguous(q_dy, sf_dy, q_wt, sf_wt, offsets.to(dev), dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ends = []
+    for g in range(e):
+        if counts[g] > 0:
+            ends += [int(offsets[g]), int(offsets[g]) + int(counts[g]) - 1]
+    rows = sampled_rows(t, 256, seed=3, extra=ends)
+    r_dy, rs_dy = oracle.quantize(dy.view(torch.int16).numpy().view(np.uint16))
+    r_wt, rs_wt = oracle.quantize_transposed(w)
+    d_ref, absd = oracle.grouped_contiguous(r_dy, rs_dy, r_wt.reshape(e, k_in, n_out), rs_wt,
+                                            offsets.numpy().astype(np.int32), rows=rows)
+    dg = dx[torch.as_tensor(rows, device=dev)]
+    assert_gemm_close(to_np_f64(dg), d_ref, absd, "MoE dgrad (sampled)")
