@@ -418,6 +418,22 @@ mx_status mx_moe_combine_peer(const void *const *y_peers, int32_t ranks, int64_t
                               const int32_t *src_rank, const int32_t *src_row, const float *w, int64_t tokens,
                               int32_t topk, void *out_bf16, int32_t *dev_status, mx_stream_t stream);
 
+/* Failure detection (no counterpart on the pages; a property of this
+ * implementation).  Every wait inside the GEMM kernels (a pipeline stage
+ * landing, an accumulator being drained, ...) is bounded: a wait that runs
+ * longer than the limit gives up, the kernel sets MX_DEV_TIMEOUT in the
+ * status word, stops issuing work, waits for the tensor-core work and copies
+ * it already issued, frees its tensor memory and returns -- it never traps or
+ * hangs, and the context stays usable; the output of that call is invalid.
+ * The limit defaults to 2 s (far above any legitimate wait).  This sets it,
+ * in nanoseconds, for the GEMM launches that follow, from any thread
+ * (ns == 0 restores the default); a limit below a kernel's legitimate waits
+ * makes its calls fail with MX_DEV_TIMEOUT, which is how the failure path is
+ * tested.  Never fails. */
+mx_status mx_set_wait_limit_ns(uint64_t ns);
+/* The current limit in nanoseconds. */
+uint64_t mx_wait_limit_ns(void);
+
 /* Copies the library-internal device status word (used when a call got
  * dev_status == NULL) to *host_out and, if clear != 0, resets it.
  * Synchronises the device. */

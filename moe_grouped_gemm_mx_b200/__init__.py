@@ -53,6 +53,7 @@ C_SYMBOLS = [
     "mx_quantize_bf16_to_e4m3_block128x128", "mx_gemm_tilewise", "mx_grouped_gemm_contiguous_tilewise",
     "mx_moe_max_rows", "mx_moe_route", "mx_moe_dispatch_quant", "mx_moe_scatter_rows", "mx_gather_rows",
     "mx_moe_combine", "mx_moe_peer_plan", "mx_moe_dispatch_quant_peer", "mx_moe_combine_peer",
+    "mx_set_wait_limit_ns", "mx_wait_limit_ns",
 ]
 
 
@@ -128,6 +129,10 @@ def _load():
     L.mx_moe_combine_peer.restype = ctypes.c_int
     L.mx_read_internal_status.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
     L.mx_read_internal_status.restype = ctypes.c_int
+    L.mx_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.mx_set_wait_limit_ns.restype = ctypes.c_int
+    L.mx_wait_limit_ns.argtypes = []
+    L.mx_wait_limit_ns.restype = ctypes.c_uint64
     return L
 
 
@@ -704,3 +709,16 @@ def read_internal_status(clear: bool = True) -> int:
     out = ctypes.c_int32(0)
     _raise(_lib.mx_read_internal_status(ctypes.byref(out), int(clear)), "mx_read_internal_status")
     return int(out.value)
+
+
+def mx_set_wait_limit_ns(ns: int) -> None:
+    """Bound, in nanoseconds, of every wait inside the GEMM kernels launched
+    from now on (0 restores the default of 2 s).  A wait that runs longer
+    makes the kernel give up cleanly and set MX_DEV_TIMEOUT; a limit below a
+    kernel's legitimate waits is how that failure path is exercised."""
+    _raise(_lib.mx_set_wait_limit_ns(int(ns)), "mx_set_wait_limit_ns")
+
+
+def mx_wait_limit_ns() -> int:
+    """The current wait bound in nanoseconds."""
+    return int(_lib.mx_wait_limit_ns())

@@ -3,6 +3,7 @@
 // memory is allocated per call; the only device memory the library owns is the
 // 4-byte internal status word below.
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/mx.h"
@@ -39,7 +40,12 @@ int32_t* internal_status_ptr() {
 
 mx_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
 
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+
 }  // namespace
+
+uint64_t mxk::wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 extern "C" {
 
@@ -564,6 +570,13 @@ mx_status mx_moe_combine_peer(const void* const* y_peers, int32_t ranks, int64_t
   return from_cuda(mxk::launch_moe_combine(nullptr, y_peers, src_rank, ranks, y_rows, n_cols, src_row, w, tokens,
                                            topk, out_bf16, status, static_cast<cudaStream_t>(stream)));
 }
+
+mx_status mx_set_wait_limit_ns(uint64_t ns) {
+  g_wait_ns.store(ns == 0 ? kDefaultWaitNs : ns, std::memory_order_relaxed);
+  return MX_OK;
+}
+
+uint64_t mx_wait_limit_ns(void) { return g_wait_ns.load(std::memory_order_relaxed); }
 
 mx_status mx_read_internal_status(int32_t* host_out, int clear) {
   if (!host_out) return MX_ERR_INVALID_ARGUMENT;

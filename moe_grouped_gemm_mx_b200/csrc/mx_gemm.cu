@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int nsfb = args.n_sf_tiles - sfb_tile0;
         nsfb = nsfb > L::SFB_TILES ? L::SFB_TILES : nsfb;
         for (int kt = kt_begin; kt < kt_end; ++kt) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
           // only the A rows that exist are loaded when M is small; the MMA's
           // remaining A rows read stale shared memory and only feed
           // accumulator rows that are never stored
@@ -257,12 +257,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
+      if (!ok) {  // loads already in flight land during the teardown's linger
         report(args.status, 0x4);
         *abort_flag = 1;
-        // give copies already in flight time to land before the CTA can exit
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 1000000ull) { }
       }
     }
   } else if (warp == 1) {
@@ -275,12 +272,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
-        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_t = tmem_base + acc * BN;
         for (int kt = kt_begin; kt < kt_end; ++kt) {
           // the copier's commit implies the stage's operands have landed too
-          if (!mbar_wait(sfready_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(sfready_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
           const uint32_t sfb_t = sfa_t + 4;
@@ -303,10 +300,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) {
         report(args.status, 0x4);
         *abort_flag = 1;
-        // every MMA this thread issued must finish before TMEM is freed
-        tc_commit(drain_bar);
-        mbar_wait(drain_bar, 0, nullptr, 100000000ull);
       }
+      // every MMA this thread issued must finish before TMEM is freed (also
+      // when another role gave up while they ran)
+      tc_commit(drain_bar);
+      mbar_wait(drain_bar, 0, nullptr, 100000000ull);
     }
   } else if (warp == 6) {
     if (lane == 0) {
@@ -318,7 +316,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
         for (int kt = kt_begin; kt < kt_end; ++kt) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
           tc_cp_32x128b_warpx4(sfa_t, desc_sf_32x16(sbase + L::OFF_SFA + stage * L::SFA_BYTES));
@@ -349,7 +347,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // every lane polls; the vote over all four epilogue warps re-converges
       // them before the warp-collective (.sync.aligned) TMEM loads and makes
       // the give-up decision uniform (the warps share named barriers below)
-      const bool got = mbar_wait(accf_bar(acc), acc_phase, abort_flag, kWaitLimitNs);
+      const bool got = mbar_wait(accf_bar(acc), acc_phase, abort_flag, args.wait_ns);
       if (!named_barrier_and(2, 128, got)) {
         if (threadIdx.x == 64) report(args.status, 0x4);
         *abort_flag = 1;
@@ -480,6 +478,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
+  if (threadIdx.x == 0 && *abort_flag) linger_after_abort();
 }
 
 // ======================================================================= host
@@ -547,6 +546,7 @@ static cudaError_t launch_gemm_cfg(const GemmProblem& p, int num_sms, cudaStream
   a.group_offsets = p.group_offsets;
   a.masked_m = p.masked_m;
   a.status = p.status;
+  a.wait_ns = wait_limit_ns();
   a.k_tiles = static_cast<int>(p.k / BK);
   a.sfa_group_bytes = ((p.m + 127) / 128) * 128 * (p.k / 32);
   a.sfb_group_bytes = ((p.n + 127) / 128) * 128 * (p.k / 32);

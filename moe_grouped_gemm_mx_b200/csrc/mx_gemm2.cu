@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int kc0 = tile_kc0(tl);
         const int k_stages = (tile_chunks(tl) + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
           if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), bytes_pair);
           const int kc = kc0 + ks * kPairKC;
@@ -310,11 +310,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
+      if (!ok) {  // loads already in flight land during the teardown's linger
         report(args.status, 0x4);
         *abort_flag = 1;
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 1000000ull) { }
       }
     }
   } else if (warp == 1) {
@@ -326,13 +324,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs) {
-        if (!mbar_wait(acce_bar, acc_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        if (!mbar_wait(acce_bar, acc_phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const int chunks = tile_chunks(decode_pair_tile(args, tab0, tab1, t));
         const int k_stages = (chunks + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
           // the copier's commit implies both CTAs' operands of the stage have landed
-          if (!mbar_wait(sfready_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(sfready_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < kPairKC; ++c) {
@@ -363,9 +361,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) {
         report(args.status, 0x4);
         *abort_flag = 1;
-        tc_commit_pair_multicast(drain_bar, 0x1);
-        mbar_wait(drain_bar, 0, nullptr, 100000000ull);
       }
+      // every pair MMA issued must finish before either CTA frees its TMEM
+      // (also when another role gave up while they ran)
+      tc_commit_pair_multicast(drain_bar, 0x1);
+      mbar_wait(drain_bar, 0, nullptr, 100000000ull);
     }
   } else if (warp == 6) {
     if (lane == 0 && rank == 0) {
@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = pair; t < total && ok; t += npairs) {
         const int k_stages = (tile_chunks(decode_pair_tile(args, tab0, tab1, t)) + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < kPairKC; ++c) {
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     uint32_t stg_count = 0;
     for (int t = pair; t < total; t += npairs) {
-      const bool got = mbar_wait(accf_bar, acc_phase, abort_flag, kWaitLimitNs);
+      const bool got = mbar_wait(accf_bar, acc_phase, abort_flag, args.wait_ns);
       if (!named_barrier_and(2, 128, got)) {
         if (threadIdx.x == 64) report(args.status, 0x4);
         *abort_flag = 1;
@@ -530,8 +530,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   // ---------------------------------------------------------------- teardown
   // neither CTA may leave while its peer can still signal its barriers,
-  // read its shared memory or write its TMEM
+  // read its shared memory or write its TMEM; a CTA that gave up lingers
+  // before the second barrier, which keeps its peer resident too (the
+  // peer's loads complete on the leader's barriers)
   tc_fence_before();
+  cluster_sync();
+  if (threadIdx.x == 0 && *abort_flag) linger_after_abort();
   cluster_sync();
   if (warp == 1) {
     tc_fence_after();
@@ -642,6 +646,7 @@ static cudaError_t launch_pair(const GemmProblem& p, int num_sms, cudaStream_t s
   a.group_offsets = p.group_offsets;
   a.masked_m = p.masked_m;
   a.status = p.status;
+  a.wait_ns = wait_limit_ns();
   a.k_tiles = static_cast<int>(p.k / BK);
   a.sfa_group_bytes = ((p.m + 127) / 128) * 128 * (p.k / 32);
   a.sfb_group_bytes = ((p.n + 127) / 128) * 128 * (p.k / 32);

@@ -15,7 +15,7 @@ constexpr int BM = 128;              // MMA M (rows of A per tile)
 constexpr int BK = 128;              // K elements per pipeline stage (4 scale blocks)
 constexpr int kMaxGroups = 1024;
 constexpr int kGemmThreads = 224;  // 7 warps: producer, MMA, 4 epilogue, scale copier
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // default wait bound, 2 s: far above any legitimate wait
 
 enum GemmMode : int { kDense = 0, kContiguous = 1, kMasked = 2, kKGrouped = 3 };
 
@@ -42,6 +42,7 @@ struct GemmArgs {
   int swiglu_i;             // 0: plain BF16 epilogue
   uint8_t* sfh;             // tiled UE8M0 scales of H
   int64_t sfh_group_bytes;  // masked form: tiled scale bytes of H per expert
+  uint64_t wait_ns;         // bound of every pipeline wait (mx_set_wait_limit_ns)
 };
 
 struct Tile {
@@ -85,6 +86,16 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& a, const int32_t* ta
 
 __device__ __forceinline__ void report(int32_t* status, int bits) {
   atomicOr(status, bits);
+}
+
+// Teardown of a CTA that gave up: every role has stopped issuing, the MMAs
+// and scale copies it issued are drained, but TMA loads issued before the
+// give-up may still be landing in its shared memory.  The CTA stays resident
+// for 1 ms more (one thread spins; the CTA ends when its last thread does),
+// so that they land here and not in the shared memory of a later CTA.
+__device__ __forceinline__ void linger_after_abort() {
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 < 1000000ull) { }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32) {

@@ -66,6 +66,7 @@ struct TwArgs {
   const int32_t* group_offsets;  // contiguous form: [groups + 1]
   int32_t* status;
   int m, n, k_tiles, n_tiles, groups, mode;  // mode 0 dense, 1 contiguous
+  uint64_t wait_ns;                          // bound of every pipeline wait
 };
 
 // Split-K reduction buffer (reuses the operand ring after the mainloop):
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(kTwThreads, 1)
         int group, m_blk, n_blk;
         decode(t, group, m_blk, n_blk);
         for (int kt = kt_begin; kt < kt_end; ++kt) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(stage), L::A_BYTES + L::B_BYTES);
           tma_load_3d(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, full_bar(stage), kt * BK, m_blk * BM, 0);
           tma_load_3d(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, full_bar(stage), kt * BK, n_blk * 128,
@@ -206,11 +207,9 @@ __global__ void __launch_bounds__(kTwThreads, 1)
           if (++stage == kTwStages) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
+      if (!ok) {  // loads already in flight land during the teardown's linger
         report(args.status, 0x4);
         *abort_flag = 1;
-        const uint64_t t0 = global_timer_ns();
-        while (global_timer_ns() - t0 < 1000000ull) { }
       }
     }
   } else if (warp == 1) {
@@ -224,8 +223,8 @@ __global__ void __launch_bounds__(kTwThreads, 1)
       for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
         for (int kt = kt_begin; kt < kt_end; ++kt, ++ib) {
           const uint32_t b = ib % kTwBufs;
-          if (!mbar_wait(acce_bar(b), ((ib / kTwBufs) & 1u) ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(acce_bar(b), ((ib / kTwBufs) & 1u) ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = sbase + L::OFF_A + stage * L::A_BYTES;
           const uint32_t b_addr = sbase + L::OFF_B + stage * L::B_BYTES;
@@ -241,9 +240,10 @@ __global__ void __launch_bounds__(kTwThreads, 1)
       if (!ok) {
         report(args.status, 0x4);
         *abort_flag = 1;
-        tc_commit(drain_bar);
-        mbar_wait(drain_bar, 0, nullptr, 100000000ull);
       }
+      // every MMA issued must finish before TMEM is freed
+      tc_commit(drain_bar);
+      mbar_wait(drain_bar, 0, nullptr, 100000000ull);
     }
   } else {
     // ===== promotion and epilogue (warps 2..5 -> TMEM lane quarters 2,3,0,1)
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kTwThreads, 1)
         }
         // each warp reads only its own TMEM lane quarter: a warp-uniform
         // decision is enough (the aligned TMEM loads need one)
-        const bool got = mbar_wait(accf_bar(b), (ib / kTwBufs) & 1u, abort_flag, kWaitLimitNs);
+        const bool got = mbar_wait(accf_bar(b), (ib / kTwBufs) & 1u, abort_flag, args.wait_ns);
         if (!__all_sync(0xFFFFFFFFu, got)) {
           if (lane == 0) report(args.status, 0x4);
           *abort_flag = 1;
@@ -371,6 +371,7 @@ __global__ void __launch_bounds__(kTwThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
+  if (threadIdx.x == 0 && *abort_flag) linger_after_abort();
 }
 
 template <int SPLIT>
@@ -423,6 +424,7 @@ static cudaError_t launch_tw(const TwProblem& p, int num_sms, cudaStream_t strea
   a.sb = p.sb;
   a.group_offsets = p.group_offsets;
   a.status = p.status;
+  a.wait_ns = wait_limit_ns();
   a.m = static_cast<int>(p.m);
   a.n = static_cast<int>(p.n);
   a.k_tiles = static_cast<int>(p.k / BK);

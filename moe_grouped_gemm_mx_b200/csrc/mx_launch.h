@@ -8,6 +8,10 @@ namespace mxk {
 
 constexpr int kMaxQuantJobs = 8;  // tensors one quantiser launch handles
 
+// Bound, in ns, of every pipeline wait of the GEMM kernels launched from now
+// on (mx_set_wait_limit_ns; 2 s unless changed).
+uint64_t wait_limit_ns();
+
 struct QuantSpec {
   const void* x;            // BF16 [groups, rows, k]
   void* q;                  // E4M3 out, same shape

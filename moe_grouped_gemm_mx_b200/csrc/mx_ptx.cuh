@@ -57,9 +57,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
+  // try_wait may suspend the thread for a microsecond or more before it
+  // reports "not yet", so the bound and the abort flag are checked every 16
+  // attempts: a limit is honoured to within a few tens of microseconds
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
+    if ((it & 15u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (global_timer_ns() - t0 > limit_ns) return false;
     }

@@ -89,8 +89,9 @@ class LibraryOps:
         self.mx.mx_moe_dispatch_quant_peer(x, dst_rank, dst_row, topk, bufs.q_ptrs, bufs.sf_ptrs, bufs.m_cap,
                                            bufs.q, bufs.sf, counts_l, offsets_l, pad, dev_status=self.status)
 
-    def combine_peer(self, bufs, n, dst_rank, dst_row, w):
-        return self.mx.mx_moe_combine_peer(bufs.y_ptrs, bufs.m_cap, n, dst_rank, dst_row, w, dev_status=self.status)
+    def combine_peer(self, bufs, n, dst_rank, dst_row, w, out=None):
+        return self.mx.mx_moe_combine_peer(bufs.y_ptrs, bufs.m_cap, n, dst_rank, dst_row, w, out=out,
+                                           dev_status=self.status)
 
     def check(self, what: str = "expert layer"):
         """Raise if any call since the last check reported a device error
@@ -242,6 +243,10 @@ class PeerBuffers:
         ``group`` (one process per GPU; peers reached over NVLink)."""
         if mx is None:
             import moe_grouped_gemm_mx_b200 as mx
+        import os
+        # the kernels use plain peer loads and stores: no NVLink multicast
+        # object is needed for these buffers
+        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
         import torch.distributed._symmetric_memory as symm
         group = dist.group.WORLD if group is None else group
         device = torch.device("cuda", torch.cuda.current_device())
@@ -254,15 +259,41 @@ class PeerBuffers:
         return cls(*bufs, *tables, dist.get_rank(group))
 
 
-def peer_dispatch(x, ids, experts, count_table, bufs: PeerBuffers, ops=None, pad: int = 128):
+def peer_route(ids, experts, ops=None):
+    """This rank's entries routed with pad 1: (counts [E], row_send [n]) --
+    the row of the count table every rank contributes, and each entry's
+    place in expert order (the placement plan's input)."""
+    ops = LibraryOps() if ops is None else ops
+    counts, _, row_send = ops.route(ids.reshape(-1), experts, 1)
+    return counts, row_send
+
+
+def count_table(counts, group=None):
+    """[ranks, experts] table of every rank's per-expert counts (one NCCL
+    all-gather; the single row itself with one rank)."""
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    if world == 1:
+        return counts.view(1, -1)
+    if counts.is_cuda:   # NCCL gathers straight into the table
+        table = torch.empty((world, counts.numel()), dtype=counts.dtype, device=counts.device)
+        dist.all_gather_into_tensor(table, counts, group=group)
+        return table
+    parts = [torch.empty_like(counts) for _ in range(world)]   # gloo (CPU ranks)
+    dist.all_gather(parts, counts, group=group)
+    return torch.stack(parts)
+
+
+def peer_dispatch(x, ids, experts, table, bufs: PeerBuffers, ops=None, pad: int = 128, row_send=None):
     """Phase 1 on one rank: plan this rank's entries against the all-ranks
     count table and store every routed MXFP8 row in its owner's receive
-    buffer.  Returns the plan (dst_rank, dst_row, counts_local, offsets_local)."""
+    buffer.  ``row_send``: peer_route's, if already computed.  Returns the
+    plan (dst_rank, dst_row, counts_local, offsets_local)."""
     ops = LibraryOps() if ops is None else ops
     T, topk = ids.shape
     flat = ids.reshape(-1)
-    _, _, row_send = ops.route(flat, experts, 1)
-    dst_rank, dst_row, counts_l, offsets_l = ops.peer_plan(flat, row_send, count_table, bufs.rank, experts, pad)
+    if row_send is None:
+        _, row_send = peer_route(flat, experts, ops)
+    dst_rank, dst_row, counts_l, offsets_l = ops.peer_plan(flat, row_send, table, bufs.rank, experts, pad)
     ops.dispatch_peer(x, dst_rank, dst_row, topk, bufs, counts_l, offsets_l, pad)
     return dst_rank, dst_row, counts_l, offsets_l
 
@@ -276,18 +307,19 @@ def peer_experts(bufs: PeerBuffers, plan, q13, sf13, q2, sf2, ops=None):
     ops.down(qh, sfh, q2, sf2, offsets_l, d=bufs.y)
 
 
-def peer_combine(bufs: PeerBuffers, plan, gate_w, n: int, ops=None):
+def peer_combine(bufs: PeerBuffers, plan, gate_w, n: int, ops=None, out=None):
     """Phase 3 on one rank: the gate-weighted sum of its tokens' expert
-    outputs, loaded from their owners' output buffers."""
+    outputs, loaded from their owners' output buffers (into ``out`` if
+    given)."""
     ops = LibraryOps() if ops is None else ops
-    return ops.combine_peer(bufs, n, plan[0], plan[1], gate_w)
+    if out is None:
+        return ops.combine_peer(bufs, n, plan[0], plan[1], gate_w)
+    return ops.combine_peer(bufs, n, plan[0], plan[1], gate_w, out=out)
 
 
 def route_counts(ids, experts, ops=None):
     """This rank's entries per global expert (the row of the count table)."""
-    ops = LibraryOps() if ops is None else ops
-    counts, _, _ = ops.route(ids.reshape(-1), experts, 1)
-    return counts
+    return peer_route(ids, experts, ops)[0]
 
 
 def _stream_barrier(group, device):
@@ -299,36 +331,34 @@ def _stream_barrier(group, device):
 
 
 def ep_moe_layer_peer(x: torch.Tensor, ids: torch.Tensor, gate_w: torch.Tensor, experts: int,
-                      q13, sf13, q2, sf2, bufs: PeerBuffers, group=None, ops=None, pad: int = 128) -> torch.Tensor:
+                      q13, sf13, q2, sf2, bufs: PeerBuffers, group=None, ops=None, pad: int = 128,
+                      check: bool = True, out: torch.Tensor | None = None) -> torch.Tensor:
     """One expert-parallel MoE layer on this rank with the exchange over peer
     memory (arguments as ep_moe_layer; ``bufs`` from PeerBuffers.symmetric).
-    With the default ops the layer checks, before it returns, that no kernel
-    reported an error -- in particular that every owner's plan fitted its
-    receive buffer (rows beyond bufs.m_cap are skipped by the dispatch and
-    reported, and would leave stale expert outputs behind): a RuntimeError
-    otherwise.  Returns BF16 [T, N]."""
+    With the default ops and ``check`` the layer verifies, before it
+    returns, that no kernel reported an error -- in particular that every
+    owner's plan fitted its receive buffer (rows beyond bufs.m_cap are
+    skipped by the dispatch and reported, and would leave stale expert
+    outputs behind): a RuntimeError otherwise.  ``check=False`` skips that
+    device-to-host read (the caller reads ``ops.status`` later, e.g. after
+    a timed loop).  Returns BF16 [T, N] (``out`` if given)."""
     _check_pad(pad)
     ops, own_status = _default_ops(ops, x.device)
     world = dist.get_world_size(group) if dist.is_initialized() else 1
     if experts % world or bufs.ranks != world:
         raise ValueError("the experts must divide evenly over the ranks, one buffer set per rank")
-    counts = route_counts(ids, experts, ops)
-    if world > 1:
-        parts = [torch.empty_like(counts) for _ in range(world)]
-        dist.all_gather(parts, counts, group=group)
-        table = torch.stack(parts)
-    else:
-        table = counts.view(1, experts)
-    plan = peer_dispatch(x, ids, experts, table, bufs, ops, pad)
+    counts, row_send = peer_route(ids, experts, ops)
+    table = count_table(counts, group)
+    plan = peer_dispatch(x, ids, experts, table, bufs, ops, pad, row_send=row_send)
     if world > 1:
         _stream_barrier(group, x.device)
     peer_experts(bufs, plan, q13, sf13, q2, sf2, ops)
     if world > 1:
         _stream_barrier(group, x.device)
-    out = peer_combine(bufs, plan, gate_w, bufs.y.shape[1], ops)
+    out = peer_combine(bufs, plan, gate_w, bufs.y.shape[1], ops, out=out)
     if world > 1:
         _stream_barrier(group, x.device)  # the outputs are read before any rank overwrites its buffers
-    if own_status:
+    if own_status and check:
         ops.check("ep_moe_layer_peer")
     return out
 

@@ -104,11 +104,15 @@ class OracleOps:
             bufs.q[ol[l] + cl[l]:ol[l + 1]] = 0
             bufs.sf[ol[l] + cl[l]:ol[l + 1]] = 0
 
-    def combine_peer(self, bufs, n, dst_rank, dst_row, w):
+    def combine_peer(self, bufs, n, dst_rank, dst_row, w, out=None):
         dr, drow = _np(dst_rank).reshape(-1), _np(dst_row).reshape(-1)
         y = torch.zeros((dr.size, n), dtype=torch.bfloat16)
         for i, (rk, r) in enumerate(zip(dr.tolist(), drow.tolist())):
             if r >= 0:
                 y[i] = bufs.peer_y[rk][r]
         rows = np.where(drow >= 0, np.arange(dr.size), -1).astype(np.int32)
-        return self.combine(y, rows, w)
+        res = self.combine(y, rows, w)
+        if out is None:
+            return res
+        out.copy_(res)
+        return out

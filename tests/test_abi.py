@@ -261,3 +261,15 @@ def test_moe_peer_argument_checks(lib):
     assert comb(None, 2, 8, 16, B, C, D, 4, 2, E, None, None) == MX_ERR_INVALID_ARGUMENT
     assert comb(A + 4, 2, 8, 16, B, C, D, 4, 2, E, None, None) == MX_ERR_MISALIGNED
     assert comb(A, 2, 8, 16, B, C, D, 0, 2, E, None, None) == MX_OK
+
+
+def test_wait_limit_setter(lib):
+    """The GEMM kernels' wait bound: 2 s by default, settable, 0 restores the
+    default (host-side state; no GPU needed)."""
+    lib.mx_wait_limit_ns.restype = ctypes.c_uint64
+    lib.mx_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    assert lib.mx_wait_limit_ns() == 2_000_000_000
+    assert lib.mx_set_wait_limit_ns(1000) == MX_OK
+    assert lib.mx_wait_limit_ns() == 1000
+    assert lib.mx_set_wait_limit_ns(0) == MX_OK
+    assert lib.mx_wait_limit_ns() == 2_000_000_000

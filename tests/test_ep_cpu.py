@@ -180,3 +180,90 @@ def test_ep_layers_reject_pad_off_the_gemm_grid(pad):
                        torch.zeros((128, N), dtype=torch.bfloat16), table, table, table, 0)
     with pytest.raises(ValueError, match="pad"):
         ep_moe_layer_peer(x, torch.from_numpy(ids), torch.from_numpy(gw), E, *w, bufs, ops=OracleOps(), pad=pad)
+
+
+# ---------------------------------------------------------------- bench plumbing
+
+BT, BE, BH, BI, BN = 48, 16, 128, 128, 96     # tokens per rank, experts, hidden, intermediate, output
+
+
+def _rank_main_bench(rank, world, port, shared, out):
+    """One rank of `bench.py --workload moe_layer_ep` at toy size: the bench's
+    own process-group set-up, rank problem and max-over-ranks timing
+    reduction around the peer-memory layer (oracle stand-ins for the
+    kernels, shared CPU tensors for the mapped buffers)."""
+    sys.path[:0] = [ROOT, TESTS]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import bench
+    import mx_inputs
+    import oracle
+    import torch.distributed as dist
+    from ep_ref_ops import OracleOps
+    from moe_grouped_gemm_mx_b200.ep import PeerBuffers, ep_moe_layer_peer
+    w, r, local = bench.dist_init(None)
+    try:
+        assert (w, r, local) == (world, rank, rank)
+        bench.EP_CTX.update(world=w, rank=r, mode="peer")
+        x, ids, gw, w13, w2 = bench.ep_rank_problem(mx_inputs, r, w, BT, BE, BH, BI, BN, seed=5)
+        el = BE // w
+        q13, sf13 = oracle.quantize(w13)
+        q2, sf2 = oracle.quantize(w2)
+        q_all, sf_all, y_all = shared
+        no_table = torch.zeros(w, dtype=torch.int64)
+        bufs = PeerBuffers(q_all[r], sf_all[r], y_all[r], no_table, no_table, no_table, r)
+        bufs.peer_q, bufs.peer_sf, bufs.peer_y = q_all, sf_all, y_all
+        y = ep_moe_layer_peer(x, ids, torch.as_tensor(gw), BE,
+                              torch.from_numpy(q13.reshape(el, 2 * BI, BH)),
+                              torch.from_numpy(sf13.reshape(el, 2 * BI, BH // 32)),
+                              torch.from_numpy(q2.reshape(el, BN, BI)), torch.from_numpy(sf2.reshape(el, BN, BI // 32)),
+                              bufs, ops=OracleOps())
+        t_max = bench.max_over_ranks(w, 1.0 + r, torch.device("cpu"))
+        out[r] = (y.view(torch.int16).numpy().copy(), t_max)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_ep_workload_plumbing():
+    """Two gloo ranks through bench.py's moe_layer_ep plumbing: every rank's
+    output equals the one-process layer over all ranks' tokens and all
+    experts (the ranks' expert shares together are one set of experts), the
+    step time is the max over ranks, and the interleaved expert placement
+    gives each rank every W-th popularity rank."""
+    import bench
+    import mx_inputs
+    import oracle
+    from ep_ref_ops import OracleOps
+    from moe_grouped_gemm_mx_b200.ep import ep_moe_layer
+    world = 2
+    el = BE // world
+    assert [bench.ep_expert_label(p, BE, world) // el for p in range(BE)] == [p % world for p in range(BE)]
+    entries = world * BT * min(8, BE)
+    m_cap = (entries + el * 127 + 127) // 128 * 128
+    shared = ([torch.full((m_cap, BH), 0xAB, dtype=torch.uint8).share_memory_() for _ in range(world)],
+              [torch.full((m_cap, BH // 32), 0xCD, dtype=torch.uint8).share_memory_() for _ in range(world)],
+              [torch.zeros((m_cap, BN), dtype=torch.bfloat16).share_memory_() for _ in range(world)])
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.spawn(_rank_main_bench, args=(world, port, shared, out), nprocs=world, join=True)
+    parts = [bench.ep_rank_problem(mx_inputs, r, world, BT, BE, BH, BI, BN, seed=5) for r in range(world)]
+    one = bench.ep_rank_problem(mx_inputs, 0, 1, BT, BE, BH, BI, BN, seed=5)
+    w13 = torch.cat([p[3] for p in parts])
+    w2 = torch.cat([p[4] for p in parts])
+    assert torch.equal(w13.view(torch.int16), one[3].view(torch.int16))   # expert e's weights depend on e only
+    q13, sf13 = oracle.quantize(w13)
+    q2, sf2 = oracle.quantize(w2)
+    x = torch.cat([p[0] for p in parts])
+    ids = torch.cat([p[1] for p in parts])
+    gw = torch.cat([torch.as_tensor(p[2]) for p in parts])
+    ref = ep_moe_layer(x, ids, gw, BE, torch.from_numpy(q13.reshape(BE, 2 * BI, BH)),
+                       torch.from_numpy(sf13.reshape(BE, 2 * BI, BH // 32)), torch.from_numpy(q2.reshape(BE, BN, BI)),
+                       torch.from_numpy(sf2.reshape(BE, BN, BI // 32)), ops=OracleOps())
+    ref_bits = ref.view(torch.int16).numpy()
+    for r in range(world):
+        y_bits, t_max = out[r]
+        assert np.array_equal(y_bits, ref_bits[r * BT:(r + 1) * BT]), f"rank {r}"
+        assert t_max == float(world)
+    assert np.abs(ref.float().numpy()).max() > 0
