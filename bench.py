@@ -29,10 +29,17 @@ Workloads (shapes from the pages; data synthetic and seeded):
   moe_layer   a whole expert layer: route, dispatch, gate/up.SwiGLU, down, combine
   moe_layer_peer  the same layer through the expert-parallel peer-memory kernels
               (placement plan, dispatch and combine through pointer tables), one rank
+  moe_layer_ep  the expert layer with expert parallelism over the job's ranks: each
+              rank holds 8192 tokens and 32/N of the experts; the exchange runs
+              over peer memory (--ep peer: symmetric-memory buffers, the dispatch
+              and combine kernels store to / load from the owners) or NCCL
+              all-to-alls (--ep nccl)
 
 With torchrun (N > 1) every rank runs its own independent batch (the work
 units are independent problems; no data-path collective), the step time is
-the max over ranks and `value` counts the work of all ranks ("weak" scaling).
+the max over ranks and `value` counts the work of all ranks ("weak" scaling);
+moe_layer_ep is the exception: its ranks exchange tokens and expert outputs
+every step.
 `--impl reference` times the CPU oracle (rank 0 only) on a bounded sample of
 the same workload, in the same unit.
 """
@@ -59,6 +66,10 @@ FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 QUANT_BYTES_PER_ELT = 2.0 + 1.0 + 1.0 / 32.0
 METRIC = "MXFP8 GEMM & grouped-GEMM TFLOPS on 1 B200; % of dense FP8 tensor peak"
 
+
+# expert-parallel workload: this process's rank, the job's ranks and the
+# exchange form (set from the launch environment and --ep)
+EP_CTX = {"world": 1, "rank": 0, "mode": "peer"}
 
 # MoE problem size: the configured 32 experts x 8192 tokens unless
 # --experts / --tokens override it (used only to make small ncu captures)
@@ -103,6 +114,18 @@ def static_config(name: str, seed: int) -> dict:
                     "padded_rows": int(I.padded_offsets(counts)[-1]),
                     "gemms": ["dgrad dX[T,7168] = dY[T,4096] W13 (contiguous, W13 quantised along N)",
                               "wgrad dW13[32,4096,7168] = dY^T X per expert (K-grouped over tokens)"]})
+    elif name == "moe_layer_ep":
+        tokens = MOE_OVERRIDE["tokens"] or I.MOE_TOKENS
+        experts = MOE_OVERRIDE["experts"] or I.MOE_EXPERTS
+        world = EP_CTX["world"]
+        cfg.update({"experts": experts, "ranks": world, "experts_per_rank": experts // max(1, world),
+                    "tokens_per_rank": tokens, "topk": I.MOE_TOPK, "zipf_s": I.MOE_ZIPF_S,
+                    "hidden": I.MOE_GATE_NK[1], "intermediate": I.MOE_DOWN_NK[1],
+                    "exchange": ("NCCL all-to-alls" if EP_CTX["mode"] == "nccl" else
+                                 "peer memory (dispatch stores into / combine loads from the owners' buffers)"),
+                    "expert_placement": "popularity rank p -> label (p % ranks) * (E / ranks) + p // ranks; "
+                                        "rank r owns labels [r E/ranks, (r+1) E/ranks)",
+                    "gate_weights": "softmax over N(0,1) logits"})
     elif name in ("moe_layer", "moe_layer_peer"):
         import numpy as np
         tokens = MOE_OVERRIDE["tokens"] or I.MOE_TOKENS
@@ -151,7 +174,9 @@ def parse_args():
     p.add_argument("--steps", type=int, default=100)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="contiguous", choices=["page", "pr1", "large", "contiguous", "masked", "moe_mlp", "moe_bwd",
-                                                            "moe_layer", "moe_layer_peer"])
+                                                            "moe_layer", "moe_layer_peer", "moe_layer_ep"])
+    p.add_argument("--ep", default="peer", choices=["peer", "nccl"],
+                   help="moe_layer_ep: exchange over peer memory (default) or NCCL all-to-alls")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -269,6 +294,39 @@ def system_info(dev, smi_id: str) -> dict:
 
 # ---------------------------------------------------------------- workloads
 
+def ep_expert_label(p: int, experts: int, world: int) -> int:
+    """Label of the expert of popularity rank p when the experts are spread
+    over ``world`` ranks: rank r owns labels [r E/W, (r+1) E/W) and gets the
+    popularity ranks r, r + W, r + 2W, ... (owning a contiguous block of
+    popularity ranks would give rank 0 all the hottest experts)."""
+    el = experts // world
+    return (p % world) * el + p // world
+
+
+def ep_rank_problem(I, rank: int, world: int, tokens: int, experts: int, hidden: int, inter: int, n_out: int,
+                    seed: int, device="cpu"):
+    """One rank's share of the expert-parallel layer: its ``tokens`` BF16 rows
+    x [T, hidden], their top-k expert labels ids int32 [T, topk] (Zipf
+    popularity, relabelled by ep_expert_label) and gate weights float32
+    [T, topk], and the weights of the experts it owns: w13 [E/W, 2*inter,
+    hidden] ([gate; up]) and w2 [E/W, n_out, inter].  Expert e's weights
+    depend only on e, so the ranks' shares together are one set of experts."""
+    import numpy as np
+    import torch
+    topk = min(I.MOE_TOPK, experts)
+    el = experts // world
+    pop = I.topk_ids(tokens, topk, experts, seed=seed + 7919 * rank)
+    lut = np.array([ep_expert_label(p, experts, world) for p in range(experts)], dtype=np.int32)
+    ids = torch.from_numpy(lut[pop]).to(device)
+    gw = torch.from_numpy(I.gate_weights(tokens, topk, seed=seed + 7919 * rank)).to(device)
+    x = I.normal_bf16((tokens, hidden), 1.0, seed + 7 + 7919 * rank, device)
+    own = range(rank * el, (rank + 1) * el)
+    w13 = torch.stack([I.normal_bf16((2 * inter, hidden), 0.02, seed + 2_000_003 + 31 * e, device) for e in own])
+    w2 = torch.stack([I.normal_bf16((n_out, inter), 0.02, seed + 4_000_037 + 31 * e, device) for e in own])
+    return x, ids, gw, w13, w2
+
+
+
 class Workload:
     """Device-resident inputs/outputs and the list of kernel launches of one step."""
 
@@ -289,6 +347,11 @@ class Workload:
         # on parallel streams / graph branches after the launches in none
         self.branches = None
         self._side = []
+        # launches timed one by one for the per-kernel table but not part of
+        # the step (a step whose launches cannot be replayed alone times its
+        # GEMMs this way), and our kernels per step when a launch runs several
+        self.timing_launches = []
+        self.kernels_per_step = None
         if fmt == "tilewise":
             if name not in ("pr1", "page", "large", "contiguous"):
                 raise SystemExit(f"--fmt tilewise applies to the dense and contiguous workloads, not {name}")
@@ -623,6 +686,82 @@ class Workload:
                             "exchange": "peer-memory kernels through device pointer tables (one rank: local)",
                             "gate_weights": "softmax over N(0,1) logits"})
 
+    def _build_moe_layer_ep(self, seed, I):
+        """The expert layer with expert parallelism over the job's ranks
+        (ep_moe_layer_peer or, with --ep nccl, ep_moe_layer): this rank's
+        8192 tokens and its 32/W experts' weights (quantised every step), the
+        exchange over peer memory or NCCL.  One rank: the same call with the
+        pointer tables pointing at local memory.  The step is the layer call
+        as a user makes it; the two grouped GEMMs are also replayed alone (on
+        a plan computed once) for the per-kernel table."""
+        import torch
+        from moe_grouped_gemm_mx_b200 import ep
+        mx = self.mx
+        world, rank, mode = EP_CTX["world"], EP_CTX["rank"], EP_CTX["mode"]
+        T = MOE_OVERRIDE["tokens"] or I.MOE_TOKENS
+        E = MOE_OVERRIDE["experts"] or I.MOE_EXPERTS
+        if E % world:
+            raise SystemExit(f"moe_layer_ep: {E} experts do not divide over {world} ranks")
+        el = E // world
+        topk = min(I.MOE_TOPK, E)
+        n13, hdim = I.MOE_GATE_NK
+        n2, i_dim = I.MOE_DOWN_NK
+        x, ids, gw, w13, w2 = ep_rank_problem(I, rank, world, T, E, hdim, n13 // 2, n2, seed % 1000, self.dev)
+        for t in (x, ids, gw, w13, w2):
+            self._add_input(t)
+        q13, sf13 = self._quant(w13, "W13 (own experts)")
+        q2, sf2 = self._quant(w2, "W2 (own experts)")
+        ops = ep.LibraryOps(mx, status=self.status)
+        out = torch.empty((T, n2), dtype=torch.bfloat16, device=self.dev)
+        self.outputs.append(out)
+        n = T * topk
+        if mode == "peer":
+            # the largest plan any rank can receive: every entry of every rank
+            m_cap = mx.mx_moe_max_rows(world * n, el, 128)
+            bufs = (ep.PeerBuffers.symmetric(m_cap, hdim, n2) if world > 1 else
+                    ep.PeerBuffers.emulated(1, m_cap, hdim, n2, self.dev)[0])
+
+            def layer(x, ids, gw, q13, sf13, q2, sf2):
+                ep.ep_moe_layer_peer(x, ids, gw, E, q13, sf13, q2, sf2, bufs, ops=ops, check=False, out=out)
+            kernels = 6   # route, placement plan, dispatch, gate/up+SwiGLU, down, combine
+        else:
+            def layer(x, ids, gw, q13, sf13, q2, sf2):
+                out.copy_(ep.ep_moe_layer(x, ids, gw, E, q13, sf13, q2, sf2, ops=ops))
+            kernels = 8   # route, dispatch, route, scatter, gate/up+SwiGLU, down, gather, combine
+        fl = 2.0 * n * n13 * hdim + 2.0 * n * n2 * i_dim        # this rank's tokens' entries, wherever computed
+        layer_bytes = (T * hdim * 2.0 + 2 * n * hdim * (1 + 1 / 32)          # tokens in; rows sent and received
+                       + el * (n13 * hdim + n2 * i_dim) * (1 + 1 / 32)       # own experts' weights
+                       + 2 * n * n2 * 2.0 + T * n2 * 2.0)                     # expert outputs; combined rows
+        self.launches.append(("layer", f"expert-parallel layer ({mode}, {world} rank(s))", layer, layer_bytes, fl,
+                              (x, ids, gw, q13, sf13, q2, sf2)))
+        self.flops += fl
+        self.kernels_per_step = 1 + kernels
+        # this rank's receive plan (computed once, as the layer computes it
+        # every step) for its two grouped GEMMs timed alone, on received rows
+        # that stand in for the real ones: N(0,1) tokens quantised like them
+        # (all-zero operands would draw less power and clock higher)
+        counts, row_send = ep.peer_route(ids, E, ops)
+        table = ep.count_table(counts)
+        _, _, counts_l, offsets_l = ops.peer_plan(ids.reshape(-1), row_send, table, rank, E, 128)
+        torch.cuda.synchronize()
+        rows_l = max(int(offsets_l[-1].item()), 128)
+        real_l = int(counts_l.sum().item())
+        qa, sfa = mx.mx_quantize_bf16_to_e4m3(I.normal_bf16((rows_l, hdim), 1.0, seed + 99, self.dev))
+        qh = torch.empty((rows_l, i_dim), dtype=torch.uint8, device=self.dev)
+        sfh = torch.empty(mx.scale_bytes(rows_l, i_dim), dtype=torch.uint8, device=self.dev)
+        y = torch.empty((rows_l, n2), dtype=torch.bfloat16, device=self.dev)
+        self.timing_launches.append(("gemm", "gate_up+swiglu (own experts, received rows)",
+                                     lambda qa, sfa, q13, sf13, off: mx.mx_grouped_gemm_contiguous_swiglu_quant(
+                                         qa, sfa, q13, sf13, off, qh=qh, sfh=sfh, dev_status=self.status),
+                                     (rows_l * hdim + el * n13 * hdim + rows_l * i_dim) * (1 + 1 / 32),
+                                     2.0 * real_l * n13 * hdim, (qa, sfa, q13, sf13, offsets_l)))
+        self.timing_launches.append(("gemm", "down (own experts, received rows)",
+                                     lambda qh_, sfh_, q2, sf2, off: mx.mx_grouped_gemm_contiguous(
+                                         qh_, sfh_, q2, sf2, off, d=y, dev_status=self.status),
+                                     self._gemm_bytes(rows_l, n2, i_dim, el), 2.0 * real_l * n2 * i_dim,
+                                     (qh, sfh, q2, sf2, offsets_l)))
+        self.config.update({"ranks": world, "received_rows_this_rank": real_l})
+
     def _build_moe_bwd(self, seed, I):
         """Backward of the MoE gate/up projection (the contiguous workload's
         first GEMM): input gradient dX = dY W13 per expert and weight gradient
@@ -820,7 +959,7 @@ def oracle_sample(name, seed, target_s=10.0, fmt="mxfp8"):
         jobs.append(job)
         desc = ("one expert layer on 64 rows over 2 experts: quantise rows and weights, gate/up GEMM, "
                 "SwiGLU, requantise, down GEMM")
-    elif name in ("moe_layer", "moe_layer_peer"):
+    elif name in ("moe_layer", "moe_layer_peer", "moe_layer_ep"):
         n13, k = I.MOE_GATE_NK
         n2, i_dim = I.MOE_DOWN_NK
         T, topk, E = 8, I.MOE_TOPK, 8
@@ -987,7 +1126,10 @@ def run_ours(args, world, rank, local):
     wl = Workload(args.workload, dev, args.seed + 1000 * rank, mx, mx_inputs, fmt=args.fmt)
     stream = torch.cuda.Stream(device=dev)
     flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    n_k = len(wl.launches)
+    # launches timed one by one: the step's own (except a whole-layer call,
+    # whose collectives cannot be replayed alone) and the timing-only ones
+    timed = [l for l in wl.launches if l[0] != "layer"] + wl.timing_launches
+    n_k = len(timed)
 
     # one eager pass (sets kernel attributes), then capture the step
     with torch.cuda.stream(stream):
@@ -1064,7 +1206,7 @@ def run_ours(args, world, rank, local):
     t_k0 = time.time()
     kernel_reps = max(3, min(args.steps, 10))
     l2_cover = 256 * 1024 * 1024
-    for i, (_, _, fn, _, _, inputs) in enumerate(wl.launches):
+    for i, (_, _, fn, _, _, inputs) in enumerate(timed):
         in_bytes = sum(t.numel() * t.element_size() for t in inputs)
         copies = max(1, min(32, -(-l2_cover // max(in_bytes, 1))))
         bufs = [inputs] + [tuple(t.clone() for t in inputs) for _ in range(copies - 1)]
@@ -1113,7 +1255,7 @@ def run_ours(args, world, rank, local):
 
     # per-kernel breakdown and the roofline of the dominant kernel kind
     per_launch = []
-    for i, (kind, label, _, nbytes, fl, _) in enumerate(wl.launches):
+    for i, (kind, label, _, nbytes, fl, _) in enumerate(timed):
         per_launch.append({"kind": kind, "label": label, "ms": statistics.mean(kern_ms[i]),
                            "bytes": nbytes, "flops": fl})
     kinds = {}
@@ -1183,7 +1325,7 @@ def run_ours(args, world, rank, local):
         rate, desc, threads = oracle_sample(args.workload, args.seed, target_s=10.0, fmt=args.fmt)
         cpu = {"value": rate / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
 
-    launches_per_step = sum(1 for r in per_launch)
+    launches_per_step = wl.kernels_per_step or len(wl.launches)
     line = {
         "metric": METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -1212,6 +1354,11 @@ def main():
     MOE_OVERRIDE["experts"] = args.experts
     MOE_OVERRIDE["tokens"] = args.tokens
     world, rank, local = dist_init(args)
+    EP_CTX.update(world=world, rank=rank, mode=args.ep)
+    if args.workload == "moe_layer_ep" and (world > 1 or args.ep == "nccl"):
+        # the step holds NCCL collectives (and, for the NCCL form, a host read
+        # of the row counts): launched eagerly, not captured in a graph
+        args.eager = True
     try:
         if args.impl == "reference":
             rc = run_reference(args, world, rank)
