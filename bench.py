@@ -20,7 +20,7 @@ Workloads (shapes from the pages; data synthetic and seeded):
   contiguous  MoE grouped, 32 experts, 8192 tokens top-8 Zipf: gate/up N=4096 K=7168,
               then down N=7168 K=2048 (default: the largest configuration, tensor-bound)
   page        dense 64x2112x7168, 64x24576x1536, 128x7168x2048; the three
-              independent shapes' GEMMs run on parallel streams
+              independent shapes' GEMMs in one mx_gemm_batch launch
   pr1         dense 128x256x512
   large       dense M=8192, (N,K) in {(7168,2048),(2112,7168),(4096,7168)}
   masked      MoE masked grouped, 32 experts x 256 rows, masked_m ~ U{0..256}, N=4096 K=7168
@@ -152,6 +152,13 @@ def static_config(name: str, seed: int) -> dict:
     elif name == "moe_layer_peer":
         cfg["step"] = ("the moe_layer step through the expert-parallel peer-memory kernels on one rank: "
                        "route (pad 1), placement plan, dispatch and combine through device pointer tables")
+    elif name == "moe_layer_ep":
+        cfg["step"] = ("quantise this rank's experts' weights, then one expert-parallel layer call: route, "
+                       "count exchange, placement plan, dispatch to the owners, fused gate/up GEMM -> SwiGLU "
+                       "-> MXFP8 and down GEMM on the received rows, combine from the owners")
+    elif name == "page":
+        cfg["step"] = ("quantise activations + weights of the three shapes (one batched launch), then their "
+                       "three GEMMs in one mx_gemm_batch launch with BF16 epilogue")
     else:
         cfg["step"] = ("quantise activations + weights (one batched launch), then the GEMM(s) "
                        "with BF16 epilogue")
@@ -443,19 +450,37 @@ class Workload:
         self.config.update({"shapes": ["128x256x512"]})
 
     def _build_page(self, seed, I):
-        for (m, n, k) in I.PAGE_SHAPES:
-            a, b = I.dense_problem(m, n, k, seed=seed, kind="outlier", device=self.dev)
-            self._dense(a, b, f"{m}x{n}x{k}")
-        # the three shapes are independent problems: their GEMMs run on
-        # parallel streams (branches of the step's graph), so that their fixed
-        # costs overlap -- after the one batched quantiser launch (MXFP8), or
-        # each behind its own two quantiser launches (tile-wise)
-        if self.fmt == "mxfp8":
-            self.branches = [[1], [2], [3]]
-            self.config["gemms"] = "three independent GEMMs on parallel streams / graph branches after the quantiser"
-        else:
+        if self.fmt == "tilewise":
+            for (m, n, k) in I.PAGE_SHAPES:
+                a, b = I.dense_problem(m, n, k, seed=seed, kind="outlier", device=self.dev)
+                self._dense(a, b, f"{m}x{n}x{k}")
+            # per shape: quantise A, quantise B, GEMM; the three shapes on parallel streams
             self.branches = [[0, 1, 2], [3, 4, 5], [6, 7, 8]]
             self.config["gemms"] = "per shape: quantise A, quantise B, GEMM, the three shapes on parallel streams"
+        else:
+            # the three independent problems' GEMMs in one mx_gemm_batch
+            # launch (the GPU shared among them), after the batched quantiser
+            import torch
+            mx = self.mx
+            qs, ds, fl, nbytes, labels = [], [], 0.0, 0.0, []
+            for (m, n, k) in I.PAGE_SHAPES:
+                a, b = I.dense_problem(m, n, k, seed=seed, kind="outlier", device=self.dev)
+                self._add_input(a)
+                self._add_input(b)
+                lab = f"{m}x{n}x{k}"
+                qa, sfa = self._quant(a, lab + ":A")
+                qb, sfb = self._quant(b, lab + ":B")
+                d = torch.empty((m, n), dtype=torch.bfloat16, device=self.dev)
+                self.outputs.append(d)
+                qs += [qa, sfa, qb, sfb]
+                ds.append(d)
+                fl += 2.0 * m * n * k
+                nbytes += self._gemm_bytes(m, n, k)
+                labels.append(lab)
+            self.launches.append(("gemm", "batch " + "+".join(labels), lambda *t: mx.mx_gemm_batch(
+                [t[4 * i:4 * i + 4] for i in range(len(ds))], outs=ds, dev_status=self.status), nbytes, fl, tuple(qs)))
+            self.flops += fl
+            self.config["gemms"] = "the three independent GEMMs in one mx_gemm_batch launch after the quantiser"
         self.config.update({"shapes": [f"{m}x{n}x{k}" for m, n, k in I.PAGE_SHAPES],
                             "a": "N(0,1) with 0.5% x64 outliers", "b": "N(0,0.02)"})
 

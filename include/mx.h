@@ -130,6 +130,34 @@ mx_status mx_gemm(const void *qa, const void *sfa, const void *qb, const void *s
                   int64_t m, int64_t n, int64_t k, int32_t *dev_status, mx_stream_t stream);
 
 /*
+ * Several independent dense MXFP8 GEMMs in ONE launch: D_i = A_i * B_i^T for
+ * i < count ("DeepGEMM" summary page, CUTLASS comparison table: the dense
+ * shapes it lists are separate small-M problems of one model, e.g.
+ * 64x2112x7168, 64x24576x1536 and 128x7168x2048).  Each problem follows
+ * mx_gemm's contract (layouts, alignment, k % 128 == 0, n % 16 == 0, the
+ * same result up to FP32 summation order); problems with m == 0 or n == 0
+ * are no-ops.  The GPU is shared among the problems so that all of them
+ * stream their operands at once instead of one launch after another: each
+ * gets a share of the SMs sized to its bytes, with K split across a cluster
+ * where that shortens it.  Meant for problems too small to fill the GPU
+ * alone; every problem uses 128 x 128 tiles.
+ *   problems  host array of `count` descriptors, read during the call;
+ *   1 <= count <= MX_GEMM_BATCH_MAX (else MX_ERR_INVALID_ARGUMENT).
+ * One status word for all problems (dev_status, nullable).
+ */
+#define MX_GEMM_BATCH_MAX 4
+typedef struct {
+    const void *qa;   /* [m, k] E4M3 */
+    const void *sfa;  /* mx_scale_bytes(m, k) tiled scales of A */
+    const void *qb;   /* [n, k] E4M3 */
+    const void *sfb;  /* mx_scale_bytes(n, k) tiled scales of B */
+    void *d_bf16;     /* [m, n] BF16 out */
+    int64_t m, n, k;
+} mx_gemm_problem;
+
+mx_status mx_gemm_batch(const mx_gemm_problem *problems, int32_t count, int32_t *dev_status, mx_stream_t stream);
+
+/*
  * Contiguous-layout MoE grouped GEMM ("DeepGEMM" release page, section 4:
  * token sequences of all experts grouped into one M dimension).
  *   qa [m_total, k] holds the groups back to back; group e owns rows

@@ -53,13 +53,21 @@ C_SYMBOLS = [
     "mx_quantize_bf16_to_e4m3_block128x128", "mx_gemm_tilewise", "mx_grouped_gemm_contiguous_tilewise",
     "mx_moe_max_rows", "mx_moe_route", "mx_moe_dispatch_quant", "mx_moe_scatter_rows", "mx_gather_rows",
     "mx_moe_combine", "mx_moe_peer_plan", "mx_moe_dispatch_quant_peer", "mx_moe_combine_peer",
-    "mx_set_wait_limit_ns", "mx_wait_limit_ns",
+    "mx_set_wait_limit_ns", "mx_wait_limit_ns", "mx_gemm_batch",
 ]
+
+MX_GEMM_BATCH_MAX = 4
 
 
 class _QuantJob(ctypes.Structure):
     _fields_ = [("x_bf16", ctypes.c_void_p), ("groups", ctypes.c_int64), ("rows", ctypes.c_int64),
                 ("k", ctypes.c_int64), ("q_e4m3", ctypes.c_void_p), ("sf_ue8m0", ctypes.c_void_p)]
+
+
+class _GemmProblem(ctypes.Structure):
+    _fields_ = [("qa", ctypes.c_void_p), ("sfa", ctypes.c_void_p), ("qb", ctypes.c_void_p),
+                ("sfb", ctypes.c_void_p), ("d_bf16", ctypes.c_void_p), ("m", ctypes.c_int64),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64)]
 
 
 class MXError(RuntimeError):
@@ -129,6 +137,8 @@ def _load():
     L.mx_moe_combine_peer.restype = ctypes.c_int
     L.mx_read_internal_status.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int]
     L.mx_read_internal_status.restype = ctypes.c_int
+    L.mx_gemm_batch.argtypes = [ctypes.POINTER(_GemmProblem), I32, P, P]
+    L.mx_gemm_batch.restype = ctypes.c_int
     L.mx_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     L.mx_set_wait_limit_ns.restype = ctypes.c_int
     L.mx_wait_limit_ns.argtypes = []
@@ -275,6 +285,32 @@ def mx_gemm(qa, sfa, qb, sfb, d: torch.Tensor | None = None, dev_status: torch.T
                       _status_arg(dev_status), _stream(stream))
     _raise(st, "mx_gemm")
     return d
+
+
+def mx_gemm_batch(problems, outs=None, dev_status: torch.Tensor | None = None, stream=None):
+    """Up to MX_GEMM_BATCH_MAX independent dense GEMMs in one launch.
+    problems: sequence of (qa, sfa, qb, sfb) as for mx_gemm; outs: optional
+    BF16 [M_i, N_i] outputs.  Returns the list of D_i."""
+    count = len(problems)
+    if not 1 <= count <= MX_GEMM_BATCH_MAX:
+        raise ValueError(f"1 to {MX_GEMM_BATCH_MAX} problems per batch")
+    arr = (_GemmProblem * count)()
+    ds = []
+    for i, (qa, sfa, qb, sfb) in enumerate(problems):
+        for t, nm in ((qa, "qa"), (sfa, "sfa"), (qb, "qb"), (sfb, "sfb")):
+            _check(t, torch.uint8, nm)
+        m, k = qa.shape
+        n = qb.shape[0]
+        if qb.shape[1] != k:
+            raise ValueError(f"problem {i}: K mismatch")
+        d = outs[i] if outs is not None else torch.empty((m, n), dtype=torch.bfloat16, device=qa.device)
+        _check(d, torch.bfloat16, "d")
+        if tuple(d.shape) != (m, n):
+            raise ValueError(f"problem {i}: D must be [{m}, {n}]")
+        arr[i] = _GemmProblem(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(d), m, n, k)
+        ds.append(d)
+    _raise(_lib.mx_gemm_batch(arr, count, _status_arg(dev_status), _stream(stream)), "mx_gemm_batch")
+    return ds
 
 
 def mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, group_offsets: torch.Tensor,

@@ -181,6 +181,37 @@ mx_status mx_gemm(const void* qa, const void* sfa, const void* qb, const void* s
   return from_cuda(mxk::launch_gemm(p, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
 }
 
+mx_status mx_gemm_batch(const mx_gemm_problem* problems, int32_t count, int32_t* dev_status, mx_stream_t stream) {
+  static_assert(MX_GEMM_BATCH_MAX == mxk::kMaxBatch, "batch limit");
+  if (!problems || count < 1 || count > MX_GEMM_BATCH_MAX) return MX_ERR_INVALID_ARGUMENT;
+  mxk::GemmProblem ps[MX_GEMM_BATCH_MAX];
+  int32_t* status = nullptr;
+  int n_live = 0;
+  for (int32_t i = 0; i < count; ++i) {  // every problem checked before anything is launched
+    const mx_gemm_problem& q = problems[i];
+    if (q.m < 0 || q.n < 0 || q.k < 0) return MX_ERR_INVALID_ARGUMENT;
+    if (q.m == 0 || q.n == 0) {
+      if (q.k % 128 != 0 || q.k == 0 || q.n % 16 != 0) return MX_ERR_UNSUPPORTED_SHAPE;
+      continue;
+    }
+    mx_status st = check_gemm_common(q.qa, q.sfa, q.qb, q.sfb, q.d_bf16, q.m, q.n, q.k, 1);
+    if (st != MX_OK) return st;
+    ++n_live;
+  }
+  if (n_live == 0) return MX_OK;
+  const int sms = num_sms();
+  if (sms <= 0) return MX_ERR_CUDA;
+  status = dev_status ? dev_status : internal_status_ptr();
+  if (!status) return MX_ERR_CUDA;
+  int n = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    const mx_gemm_problem& q = problems[i];
+    if (q.m == 0 || q.n == 0) continue;
+    ps[n++] = mxk::GemmProblem{q.qa, q.sfa, q.qb, q.sfb, q.d_bf16, nullptr, nullptr, status, q.m, q.n, q.k, 1, 0};
+  }
+  return from_cuda(mxk::launch_gemm_batch(ps, n, sms, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
 mx_status mx_grouped_gemm_contiguous(const void* qa, const void* sfa, const void* qb, const void* sfb,
                                      const int32_t* group_offsets, int32_t groups, int64_t m_total, int64_t n,
                                      int64_t k, void* d_bf16, int32_t* dev_status, mx_stream_t stream) {

@@ -94,18 +94,19 @@ struct Layout {
   __host__ __device__ static constexpr int quad_owner(int q) { return (q * SPLIT) / QUADS; }
 };
 
-template <int BN, int STAGES, int ACC, int SPLIT, int BMA>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                   const __grid_constant__ CUtensorMap tmap_d, const GemmArgs args) {
-  using L = Layout<BN, STAGES, ACC, SPLIT, BMA>;
-  // SPLIT > 1 (dense form only): a cluster of SPLIT CTAs shares one output
-  // tile, each CTA accumulating a contiguous share of the K tiles; the FP32
-  // partials are reduced through distributed shared memory.
-  const int split_rank = SPLIT > 1 ? static_cast<int>(cluster_ctarank()) : 0;
-  const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT : static_cast<int>(blockIdx.x);
-  const int kt_begin = SPLIT > 1 ? split_rank * args.k_tiles / SPLIT : 0;
-  const int kt_end = SPLIT > 1 ? (split_rank + 1) * args.k_tiles / SPLIT : args.k_tiles;
+// One CTA of the GEMM: tiles t_first, t_first + t_stride, ... of the problem
+// in `args` (operands through the three tensor maps), or, with split > 1
+// (dense form only, split == SPLIT_MAX), the K tiles [kt_begin, kt_end) of
+// the single tile t_first, which the `split` CTAs of this cluster share: each
+// accumulates a contiguous share of K and the FP32 partials are reduced
+// through distributed shared memory.  Every CTA of a cluster has the same
+// split.
+template <int BN, int STAGES, int ACC, int SPLIT_MAX, int BMA>
+__device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtensorMap* tmap_b,
+                                         const CUtensorMap* tmap_d, const GemmArgs& args, const int split,
+                                         const int split_rank, const int t_first, const int t_stride,
+                                         const int kt_begin, const int kt_end) {
+  using L = Layout<BN, STAGES, ACC, SPLIT_MAX, BMA>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -145,9 +146,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     *abort_flag = 0;
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmap_a);
-    prefetch_tmap(&tmap_b);
-    prefetch_tmap(&tmap_d);
+    prefetch_tmap(tmap_a);
+    prefetch_tmap(tmap_b);
+    prefetch_tmap(tmap_d);
   }
   // Everything above touches only this CTA's shared memory and the kernel
   // parameters.  With programmatic dependent launch the next kernel may begin
@@ -227,7 +228,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
+      for (int t = t_first; t < total && ok; t = split > 1 ? total : t + t_stride) {
         const Tile tl = decode_tile(args, tab0, t);
         const int a_row = tl.m_blk * BM;
         const int a_z = (args.mode == kMasked) ? tl.group : 0;
@@ -245,8 +246,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // accumulator rows that are never stored
           const uint32_t bytes = args.a_box_rows * BK + L::B_BYTES + L::SFA_BYTES + 512u * nsfb;
           mbar_arrive_expect_tx(full_bar(stage), bytes);
-          tma_load_3d(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, full_bar(stage), kt * BK, a_row, a_z);
-          tma_load_3d(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, full_bar(stage), kt * BK,
+          tma_load_3d(sbase + L::OFF_A + stage * L::A_BYTES, tmap_a, full_bar(stage), kt * BK, a_row, a_z);
+          tma_load_3d(sbase + L::OFF_B + stage * L::B_BYTES, tmap_b, full_bar(stage), kt * BK,
                       tl.n_blk * BN, b_z);
           bulk_load(sbase + L::OFF_SFA + stage * L::SFA_BYTES, sfa_base + kt * 512, 512, full_bar(stage));
           for (int j = 0; j < nsfb; ++j)
@@ -271,7 +272,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
+      for (int t = t_first; t < total && ok; t = split > 1 ? total : t + t_stride) {
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_t = tmem_base + acc * BN;
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = t_first; t < total && ok; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
+      for (int t = t_first; t < total && ok; t = split > 1 ? total : t + t_stride) {
         for (int kt = kt_begin; kt < kt_end; ++kt) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t stg_count = 0;  // staging chunks used so far (buffer = count & 1)
-    for (int t = t_first; t < total; t = SPLIT > 1 ? total : t + static_cast<int>(gridDim.x)) {
+    for (int t = t_first; t < total; t = split > 1 ? total : t + t_stride) {
       // every lane polls; the vote over all four epilogue warps re-converges
       // them before the warp-collective (.sync.aligned) TMEM loads and makes
       // the give-up decision uniform (the warps share named barriers below)
@@ -354,7 +355,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      if (SPLIT > 1) break;  // the split-K reduction below finishes this tile
+      if (split > 1) break;  // the split-K reduction below finishes this tile
       const Tile tl = decode_tile(args, tab0, t);
       int64_t drow;
       bool valid;
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_row_to_bf16<BN>(t_row, packed);
         tc_fence_before();
         mbar_arrive(acce_bar(acc));
-        store_rows_tma<BN>(packed, r_local, sbase + L::OFF_STG, stg_count, &tmap_d, tl.n_blk * BN, tl.m_blk * BM,
+        store_rows_tma<BN>(packed, r_local, sbase + L::OFF_STG, stg_count, tmap_d, tl.n_blk * BN, tl.m_blk * BM,
                            args.mode == kMasked ? tl.group : 0);
       } else {
         __nv_bfloat16* drow_ptr = args.d + drow * args.n;
@@ -413,7 +414,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (threadIdx.x == 64) bulk_wait_group_all();
   }
 
-  if constexpr (SPLIT > 1) {
+  if (SPLIT_MAX > 1 && split > 1) {
     // ---------------------------------------------------------- split-K reduction
     // 1) every CTA of the cluster is past its mainloop, so every operand ring
     //    is free to receive partials; 2) each CTA sends column slice j of its
@@ -455,7 +456,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
       for (int q = q_begin; q < q_end; ++q) {
         float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = 0; src < SPLIT; ++src) {
+        for (int src = 0; src < SPLIT_MAX; ++src) {
           const float4 x = *reinterpret_cast<const float4*>(
               red + ((src * L::MAX_SLICE_QUADS + (q - q_begin)) * BM + r_local) * 4);
           sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
@@ -479,6 +480,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_dealloc(tmem_base, L::TMEM_COLS);
   }
   if (threadIdx.x == 0 && *abort_flag) linger_after_abort();
+}
+
+template <int BN, int STAGES, int ACC, int SPLIT, int BMA>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ CUtensorMap tmap_d, const GemmArgs args) {
+  // persistent over the problem's tiles, or (SPLIT > 1) one cluster of SPLIT
+  // CTAs per tile
+  const int split_rank = SPLIT > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT : static_cast<int>(blockIdx.x);
+  const int kt_begin = SPLIT > 1 ? split_rank * args.k_tiles / SPLIT : 0;
+  const int kt_end = SPLIT > 1 ? (split_rank + 1) * args.k_tiles / SPLIT : args.k_tiles;
+  gemm_cta<BN, STAGES, ACC, SPLIT, BMA>(&tmap_a, &tmap_b, &tmap_d, args, SPLIT, split_rank, t_first,
+                                        static_cast<int>(gridDim.x), kt_begin, kt_end);
 }
 
 // ======================================================================= host
@@ -710,6 +725,249 @@ cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, 
     case kCfgSplit6: return launch_gemm_cfg<128, 6, 1, 6>(p, num_sms, stream, launches);
     case kCfgSplit8: return launch_gemm_cfg<128, 6, 1, 8>(p, num_sms, stream, launches);
     default: return launch_gemm_cfg<256, 4, 1, 1>(p, num_sms, stream, launches);
+  }
+}
+
+// ======================================================================= batch
+
+// Independent dense problems in ONE launch.  Each CTA belongs to one problem
+// (problem p owns CTAs [cta0[p], cta0[p+1]), a whole number of clusters) and
+// runs the one-CTA kernel's body on it with 128 x BN tiles (BN = 128: six
+// stages and two accumulators; BN = 256: four stages, one accumulator, half
+// the re-reads of A): persistently over the problem's tiles, or with K split
+// over the CS CTAs of each of its clusters (one tile per cluster, partials
+// reduced through distributed shared memory).  The host sizes every
+// problem's share of the GPU so that all of them finish at about the same
+// time: small problems stream their operands on all SMs at once instead of
+// one after another.
+template <int BN>
+struct BatchCfg {
+  static constexpr int STAGES = BN == 128 ? 6 : 4;
+  static constexpr int ACC = BN == 128 ? 2 : 1;
+};
+
+struct BatchMaps {
+  CUtensorMap a[kMaxBatch];
+  CUtensorMap b[kMaxBatch];
+  CUtensorMap d[kMaxBatch];
+};
+
+struct BatchArgs {
+  GemmArgs args[kMaxBatch];
+  int cta0[kMaxBatch + 1];
+  int split[kMaxBatch];  // 1, or CS: the CTAs of a cluster share one tile
+  int count;
+};
+
+template <int BN, int CS>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    mx_gemm_batch_kernel(const __grid_constant__ BatchMaps maps, const __grid_constant__ BatchArgs bat) {
+  const int cta = static_cast<int>(blockIdx.x);
+  int p = 0;
+  while (p + 1 < bat.count && cta >= bat.cta0[p + 1]) ++p;
+  const GemmArgs& args = bat.args[p];
+  const int local = cta - bat.cta0[p];
+  const int ctas = bat.cta0[p + 1] - bat.cta0[p];
+  const int split = bat.split[p];
+  const int split_rank = split > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int kt_begin = split > 1 ? split_rank * args.k_tiles / split : 0;
+  const int kt_end = split > 1 ? (split_rank + 1) * args.k_tiles / split : args.k_tiles;
+  gemm_cta<BN, BatchCfg<BN>::STAGES, BatchCfg<BN>::ACC, CS, BM>(&maps.a[p], &maps.b[p], &maps.d[p], args, split,
+                                                                 split_rank, local / split, ctas / split, kt_begin,
+                                                                 kt_end);
+}
+
+template <int BN, int CS>
+using BatchLayout = Layout<BN, BatchCfg<BN>::STAGES, BatchCfg<BN>::ACC, CS, BM>;
+
+template <int BN, int CS>
+static cudaError_t prepare_batch_kernel() {
+  static cudaError_t state = cudaErrorNotReady;
+  if (state == cudaErrorNotReady)
+    state = cudaFuncSetAttribute(mx_gemm_batch_kernel<BN, CS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 BatchLayout<BN, CS>::ALLOC);
+  return state;
+}
+
+// Clusters of CS CTAs the GPU holds at once (0 if unknown).
+template <int BN, int CS>
+static int batch_max_clusters() {
+  static int v = -1;
+  if (v < 0) {
+    v = 0;
+    if (prepare_batch_kernel<BN, CS>() == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      cfg.gridDim = dim3(CS, 1, 1);
+      cfg.blockDim = dim3(kGemmThreads, 1, 1);
+      cfg.dynamicSmemBytes = BatchLayout<BN, CS>::ALLOC;
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = CS;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, mx_gemm_batch_kernel<BN, CS>, &cfg) == cudaSuccess) v = n;
+      cudaGetLastError();
+    }
+  }
+  return v;
+}
+
+// Share of the GPU for each problem: a time model (a CTA of this kernel
+// streams its operands at ~62 GB/s with 128-wide tiles and ~52 GB/s with
+// 256-wide ones, fitted to the page shapes' batch; a tile costs ~0.5 us
+// more, a split-K exchange ~3 us).  Every problem gets a cluster, then each further
+// cluster goes to the problem that would finish last, with the better of
+// "no split" and "split K over the cluster" for its share.
+struct BatchPlan {
+  int ctas[kMaxBatch];
+  int split[kMaxBatch];
+  double time;
+};
+
+static double batch_time(int64_t tiles, double tile_bytes, int64_t k_tiles, int ctas, int bn, int cs, int* split) {
+  const double rate = bn == 128 ? 6.2e10 : 5.2e10, per_tile = 0.5e-6, exchange = 3.0e-6;
+  const int64_t groups1 = ctas;
+  double best = static_cast<double>((tiles + groups1 - 1) / groups1) * (tile_bytes / rate + per_tile);
+  *split = 1;
+  const int64_t groups_s = ctas / cs;
+  if (cs > 1 && k_tiles >= cs && groups_s >= tiles) {  // one tile per cluster
+    const double t = tile_bytes / cs / rate + per_tile + exchange;
+    if (t < best) {
+      best = t;
+      *split = cs;
+    }
+  }
+  return best;
+}
+
+static BatchPlan plan_batch(const GemmProblem* ps, int count, int bn, int cs, int clusters) {
+  BatchPlan pl = {};
+  int64_t tiles[kMaxBatch];
+  double tile_bytes[kMaxBatch];
+  double t[kMaxBatch];
+  int left = clusters;
+  for (int i = 0; i < count; ++i) {
+    tiles[i] = ((ps[i].m + BM - 1) / BM) * ((ps[i].n + bn - 1) / bn);
+    const int64_t a_rows = ps[i].m < BM ? (ps[i].m <= 32 ? 32 : ps[i].m <= 64 ? 64 : BM) : BM;
+    tile_bytes[i] = static_cast<double>((a_rows + bn) * ps[i].k) * (1.0 + 1.0 / 32.0);
+    pl.ctas[i] = cs;
+    --left;
+    t[i] = batch_time(tiles[i], tile_bytes[i], ps[i].k / BK, pl.ctas[i], bn, cs, &pl.split[i]);
+  }
+  while (left > 0) {
+    int worst = -1;
+    for (int i = 0; i < count; ++i) {
+      const bool useful = pl.ctas[i] < tiles[i] * cs;  // more CTAs than tiles x cluster size cannot help
+      if (useful && (worst < 0 || t[i] > t[worst])) worst = i;
+    }
+    if (worst < 0) break;
+    pl.ctas[worst] += cs;
+    --left;
+    t[worst] =
+        batch_time(tiles[worst], tile_bytes[worst], ps[worst].k / BK, pl.ctas[worst], bn, cs, &pl.split[worst]);
+  }
+  pl.time = 0.0;
+  for (int i = 0; i < count; ++i) pl.time = t[i] > pl.time ? t[i] : pl.time;
+  return pl;
+}
+
+template <int BN, int CS>
+static cudaError_t launch_batch_cs(const GemmProblem* ps, int count, const BatchPlan& pl, cudaStream_t stream,
+                                   int* launches) {
+  using L = BatchLayout<BN, CS>;
+  {
+    cudaError_t e = prepare_batch_kernel<BN, CS>();
+    if (e != cudaSuccess) return e;
+  }
+  BatchMaps maps;
+  BatchArgs bat = {};
+  bat.count = count;
+  int cta = 0;
+  for (int i = 0; i < count; ++i) {
+    const GemmProblem& p = ps[i];
+    const int a_box_rows = p.m <= 32 ? 32 : p.m <= 64 ? 64 : BM;
+    if (!make_tmap(&maps.a[i], p.qa, p.k, p.m, 1, a_box_rows)) return cudaErrorInvalidValue;
+    if (!make_tmap(&maps.b[i], p.qb, p.k, p.n, 1, BN)) return cudaErrorInvalidValue;
+    if (!make_tmap_d(&maps.d[i], p.d, p.n, p.m, 1)) return cudaErrorInvalidValue;
+    GemmArgs& a = bat.args[i];
+    a.sfa = static_cast<const uint8_t*>(p.sfa);
+    a.sfb = static_cast<const uint8_t*>(p.sfb);
+    a.d = static_cast<__nv_bfloat16*>(p.d);
+    a.status = p.status;
+    a.wait_ns = wait_limit_ns();
+    a.k_tiles = static_cast<int>(p.k / BK);
+    a.sfa_group_bytes = ((p.m + 127) / 128) * 128 * (p.k / 32);
+    a.sfb_group_bytes = ((p.n + 127) / 128) * 128 * (p.k / 32);
+    a.m = static_cast<int>(p.m);
+    a.n = static_cast<int>(p.n);
+    a.n_tiles = static_cast<int>((p.n + BN - 1) / BN);
+    a.n_sf_tiles = static_cast<int>((p.n + 127) / 128);
+    a.groups = 1;
+    a.mode = kDense;
+    a.a_box_rows = a_box_rows;
+    bat.cta0[i] = cta;
+    bat.split[i] = pl.split[i];
+    cta += pl.ctas[i];
+  }
+  bat.cta0[count] = cta;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  cfg.gridDim = dim3(static_cast<unsigned>(cta), 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::ALLOC;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mx_gemm_batch_kernel<BN, CS>, maps, bat);
+  if (e != cudaSuccess) return e;
+  if (launches) *launches += 1;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_batch(const GemmProblem* ps_in, int count, int num_sms, cudaStream_t stream, int* launches) {
+  (void)num_sms;
+  if (count < 0 || count > kMaxBatch) return cudaErrorInvalidValue;
+  GemmProblem ps[kMaxBatch];
+  int n = 0;
+  for (int i = 0; i < count; ++i)  // empty problems take no CTAs
+    if (ps_in[i].m > 0 && ps_in[i].n > 0 && ps_in[i].k > 0) ps[n++] = ps_in[i];
+  if (n == 0) return cudaSuccess;
+  static int forced_cs = -2, forced_bn = -2;  // tuning overrides: cluster size 2 or 4, tile width 128 or 256
+  if (forced_cs == -2) {
+    const char* env = getenv("MX_BATCH_CLUSTER");
+    forced_cs = env ? atoi(env) : -1;
+    env = getenv("MX_BATCH_BN");
+    forced_bn = env ? atoi(env) : -1;
+  }
+  // candidate (tile width, cluster size) forms; the one the model finishes first
+  const int cl[4] = {batch_max_clusters<128, 2>(), batch_max_clusters<128, 4>(), batch_max_clusters<256, 2>(),
+                     batch_max_clusters<256, 4>()};
+  const int bns[4] = {128, 128, 256, 256}, css[4] = {2, 4, 2, 4};
+  int best = -1;
+  BatchPlan plans[4];
+  for (int c = 0; c < 4; ++c) {
+    if (cl[c] < n) continue;
+    if ((forced_cs == 2 || forced_cs == 4) && css[c] != forced_cs) continue;
+    if ((forced_bn == 128 || forced_bn == 256) && bns[c] != forced_bn) continue;
+    plans[c] = plan_batch(ps, n, bns[c], css[c], cl[c]);
+    if (best < 0 || plans[c].time < plans[best].time) best = c;
+  }
+  switch (best) {
+    case 0: return launch_batch_cs<128, 2>(ps, n, plans[0], stream, launches);
+    case 1: return launch_batch_cs<128, 4>(ps, n, plans[1], stream, launches);
+    case 2: return launch_batch_cs<256, 2>(ps, n, plans[2], stream, launches);
+    case 3: return launch_batch_cs<256, 4>(ps, n, plans[3], stream, launches);
+    default: return cudaErrorInvalidConfiguration;
   }
 }
 

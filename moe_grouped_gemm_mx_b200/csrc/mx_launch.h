@@ -48,6 +48,11 @@ struct GemmProblem {
 
 cudaError_t launch_gemm(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches);
 
+// Up to kMaxBatch independent dense problems (mode 0) in one launch, the
+// GPU shared among them (mx_gemm.cu).  Empty problems are skipped.
+constexpr int kMaxBatch = 4;
+cudaError_t launch_gemm_batch(const GemmProblem* ps, int count, int num_sms, cudaStream_t stream, int* launches);
+
 // CTA-pair (2-SM MMA) kernel for large problems, any of the three forms.
 cudaError_t launch_gemm_pair(const GemmProblem& p, int num_sms, cudaStream_t stream, int* launches);
 

@@ -273,3 +273,36 @@ def test_wait_limit_setter(lib):
     assert lib.mx_wait_limit_ns() == 1000
     assert lib.mx_set_wait_limit_ns(0) == MX_OK
     assert lib.mx_wait_limit_ns() == 2_000_000_000
+
+
+class _Prob(ctypes.Structure):
+    _fields_ = [("qa", ctypes.c_void_p), ("sfa", ctypes.c_void_p), ("qb", ctypes.c_void_p),
+                ("sfb", ctypes.c_void_p), ("d_bf16", ctypes.c_void_p), ("m", ctypes.c_int64),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64)]
+
+
+def test_gemm_batch_argument_checks(lib):
+    """mx_gemm_batch: 1..4 problems, each with mx_gemm's rules; every problem
+    is checked before anything is launched; an all-empty batch is a no-op
+    (no GPU needed for any of these)."""
+    f = lib.mx_gemm_batch
+    f.argtypes = [ctypes.POINTER(_Prob), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+    A, B, C, D, E = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+    good = _Prob(A, B, C, D, E, 64, 256, 512)
+    arr = (_Prob * 5)(*([good] * 5))
+    assert f(arr, 0, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert f(arr, 5, None, None) == MX_ERR_INVALID_ARGUMENT
+    assert f(None, 1, None, None) == MX_ERR_INVALID_ARGUMENT
+    bad = (_Prob * 2)(good, _Prob(A, B, C, D, E, 64, 256, 500))           # second problem: k % 128
+    assert f(bad, 2, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    bad = (_Prob * 2)(good, _Prob(A, B, C, D, E, 64, 250, 512))           # n % 16
+    assert f(bad, 2, None, None) == MX_ERR_UNSUPPORTED_SHAPE
+    bad = (_Prob * 2)(good, _Prob(A + 8, B, C, D, E, 64, 256, 512))       # misaligned A
+    assert f(bad, 2, None, None) == MX_ERR_MISALIGNED
+    bad = (_Prob * 2)(good, _Prob(None, B, C, D, E, 64, 256, 512))        # null A
+    assert f(bad, 2, None, None) == MX_ERR_INVALID_ARGUMENT
+    bad = (_Prob * 1)(_Prob(A, B, C, D, E, -1, 256, 512))
+    assert f(bad, 1, None, None) == MX_ERR_INVALID_ARGUMENT
+    empty = (_Prob * 2)(_Prob(None, None, None, None, None, 0, 256, 512),
+                        _Prob(None, None, None, None, None, 64, 0, 512))
+    assert f(empty, 2, None, None) == MX_OK

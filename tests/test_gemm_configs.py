@@ -114,3 +114,45 @@ def test_forced_config_grouped(oracle, cfg):
             if mm[e]:
                 assert_gemm_close(got["masked"][e, :mm[e]].astype(np.float64), d2_ref[e, :mm[e]],
                                   abs2[e, :mm[e]], f"cfg {cfg} masked e={e}")
+
+
+CHILD_BATCH = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import moe_grouped_gemm_mx_b200 as mx, mx_inputs
+out = sys.argv[2]
+qs = []
+for (m, n, k) in %r:
+    a, b = mx_inputs.dense_problem(m, n, k, seed=m + n, kind="outlier")
+    qa, sfa = mx.mx_quantize_bf16_to_e4m3(a.cuda())
+    qb, sfb = mx.mx_quantize_bf16_to_e4m3(b.cuda())
+    qs.append((qa, sfa, qb, sfb))
+st = torch.zeros(1, dtype=torch.int32, device="cuda")
+ds = mx.mx_gemm_batch(qs, dev_status=st)
+torch.cuda.synchronize()
+assert int(st.item()) == 0, hex(int(st.item()))
+np.savez(out, **{f"{m}x{n}x{k}": d.float().cpu().numpy() for (m, n, k), d in zip(%r, ds)})
+""" % (SHAPES, SHAPES)
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("cluster", [2, 4])
+def test_batch_forced_cluster(oracle, cluster, bn):
+    """mx_gemm_batch over the four shapes above with its cluster size and tile
+    width forced (MX_BATCH_CLUSTER, MX_BATCH_BN, read once per process): the
+    planner's split-K over clusters of 2 or 4 and its persistent shares, with
+    128- and 256-wide tiles, against the oracle."""
+    with tempfile.TemporaryDirectory() as td:
+        out = os.path.join(td, "d.npz")
+        env = dict(os.environ, MX_BATCH_CLUSTER=str(cluster), MX_BATCH_BN=str(bn))
+        r = subprocess.run([sys.executable, "-c", CHILD_BATCH, ROOT, out], env=env, capture_output=True, text=True,
+                           timeout=300)
+        assert r.returncode == 0, r.stderr[-2000:]
+        got = np.load(out)
+        for (m, n, k) in SHAPES:
+            a, b = mx_inputs.dense_problem(m, n, k, seed=m + n, kind="outlier")
+            qa, sfa = oracle_quantize(oracle, a)
+            qb, sfb = oracle_quantize(oracle, b)
+            d_ref, absd = oracle.gemm(qa, sfa, qb, sfb)
+            assert_gemm_close(got[f"{m}x{n}x{k}"].astype(np.float64), d_ref, absd,
+                              f"batch cluster {cluster} bn {bn} {m}x{n}x{k}")

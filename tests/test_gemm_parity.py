@@ -103,6 +103,83 @@ def test_page_shapes_all_rows(mx, oracle, shape):
     check_dense(mx, oracle, a, b, what=f"page shape {shape}")
 
 
+def gpu_batch(mx, problems):
+    """D_i of mx_gemm_batch over BF16 (A_i, B_i) pairs, with the status word."""
+    dev = torch.device("cuda")
+    qs = []
+    for a, b in problems:
+        qa, sfa = mx.mx_quantize_bf16_to_e4m3(a.to(dev))
+        qb, sfb = mx.mx_quantize_bf16_to_e4m3(b.to(dev))
+        qs.append((qa, sfa, qb, sfb))
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    ds = mx.mx_gemm_batch(qs, dev_status=st)
+    torch.cuda.synchronize()
+    return ds, int(st.item())
+
+
+def test_page_shapes_batch_all_rows(mx, oracle):
+    """The three page shapes as one mx_gemm_batch launch (the GPU shared
+    among them, K split over clusters where the model says so): every row of
+    every problem against the oracle."""
+    probs = [mx_inputs.dense_problem(m, n, k, seed=0, kind="outlier") for (m, n, k) in mx_inputs.PAGE_SHAPES]
+    ds, st = gpu_batch(mx, probs)
+    assert st == 0
+    for (a, b), d, shape in zip(probs, ds, mx_inputs.PAGE_SHAPES):
+        qa, sfa = oracle_quantize(oracle, a)
+        qb, sfb = oracle_quantize(oracle, b)
+        d_ref, absd = oracle.gemm(qa, sfa, qb, sfb)
+        assert_gemm_close(to_np_f64(d), d_ref, absd, f"batch page shape {shape}")
+
+
+@pytest.mark.parametrize("shapes", [
+    [(1, 16, 128), (63, 144, 384), (200, 272, 1152), (129, 400, 256)],
+    [(17, 528, 2048), (64, 256, 128)],
+    [(300, 400, 256)],
+], ids=["four-ragged", "two", "one"])
+def test_batch_ragged(mx, oracle, shapes):
+    """Ragged batches: M of 1, 63, 129, 200, 300 rows, N not a multiple of
+    128, K of one 128-element tile (no split possible) to 2048; one problem
+    alone is mx_gemm's problem."""
+    probs = [mx_inputs.dense_problem(m, n, k, seed=m + n + k, kind="outlier") for (m, n, k) in shapes]
+    ds, st = gpu_batch(mx, probs)
+    assert st == 0
+    for (a, b), d, shape in zip(probs, ds, shapes):
+        qa, sfa = oracle_quantize(oracle, a)
+        qb, sfb = oracle_quantize(oracle, b)
+        d_ref, absd = oracle.gemm(qa, sfa, qb, sfb)
+        assert_gemm_close(to_np_f64(d), d_ref, absd, f"batch {shape}")
+
+
+def test_batch_with_empty_problem_and_sentinels(mx, oracle):
+    """An empty problem in the batch takes no work; the others' outputs are
+    written exactly in their [M, N] (sentinel rows around each untouched)."""
+    dev = torch.device("cuda")
+    shapes = [(64, 2112, 1024), (0, 256, 512), (128, 512, 768)]
+    qs, refs, bufs = [], [], []
+    for (m, n, k) in shapes:
+        a, b = mx_inputs.dense_problem(max(m, 1), n, k, seed=7 + n, kind="outlier")
+        a = a[:m]
+        qa, sfa = mx.mx_quantize_bf16_to_e4m3(a.to(dev)) if m else (torch.empty((0, k), dtype=torch.uint8, device=dev),
+                                                                  torch.zeros(16, dtype=torch.uint8, device=dev))
+        qb, sfb = mx.mx_quantize_bf16_to_e4m3(b.to(dev))
+        qs.append((qa, sfa, qb, sfb))
+        buf = sentinel_fill((m + 2, n))
+        bufs.append(buf)
+        refs.append((a, b))
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    mx.mx_gemm_batch(qs, outs=[bf[1:1 + m] for bf, (m, _, _) in zip(bufs, shapes)], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for (a, b), bf, (m, n, k) in zip(refs, bufs, shapes):
+        assert bool(is_sentinel(bf[0]).all()) and bool(is_sentinel(bf[m + 1]).all()), f"{(m, n, k)}: guard rows"
+        if m == 0:
+            continue
+        qa, sfa = oracle_quantize(oracle, a)
+        qb, sfb = oracle_quantize(oracle, b)
+        d_ref, absd = oracle.gemm(qa, sfa, qb, sfb)
+        assert_gemm_close(to_np_f64(bf[1:1 + m]), d_ref, absd, f"batch {(m, n, k)}")
+
+
 @pytest.mark.parametrize("nk", mx_inputs.LARGE_NK, ids=lambda s: "x".join(map(str, s)))
 def test_large_dense_sampled_rows(mx, oracle, nk):
     n, k = nk
