@@ -94,18 +94,38 @@ struct Layout {
   __host__ __device__ static constexpr int quad_owner(int q) { return (q * SPLIT) / QUADS; }
 };
 
-// One CTA of the GEMM: tiles t_first, t_first + t_stride, ... of the problem
-// in `args` (operands through the three tensor maps), or, with split > 1
-// (dense form only, split == SPLIT_MAX), the K tiles [kt_begin, kt_end) of
-// the single tile t_first, which the `split` CTAs of this cluster share: each
-// accumulates a contiguous share of K and the FP32 partials are reduced
-// through distributed shared memory.  Every CTA of a cluster has the same
-// split.
+// How the tiles of a problem are shared out.  Tiles [0, bulk) are whole-K
+// tiles dealt round robin: a CTA takes first, first + stride, ...  After
+// them, cluster `cluster` (of cs CTAs) shares at most one more tile, bulk +
+// cluster, each CTA accumulating the K tiles of its rank's share; the cluster
+// reduces those partials through distributed shared memory.  `bulk` is all
+// tiles (persistent CTAs) or none (one split tile per cluster).
+enum BulkMode : int { kBulkAll = 0, kBulkNone = 1 };
+
+struct CtaSchedule {
+  int first, stride, cluster, cs, rank, bulk, total, k_tiles;
+  __device__ __forceinline__ int split_tile() const {
+    return (cs > 1 && bulk + cluster < total) ? bulk + cluster : total;
+  }
+  __device__ __forceinline__ int begin() const { return first < bulk ? first : split_tile(); }
+  __device__ __forceinline__ int next(int t) const {
+    if (t >= bulk) return total;
+    return t + stride < bulk ? t + stride : split_tile();
+  }
+  __device__ __forceinline__ bool split(int t) const { return t >= bulk; }
+  __device__ __forceinline__ int kt_begin(int t) const { return t >= bulk ? rank * k_tiles / cs : 0; }
+  __device__ __forceinline__ int kt_end(int t) const { return t >= bulk ? (rank + 1) * k_tiles / cs : k_tiles; }
+};
+
+// One CTA of the GEMM on the problem in `args` (operands through the three
+// tensor maps): the tiles of its schedule (CtaSchedule; `bulk` from
+// bulk_mode once the tile count is known on the device).  Split tiles need
+// cs == SPLIT_MAX; every CTA of a cluster has the same schedule parameters.
 template <int BN, int STAGES, int ACC, int SPLIT_MAX, int BMA>
 __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtensorMap* tmap_b,
-                                         const CUtensorMap* tmap_d, const GemmArgs& args, const int split,
-                                         const int split_rank, const int t_first, const int t_stride,
-                                         const int kt_begin, const int kt_end) {
+                                         const CUtensorMap* tmap_d, const GemmArgs& args, const int bulk_mode,
+                                         const int first, const int stride, const int cluster, const int cs,
+                                         const int rank) {
   using L = Layout<BN, STAGES, ACC, SPLIT_MAX, BMA>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -219,6 +239,17 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = *total_slot;
+  CtaSchedule sch;
+  sch.first = first;
+  sch.stride = stride;
+  sch.cluster = cluster;
+  sch.cs = cs;
+  sch.rank = rank;
+  sch.total = total;
+  sch.k_tiles = args.k_tiles;
+  sch.bulk = bulk_mode == kBulkNone ? 0 : total;
+
+  int red_acc = 0;  // epilogue threads: the accumulator holding this CTA's split tile
 
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
@@ -228,7 +259,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int t = t_first; t < total && ok; t = split > 1 ? total : t + t_stride) {
+      for (int t = sch.begin(); t < total && ok; t = sch.next(t)) {
         const Tile tl = decode_tile(args, tab0, t);
         const int a_row = tl.m_blk * BM;
         const int a_z = (args.mode == kMasked) ? tl.group : 0;
@@ -239,6 +270,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
         const int sfb_tile0 = tl.n_blk * L::SFB_TILES;
         int nsfb = args.n_sf_tiles - sfb_tile0;
         nsfb = nsfb > L::SFB_TILES ? L::SFB_TILES : nsfb;
+        const int kt_begin = sch.kt_begin(t), kt_end = sch.kt_end(t);
         for (int kt = kt_begin; kt < kt_end; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
           // only the A rows that exist are loaded when M is small; the MMA's
@@ -272,10 +304,11 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = t_first; t < total && ok; t = split > 1 ? total : t + t_stride) {
+      for (int t = sch.begin(); t < total && ok; t = sch.next(t)) {
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_t = tmem_base + acc * BN;
+        const int kt_begin = sch.kt_begin(t), kt_end = sch.kt_end(t);
         for (int kt = kt_begin; kt < kt_end; ++kt) {
           // the copier's commit implies the stage's operands have landed too
           if (!mbar_wait(sfready_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
@@ -315,8 +348,8 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = t_first; t < total && ok; t = split > 1 ? total : t + t_stride) {
-        for (int kt = kt_begin; kt < kt_end; ++kt) {
+      for (int t = sch.begin(); t < total && ok; t = sch.next(t)) {
+        for (int kt = sch.kt_begin(t); kt < sch.kt_end(t); ++kt) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sfa_t = tmem_base + L::SF_COL0 + stage * L::SF_COLS;
@@ -344,7 +377,7 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t stg_count = 0;  // staging chunks used so far (buffer = count & 1)
-    for (int t = t_first; t < total; t = split > 1 ? total : t + t_stride) {
+    for (int t = sch.begin(); t < total; t = sch.next(t)) {
       // every lane polls; the vote over all four epilogue warps re-converges
       // them before the warp-collective (.sync.aligned) TMEM loads and makes
       // the give-up decision uniform (the warps share named barriers below)
@@ -355,7 +388,10 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
         break;
       }
       tc_fence_after();
-      if (split > 1) break;  // the split-K reduction below finishes this tile
+      if (sch.split(t)) {  // the split-K reduction below finishes this tile
+        red_acc = acc;
+        break;
+      }
       const Tile tl = decode_tile(args, tab0, t);
       int64_t drow;
       bool valid;
@@ -414,22 +450,28 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
     if (threadIdx.x == 64) bulk_wait_group_all();
   }
 
-  if (SPLIT_MAX > 1 && split > 1) {
+  const int split_t = sch.split_tile();
+  if (SPLIT_MAX > 1 && split_t < total) {
     // ---------------------------------------------------------- split-K reduction
+    // (the cluster's split tile; uniform over the cluster, cs == SPLIT_MAX)
     // 1) every CTA of the cluster is past its mainloop, so every operand ring
     //    is free to receive partials; 2) each CTA sends column slice j of its
-    //    FP32 partial to CTA j; 3) each CTA sums the SPLIT partials of its
+    //    FP32 partial to CTA j; 3) each CTA sums the SPLIT_MAX partials of its
     //    slice in rank order (deterministic) and stores BF16.
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
     const int quarter = warp & 3;
     const int r_local = quarter * 32 + lane;
-    const Tile tl = decode_tile(args, tab0, t_first);
+    const Tile tl = decode_tile(args, tab0, split_t);
     const int row = tl.m_blk * BM + r_local;
-    const bool valid = row < args.m && !*abort_flag;
-    if (warp >= 2 && warp <= 5 && t_first < total) {
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    // D row of this accumulator row, and whether it is stored (masked form:
+    // rows at or beyond the expert's masked_m are not)
+    const bool is_masked = args.mode == kMasked;
+    const int64_t drow = is_masked ? static_cast<int64_t>(tl.group) * args.m + row : row;
+    const bool valid = (is_masked ? row < tab1[tl.group] : row < args.m) && !*abort_flag;
+    if (warp >= 2 && warp <= 5) {
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + red_acc * BN;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
@@ -441,18 +483,18 @@ __device__ __forceinline__ void gemm_cta(const CUtensorMap* tmap_a, const CUtens
             const int q = c * 8 + q4;
             const int owner = L::quad_owner(q);
             const int cin = (q - L::slice_start(owner)) * 4;
-            const uint32_t local = sbase + ((split_rank * L::MAX_SLICE_QUADS + cin / 4) * BM + r_local) * 16;
+            const uint32_t local = sbase + ((rank * L::MAX_SLICE_QUADS + cin / 4) * BM + r_local) * 16;
             st_cluster_v4(map_to_rank(local, owner), v[q4 * 4 + 0], v[q4 * 4 + 1], v[q4 * 4 + 2], v[q4 * 4 + 3]);
           }
         }
       }
     }
     cluster_sync();
-    if (warp >= 2 && warp <= 5 && t_first < total && valid) {
+    if (warp >= 2 && warp <= 5 && valid) {
       const float* red = reinterpret_cast<const float*>(smem);
-      __nv_bfloat16* drow_ptr = args.d + static_cast<int64_t>(row) * args.n;
-      const int q_begin = L::slice_start(split_rank);
-      const int q_end = L::slice_start(split_rank + 1);
+      __nv_bfloat16* drow_ptr = args.d + drow * args.n;
+      const int q_begin = L::slice_start(rank);
+      const int q_end = L::slice_start(rank + 1);
 #pragma unroll 1
       for (int q = q_begin; q < q_end; ++q) {
         float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -488,12 +530,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const __grid_constant__ CUtensorMap tmap_d, const GemmArgs args) {
   // persistent over the problem's tiles, or (SPLIT > 1) one cluster of SPLIT
   // CTAs per tile
-  const int split_rank = SPLIT > 1 ? static_cast<int>(cluster_ctarank()) : 0;
-  const int t_first = SPLIT > 1 ? static_cast<int>(blockIdx.x) / SPLIT : static_cast<int>(blockIdx.x);
-  const int kt_begin = SPLIT > 1 ? split_rank * args.k_tiles / SPLIT : 0;
-  const int kt_end = SPLIT > 1 ? (split_rank + 1) * args.k_tiles / SPLIT : args.k_tiles;
-  gemm_cta<BN, STAGES, ACC, SPLIT, BMA>(&tmap_a, &tmap_b, &tmap_d, args, SPLIT, split_rank, t_first,
-                                        static_cast<int>(gridDim.x), kt_begin, kt_end);
+  const int cta = static_cast<int>(blockIdx.x);
+  const int rank = SPLIT > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  gemm_cta<BN, STAGES, ACC, SPLIT, BMA>(&tmap_a, &tmap_b, &tmap_d, args, SPLIT > 1 ? kBulkNone : kBulkAll, cta,
+                                        static_cast<int>(gridDim.x), cta / SPLIT, SPLIT, rank);
 }
 
 // ======================================================================= host
@@ -769,12 +809,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int local = cta - bat.cta0[p];
   const int ctas = bat.cta0[p + 1] - bat.cta0[p];
   const int split = bat.split[p];
-  const int split_rank = split > 1 ? static_cast<int>(cluster_ctarank()) : 0;
-  const int kt_begin = split > 1 ? split_rank * args.k_tiles / split : 0;
-  const int kt_end = split > 1 ? (split_rank + 1) * args.k_tiles / split : args.k_tiles;
-  gemm_cta<BN, BatchCfg<BN>::STAGES, BatchCfg<BN>::ACC, CS, BM>(&maps.a[p], &maps.b[p], &maps.d[p], args, split,
-                                                                 split_rank, local / split, ctas / split, kt_begin,
-                                                                 kt_end);
+  const int rank = split > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  gemm_cta<BN, BatchCfg<BN>::STAGES, BatchCfg<BN>::ACC, CS, BM>(&maps.a[p], &maps.b[p], &maps.d[p], args,
+                                                                 split > 1 ? kBulkNone : kBulkAll, local, ctas,
+                                                                 local / split, split, rank);
 }
 
 template <int BN, int CS>
