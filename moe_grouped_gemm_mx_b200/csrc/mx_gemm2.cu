@@ -9,15 +9,19 @@
 // 128 x 256 tile needs for the same math, which lowers the operand feed each
 // SM must sustain -- the limit of the one-CTA kernel on large problems.
 //
-//   warp 0 (both CTAs)   TMA producer: own A half, own B half, the 512-byte
-//                        scale chunk of its own 128 A rows and the two chunks
-//                        of all 256 B rows (every CTA's MMA half needs all N
-//                        scales).  Every load completes on the LEADER's
-//                        full barrier; the leader announces both CTAs' bytes.
-//   warp 6 (leader)      scale chunks of each landed stage -> that stage's
-//                        TMEM scale buffer (tcgen05.cp, both CTAs), commit
-//                        to the stage's "scales ready" barrier.
-//   warp 1 (leader)      4 pair MMAs per K tile once its scales are ready,
+//   warp 0 (both CTAs)   TMA producer: the 512-byte scale chunk of its own
+//                        128 A rows and the two chunks of all 256 B rows
+//                        (every CTA's MMA half needs all N scales), then its
+//                        own A half and B half.  Every load completes on a
+//                        barrier of the LEADER (scales and operands on two
+//                        barriers per stage); the leader announces both
+//                        CTAs' bytes.
+//   warp 6 (leader)      scale chunks of each stage -> that stage's TMEM
+//                        scale buffer (tcgen05.cp, both CTAs) as soon as
+//                        they land, while the operands are still in flight;
+//                        commit to the stage's "scales ready" barrier.
+//   warp 1 (leader)      4 pair MMAs per K tile once its operands have landed
+//                        and its scales are ready,
 //                        commits multicast to both CTAs' "empty" /
 //                        "accumulator full" barriers.
 //   warps 2-5 (both)     epilogue of the CTA's own 128 accumulator rows
@@ -66,9 +70,9 @@ struct PairLayout {
   static constexpr int STG_BYTES = 128 * 32 * 2;
   static constexpr int OFF_STG = (OFF_SFB + STAGES * SFB_BYTES + 1023) / 1024 * 1024;
   static constexpr int OFF_BAR = OFF_STG + 2 * STG_BYTES;
-  // full / empty / scales-ready per stage, accf, acce, and the drain barriers
-  // of the MMA issuer and the scale copier
-  static constexpr int NUM_BARS = 3 * STAGES + 4;
+  // full (operands) / empty / scales-ready / scales-landed per stage, accf,
+  // acce, and the drain barriers of the MMA issuer and the scale copier
+  static constexpr int NUM_BARS = 4 * STAGES + 4;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB0 = OFF_MISC + 16;
   static constexpr int OFF_TAB1 = OFF_TAB0 + (kMaxGroups + 1) * 4;
@@ -161,6 +165,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t drain_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 2);
   const uint32_t sf_drain_bar = sbase + L::OFF_BAR + 8u * (2 * STAGES + 3);
   auto sfready_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (2 * STAGES + 4 + s); };
+  auto sffull_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (3 * STAGES + 4 + s); };
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -168,6 +173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(full_bar(s), 1);   // the leader's producer announces both CTAs' bytes
       mbar_init(empty_bar(s), 1);  // the leader's commit, multicast to both CTAs
       mbar_init(sfready_bar(s), 1);  // the leader's scale-copy commit (leader only)
+      mbar_init(sffull_bar(s), 1);   // the leader's producer announces both CTAs' scale bytes
     }
     mbar_init(accf_bar, 1);
     mbar_init(acce_bar, 8);        // one lane of each epilogue warp of both CTAs, after the warp's loads
@@ -267,13 +273,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
     if (lane == 0) {
-      // ===== TMA producer (both CTAs); every load completes on the leader's full barrier
+      // ===== TMA producer (both CTAs); every load completes on a barrier of
+      // the leader: the scale tiles on the stage's "scales landed" barrier,
+      // issued first, so that the copier moves them into TMEM while the
+      // operands are still in flight and the MMAs wait for the operands only
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       // the leader announces the bytes of both CTAs' loads for a stage (boxes
       // reaching past the tensor are zero-filled and still count in full)
-      const uint32_t bytes_pair = 2u * (L::A_BYTES + L::B_BYTES + L::SFA_BYTES + L::SFB_BYTES);
+      const uint32_t bytes_ab = 2u * (L::A_BYTES + L::B_BYTES);
+      const uint32_t bytes_sf = 2u * (L::SFA_BYTES + L::SFB_BYTES);
       for (int t = pair; t < total && ok; t += npairs) {
         const PairTile tl = decode_pair_tile(args, tab0, tab1, t);
         const int a_row = tl.row0 + 128 * static_cast<int>(rank);
@@ -295,18 +305,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
           const uint32_t fb = map_to_rank(full_bar(stage), 0);
-          if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), bytes_pair);
+          const uint32_t sb = map_to_rank(sffull_bar(stage), 0);
+          if (rank == 0) {
+            mbar_arrive_expect_tx(sffull_bar(stage), bytes_sf);
+            mbar_arrive_expect_tx(full_bar(stage), bytes_ab);
+          }
           const int kc = kc0 + ks * kPairKC;
-          tma_load_4d_pair(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, fb, 0, a_row, kc, a_z);
-          tma_load_4d_pair(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, fb, 0, b_row, kc, b_z);
-          tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, fb, 0, kc, sfa_blk);
+          tma_load_3d_pair(sbase + L::OFF_SFA + stage * L::SFA_BYTES, &tmap_sfa, sb, 0, kc, sfa_blk);
           if (SWIGLU) {  // gate and up scale blocks are i/128 blocks apart: two boxes of one block
-            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES, &tmap_sfb, fb, 0, kc, sfb_blk);
-            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES + kPairKC * 512, &tmap_sfb, fb, 0, kc,
+            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES, &tmap_sfb, sb, 0, kc, sfb_blk);
+            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES + kPairKC * 512, &tmap_sfb, sb, 0, kc,
                              sfb_blk + args.swiglu_i / 128);
           } else {
-            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES, &tmap_sfb, fb, 0, kc, sfb_blk);
+            tma_load_3d_pair(sbase + L::OFF_SFB + stage * L::SFB_BYTES, &tmap_sfb, sb, 0, kc, sfb_blk);
           }
+          tma_load_4d_pair(sbase + L::OFF_A + stage * L::A_BYTES, &tmap_a, fb, 0, a_row, kc, a_z);
+          tma_load_4d_pair(sbase + L::OFF_B + stage * L::B_BYTES, &tmap_b, fb, 0, b_row, kc, b_z);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -329,7 +343,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int chunks = tile_chunks(decode_pair_tile(args, tab0, tab1, t));
         const int k_stages = (chunks + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
-          // the copier's commit implies both CTAs' operands of the stage have landed
+          // both CTAs' operands of the stage have landed, and its scales are in TMEM
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           if (!mbar_wait(sfready_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
@@ -369,17 +384,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 6) {
     if (lane == 0 && rank == 0) {
-      // ===== scale copier (leader only): once both CTAs' stage s has landed,
-      // copy each CTA's scale chunks into its TMEM scale buffer s.  Buffer s
-      // is free again once the stage's MMAs completed, which both producers
-      // have seen (empty) before refilling the stage (full).
+      // ===== scale copier (leader only): once both CTAs' scale tiles of
+      // stage s have landed, copy each CTA's scale chunks into its TMEM scale
+      // buffer s.  Buffer s is free again once the stage's MMAs completed,
+      // which both producers have seen (empty) before refilling the stage.
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs) {
         const int k_stages = (tile_chunks(decode_pair_tile(args, tab0, tab1, t)) + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
+          if (!mbar_wait(sffull_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < kPairKC; ++c) {
