@@ -140,7 +140,8 @@ mx_status mx_gemm(const void *qa, const void *sfa, const void *qb, const void *s
  * stream their operands at once instead of one launch after another: each
  * gets a share of the SMs sized to its bytes, with K split across a cluster
  * where that shortens it.  Meant for problems too small to fill the GPU
- * alone; every problem uses 128 x 128 tiles.
+ * alone; every problem uses one-CTA tiles of 128 rows (128 or 256 columns,
+ * one width for the whole batch).
  *   problems  host array of `count` descriptors, read during the call;
  *   1 <= count <= MX_GEMM_BATCH_MAX (else MX_ERR_INVALID_ARGUMENT).
  * One status word for all problems (dev_status, nullable).
