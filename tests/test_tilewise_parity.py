@@ -180,6 +180,78 @@ def test_tilewise_quant_midpoints_and_tiny_scales(mx, oracle, blocks):
     check_quant(mx, oracle, big, blocks)
 
 
+def _near_boundary_counts(x: torch.Tensor, s: np.ndarray, blocks: bool):
+    """Elements of x whose approximate quotient RN(|x| * RN(1 / s)) lies within
+    8 FP32 grid steps of an E4M3 rounding boundary -- the ones whose code a
+    quotient a few ulp off would change: returns (how many, how many of those
+    are not exact quotients).  Counts coverage only; the codes themselves are
+    compared with the oracle."""
+    a = np.abs(x.float().numpy())
+    rows, k = a.shape
+    if blocks:
+        st = np.repeat(np.repeat(s, 128, axis=0)[:rows], 128, axis=1)
+    else:
+        st = np.repeat(s.T, 128, axis=1)
+    st = st.astype(np.float32)
+    ok = np.isfinite(st) & (st >= np.float32(2.0 ** -64))
+    r = np.float32(1.0) / st
+    q0 = (a.astype(np.float32) * r).astype(np.float32)
+    b = q0.view(np.uint32).astype(np.int64)
+    lo = np.maximum(b - 8, 0).astype(np.uint32).view(np.float32)
+    hi = (b + 8).astype(np.uint32).view(np.float32)
+
+    def code(v):
+        return torch.from_numpy(np.minimum(v, np.float32(448.0))).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    near = (code(lo) != code(hi)) & ok
+    inexact = near & (a.astype(np.float64) != q0.astype(np.float64) * st.astype(np.float64))
+    return int(near.sum()), int(inexact.sum())
+
+
+@pytest.mark.parametrize("blocks", [False, True])
+def test_tilewise_quant_near_rounding_boundaries(mx, oracle, blocks):
+    """Random tiles over many binades, large enough that thousands of
+    quotients x / s sit on or within a few ulp of an E4M3 rounding boundary
+    (exact ties against scales with short significands, and thousands of
+    inexact near-ties), bit-exact against the oracle."""
+    g = torch.Generator().manual_seed(91)
+    x = torch.randn(4096, 2048, generator=g) * torch.exp(torch.randn(4096, 1, generator=g) * 3.0)
+    x = x.to(torch.bfloat16)
+    _, rs = (oracle.tw_quantize_blocks if blocks else oracle.tw_quantize_rows)(x)
+    near, inexact = _near_boundary_counts(x, rs, blocks)
+    assert near >= 1000 and inexact >= 20, (near, inexact)
+    check_quant(mx, oracle, x, blocks)
+
+
+def _every_significand_pair() -> torch.Tensor:
+    """128 blocks of 128 x 128 BF16 values.  Block b's largest magnitude has
+    significand 1 + b/128 (element [0, 0], one binade above the rest); row i
+    of a block peaks at significand 1 + ((b + i) % 128)/128; every other
+    element takes each of the 128 BF16 significands at 0 to 12 binades below
+    its row's peak, with random signs.  So both kernels see every scale
+    significand (a scale RN(amax / 448) has one per amax significand), each
+    paired with every element significand across the E4M3 normal and
+    subnormal ranges of the quotient.  Every value is exact in BF16."""
+    g = np.random.default_rng(123)
+    blocks = []
+    sig = 1.0 + np.arange(128) / 128.0
+    for b in range(128):
+        blk = np.empty((128, 128), dtype=np.float64)
+        for i in range(128):
+            peak = sig[(b + i) % 128]
+            j = g.permutation(128)[:127]
+            d = g.integers(0, 13, 127)
+            blk[i, 1:] = sig[j] * np.exp2(-d - 1.0) * np.where(g.random(127) < 0.5, -1.0, 1.0)
+            blk[i, 0] = peak
+        blk[0, 0] = sig[b] * 2.0
+        blocks.append(blk * 2.0 ** (b % 7 - 3))
+    return torch.from_numpy(np.concatenate(blocks)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("blocks", [False, True])
+def test_tilewise_quant_every_significand_pair(mx, oracle, blocks):
+    check_quant(mx, oracle, _every_significand_pair(), blocks)
+
+
 # ---------------------------------------------------------------- split-K over a cluster
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
