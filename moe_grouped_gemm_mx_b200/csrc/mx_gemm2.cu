@@ -449,25 +449,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (lane == 0) mbar_arrive_cluster(acce_leader);
           continue;
         }
-        uint32_t qw[32];  // the row's 128 E4M3 bytes
-        uint32_t sfw = 0; // its 4 scale bytes (column blocks 4*n_blk .. 4*n_blk+3)
+        // H for the row's 128 columns first; the accumulator goes back to the
+        // MMA warp before the requantisation
+        float h[4][32];
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           uint32_t g[32], u[32];
           tc_ld_32x32b_x32(t_row + b * 32, g);
           tc_ld_32x32b_x32(t_row + 128 + b * 32, u);
           tc_wait_ld();
-          float h[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) h[j] = swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]));
-          uint32_t q8[8];
-          sfw |= quant_block32_f32(h, q8) << (8 * b);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) qw[b * 8 + i] = q8[i];
+          for (int j = 0; j < 32; ++j) h[b][j] = swiglu_f32(__uint_as_float(g[j]), __uint_as_float(u[j]));
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acce_leader);  // TMEM back to the leader's MMA warp before any store
+        uint32_t qw[32];  // the row's 128 E4M3 bytes
+        uint32_t sfw = 0; // its 4 scale bytes (column blocks 4*n_blk .. 4*n_blk+3)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          uint32_t q8[8];
+          sfw |= quant_block32_f32(h[b], q8) << (8 * b);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) qw[b * 8 + i] = q8[i];
+        }
         const int r = my_row0 + r_local;   // absolute row (dense, contiguous) or row within the expert (masked)
         const bool valid = r < tl.rows_end;
         // scales: the 4 bytes of this row for column blocks 4*n_blk..+3 are
