@@ -17,7 +17,7 @@
 //    tile (32 elements, four 16-byte loads per lane, all in flight before the
 //    arithmetic); HBM-bound.
 //  * blocks kernel (weights, [rows, k], scales [ceil(rows/128), k/128]): one
-//    512-thread CTA per 128 x 128 block, a half-warp per row segment, 32
+//    256-thread CTA per 128 x 128 block, a half-warp per row segment, 64
 //    elements per thread held in registers across the block-wide amax
 //    reduction.
 #include <cuda_bf16.h>
@@ -136,28 +136,30 @@ __global__ void __launch_bounds__(256) tw_quant_rows_kernel(const uint4* __restr
   for (int i = 0; i < 4; ++i) q[base + 4 * i] = nonfinite ? make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu) : tw_codes8(v[i], sc, r);
 }
 
-// Weights: one 512-thread CTA per 128 x 128 block; a half-warp reads one row's
-// 256 contiguous bytes per load, a warp 8 rows (4 loads per thread, all in
-// flight); block-wide amax through shared memory.
-__global__ void __launch_bounds__(512) tw_quant_blocks_kernel(const uint4* __restrict__ x, uint2* __restrict__ q,
+// Weights: one 256-thread CTA per 128 x 128 block; a half-warp reads one row's
+// 256 contiguous bytes per load, a warp 16 rows (8 loads per thread, all in
+// flight); block-wide amax through shared memory.  At 62 registers four CTAs
+// fit on an SM (three of the 512-thread form did), which shortens the last
+// partial wave of the small weight tensors.
+__global__ void __launch_bounds__(256, 4) tw_quant_blocks_kernel(const uint4* __restrict__ x, uint2* __restrict__ q,
                                                                float* __restrict__ s, int rows, int ktiles) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ uint32_t warp_max[16];
+  __shared__ uint32_t warp_max[8];
   const int kt = blockIdx.x % ktiles;
   const int rb = blockIdx.x / ktiles;
   const int t = threadIdx.x;
   const int warp = t >> 5, lane = t & 31;
   const int hl = lane & 15;
   const int64_t k8 = static_cast<int64_t>(ktiles) * 16;  // row length in 8-element units
-  const int r0 = rb * 128 + warp * 8 + (lane >> 4);  // this thread's rows: r0, r0 + 2, r0 + 4, r0 + 6
+  const int r0 = rb * 128 + warp * 16 + (lane >> 4);  // this thread's rows: r0, r0 + 2, ..., r0 + 14
   const int64_t base = static_cast<int64_t>(r0) * k8 + kt * 16 + hl;
-  uint4 v[4];
+  uint4 v[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = r0 + 2 * i < rows ? x[base + 2 * i * k8] : make_uint4(0, 0, 0, 0);
+  for (int i = 0; i < 8; ++i) v[i] = r0 + 2 * i < rows ? x[base + 2 * i * k8] : make_uint4(0, 0, 0, 0);
   uint32_t m2 = 0;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) m2 = fold_amax(m2, v[i]);
+  for (int i = 0; i < 8; ++i) m2 = fold_amax(m2, v[i]);
   uint32_t m = max(m2 & 0xFFFFu, m2 >> 16) << 16;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -165,13 +167,13 @@ __global__ void __launch_bounds__(512) tw_quant_blocks_kernel(const uint4* __res
   __syncthreads();
   m = warp_max[0];
 #pragma unroll
-  for (int i = 1; i < 16; ++i) m = max(m, warp_max[i]);
+  for (int i = 1; i < 8; ++i) m = max(m, warp_max[i]);
   const bool nonfinite = m >= 0x7F800000u;
   const float sc = tw_scale(m);
   if (t == 0) s[static_cast<int64_t>(rb) * ktiles + kt] = sc;
   const float r = __frcp_rn(sc);
 #pragma unroll
-  for (int i = 0; i < 4; ++i)  // 8 elements -> 8 bytes at the same unit index
+  for (int i = 0; i < 8; ++i)  // 8 elements -> 8 bytes at the same unit index
     if (r0 + 2 * i < rows) q[base + 2 * i * k8] = nonfinite ? make_uint2(0x7F7F7F7Fu, 0x7F7F7F7Fu) : tw_codes8(v[i], sc, r);
 }
 
@@ -208,7 +210,7 @@ cudaError_t launch_tw_quant(const void* x, int64_t rows, int64_t k, void* q, flo
     const uint4* xp = static_cast<const uint4*>(x);
     uint2* qp = static_cast<uint2*>(q);
     void* args[] = {&xp, &qp, &s, &r, &kt};
-    e = launch_pdl(reinterpret_cast<const void*>(tw_quant_blocks_kernel), dim3(static_cast<unsigned>(grid)), dim3(512),
+    e = launch_pdl(reinterpret_cast<const void*>(tw_quant_blocks_kernel), dim3(static_cast<unsigned>(grid)), dim3(256),
                    args, stream);
   }
   if (e != cudaSuccess) return e;
