@@ -283,7 +283,11 @@ mx_status mx_grouped_gemm_masked_swiglu_quant(const void *qa, const void *sfa, c
  * elements 0x7F.  Scales are plain FP32 arrays:
  *   1 x 128:   scales [k/128, rows]          (K-tile major)
  *   128 x 128: scales [ceil(rows/128), k/128]
- * x [rows, k] BF16 16-byte aligned, q [rows, k]; requires k % 128 == 0.
+ * x [rows, k] BF16 16-byte aligned, q [rows, k], scales 4-byte aligned;
+ * requires k % 128 == 0 (else MX_ERR_UNSUPPORTED_SHAPE), rows and k at most
+ * 2^31 - 1 and fewer than 2^32 - 16 groups of 8 rows x 128 columns (else
+ * MX_ERR_UNSUPPORTED_SHAPE).  rows == 0 is a no-op.  Null pointers give
+ * MX_ERR_INVALID_ARGUMENT, misaligned ones MX_ERR_MISALIGNED.
  */
 mx_status mx_quantize_bf16_to_e4m3_tile1x128(const void *x_bf16, int64_t rows, int64_t k, void *q_e4m3,
                                              float *scales, mx_stream_t stream);

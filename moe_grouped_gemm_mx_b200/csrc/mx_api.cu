@@ -278,6 +278,8 @@ static mx_status tw_quantize(const void* x, int64_t rows, int64_t k, void* q, fl
   if (!x || !q || !s) return MX_ERR_INVALID_ARGUMENT;
   if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s) & 3u)) return MX_ERR_MISALIGNED;
   if (rows > kMaxDim || k > kMaxDim) return MX_ERR_UNSUPPORTED_SHAPE;
+  // the 1 x 128 kernel numbers its (8 rows x 128 columns) items in 32 bits
+  if ((rows + 7) / 8 * (k / 128) > 0xFFFFFFF0LL) return MX_ERR_UNSUPPORTED_SHAPE;
   return from_cuda(mxk::launch_tw_quant(x, rows, k, q, s, blocks, reinterpret_cast<cudaStream_t>(stream)));
 }
 

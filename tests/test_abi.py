@@ -180,6 +180,8 @@ def test_tilewise_argument_checks(lib):
         assert q(FAKE, 4, 128, FAKE, None, None) == MX_ERR_INVALID_ARGUMENT
         assert q(FAKE, 4, 128, FAKE, FAKE + 2, None) == MX_ERR_MISALIGNED
         assert q(None, 0, 128, None, None, None) == MX_OK
+        # more than 2^32 - 16 groups of 8 rows x 128 columns
+        assert q(FAKE, (1 << 31) - 1, 1 << 30, FAKE, FAKE, None) == MX_ERR_UNSUPPORTED_SHAPE
     g = lib.mx_gemm_tilewise
     assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 96, None, None) == MX_ERR_UNSUPPORTED_SHAPE
     assert g(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 24, 128, None, None) == MX_ERR_UNSUPPORTED_SHAPE
