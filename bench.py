@@ -168,11 +168,18 @@ def static_config(name: str, seed: int) -> dict:
 def run_config(args, world: int) -> dict:
     """The `config` object of the JSON line, identical in both arms: the
     workload, the operand format and how the GPU arm times it (L2 flushed
-    before every timed step, CUDA-graph replays unless --eager)."""
+    before every timed step, CUDA-graph replays unless --eager).  Under N
+    ranks every workload runs one independent problem per rank, except
+    moe_layer_ep, whose ranks share the experts and exchange tokens."""
+    if world <= 1:
+        par = "single GPU"
+    elif args.workload == "moe_layer_ep":
+        par = f"expert parallel x{world} ({'NCCL all-to-all' if args.ep == 'nccl' else 'peer memory'})"
+    else:
+        par = f"replicas x{world}"
     return dict(static_config(args.workload, args.seed), format=args.fmt,
                 l2="flushed (512 MiB write) before every timed step",
-                parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                graph=not args.eager)
+                parallelism=par, graph=not args.eager)
 
 
 def parse_args():
