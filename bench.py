@@ -82,7 +82,7 @@ def moe_counts(I, seed):
     return I.zipf_routing_counts(tokens=tokens, experts=experts, topk=min(I.MOE_TOPK, experts), seed=seed)
 
 
-def static_config(name: str, seed: int) -> dict:
+def static_config(name: str, seed: int, fmt: str = "mxfp8") -> dict:
     """Workload description shared by both arms (no GPU needed)."""
     import mx_inputs as I
     cfg = {"workload": name, "seed": seed}
@@ -159,6 +159,11 @@ def static_config(name: str, seed: int) -> dict:
     elif name == "page":
         cfg["step"] = ("quantise activations + weights of the three shapes (one batched launch), then their "
                        "three GEMMs in one mx_gemm_batch launch with BF16 epilogue")
+    elif name == "contiguous" and fmt == "mxfp8":
+        cfg["step"] = ("quantise the gate/up activations + weights (one batched launch), then the gate/up GEMM; "
+                       "the down activations + weights are quantised on a parallel stream by the lean form of the "
+                       "quantiser (no shared memory, one CTA per SM), which runs beside the quantisation and "
+                       "GEMM of the other stream; then the down GEMM, BF16 epilogues")
     else:
         cfg["step"] = ("quantise activations + weights (one batched launch), then the GEMM(s) "
                        "with BF16 epilogue")
@@ -177,7 +182,7 @@ def run_config(args, world: int) -> dict:
         par = f"expert parallel x{world} ({'NCCL all-to-all' if args.ep == 'nccl' else 'peer memory'})"
     else:
         par = f"replicas x{world}"
-    return dict(static_config(args.workload, args.seed), format=args.fmt,
+    return dict(static_config(args.workload, args.seed, args.fmt), format=args.fmt,
                 l2="flushed (512 MiB write) before every timed step",
                 parallelism=par, graph=not args.eager)
 
@@ -356,10 +361,12 @@ class Workload:
         self.config = {"workload": name}
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.quant_jobs = []
+        self.lean_jobs = []     # quantised by the lean form, on a branch of their own (see _finish)
         self.fmt = fmt
         # independent chains of launches (lists of indices into launches), run
         # on parallel streams / graph branches after the launches in none
         self.branches = None
+        self.after = []         # launches run after the branches have joined
         self._side = []
         # launches timed one by one for the per-kernel table but not part of
         # the step (a step whose launches cannot be replayed alone times its
@@ -374,30 +381,34 @@ class Workload:
         self._finish()
 
     # -- helpers
-    def _quant(self, x, label):
-        """Register x for the step's single batched quantisation launch."""
+    def _quant(self, x, label, lean=False):
+        """Register x for the step's batched quantisation launch (or, with
+        lean, for the lean-form launch)."""
         import torch
         mx = self.mx
         groups = 1 if x.dim() == 2 else x.shape[0]
         rows, k = x.shape[-2], x.shape[-1]
         q = torch.empty(x.shape, dtype=torch.uint8, device=self.dev)
         sf = torch.empty(groups * mx.scale_bytes(rows, k), dtype=torch.uint8, device=self.dev)
-        self.quant_jobs.append((x, q, sf, label))
+        (self.lean_jobs if lean else self.quant_jobs).append((x, q, sf, label))
         return q, sf
 
     def _finish(self):
         """All MXFP8 quantisations of the step go in one launch (up to 8
-        tensors), ahead of the GEMMs."""
-        if not self.quant_jobs:
-            return
+        tensors), ahead of the GEMMs; lean jobs go in a second launch of the
+        lean form, placed by the workload's branches."""
         mx = self.mx
-        xs = [j[0] for j in self.quant_jobs]
-        outs = [(j[1], j[2]) for j in self.quant_jobs]
-        nbytes = sum(x.numel() for x in xs) * QUANT_BYTES_PER_ELT
-        label = "+".join(j[3] for j in self.quant_jobs)
-        assert len(xs) <= 8
-        self.launches.insert(0, ("quant", label, lambda *xs_: mx.mx_quantize_bf16_to_e4m3_multi(list(xs_), outs),
-                                 nbytes, 0.0, tuple(xs)))
+        for jobs, lean in ((self.lean_jobs, True), (self.quant_jobs, False)):
+            if not jobs:
+                continue
+            xs = [j[0] for j in jobs]
+            outs = [(j[1], j[2]) for j in jobs]
+            nbytes = sum(x.numel() for x in xs) * QUANT_BYTES_PER_ELT
+            label = "+".join(j[3] for j in jobs) + (" (lean, beside the GEMM)" if lean else "")
+            assert len(xs) <= 8
+            self.launches.insert(0, ("quant", label, lambda *xs_, outs=outs, lean=lean:
+                                     mx.mx_quantize_bf16_to_e4m3_multi(list(xs_), outs, lean=lean),
+                                     nbytes, 0.0, tuple(xs)))
 
     def _add_input(self, t):
         import torch
@@ -525,12 +536,19 @@ class Workload:
                                       nbytes, fl, (qa, sa, qb, sb, off)))
                 self.flops += fl
                 continue
-            qa, sfa = self._quant(prob.a, tag + ":A")
-            qb, sfb = self._quant(prob.b, tag + ":B")
+            # the down GEMM's operands are quantised by the lean form beside
+            # the gate/up quantisation and GEMM (branches below)
+            qa, sfa = self._quant(prob.a, tag + ":A", lean=tag == "down")
+            qb, sfb = self._quant(prob.b, tag + ":B", lean=tag == "down")
             self.launches.append(("gemm", tag, lambda qa, sfa, qb, sfb, off, d=d:
                                   mx.mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, off, d=d, dev_status=self.status),
                                   self._gemm_bytes(m_total, n, k, experts), fl, (qa, sfa, qb, sfb, off)))
             self.flops += fl
+        if self.fmt == "mxfp8":
+            # launches after _finish: 0 quantise gate/up operands, 1 quantise down
+            # operands (lean form), 2 gate/up GEMM, 3 down GEMM
+            self.branches = [[0, 2], [1]]
+            self.after = [3]
         self.config.update({"experts": len(counts), "tokens": MOE_OVERRIDE["tokens"] or I.MOE_TOKENS, "topk": I.MOE_TOPK,
                             "zipf_s": I.MOE_ZIPF_S, "real_rows": real,
                             "padded_rows": int(I.padded_offsets(counts)[-1]),
@@ -874,7 +892,7 @@ class Workload:
         cur = torch.cuda.current_stream()
         in_branch = {i for br in self.branches for i in br}
         for i, (_, _, fn, _, _, inputs) in enumerate(self.launches):
-            if i not in in_branch:
+            if i not in in_branch and i not in self.after:
                 fn(*inputs)
         nside = len(self.branches) - 1
         while len(self._side) < nside:
@@ -888,6 +906,9 @@ class Workload:
                     fn(*inputs)
         for st in self._side[:nside]:
             cur.wait_stream(st)
+        for i in self.after:
+            _, _, fn, _, _, inputs = self.launches[i]
+            fn(*inputs)
 
 
 # ---------------------------------------------------------------- oracle (CPU) timing

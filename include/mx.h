@@ -118,6 +118,18 @@ typedef struct mx_quant_job {
 mx_status mx_quantize_bf16_to_e4m3_multi(const mx_quant_job *jobs, int32_t count, mx_stream_t stream);
 
 /*
+ * The same jobs, the same bytes out and the same argument checks as
+ * mx_quantize_bf16_to_e4m3_multi, from a form of the kernel that uses no
+ * shared memory and one CTA per SM.  It is meant to run concurrently with a
+ * GEMM launched on another stream: the GEMM's CTAs hold nearly all of each
+ * SM's shared memory, so the normal form cannot share an SM with them, and
+ * the quantisation (HBM-bound) then proceeds underneath the GEMM
+ * (tensor-bound) instead of before or after it.  Alone it is slower than the
+ * normal form.
+ */
+mx_status mx_quantize_bf16_to_e4m3_multi_lean(const mx_quant_job *jobs, int32_t count, mx_stream_t stream);
+
+/*
  * Dense MXFP8 GEMM, D = A * B^T ("DeepGEMM" summary page: the plain FP8
  * GEMM; the dense shapes of its CUTLASS comparison table).
  *   qa [m, k], sfa = scales of A (mx_scale_bytes(m, k));

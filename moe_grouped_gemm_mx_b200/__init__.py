@@ -45,7 +45,8 @@ MX_DEV_BAD_INDEX = 0x8
 # every symbol include/mx.h declares
 C_SYMBOLS = [
     "mx_status_string", "mx_scale_bytes", "mx_quantize_bf16_to_e4m3",
-    "mx_quantize_bf16_to_e4m3_grouped", "mx_quantize_bf16_to_e4m3_multi", "mx_gemm",
+    "mx_quantize_bf16_to_e4m3_grouped", "mx_quantize_bf16_to_e4m3_multi", "mx_quantize_bf16_to_e4m3_multi_lean",
+    "mx_gemm",
     "mx_grouped_gemm_contiguous",
     "mx_grouped_gemm_masked", "mx_read_internal_status", "mx_gemm_swiglu_quant",
     "mx_grouped_gemm_contiguous_swiglu_quant", "mx_grouped_gemm_masked_swiglu_quant",
@@ -93,6 +94,8 @@ def _load():
     L.mx_quantize_bf16_to_e4m3_grouped.restype = ctypes.c_int
     L.mx_quantize_bf16_to_e4m3_multi.argtypes = [ctypes.POINTER(_QuantJob), I32, P]
     L.mx_quantize_bf16_to_e4m3_multi.restype = ctypes.c_int
+    L.mx_quantize_bf16_to_e4m3_multi_lean.argtypes = [ctypes.POINTER(_QuantJob), I32, P]
+    L.mx_quantize_bf16_to_e4m3_multi_lean.restype = ctypes.c_int
     L.mx_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, P, P]
     L.mx_gemm.restype = ctypes.c_int
     L.mx_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, I32, I64, I64, I64, P, P, P]
@@ -210,10 +213,12 @@ def mx_quantize_bf16_to_e4m3(x: torch.Tensor, q: torch.Tensor | None = None,
     return q, sf
 
 
-def mx_quantize_bf16_to_e4m3_multi(xs, outs=None, stream=None):
+def mx_quantize_bf16_to_e4m3_multi(xs, outs=None, stream=None, lean=False):
     """Quantise several BF16 tensors ([rows, K] or [groups, rows, K]) in one
     kernel launch.  ``outs`` optionally gives a (q, sf) pair per tensor.
-    Returns the list of (q, sf)."""
+    ``lean`` selects mx_quantize_bf16_to_e4m3_multi_lean (the same bytes from
+    a form without shared memory, one CTA per SM, to run beside a GEMM on
+    another stream).  Returns the list of (q, sf)."""
     xs = list(xs)
     res = []
     jobs = (_QuantJob * max(1, len(xs)))()
@@ -234,7 +239,8 @@ def mx_quantize_bf16_to_e4m3_multi(xs, outs=None, stream=None):
             raise ValueError("output buffers too small")
         jobs[i] = _QuantJob(_ptr(x), groups, rows, k, _ptr(q), _ptr(sf))
         res.append((q, sf))
-    _raise(_lib.mx_quantize_bf16_to_e4m3_multi(jobs, len(xs), _stream(stream)), "mx_quantize_bf16_to_e4m3_multi")
+    name = "mx_quantize_bf16_to_e4m3_multi_lean" if lean else "mx_quantize_bf16_to_e4m3_multi"
+    _raise(getattr(_lib, name)(jobs, len(xs), _stream(stream)), name)
     return res
 
 

@@ -104,7 +104,7 @@ mx_status mx_quantize_bf16_to_e4m3_grouped(const void* x_bf16, int64_t groups, i
   return quantize_impl(x_bf16, groups, rows, k, q_e4m3, sf_ue8m0, stream);
 }
 
-mx_status mx_quantize_bf16_to_e4m3_multi(const mx_quant_job* jobs, int32_t count, mx_stream_t stream) {
+static mx_status quantize_multi(const mx_quant_job* jobs, int32_t count, mx_stream_t stream, bool lean) {
   if (count < 0 || (count > 0 && !jobs)) return MX_ERR_INVALID_ARGUMENT;
   // validate everything before launching anything
   int nonempty = 0;
@@ -126,16 +126,24 @@ mx_status mx_quantize_bf16_to_e4m3_multi(const mx_quant_job* jobs, int32_t count
     specs[n++] = mxk::QuantSpec{j.x_bf16, j.q_e4m3, j.sf_ue8m0, j.groups, j.rows, j.k,
                                 static_cast<int64_t>(mx_scale_bytes(j.rows, j.k))};
     if (n == mxk::kMaxQuantJobs) {
-      cudaError_t e = mxk::launch_quant_batch(specs, n, sms, reinterpret_cast<cudaStream_t>(stream), nullptr);
+      cudaError_t e = mxk::launch_quant_batch(specs, n, sms, reinterpret_cast<cudaStream_t>(stream), nullptr, lean);
       if (e != cudaSuccess) return MX_ERR_CUDA;
       n = 0;
     }
   }
   if (n > 0) {
-    cudaError_t e = mxk::launch_quant_batch(specs, n, sms, reinterpret_cast<cudaStream_t>(stream), nullptr);
+    cudaError_t e = mxk::launch_quant_batch(specs, n, sms, reinterpret_cast<cudaStream_t>(stream), nullptr, lean);
     if (e != cudaSuccess) return MX_ERR_CUDA;
   }
   return MX_OK;
+}
+
+mx_status mx_quantize_bf16_to_e4m3_multi(const mx_quant_job* jobs, int32_t count, mx_stream_t stream) {
+  return quantize_multi(jobs, count, stream, false);
+}
+
+mx_status mx_quantize_bf16_to_e4m3_multi_lean(const mx_quant_job* jobs, int32_t count, mx_stream_t stream) {
+  return quantize_multi(jobs, count, stream, true);
 }
 
 mx_status mx_quantize_bf16_to_e4m3_transposed(const void* x_bf16, int64_t groups, int64_t rows, int64_t cols,

@@ -75,8 +75,10 @@ struct PairLayout {
   static constexpr int NUM_BARS = 4 * STAGES + 4;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB0 = OFF_MISC + 16;
-  static constexpr int OFF_TAB1 = OFF_TAB0 + (kMaxGroups + 1) * 4;
-  static constexpr int BYTES = OFF_TAB1 + (kMaxGroups + 1) * 4;
+  // (the groups' offsets / masks are read from global memory where needed:
+  // a second table here would leave no room on the SM for another kernel's
+  // CTA without shared memory, e.g. a quantisation running underneath)
+  static constexpr int BYTES = OFF_TAB0 + (kMaxGroups + 1) * 4;
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM scale buffer of one stage: per K chunk [SFA 4 cols | SFB 8 cols]
@@ -95,8 +97,18 @@ struct PairTile {
   int n_blk;     // 256-wide column block
 };
 
-__device__ __forceinline__ PairTile decode_pair_tile(const GemmArgs& a, const int32_t* tab0, const int32_t* tab1,
-                                                     int t) {
+// Group i's row offset (contiguous), token offset (K-grouped; i in [0,
+// groups]) or valid rows clamped to [0, m] (masked; i < groups), from global
+// memory (read once per tile, cached).
+__device__ __forceinline__ int32_t group_val(const GemmArgs& a, int i) {
+  if (a.mode == kMasked) {
+    const int32_t mm = __ldg(a.masked_m + i);
+    return mm < 0 ? 0 : (mm > a.m ? a.m : mm);
+  }
+  return __ldg(a.group_offsets + i);
+}
+
+__device__ __forceinline__ PairTile decode_pair_tile(const GemmArgs& a, const int32_t* tab0, int t) {
   PairTile r;
   if (a.mode == kDense) {
     const int mb = t / a.n_tiles;
@@ -110,15 +122,15 @@ __device__ __forceinline__ PairTile decode_pair_tile(const GemmArgs& a, const in
     const int mb = local / a.n_tiles;
     r.group = e;
     r.n_blk = local - mb * a.n_tiles;
-    if (a.mode == kContiguous) {  // tab1: group offsets
-      r.row0 = tab1[e] + mb * kPairM;
-      r.rows_end = tab1[e + 1];
+    if (a.mode == kContiguous) {
+      r.row0 = group_val(a, e) + mb * kPairM;
+      r.rows_end = group_val(a, e + 1);
     } else if (a.mode == kKGrouped) {  // every expert has the full [m, n] output
       r.row0 = mb * kPairM;
       r.rows_end = a.m;
-    } else {  // tab1: clamped masked_m
+    } else {  // masked
       r.row0 = mb * kPairM;
-      r.rows_end = tab1[e];
+      r.rows_end = group_val(a, e);
     }
   }
   return r;
@@ -156,7 +168,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* total_slot = reinterpret_cast<volatile int*>(misc + 2);
   int32_t* tab0 = reinterpret_cast<int32_t*>(smem + L::OFF_TAB0);
-  int32_t* tab1 = reinterpret_cast<int32_t*>(smem + L::OFF_TAB1);
 
   auto full_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * s; };
   auto empty_bar = [&](int s) { return sbase + L::OFF_BAR + 8u * (STAGES + s); };
@@ -192,28 +203,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_launch_dependents();
   pdl_wait_prior();
 
-  // scheduling tables: tab1 = offsets (contiguous) / clamped masks (masked),
-  // tab0 = exclusive prefix of pair tiles per expert
+  // scheduling table: tab0 = exclusive prefix of pair tiles per expert,
+  // after checking the offsets (contiguous, K-grouped) or masks (masked)
   int bad = 0;
   if (args.mode != kDense) {
     if (args.mode == kContiguous || args.mode == kKGrouped) {
       // offsets along M (contiguous) or along K (K-grouped: the token ranges)
       const int limit = args.mode == kContiguous ? args.m : args.k_tiles * BK;
-      for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) tab1[i] = __ldg(args.group_offsets + i);
-      __syncthreads();
       for (int i = threadIdx.x; i <= args.groups; i += blockDim.x) {
-        const int32_t v = tab1[i];
+        const int32_t v = __ldg(args.group_offsets + i);
         if (v < 0 || (v % BM) != 0 || v > limit) bad = 1;
-        if (i > 0 && v < tab1[i - 1]) bad = 1;
+        if (i > 0 && v < __ldg(args.group_offsets + i - 1)) bad = 1;
       }
     } else {
       for (int i = threadIdx.x; i < args.groups; i += blockDim.x) {
-        int32_t mm = __ldg(args.masked_m + i);
-        if (mm < 0 || mm > args.m) {
-          bad = 1;
-          mm = mm < 0 ? 0 : args.m;
-        }
-        tab1[i] = mm;
+        const int32_t mm = __ldg(args.masked_m + i);
+        if (mm < 0 || mm > args.m) bad = 1;  // clamped where it is read (group_val)
       }
     }
     bad = __syncthreads_or(bad);
@@ -222,7 +227,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int lo = lane * per;
       auto tiles_of = [&](int e) -> int {
         if (args.mode == kKGrouped) return bad ? 0 : (args.m + kPairM - 1) / kPairM * args.n_tiles;
-        const int rows = args.mode == kContiguous ? (bad ? 0 : tab1[e + 1] - tab1[e]) : tab1[e];
+        const int rows = args.mode == kContiguous ? (bad ? 0 : group_val(args, e + 1) - group_val(args, e))
+                                                  : group_val(args, e);
         return (rows + kPairM - 1) / kPairM * args.n_tiles;
       };
       int sum = 0;
@@ -264,10 +270,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // K range of a tile in 128-byte chunks: all of K, or (K-grouped) the
   // expert's own token range [off[e], off[e+1])
   auto tile_kc0 = [&](const PairTile& tl) -> int {
-    return args.mode == kKGrouped ? tab1[tl.group] / BK : 0;
+    return args.mode == kKGrouped ? group_val(args, tl.group) / BK : 0;
   };
   auto tile_chunks = [&](const PairTile& tl) -> int {
-    return args.mode == kKGrouped ? (tab1[tl.group + 1] - tab1[tl.group]) / BK : args.k_tiles;
+    return args.mode == kKGrouped ? (group_val(args, tl.group + 1) - group_val(args, tl.group)) / BK : args.k_tiles;
   };
 
   // ---------------------------------------------------------------- roles
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t bytes_ab = 2u * (L::A_BYTES + L::B_BYTES);
       const uint32_t bytes_sf = 2u * (L::SFA_BYTES + L::SFB_BYTES);
       for (int t = pair; t < total && ok; t += npairs) {
-        const PairTile tl = decode_pair_tile(args, tab0, tab1, t);
+        const PairTile tl = decode_pair_tile(args, tab0, t);
         const int a_row = tl.row0 + 128 * static_cast<int>(rank);
         const int a_z = args.mode == kMasked ? tl.group : 0;
         const int b_z = (args.mode == kDense || args.mode == kKGrouped) ? 0 : tl.group;
@@ -340,7 +346,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = pair; t < total && ok; t += npairs) {
         if (!mbar_wait(acce_bar, acc_phase ^ 1u, abort_flag, args.wait_ns)) { ok = false; break; }
         tc_fence_after();
-        const int chunks = tile_chunks(decode_pair_tile(args, tab0, tab1, t));
+        const int chunks = tile_chunks(decode_pair_tile(args, tab0, t));
         const int k_stages = (chunks + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
           // both CTAs' operands of the stage have landed, and its scales are in TMEM
@@ -392,7 +398,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += npairs) {
-        const int k_stages = (tile_chunks(decode_pair_tile(args, tab0, tab1, t)) + kPairKC - 1) / kPairKC;
+        const int k_stages = (tile_chunks(decode_pair_tile(args, tab0, t)) + kPairKC - 1) / kPairKC;
         for (int ks = 0; ks < k_stages; ++ks) {
           if (!mbar_wait(sffull_bar(stage), phase, abort_flag, args.wait_ns)) { ok = false; break; }
           tc_fence_after();
@@ -432,7 +438,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       acc_phase ^= 1u;
       tc_fence_after();
-      const PairTile tl = decode_pair_tile(args, tab0, tab1, t);
+      const PairTile tl = decode_pair_tile(args, tab0, t);
       const int my_row0 = tl.row0 + 128 * static_cast<int>(rank);
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
       // dense rows past M are clipped by the tensor map; grouped rows past the

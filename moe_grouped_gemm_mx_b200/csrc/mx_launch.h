@@ -20,7 +20,9 @@ struct QuantSpec {
   int64_t sf_group_bytes;
 };
 
-cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, cudaStream_t stream, int* launches);
+// lean: the shared-memory-free form, one CTA per SM (to run beside a GEMM)
+cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, cudaStream_t stream, int* launches,
+                               bool lean = false);
 
 // Quantisation along the rows of x [groups, rows, cols] into q [groups, cols,
 // rows] with per-group tiled scales of the [cols, rows] operand.

@@ -106,9 +106,14 @@ __device__ __forceinline__ void store_out(uint4* p, const uint4& v) {
     __stcs(p, v);
 }
 
-template <bool KEEP>
+// STAGED: the coalesced loads go through a per-warp shared-memory stage (the
+// normal form).  Without it (the lean form) each lane loads its own block's
+// four pieces straight from global memory: no shared memory at all, so one
+// CTA of it fits on an SM beside a GEMM CTA that holds nearly all of the
+// shared memory, and the quantisation runs underneath the GEMM.
+template <bool KEEP, bool STAGED>
 __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_constant__ QuantBatch B) {
-  __shared__ uint4 quant_stage[(kQuantThreads / 32) * kQuantUnroll * 128];  // 2 KiB per warp and step
+  __shared__ uint4 quant_stage[STAGED ? (kQuantThreads / 32) * kQuantUnroll * 128 : 1];  // 2 KiB per warp and step
   // with programmatic dependent launch the next kernel may start its
   // prologue now; our own reads and writes wait for the previous kernel
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -138,43 +143,53 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_co
     const QuantJob& jb = B.job[jn];
     const uint32_t base = (slot - jb.slot0) * kSlotBlocks;
 
-    // Coalesced loads: instruction j of step u brings the 16-byte piece
-    // 32j + lane of the step's 2 KiB (512 contiguous bytes per instruction);
-    // the pieces go through a per-warp shared-memory stage, swizzled (piece
-    // p at slot p ^ ((p >> 3) & 7)) so that both the writes here and each
-    // lane's read of its own block's four pieces below are free of bank
-    // conflicts.
-    uint4* stage = quant_stage + (threadIdx.x >> 5) * (kQuantUnroll * 128);
-    {
-      uint4 g[kQuantUnroll][4];
+    uint4 v[kQuantUnroll][4];
+    if constexpr (!STAGED) {  // lean form: each lane's own 64 bytes, four 16-byte loads
 #pragma unroll
       for (int u = 0; u < kQuantUnroll; ++u) {
-        const uint32_t b0 = base + u * 32;  // first block of the step
-        const uint4* src = jb.x + static_cast<size_t>(b0) * 4;
+        const uint32_t b = base + u * 32 + lane;
+        const uint4* src = jb.x + static_cast<size_t>(b) * 4;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t p = 32 * j + lane;  // piece p belongs to block b0 + p / 4
-          g[u][j] = b0 + (p >> 2) < jb.nblk ? __ldcs(src + p) : make_uint4(0, 0, 0, 0);
-        }
+        for (int q = 0; q < 4; ++q) v[u][q] = b < jb.nblk ? __ldcs(src + q) : make_uint4(0, 0, 0, 0);
       }
+    } else {
+      // Coalesced loads: instruction j of step u brings the 16-byte piece
+      // 32j + lane of the step's 2 KiB (512 contiguous bytes per instruction);
+      // the pieces go through a per-warp shared-memory stage, swizzled (piece
+      // p at slot p ^ ((p >> 3) & 7)) so that both the writes here and each
+      // lane's read of its own block's four pieces below are free of bank
+      // conflicts.
+      uint4* stage = quant_stage + (threadIdx.x >> 5) * (kQuantUnroll * 128);
+      {
+        uint4 g[kQuantUnroll][4];
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+          const uint32_t b0 = base + u * 32;  // first block of the step
+          const uint4* src = jb.x + static_cast<size_t>(b0) * 4;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t p = 32 * j + lane;  // piece p belongs to block b0 + p / 4
+            g[u][j] = b0 + (p >> 2) < jb.nblk ? __ldcs(src + p) : make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t p = 32 * j + lane;
+            stage[u * 128 + (p ^ ((p >> 3) & 7u))] = g[u][j];
+          }
+      }
+      __syncwarp();
 #pragma unroll
       for (int u = 0; u < kQuantUnroll; ++u)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t p = 32 * j + lane;
-          stage[u * 128 + (p ^ ((p >> 3) & 7u))] = g[u][j];
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t p = 4 * lane + q;
+          v[u][q] = stage[u * 128 + (p ^ ((p >> 3) & 7u))];
         }
+      __syncwarp();  // the stage is rewritten by the warp's next slot
     }
-    __syncwarp();
-    uint4 v[kQuantUnroll][4];
-#pragma unroll
-    for (int u = 0; u < kQuantUnroll; ++u)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t p = 4 * lane + q;
-        v[u][q] = stage[u * 128 + (p ^ ((p >> 3) & 7u))];
-      }
-    __syncwarp();  // the stage is rewritten by the warp's next slot
 #pragma unroll
     for (int u = 0; u < kQuantUnroll; ++u) {
       const uint32_t b = base + u * 32 + lane;
@@ -227,11 +242,13 @@ __global__ void __launch_bounds__(kQuantThreads) mx_quant_kernel(const __grid_co
 
 // Launch helper used by the C ABI (validation happens there): up to
 // kMaxQuantJobs tensors in one launch.  Each job needs groups*rows*(k/32) < 2^31.
-cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, cudaStream_t stream, int* launches) {
+cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, cudaStream_t stream, int* launches,
+                               bool lean) {
   static int resident = 0;  // CTAs of the kernel one SM holds
   static int64_t l2_bytes = 0;
   if (resident == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, mx_quant_kernel<false>, kQuantThreads, 0);
+    cudaError_t e =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, mx_quant_kernel<false, true>, kQuantThreads, 0);
     if (e != cudaSuccess || resident <= 0) resident = 2048 / kQuantThreads;
     int dev = 0, l2 = 0;
     if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) == cudaSuccess)
@@ -274,7 +291,8 @@ cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, c
   B.total_slots = slots;
   B.pad_total = pads;
   const int64_t ctas_needed = (static_cast<int64_t>(slots) + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
-  const int64_t max_ctas = static_cast<int64_t>(num_sms) * resident;
+  // the lean form runs one CTA per SM, beside whatever else the SM holds
+  const int64_t max_ctas = static_cast<int64_t>(num_sms) * (lean ? 1 : resident);
   B.main_blocks = static_cast<int>(ctas_needed < max_ctas ? ctas_needed : max_ctas);
   int pad_blocks = 0;
   if (pads > 0) {
@@ -294,8 +312,10 @@ cudaError_t launch_quant_batch(const QuantSpec* specs, int count, int num_sms, c
   cfg.numAttrs = 1;
   // outputs that fit in three quarters of L2 are kept there for their consumer
   const bool keep = out_bytes <= l2_bytes / 4 * 3;
-  cudaError_t e = keep ? cudaLaunchKernelEx(&cfg, mx_quant_kernel<true>, B)
-                       : cudaLaunchKernelEx(&cfg, mx_quant_kernel<false>, B);
+  cudaError_t e = lean   ? (keep ? cudaLaunchKernelEx(&cfg, mx_quant_kernel<true, false>, B)
+                                : cudaLaunchKernelEx(&cfg, mx_quant_kernel<false, false>, B))
+                  : keep ? cudaLaunchKernelEx(&cfg, mx_quant_kernel<true, true>, B)
+                         : cudaLaunchKernelEx(&cfg, mx_quant_kernel<false, true>, B);
   if (e != cudaSuccess) return e;
   if (launches) *launches += 1;
   return cudaGetLastError();

@@ -99,3 +99,10 @@ def test_peaks_are_the_measured_ones():
         assert pk["hbm_gbs"] > 1000 and pk["bf16_tflops"] >= pk["bf16_tflops_sustained"] > 100
     else:
         assert pk["source"] == "fallback"
+
+
+def test_contiguous_step_text_names_the_lean_quantisation():
+    mx8 = bench.run_config(_args("contiguous"), 1)["step"]
+    tw = bench.run_config(_args("contiguous", fmt="tilewise"), 1)["step"]
+    assert "lean form" in mx8 and "parallel stream" in mx8
+    assert "lean" not in tw

@@ -137,6 +137,34 @@ def test_multi_matches_single_and_oracle(mx, oracle):
         assert np.array_equal(gpu_sf_rowmajor(oracle, sf, groups, rows, k), sf_ref)
 
 
+def test_multi_lean_matches_normal_form(mx, oracle):
+    """The lean form (no shared memory, one CTA per SM) writes the same bytes
+    as the normal form: the nine assorted tensors of the test above (outputs
+    small enough to be kept in L2), and the contiguous MoE's down operands
+    ([67,456 x 2048] tokens and 8 experts of [7168 x 2048]: outputs larger
+    than L2, streamed), scale padding included (buffers pre-filled with a
+    sentinel)."""
+    shapes = [(64, 7168), (2112, 256), (3, 130, 160), (1, 32), (0, 64), (300, 224), (129, 96),
+              (2, 128, 512), (5, 7168)]
+    for case in (shapes, [(67456, 2048), (8, 7168, 2048)]):
+        xs = [mx_inputs.outlier_bf16(s, seed=30 + i).cuda() if len(case) > 2 else
+              mx_inputs.normal_bf16(s, 1.0 if i == 0 else 0.02, 30 + i).cuda() for i, s in enumerate(case)]
+        outs = []
+        for x in xs:
+            groups = 1 if x.dim() == 2 else x.shape[0]
+            rows, k = x.shape[-2], x.shape[-1]
+            outs.append((torch.full(x.shape, 0xAB, dtype=torch.uint8, device="cuda"),
+                         torch.full((groups * mx.scale_bytes(rows, k),), 0xCD, dtype=torch.uint8, device="cuda")))
+        mx.mx_quantize_bf16_to_e4m3_multi(xs, outs, lean=True)
+        ref = mx.mx_quantize_bf16_to_e4m3_multi(xs)
+        torch.cuda.synchronize()
+        for (q, sf), (q1, sf1) in zip(outs, ref):
+            assert torch.equal(q, q1) and torch.equal(sf, sf1)
+    x = xs[0][:4096]
+    q_ref, sf_ref = oracle_quantize(oracle, x.cpu())
+    assert np.array_equal(outs[0][0][:4096].cpu().numpy(), q_ref)
+
+
 def test_empty_is_noop(mx):
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     q, sf = mx.mx_quantize_bf16_to_e4m3(x)
