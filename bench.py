@@ -159,6 +159,11 @@ def static_config(name: str, seed: int, fmt: str = "mxfp8") -> dict:
     elif name == "page":
         cfg["step"] = ("quantise activations + weights of the three shapes (one batched launch), then their "
                        "three GEMMs in one mx_gemm_batch launch with BF16 epilogue")
+    elif name == "large" and fmt == "mxfp8":
+        cfg["step"] = ("quantise the first shape's activations + weights, then the three GEMMs in sequence with "
+                       "BF16 epilogues; the second and third shapes' operands are quantised on a parallel stream "
+                       "by the lean form of the quantiser (no shared memory, one CTA per SM), each underneath "
+                       "the GEMM before the one that needs it")
     elif name == "contiguous" and fmt == "mxfp8":
         cfg["step"] = ("quantise the gate/up activations + weights (one batched launch), then the gate/up GEMM; "
                        "the down activations + weights are quantised on a parallel stream by the lean form of the "
@@ -361,12 +366,13 @@ class Workload:
         self.config = {"workload": name}
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.quant_jobs = []
-        self.lean_jobs = []     # quantised by the lean form, on a branch of their own (see _finish)
+        self.lean_jobs = []     # job lists of lean-form launches, run on a branch of their own (see _finish)
         self.fmt = fmt
         # independent chains of launches (lists of indices into launches), run
         # on parallel streams / graph branches after the launches in none
         self.branches = None
         self.after = []         # launches run after the branches have joined
+        self.waits = {}         # launch index -> launches of other branches it waits for
         self._side = []
         # launches timed one by one for the per-kernel table but not part of
         # the step (a step whose launches cannot be replayed alone times its
@@ -381,24 +387,31 @@ class Workload:
         self._finish()
 
     # -- helpers
-    def _quant(self, x, label, lean=False):
+    def _quant(self, x, label, lean=0):
         """Register x for the step's batched quantisation launch (or, with
-        lean, for the lean-form launch)."""
+        lean = g > 0, for the g-th launch of the lean form)."""
         import torch
         mx = self.mx
         groups = 1 if x.dim() == 2 else x.shape[0]
         rows, k = x.shape[-2], x.shape[-1]
         q = torch.empty(x.shape, dtype=torch.uint8, device=self.dev)
         sf = torch.empty(groups * mx.scale_bytes(rows, k), dtype=torch.uint8, device=self.dev)
-        (self.lean_jobs if lean else self.quant_jobs).append((x, q, sf, label))
+        if lean:
+            while len(self.lean_jobs) < lean:
+                self.lean_jobs.append([])
+            self.lean_jobs[lean - 1].append((x, q, sf, label))
+        else:
+            self.quant_jobs.append((x, q, sf, label))
         return q, sf
 
     def _finish(self):
         """All MXFP8 quantisations of the step go in one launch (up to 8
-        tensors), ahead of the GEMMs; lean jobs go in a second launch of the
-        lean form, placed by the workload's branches."""
+        tensors), ahead of the GEMMs, except the lean jobs: each group of
+        them is one launch of the lean form, placed by the workload's
+        branches."""
         mx = self.mx
-        for jobs, lean in ((self.lean_jobs, True), (self.quant_jobs, False)):
+        # after this: 0 the batched launch, 1.. the lean launches in order, then the rest
+        for jobs, lean in [(j, True) for j in reversed(self.lean_jobs)] + [(self.quant_jobs, False)]:
             if not jobs:
                 continue
             xs = [j[0] for j in jobs]
@@ -433,7 +446,7 @@ class Workload:
         self.launches.append(("quant", label, lambda x2: fn(x2, q=q, s=sc), nbytes, 0.0, (x2,)))
         return q.reshape(x.shape), sc
 
-    def _dense(self, a, b, label):
+    def _dense(self, a, b, label, lean=0):
         import torch
         mx = self.mx
         m, k = a.shape
@@ -451,8 +464,8 @@ class Workload:
                 qa, sa, qb, sb, d=d, dev_status=self.status), nbytes, fl, (qa, sa, qb, sb)))
             self.flops += fl
             return
-        qa, sfa = self._quant(a, label + ":A")
-        qb, sfb = self._quant(b, label + ":B")
+        qa, sfa = self._quant(a, label + ":A", lean)
+        qb, sfb = self._quant(b, label + ":B", lean)
         d = torch.empty((m, n), dtype=torch.bfloat16, device=self.dev)
         self.outputs.append(d)
         fl = 2.0 * m * n * k
@@ -503,9 +516,15 @@ class Workload:
                             "a": "N(0,1) with 0.5% x64 outliers", "b": "N(0,0.02)"})
 
     def _build_large(self, seed, I):
-        for (n, k) in I.LARGE_NK:
+        for s, (n, k) in enumerate(I.LARGE_NK):
             a, b = I.dense_problem(I.LARGE_M, n, k, seed=seed, kind="loguniform", device=self.dev)
-            self._dense(a, b, f"{I.LARGE_M}x{n}x{k}")
+            # shape s > 0 is quantised by the lean form underneath GEMM s - 1
+            self._dense(a, b, f"{I.LARGE_M}x{n}x{k}", lean=s)
+        if self.fmt == "mxfp8":
+            # launches after _finish: 0 quantise shape 0, 1 and 2 the lean launches
+            # of shapes 1 and 2, 3..5 the GEMMs
+            self.branches = [[0, 3, 4, 5], [1, 2]]
+            self.waits = {4: [1], 5: [2]}
         self.config.update({"shapes": [f"{I.LARGE_M}x{n}x{k}" for n, k in I.LARGE_NK],
                             "a": "row-wise 2^U[-4,4] * N(0,1)", "b": "N(0,0.02)"})
 
@@ -538,8 +557,8 @@ class Workload:
                 continue
             # the down GEMM's operands are quantised by the lean form beside
             # the gate/up quantisation and GEMM (branches below)
-            qa, sfa = self._quant(prob.a, tag + ":A", lean=tag == "down")
-            qb, sfb = self._quant(prob.b, tag + ":B", lean=tag == "down")
+            qa, sfa = self._quant(prob.a, tag + ":A", lean=int(tag == "down"))
+            qb, sfb = self._quant(prob.b, tag + ":B", lean=int(tag == "down"))
             self.launches.append(("gemm", tag, lambda qa, sfa, qb, sfb, off, d=d:
                                   mx.mx_grouped_gemm_contiguous(qa, sfa, qb, sfb, off, d=d, dev_status=self.status),
                                   self._gemm_bytes(m_total, n, k, experts), fl, (qa, sfa, qb, sfb, off)))
@@ -899,11 +918,29 @@ class Workload:
             self._side.append(torch.cuda.Stream(device=self.dev))
         for st in self._side[:nside]:
             st.wait_stream(cur)
-        for b, br in enumerate(self.branches):
-            with torch.cuda.stream(cur if b == 0 else self._side[b - 1]):
-                for i in br:
-                    _, _, fn, _, _, inputs = self.launches[i]
-                    fn(*inputs)
+        # issue the branches' launches in an order in which every launch that
+        # another branch waits for (self.waits) is recorded before that wait
+        streams = [cur] + self._side[:nside]
+        pending = [list(br) for br in self.branches]
+        sources = {d for deps in self.waits.values() for d in deps}
+        recorded = {}
+        while any(pending):
+            progressed = False
+            for b, br in enumerate(pending):
+                while br and all(d in recorded for d in self.waits.get(br[0], ())):
+                    i = br.pop(0)
+                    with torch.cuda.stream(streams[b]):
+                        for d in self.waits.get(i, ()):
+                            streams[b].wait_event(recorded[d])
+                        _, _, fn, _, _, inputs = self.launches[i]
+                        fn(*inputs)
+                        if i in sources:
+                            ev = torch.cuda.Event()
+                            ev.record(streams[b])
+                            recorded[i] = ev
+                    progressed = True
+            if not progressed:
+                raise RuntimeError("branch waits form a cycle")
         for st in self._side[:nside]:
             cur.wait_stream(st)
         for i in self.after:

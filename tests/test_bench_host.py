@@ -101,8 +101,106 @@ def test_peaks_are_the_measured_ones():
         assert pk["source"] == "fallback"
 
 
-def test_contiguous_step_text_names_the_lean_quantisation():
-    mx8 = bench.run_config(_args("contiguous"), 1)["step"]
-    tw = bench.run_config(_args("contiguous", fmt="tilewise"), 1)["step"]
+@pytest.mark.parametrize("workload", ["contiguous", "large"])
+def test_step_text_names_the_lean_quantisation(workload):
+    mx8 = bench.run_config(_args(workload), 1)["step"]
+    tw = bench.run_config(_args(workload, fmt="tilewise"), 1)["step"]
     assert "lean form" in mx8 and "parallel stream" in mx8
     assert "lean" not in tw
+
+
+class _FakeCuda:
+    """Stand-ins for the torch.cuda stream/event calls run_eager makes,
+    recording the order in which launches, waits and records are issued on
+    which stream."""
+
+    def __init__(self):
+        self.log = []
+        self.current = None
+        self.main = self.Stream(self, "main")
+
+    class Stream:
+        def __init__(self, fc, name=None, device=None):
+            self.fc, self.name = fc, name or f"side{len([e for e in fc.log if e[0] == 'new'])}"
+            fc.log.append(("new", self.name))
+
+        def wait_stream(self, other):
+            self.fc.log.append(("wait_stream", self.name, other.name))
+
+        def wait_event(self, ev):
+            assert ev.recorded, "waiting on an event that was never recorded"
+            self.fc.log.append(("wait_event", self.name, ev.tag))
+
+    class Event:
+        def __init__(self, fc):
+            self.fc, self.recorded, self.tag = fc, False, None
+
+        def record(self, stream):
+            self.recorded, self.tag = True, stream.fc.current_launch
+            self.fc.log.append(("record", stream.name, self.tag))
+
+
+def test_run_eager_branch_waits(monkeypatch):
+    import contextlib
+    import torch
+    fc = _FakeCuda()
+    fc.current = fc.main
+    fc.current_launch = None
+
+    @contextlib.contextmanager
+    def stream_ctx(st):
+        prev, fc.current = fc.current, st
+        try:
+            yield
+        finally:
+            fc.current = prev
+
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: fc.current)
+    monkeypatch.setattr(torch.cuda, "Stream", lambda device=None: _FakeCuda.Stream(fc, device=device))
+    monkeypatch.setattr(torch.cuda, "Event", lambda *a, **k: _FakeCuda.Event(fc))
+    monkeypatch.setattr(torch.cuda, "stream", stream_ctx)
+
+    def launch(i):
+        def fn():
+            fc.current_launch = i
+            fc.log.append(("launch", fc.current.name, i))
+        return ("quant", f"l{i}", fn, 0.0, 0.0, ())
+
+    wl = object.__new__(bench.Workload)
+    wl.dev = "cpu"
+    wl._side = []
+    # the large workload's shape: 0 quantise, 1 and 2 lean quantisations, 3..5 GEMMs
+    wl.launches = [launch(i) for i in range(6)]
+    wl.branches = [[0, 3, 4, 5], [1, 2]]
+    wl.waits = {4: [1], 5: [2]}
+    wl.after = []
+    wl.run_eager()
+    log = fc.log
+    launches = [e for e in log if e[0] == "launch"]
+    assert sorted(e[2] for e in launches) == list(range(6))
+    on = {e[2]: e[1] for e in launches}
+    assert on[0] == on[3] == on[4] == on[5] == "main" and on[1] == on[2] != "main"
+    pos = {e[2]: k for k, e in enumerate(log) if e[0] == "launch"}
+    for i, deps in wl.waits.items():
+        for d in deps:
+            rec = next(k for k, e in enumerate(log) if e[0] == "record" and e[2] == d)
+            wait = next(k for k, e in enumerate(log) if e[0] == "wait_event" and e[2] == d and e[1] == on[i])
+            assert pos[d] < rec < wait < pos[i]
+    assert pos[3] < pos[4] < pos[5] and pos[0] < pos[3] and pos[1] < pos[2]
+    # the side stream forks from and joins back into the main stream
+    side = on[1]
+    fork = next(k for k, e in enumerate(log) if e == ("wait_stream", side, "main"))
+    join = next(k for k, e in enumerate(log) if e == ("wait_stream", "main", side))
+    assert fork < pos[1] and join > max(pos.values())
+
+    # the contiguous workload's shape: a launch after the join
+    fc.log.clear()
+    wl.launches = [launch(i) for i in range(4)]
+    wl.branches = [[0, 2], [1]]
+    wl.waits = {}
+    wl.after = [3]
+    wl.run_eager()
+    log = fc.log
+    pos = {e[2]: k for k, e in enumerate(log) if e[0] == "launch"}
+    join = next(k for k, e in enumerate(log) if e[0] == "wait_stream" and e[1] == "main")
+    assert join < pos[3] and all(pos[i] < join for i in range(3))
